@@ -1,0 +1,57 @@
+"""Seeded synthetic inputs shared by the CUDA path's tests, the bench and the oracle.
+
+This module only draws random numbers and rounds them to the storage dtype; it
+contains none of the attention arithmetic.  Recipe (fixed, so every consumer sees
+identical bits):
+
+* one CPU ``torch.Generator`` seeded with ``seed``; Q, then K, then V are drawn in
+  that order as float32 N(0,1) (``torch.randn``);
+* each is multiplied by ``input_scale`` (exact for powers of two);
+* K rows ``0 .. k_sink_rows-1`` (every batch and KV head) are multiplied by
+  ``k_sink_factor`` (x8 is exact), V is left alone;
+* the float32 values are rounded to fp16 / bf16 (round-to-nearest-even).
+
+Layouts: prefill Q [B, Sq, Hq, D], K/V [B, Sk, Hkv, D]; decode Q [B, Hq, D].
+All tensors are contiguous CPU tensors of the storage dtype.
+"""
+from __future__ import annotations
+
+import torch
+
+DTYPES = {"fp16": torch.float16, "bf16": torch.bfloat16}
+
+
+def make_qkv(B, Sq, Sk, Hq, Hkv, D, dtype="fp16", seed=0, input_scale=1.0,
+             k_sink_rows=0, k_sink_factor=1.0, decode=False):
+    g = torch.Generator(device="cpu")
+    g.manual_seed(int(seed))
+    qshape = (B, Hq, D) if decode else (B, Sq, Hq, D)
+    q = torch.randn(qshape, generator=g, dtype=torch.float32)
+    k = torch.randn((B, Sk, Hkv, D), generator=g, dtype=torch.float32)
+    v = torch.randn((B, Sk, Hkv, D), generator=g, dtype=torch.float32)
+    if input_scale != 1.0:
+        q.mul_(input_scale)
+        k.mul_(input_scale)
+        v.mul_(input_scale)
+    if k_sink_rows:
+        k[:, :k_sink_rows].mul_(k_sink_factor)
+    t = DTYPES[dtype]
+    return q.to(t).contiguous(), k.to(t).contiguous(), v.to(t).contiguous()
+
+
+def make_workload_inputs(w, seed=None):
+    """Inputs of a :class:`workloads.Workload` (decode workloads give Q as [B, Hq, D])."""
+    return make_qkv(w.B, w.Sq, w.Sk, w.Hq, w.Hkv, w.D, w.dtype,
+                    w.seed if seed is None else seed, w.input_scale,
+                    w.k_sink_rows, w.k_sink_factor, decode=(w.kind == "decode"))
+
+
+def sample_rows(Sq, n_random, seed, extra=()):
+    """Seeded set of query rows for checking a long sequence row by row: the
+    first four rows, the rows around the first 128-row tile boundaries, the last
+    row, any ``extra`` rows, plus ``n_random`` uniform rows.  Sorted, unique, < Sq."""
+    g = torch.Generator(device="cpu")
+    g.manual_seed(int(seed) + 7919)
+    fixed = [0, 1, 2, 3, 127, 128, 129, 255, 256, 257, Sq - 1] + list(extra)
+    rnd = torch.randint(0, Sq, (n_random,), generator=g).tolist() if n_random else []
+    return sorted({r for r in fixed + rnd if 0 <= r < Sq})

@@ -1,0 +1,12 @@
+"""fp64 CPU oracle for the fused online-softmax attention forward.
+
+TEST INFRASTRUCTURE ONLY: imported by ``tests/``, ``__graft_entry__.smoke()`` and
+``bench.py`` (CPU baseline and ``--impl reference``), never by the library.
+It shares no code with the CUDA path.  Every function here is pinned by
+``tests/test_oracle.py`` to closed forms, invariants and brute force; none is
+"parity unpinned".
+"""
+from .attention import (attention, attention_rows, attention_blockwise, decode,
+                        combine_lse)
+
+__all__ = ["attention", "attention_rows", "attention_blockwise", "decode", "combine_lse"]

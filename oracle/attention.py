@@ -1,0 +1,167 @@
+"""fp64 CPU oracle for fused online-softmax attention -- TEST INFRASTRUCTURE ONLY.
+
+Only ``tests/``, ``__graft_entry__.smoke()`` and ``bench.py`` (its CPU-baseline leg
+and ``--impl reference``) may import this module.  The library itself never does:
+the CUDA path must not route through here.
+
+What it computes, for every batch b, query head h and query row i:
+
+    kvh   = h // G,  G = Hq // Hkv          (consecutive query heads share a KV head:
+                                              TurboQuant "Attention API" page,
+                                              compute_hybrid_attention_store, the
+                                              (T, H_kv, G, D) view of the query)
+    V_i   = { j < Sk : not causal  or  j <= i + Sk - Sq }   (bottom-right causal
+                                              alignment; the pages only use Sq == Sk,
+                                              where every alignment agrees)
+    s_j   = scale * sum_d q[b,i,h,d] * k[b,j,kvh,d]
+    M     = max_{j in V_i} s_j                (explicit max subtraction)
+    Z     = sum_{j in V_i} exp(s_j - M)
+    O     = sum_{j in V_i} exp(s_j - M) * v[b,j,kvh,:] / Z
+    LSE   = M + log Z                          (natural log; StreamAttention page,
+                                              "Kernel Design": lse = running max +
+                                              log of the running denominator)
+    empty V_i  ->  O = 0, LSE = -inf           (TurboQuant page: no keys gives zeros)
+
+The StreamAttention page's online recurrence ("Kernel Design (Fused Online
+Softmax)") is an exact reordering of this normalisation, so the direct definition
+is the oracle; :func:`attention_blockwise` restates the recurrence itself (the
+TurboQuant page's ``online_softmax_attention`` loop) so a test can pin the two
+against each other.  Everything is float64; inputs are widened exactly from
+their storage dtype.  No blocking, fusion or reordering beyond what is stated.
+"""
+from __future__ import annotations
+
+import numpy as np
+
+NEG_INF = -np.inf
+
+
+def _f64(x):
+    return np.asarray(x, dtype=np.float64)
+
+
+def _visible(Sq, Sk, causal, rows=None):
+    """Boolean [len(rows), Sk] visibility mask (bottom-right causal alignment)."""
+    rows = np.arange(Sq) if rows is None else np.asarray(rows)
+    j = np.arange(Sk)
+    if not causal:
+        return np.ones((rows.size, Sk), dtype=bool)
+    return j[None, :] <= (rows[:, None] + (Sk - Sq))
+
+
+def _softmax_attend(qm, km, vm, scale, vis):
+    """Plain softmax attention for one (batch, head): qm [n, D], km/vm [Sk, D],
+    vis [n, Sk].  Returns O [n, D] and LSE [n] in float64."""
+    s = scale * (qm @ km.T)                      # scores, [n, Sk]
+    s = np.where(vis, s, NEG_INF)
+    n = qm.shape[0]
+    o = np.zeros((n, vm.shape[1]), dtype=np.float64)
+    lse = np.full(n, NEG_INF, dtype=np.float64)
+    has = vis.any(axis=1)
+    if has.any():
+        sh = s[has]
+        m = sh.max(axis=1)                       # M
+        e = np.exp(sh - m[:, None])              # exp(s_j - M), 0 for masked keys
+        z = e.sum(axis=1)                        # Z
+        o[has] = (e @ vm) / z[:, None]
+        lse[has] = m + np.log(z)
+    return o, lse
+
+
+def attention(q, k, v, scale, causal=False):
+    """Full oracle.  q [B,Sq,Hq,D], k/v [B,Sk,Hkv,D] -> (O [B,Sq,Hq,D], LSE [B,Hq,Sq])."""
+    q, k, v = _f64(q), _f64(k), _f64(v)
+    B, Sq, Hq, D = q.shape
+    Sk, Hkv = k.shape[1], k.shape[2]
+    if Hkv == 0 or Hq % Hkv:
+        raise ValueError("Hq must be a positive multiple of Hkv")
+    G = Hq // Hkv
+    O = np.zeros((B, Sq, Hq, D), dtype=np.float64)
+    LSE = np.full((B, Hq, Sq), NEG_INF, dtype=np.float64)
+    if Sq == 0 or Sk == 0:
+        return O, LSE
+    vis = _visible(Sq, Sk, causal)
+    for b in range(B):
+        for h in range(Hq):
+            kvh = h // G
+            O[b, :, h, :], LSE[b, h, :] = _softmax_attend(
+                q[b, :, h, :], k[b, :, kvh, :], v[b, :, kvh, :], scale, vis)
+    return O, LSE
+
+
+def attention_rows(q, k, v, scale, causal, b, h, rows):
+    """Oracle for selected query rows of one (batch, head): returns O [n, D], LSE [n].
+    Used where the full Sq x Sk score matrix would not fit (long sequences)."""
+    rows = np.asarray(rows, dtype=np.int64)
+    Sq, Hq = q.shape[1], q.shape[2]
+    Sk, Hkv = k.shape[1], k.shape[2]
+    G = Hq // Hkv
+    kvh = h // G
+    qm = _f64(q[b, rows, h, :])
+    if Sk == 0:
+        return np.zeros((rows.size, q.shape[3])), np.full(rows.size, NEG_INF)
+    vis = _visible(Sq, Sk, causal, rows)
+    return _softmax_attend(qm, _f64(k[b, :, kvh, :]), _f64(v[b, :, kvh, :]), scale, vis)
+
+
+def decode(q, k, v, scale):
+    """Single-token decode: q [B,Hq,D], k/v [B,Sk,Hkv,D]; every key is visible.
+    Returns O [B,Hq,D] and LSE [B,Hq]."""
+    O, LSE = attention(_f64(q)[:, None], k, v, scale, causal=False)
+    return O[:, 0], LSE[:, :, 0]
+
+
+def attention_blockwise(q, k, v, scale, causal=False, block=64):
+    """The online-softmax recurrence, restated in float64 (TurboQuant page,
+    ``online_softmax_attention``; StreamAttention page, "Kernel Design"): walk the
+    keys in blocks, keep a running max m, running denominator l and accumulator acc,
+    rescale both by exp(m_old - m_new) when the max grows, finish with acc / l.
+    A fully masked block leaves the state unchanged (the flash-attn-volta page's
+    fully-masked-row guard: exponentiate against 0 while the max is still -inf)."""
+    q, k, v = _f64(q), _f64(k), _f64(v)
+    B, Sq, Hq, D = q.shape
+    Sk, Hkv = k.shape[1], k.shape[2]
+    G = Hq // Hkv
+    O = np.zeros((B, Sq, Hq, D))
+    LSE = np.full((B, Hq, Sq), NEG_INF)
+    vis = _visible(Sq, Sk, causal)
+    for b in range(B):
+        for h in range(Hq):
+            kvh = h // G
+            qm = q[b, :, h, :]
+            m = np.full(Sq, NEG_INF)
+            l = np.zeros(Sq)
+            acc = np.zeros((Sq, D))
+            for start in range(0, Sk, block):
+                end = min(start + block, Sk)
+                s = scale * (qm @ k[b, start:end, kvh, :].T)
+                s = np.where(vis[:, start:end], s, NEG_INF)
+                m_new = np.maximum(m, s.max(axis=1))
+                ref = np.where(np.isneginf(m_new), 0.0, m_new)   # the guard
+                alpha = np.exp(m - ref)
+                p = np.exp(s - ref[:, None])
+                l = l * alpha + p.sum(axis=1)
+                acc = acc * alpha[:, None] + p @ v[b, start:end, kvh, :]
+                m = m_new
+            ok = l > 0
+            O[b, ok, h, :] = acc[ok] / l[ok, None]
+            LSE[b, h, ok] = m[ok] + np.log(l[ok])
+    return O, LSE
+
+
+def combine_lse(outs, lses):
+    """LSE-weighted merge of partial attention results over disjoint key sets
+    (StreamAttention page, "Distributed and Long-Context Variants": log-sum-exp
+    weighted combining; its "Engine Direction" section: partial online-softmax
+    states merged in a second kernel).  outs[s] [..., D] normalised partial outputs,
+    lses[s] [...] their natural-log LSEs.  Parts with LSE = -inf carry no weight."""
+    lses = np.stack([_f64(x) for x in lses])          # [S, ...]
+    outs = np.stack([_f64(x) for x in outs])          # [S, ..., D]
+    mx = lses.max(axis=0)
+    ref = np.where(np.isneginf(mx), 0.0, mx)
+    w = np.exp(lses - ref)                            # [S, ...]
+    den = w.sum(axis=0)
+    lse = np.where(den > 0, ref + np.log(np.where(den > 0, den, 1.0)), NEG_INF)
+    o = np.where((den > 0)[..., None],
+                 (w[..., None] * outs).sum(axis=0) / np.where(den > 0, den, 1.0)[..., None], 0.0)
+    return o, lse

@@ -1,0 +1,262 @@
+"""Pins for the fp64 oracle: closed forms, invariants and brute force.
+
+Each test fixes the oracle against something other than itself, chosen so that a
+plausible slip (a dropped scale, a wrong sign, a transposed operand, a wrong GQA
+index or causal offset, a missing max-subtraction guard) fails at least one.
+"""
+import json
+import math
+import os
+
+import numpy as np
+import pytest
+
+from oracle import attention, attention_rows, attention_blockwise, decode, combine_lse
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+TOL = 1e-12
+
+
+def rnd(shape, seed, scale=1.0):
+    return np.random.default_rng(seed).standard_normal(shape) * scale
+
+
+def qkv(B=2, Sq=9, Sk=11, Hq=4, Hkv=2, D=8, seed=0, s=1.0):
+    return (rnd((B, Sq, Hq, D), seed, s), rnd((B, Sk, Hkv, D), seed + 1, s),
+            rnd((B, Sk, Hkv, D), seed + 2, s))
+
+
+def visible_count(i, Sq, Sk, causal):
+    return Sk if not causal else max(0, min(Sk, i + Sk - Sq + 1))
+
+
+def test_hand_worked_example():
+    g = json.load(open(os.path.join(GOLDEN, "hand_example.json")))
+    q = np.array(g["q"])[None, :, None, :]
+    k = np.array(g["k"])[None, :, None, :]
+    v = np.array(g["v"])[None, :, None, :]
+    for mode, causal in (("noncausal", False), ("causal", True)):
+        O, L = attention(q, k, v, g["scale"], causal)
+        np.testing.assert_allclose(O[0, :, 0, :], g[mode]["O"], atol=1e-14)
+        np.testing.assert_allclose(L[0, 0], g[mode]["LSE"], atol=1e-14)
+
+
+@pytest.mark.parametrize("causal", [False, True])
+@pytest.mark.parametrize("Sq,Sk", [(7, 7), (5, 9), (9, 5)])
+def test_zero_query_gives_mean_of_visible_values(causal, Sq, Sk):
+    # all scores equal -> uniform weights over the visible keys
+    _, k, v = qkv(Sq=Sq, Sk=Sk)
+    q = np.zeros((2, Sq, 4, 8))
+    O, L = attention(q, k, v, 0.37, causal)
+    for b in range(2):
+        for h in range(4):
+            for i in range(Sq):
+                n = visible_count(i, Sq, Sk, causal)
+                if n == 0:
+                    assert np.all(O[b, i, h] == 0) and L[b, h, i] == -np.inf
+                    continue
+                mean = np.mean(v[b, :n, h // 2, :], axis=0)
+                np.testing.assert_allclose(O[b, i, h], mean, atol=TOL)
+                assert abs(L[b, h, i] - math.log(n)) < TOL
+
+
+def test_zero_scale_gives_mean_of_values():
+    q, k, v = qkv()
+    O, L = attention(q, k, v, 0.0, False)
+    np.testing.assert_allclose(O, np.broadcast_to(
+        np.repeat(v.mean(axis=1), 2, axis=1)[:, None], O.shape), atol=TOL)
+    np.testing.assert_allclose(L, math.log(11), atol=TOL)
+
+
+def test_single_key_returns_its_value():
+    q, k, v = qkv(Sk=1)
+    scale = 0.41
+    O, L = attention(q, k, v, scale, False)
+    for b in range(2):
+        for h in range(4):
+            for i in range(9):
+                np.testing.assert_allclose(O[b, i, h], v[b, 0, h // 2], atol=TOL)
+                ref = scale * math.fsum(q[b, i, h, d] * k[b, 0, h // 2, d] for d in range(8))
+                assert abs(L[b, h, i] - ref) < TOL
+
+
+def test_one_hot_dominant_score_selects_one_value():
+    D, Sk, alpha, beta, scale = 8, 8, 4.0, 5.0, 4.0      # scale*alpha*beta = 80
+    k = np.zeros((1, Sk, 1, D))
+    for j in range(Sk):
+        k[0, j, 0, j] = alpha
+    v = rnd((1, Sk, 1, D), 3)
+    for jstar in range(Sk):
+        q = np.zeros((1, 1, 1, D))
+        q[0, 0, 0, jstar] = beta
+        O, L = attention(q, k, v, scale, False)
+        np.testing.assert_allclose(O[0, 0, 0], v[0, jstar, 0], atol=(Sk - 1) * math.exp(-80) * 10)
+        assert abs(L[0, 0, 0] - 80.0) < 1e-12
+
+
+def test_lse_matches_brute_force_sum_of_exponentials():
+    # small scores, so log(sum exp(s)) needs no max-subtraction
+    q, k, v = qkv(B=1, Sq=4, Sk=6, Hq=2, Hkv=1, D=5, s=0.5)
+    scale = 0.7
+    _, L = attention(q, k, v, scale, False)
+    for h in range(2):
+        for i in range(4):
+            tot = math.fsum(math.exp(scale * math.fsum(q[0, i, h, d] * k[0, j, 0, d] for d in range(5)))
+                            for j in range(6))
+            assert abs(L[0, h, i] - math.log(tot)) < 1e-13
+
+
+def test_output_matches_brute_force_softmax_weights():
+    # V = identity rows: O row i is exactly the softmax probability vector
+    Sk = D = 6
+    q = rnd((1, 3, 1, D), 11)
+    k = rnd((1, Sk, 1, D), 12)
+    v = np.eye(Sk)[None, :, None, :]
+    scale = 0.9
+    O, _ = attention(q, k, v, scale, False)
+    for i in range(3):
+        e = [math.exp(scale * math.fsum(q[0, i, 0, d] * k[0, j, 0, d] for d in range(D)))
+             for j in range(Sk)]
+        z = math.fsum(e)
+        np.testing.assert_allclose(O[0, i, 0], [x / z for x in e], atol=1e-14)
+
+
+def test_causal_row_zero_is_first_value():
+    q, k, v = qkv(Sq=10, Sk=10)
+    scale = 0.3
+    O, L = attention(q, k, v, scale, True)
+    for b in range(2):
+        for h in range(4):
+            np.testing.assert_allclose(O[b, 0, h], v[b, 0, h // 2], atol=TOL)
+            ref = scale * math.fsum(q[b, 0, h, d] * k[b, 0, h // 2, d] for d in range(8))
+            assert abs(L[b, h, 0] - ref) < TOL
+
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_affine_in_values(causal):
+    q, k, v = qkv()
+    a, c = -1.7, 0.25
+    O, L = attention(q, k, v, 0.5, causal)
+    O2, L2 = attention(q, k, a * v + c, 0.5, causal)
+    np.testing.assert_allclose(O2, a * O + c, atol=1e-12)
+    np.testing.assert_array_equal(L, L2)
+
+
+def test_key_permutation_invariance():
+    q, k, v = qkv()
+    perm = np.random.default_rng(5).permutation(11)
+    O, L = attention(q, k, v, 0.5, False)
+    O2, L2 = attention(q, k[:, perm], v[:, perm], 0.5, False)
+    np.testing.assert_allclose(O2, O, atol=TOL)
+    np.testing.assert_allclose(L2, L, atol=TOL)
+
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_score_shift(causal):
+    # k_j += u for every j adds scale*q.u to every score of a row: O unchanged
+    q, k, v = qkv()
+    u = rnd((2, 1, 2, 8), 9)
+    scale = 0.45
+    O, L = attention(q, k, v, scale, causal)
+    O2, L2 = attention(q, k + u, v, scale, causal)
+    np.testing.assert_allclose(O2, O, atol=1e-12)
+    shift = scale * np.einsum("bihd,bhd->bhi", q, np.repeat(u[:, 0], 2, axis=1))
+    np.testing.assert_allclose(L2, L + shift, atol=1e-12)
+
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_gqa_equals_mha_on_repeated_kv(causal):
+    # repeat_kv: KV head j serves query heads j*G .. j*G+G-1
+    q, k, v = qkv(Hq=6, Hkv=2)
+    O, L = attention(q, k, v, 0.5, causal)
+    kk, vv = np.repeat(k, 3, axis=2), np.repeat(v, 3, axis=2)
+    O2, L2 = attention(q, kk, vv, 0.5, causal)
+    np.testing.assert_array_equal(O, O2)
+    np.testing.assert_array_equal(L, L2)
+    # and not the interleaved (h % Hkv) mapping
+    O3, _ = attention(q, np.tile(k, (1, 1, 3, 1)), np.tile(v, (1, 1, 3, 1)), 0.5, causal)
+    assert not np.allclose(O, O3)
+
+
+def test_split_combine_equals_whole():
+    q, k, v = qkv(Sk=13)
+    O, L = attention(q, k, v, 0.5, False)
+    parts = [(0, 5), (5, 6), (6, 13)]
+    outs, lses = zip(*[attention(q, k[:, a:b], v[:, a:b], 0.5, False) for a, b in parts])
+    lses = [x.transpose(0, 2, 1) for x in lses]          # [B, Sq, Hq]
+    Oc, Lc = combine_lse(outs, lses)
+    np.testing.assert_allclose(Oc, O, atol=1e-12)
+    np.testing.assert_allclose(Lc, L.transpose(0, 2, 1), atol=1e-12)
+
+
+def test_combine_ignores_empty_parts():
+    o = rnd((3, 4), 1)
+    l = rnd((3,), 2)
+    Oc, Lc = combine_lse([o, np.zeros((3, 4))], [l, np.full(3, -np.inf)])
+    np.testing.assert_allclose(Oc, o, atol=TOL)
+    np.testing.assert_allclose(Lc, l, atol=TOL)
+    Oc, Lc = combine_lse([o, o], [np.full(3, -np.inf)] * 2)
+    assert np.all(Oc == 0) and np.all(Lc == -np.inf)
+
+
+@pytest.mark.parametrize("causal", [False, True])
+@pytest.mark.parametrize("Sq,Sk,block", [(9, 11, 4), (16, 16, 64), (20, 7, 3), (3, 130, 64)])
+def test_blockwise_recurrence_equals_direct(causal, Sq, Sk, block):
+    q, k, v = qkv(Sq=Sq, Sk=Sk, s=2.0)
+    O, L = attention(q, k, v, 0.6, causal)
+    O2, L2 = attention_blockwise(q, k, v, 0.6, causal, block)
+    np.testing.assert_allclose(O2, O, atol=1e-12)
+    np.testing.assert_allclose(L2, L, atol=1e-12)
+
+
+def test_causal_leak_rows_ignore_future_keys():
+    q, k, v = qkv(Sq=12, Sk=12)
+    O, L = attention(q, k, v, 0.5, True)
+    for i in range(12):
+        k2, v2 = k.copy(), v.copy()
+        k2[:, i + 1:] += 100.0
+        v2[:, i + 1:] -= 50.0
+        O2, L2 = attention(q, k2, v2, 0.5, True)
+        np.testing.assert_array_equal(O2[:, :i + 1], O[:, :i + 1])
+        np.testing.assert_array_equal(L2[:, :, :i + 1], L[:, :, :i + 1])
+
+
+def test_empty_and_fully_masked():
+    q, k, v = qkv(Sk=0)
+    O, L = attention(q, k, v, 0.5, False)
+    assert np.all(O == 0) and np.all(L == -np.inf)
+    q, k, v = qkv(Sq=9, Sk=4)           # causal, Sq > Sk: rows 0..4 see nothing
+    O, L = attention(q, k, v, 0.5, True)
+    assert np.all(O[:, :5] == 0) and np.all(L[:, :, :5] == -np.inf)
+    assert np.all(np.isfinite(L[:, :, 5:]))
+    np.testing.assert_allclose(O[:, 5, :, :], np.repeat(v[:, 0], 2, axis=1), atol=TOL)
+
+
+def test_decode_is_last_causal_row():
+    # bottom-right alignment: a single query sees every key, like the last causal row
+    q, k, v = qkv(Sq=6, Sk=6)
+    O, L = attention(q, k, v, 0.5, True)
+    Od, Ld = decode(q[:, -1], k, v, 0.5)
+    np.testing.assert_allclose(Od, O[:, -1], atol=TOL)
+    np.testing.assert_allclose(Ld, L[:, :, -1], atol=TOL)
+    Oc, Lc = attention(q[:, -1:], k, v, 0.5, True)          # Sq=1 causal == all visible
+    np.testing.assert_allclose(Oc[:, 0], Od, atol=TOL)
+
+
+def test_rows_match_full():
+    q, k, v = qkv(Sq=10, Sk=12)
+    O, L = attention(q, k, v, 0.5, True)
+    rows = [0, 3, 9]
+    for b in range(2):
+        for h in range(4):
+            Or, Lr = attention_rows(q, k, v, 0.5, True, b, h, rows)
+            np.testing.assert_allclose(Or, O[b, rows, h], atol=TOL)
+            np.testing.assert_allclose(Lr, L[b, h, rows], atol=TOL)
+
+
+def test_large_scores_stay_finite():
+    # max-subtraction: scores ~ 1e3 would overflow exp() without it
+    q, k, v = qkv(s=30.0)
+    O, L = attention(q, k, v, 1.0, True)
+    assert np.all(np.isfinite(O)) and np.all(np.isfinite(L))
+    assert np.all(np.abs(O) <= np.abs(v).max() + 1e-9)
