@@ -1,0 +1,125 @@
+/*
+ * sa_attn.h -- C ABI of the B200 (sm_100a) fused online-softmax attention library.
+ *
+ * What is computed (for batch b, query head h, query row i; G = Hq / Hkv):
+ *   kvh = h / G                                   GQA: consecutive query heads share a
+ *                                                 KV head (TurboQuant "Attention API" page,
+ *                                                 compute_hybrid_attention_store, the
+ *                                                 (T, H_kv, G, D) query view)
+ *   visible keys j: j < Sk, and j <= i + Sk - Sq when causal (bottom-right alignment;
+ *                                                 the pages use Sq == Sk only)
+ *   s_j = scale * <q[b,i,h,:], k[b,j,kvh,:]>
+ *   O   = sum_j softmax(s)_j * v[b,j,kvh,:]       StreamAttention page, "Kernel Design
+ *   LSE = log sum_j exp(s_j)  (natural log)       (Fused Online Softmax)": one streaming
+ *                                                 pass with running max, running sum and a
+ *                                                 rescaled accumulator; lse = running max
+ *                                                 + log(denominator)
+ *   no visible key -> O = 0 and LSE = -inf        (TurboQuant page: empty KV gives zeros)
+ *
+ * Layouts (all contiguous, row-major, elements of `dtype` unless stated):
+ *   prefill  q [B, Sq, Hq, D]   k, v [B, Sk, Hkv, D]   o [B, Sq, Hq, D]   lse [B, Hq, Sq] fp32
+ *   decode   q [B, Hq, D]       k, v [B, Sk, Hkv, D]   o [B, Hq, D]       lse [B, Hq]     fp32
+ *
+ * Conventions shared by every entry point:
+ *   - All tensor pointers are DEVICE pointers owned by the caller; the library keeps no
+ *     reference after the call returns and allocates no device memory on these paths.
+ *   - Work is enqueued asynchronously on `stream` (NULL = legacy default stream); nothing
+ *     synchronises.  A return of SA_OK means "validated and launched".
+ *   - Pointers must be 16-byte aligned (tensor-memory-access copies need it).
+ *   - Arguments are checked on the host before anything is launched; the first failing
+ *     check is returned and sa_last_error() describes it.  Nothing is written then.
+ *   - Every device-side wait is bounded; if one expires the kernel records it in a device
+ *     status word and returns early (outputs are then undefined).  sa_check_status()
+ *     reports and clears that word.
+ *   - D must be 64 or 128; dtype SA_FP16 or SA_BF16; Hq a positive multiple of Hkv.
+ *   - B == 0, Sq == 0 or Hq == 0: SA_OK, nothing launched.  Sk == 0: O = 0, LSE = -inf.
+ */
+#ifndef SA_ATTN_H
+#define SA_ATTN_H
+
+#include <stddef.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Same handle type as cudaStream_t / CUstream. */
+typedef struct CUstream_st* sa_stream_t;
+
+typedef enum { SA_FP16 = 0, SA_BF16 = 1 } sa_dtype_t;
+
+typedef enum {
+    SA_OK = 0,
+    SA_ERR_INVALID = -1,      /* null pointer, negative size, Hq % Hkv, misalignment, bad scale */
+    SA_ERR_UNSUPPORTED = -2,  /* D not in {64,128}, unknown dtype, size beyond a stated limit */
+    SA_ERR_CUDA = -3,         /* a CUDA call failed; sa_last_error() has the CUDA message */
+    SA_ERR_TIMEOUT = -4,      /* a bounded device wait expired (reported by sa_check_status) */
+    SA_ERR_WORKSPACE = -5     /* decode workspace missing or smaller than required */
+} sa_status_t;
+
+/*
+ * Prefill / full attention forward (StreamAttention page, "Kernel Design (Fused Online
+ * Softmax)"; flash-attn-volta page, flash_attn_forward with return_softmax_lse).
+ *   q, k, v, o : device tensors as laid out above.
+ *   lse        : device fp32 [B, Hq, Sq], or NULL to skip it.
+ *   causal     : 0 or 1 (bottom-right aligned when Sq != Sk).
+ *   scale      : softmax scale, used as given (finite); callers usually pass 1/sqrt(D).
+ *   dtype      : SA_FP16 or SA_BF16 for q, k, v and o.
+ * Runs the persistent tcgen05 (tensor-memory) kernel.
+ */
+int sa_attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse,
+                int B, int Sq, int Sk, int Hq, int Hkv, int D, int causal,
+                float scale, int dtype, sa_stream_t stream);
+
+/*
+ * Bytes of decode workspace needed for `num_splits` (0 = the automatic choice).  The
+ * workspace holds, per (b, h, split), the split's unnormalised fp32 output row and its
+ * running max and sum (StreamAttention page, "Engine Direction": partial online-softmax
+ * states merged by a second kernel).  Returns 0 for empty problems or invalid sizes.
+ */
+size_t sa_attn_decode_workspace_size(int B, int Sk, int Hq, int Hkv, int D, int num_splits);
+
+/* The split count sa_attn_decode uses for num_splits = 0 on the current device (>= 1),
+ * or 0 for invalid sizes. */
+int sa_attn_decode_num_splits(int B, int Sk, int Hq, int Hkv, int D);
+
+/*
+ * Single-token split-KV decode with an LSE-weighted combine (StreamAttention page,
+ * "Engine Direction" and "Distributed and Long-Context Variants": partial states merged
+ * with log-sum-exp weights).
+ *   q [B, Hq, D], k/v [B, Sk, Hkv, D], o [B, Hq, D]; lse [B, Hq] fp32 or NULL.
+ *   num_splits : KV splits per (b, kv head); 0 = automatic; clamped to ceil(Sk / 64).
+ *   workspace  : device buffer of at least sa_attn_decode_workspace_size(...) bytes,
+ *                16-byte aligned, owned by the caller; overwritten; must not be shared
+ *                by calls that may run concurrently.
+ * Launches the split kernel and, on the same stream, the combine kernel.
+ */
+int sa_attn_decode(const void* q, const void* k, const void* v, void* o, float* lse,
+                   int B, int Sk, int Hq, int Hkv, int D, float scale, int dtype,
+                   int num_splits, void* workspace, size_t workspace_bytes,
+                   sa_stream_t stream);
+
+/*
+ * Diagnostic only: the same forward as sa_attn_fwd computed by a plain CUDA-core kernel
+ * (one thread per query row, fp32 online softmax).  Slow; used to cross-check the
+ * tensor-core path.  Same arguments and conventions as sa_attn_fwd.
+ */
+int sa_attn_fwd_simple(const void* q, const void* k, const void* v, void* o, float* lse,
+                       int B, int Sq, int Sk, int Hq, int Hkv, int D, int causal,
+                       float scale, int dtype, sa_stream_t stream);
+
+/* Thread-local description of the last non-OK return of this thread ("" if none). */
+const char* sa_last_error(void);
+
+/* Synchronises `stream`, then returns SA_ERR_TIMEOUT (and clears the word) if a device
+ * wait expired since the last check, SA_ERR_CUDA on a CUDA error, else SA_OK. */
+int sa_check_status(sa_stream_t stream);
+
+/* Library version, "major.minor.patch". */
+const char* sa_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* SA_ATTN_H */

@@ -1,0 +1,11 @@
+"""B200 (sm_100a) fused online-softmax attention: prefill forward and split-KV decode.
+
+The computation runs in hand-written CUDA kernels behind the C ABI of
+``include/sa_attn.h`` (``libsa_attn.so``); :mod:`.sa_attn` is its Python binding.
+"""
+from .sa_attn import (sa_attn_fwd, sa_attn_fwd_simple, sa_attn_decode,
+                      sa_attn_decode_workspace_size, sa_attn_decode_num_splits,
+                      sa_check_status, sa_version, SAError, lib)
+
+__all__ = ["sa_attn_fwd", "sa_attn_fwd_simple", "sa_attn_decode", "sa_attn_decode_workspace_size",
+           "sa_attn_decode_num_splits", "sa_check_status", "sa_version", "SAError", "lib"]

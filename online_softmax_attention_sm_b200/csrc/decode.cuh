@@ -1,0 +1,344 @@
+// decode.cuh -- split-KV single-token decode and its LSE-weighted combine, sm_100a.
+//
+// Method: the StreamAttention page's split-state prototype ("Engine Direction": write
+// partial online-softmax states, merge them in a second kernel) and its log-sum-exp
+// weighted combining ("Distributed and Long-Context Variants").  Each split runs the
+// online-softmax recurrence of "Kernel Design" over its slice of keys; the combine
+// rescales every split's state to the common max and divides once.
+//
+// B200 design:
+//   * grid (split, KV head x head-group, batch); the G = Hq/Hkv query heads that share a
+//     KV head are packed as the rows of one 16-row mma.sync tile, so every K/V byte is
+//     read from HBM exactly once (never once per query head);
+//   * thread 0 streams 64-token K and V slices with TMA tensor loads (128-byte swizzle)
+//     into a ring of shared-memory stages; 4 warps each take 16 tokens of a stage;
+//   * S = Q K^T and O += P V on mma.sync.m16n8k16 (fp32 accumulate), fragments from
+//     ldmatrix; row max / sum by quad shuffles; the 4 warps merge through shared memory;
+//   * the split writes (unnormalised O, running max, running sum) in fp32; the combine
+//     kernel (one warp per (batch, query head)) is launched with programmatic dependent
+//     launch so its launch overlaps the split kernel's tail.
+#pragma once
+#include "ptx.cuh"
+#include <cuda_fp16.h>
+#include <cuda_bf16.h>
+#include <type_traits>
+
+namespace sa {
+
+template <int D>
+struct DecCfg {
+  static constexpr int TOK = 64;                       // tokens per stage
+  static constexpr int KCH = D / 64;
+  static constexpr int CHUNK_BYTES = TOK * 128;        // 64 tokens x 64 elements
+  static constexpr int KV_BYTES = KCH * CHUNK_BYTES;   // one K (or V) stage
+  static constexpr int STAGES = (D == 64) ? 4 : 2;
+  static constexpr int SMEM_STAGES = STAGES * 2 * KV_BYTES;
+  static constexpr int SMEM_MERGE = 4 * 16 * D * 4 + 2 * 4 * 16 * 4;
+  static constexpr int SMEM_TOTAL = 1024 + (SMEM_STAGES > SMEM_MERGE ? SMEM_STAGES : SMEM_MERGE) + 256;
+};
+
+struct DecParams {
+  const void* q;       // [B, Hq, D]
+  float* ws_o;         // [B, Hq, nsplit, D]
+  float* ws_ml;        // [B, Hq, nsplit, 2]  (max in log2 units of c2*s, sum)
+  void* o;             // [B, Hq, D]
+  float* lse;          // [B, Hq] or null
+  int B, Sk, Hq, Hkv, G, ngrp, nsplit, chunk;
+  float c2;
+};
+
+__device__ __forceinline__ void ldsm_x4(uint32_t addr, uint32_t& r0, uint32_t& r1, uint32_t& r2, uint32_t& r3) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];"
+               : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3) : "r"(addr));
+}
+__device__ __forceinline__ void ldsm_x4_t(uint32_t addr, uint32_t& r0, uint32_t& r1, uint32_t& r2, uint32_t& r3) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0,%1,%2,%3}, [%4];"
+               : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3) : "r"(addr));
+}
+
+template <bool BF16>
+__device__ __forceinline__ void mma16816(float (&c)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
+  if (BF16) {
+    asm volatile("mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, {%0,%1,%2,%3};"
+                 : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
+                 : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+  } else {
+    asm volatile("mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, {%0,%1,%2,%3};"
+                 : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
+                 : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+  }
+}
+
+template <bool BF16>
+__device__ __forceinline__ uint32_t pack2(float lo, float hi) {
+  if (BF16) {
+    __nv_bfloat162 h = __floats2bfloat162_rn(lo, hi);
+    return *reinterpret_cast<uint32_t*>(&h);
+  } else {
+    __half2 h = __floats2half2_rn(lo, hi);
+    return *reinterpret_cast<uint32_t*>(&h);
+  }
+}
+
+// Byte offset of (row, 16-byte column chunk) inside a 128-byte-swizzled box of 128-byte rows.
+__device__ __forceinline__ uint32_t sw128(int row, int chunk16) {
+  return (uint32_t)(row * 128 + ((chunk16 ^ (row & 7)) << 4));
+}
+
+template <int D, bool BF16>
+__global__ void __launch_bounds__(128)
+attn_decode_split(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
+                  const DecParams p) {
+  using Cfg = DecCfg<D>;
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  uint8_t* smem = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
+  const int region = Cfg::SMEM_STAGES > Cfg::SMEM_MERGE ? Cfg::SMEM_STAGES : Cfg::SMEM_MERGE;
+  uint64_t* full = (uint64_t*)(smem + region);
+  volatile int* abort_flag = (volatile int*)(full + Cfg::STAGES);
+
+  // let the combine kernel get launched while this grid runs (it waits for our results)
+  asm volatile("griddepcontrol.launch_dependents;");
+
+  const int split = blockIdx.x;
+  const int kvh = blockIdx.y / p.ngrp;
+  const int grp = blockIdx.y % p.ngrp;
+  const int b = blockIdx.z;
+  const int h0 = kvh * p.G + grp * 16;                  // first query head of this tile
+  const int nrows = min(16, p.G - grp * 16);            // valid rows of the tile
+  const int tok0 = split * p.chunk;
+  const int tok1 = min(p.Sk, tok0 + p.chunk);
+  const int nstage = (tok1 - tok0 + Cfg::TOK - 1) / Cfg::TOK;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < Cfg::STAGES; ++i) mbar_init(&full[i], 1);
+    *abort_flag = 0;
+    fence_barrier_init();
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    tma_prefetch_desc(&tm_k); tma_prefetch_desc(&tm_v);
+    for (int s = 0; s < Cfg::STAGES && s < nstage; ++s) {
+      uint8_t* dk = smem + s * 2 * Cfg::KV_BYTES;
+      mbar_arrive_expect_tx(&full[s], 2 * Cfg::KV_BYTES);
+      for (int c = 0; c < Cfg::KCH; ++c) {
+        tma_load_4d(dk + c * Cfg::CHUNK_BYTES, &tm_k, &full[s], c * 64, kvh, tok0 + s * Cfg::TOK, b);
+        tma_load_4d(dk + Cfg::KV_BYTES + c * Cfg::CHUNK_BYTES, &tm_v, &full[s], c * 64, kvh, tok0 + s * Cfg::TOK, b);
+      }
+    }
+  }
+
+  // Q fragments (A operand, 16 rows = packed query heads, K = D), rows >= nrows are 0
+  uint32_t qa[D / 16][4];
+  {
+    const uint16_t* q16 = reinterpret_cast<const uint16_t*>(p.q);
+    const int r0 = lane >> 2, r1 = r0 + 8, cc = (lane & 3) * 2;
+    const size_t base = ((size_t)b * p.Hq + h0) * D;
+#pragma unroll
+    for (int kk = 0; kk < D / 16; ++kk) {
+      const int d0 = kk * 16 + cc;
+      auto ld = [&](int r, int d) -> uint32_t {
+        return r < nrows ? *reinterpret_cast<const uint32_t*>(q16 + base + (size_t)r * D + d) : 0u;
+      };
+      qa[kk][0] = ld(r0, d0);
+      qa[kk][1] = ld(r1, d0);
+      qa[kk][2] = ld(r0, d0 + 8);
+      qa[kk][3] = ld(r1, d0 + 8);
+    }
+  }
+
+  float o[D / 8][4];
+#pragma unroll
+  for (int n = 0; n < D / 8; ++n) o[n][0] = o[n][1] = o[n][2] = o[n][3] = 0.f;
+  float m0 = -INFINITY, m1 = -INFINITY, l0 = 0.f, l1 = 0.f;
+  const float c2 = p.c2;
+  const uint32_t smem_addr = smem_u32(smem);
+  bool ok = true;
+  int issued = min(Cfg::STAGES, nstage);               // stages whose loads were issued
+
+  for (int st = 0; st < nstage; ++st) {
+    const int slot = st % Cfg::STAGES;
+    // on a failed wait the stage's contents are stale but in bounds; the CTA-wide vote
+    // after the compute decides whether to stop
+    const bool landed = mbar_wait(&full[slot], (st / Cfg::STAGES) & 1, abort_flag, 40);
+    const uint32_t kb = smem_addr + slot * 2 * Cfg::KV_BYTES;
+    const uint32_t vb = kb + Cfg::KV_BYTES;
+    const int wt = warp * 16;                          // this warp's first token in the stage
+    // ---- S (16 heads x 16 tokens) = Q K^T
+    float s[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
+#pragma unroll
+    for (int kk = 0; kk < D / 16; ++kk) {
+      // matrices: (tok 0-7, d 0-7), (tok 0-7, d 8-15), (tok 8-15, d 0-7), (tok 8-15, d 8-15)
+      const int mi = lane >> 3, rr = lane & 7;
+      const int tok = wt + ((mi >> 1) << 3) + rr;
+      const int dchunk = (kk & 3) * 2 + (mi & 1);      // 16-byte chunk within the 64-wide box
+      uint32_t b0, b1, b2, b3;
+      ldsm_x4(kb + (kk >> 2) * Cfg::CHUNK_BYTES + sw128(tok, dchunk), b0, b1, b2, b3);
+      mma16816<BF16>(s[0], qa[kk], b0, b1);
+      mma16816<BF16>(s[1], qa[kk], b2, b3);
+    }
+    // ---- scale, mask tokens outside [tok0, tok1), online softmax
+    const int tbase = tok0 + st * Cfg::TOK + wt + (lane & 3) * 2;
+    float x[2][4];
+#pragma unroll
+    for (int n = 0; n < 2; ++n)
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const int tk = tbase + n * 8 + (e & 1);
+        x[n][e] = (tk < tok1) ? s[n][e] * c2 : -INFINITY;
+      }
+    float mx0 = fmaxf(fmaxf(x[0][0], x[0][1]), fmaxf(x[1][0], x[1][1]));
+    float mx1 = fmaxf(fmaxf(x[0][2], x[0][3]), fmaxf(x[1][2], x[1][3]));
+    mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, 1));
+    mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, 2));
+    mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, 1));
+    mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, 2));
+    const float mn0 = fmaxf(m0, mx0), mn1 = fmaxf(m1, mx1);
+    const float u0 = (mn0 == -INFINITY) ? 0.f : mn0, u1 = (mn1 == -INFINITY) ? 0.f : mn1;
+    const float a0 = ex2(m0 - u0), a1 = ex2(m1 - u1);
+    m0 = mn0; m1 = mn1;
+    float pr[2][4];
+#pragma unroll
+    for (int n = 0; n < 2; ++n) {
+      pr[n][0] = ex2(x[n][0] - u0); pr[n][1] = ex2(x[n][1] - u0);
+      pr[n][2] = ex2(x[n][2] - u1); pr[n][3] = ex2(x[n][3] - u1);
+    }
+    l0 = l0 * a0 + pr[0][0] + pr[0][1] + pr[1][0] + pr[1][1];
+    l1 = l1 * a1 + pr[0][2] + pr[0][3] + pr[1][2] + pr[1][3];
+#pragma unroll
+    for (int n = 0; n < D / 8; ++n) { o[n][0] *= a0; o[n][1] *= a0; o[n][2] *= a1; o[n][3] *= a1; }
+    // P as the A operand (16 heads x 16 tokens)
+    uint32_t pa[4];
+    pa[0] = pack2<BF16>(pr[0][0], pr[0][1]);
+    pa[1] = pack2<BF16>(pr[0][2], pr[0][3]);
+    pa[2] = pack2<BF16>(pr[1][0], pr[1][1]);
+    pa[3] = pack2<BF16>(pr[1][2], pr[1][3]);
+    // ---- O (16 x D) += P V; V slice [16 tokens][D] via transposed ldmatrix
+#pragma unroll
+    for (int n = 0; n < D / 8; n += 2) {
+      // matrices: (tok 0-7, d n*8..), (tok 8-15, d n*8..), (tok 0-7, d (n+1)*8..), (tok 8-15, d (n+1)*8..)
+      const int mi = lane >> 3, rr = lane & 7;
+      const int tok = wt + ((mi & 1) << 3) + rr;
+      const int dcol = n + (mi >> 1);                  // 8-element column block 0..D/8-1
+      uint32_t b0, b1, b2, b3;
+      ldsm_x4_t(vb + (dcol >> 3) * Cfg::CHUNK_BYTES + sw128(tok, dcol & 7), b0, b1, b2, b3);
+      mma16816<BF16>(o[n], pa, b0, b1);
+      mma16816<BF16>(o[n + 1], pa, b2, b3);
+    }
+    // every warp is done with this slot, and every thread saw its data land
+    if (!__syncthreads_and(landed)) { ok = false; break; }
+    if (threadIdx.x == 0 && st + Cfg::STAGES < nstage) {
+      const int ns = st + Cfg::STAGES;
+      issued = ns + 1;
+      uint8_t* dk = smem + slot * 2 * Cfg::KV_BYTES;
+      mbar_arrive_expect_tx(&full[slot], 2 * Cfg::KV_BYTES);
+      for (int c = 0; c < Cfg::KCH; ++c) {
+        tma_load_4d(dk + c * Cfg::CHUNK_BYTES, &tm_k, &full[slot], c * 64, kvh, tok0 + ns * Cfg::TOK, b);
+        tma_load_4d(dk + Cfg::KV_BYTES + c * Cfg::CHUNK_BYTES, &tm_v, &full[slot], c * 64, kvh, tok0 + ns * Cfg::TOK, b);
+      }
+    }
+  }
+  if (!ok) {
+    // drain loads still in flight before shared memory is released
+    if (threadIdx.x == 0) {
+      // loads were issued for stages 0 .. issued-1; those not yet consumed may be pending
+      // (each slot's most recent load is among the last STAGES issued)
+      for (int st = max(0, issued - Cfg::STAGES); st < issued; ++st)
+        mbar_wait(&full[st % Cfg::STAGES], (st / Cfg::STAGES) & 1, nullptr, 41);
+    }
+    __syncthreads();
+    return;
+  }
+
+  // ---- merge the 4 warps: per row, rescale to the CTA max and add
+  l0 += __shfl_xor_sync(0xffffffffu, l0, 1);
+  l0 += __shfl_xor_sync(0xffffffffu, l0, 2);
+  l1 += __shfl_xor_sync(0xffffffffu, l1, 1);
+  l1 += __shfl_xor_sync(0xffffffffu, l1, 2);
+  float* sm_o = reinterpret_cast<float*>(smem);              // [4][16][D] (stages are drained)
+  float* sm_m = sm_o + 4 * 16 * D;                           // [4][16]
+  float* sm_l = sm_m + 64;                                   // [4][16]
+  const int r0 = lane >> 2, r1 = r0 + 8;
+  if ((lane & 3) == 0) {
+    sm_m[warp * 16 + r0] = m0; sm_m[warp * 16 + r1] = m1;
+    sm_l[warp * 16 + r0] = l0; sm_l[warp * 16 + r1] = l1;
+  }
+  __syncthreads();
+  float M0 = -INFINITY, M1 = -INFINITY;
+#pragma unroll
+  for (int w = 0; w < 4; ++w) { M0 = fmaxf(M0, sm_m[w * 16 + r0]); M1 = fmaxf(M1, sm_m[w * 16 + r1]); }
+  const float w0 = (m0 == -INFINITY) ? 0.f : ex2(m0 - M0);
+  const float w1 = (m1 == -INFINITY) ? 0.f : ex2(m1 - M1);
+#pragma unroll
+  for (int n = 0; n < D / 8; ++n) {
+    const int c = n * 8 + (lane & 3) * 2;
+    sm_o[(warp * 16 + r0) * D + c] = o[n][0] * w0;
+    sm_o[(warp * 16 + r0) * D + c + 1] = o[n][1] * w0;
+    sm_o[(warp * 16 + r1) * D + c] = o[n][2] * w1;
+    sm_o[(warp * 16 + r1) * D + c + 1] = o[n][3] * w1;
+  }
+  __syncthreads();
+  const size_t ws_row0 = ((size_t)b * p.Hq + h0) * p.nsplit + split;   // row r -> + r * nsplit
+  for (int i = threadIdx.x; i < nrows * D; i += blockDim.x) {
+    const int r = i / D, d = i % D;
+    float acc = 0.f;
+#pragma unroll
+    for (int w = 0; w < 4; ++w) acc += sm_o[(w * 16 + r) * D + d];
+    p.ws_o[(ws_row0 + (size_t)r * p.nsplit) * D + d] = acc;
+  }
+  if (threadIdx.x < nrows) {
+    const int r = threadIdx.x;
+    float M = -INFINITY;
+#pragma unroll
+    for (int w = 0; w < 4; ++w) M = fmaxf(M, sm_m[w * 16 + r]);
+    float L = 0.f;
+#pragma unroll
+    for (int w = 0; w < 4; ++w) {
+      const float mw = sm_m[w * 16 + r];
+      L += (mw == -INFINITY) ? 0.f : sm_l[w * 16 + r] * ex2(mw - M);
+    }
+    float* ml = p.ws_ml + (ws_row0 + (size_t)r * p.nsplit) * 2;
+    ml[0] = M;
+    ml[1] = L;
+  }
+}
+
+// One warp per (batch, query head): O = sum_s w_s O_s / sum_s w_s l_s, w_s = 2^(m_s - M).
+template <int D, bool BF16>
+__global__ void __launch_bounds__(128)
+attn_decode_combine(const DecParams p) {
+  asm volatile("griddepcontrol.wait;" ::: "memory");   // split results are complete
+  const int gw = blockIdx.x * 4 + (threadIdx.x >> 5);
+  const int lane = threadIdx.x & 31;
+  if (gw >= p.B * p.Hq) return;
+  const float* ml = p.ws_ml + (size_t)gw * p.nsplit * 2;
+  const float* os = p.ws_o + (size_t)gw * p.nsplit * D;
+  float M = -INFINITY;
+  for (int s = lane; s < p.nsplit; s += 32) M = fmaxf(M, ml[2 * s]);
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
+  constexpr int E = D / 32;                            // elements per lane
+  float acc[E];
+#pragma unroll
+  for (int e = 0; e < E; ++e) acc[e] = 0.f;
+  float L = 0.f;
+  for (int s = 0; s < p.nsplit; ++s) {
+    const float ms = ml[2 * s];
+    const float w = (ms == -INFINITY) ? 0.f : ex2(ms - M);
+    L += w * ml[2 * s + 1];
+#pragma unroll
+    for (int e = 0; e < E; ++e) acc[e] += w * os[(size_t)s * D + lane * E + e];
+  }
+  const float inv = L > 0.f ? 1.f / L : 0.f;
+  using T = typename std::conditional<BF16, __nv_bfloat16, __half>::type;
+  T* out = reinterpret_cast<T*>(p.o) + (size_t)gw * D + lane * E;
+#pragma unroll
+  for (int e = 0; e < E; e += 2) {
+    uint32_t v = pack2<BF16>(acc[e] * inv, acc[e + 1] * inv);
+    *reinterpret_cast<uint32_t*>(out + e) = v;
+  }
+  if (p.lse && lane == 0)
+    p.lse[gw] = L > 0.f ? (M + __log2f(L)) * 0.69314718055994531f : -INFINITY;
+}
+
+}  // namespace sa

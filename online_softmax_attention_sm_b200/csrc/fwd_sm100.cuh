@@ -1,0 +1,440 @@
+// fwd_sm100.cuh -- persistent fused attention forward for sm_100a.
+//
+// Method: the online-softmax forward of the StreamAttention page ("Kernel Design (Fused
+// Online Softmax)"): stream K/V tiles, keep per query row a running max, a running
+// denominator and a rescaled accumulator, finish with acc / den and
+// lse = max + log(den).  Fully masked rows follow the flash-attn-volta page's guard
+// (section "Stability"): exponentiate against 0 while the running max is still -inf.
+//
+// B200 design:
+//   * unit of work = (batch, query head, 256 query rows) = two 128-row Q tiles that
+//     share every K/V tile; a persistent grid of one CTA per SM walks the units in
+//     longest-first order (causal units with more K/V tiles first);
+//   * warp 8 (one lane) issues TMA tensor loads: the two Q tiles once per unit, then
+//     K and V tiles into a ring of shared-memory slots (full/empty mbarriers);
+//   * warp 9 (one lane) issues tcgen05.mma: S_t = Q_t K^T (128x128, fp32 in tensor
+//     memory) and O_t += P_t V (P_t read from tensor memory, O_t fp32 in tensor memory);
+//   * warpgroups 0 and 1 run the softmax of Q tile 0 and 1: each thread owns one row of
+//     S (tcgen05.ld 32x32b), computes the row max, p = 2^(c*s - m) with c = scale*log2(e),
+//     the row sum, writes P as 16-bit into tensor memory over S, and rescales its O row
+//     only when the reference max moves by more than kRescaleThresh (exact after the
+//     final division; keeps p <= 2^kRescaleThresh);
+//   * the epilogue (same warpgroups) divides O by the row sum, rounds to the I/O dtype
+//     and writes O and the natural-log LSE.
+// Causal: K/V tiles past the diagonal are never loaded or multiplied; only tiles that
+// cross the diagonal or the ragged end of K are masked.
+#pragma once
+#include "ptx.cuh"
+#include <cuda_fp16.h>
+#include <cuda_bf16.h>
+#include <type_traits>
+
+namespace sa {
+
+template <int D>
+struct FwdCfg {
+  static constexpr int BM = 128;                     // query rows per Q tile
+  static constexpr int BN = 128;                     // keys per K/V tile
+  static constexpr int KCH = D / 64;                 // 128-byte chunks along D
+  static constexpr int CHUNK_BYTES = 128 * 128;      // one 128-row x 64-element box
+  static constexpr int TILE_BYTES = KCH * CHUNK_BYTES;
+  static constexpr int STAGES = (D == 128) ? 4 : 8;  // K/V ring slots
+  static constexpr int SMEM_Q = 2 * TILE_BYTES;
+  static constexpr int SMEM_RING = STAGES * TILE_BYTES;
+  static constexpr int SMEM_BARS = 1024;
+  static constexpr int SMEM_TOTAL = 1024 /*align slack*/ + SMEM_Q + SMEM_RING + SMEM_BARS;
+  static constexpr int THREADS = 384;                // 2 softmax WGs + load/MMA WG
+  static constexpr uint32_t TMEM_COLS = 512;
+  // tensor-memory column map: S_t at 128 t, O_t at 256 + D t, P_t over S_t (16-bit)
+  __host__ __device__ static constexpr uint32_t S_COL(int t) { return 128u * t; }
+  __host__ __device__ static constexpr uint32_t O_COL(int t) { return 256u + (uint32_t)D * t; }
+  __host__ __device__ static constexpr uint32_t P_COL(int t) { return 128u * t; }
+};
+
+constexpr float kRescaleThresh = 8.0f;   // log2 units
+
+struct FwdParams {
+  void* o;
+  float* lse;
+  int B, Sq, Sk, Hq, Hkv, causal;
+  int n_qblk;        // ceil(Sq / 256)
+  int n_units;       // B * Hq * n_qblk
+  float c2;          // scale * log2(e)
+};
+
+struct UnitInfo {
+  int b, h, kvh, q0;         // q0: first query row of the unit
+  int nkv[2];                // K/V tiles needed by Q tile 0 / 1 (0: tile has no work)
+  int nkv_max;
+};
+
+__device__ __forceinline__ int fwd_kv_tiles(const FwdParams& p, int r0) {
+  if (r0 >= p.Sq) return 0;
+  int kend = p.Sk;
+  if (p.causal) {
+    int rmax = min(r0 + 127, p.Sq - 1);
+    kend = min(p.Sk, rmax + p.Sk - p.Sq + 1);
+  }
+  return kend > 0 ? (kend + 127) / 128 : 0;
+}
+
+// Units are numbered longest-first: query block descending, then (b, h) with heads of
+// one KV head adjacent.
+__device__ __forceinline__ UnitInfo fwd_unit(const FwdParams& p, int u) {
+  UnitInfo x;
+  int bh = p.B * p.Hq;
+  int qb = p.n_qblk - 1 - u / bh;
+  int r = u % bh;
+  x.b = r / p.Hq;
+  x.h = r % p.Hq;
+  x.kvh = x.h / (p.Hq / p.Hkv);
+  x.q0 = qb * 256;
+  x.nkv[0] = fwd_kv_tiles(p, x.q0);
+  x.nkv[1] = fwd_kv_tiles(p, x.q0 + 128);
+  x.nkv_max = max(x.nkv[0], x.nkv[1]);
+  return x;
+}
+
+// Snake assignment of the longest-first unit list over the persistent CTAs.
+__device__ __forceinline__ int fwd_unit_of(int round, int cta, int ncta) {
+  return round * ncta + ((round & 1) ? (ncta - 1 - cta) : cta);
+}
+
+template <int D, bool BF16>
+__global__ void __launch_bounds__(384, 1)
+attn_fwd_sm100(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+               const __grid_constant__ CUtensorMap tm_v, const FwdParams p) {
+  using Cfg = FwdCfg<D>;
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  uint8_t* smem = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
+  uint8_t* sQ = smem;                                   // [2][TILE]
+  uint8_t* sRing = smem + Cfg::SMEM_Q;                  // [STAGES][TILE]
+  uint64_t* bars = (uint64_t*)(smem + Cfg::SMEM_Q + Cfg::SMEM_RING);
+  uint64_t* kv_full = bars;                             // [STAGES]
+  uint64_t* kv_empty = bars + Cfg::STAGES;              // [STAGES]
+  uint64_t* q_full = bars + 2 * Cfg::STAGES;            // [2]
+  uint64_t* q_empty = q_full + 2;                       // [2]
+  uint64_t* s_full = q_full + 4;                        // [2]
+  uint64_t* p_full = q_full + 6;                        // [2]
+  uint64_t* o_done = q_full + 8;                        // [2]
+  uint64_t* fin_bar = q_full + 10;                      // [1]
+  uint32_t* tmem_holder = (uint32_t*)(q_full + 12);
+  volatile int* abort_flag = (volatile int*)(tmem_holder + 1);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const int ncta = gridDim.x;
+  const int cta = blockIdx.x;
+
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < Cfg::STAGES; ++i) { mbar_init(&kv_full[i], 1); mbar_init(&kv_empty[i], 1); }
+    for (int t = 0; t < 2; ++t) {
+      mbar_init(&q_full[t], 1); mbar_init(&q_empty[t], 1);
+      mbar_init(&s_full[t], 1); mbar_init(&p_full[t], 128); mbar_init(&o_done[t], 1);
+    }
+    mbar_init(fin_bar, 1);
+    *abort_flag = 0;
+    fence_barrier_init();
+  }
+  if (warp == 9) {
+    tmem_alloc(tmem_holder, Cfg::TMEM_COLS);
+    tmem_relinquish();
+  }
+  if (warp == 8 && lane == 0) {
+    tma_prefetch_desc(&tm_q); tma_prefetch_desc(&tm_k); tma_prefetch_desc(&tm_v);
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_holder;
+
+  if (warp == 8) {
+    // ------------------------------------------------------------ TMA producer
+    if (lane == 0) {
+      int slot = 0, ring_n = 0;            // ring position and total loads issued
+      int q_loads[2] = {0, 0};
+      bool ok = true;
+      for (int round = 0; ok; ++round) {
+        int u = fwd_unit_of(round, cta, ncta);
+        if (u >= p.n_units) break;
+        UnitInfo x = fwd_unit(p, u);
+        for (int j = 0; j < x.nkv_max && ok; ++j) {
+          for (int kv = 0; kv < 2 && ok; ++kv) {
+            if (ring_n >= Cfg::STAGES) {
+              ok = mbar_wait(&kv_empty[slot], ((ring_n / Cfg::STAGES) - 1) & 1, abort_flag, 1);
+              if (!ok) break;
+            }
+            uint8_t* dst = sRing + slot * Cfg::TILE_BYTES;
+            mbar_arrive_expect_tx(&kv_full[slot], Cfg::TILE_BYTES);
+            const CUtensorMap* tm = kv ? &tm_v : &tm_k;
+            for (int c = 0; c < Cfg::KCH; ++c)
+              tma_load_4d(dst + c * Cfg::CHUNK_BYTES, tm, &kv_full[slot], c * 64, x.kvh, j * 128, x.b);
+            ++ring_n;
+            slot = (slot + 1 == Cfg::STAGES) ? 0 : slot + 1;
+            if (j == 0 && kv == 0) {
+              // Q tiles after the first K tile, so K0 is in flight while Q waits for its slot
+              for (int t = 0; t < 2 && ok; ++t) {
+                if (x.nkv[t] == 0) continue;
+                if (q_loads[t] > 0) {
+                  ok = mbar_wait(&q_empty[t], (q_loads[t] - 1) & 1, abort_flag, 2);
+                  if (!ok) break;
+                }
+                uint8_t* qd = sQ + t * Cfg::TILE_BYTES;
+                mbar_arrive_expect_tx(&q_full[t], Cfg::TILE_BYTES);
+                for (int c = 0; c < Cfg::KCH; ++c)
+                  tma_load_4d(qd + c * Cfg::CHUNK_BYTES, &tm_q, &q_full[t], c * 64, x.h, x.q0 + t * 128, x.b);
+                ++q_loads[t];
+              }
+            }
+          }
+        }
+      }
+      if (!ok) {
+        // drain: every load issued must land before the CTA's shared memory goes away
+        int first = ring_n > Cfg::STAGES ? ring_n - Cfg::STAGES : 0;
+        for (int n = first; n < ring_n; ++n)
+          mbar_wait(&kv_full[n % Cfg::STAGES], (n / Cfg::STAGES) & 1, nullptr, 3);
+        for (int t = 0; t < 2; ++t)
+          if (q_loads[t] > 0) mbar_wait(&q_full[t], (q_loads[t] - 1) & 1, nullptr, 4);
+      }
+    }
+    __syncwarp();
+  } else if (warp == 9) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      constexpr uint32_t IDESC_QK = idesc_f16(BF16 ? 1 : 0, 128, 128, 0, 0);
+      constexpr uint32_t IDESC_PV = idesc_f16(BF16 ? 1 : 0, 128, D, 0, 1);
+      const uint32_t sQ_addr = smem_u32(sQ);
+      const uint32_t sRing_addr = smem_u32(sRing);
+      int slot = 0, ring_n = 0;
+      int q_uses[2] = {0, 0}, pv_n[2] = {0, 0};
+      bool ok = true;
+      for (int round = 0; ok; ++round) {
+        int u = fwd_unit_of(round, cta, ncta);
+        if (u >= p.n_units) break;
+        UnitInfo x = fwd_unit(p, u);
+        for (int j = 0; j < x.nkv_max && ok; ++j) {
+          // ---- S_t = Q_t K_j^T
+          ok = mbar_wait(&kv_full[slot], (ring_n / Cfg::STAGES) & 1, abort_flag, 10);
+          if (!ok) break;
+          const uint32_t k_addr = sRing_addr + slot * Cfg::TILE_BYTES;
+          for (int t = 0; t < 2; ++t) {
+            if (j >= x.nkv[t]) continue;
+            if (j == 0) {
+              ok = mbar_wait(&q_full[t], q_uses[t] & 1, abort_flag, 11);
+              if (!ok) break;
+            }
+            if (pv_n[t] > 0) {   // P_t lives over S_t: the previous P_t V must be done
+              ok = mbar_wait(&o_done[t], (pv_n[t] - 1) & 1, abort_flag, 12);
+              if (!ok) break;
+            }
+            tc_fence_after();
+            const uint32_t q_addr = sQ_addr + t * Cfg::TILE_BYTES;
+#pragma unroll
+            for (int kk = 0; kk < D / 16; ++kk) {
+              const uint32_t off = (kk >> 2) * Cfg::CHUNK_BYTES + (kk & 3) * 32;
+              mma_ss(tmem_base + Cfg::S_COL(t), smem_desc_sw128(q_addr + off, 16, 1024),
+                     smem_desc_sw128(k_addr + off, 16, 1024), IDESC_QK, kk > 0);
+            }
+            mma_commit(&s_full[t]);
+          }
+          if (!ok) break;
+          mma_commit(&kv_empty[slot]);
+          ++ring_n;
+          slot = (slot + 1 == Cfg::STAGES) ? 0 : slot + 1;
+          if (j == x.nkv_max - 1) {
+            for (int t = 0; t < 2; ++t)
+              if (x.nkv[t] > 0) { mma_commit(&q_empty[t]); ++q_uses[t]; }
+          }
+          // ---- O_t += P_t V_j
+          ok = mbar_wait(&kv_full[slot], (ring_n / Cfg::STAGES) & 1, abort_flag, 13);
+          if (!ok) break;
+          const uint32_t v_addr = sRing_addr + slot * Cfg::TILE_BYTES;
+          for (int t = 0; t < 2; ++t) {
+            if (j >= x.nkv[t]) continue;
+            ok = mbar_wait(&p_full[t], (pv_n[t]) & 1, abort_flag, 14);
+            if (!ok) break;
+            tc_fence_after();
+#pragma unroll
+            for (int kk = 0; kk < 128 / 16; ++kk) {
+              mma_ts(tmem_base + Cfg::O_COL(t), tmem_base + Cfg::P_COL(t) + kk * 8,
+                     smem_desc_sw128(v_addr + kk * 2048, Cfg::CHUNK_BYTES, 1024), IDESC_PV,
+                     (j > 0 || kk > 0) ? 1u : 0u);
+            }
+            mma_commit(&o_done[t]);
+            ++pv_n[t];
+          }
+          if (!ok) break;
+          mma_commit(&kv_empty[slot]);
+          ++ring_n;
+          slot = (slot + 1 == Cfg::STAGES) ? 0 : slot + 1;
+        }
+      }
+      // every MMA issued above completes before tensor memory is released
+      mma_commit(fin_bar);
+      mbar_wait(fin_bar, 0, nullptr, 15);
+    }
+    __syncwarp();
+  } else if (warp < 8) {
+    // ------------------------------------------------------------ softmax / epilogue
+    const int t = warp >> 2;                  // Q tile of this warpgroup
+    const int wl = warp & 3;                  // TMEM lane quarter
+    const int row_in_tile = wl * 32 + lane;
+    const uint32_t lane_addr = tmem_base + ((uint32_t)(wl * 32) << 16);
+    const float c2 = p.c2;
+    int s_n = 0, o_n = 0;                     // s_full / o_done phases consumed
+    bool ok = true;
+    for (int round = 0; ok; ++round) {
+      int u = fwd_unit_of(round, cta, ncta);
+      if (u >= p.n_units) break;
+      UnitInfo x = fwd_unit(p, u);
+      const int nkv = x.nkv[t];
+      const int row = x.q0 + t * 128 + row_in_tile;
+      int klim = p.Sk;
+      if (p.causal) klim = min(p.Sk, row + p.Sk - p.Sq + 1);
+      // the first key tile that any row of this Q tile must mask
+      const int r0 = x.q0 + t * 128;
+      int kvis = p.Sk;                        // keys every row of the tile can see
+      if (p.causal) kvis = min(kvis, max(0, r0 + p.Sk - p.Sq + 1));
+      const int mask_from = kvis / 128;
+      float m_ref = -INFINITY, l_sum = 0.f;
+      for (int j = 0; j < nkv; ++j) {
+        ok = __all_sync(0xffffffffu, mbar_wait(&s_full[t], s_n & 1, abort_flag, 20 + t));
+        if (!ok) break;
+        ++s_n;
+        tc_fence_after();
+        float s[128];
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+          uint32_t r[32];
+          tmem_ld32(lane_addr + Cfg::S_COL(t) + c * 32, r);
+#pragma unroll
+          for (int i = 0; i < 32; ++i) s[c * 32 + i] = __uint_as_float(r[i]);
+        }
+        tmem_wait_ld();
+        const bool masked = (j >= mask_from);
+        float m_tile;
+        if (masked) {
+          const int kl = klim - j * 128;     // keys >= kl are invisible to this row
+#pragma unroll
+          for (int i = 0; i < 128; ++i) s[i] = (i < kl) ? s[i] * c2 : -INFINITY;
+          m_tile = s[0];
+#pragma unroll
+          for (int i = 1; i < 128; ++i) m_tile = fmaxf(m_tile, s[i]);
+        } else {
+          float mx = s[0];
+          if (c2 >= 0.f) {
+#pragma unroll
+            for (int i = 1; i < 128; ++i) mx = fmaxf(mx, s[i]);
+          } else {
+#pragma unroll
+            for (int i = 1; i < 128; ++i) mx = fminf(mx, s[i]);
+          }
+          m_tile = mx * c2;
+        }
+        // lazy rescale: move the reference max only when it grows by more than the threshold
+        const bool need = m_tile > m_ref + kRescaleThresh;
+        float alpha = 1.f;
+        if (need) {
+          alpha = ex2(m_ref - m_tile);       // 0 when m_ref == -inf
+          l_sum *= alpha;
+          m_ref = m_tile;
+        }
+        const float m_use = (m_ref == -INFINITY) ? 0.f : m_ref;
+        float rs = 0.f;
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+          uint32_t pk[16];
+#pragma unroll
+          for (int i = 0; i < 16; ++i) {
+            float a, b2;
+            if (masked) {
+              a = ex2(s[c * 32 + 2 * i] - m_use);
+              b2 = ex2(s[c * 32 + 2 * i + 1] - m_use);
+            } else {
+              a = ex2(fmaf(s[c * 32 + 2 * i], c2, -m_use));
+              b2 = ex2(fmaf(s[c * 32 + 2 * i + 1], c2, -m_use));
+            }
+            rs += a + b2;
+            if (BF16) {
+              __nv_bfloat162 h2 = __floats2bfloat162_rn(a, b2);
+              pk[i] = *reinterpret_cast<uint32_t*>(&h2);
+            } else {
+              __half2 h2 = __floats2half2_rn(a, b2);
+              pk[i] = *reinterpret_cast<uint32_t*>(&h2);
+            }
+          }
+          tmem_st16(lane_addr + Cfg::P_COL(t) + c * 16, pk);
+        }
+        l_sum += rs;
+        // O_t holds P V up to tile j-1 (complete: S_t(j) was issued after it finished)
+        if (j > 0 && __any_sync(0xffffffffu, need)) {
+#pragma unroll 1
+          for (int c = 0; c < D / 32; ++c) {
+            uint32_t r[32];
+            tmem_ld32(lane_addr + Cfg::O_COL(t) + c * 32, r);
+            tmem_wait_ld();
+#pragma unroll
+            for (int i = 0; i < 32; ++i) r[i] = __float_as_uint(__uint_as_float(r[i]) * alpha);
+            tmem_st32(lane_addr + Cfg::O_COL(t) + c * 32, r);
+          }
+        }
+        tmem_wait_st();
+        tc_fence_before();
+        mbar_arrive(&p_full[t]);
+      }
+      if (!ok) break;
+      // ---------------- epilogue: O / l, LSE
+      if (nkv > 0) {
+        ok = __all_sync(0xffffffffu, mbar_wait(&o_done[t], (o_n + nkv - 1) & 1, abort_flag, 22 + t));
+        if (!ok) break;
+        o_n += nkv;
+        tc_fence_after();
+      }
+      const bool store = row < p.Sq;
+      const float inv_l = l_sum > 0.f ? 1.f / l_sum : 0.f;
+      using T = typename std::conditional<BF16, __nv_bfloat16, __half>::type;
+      T* orow = reinterpret_cast<T*>(p.o) + (((size_t)x.b * p.Sq + row) * p.Hq + x.h) * D;
+#pragma unroll 1
+      for (int c = 0; c < D / 32; ++c) {
+        uint32_t r[32];
+        if (nkv > 0) {
+          tmem_ld32(lane_addr + Cfg::O_COL(t) + c * 32, r);
+          tmem_wait_ld();
+        } else {
+#pragma unroll
+          for (int i = 0; i < 32; ++i) r[i] = 0u;
+        }
+        uint32_t pk[16];
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+          float a = __uint_as_float(r[2 * i]) * inv_l, b2 = __uint_as_float(r[2 * i + 1]) * inv_l;
+          if (BF16) {
+            __nv_bfloat162 h2 = __floats2bfloat162_rn(a, b2);
+            pk[i] = *reinterpret_cast<uint32_t*>(&h2);
+          } else {
+            __half2 h2 = __floats2half2_rn(a, b2);
+            pk[i] = *reinterpret_cast<uint32_t*>(&h2);
+          }
+        }
+        if (store) {
+          uint4* dst = reinterpret_cast<uint4*>(orow + c * 32);
+#pragma unroll
+          for (int i = 0; i < 4; ++i) dst[i] = make_uint4(pk[4 * i], pk[4 * i + 1], pk[4 * i + 2], pk[4 * i + 3]);
+        }
+      }
+      if (store && p.lse) {
+        float lse = l_sum > 0.f ? (m_ref + __log2f(l_sum)) * 0.69314718055994531f : -INFINITY;
+        p.lse[((size_t)x.b * p.Hq + x.h) * p.Sq + row] = lse;
+      }
+      tc_fence_before();
+    }
+  }
+  // warps 10, 11 have no role
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == 9) tmem_dealloc(tmem_base, Cfg::TMEM_COLS);
+}
+
+}  // namespace sa

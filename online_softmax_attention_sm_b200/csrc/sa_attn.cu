@@ -1,0 +1,306 @@
+// sa_attn.cu -- host side of the C ABI declared in include/sa_attn.h: argument checks,
+// tensor-map construction, split planning and kernel launches.  Nothing here allocates
+// device memory; every device pointer belongs to the caller.
+#include "../../include/sa_attn.h"
+#include "ptx.cuh"
+#include "fwd_sm100.cuh"
+#include "fwd_simple.cuh"
+#include "decode.cuh"
+
+#include <cmath>
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+#include <mutex>
+#include <string>
+
+namespace {
+
+thread_local std::string g_err;
+
+int fail(int code, const char* fmt, ...) {
+  char buf[512];
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(buf, sizeof(buf), fmt, ap);
+  va_end(ap);
+  g_err = buf;
+  return code;
+}
+
+int cuda_fail(cudaError_t e, const char* what) {
+  return fail(SA_ERR_CUDA, "%s: %s (%s)", what, cudaGetErrorName(e), cudaGetErrorString(e));
+}
+
+// ---------------------------------------------------------------- tensor maps
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                   const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                   const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                   CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn get_encode() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  });
+  return fn;
+}
+
+// View a [B, S, H, D] 16-bit tensor as 4-D (D, H, S, B); box = 64 elements x 1 head x
+// `rows` rows x 1 batch, 128-byte swizzle.  Rows past S read as zero.
+int make_map(CUtensorMap* m, const void* ptr, int dtype, int D, int H, int S, int B, int rows) {
+  EncodeTiledFn enc = get_encode();
+  if (!enc) return fail(SA_ERR_CUDA, "cuTensorMapEncodeTiled is not available from the driver");
+  cuuint64_t dims[4] = {(cuuint64_t)D, (cuuint64_t)H, (cuuint64_t)S, (cuuint64_t)B};
+  cuuint64_t strides[3] = {(cuuint64_t)D * 2, (cuuint64_t)H * D * 2, (cuuint64_t)S * H * D * 2};
+  cuuint32_t box[4] = {64, 1, (cuuint32_t)rows, 1};
+  cuuint32_t estr[4] = {1, 1, 1, 1};
+  CUresult r = enc(m, dtype == SA_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16,
+                   4, const_cast<void*>(ptr), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                   CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return fail(SA_ERR_CUDA, "cuTensorMapEncodeTiled failed (CUresult %d)", (int)r);
+  return SA_OK;
+}
+
+// ---------------------------------------------------------------- device facts
+int num_sms() {
+  static int cache[64] = {0};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 148;
+  if (!cache[dev]) {
+    int n = 0;
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) n = 148;
+    cache[dev] = n;
+  }
+  return cache[dev];
+}
+
+constexpr float kLog2e = 1.4426950408889634f;
+
+bool aligned16(const void* p) { return ((uintptr_t)p & 15u) == 0; }
+
+// Shared checks of the shape arguments.  Returns SA_OK or an error code.
+int check_dims(int B, int Sq, int Sk, int Hq, int Hkv, int D, int dtype, float scale) {
+  if (B < 0 || Sq < 0 || Sk < 0 || Hq < 0 || Hkv < 0)
+    return fail(SA_ERR_INVALID, "negative size (B=%d Sq=%d Sk=%d Hq=%d Hkv=%d)", B, Sq, Sk, Hq, Hkv);
+  if (Hq > 0 && (Hkv == 0 || Hq % Hkv != 0))
+    return fail(SA_ERR_INVALID, "Hq (%d) must be a positive multiple of Hkv (%d)", Hq, Hkv);
+  if (D != 64 && D != 128) return fail(SA_ERR_UNSUPPORTED, "head dim D=%d not supported (64 or 128)", D);
+  if (dtype != SA_FP16 && dtype != SA_BF16) return fail(SA_ERR_UNSUPPORTED, "unknown dtype %d", dtype);
+  if (!std::isfinite(scale)) return fail(SA_ERR_INVALID, "scale must be finite");
+  return SA_OK;
+}
+
+int check_ptrs(const void* q, const void* k, const void* v, const void* o, const void* lse) {
+  if (!q || !k || !v || !o) return fail(SA_ERR_INVALID, "q, k, v and o must be non-null");
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || (lse && !aligned16(lse)))
+    return fail(SA_ERR_INVALID, "tensor pointers must be 16-byte aligned");
+  return SA_OK;
+}
+
+int launch_fill(void* o, size_t n_o, float* lse, size_t n_lse, cudaStream_t st) {
+  size_t n = n_o > n_lse ? n_o : n_lse;
+  int blocks = (int)((n + 255) / 256);
+  if (blocks > 4 * num_sms()) blocks = 4 * num_sms();
+  if (blocks < 1) blocks = 1;
+  sa::attn_fill_empty<<<blocks, 256, 0, st>>>((uint16_t*)o, n_o, lse, n_lse);
+  cudaError_t e = cudaGetLastError();
+  return e == cudaSuccess ? SA_OK : cuda_fail(e, "fill launch");
+}
+
+template <int D, bool BF16>
+int launch_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Sq,
+               int Sk, int Hq, int Hkv, int causal, float scale, cudaStream_t st) {
+  using Cfg = sa::FwdCfg<D>;
+  CUtensorMap mq, mk, mv;
+  int rc;
+  if ((rc = make_map(&mq, q, BF16, D, Hq, Sq, B, 128)) != SA_OK) return rc;
+  if ((rc = make_map(&mk, k, BF16, D, Hkv, Sk, B, 128)) != SA_OK) return rc;
+  if ((rc = make_map(&mv, v, BF16, D, Hkv, Sk, B, 128)) != SA_OK) return rc;
+  sa::FwdParams p;
+  p.o = o; p.lse = lse;
+  p.B = B; p.Sq = Sq; p.Sk = Sk; p.Hq = Hq; p.Hkv = Hkv; p.causal = causal;
+  p.n_qblk = (Sq + 255) / 256;
+  long long units = (long long)B * Hq * p.n_qblk;
+  if (units > 0x7fffffffLL) return fail(SA_ERR_UNSUPPORTED, "too many work units (%lld)", units);
+  p.n_units = (int)units;
+  p.c2 = scale * kLog2e;
+  auto kern = sa::attn_fwd_sm100<D, BF16>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::SMEM_TOTAL);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(attn_fwd_sm100)");
+  int grid = p.n_units < num_sms() ? p.n_units : num_sms();
+  kern<<<grid, Cfg::THREADS, Cfg::SMEM_TOTAL, st>>>(mq, mk, mv, p);
+  e = cudaGetLastError();
+  return e == cudaSuccess ? SA_OK : cuda_fail(e, "attn_fwd_sm100 launch");
+}
+
+template <int D, bool BF16>
+int launch_simple(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Sq,
+                  int Sk, int Hq, int Hkv, int causal, float scale, cudaStream_t st) {
+  dim3 grid((Sq + 63) / 64, Hq, B);
+  if (grid.y > 65535 || grid.z > 65535) return fail(SA_ERR_UNSUPPORTED, "Hq or B too large for the simple kernel");
+  sa::attn_fwd_simple<D, BF16><<<grid, 64, 0, st>>>(q, k, v, o, lse, Sq, Sk, Hq, Hkv, causal, scale * kLog2e);
+  cudaError_t e = cudaGetLastError();
+  return e == cudaSuccess ? SA_OK : cuda_fail(e, "attn_fwd_simple launch");
+}
+
+// ---------------------------------------------------------------- decode planning
+struct DecPlan {
+  int nsplit, chunk, ngrp;
+};
+
+DecPlan plan_decode(int B, int Sk, int Hq, int Hkv, int num_splits, int sms) {
+  DecPlan pl;
+  const int G = Hq / Hkv;
+  pl.ngrp = (G + 15) / 16;
+  const long long groups = (long long)B * Hkv * pl.ngrp;
+  const int max_split = (Sk + 63) / 64;
+  long long want = num_splits > 0 ? num_splits : (2LL * sms + groups - 1) / groups;
+  if (want < 1) want = 1;
+  if (want > max_split) want = max_split;
+  int chunk = (int)((Sk + want - 1) / want);
+  chunk = (chunk + 63) / 64 * 64;
+  pl.chunk = chunk;
+  pl.nsplit = (Sk + chunk - 1) / chunk;
+  return pl;
+}
+
+template <int D, bool BF16>
+int launch_decode(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Sk,
+                  int Hq, int Hkv, float scale, const DecPlan& pl, void* ws, cudaStream_t st) {
+  using Cfg = sa::DecCfg<D>;
+  CUtensorMap mk, mv;
+  int rc;
+  if ((rc = make_map(&mk, k, BF16, D, Hkv, Sk, B, 64)) != SA_OK) return rc;
+  if ((rc = make_map(&mv, v, BF16, D, Hkv, Sk, B, 64)) != SA_OK) return rc;
+  sa::DecParams p;
+  p.q = q;
+  p.ws_o = reinterpret_cast<float*>(ws);
+  p.ws_ml = p.ws_o + (size_t)B * Hq * pl.nsplit * D;
+  p.o = o; p.lse = lse;
+  p.B = B; p.Sk = Sk; p.Hq = Hq; p.Hkv = Hkv; p.G = Hq / Hkv; p.ngrp = pl.ngrp;
+  p.nsplit = pl.nsplit; p.chunk = pl.chunk;
+  p.c2 = scale * kLog2e;
+  dim3 grid(pl.nsplit, Hkv * pl.ngrp, B);
+  if (grid.x > 0x7fffffffu || grid.y > 65535 || grid.z > 65535)
+    return fail(SA_ERR_UNSUPPORTED, "decode grid too large");
+  auto ks = sa::attn_decode_split<D, BF16>;
+  cudaError_t e = cudaFuncSetAttribute(ks, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::SMEM_TOTAL);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(attn_decode_split)");
+  ks<<<grid, 128, Cfg::SMEM_TOTAL, st>>>(mk, mv, p);
+  e = cudaGetLastError();
+  if (e != cudaSuccess) return cuda_fail(e, "attn_decode_split launch");
+  // combine: programmatic dependent launch, so it is resident and waiting when the
+  // split grid finishes
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)((B * Hq + 3) / 4));
+  cfg.blockDim = dim3(128);
+  cfg.dynamicSmemBytes = 0;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  e = cudaLaunchKernelEx(&cfg, sa::attn_decode_combine<D, BF16>, p);
+  return e == cudaSuccess ? SA_OK : cuda_fail(e, "attn_decode_combine launch");
+}
+
+}  // namespace
+
+extern "C" {
+
+int sa_attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Sq,
+                int Sk, int Hq, int Hkv, int D, int causal, float scale, int dtype, sa_stream_t stream) {
+  int rc = check_dims(B, Sq, Sk, Hq, Hkv, D, dtype, scale);
+  if (rc != SA_OK) return rc;
+  if (causal != 0 && causal != 1) return fail(SA_ERR_INVALID, "causal must be 0 or 1");
+  if (B == 0 || Sq == 0 || Hq == 0) return SA_OK;
+  if ((rc = check_ptrs(q, Sk ? k : q, Sk ? v : q, o, lse)) != SA_OK) return rc;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  if (Sk == 0) return launch_fill(o, (size_t)B * Sq * Hq * D, lse, (size_t)B * Hq * Sq, st);
+  const bool bf = dtype == SA_BF16;
+  if (D == 64) return bf ? launch_fwd<64, true>(q, k, v, o, lse, B, Sq, Sk, Hq, Hkv, causal, scale, st)
+                         : launch_fwd<64, false>(q, k, v, o, lse, B, Sq, Sk, Hq, Hkv, causal, scale, st);
+  return bf ? launch_fwd<128, true>(q, k, v, o, lse, B, Sq, Sk, Hq, Hkv, causal, scale, st)
+            : launch_fwd<128, false>(q, k, v, o, lse, B, Sq, Sk, Hq, Hkv, causal, scale, st);
+}
+
+int sa_attn_fwd_simple(const void* q, const void* k, const void* v, void* o, float* lse, int B,
+                       int Sq, int Sk, int Hq, int Hkv, int D, int causal, float scale, int dtype,
+                       sa_stream_t stream) {
+  int rc = check_dims(B, Sq, Sk, Hq, Hkv, D, dtype, scale);
+  if (rc != SA_OK) return rc;
+  if (causal != 0 && causal != 1) return fail(SA_ERR_INVALID, "causal must be 0 or 1");
+  if (B == 0 || Sq == 0 || Hq == 0) return SA_OK;
+  if ((rc = check_ptrs(q, Sk ? k : q, Sk ? v : q, o, lse)) != SA_OK) return rc;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  const bool bf = dtype == SA_BF16;
+  if (D == 64) return bf ? launch_simple<64, true>(q, k, v, o, lse, B, Sq, Sk, Hq, Hkv, causal, scale, st)
+                         : launch_simple<64, false>(q, k, v, o, lse, B, Sq, Sk, Hq, Hkv, causal, scale, st);
+  return bf ? launch_simple<128, true>(q, k, v, o, lse, B, Sq, Sk, Hq, Hkv, causal, scale, st)
+            : launch_simple<128, false>(q, k, v, o, lse, B, Sq, Sk, Hq, Hkv, causal, scale, st);
+}
+
+int sa_attn_decode_num_splits(int B, int Sk, int Hq, int Hkv, int D) {
+  if (check_dims(B, 1, Sk, Hq, Hkv, D, SA_FP16, 1.f) != SA_OK) return 0;
+  if (B == 0 || Hq == 0 || Sk == 0) return 1;
+  return plan_decode(B, Sk, Hq, Hkv, 0, num_sms()).nsplit;
+}
+
+size_t sa_attn_decode_workspace_size(int B, int Sk, int Hq, int Hkv, int D, int num_splits) {
+  if (num_splits < 0 || check_dims(B, 1, Sk, Hq, Hkv, D, SA_FP16, 1.f) != SA_OK) return 0;
+  if (B == 0 || Hq == 0 || Sk == 0) return 0;
+  DecPlan pl = plan_decode(B, Sk, Hq, Hkv, num_splits, num_sms());
+  return (size_t)B * Hq * pl.nsplit * (D + 2) * sizeof(float);
+}
+
+int sa_attn_decode(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Sk,
+                   int Hq, int Hkv, int D, float scale, int dtype, int num_splits, void* workspace,
+                   size_t workspace_bytes, sa_stream_t stream) {
+  int rc = check_dims(B, 1, Sk, Hq, Hkv, D, dtype, scale);
+  if (rc != SA_OK) return rc;
+  if (num_splits < 0) return fail(SA_ERR_INVALID, "num_splits must be >= 0");
+  if (B == 0 || Hq == 0) return SA_OK;
+  if ((rc = check_ptrs(q, Sk ? k : q, Sk ? v : q, o, lse)) != SA_OK) return rc;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  if (Sk == 0) return launch_fill(o, (size_t)B * Hq * D, lse, (size_t)B * Hq, st);
+  DecPlan pl = plan_decode(B, Sk, Hq, Hkv, num_splits, num_sms());
+  const size_t need = (size_t)B * Hq * pl.nsplit * (D + 2) * sizeof(float);
+  if (!workspace || workspace_bytes < need)
+    return fail(SA_ERR_WORKSPACE, "decode workspace of %zu bytes needed (got %zu)", need,
+                workspace ? workspace_bytes : (size_t)0);
+  if (!aligned16(workspace)) return fail(SA_ERR_INVALID, "workspace must be 16-byte aligned");
+  const bool bf = dtype == SA_BF16;
+  if (D == 64) return bf ? launch_decode<64, true>(q, k, v, o, lse, B, Sk, Hq, Hkv, scale, pl, workspace, st)
+                         : launch_decode<64, false>(q, k, v, o, lse, B, Sk, Hq, Hkv, scale, pl, workspace, st);
+  return bf ? launch_decode<128, true>(q, k, v, o, lse, B, Sk, Hq, Hkv, scale, pl, workspace, st)
+            : launch_decode<128, false>(q, k, v, o, lse, B, Sk, Hq, Hkv, scale, pl, workspace, st);
+}
+
+const char* sa_last_error(void) { return g_err.c_str(); }
+
+int sa_check_status(sa_stream_t stream) {
+  cudaError_t e = cudaStreamSynchronize(reinterpret_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "cudaStreamSynchronize");
+  int status = 0;
+  e = cudaMemcpyFromSymbol(&status, sa::g_status, sizeof(int));
+  if (e != cudaSuccess) return cuda_fail(e, "reading the device status word");
+  if (status != 0) {
+    const int zero = 0;
+    cudaMemcpyToSymbol(sa::g_status, &zero, sizeof(int));
+    return fail(SA_ERR_TIMEOUT, "a device wait expired (code %d, site %d)", status >> 16, status & 0xffff);
+  }
+  g_err.clear();
+  return SA_OK;
+}
+
+const char* sa_version(void) { return "0.1.0"; }
+
+}  // extern "C"

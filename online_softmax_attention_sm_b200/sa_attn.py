@@ -1,0 +1,156 @@
+"""Python binding of the ``sa_attn`` C ABI (``include/sa_attn.h``).
+
+Argument marshalling only: every step of the computation runs in the CUDA kernels of
+``libsa_attn.so``.  torch is used for device memory and the current stream.  The
+library must have been built (``online_softmax_attention_sm_b200.build``); if it is
+missing, loading raises -- there is no fallback path.
+"""
+from __future__ import annotations
+
+import ctypes
+import math
+import os
+
+import torch
+
+_LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libsa_attn.so")
+
+SA_OK, SA_ERR_INVALID, SA_ERR_UNSUPPORTED, SA_ERR_CUDA, SA_ERR_TIMEOUT, SA_ERR_WORKSPACE = 0, -1, -2, -3, -4, -5
+SA_FP16, SA_BF16 = 0, 1
+_DT = {torch.float16: SA_FP16, torch.bfloat16: SA_BF16}
+
+# exported symbol -> (restype, argtypes)
+_P, _I, _F, _Z = ctypes.c_void_p, ctypes.c_int, ctypes.c_float, ctypes.c_size_t
+SIGNATURES = {
+    "sa_attn_fwd": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _F, _I, _P]),
+    "sa_attn_fwd_simple": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _F, _I, _P]),
+    "sa_attn_decode_workspace_size": (_Z, [_I, _I, _I, _I, _I, _I]),
+    "sa_attn_decode_num_splits": (_I, [_I, _I, _I, _I, _I]),
+    "sa_attn_decode": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _F, _I, _I, _P, _Z, _P]),
+    "sa_last_error": (ctypes.c_char_p, []),
+    "sa_check_status": (_I, [_P]),
+    "sa_version": (ctypes.c_char_p, []),
+}
+
+_lib = None
+
+
+class SAError(RuntimeError):
+    def __init__(self, code, msg):
+        super().__init__(f"sa_attn error {code}: {msg}")
+        self.code = code
+
+
+def lib():
+    """The loaded C library (raises if it has not been built)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(_LIB_PATH):
+            raise ImportError(f"{_LIB_PATH} is missing: build it with "
+                              "`python -m online_softmax_attention_sm_b200.build`")
+        L = ctypes.CDLL(_LIB_PATH)
+        for name, (res, args) in SIGNATURES.items():
+            fn = getattr(L, name)
+            fn.restype = res
+            fn.argtypes = args
+        _lib = L
+    return _lib
+
+
+def _check(rc):
+    if rc != SA_OK:
+        raise SAError(rc, lib().sa_last_error().decode())
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream):
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream)
+
+
+def _check_tensor(name, t, dtype, device):
+    if t.dtype != dtype:
+        raise TypeError(f"{name}: dtype {t.dtype}, expected {dtype}")
+    if t.device != device:
+        raise ValueError(f"{name}: on {t.device}, expected {device}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+
+
+def sa_attn_fwd(q, k, v, causal=False, scale=None, out=None, lse=None, return_lse=True,
+                stream=None, simple=False):
+    """Attention forward.  q [B,Sq,Hq,D], k/v [B,Sk,Hkv,D] (fp16/bf16, CUDA, contiguous).
+    Returns (o [B,Sq,Hq,D], lse [B,Hq,Sq] fp32 or None)."""
+    B, Sq, Hq, D = q.shape
+    Sk, Hkv = k.shape[1], k.shape[2]
+    if k.shape != (B, Sk, Hkv, D) or v.shape != k.shape:
+        raise ValueError(f"shape mismatch q{tuple(q.shape)} k{tuple(k.shape)} v{tuple(v.shape)}")
+    if q.dtype not in _DT:
+        raise TypeError(f"unsupported dtype {q.dtype}")
+    for n, t in (("q", q), ("k", k), ("v", v)):
+        _check_tensor(n, t, q.dtype, q.device)
+    if scale is None:
+        scale = 1.0 / math.sqrt(D)
+    if out is None:
+        out = torch.empty_like(q)
+    _check_tensor("out", out, q.dtype, q.device)
+    if return_lse and lse is None:
+        lse = torch.empty((B, Hq, Sq), dtype=torch.float32, device=q.device)
+    if lse is not None:
+        _check_tensor("lse", lse, torch.float32, q.device)
+    fn = lib().sa_attn_fwd_simple if simple else lib().sa_attn_fwd
+    _check(fn(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse), B, Sq, Sk, Hq, Hkv, D,
+              int(bool(causal)), float(scale), _DT[q.dtype], _stream(stream)))
+    return out, lse
+
+
+def sa_attn_fwd_simple(q, k, v, causal=False, scale=None, **kw):
+    """The diagnostic CUDA-core forward (same contract as :func:`sa_attn_fwd`)."""
+    return sa_attn_fwd(q, k, v, causal, scale, simple=True, **kw)
+
+
+def sa_attn_decode_workspace_size(B, Sk, Hq, Hkv, D, num_splits=0):
+    return int(lib().sa_attn_decode_workspace_size(B, Sk, Hq, Hkv, D, num_splits))
+
+
+def sa_attn_decode_num_splits(B, Sk, Hq, Hkv, D):
+    return int(lib().sa_attn_decode_num_splits(B, Sk, Hq, Hkv, D))
+
+
+def sa_attn_decode(q, k, v, scale=None, num_splits=0, workspace=None, out=None, lse=None,
+                   return_lse=True, stream=None):
+    """Split-KV decode.  q [B,Hq,D], k/v [B,Sk,Hkv,D].  Returns (o [B,Hq,D], lse [B,Hq])."""
+    B, Hq, D = q.shape
+    Sk, Hkv = k.shape[1], k.shape[2]
+    if k.shape != (B, Sk, Hkv, D) or v.shape != k.shape:
+        raise ValueError(f"shape mismatch q{tuple(q.shape)} k{tuple(k.shape)} v{tuple(v.shape)}")
+    if q.dtype not in _DT:
+        raise TypeError(f"unsupported dtype {q.dtype}")
+    for n, t in (("q", q), ("k", k), ("v", v)):
+        _check_tensor(n, t, q.dtype, q.device)
+    if scale is None:
+        scale = 1.0 / math.sqrt(D)
+    if out is None:
+        out = torch.empty_like(q)
+    if return_lse and lse is None:
+        lse = torch.empty((B, Hq), dtype=torch.float32, device=q.device)
+    need = sa_attn_decode_workspace_size(B, Sk, Hq, Hkv, D, num_splits)
+    if workspace is None:
+        workspace = torch.empty(max(need, 16), dtype=torch.uint8, device=q.device)
+    _check(lib().sa_attn_decode(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse), B, Sk, Hq, Hkv, D,
+                                float(scale), _DT[q.dtype], int(num_splits), _ptr(workspace),
+                                workspace.numel() * workspace.element_size(), _stream(stream)))
+    return out, lse
+
+
+def sa_check_status(stream=None):
+    """Synchronise the stream and raise if a bounded device wait expired."""
+    _check(lib().sa_check_status(_stream(stream)))
+
+
+def sa_version():
+    return lib().sa_version().decode()

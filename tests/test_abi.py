@@ -1,0 +1,132 @@
+"""C-ABI checks that need no GPU: the library loads, exports every symbol the header
+declares, and rejects invalid arguments on the host before any device work."""
+import ctypes
+import math
+import os
+import re
+
+import pytest
+
+from online_softmax_attention_sm_b200 import build as build_mod
+from online_softmax_attention_sm_b200 import sa_attn as sa
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "sa_attn.h")
+
+
+@pytest.fixture(scope="module")
+def L():
+    build_mod.build()
+    return sa.lib()
+
+
+def header_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(sa_[a-z0-9_]+)\s*\(", text)))
+
+
+def test_header_declares_the_boundary():
+    names = header_functions()
+    for n in ("sa_attn_fwd", "sa_attn_decode", "sa_attn_decode_workspace_size", "sa_last_error",
+              "sa_check_status"):
+        assert n in names
+
+
+def test_every_declared_symbol_is_exported(L):
+    for n in header_functions():
+        assert hasattr(L, n), f"{n} declared in sa_attn.h but not exported"
+        assert n in sa.SIGNATURES, f"{n} has no binding signature"
+
+
+def test_binding_names_match_header():
+    assert set(sa.SIGNATURES) == set(header_functions())
+
+
+NULL = None
+FAKE = ctypes.c_void_p(1 << 20)          # 16-byte aligned, never dereferenced: checks fail first
+
+
+def fwd(L, q=FAKE, k=FAKE, v=FAKE, o=FAKE, lse=NULL, B=1, Sq=8, Sk=8, Hq=2, Hkv=2, D=64, causal=0,
+        scale=0.125, dtype=0):
+    return L.sa_attn_fwd(q, k, v, o, lse, B, Sq, Sk, Hq, Hkv, D, causal, scale, dtype, None)
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(q=NULL), sa.SA_ERR_INVALID),
+    (dict(o=NULL), sa.SA_ERR_INVALID),
+    (dict(k=NULL), sa.SA_ERR_INVALID),
+    (dict(B=-1), sa.SA_ERR_INVALID),
+    (dict(Sk=-3), sa.SA_ERR_INVALID),
+    (dict(Hq=3, Hkv=2), sa.SA_ERR_INVALID),
+    (dict(Hq=2, Hkv=0), sa.SA_ERR_INVALID),
+    (dict(D=96), sa.SA_ERR_UNSUPPORTED),
+    (dict(D=256), sa.SA_ERR_UNSUPPORTED),
+    (dict(dtype=7), sa.SA_ERR_UNSUPPORTED),
+    (dict(scale=math.nan), sa.SA_ERR_INVALID),
+    (dict(scale=math.inf), sa.SA_ERR_INVALID),
+    (dict(causal=2), sa.SA_ERR_INVALID),
+    (dict(q=ctypes.c_void_p((1 << 20) + 8)), sa.SA_ERR_INVALID),
+    (dict(lse=ctypes.c_void_p((1 << 20) + 4)), sa.SA_ERR_INVALID),
+])
+def test_fwd_rejects_invalid_arguments(L, kw, code):
+    assert fwd(L, **kw) == code
+    assert L.sa_last_error().decode() != ""
+    assert L.sa_attn_fwd_simple(*[kw.get(n, d) for n, d in
+                                  (("q", FAKE), ("k", FAKE), ("v", FAKE), ("o", FAKE), ("lse", NULL))],
+                                kw.get("B", 1), kw.get("Sq", 8), kw.get("Sk", 8), kw.get("Hq", 2),
+                                kw.get("Hkv", 2), kw.get("D", 64), kw.get("causal", 0),
+                                kw.get("scale", 0.125), kw.get("dtype", 0), None) == code
+
+
+@pytest.mark.parametrize("kw", [dict(B=0), dict(Sq=0), dict(Hq=0, Hkv=0), dict(Hq=0, Hkv=2)])
+def test_fwd_empty_problem_is_a_no_op(L, kw):
+    # nothing is launched, so null pointers are fine
+    assert fwd(L, q=NULL, k=NULL, v=NULL, o=NULL, **kw) == sa.SA_OK
+
+
+def dec(L, q=FAKE, k=FAKE, v=FAKE, o=FAKE, lse=NULL, B=1, Sk=64, Hq=2, Hkv=1, D=64, scale=0.125,
+        dtype=0, ns=0, ws=FAKE, wsb=1 << 30):
+    return L.sa_attn_decode(q, k, v, o, lse, B, Sk, Hq, Hkv, D, scale, dtype, ns, ws, wsb, None)
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(q=NULL), sa.SA_ERR_INVALID),
+    (dict(Hq=3, Hkv=2), sa.SA_ERR_INVALID),
+    (dict(D=32), sa.SA_ERR_UNSUPPORTED),
+    (dict(dtype=2), sa.SA_ERR_UNSUPPORTED),
+    (dict(ns=-1), sa.SA_ERR_INVALID),
+    (dict(scale=math.nan), sa.SA_ERR_INVALID),
+    (dict(ws=NULL), sa.SA_ERR_WORKSPACE),
+    (dict(wsb=16), sa.SA_ERR_WORKSPACE),
+    (dict(ws=ctypes.c_void_p((1 << 20) + 4)), sa.SA_ERR_INVALID),
+])
+def test_decode_rejects_invalid_arguments(L, kw, code):
+    assert dec(L, **kw) == code
+
+
+def test_decode_empty_is_a_no_op(L):
+    assert dec(L, q=NULL, k=NULL, v=NULL, o=NULL, B=0) == sa.SA_OK
+
+
+def test_workspace_size(L):
+    # explicit split counts: (D + 2) floats per (b, h, split)
+    assert L.sa_attn_decode_workspace_size(4, 32768, 14, 2, 64, 1) == 4 * 14 * 1 * 66 * 4
+    assert L.sa_attn_decode_workspace_size(4, 32768, 14, 2, 64, 8) == 4 * 14 * 8 * 66 * 4
+    # clamped to ceil(Sk / 64) splits
+    assert L.sa_attn_decode_workspace_size(1, 100, 2, 1, 128, 50) == 1 * 2 * 2 * 130 * 4
+    assert L.sa_attn_decode_workspace_size(1, 100, 3, 2, 64, 1) == 0      # invalid GQA
+    assert L.sa_attn_decode_workspace_size(0, 100, 2, 2, 64, 1) == 0      # empty
+    assert L.sa_attn_decode_num_splits(1, 100, 3, 2, 64) == 0
+    assert L.sa_attn_decode_num_splits(4, 32768, 14, 2, 64) >= 1
+
+
+def test_version(L):
+    assert re.fullmatch(r"\d+\.\d+\.\d+", sa.sa_version())
+
+
+def test_library_has_no_cpu_path():
+    # the package exposes no host-side compute: every entry point goes through the C ABI
+    import online_softmax_attention_sm_b200 as pkg
+    src = open(os.path.join(os.path.dirname(pkg.__file__), "sa_attn.py")).read()
+    assert "oracle" not in src and "scaled_dot_product" not in src and "softmax(" not in src
