@@ -1,0 +1,378 @@
+#!/usr/bin/env python
+"""Benchmark of the fused online-softmax attention hot path on B200.
+
+One step = one pass of the whole hot path over one batch of synthetic input:
+  * prefill: the 32768-token GQA causal forward (bf16, B=1, Hq=32, Hkv=8, D=128, K rows
+    0..3 scaled x8), sa_attn_fwd -> persistent tcgen05 kernel;
+  * decode: the 32768-token GQA split-KV decode (fp16, B=4, Hq=14, Hkv=2, D=64),
+    sa_attn_decode -> split kernel + combine kernel.
+value = prefill FLOPs (4*B*Hq*Sq*Sk*D/2, causal) per second of whole step, TFLOP/s.
+The decode's KV bandwidth is reported beside it ("decode"), timed with its own events.
+
+Multi-GPU (torchrun): every rank runs its own independent copy of the workload (the
+work units -- batches and heads -- are independent, so nothing is exchanged); value is
+the FLOPs of all ranks over the slowest rank's time ("scaling": "weak").
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference]
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+PREFILL = "gqa_causal_s32768_d128_bf16_sinks"
+DECODE = "gqa_decode_sk32768_d64_fp16"
+METRIC = "attn fwd TFLOP/s (prefill) and KV GB/s (decode) vs B200 roofline, 1 GPU"
+
+
+def dist_env():
+    return int(os.environ.get("RANK", "0")), int(os.environ.get("WORLD_SIZE", "1")), \
+        int(os.environ.get("LOCAL_RANK", "0"))
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return {"hbm_gbs": d["hbm_gbs"], "bf16_tflops": d["bf16_tflops"],
+                "bf16_tflops_sustained": d.get("bf16_tflops_sustained", d["bf16_tflops"]),
+                "source": "measured"}
+    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0,
+            "source": "fallback"}
+
+
+# ------------------------------------------------------------------ clocks
+class ClockSampler:
+    """nvidia-smi sampling of SM clocks and throttle reasons during the timed region."""
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index):
+        self.gpu = gpu_index
+        self.proc = None
+        self.path = None
+
+    def __enter__(self):
+        fd, self.path = tempfile.mkstemp(suffix=".csv")
+        os.close(fd)
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+            time.sleep(0.3)
+        except (OSError, FileNotFoundError):
+            self.proc = None
+        return self
+
+    def __exit__(self, *a):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+
+    def summary(self):
+        rows = []
+        if self.path and os.path.exists(self.path):
+            for line in open(self.path):
+                f = [x.strip() for x in line.split(",")]
+                if len(f) < 9:
+                    continue
+                try:
+                    rows.append((float(f[1]), float(f[2]), float(f[3]) if f[3] not in ("[N/A]", "N/A") else 0.0,
+                                 f[5], f[6], f[7], f[8]))
+                except ValueError:
+                    continue
+            os.unlink(self.path)
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"]}
+        load = [r for r in rows if r[2] > 200.0] or rows
+        reasons = set()
+        for r in load:
+            for name, val in zip(("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"),
+                                 r[3:]):
+                if val.lower().startswith("active"):
+                    reasons.add(name)
+        return {"sm_mhz": statistics.median(r[0] for r in load), "sm_max_mhz": max(r[1] for r in load),
+                "samples": len(load), "power_w_max": max(r[2] for r in load), "reasons": sorted(reasons)}
+
+
+# ------------------------------------------------------------------ CPU oracle baseline
+def oracle_prefill_sample(w, q, k, v, seconds, rng_seed=0, max_rows=None):
+    """Time the fp64 oracle on sampled query rows of the prefill workload for about
+    `seconds`; returns (flops done, elapsed s, description).  FLOPs per row follow the
+    forward convention: 4*D per visible key."""
+    import numpy as np
+    import oracle
+    # bf16/fp16 -> float32 is exact; the oracle widens to float64 itself
+    qn, kn, vn = (x.float().numpy() if hasattr(x, "float") else x for x in (q, k, v))
+    g = np.random.default_rng(rng_seed)
+    flops, rows_done, t0 = 0.0, 0, time.perf_counter()
+    while True:
+        h = int(g.integers(0, w.Hq))
+        rows = np.sort(g.choice(w.Sq, size=64, replace=False))
+        oracle.attention_rows(qn, kn, vn, w.scale, w.causal, 0, h, rows)
+        vis = (rows + 1 + (w.Sk - w.Sq)).clip(0, w.Sk) if w.causal else np.full(rows.size, w.Sk)
+        flops += 4.0 * w.D * float(vis.sum())
+        rows_done += rows.size
+        el = time.perf_counter() - t0
+        if el >= seconds or (max_rows and rows_done >= max_rows):
+            break
+    return flops, el, f"{rows_done} random query rows (64 per head draw) of {w.name}"
+
+
+def blas_threads():
+    try:
+        from threadpoolctl import threadpool_info
+        n = [i["num_threads"] for i in threadpool_info() if i.get("user_api") == "blas"]
+        return int(max(n)) if n else os.cpu_count()
+    except Exception:
+        return os.cpu_count()
+
+
+# ------------------------------------------------------------------ reference arm
+def run_reference(args):
+    rank, world, _ = dist_env()
+    if rank != 0:
+        return 0
+    import torch
+    from online_softmax_attention_sm_b200.inputs import make_workload_inputs
+    from online_softmax_attention_sm_b200.workloads import WORKLOADS
+    import oracle
+    wp, wd = WORKLOADS[PREFILL], WORKLOADS[DECODE]
+    q, k, v = (x.float().numpy() for x in make_workload_inputs(wp))
+    dq, dk, dv = make_workload_inputs(wd)
+    dqn, dkn, dvn = dq.double().numpy(), dk.double().numpy(), dv.double().numpy()
+    per_step = 2.0
+    times, flops_tot = [], 0.0
+    for i in range(args.warmup + args.steps):
+        t0 = time.perf_counter()
+        f, _, desc = oracle_prefill_sample(wp, q, k, v, per_step, rng_seed=i)
+        oracle.decode(dqn, dkn, dvn, wd.scale)
+        el = time.perf_counter() - t0
+        if i >= args.warmup:
+            times.append(el)
+            flops_tot += f
+    total = sum(times)
+    value = flops_tot / total / 1e12
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * total / args.steps,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic",
+        "config": {"workload": f"{PREFILL} (sampled rows) + {DECODE}", "parallelism": "none (CPU oracle)"},
+        "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": blas_threads(), "kind": "oracle",
+                         "sample": f"per step ~{per_step:.0f} s of {desc}, plus the full decode workload"},
+        "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# ------------------------------------------------------------------ our arm
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--cpu-seconds", type=float, default=12.0)
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--only", default="all", choices=["all", "prefill", "decode"],
+                    help="profiling aid: run only one half of the step (the JSON line is then partial)")
+    ap.add_argument("--prefill-seq", type=int, default=0,
+                    help="profiling aid: shorter prefill sequence (same heads, dtype, sinks)")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+    if args.impl == "reference":
+        return run_reference(args)
+
+    import numpy as np
+    import torch
+    import torch.distributed as dist
+    from online_softmax_attention_sm_b200 import (sa_attn_decode, sa_attn_decode_workspace_size,
+                                                   sa_attn_fwd, sa_check_status)
+    from online_softmax_attention_sm_b200.inputs import make_workload_inputs
+    from online_softmax_attention_sm_b200.workloads import WORKLOADS
+
+    rank, world, local = dist_env()
+    if world > 1:
+        torch.cuda.set_device(local)
+        from datetime import timedelta
+        dist.init_process_group("nccl", timeout=timedelta(seconds=120))
+    dev = torch.device("cuda", local if world > 1 else 0)
+    torch.cuda.set_device(dev)
+
+    wp, wd = WORKLOADS[PREFILL], WORKLOADS[DECODE]
+    if args.prefill_seq:
+        import dataclasses
+        wp = dataclasses.replace(wp, name=f"{wp.name}_seq{args.prefill_seq}", Sq=args.prefill_seq,
+                                 Sk=args.prefill_seq)
+    run_pre, run_dec = args.only in ("all", "prefill"), args.only in ("all", "decode")
+    q_h, k_h, v_h = make_workload_inputs(wp, seed=wp.seed + 1000 * rank)
+    dq_h, dk_h, dv_h = make_workload_inputs(wd, seed=wd.seed + 1000 * rank)
+    q, k, v = q_h.to(dev), k_h.to(dev), v_h.to(dev)
+    dq, dk, dv = dq_h.to(dev), dk_h.to(dev), dv_h.to(dev)
+    o = torch.empty_like(q)
+    lse = torch.empty((wp.B, wp.Hq, wp.Sq), dtype=torch.float32, device=dev)
+    do = torch.empty_like(dq)
+    dlse = torch.empty((wd.B, wd.Hq), dtype=torch.float32, device=dev)
+    ws = torch.empty(sa_attn_decode_workspace_size(wd.B, wd.Sk, wd.Hq, wd.Hkv, wd.D), dtype=torch.uint8,
+                     device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def step(ev=None):
+        if ev:
+            ev[0].record(stream)
+        if run_pre:
+            sa_attn_fwd(q, k, v, causal=True, scale=wp.scale, out=o, lse=lse, stream=stream)
+        if ev:
+            ev[1].record(stream)
+        if run_dec:
+            sa_attn_decode(dq, dk, dv, scale=wd.scale, workspace=ws, out=do, lse=dlse, stream=stream)
+        if ev:
+            ev[2].record(stream)
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+        torch.cuda.synchronize(dev)
+
+    for _ in range(args.warmup):
+        step()
+    sa_check_status(stream)
+
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(args.steps)]
+    t_start, t_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with ClockSampler(dev.index) as clk:
+        barrier()
+        t_start.record(stream)
+        for i in range(args.steps):
+            step(evs[i])
+        t_end.record(stream)
+        barrier()
+    sa_check_status(stream)
+    ms_total = t_start.elapsed_time(t_end)
+    pre_ms = [e[0].elapsed_time(e[1]) for e in evs]
+    dec_ms = [e[1].elapsed_time(e[2]) for e in evs]
+
+    # decode alone with a cold L2: a 2x-L2 scrub write between iterations, outside the events
+    scrub = torch.empty(2 * torch.cuda.get_device_properties(dev).L2_cache_size, dtype=torch.uint8, device=dev)
+    cold = []
+    for i in range(args.warmup + args.steps if run_dec else 0):
+        scrub.fill_(i & 0xFF)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        sa_attn_decode(dq, dk, dv, scale=wd.scale, workspace=ws, out=do, lse=dlse, stream=stream)
+        e1.record(stream)
+        if i >= args.warmup:
+            cold.append((e0, e1))
+    torch.cuda.synchronize(dev)
+    cold_ms = [a.elapsed_time(b) for a, b in cold] or [float("nan")]
+    del scrub
+
+    # e2e through the public API with host buffers: H2D of the step's inputs, D2H of outputs
+    e2e_ms = None
+    h2d = sum(t.numel() * t.element_size() for t in (q_h, k_h, v_h, dq_h, dk_h, dv_h))
+    d2h = sum(t.numel() * t.element_size() for t in (o, lse, do, dlse))
+    if not args.no_e2e:
+        pin = [t.pin_memory() for t in (q_h, k_h, v_h, dq_h, dk_h, dv_h)]
+        outs_h = [torch.empty(t.shape, dtype=t.dtype, pin_memory=True) for t in (o, lse, do, dlse)]
+
+        def e2e_step():
+            for src, dst in zip(pin, (q, k, v, dq, dk, dv)):
+                dst.copy_(src, non_blocking=True)
+            step()
+            for src, dst in zip((o, lse, do, dlse), outs_h):
+                dst.copy_(src, non_blocking=True)
+
+        for _ in range(3):
+            e2e_step()
+        barrier()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        n_e2e = max(3, args.steps // 2)
+        for _ in range(n_e2e):
+            e2e_step()
+        b.record(stream)
+        barrier()
+        e2e_ms = a.elapsed_time(b) / n_e2e
+        sa_check_status(stream)
+
+    def max_over_ranks(x):
+        if world == 1:
+            return x
+        t = torch.tensor([x], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        return float(t.item())
+
+    ms_step = max_over_ranks(ms_total / args.steps)
+    pre_avg = max_over_ranks(sum(pre_ms) / len(pre_ms))
+    dec_avg = max_over_ranks(sum(dec_ms) / len(dec_ms))
+    cold_avg = max_over_ranks(sum(cold_ms) / len(cold_ms))
+    e2e_ms = max_over_ranks(e2e_ms) if e2e_ms is not None else None
+
+    if rank == 0:
+        peaks = load_peaks()
+        value = world * wp.flops / (ms_step * 1e-3) / 1e12
+        pre_tf = wp.flops / (pre_avg * 1e-3) / 1e12
+        peak = peaks["bf16_tflops_sustained"]
+        dec_gbs_cold = wd.kv_bytes / (cold_avg * 1e-3) / 1e9
+        dec_gbs_step = wd.kv_bytes / (dec_avg * 1e-3) / 1e9
+        traffic = None
+        prof = os.path.join(ROOT, "profiles", "traffic.json")
+        if os.path.exists(prof):
+            traffic = json.load(open(prof)).get("attn_fwd_sm100")
+        line = {
+            "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_step,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+            "data": "synthetic",
+            "config": {"workload": f"{PREFILL} + {DECODE}",
+                       "prefill": {"B": wp.B, "Sq": wp.Sq, "Sk": wp.Sk, "Hq": wp.Hq, "Hkv": wp.Hkv, "D": wp.D,
+                                   "causal": True, "dtype": "bf16", "k_sink_rows": 4},
+                       "decode": {"B": wd.B, "Sk": wd.Sk, "Hq": wd.Hq, "Hkv": wd.Hkv, "D": wd.D, "dtype": "fp16"},
+                       "global_batch": wp.B * world, "seq_len": wp.Sq,
+                       "parallelism": f"independent replicas x{world}" if world > 1 else "single GPU",
+                       "l2": "prefill inputs+outputs (640 MB) exceed L2; decode timed alone after a 2xL2 scrub"},
+            "roofline": {"bound": "tensor", "kernel": "attn_fwd_sm100", "achieved": pre_tf, "peak": peak,
+                         "unit": "TFLOP/s", "frac": pre_tf / peak,
+                         "peak_source": f"{peaks['source']} bf16 cuBLAS, sustained (kernel runs inside a long loop)",
+                         "traffic": traffic},
+            "decode": {"value": dec_gbs_cold, "unit": "GB/s", "bound": "hbm", "peak": peaks["hbm_gbs"],
+                       "frac": dec_gbs_cold / peaks["hbm_gbs"], "us": cold_avg * 1e3, "l2": "cold (2xL2 scrub)",
+                       "in_step_gbs": dec_gbs_step, "kernels": "attn_decode_split + attn_decode_combine"},
+            "prefill_ms": pre_avg,
+            "gpu_launches": (int(run_pre) + 2 * int(run_dec)) * args.steps,
+            "clocks": clk.summary(),
+        }
+        if e2e_ms is not None:
+            line["e2e"] = {"value": world * wp.flops / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOP/s",
+                           "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms}
+        if world == 1 and args.cpu_seconds > 0:
+            f, el, desc = oracle_prefill_sample(wp, q_h, k_h, v_h, args.cpu_seconds)
+            line["cpu_baseline"] = {"value": f / el / 1e12, "unit": "TFLOP/s", "cores": blas_threads(),
+                                    "kind": "oracle", "sample": f"{desc}, {el:.1f} s"}
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -80,6 +80,13 @@ __device__ __forceinline__ uint32_t pack2(float lo, float hi) {
   }
 }
 
+template <bool BF16>
+__device__ __forceinline__ float unpack_sum(uint32_t v) {
+  if (BF16) return __uint_as_float(v << 16) + __uint_as_float(v & 0xffff0000u);
+  const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&v));
+  return f.x + f.y;
+}
+
 // Byte offset of (row, 16-byte column chunk) inside a 128-byte-swizzled box of 128-byte rows.
 __device__ __forceinline__ uint32_t sw128(int row, int chunk16) {
   return (uint32_t)(row * 128 + ((chunk16 ^ (row & 7)) << 4));
@@ -203,16 +210,17 @@ attn_decode_split(const __grid_constant__ CUtensorMap tm_k, const __grid_constan
       pr[n][0] = ex2(x[n][0] - u0); pr[n][1] = ex2(x[n][1] - u0);
       pr[n][2] = ex2(x[n][2] - u1); pr[n][3] = ex2(x[n][3] - u1);
     }
-    l0 = l0 * a0 + pr[0][0] + pr[0][1] + pr[1][0] + pr[1][1];
-    l1 = l1 * a1 + pr[0][2] + pr[0][3] + pr[1][2] + pr[1][3];
 #pragma unroll
     for (int n = 0; n < D / 8; ++n) { o[n][0] *= a0; o[n][1] *= a0; o[n][2] *= a1; o[n][3] *= a1; }
-    // P as the A operand (16 heads x 16 tokens)
+    // P as the A operand (16 heads x 16 tokens); the row sums add the rounded weights
+    // the MMA uses, so O / l stays an exact weighted average of V
     uint32_t pa[4];
     pa[0] = pack2<BF16>(pr[0][0], pr[0][1]);
     pa[1] = pack2<BF16>(pr[0][2], pr[0][3]);
     pa[2] = pack2<BF16>(pr[1][0], pr[1][1]);
     pa[3] = pack2<BF16>(pr[1][2], pr[1][3]);
+    l0 = l0 * a0 + unpack_sum<BF16>(pa[0]) + unpack_sum<BF16>(pa[2]);
+    l1 = l1 * a1 + unpack_sum<BF16>(pa[1]) + unpack_sum<BF16>(pa[3]);
     // ---- O (16 x D) += P V; V slice [16 tokens][D] via transposed ldmatrix
 #pragma unroll
     for (int n = 0; n < D / 8; n += 2) {

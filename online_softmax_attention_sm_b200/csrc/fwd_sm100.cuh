@@ -355,13 +355,17 @@ attn_fwd_sm100(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
               a = ex2(fmaf(s[c * 32 + 2 * i], c2, -m_use));
               b2 = ex2(fmaf(s[c * 32 + 2 * i + 1], c2, -m_use));
             }
-            rs += a + b2;
+            // the row sum adds the 16-bit weights the tensor core multiplies with, so
+            // O / l is an exact weighted average of V (no bias on one-key-dominated rows)
             if (BF16) {
               __nv_bfloat162 h2 = __floats2bfloat162_rn(a, b2);
               pk[i] = *reinterpret_cast<uint32_t*>(&h2);
+              rs += __uint_as_float(pk[i] << 16) + __uint_as_float(pk[i] & 0xffff0000u);
             } else {
               __half2 h2 = __floats2half2_rn(a, b2);
               pk[i] = *reinterpret_cast<uint32_t*>(&h2);
+              const float2 f = __half22float2(h2);
+              rs += f.x + f.y;
             }
           }
           tmem_st16(lane_addr + Cfg::P_COL(t) + c * 16, pk);

@@ -61,8 +61,16 @@ def test_fwd_zero_query_is_mean_of_values():
 
 
 def test_fwd_large_magnitudes_stay_finite():
-    # scores of several hundred: no overflow thanks to the running max
-    run_fwd_case(1, 600, 600, 2, 2, 128, True, "bf16", seed=6, in_scale=6.0)
+    # scores of several hundred: no overflow thanks to the running max.  Inputs are 6x the
+    # workloads' N(0,1), so |O| reaches ~20 and rounding O to bf16 alone costs up to half
+    # an ulp there (0.0625): the absolute tolerance scales with the values, here by 8.
+    q, k, v = make_qkv(1, 600, 600, 2, 2, 128, "bf16", seed=6, input_scale=6.0)
+    o, lse = sa_attn_fwd(q.to(dev()), k.to(dev()), v.to(dev()), causal=True)
+    sa_check_status()
+    O, L = oracle.attention(f64(q), f64(k), f64(v), 1 / math.sqrt(128), True)
+    assert np.all(np.isfinite(f64(o))) and np.all(np.isfinite(f64(lse)))
+    assert np.abs(f64(o) - O).max() <= 8e-2
+    assert np.abs(f64(lse) - L).max() <= 1e-3
 
 
 def test_fwd_causal_leak_bit_identical():
