@@ -72,10 +72,12 @@ int sa_attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse
                 float scale, int dtype, sa_stream_t stream);
 
 /*
- * Bytes of decode workspace needed for `num_splits` (0 = the automatic choice).  The
- * workspace holds, per (b, h, split), the split's unnormalised fp32 output row and its
- * running max and sum (StreamAttention page, "Engine Direction": partial online-softmax
- * states merged by a second kernel).  Returns 0 for empty problems or invalid sizes.
+ * Bytes of decode workspace needed for `num_splits` (0 = the automatic choice):
+ * B * Hq * splits * (D + 3) * 4.  The workspace holds, per (b, h, split), the split's
+ * unnormalised fp32 output row, its running max and two running sums (of the 16-bit
+ * weights the MMA used, and of the fp32 weights for the LSE) -- the partial
+ * online-softmax states of the StreamAttention page, "Engine Direction", merged by a
+ * second kernel.  Returns 0 for empty problems or invalid sizes.
  */
 size_t sa_attn_decode_workspace_size(int B, int Sk, int Hq, int Hkv, int D, int num_splits);
 

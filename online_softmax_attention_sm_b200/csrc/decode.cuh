@@ -33,14 +33,14 @@ struct DecCfg {
   static constexpr int KV_BYTES = KCH * CHUNK_BYTES;   // one K (or V) stage
   static constexpr int STAGES = (D == 64) ? 4 : 2;
   static constexpr int SMEM_STAGES = STAGES * 2 * KV_BYTES;
-  static constexpr int SMEM_MERGE = 4 * 16 * D * 4 + 2 * 4 * 16 * 4;
+  static constexpr int SMEM_MERGE = 4 * 16 * D * 4 + 3 * 4 * 16 * 4;
   static constexpr int SMEM_TOTAL = 1024 + (SMEM_STAGES > SMEM_MERGE ? SMEM_STAGES : SMEM_MERGE) + 256;
 };
 
 struct DecParams {
   const void* q;       // [B, Hq, D]
   float* ws_o;         // [B, Hq, nsplit, D]
-  float* ws_ml;        // [B, Hq, nsplit, 2]  (max in log2 units of c2*s, sum)
+  float* ws_ml;        // [B, Hq, nsplit, 3]: max (log2 units of c2*s), 16-bit-weight sum, fp32 sum
   void* o;             // [B, Hq, D]
   float* lse;          // [B, Hq] or null
   int B, Sk, Hq, Hkv, G, ngrp, nsplit, chunk;
@@ -157,7 +157,8 @@ attn_decode_split(const __grid_constant__ CUtensorMap tm_k, const __grid_constan
   float o[D / 8][4];
 #pragma unroll
   for (int n = 0; n < D / 8; ++n) o[n][0] = o[n][1] = o[n][2] = o[n][3] = 0.f;
-  float m0 = -INFINITY, m1 = -INFINITY, l0 = 0.f, l1 = 0.f;
+  // l: sums of the 16-bit weights (normalise O); e: sums of the fp32 weights (LSE)
+  float m0 = -INFINITY, m1 = -INFINITY, l0 = 0.f, l1 = 0.f, e0 = 0.f, e1 = 0.f;
   const float c2 = p.c2;
   const uint32_t smem_addr = smem_u32(smem);
   bool ok = true;
@@ -221,6 +222,8 @@ attn_decode_split(const __grid_constant__ CUtensorMap tm_k, const __grid_constan
     pa[3] = pack2<BF16>(pr[1][2], pr[1][3]);
     l0 = l0 * a0 + unpack_sum<BF16>(pa[0]) + unpack_sum<BF16>(pa[2]);
     l1 = l1 * a1 + unpack_sum<BF16>(pa[1]) + unpack_sum<BF16>(pa[3]);
+    e0 = e0 * a0 + pr[0][0] + pr[0][1] + pr[1][0] + pr[1][1];
+    e1 = e1 * a1 + pr[0][2] + pr[0][3] + pr[1][2] + pr[1][3];
     // ---- O (16 x D) += P V; V slice [16 tokens][D] via transposed ldmatrix
 #pragma unroll
     for (int n = 0; n < D / 8; n += 2) {
@@ -263,13 +266,19 @@ attn_decode_split(const __grid_constant__ CUtensorMap tm_k, const __grid_constan
   l0 += __shfl_xor_sync(0xffffffffu, l0, 2);
   l1 += __shfl_xor_sync(0xffffffffu, l1, 1);
   l1 += __shfl_xor_sync(0xffffffffu, l1, 2);
+  e0 += __shfl_xor_sync(0xffffffffu, e0, 1);
+  e0 += __shfl_xor_sync(0xffffffffu, e0, 2);
+  e1 += __shfl_xor_sync(0xffffffffu, e1, 1);
+  e1 += __shfl_xor_sync(0xffffffffu, e1, 2);
   float* sm_o = reinterpret_cast<float*>(smem);              // [4][16][D] (stages are drained)
   float* sm_m = sm_o + 4 * 16 * D;                           // [4][16]
   float* sm_l = sm_m + 64;                                   // [4][16]
+  float* sm_e = sm_l + 64;                                   // [4][16]
   const int r0 = lane >> 2, r1 = r0 + 8;
   if ((lane & 3) == 0) {
     sm_m[warp * 16 + r0] = m0; sm_m[warp * 16 + r1] = m1;
     sm_l[warp * 16 + r0] = l0; sm_l[warp * 16 + r1] = l1;
+    sm_e[warp * 16 + r0] = e0; sm_e[warp * 16 + r1] = e1;
   }
   __syncthreads();
   float M0 = -INFINITY, M1 = -INFINITY;
@@ -299,15 +308,18 @@ attn_decode_split(const __grid_constant__ CUtensorMap tm_k, const __grid_constan
     float M = -INFINITY;
 #pragma unroll
     for (int w = 0; w < 4; ++w) M = fmaxf(M, sm_m[w * 16 + r]);
-    float L = 0.f;
+    float L = 0.f, E = 0.f;
 #pragma unroll
     for (int w = 0; w < 4; ++w) {
       const float mw = sm_m[w * 16 + r];
-      L += (mw == -INFINITY) ? 0.f : sm_l[w * 16 + r] * ex2(mw - M);
+      const float sc = (mw == -INFINITY) ? 0.f : ex2(mw - M);
+      L += sm_l[w * 16 + r] * sc;
+      E += sm_e[w * 16 + r] * sc;
     }
-    float* ml = p.ws_ml + (ws_row0 + (size_t)r * p.nsplit) * 2;
+    float* ml = p.ws_ml + (ws_row0 + (size_t)r * p.nsplit) * 3;
     ml[0] = M;
     ml[1] = L;
+    ml[2] = E;
   }
 }
 
@@ -319,34 +331,35 @@ attn_decode_combine(const DecParams p) {
   const int gw = blockIdx.x * 4 + (threadIdx.x >> 5);
   const int lane = threadIdx.x & 31;
   if (gw >= p.B * p.Hq) return;
-  const float* ml = p.ws_ml + (size_t)gw * p.nsplit * 2;
+  const float* ml = p.ws_ml + (size_t)gw * p.nsplit * 3;
   const float* os = p.ws_o + (size_t)gw * p.nsplit * D;
   float M = -INFINITY;
-  for (int s = lane; s < p.nsplit; s += 32) M = fmaxf(M, ml[2 * s]);
+  for (int s = lane; s < p.nsplit; s += 32) M = fmaxf(M, ml[3 * s]);
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
-  constexpr int E = D / 32;                            // elements per lane
-  float acc[E];
+  constexpr int NE = D / 32;                           // elements per lane
+  float acc[NE];
 #pragma unroll
-  for (int e = 0; e < E; ++e) acc[e] = 0.f;
-  float L = 0.f;
+  for (int e = 0; e < NE; ++e) acc[e] = 0.f;
+  float L = 0.f, E = 0.f;
   for (int s = 0; s < p.nsplit; ++s) {
-    const float ms = ml[2 * s];
+    const float ms = ml[3 * s];
     const float w = (ms == -INFINITY) ? 0.f : ex2(ms - M);
-    L += w * ml[2 * s + 1];
+    L += w * ml[3 * s + 1];
+    E += w * ml[3 * s + 2];
 #pragma unroll
-    for (int e = 0; e < E; ++e) acc[e] += w * os[(size_t)s * D + lane * E + e];
+    for (int e = 0; e < NE; ++e) acc[e] += w * os[(size_t)s * D + lane * NE + e];
   }
   const float inv = L > 0.f ? 1.f / L : 0.f;
   using T = typename std::conditional<BF16, __nv_bfloat16, __half>::type;
-  T* out = reinterpret_cast<T*>(p.o) + (size_t)gw * D + lane * E;
+  T* out = reinterpret_cast<T*>(p.o) + (size_t)gw * D + lane * NE;
 #pragma unroll
-  for (int e = 0; e < E; e += 2) {
+  for (int e = 0; e < NE; e += 2) {
     uint32_t v = pack2<BF16>(acc[e] * inv, acc[e + 1] * inv);
     *reinterpret_cast<uint32_t*>(out + e) = v;
   }
   if (p.lse && lane == 0)
-    p.lse[gw] = L > 0.f ? (M + __log2f(L)) * 0.69314718055994531f : -INFINITY;
+    p.lse[gw] = E > 0.f ? (M + __log2f(E)) * 0.69314718055994531f : -INFINITY;
 }
 
 }  // namespace sa

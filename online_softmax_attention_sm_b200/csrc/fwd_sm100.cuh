@@ -206,53 +206,58 @@ attn_fwd_sm100(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
       constexpr uint32_t IDESC_PV = idesc_f16(BF16 ? 1 : 0, 128, D, 0, 1);
       const uint32_t sQ_addr = smem_u32(sQ);
       const uint32_t sRing_addr = smem_u32(sRing);
-      int slot = 0, ring_n = 0;
-      int q_uses[2] = {0, 0}, pv_n[2] = {0, 0};
+      int ring_n = 0;                       // ring position of this unit's first K tile
+      int q_use0 = 0, q_use1 = 0;           // Q tile loads consumed (q_full phases)
+      int pv0 = 0, pv1 = 0;                 // P_t V products issued (p_full phases)
       bool ok = true;
+      auto issue_qk = [&](int t, uint32_t k_addr) {
+        const uint32_t q_addr = sQ_addr + t * Cfg::TILE_BYTES;
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t off = (kk >> 2) * Cfg::CHUNK_BYTES + (kk & 3) * 32;
+          mma_ss(tmem_base + Cfg::S_COL(t), smem_desc_sw128(q_addr + off, 16, 1024),
+                 smem_desc_sw128(k_addr + off, 16, 1024), IDESC_QK, kk > 0);
+        }
+        mma_commit(&s_full[t]);
+      };
+      // Issue order per K/V step j:  PV_0(j), QK_0(j+1), PV_1(j), QK_1(j+1).
+      // P_t lives in S_t's tensor-memory columns; QK_t(j+1) overwrites them right after
+      // PV_t(j) read them.  tcgen05.mma instructions issued by one thread execute in
+      // issue order, so the overwrite cannot overtake the read, and each softmax
+      // warpgroup gets the other tile's PV + QK as cover for its exponentials.
       for (int round = 0; ok; ++round) {
         int u = fwd_unit_of(round, cta, ncta);
         if (u >= p.n_units) break;
         UnitInfo x = fwd_unit(p, u);
-        for (int j = 0; j < x.nkv_max && ok; ++j) {
-          // ---- S_t = Q_t K_j^T
-          ok = mbar_wait(&kv_full[slot], (ring_n / Cfg::STAGES) & 1, abort_flag, 10);
+        if (x.nkv_max == 0) continue;
+        const int base = ring_n;                 // K(j) at base + 2j, V(j) at base + 2j + 1
+        // ---- prologue: S_t = Q_t K_0^T
+        {
+          const int pos = base;
+          ok = mbar_wait(&kv_full[pos % Cfg::STAGES], (pos / Cfg::STAGES) & 1, abort_flag, 10);
           if (!ok) break;
-          const uint32_t k_addr = sRing_addr + slot * Cfg::TILE_BYTES;
-          for (int t = 0; t < 2; ++t) {
-            if (j >= x.nkv[t]) continue;
-            if (j == 0) {
-              ok = mbar_wait(&q_full[t], q_uses[t] & 1, abort_flag, 11);
-              if (!ok) break;
-            }
-            if (pv_n[t] > 0) {   // P_t lives over S_t: the previous P_t V must be done
-              ok = mbar_wait(&o_done[t], (pv_n[t] - 1) & 1, abort_flag, 12);
-              if (!ok) break;
-            }
+          const uint32_t k_addr = sRing_addr + (pos % Cfg::STAGES) * Cfg::TILE_BYTES;
+          for (int t = 0; t < 2 && ok; ++t) {
+            if (x.nkv[t] == 0) continue;
+            ok = mbar_wait(&q_full[t], (t ? q_use1 : q_use0) & 1, abort_flag, 11);
+            if (!ok) break;
             tc_fence_after();
-            const uint32_t q_addr = sQ_addr + t * Cfg::TILE_BYTES;
-#pragma unroll
-            for (int kk = 0; kk < D / 16; ++kk) {
-              const uint32_t off = (kk >> 2) * Cfg::CHUNK_BYTES + (kk & 3) * 32;
-              mma_ss(tmem_base + Cfg::S_COL(t), smem_desc_sw128(q_addr + off, 16, 1024),
-                     smem_desc_sw128(k_addr + off, 16, 1024), IDESC_QK, kk > 0);
-            }
-            mma_commit(&s_full[t]);
+            issue_qk(t, k_addr);
           }
           if (!ok) break;
-          mma_commit(&kv_empty[slot]);
-          ++ring_n;
-          slot = (slot + 1 == Cfg::STAGES) ? 0 : slot + 1;
-          if (j == x.nkv_max - 1) {
-            for (int t = 0; t < 2; ++t)
-              if (x.nkv[t] > 0) { mma_commit(&q_empty[t]); ++q_uses[t]; }
-          }
-          // ---- O_t += P_t V_j
-          ok = mbar_wait(&kv_full[slot], (ring_n / Cfg::STAGES) & 1, abort_flag, 13);
+          mma_commit(&kv_empty[pos % Cfg::STAGES]);
+        }
+        for (int j = 0; j < x.nkv_max && ok; ++j) {
+          const int vpos = base + 2 * j + 1, kpos = base + 2 * j + 2;
+          ok = mbar_wait(&kv_full[vpos % Cfg::STAGES], (vpos / Cfg::STAGES) & 1, abort_flag, 13);
           if (!ok) break;
-          const uint32_t v_addr = sRing_addr + slot * Cfg::TILE_BYTES;
+          const uint32_t v_addr = sRing_addr + (vpos % Cfg::STAGES) * Cfg::TILE_BYTES;
+          const uint32_t k_addr = sRing_addr + (kpos % Cfg::STAGES) * Cfg::TILE_BYTES;
+          bool k_ready = false;
           for (int t = 0; t < 2; ++t) {
             if (j >= x.nkv[t]) continue;
-            ok = mbar_wait(&p_full[t], (pv_n[t]) & 1, abort_flag, 14);
+            // ---- O_t += P_t V_j
+            ok = mbar_wait(&p_full[t], (t ? pv1 : pv0) & 1, abort_flag, 14);
             if (!ok) break;
             tc_fence_after();
 #pragma unroll
@@ -262,13 +267,32 @@ attn_fwd_sm100(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
                      (j > 0 || kk > 0) ? 1u : 0u);
             }
             mma_commit(&o_done[t]);
-            ++pv_n[t];
+            if (t) ++pv1; else ++pv0;
+            // ---- S_t = Q_t K_{j+1}^T
+            if (j + 1 < x.nkv[t]) {
+              if (!k_ready) {
+                ok = mbar_wait(&kv_full[kpos % Cfg::STAGES], (kpos / Cfg::STAGES) & 1, abort_flag, 10);
+                if (!ok) break;
+                k_ready = true;
+              }
+              issue_qk(t, k_addr);
+            }
           }
           if (!ok) break;
-          mma_commit(&kv_empty[slot]);
-          ++ring_n;
-          slot = (slot + 1 == Cfg::STAGES) ? 0 : slot + 1;
+          mma_commit(&kv_empty[vpos % Cfg::STAGES]);
+          if (j + 1 < x.nkv_max) {
+            if (!k_ready) {
+              // no Q tile needed K(j+1) (cannot happen: the tile with most K/V tiles does)
+              ok = mbar_wait(&kv_full[kpos % Cfg::STAGES], (kpos / Cfg::STAGES) & 1, abort_flag, 16);
+              if (!ok) break;
+            }
+            mma_commit(&kv_empty[kpos % Cfg::STAGES]);
+          }
         }
+        if (!ok) break;
+        ring_n = base + 2 * x.nkv_max;
+        if (x.nkv[0] > 0) { mma_commit(&q_empty[0]); ++q_use0; }
+        if (x.nkv[1] > 0) { mma_commit(&q_empty[1]); ++q_use1; }
       }
       // every MMA issued above completes before tensor memory is released
       mma_commit(fin_bar);
@@ -297,7 +321,9 @@ attn_fwd_sm100(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
       int kvis = p.Sk;                        // keys every row of the tile can see
       if (p.causal) kvis = min(kvis, max(0, r0 + p.Sk - p.Sq + 1));
       const int mask_from = kvis / 128;
-      float m_ref = -INFINITY, l_sum = 0.f;
+      // l_sum: sum of the 16-bit weights (normalises O, matching what the MMA multiplied);
+      // l_lse: sum of the fp32 weights (gives the LSE without the 16-bit rounding bias)
+      float m_ref = -INFINITY, l_sum = 0.f, l_lse = 0.f;
       for (int j = 0; j < nkv; ++j) {
         ok = __all_sync(0xffffffffu, mbar_wait(&s_full[t], s_n & 1, abort_flag, 20 + t));
         if (!ok) break;
@@ -338,10 +364,11 @@ attn_fwd_sm100(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
         if (need) {
           alpha = ex2(m_ref - m_tile);       // 0 when m_ref == -inf
           l_sum *= alpha;
+          l_lse *= alpha;
           m_ref = m_tile;
         }
         const float m_use = (m_ref == -INFINITY) ? 0.f : m_ref;
-        float rs = 0.f;
+        float rs = 0.f, rse = 0.f;
 #pragma unroll
         for (int c = 0; c < 4; ++c) {
           uint32_t pk[16];
@@ -357,6 +384,7 @@ attn_fwd_sm100(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
             }
             // the row sum adds the 16-bit weights the tensor core multiplies with, so
             // O / l is an exact weighted average of V (no bias on one-key-dominated rows)
+            rse += a + b2;
             if (BF16) {
               __nv_bfloat162 h2 = __floats2bfloat162_rn(a, b2);
               pk[i] = *reinterpret_cast<uint32_t*>(&h2);
@@ -371,6 +399,7 @@ attn_fwd_sm100(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
           tmem_st16(lane_addr + Cfg::P_COL(t) + c * 16, pk);
         }
         l_sum += rs;
+        l_lse += rse;
         // O_t holds P V up to tile j-1 (complete: S_t(j) was issued after it finished)
         if (j > 0 && __any_sync(0xffffffffu, need)) {
 #pragma unroll 1
@@ -428,7 +457,7 @@ attn_fwd_sm100(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
         }
       }
       if (store && p.lse) {
-        float lse = l_sum > 0.f ? (m_ref + __log2f(l_sum)) * 0.69314718055994531f : -INFINITY;
+        float lse = l_lse > 0.f ? (m_ref + __log2f(l_lse)) * 0.69314718055994531f : -INFINITY;
         p.lse[((size_t)x.b * p.Hq + x.h) * p.Sq + row] = lse;
       }
       tc_fence_before();

@@ -258,7 +258,7 @@ size_t sa_attn_decode_workspace_size(int B, int Sk, int Hq, int Hkv, int D, int 
   if (num_splits < 0 || check_dims(B, 1, Sk, Hq, Hkv, D, SA_FP16, 1.f) != SA_OK) return 0;
   if (B == 0 || Hq == 0 || Sk == 0) return 0;
   DecPlan pl = plan_decode(B, Sk, Hq, Hkv, num_splits, num_sms());
-  return (size_t)B * Hq * pl.nsplit * (D + 2) * sizeof(float);
+  return (size_t)B * Hq * pl.nsplit * (D + 3) * sizeof(float);
 }
 
 int sa_attn_decode(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Sk,
@@ -272,7 +272,7 @@ int sa_attn_decode(const void* q, const void* k, const void* v, void* o, float* 
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   if (Sk == 0) return launch_fill(o, (size_t)B * Hq * D, lse, (size_t)B * Hq, st);
   DecPlan pl = plan_decode(B, Sk, Hq, Hkv, num_splits, num_sms());
-  const size_t need = (size_t)B * Hq * pl.nsplit * (D + 2) * sizeof(float);
+  const size_t need = (size_t)B * Hq * pl.nsplit * (D + 3) * sizeof(float);
   if (!workspace || workspace_bytes < need)
     return fail(SA_ERR_WORKSPACE, "decode workspace of %zu bytes needed (got %zu)", need,
                 workspace ? workspace_bytes : (size_t)0);

@@ -72,7 +72,7 @@ def test_decode_workspace_contract():
     B, Sk, Hq, Hkv, D = 4, 32768, 14, 2, 64
     ns = sa_attn_decode_num_splits(B, Sk, Hq, Hkv, D)
     assert 1 <= ns <= Sk // 64
-    assert sa_attn_decode_workspace_size(B, Sk, Hq, Hkv, D) == B * Hq * ns * (D + 2) * 4
+    assert sa_attn_decode_workspace_size(B, Sk, Hq, Hkv, D) == B * Hq * ns * (D + 3) * 4
     q, k, v = make_qkv(B, 1, Sk, Hq, Hkv, D, "fp16", seed=25, decode=True)
     ws = torch.full((sa_attn_decode_workspace_size(B, Sk, Hq, Hkv, D) + 4096,), 0x5A,
                     dtype=torch.uint8, device=dev())
