@@ -323,42 +323,74 @@ attn_decode_split(const __grid_constant__ CUtensorMap tm_k, const __grid_constan
   }
 }
 
-// One warp per (batch, query head): O = sum_s w_s O_s / sum_s w_s l_s, w_s = 2^(m_s - M).
+// One 128-thread block per (batch, query head):
+//   M = max_s m_s,  w_s = 2^(m_s - M),  O = sum_s w_s O_s / sum_s w_s l_s,
+//   LSE = (M + log2 sum_s w_s e_s) * ln 2.
+// Thread t owns column d = t % D and the splits s = t / D, t / D + 128 / D, ...; the
+// (128 / D) partial sums per column are added through shared memory.
+constexpr int kCombineMaxSplits = 1024;
+
 template <int D, bool BF16>
 __global__ void __launch_bounds__(128)
 attn_decode_combine(const DecParams p) {
   asm volatile("griddepcontrol.wait;" ::: "memory");   // split results are complete
-  const int gw = blockIdx.x * 4 + (threadIdx.x >> 5);
-  const int lane = threadIdx.x & 31;
-  if (gw >= p.B * p.Hq) return;
+  __shared__ float s_w[kCombineMaxSplits];
+  __shared__ float s_red[2][4];
+  __shared__ float s_acc[128];
+  const int gw = blockIdx.x;                           // (b, h)
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const float* ml = p.ws_ml + (size_t)gw * p.nsplit * 3;
   const float* os = p.ws_o + (size_t)gw * p.nsplit * D;
+  const int ns = p.nsplit;
   float M = -INFINITY;
-  for (int s = lane; s < p.nsplit; s += 32) M = fmaxf(M, ml[3 * s]);
+  for (int s = tid; s < ns; s += 128) M = fmaxf(M, ml[3 * s]);
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
-  constexpr int NE = D / 32;                           // elements per lane
-  float acc[NE];
-#pragma unroll
-  for (int e = 0; e < NE; ++e) acc[e] = 0.f;
+  if (lane == 0) s_red[0][warp] = M;
+  __syncthreads();
+  M = fmaxf(fmaxf(s_red[0][0], s_red[0][1]), fmaxf(s_red[0][2], s_red[0][3]));
   float L = 0.f, E = 0.f;
-  for (int s = 0; s < p.nsplit; ++s) {
+  for (int s = tid; s < ns; s += 128) {
     const float ms = ml[3 * s];
     const float w = (ms == -INFINITY) ? 0.f : ex2(ms - M);
+    s_w[s] = w;
     L += w * ml[3 * s + 1];
     E += w * ml[3 * s + 2];
-#pragma unroll
-    for (int e = 0; e < NE; ++e) acc[e] += w * os[(size_t)s * D + lane * NE + e];
   }
-  const float inv = L > 0.f ? 1.f / L : 0.f;
-  using T = typename std::conditional<BF16, __nv_bfloat16, __half>::type;
-  T* out = reinterpret_cast<T*>(p.o) + (size_t)gw * D + lane * NE;
 #pragma unroll
-  for (int e = 0; e < NE; e += 2) {
-    uint32_t v = pack2<BF16>(acc[e] * inv, acc[e + 1] * inv);
-    *reinterpret_cast<uint32_t*>(out + e) = v;
+  for (int o = 16; o > 0; o >>= 1) {
+    L += __shfl_xor_sync(0xffffffffu, L, o);
+    E += __shfl_xor_sync(0xffffffffu, E, o);
   }
-  if (p.lse && lane == 0)
+  __syncthreads();                                     // s_red[0] reads done, s_w written
+  if (lane == 0) { s_red[0][warp] = L; s_red[1][warp] = E; }
+  __syncthreads();
+  L = (s_red[0][0] + s_red[0][1]) + (s_red[0][2] + s_red[0][3]);
+  E = (s_red[1][0] + s_red[1][1]) + (s_red[1][2] + s_red[1][3]);
+  constexpr int GRP = 128 / D;                         // threads per column
+  const int d = tid % D, g = tid / D;
+  float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;        // independent chains
+  int s = g;
+  for (; s + 3 * GRP < ns; s += 4 * GRP) {
+    a0 += s_w[s] * os[(size_t)s * D + d];
+    a1 += s_w[s + GRP] * os[(size_t)(s + GRP) * D + d];
+    a2 += s_w[s + 2 * GRP] * os[(size_t)(s + 2 * GRP) * D + d];
+    a3 += s_w[s + 3 * GRP] * os[(size_t)(s + 3 * GRP) * D + d];
+  }
+  for (; s < ns; s += GRP) a0 += s_w[s] * os[(size_t)s * D + d];
+  s_acc[tid] = (a0 + a1) + (a2 + a3);
+  __syncthreads();
+  if (tid < D) {
+    float acc = 0.f;
+#pragma unroll
+    for (int k = 0; k < GRP; ++k) acc += s_acc[k * D + tid];
+    const float inv = L > 0.f ? 1.f / L : 0.f;
+    using T = typename std::conditional<BF16, __nv_bfloat16, __half>::type;
+    T* out = reinterpret_cast<T*>(p.o) + (size_t)gw * D + tid;
+    if (BF16) *reinterpret_cast<__nv_bfloat16*>(out) = __float2bfloat16_rn(acc * inv);
+    else *reinterpret_cast<__half*>(out) = __float2half_rn(acc * inv);
+  }
+  if (p.lse && tid == 0)
     p.lse[gw] = E > 0.f ? (M + __log2f(E)) * 0.69314718055994531f : -INFINITY;
 }
 

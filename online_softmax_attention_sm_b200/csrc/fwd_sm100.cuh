@@ -13,10 +13,12 @@
 //   * warp 8 (one lane) issues TMA tensor loads: the two Q tiles once per unit, then
 //     K and V tiles into a ring of shared-memory slots (full/empty mbarriers);
 //   * warp 9 (one lane) issues tcgen05.mma: S_t = Q_t K^T (128x128, fp32 in tensor
-//     memory) and O_t += P_t V (P_t read from tensor memory, O_t fp32 in tensor memory);
+//     memory) and O_t += P_t V (P_t read from tensor memory, O_t fp32 in tensor memory),
+//     in the order PV_0(j), QK_0(j+1), PV_1(j), QK_1(j+1) so that each softmax
+//     warpgroup works while the tensor core serves the other Q tile;
 //   * warpgroups 0 and 1 run the softmax of Q tile 0 and 1: each thread owns one row of
 //     S (tcgen05.ld 32x32b), computes the row max, p = 2^(c*s - m) with c = scale*log2(e),
-//     the row sum, writes P as 16-bit into tensor memory over S, and rescales its O row
+//     the row sums, writes P as 16-bit into tensor memory over S, and rescales its O row
 //     only when the reference max moves by more than kRescaleThresh (exact after the
 //     final division; keeps p <= 2^kRescaleThresh);
 //   * the epilogue (same warpgroups) divides O by the row sum, rounds to the I/O dtype
@@ -44,6 +46,11 @@ struct FwdCfg {
   static constexpr int SMEM_BARS = 1024;
   static constexpr int SMEM_TOTAL = 1024 /*align slack*/ + SMEM_Q + SMEM_RING + SMEM_BARS;
   static constexpr int THREADS = 384;                // 2 softmax WGs + load/MMA WG
+  // per-thread registers after reallocation: softmax warpgroups / load+MMA warpgroup.
+  // 2*128*REGS_SOFTMAX + 128*REGS_OTHER must not exceed the block's launch registers
+  // (384 * registers per thread); the host checks this before launching.
+  static constexpr uint32_t REGS_SOFTMAX = 192;
+  static constexpr uint32_t REGS_OTHER = 120;
   static constexpr uint32_t TMEM_COLS = 512;
   // tensor-memory column map: S_t at 128 t, O_t at 256 + D t, P_t over S_t (16-bit)
   __host__ __device__ static constexpr uint32_t S_COL(int t) { return 128u * t; }
@@ -100,6 +107,395 @@ __device__ __forceinline__ int fwd_unit_of(int round, int cta, int ncta) {
   return round * ncta + ((round & 1) ? (ncta - 1 - cta) : cta);
 }
 
+// Shared-memory map: Q tiles, K/V ring, then the barriers and two words.
+template <int D>
+struct FwdSmem {
+  using Cfg = FwdCfg<D>;
+  uint8_t* q;          // [2][TILE]
+  uint8_t* ring;       // [STAGES][TILE]
+  uint64_t* kv_full;   // [STAGES]
+  uint64_t* kv_empty;  // [STAGES]
+  uint64_t* q_full;    // [2]
+  uint64_t* q_empty;   // [2]
+  uint64_t* s_full;    // [2]  S_t written (tcgen05.commit)
+  uint64_t* p_full;    // [2]  P_t written and O_t rescaled (128 softmax threads)
+  uint64_t* o_done;    // [2]  P_t V complete (tcgen05.commit)
+  uint64_t* fin;       // [1]  every MMA of this CTA complete
+  uint32_t* tmem_holder;
+  volatile int* abort_flag;
+  __device__ explicit FwdSmem(uint8_t* s) {
+    q = s;
+    ring = s + Cfg::SMEM_Q;
+    uint64_t* b = (uint64_t*)(s + Cfg::SMEM_Q + Cfg::SMEM_RING);
+    kv_full = b;
+    kv_empty = b + Cfg::STAGES;
+    q_full = b + 2 * Cfg::STAGES;
+    q_empty = q_full + 2;
+    s_full = q_full + 4;
+    p_full = q_full + 6;
+    o_done = q_full + 8;
+    fin = q_full + 10;
+    tmem_holder = (uint32_t*)(q_full + 12);
+    abort_flag = (volatile int*)(tmem_holder + 1);
+  }
+};
+
+// ------------------------------------------------------------------ TMA producer
+template <int D, bool BF16>
+__device__ __forceinline__ void fwd_producer(const CUtensorMap* tm_q, const CUtensorMap* tm_k,
+                                             const CUtensorMap* tm_v, const FwdParams& p,
+                                             const FwdSmem<D>& sm, int lane, int cta, int ncta) {
+  using Cfg = FwdCfg<D>;
+  if (lane == 0) {
+    int slot = 0, ring_n = 0;            // ring position and total loads issued
+    int q_load0 = 0, q_load1 = 0;        // Q tile loads issued
+    bool ok = true;
+    for (int round = 0; ok; ++round) {
+      int u = fwd_unit_of(round, cta, ncta);
+      if (u >= p.n_units) break;
+      UnitInfo x = fwd_unit(p, u);
+      for (int j = 0; j < x.nkv_max && ok; ++j) {
+        for (int kv = 0; kv < 2 && ok; ++kv) {
+          if (ring_n >= Cfg::STAGES) {
+            ok = mbar_wait(&sm.kv_empty[slot], ((ring_n / Cfg::STAGES) - 1) & 1, sm.abort_flag, 1);
+            if (!ok) break;
+          }
+          uint8_t* dst = sm.ring + slot * Cfg::TILE_BYTES;
+          mbar_arrive_expect_tx(&sm.kv_full[slot], Cfg::TILE_BYTES);
+          const CUtensorMap* tm = kv ? tm_v : tm_k;
+#pragma unroll
+          for (int c = 0; c < Cfg::KCH; ++c)
+            tma_load_4d(dst + c * Cfg::CHUNK_BYTES, tm, &sm.kv_full[slot], c * 64, x.kvh, j * 128, x.b);
+          ++ring_n;
+          slot = (slot + 1 == Cfg::STAGES) ? 0 : slot + 1;
+          if (j == 0 && kv == 0) {
+            // Q tiles after the first K tile, so K0 is in flight while Q waits for its slot
+            for (int t = 0; t < 2 && ok; ++t) {
+              if (x.nkv[t] == 0) continue;
+              int& ql = t ? q_load1 : q_load0;
+              if (ql > 0) {
+                ok = mbar_wait(&sm.q_empty[t], (ql - 1) & 1, sm.abort_flag, 2);
+                if (!ok) break;
+              }
+              uint8_t* qd = sm.q + t * Cfg::TILE_BYTES;
+              mbar_arrive_expect_tx(&sm.q_full[t], Cfg::TILE_BYTES);
+#pragma unroll
+              for (int c = 0; c < Cfg::KCH; ++c)
+                tma_load_4d(qd + c * Cfg::CHUNK_BYTES, tm_q, &sm.q_full[t], c * 64, x.h, x.q0 + t * 128, x.b);
+              ++ql;
+            }
+          }
+        }
+      }
+    }
+    if (!ok) {
+      // drain: every load issued must land before the CTA's shared memory goes away
+      // (each slot's most recent load is among the last STAGES issued)
+      int first = ring_n > Cfg::STAGES ? ring_n - Cfg::STAGES : 0;
+      for (int n = first; n < ring_n; ++n)
+        mbar_wait(&sm.kv_full[n % Cfg::STAGES], (n / Cfg::STAGES) & 1, nullptr, 3);
+      if (q_load0 > 0) mbar_wait(&sm.q_full[0], (q_load0 - 1) & 1, nullptr, 4);
+      if (q_load1 > 0) mbar_wait(&sm.q_full[1], (q_load1 - 1) & 1, nullptr, 4);
+    }
+  }
+  __syncwarp();
+}
+
+// ------------------------------------------------------------------ MMA issuer
+template <int D, bool BF16>
+__device__ __forceinline__ void fwd_mma(const FwdParams& p, const FwdSmem<D>& sm, uint32_t tmem_base,
+                                        int lane, int cta, int ncta) {
+  using Cfg = FwdCfg<D>;
+  if (lane == 0) {
+    constexpr uint32_t IDESC_QK = idesc_f16(BF16 ? 1 : 0, 128, 128, 0, 0);
+    constexpr uint32_t IDESC_PV = idesc_f16(BF16 ? 1 : 0, 128, D, 0, 1);
+    const uint32_t sQ_addr = smem_u32(sm.q);
+    const uint32_t sRing_addr = smem_u32(sm.ring);
+    int ring_n = 0;                       // ring position of this unit's first K tile
+    int q_use0 = 0, q_use1 = 0;           // Q tile loads consumed (q_full phases)
+    int pv0 = 0, pv1 = 0;                 // P_t V products issued (p_full phases)
+    bool ok = true;
+    auto issue_qk = [&](int t, uint32_t k_addr) {
+      const uint32_t q_addr = sQ_addr + t * Cfg::TILE_BYTES;
+#pragma unroll
+      for (int kk = 0; kk < D / 16; ++kk) {
+        const uint32_t off = (kk >> 2) * Cfg::CHUNK_BYTES + (kk & 3) * 32;
+        mma_ss(tmem_base + Cfg::S_COL(t), smem_desc_sw128(q_addr + off, 16, 1024),
+               smem_desc_sw128(k_addr + off, 16, 1024), IDESC_QK, kk > 0);
+      }
+      mma_commit(&sm.s_full[t]);
+    };
+    // Issue order per K/V step j:  PV_0(j), QK_0(j+1), PV_1(j), QK_1(j+1).
+    // P_t lives in S_t's tensor-memory columns; QK_t(j+1) overwrites them right after
+    // PV_t(j) read them.  tcgen05.mma instructions issued by one thread execute in
+    // issue order, so the overwrite cannot overtake the read, and each softmax
+    // warpgroup gets the other tile's PV + QK as cover for its exponentials.
+    for (int round = 0; ok; ++round) {
+      int u = fwd_unit_of(round, cta, ncta);
+      if (u >= p.n_units) break;
+      UnitInfo x = fwd_unit(p, u);
+      if (x.nkv_max == 0) continue;
+      const int base = ring_n;                 // K(j) at base + 2j, V(j) at base + 2j + 1
+      // ---- prologue: S_t = Q_t K_0^T
+      {
+        const int pos = base;
+        ok = mbar_wait(&sm.kv_full[pos % Cfg::STAGES], (pos / Cfg::STAGES) & 1, sm.abort_flag, 10);
+        if (!ok) break;
+        const uint32_t k_addr = sRing_addr + (pos % Cfg::STAGES) * Cfg::TILE_BYTES;
+        for (int t = 0; t < 2 && ok; ++t) {
+          if (x.nkv[t] == 0) continue;
+          ok = mbar_wait(&sm.q_full[t], (t ? q_use1 : q_use0) & 1, sm.abort_flag, 11);
+          if (!ok) break;
+          tc_fence_after();
+          issue_qk(t, k_addr);
+        }
+        if (!ok) break;
+        mma_commit(&sm.kv_empty[pos % Cfg::STAGES]);
+      }
+      for (int j = 0; j < x.nkv_max && ok; ++j) {
+        const int vpos = base + 2 * j + 1, kpos = base + 2 * j + 2;
+        ok = mbar_wait(&sm.kv_full[vpos % Cfg::STAGES], (vpos / Cfg::STAGES) & 1, sm.abort_flag, 13);
+        if (!ok) break;
+        const uint32_t v_addr = sRing_addr + (vpos % Cfg::STAGES) * Cfg::TILE_BYTES;
+        const uint32_t k_addr = sRing_addr + (kpos % Cfg::STAGES) * Cfg::TILE_BYTES;
+        bool k_ready = false;
+        for (int t = 0; t < 2; ++t) {
+          if (j >= x.nkv[t]) continue;
+          // ---- O_t += P_t V_j
+          ok = mbar_wait(&sm.p_full[t], (t ? pv1 : pv0) & 1, sm.abort_flag, 14);
+          if (!ok) break;
+          tc_fence_after();
+#pragma unroll
+          for (int kk = 0; kk < 128 / 16; ++kk) {
+            mma_ts(tmem_base + Cfg::O_COL(t), tmem_base + Cfg::P_COL(t) + kk * 8,
+                   smem_desc_sw128(v_addr + kk * 2048, Cfg::CHUNK_BYTES, 1024), IDESC_PV,
+                   (j > 0 || kk > 0) ? 1u : 0u);
+          }
+          mma_commit(&sm.o_done[t]);
+          if (t) ++pv1; else ++pv0;
+          // ---- S_t = Q_t K_{j+1}^T
+          if (j + 1 < x.nkv[t]) {
+            if (!k_ready) {
+              ok = mbar_wait(&sm.kv_full[kpos % Cfg::STAGES], (kpos / Cfg::STAGES) & 1, sm.abort_flag, 10);
+              if (!ok) break;
+              k_ready = true;
+            }
+            issue_qk(t, k_addr);
+          }
+        }
+        if (!ok) break;
+        mma_commit(&sm.kv_empty[vpos % Cfg::STAGES]);
+        if (j + 1 < x.nkv_max) {
+          if (!k_ready) {
+            // (cannot happen: the Q tile with the most K/V tiles needs K(j+1))
+            ok = mbar_wait(&sm.kv_full[kpos % Cfg::STAGES], (kpos / Cfg::STAGES) & 1, sm.abort_flag, 16);
+            if (!ok) break;
+          }
+          mma_commit(&sm.kv_empty[kpos % Cfg::STAGES]);
+        }
+      }
+      if (!ok) break;
+      ring_n = base + 2 * x.nkv_max;
+      if (x.nkv[0] > 0) { mma_commit(&sm.q_empty[0]); ++q_use0; }
+      if (x.nkv[1] > 0) { mma_commit(&sm.q_empty[1]); ++q_use1; }
+    }
+    // every MMA issued above completes before tensor memory is released
+    mma_commit(sm.fin);
+    mbar_wait(sm.fin, 0, nullptr, 15);
+  }
+  __syncwarp();
+}
+
+// ------------------------------------------------------------------ softmax + epilogue
+template <int D, bool BF16>
+__device__ __forceinline__ void fwd_softmax(const FwdParams& p, const FwdSmem<D>& sm, uint32_t tmem_base,
+                                            int warp, int lane, int cta, int ncta) {
+  using Cfg = FwdCfg<D>;
+  const int t = warp >> 2;                  // Q tile of this warpgroup
+  const int wl = warp & 3;                  // TMEM lane quarter
+  const int row_in_tile = wl * 32 + lane;
+  const uint32_t lane_addr = tmem_base + ((uint32_t)(wl * 32) << 16);
+  const float c2 = p.c2;
+  int s_n = 0, o_n = 0;                     // s_full / o_done phases consumed
+  bool ok = true;
+  for (int round = 0; ok; ++round) {
+    int u = fwd_unit_of(round, cta, ncta);
+    if (u >= p.n_units) break;
+    UnitInfo x = fwd_unit(p, u);
+    const int nkv = x.nkv[t];
+    const int row = x.q0 + t * 128 + row_in_tile;
+    int klim = p.Sk;
+    if (p.causal) klim = min(p.Sk, row + p.Sk - p.Sq + 1);
+    // the first key tile that any row of this Q tile must mask
+    const int r0 = x.q0 + t * 128;
+    int kvis = p.Sk;                        // keys every row of the tile can see
+    if (p.causal) kvis = min(kvis, max(0, r0 + p.Sk - p.Sq + 1));
+    const int mask_from = kvis / 128;
+    // l_sum: sum of the 16-bit weights (normalises O, matching what the MMA multiplied);
+    // l_lse: sum of the fp32 weights (gives the LSE without the 16-bit rounding bias)
+    float m_ref = -INFINITY, l_sum = 0.f, l_lse = 0.f;
+    for (int j = 0; j < nkv; ++j) {
+      ok = __all_sync(0xffffffffu, mbar_wait(&sm.s_full[t], s_n & 1, sm.abort_flag, 20 + t));
+      if (!ok) break;
+      ++s_n;
+      tc_fence_after();
+      float s[128];
+#pragma unroll
+      for (int c = 0; c < 4; ++c) {
+        uint32_t r[32];
+        tmem_ld32(lane_addr + Cfg::S_COL(t) + c * 32, r);
+#pragma unroll
+        for (int i = 0; i < 32; ++i) s[c * 32 + i] = __uint_as_float(r[i]);
+      }
+      tmem_wait_ld();
+      const bool masked = (j >= mask_from);
+      // row max as 8 independent chains (a single 128-long chain is latency-bound)
+      float mx[8];
+      if (masked) {
+        const int kl = klim - j * 128;     // keys >= kl are invisible to this row
+#pragma unroll
+        for (int i = 0; i < 128; ++i) s[i] = (i < kl) ? s[i] * c2 : -INFINITY;
+#pragma unroll
+        for (int k = 0; k < 8; ++k) mx[k] = s[k];
+#pragma unroll
+        for (int i = 8; i < 128; ++i) mx[i & 7] = fmaxf(mx[i & 7], s[i]);
+      } else if (c2 >= 0.f) {
+#pragma unroll
+        for (int k = 0; k < 8; ++k) mx[k] = s[k];
+#pragma unroll
+        for (int i = 8; i < 128; ++i) mx[i & 7] = fmaxf(mx[i & 7], s[i]);
+      } else {
+#pragma unroll
+        for (int k = 0; k < 8; ++k) mx[k] = s[k];
+#pragma unroll
+        for (int i = 8; i < 128; ++i) mx[i & 7] = fminf(mx[i & 7], s[i]);
+      }
+      float m_tile;
+      if (masked || c2 >= 0.f) {
+        m_tile = fmaxf(fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])),
+                       fmaxf(fmaxf(mx[4], mx[5]), fmaxf(mx[6], mx[7])));
+      } else {
+        m_tile = fminf(fminf(fminf(mx[0], mx[1]), fminf(mx[2], mx[3])),
+                       fminf(fminf(mx[4], mx[5]), fminf(mx[6], mx[7])));
+      }
+      if (!masked) m_tile *= c2;
+      // lazy rescale: move the reference max only when it grows by more than the threshold
+      const bool need = m_tile > m_ref + kRescaleThresh;
+      float alpha = 1.f;
+      if (need) {
+        alpha = ex2(m_ref - m_tile);       // 0 when m_ref == -inf
+        l_sum *= alpha;
+        l_lse *= alpha;
+        m_ref = m_tile;
+      }
+      const float m_use = (m_ref == -INFINITY) ? 0.f : m_ref;
+      float rs[4] = {0.f, 0.f, 0.f, 0.f}, rse[4] = {0.f, 0.f, 0.f, 0.f};   // 4 chains each
+#pragma unroll
+      for (int c = 0; c < 4; ++c) {
+        uint32_t pk[16];
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+          float a, b2;
+          if (masked) {
+            a = ex2(s[c * 32 + 2 * i] - m_use);
+            b2 = ex2(s[c * 32 + 2 * i + 1] - m_use);
+          } else {
+            a = ex2(fmaf(s[c * 32 + 2 * i], c2, -m_use));
+            b2 = ex2(fmaf(s[c * 32 + 2 * i + 1], c2, -m_use));
+          }
+          // the row sum adds the 16-bit weights the tensor core multiplies with, so
+          // O / l is an exact weighted average of V (no bias on one-key-dominated rows)
+          rse[i & 3] += a + b2;
+          if (BF16) {
+            __nv_bfloat162 h2 = __floats2bfloat162_rn(a, b2);
+            pk[i] = *reinterpret_cast<uint32_t*>(&h2);
+            rs[i & 3] += __uint_as_float(pk[i] << 16) + __uint_as_float(pk[i] & 0xffff0000u);
+          } else {
+            __half2 h2 = __floats2half2_rn(a, b2);
+            pk[i] = *reinterpret_cast<uint32_t*>(&h2);
+            const float2 f = __half22float2(h2);
+            rs[i & 3] += f.x + f.y;
+          }
+        }
+        tmem_st16(lane_addr + Cfg::P_COL(t) + c * 16, pk);
+      }
+      l_sum += (rs[0] + rs[1]) + (rs[2] + rs[3]);
+      l_lse += (rse[0] + rse[1]) + (rse[2] + rse[3]);
+      // O_t holds P V up to tile j-1, complete: S_t(j)'s commit covers every earlier MMA
+      if (j > 0 && __any_sync(0xffffffffu, need)) {
+#pragma unroll 1
+        for (int c = 0; c < D / 32; ++c) {
+          uint32_t r[32];
+          tmem_ld32(lane_addr + Cfg::O_COL(t) + c * 32, r);
+          tmem_wait_ld();
+#pragma unroll
+          for (int i = 0; i < 32; ++i) r[i] = __float_as_uint(__uint_as_float(r[i]) * alpha);
+          tmem_st32(lane_addr + Cfg::O_COL(t) + c * 32, r);
+        }
+      }
+      tmem_wait_st();
+      tc_fence_before();
+      mbar_arrive(&sm.p_full[t]);
+    }
+    if (!ok) break;
+    // ---------------- epilogue: O / l, LSE
+    if (nkv > 0) {
+      ok = __all_sync(0xffffffffu, mbar_wait(&sm.o_done[t], (o_n + nkv - 1) & 1, sm.abort_flag, 22 + t));
+      if (!ok) break;
+      o_n += nkv;
+      tc_fence_after();
+    }
+    const bool store = row < p.Sq;
+    const float inv_l = l_sum > 0.f ? 1.f / l_sum : 0.f;
+    using T = typename std::conditional<BF16, __nv_bfloat16, __half>::type;
+    T* orow = reinterpret_cast<T*>(p.o) + (((size_t)x.b * p.Sq + row) * p.Hq + x.h) * D;
+#pragma unroll 1
+    for (int c = 0; c < D / 32; ++c) {
+      uint32_t r[32];
+      if (nkv > 0) {
+        tmem_ld32(lane_addr + Cfg::O_COL(t) + c * 32, r);
+        tmem_wait_ld();
+      } else {
+#pragma unroll
+        for (int i = 0; i < 32; ++i) r[i] = 0u;
+      }
+      uint32_t pk[16];
+#pragma unroll
+      for (int i = 0; i < 16; ++i) {
+        float a = __uint_as_float(r[2 * i]) * inv_l, b2 = __uint_as_float(r[2 * i + 1]) * inv_l;
+        if (BF16) {
+          __nv_bfloat162 h2 = __floats2bfloat162_rn(a, b2);
+          pk[i] = *reinterpret_cast<uint32_t*>(&h2);
+        } else {
+          __half2 h2 = __floats2half2_rn(a, b2);
+          pk[i] = *reinterpret_cast<uint32_t*>(&h2);
+        }
+      }
+      if (store) {
+        uint4* dst = reinterpret_cast<uint4*>(orow + c * 32);
+#pragma unroll
+        for (int i = 0; i < 4; ++i) dst[i] = make_uint4(pk[4 * i], pk[4 * i + 1], pk[4 * i + 2], pk[4 * i + 3]);
+      }
+    }
+    if (store && p.lse) {
+      float lse = l_lse > 0.f ? (m_ref + __log2f(l_lse)) * 0.69314718055994531f : -INFINITY;
+      p.lse[((size_t)x.b * p.Hq + x.h) * p.Sq + row] = lse;
+    }
+    tc_fence_before();
+  }
+}
+
+// Every role ends here: one block-wide named barrier (id 1, all 384 threads), then the
+// warp that allocated tensor memory releases it.
+__device__ __forceinline__ void fwd_teardown(bool owner, uint32_t tmem_base, uint32_t ncols) {
+  tc_fence_before();
+  asm volatile("bar.sync 1, 384;" ::: "memory");
+  if (owner) {
+    tc_fence_after();
+    tmem_dealloc(tmem_base, ncols);
+  }
+}
+
 template <int D, bool BF16>
 __global__ void __launch_bounds__(384, 1)
 attn_fwd_sm100(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
@@ -107,37 +503,24 @@ attn_fwd_sm100(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
   using Cfg = FwdCfg<D>;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
-  uint8_t* sQ = smem;                                   // [2][TILE]
-  uint8_t* sRing = smem + Cfg::SMEM_Q;                  // [STAGES][TILE]
-  uint64_t* bars = (uint64_t*)(smem + Cfg::SMEM_Q + Cfg::SMEM_RING);
-  uint64_t* kv_full = bars;                             // [STAGES]
-  uint64_t* kv_empty = bars + Cfg::STAGES;              // [STAGES]
-  uint64_t* q_full = bars + 2 * Cfg::STAGES;            // [2]
-  uint64_t* q_empty = q_full + 2;                       // [2]
-  uint64_t* s_full = q_full + 4;                        // [2]
-  uint64_t* p_full = q_full + 6;                        // [2]
-  uint64_t* o_done = q_full + 8;                        // [2]
-  uint64_t* fin_bar = q_full + 10;                      // [1]
-  uint32_t* tmem_holder = (uint32_t*)(q_full + 12);
-  volatile int* abort_flag = (volatile int*)(tmem_holder + 1);
-
+  const FwdSmem<D> sm(smem);
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
   const int ncta = gridDim.x;
   const int cta = blockIdx.x;
 
   if (threadIdx.x == 0) {
-    for (int i = 0; i < Cfg::STAGES; ++i) { mbar_init(&kv_full[i], 1); mbar_init(&kv_empty[i], 1); }
+    for (int i = 0; i < Cfg::STAGES; ++i) { mbar_init(&sm.kv_full[i], 1); mbar_init(&sm.kv_empty[i], 1); }
     for (int t = 0; t < 2; ++t) {
-      mbar_init(&q_full[t], 1); mbar_init(&q_empty[t], 1);
-      mbar_init(&s_full[t], 1); mbar_init(&p_full[t], 128); mbar_init(&o_done[t], 1);
+      mbar_init(&sm.q_full[t], 1); mbar_init(&sm.q_empty[t], 1);
+      mbar_init(&sm.s_full[t], 1); mbar_init(&sm.p_full[t], 128); mbar_init(&sm.o_done[t], 1);
     }
-    mbar_init(fin_bar, 1);
-    *abort_flag = 0;
+    mbar_init(sm.fin, 1);
+    *sm.abort_flag = 0;
     fence_barrier_init();
   }
   if (warp == 9) {
-    tmem_alloc(tmem_holder, Cfg::TMEM_COLS);
+    tmem_alloc(sm.tmem_holder, Cfg::TMEM_COLS);
     tmem_relinquish();
   }
   if (warp == 8 && lane == 0) {
@@ -146,328 +529,19 @@ attn_fwd_sm100(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
-  const uint32_t tmem_base = *tmem_holder;
+  const uint32_t tmem_base = *sm.tmem_holder;
 
-  if (warp == 8) {
-    // ------------------------------------------------------------ TMA producer
-    if (lane == 0) {
-      int slot = 0, ring_n = 0;            // ring position and total loads issued
-      int q_loads[2] = {0, 0};
-      bool ok = true;
-      for (int round = 0; ok; ++round) {
-        int u = fwd_unit_of(round, cta, ncta);
-        if (u >= p.n_units) break;
-        UnitInfo x = fwd_unit(p, u);
-        for (int j = 0; j < x.nkv_max && ok; ++j) {
-          for (int kv = 0; kv < 2 && ok; ++kv) {
-            if (ring_n >= Cfg::STAGES) {
-              ok = mbar_wait(&kv_empty[slot], ((ring_n / Cfg::STAGES) - 1) & 1, abort_flag, 1);
-              if (!ok) break;
-            }
-            uint8_t* dst = sRing + slot * Cfg::TILE_BYTES;
-            mbar_arrive_expect_tx(&kv_full[slot], Cfg::TILE_BYTES);
-            const CUtensorMap* tm = kv ? &tm_v : &tm_k;
-            for (int c = 0; c < Cfg::KCH; ++c)
-              tma_load_4d(dst + c * Cfg::CHUNK_BYTES, tm, &kv_full[slot], c * 64, x.kvh, j * 128, x.b);
-            ++ring_n;
-            slot = (slot + 1 == Cfg::STAGES) ? 0 : slot + 1;
-            if (j == 0 && kv == 0) {
-              // Q tiles after the first K tile, so K0 is in flight while Q waits for its slot
-              for (int t = 0; t < 2 && ok; ++t) {
-                if (x.nkv[t] == 0) continue;
-                if (q_loads[t] > 0) {
-                  ok = mbar_wait(&q_empty[t], (q_loads[t] - 1) & 1, abort_flag, 2);
-                  if (!ok) break;
-                }
-                uint8_t* qd = sQ + t * Cfg::TILE_BYTES;
-                mbar_arrive_expect_tx(&q_full[t], Cfg::TILE_BYTES);
-                for (int c = 0; c < Cfg::KCH; ++c)
-                  tma_load_4d(qd + c * Cfg::CHUNK_BYTES, &tm_q, &q_full[t], c * 64, x.h, x.q0 + t * 128, x.b);
-                ++q_loads[t];
-              }
-            }
-          }
-        }
-      }
-      if (!ok) {
-        // drain: every load issued must land before the CTA's shared memory goes away
-        int first = ring_n > Cfg::STAGES ? ring_n - Cfg::STAGES : 0;
-        for (int n = first; n < ring_n; ++n)
-          mbar_wait(&kv_full[n % Cfg::STAGES], (n / Cfg::STAGES) & 1, nullptr, 3);
-        for (int t = 0; t < 2; ++t)
-          if (q_loads[t] > 0) mbar_wait(&q_full[t], (q_loads[t] - 1) & 1, nullptr, 4);
-      }
-    }
-    __syncwarp();
-  } else if (warp == 9) {
-    // ------------------------------------------------------------ MMA issuer
-    if (lane == 0) {
-      constexpr uint32_t IDESC_QK = idesc_f16(BF16 ? 1 : 0, 128, 128, 0, 0);
-      constexpr uint32_t IDESC_PV = idesc_f16(BF16 ? 1 : 0, 128, D, 0, 1);
-      const uint32_t sQ_addr = smem_u32(sQ);
-      const uint32_t sRing_addr = smem_u32(sRing);
-      int ring_n = 0;                       // ring position of this unit's first K tile
-      int q_use0 = 0, q_use1 = 0;           // Q tile loads consumed (q_full phases)
-      int pv0 = 0, pv1 = 0;                 // P_t V products issued (p_full phases)
-      bool ok = true;
-      auto issue_qk = [&](int t, uint32_t k_addr) {
-        const uint32_t q_addr = sQ_addr + t * Cfg::TILE_BYTES;
-#pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk) {
-          const uint32_t off = (kk >> 2) * Cfg::CHUNK_BYTES + (kk & 3) * 32;
-          mma_ss(tmem_base + Cfg::S_COL(t), smem_desc_sw128(q_addr + off, 16, 1024),
-                 smem_desc_sw128(k_addr + off, 16, 1024), IDESC_QK, kk > 0);
-        }
-        mma_commit(&s_full[t]);
-      };
-      // Issue order per K/V step j:  PV_0(j), QK_0(j+1), PV_1(j), QK_1(j+1).
-      // P_t lives in S_t's tensor-memory columns; QK_t(j+1) overwrites them right after
-      // PV_t(j) read them.  tcgen05.mma instructions issued by one thread execute in
-      // issue order, so the overwrite cannot overtake the read, and each softmax
-      // warpgroup gets the other tile's PV + QK as cover for its exponentials.
-      for (int round = 0; ok; ++round) {
-        int u = fwd_unit_of(round, cta, ncta);
-        if (u >= p.n_units) break;
-        UnitInfo x = fwd_unit(p, u);
-        if (x.nkv_max == 0) continue;
-        const int base = ring_n;                 // K(j) at base + 2j, V(j) at base + 2j + 1
-        // ---- prologue: S_t = Q_t K_0^T
-        {
-          const int pos = base;
-          ok = mbar_wait(&kv_full[pos % Cfg::STAGES], (pos / Cfg::STAGES) & 1, abort_flag, 10);
-          if (!ok) break;
-          const uint32_t k_addr = sRing_addr + (pos % Cfg::STAGES) * Cfg::TILE_BYTES;
-          for (int t = 0; t < 2 && ok; ++t) {
-            if (x.nkv[t] == 0) continue;
-            ok = mbar_wait(&q_full[t], (t ? q_use1 : q_use0) & 1, abort_flag, 11);
-            if (!ok) break;
-            tc_fence_after();
-            issue_qk(t, k_addr);
-          }
-          if (!ok) break;
-          mma_commit(&kv_empty[pos % Cfg::STAGES]);
-        }
-        for (int j = 0; j < x.nkv_max && ok; ++j) {
-          const int vpos = base + 2 * j + 1, kpos = base + 2 * j + 2;
-          ok = mbar_wait(&kv_full[vpos % Cfg::STAGES], (vpos / Cfg::STAGES) & 1, abort_flag, 13);
-          if (!ok) break;
-          const uint32_t v_addr = sRing_addr + (vpos % Cfg::STAGES) * Cfg::TILE_BYTES;
-          const uint32_t k_addr = sRing_addr + (kpos % Cfg::STAGES) * Cfg::TILE_BYTES;
-          bool k_ready = false;
-          for (int t = 0; t < 2; ++t) {
-            if (j >= x.nkv[t]) continue;
-            // ---- O_t += P_t V_j
-            ok = mbar_wait(&p_full[t], (t ? pv1 : pv0) & 1, abort_flag, 14);
-            if (!ok) break;
-            tc_fence_after();
-#pragma unroll
-            for (int kk = 0; kk < 128 / 16; ++kk) {
-              mma_ts(tmem_base + Cfg::O_COL(t), tmem_base + Cfg::P_COL(t) + kk * 8,
-                     smem_desc_sw128(v_addr + kk * 2048, Cfg::CHUNK_BYTES, 1024), IDESC_PV,
-                     (j > 0 || kk > 0) ? 1u : 0u);
-            }
-            mma_commit(&o_done[t]);
-            if (t) ++pv1; else ++pv0;
-            // ---- S_t = Q_t K_{j+1}^T
-            if (j + 1 < x.nkv[t]) {
-              if (!k_ready) {
-                ok = mbar_wait(&kv_full[kpos % Cfg::STAGES], (kpos / Cfg::STAGES) & 1, abort_flag, 10);
-                if (!ok) break;
-                k_ready = true;
-              }
-              issue_qk(t, k_addr);
-            }
-          }
-          if (!ok) break;
-          mma_commit(&kv_empty[vpos % Cfg::STAGES]);
-          if (j + 1 < x.nkv_max) {
-            if (!k_ready) {
-              // no Q tile needed K(j+1) (cannot happen: the tile with most K/V tiles does)
-              ok = mbar_wait(&kv_full[kpos % Cfg::STAGES], (kpos / Cfg::STAGES) & 1, abort_flag, 16);
-              if (!ok) break;
-            }
-            mma_commit(&kv_empty[kpos % Cfg::STAGES]);
-          }
-        }
-        if (!ok) break;
-        ring_n = base + 2 * x.nkv_max;
-        if (x.nkv[0] > 0) { mma_commit(&q_empty[0]); ++q_use0; }
-        if (x.nkv[1] > 0) { mma_commit(&q_empty[1]); ++q_use1; }
-      }
-      // every MMA issued above completes before tensor memory is released
-      mma_commit(fin_bar);
-      mbar_wait(fin_bar, 0, nullptr, 15);
-    }
-    __syncwarp();
-  } else if (warp < 8) {
-    // ------------------------------------------------------------ softmax / epilogue
-    const int t = warp >> 2;                  // Q tile of this warpgroup
-    const int wl = warp & 3;                  // TMEM lane quarter
-    const int row_in_tile = wl * 32 + lane;
-    const uint32_t lane_addr = tmem_base + ((uint32_t)(wl * 32) << 16);
-    const float c2 = p.c2;
-    int s_n = 0, o_n = 0;                     // s_full / o_done phases consumed
-    bool ok = true;
-    for (int round = 0; ok; ++round) {
-      int u = fwd_unit_of(round, cta, ncta);
-      if (u >= p.n_units) break;
-      UnitInfo x = fwd_unit(p, u);
-      const int nkv = x.nkv[t];
-      const int row = x.q0 + t * 128 + row_in_tile;
-      int klim = p.Sk;
-      if (p.causal) klim = min(p.Sk, row + p.Sk - p.Sq + 1);
-      // the first key tile that any row of this Q tile must mask
-      const int r0 = x.q0 + t * 128;
-      int kvis = p.Sk;                        // keys every row of the tile can see
-      if (p.causal) kvis = min(kvis, max(0, r0 + p.Sk - p.Sq + 1));
-      const int mask_from = kvis / 128;
-      // l_sum: sum of the 16-bit weights (normalises O, matching what the MMA multiplied);
-      // l_lse: sum of the fp32 weights (gives the LSE without the 16-bit rounding bias)
-      float m_ref = -INFINITY, l_sum = 0.f, l_lse = 0.f;
-      for (int j = 0; j < nkv; ++j) {
-        ok = __all_sync(0xffffffffu, mbar_wait(&s_full[t], s_n & 1, abort_flag, 20 + t));
-        if (!ok) break;
-        ++s_n;
-        tc_fence_after();
-        float s[128];
-#pragma unroll
-        for (int c = 0; c < 4; ++c) {
-          uint32_t r[32];
-          tmem_ld32(lane_addr + Cfg::S_COL(t) + c * 32, r);
-#pragma unroll
-          for (int i = 0; i < 32; ++i) s[c * 32 + i] = __uint_as_float(r[i]);
-        }
-        tmem_wait_ld();
-        const bool masked = (j >= mask_from);
-        float m_tile;
-        if (masked) {
-          const int kl = klim - j * 128;     // keys >= kl are invisible to this row
-#pragma unroll
-          for (int i = 0; i < 128; ++i) s[i] = (i < kl) ? s[i] * c2 : -INFINITY;
-          m_tile = s[0];
-#pragma unroll
-          for (int i = 1; i < 128; ++i) m_tile = fmaxf(m_tile, s[i]);
-        } else {
-          float mx = s[0];
-          if (c2 >= 0.f) {
-#pragma unroll
-            for (int i = 1; i < 128; ++i) mx = fmaxf(mx, s[i]);
-          } else {
-#pragma unroll
-            for (int i = 1; i < 128; ++i) mx = fminf(mx, s[i]);
-          }
-          m_tile = mx * c2;
-        }
-        // lazy rescale: move the reference max only when it grows by more than the threshold
-        const bool need = m_tile > m_ref + kRescaleThresh;
-        float alpha = 1.f;
-        if (need) {
-          alpha = ex2(m_ref - m_tile);       // 0 when m_ref == -inf
-          l_sum *= alpha;
-          l_lse *= alpha;
-          m_ref = m_tile;
-        }
-        const float m_use = (m_ref == -INFINITY) ? 0.f : m_ref;
-        float rs = 0.f, rse = 0.f;
-#pragma unroll
-        for (int c = 0; c < 4; ++c) {
-          uint32_t pk[16];
-#pragma unroll
-          for (int i = 0; i < 16; ++i) {
-            float a, b2;
-            if (masked) {
-              a = ex2(s[c * 32 + 2 * i] - m_use);
-              b2 = ex2(s[c * 32 + 2 * i + 1] - m_use);
-            } else {
-              a = ex2(fmaf(s[c * 32 + 2 * i], c2, -m_use));
-              b2 = ex2(fmaf(s[c * 32 + 2 * i + 1], c2, -m_use));
-            }
-            // the row sum adds the 16-bit weights the tensor core multiplies with, so
-            // O / l is an exact weighted average of V (no bias on one-key-dominated rows)
-            rse += a + b2;
-            if (BF16) {
-              __nv_bfloat162 h2 = __floats2bfloat162_rn(a, b2);
-              pk[i] = *reinterpret_cast<uint32_t*>(&h2);
-              rs += __uint_as_float(pk[i] << 16) + __uint_as_float(pk[i] & 0xffff0000u);
-            } else {
-              __half2 h2 = __floats2half2_rn(a, b2);
-              pk[i] = *reinterpret_cast<uint32_t*>(&h2);
-              const float2 f = __half22float2(h2);
-              rs += f.x + f.y;
-            }
-          }
-          tmem_st16(lane_addr + Cfg::P_COL(t) + c * 16, pk);
-        }
-        l_sum += rs;
-        l_lse += rse;
-        // O_t holds P V up to tile j-1 (complete: S_t(j) was issued after it finished)
-        if (j > 0 && __any_sync(0xffffffffu, need)) {
-#pragma unroll 1
-          for (int c = 0; c < D / 32; ++c) {
-            uint32_t r[32];
-            tmem_ld32(lane_addr + Cfg::O_COL(t) + c * 32, r);
-            tmem_wait_ld();
-#pragma unroll
-            for (int i = 0; i < 32; ++i) r[i] = __float_as_uint(__uint_as_float(r[i]) * alpha);
-            tmem_st32(lane_addr + Cfg::O_COL(t) + c * 32, r);
-          }
-        }
-        tmem_wait_st();
-        tc_fence_before();
-        mbar_arrive(&p_full[t]);
-      }
-      if (!ok) break;
-      // ---------------- epilogue: O / l, LSE
-      if (nkv > 0) {
-        ok = __all_sync(0xffffffffu, mbar_wait(&o_done[t], (o_n + nkv - 1) & 1, abort_flag, 22 + t));
-        if (!ok) break;
-        o_n += nkv;
-        tc_fence_after();
-      }
-      const bool store = row < p.Sq;
-      const float inv_l = l_sum > 0.f ? 1.f / l_sum : 0.f;
-      using T = typename std::conditional<BF16, __nv_bfloat16, __half>::type;
-      T* orow = reinterpret_cast<T*>(p.o) + (((size_t)x.b * p.Sq + row) * p.Hq + x.h) * D;
-#pragma unroll 1
-      for (int c = 0; c < D / 32; ++c) {
-        uint32_t r[32];
-        if (nkv > 0) {
-          tmem_ld32(lane_addr + Cfg::O_COL(t) + c * 32, r);
-          tmem_wait_ld();
-        } else {
-#pragma unroll
-          for (int i = 0; i < 32; ++i) r[i] = 0u;
-        }
-        uint32_t pk[16];
-#pragma unroll
-        for (int i = 0; i < 16; ++i) {
-          float a = __uint_as_float(r[2 * i]) * inv_l, b2 = __uint_as_float(r[2 * i + 1]) * inv_l;
-          if (BF16) {
-            __nv_bfloat162 h2 = __floats2bfloat162_rn(a, b2);
-            pk[i] = *reinterpret_cast<uint32_t*>(&h2);
-          } else {
-            __half2 h2 = __floats2half2_rn(a, b2);
-            pk[i] = *reinterpret_cast<uint32_t*>(&h2);
-          }
-        }
-        if (store) {
-          uint4* dst = reinterpret_cast<uint4*>(orow + c * 32);
-#pragma unroll
-          for (int i = 0; i < 4; ++i) dst[i] = make_uint4(pk[4 * i], pk[4 * i + 1], pk[4 * i + 2], pk[4 * i + 3]);
-        }
-      }
-      if (store && p.lse) {
-        float lse = l_lse > 0.f ? (m_ref + __log2f(l_lse)) * 0.69314718055994531f : -INFINITY;
-        p.lse[((size_t)x.b * p.Hq + x.h) * p.Sq + row] = lse;
-      }
-      tc_fence_before();
-    }
+  if (warp >= 8) {
+    // load / MMA warpgroup (warps 10 and 11 have no role) gives registers away
+    regs_dec<Cfg::REGS_OTHER>();
+    if (warp == 8) fwd_producer<D, BF16>(&tm_q, &tm_k, &tm_v, p, sm, lane, cta, ncta);
+    else if (warp == 9) fwd_mma<D, BF16>(p, sm, tmem_base, lane, cta, ncta);
+    fwd_teardown(warp == 9, tmem_base, Cfg::TMEM_COLS);
+  } else {
+    regs_inc<Cfg::REGS_SOFTMAX>();
+    fwd_softmax<D, BF16>(p, sm, tmem_base, warp, lane, cta, ncta);
+    fwd_teardown(false, tmem_base, Cfg::TMEM_COLS);
   }
-  // warps 10, 11 have no role
-  tc_fence_before();
-  __syncthreads();
-  tc_fence_after();
-  if (warp == 9) tmem_dealloc(tmem_base, Cfg::TMEM_COLS);
 }
 
 }  // namespace sa

@@ -134,6 +134,14 @@ int launch_fwd(const void* q, const void* k, const void* v, void* o, float* lse,
   auto kern = sa::attn_fwd_sm100<D, BF16>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::SMEM_TOTAL);
   if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(attn_fwd_sm100)");
+  // the in-kernel register reallocation must fit in what the block is launched with,
+  // otherwise the increasing warpgroups would wait forever
+  cudaFuncAttributes fa;
+  e = cudaFuncGetAttributes(&fa, kern);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaFuncGetAttributes(attn_fwd_sm100)");
+  if ((long long)fa.numRegs * Cfg::THREADS < 256LL * Cfg::REGS_SOFTMAX + 128LL * Cfg::REGS_OTHER)
+    return fail(SA_ERR_UNSUPPORTED, "attn_fwd_sm100 launches with %d registers per thread, too few for "
+                "its register split", fa.numRegs);
   int grid = p.n_units < num_sms() ? p.n_units : num_sms();
   kern<<<grid, Cfg::THREADS, Cfg::SMEM_TOTAL, st>>>(mq, mk, mv, p);
   e = cudaGetLastError();
@@ -160,7 +168,8 @@ DecPlan plan_decode(int B, int Sk, int Hq, int Hkv, int num_splits, int sms) {
   const int G = Hq / Hkv;
   pl.ngrp = (G + 15) / 16;
   const long long groups = (long long)B * Hkv * pl.ngrp;
-  const int max_split = (Sk + 63) / 64;
+  int max_split = (Sk + 63) / 64;
+  if (max_split > sa::kCombineMaxSplits) max_split = sa::kCombineMaxSplits;
   long long want = num_splits > 0 ? num_splits : (2LL * sms + groups - 1) / groups;
   if (want < 1) want = 1;
   if (want > max_split) want = max_split;
@@ -188,7 +197,7 @@ int launch_decode(const void* q, const void* k, const void* v, void* o, float* l
   p.nsplit = pl.nsplit; p.chunk = pl.chunk;
   p.c2 = scale * kLog2e;
   dim3 grid(pl.nsplit, Hkv * pl.ngrp, B);
-  if (grid.x > 0x7fffffffu || grid.y > 65535 || grid.z > 65535)
+  if ((long long)B * Hq > 0x7fffffffLL || grid.y > 65535 || grid.z > 65535)
     return fail(SA_ERR_UNSUPPORTED, "decode grid too large");
   auto ks = sa::attn_decode_split<D, BF16>;
   cudaError_t e = cudaFuncSetAttribute(ks, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::SMEM_TOTAL);
@@ -199,7 +208,7 @@ int launch_decode(const void* q, const void* k, const void* v, void* o, float* l
   // combine: programmatic dependent launch, so it is resident and waiting when the
   // split grid finishes
   cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3((unsigned)((B * Hq + 3) / 4));
+  cfg.gridDim = dim3((unsigned)(B * Hq));
   cfg.blockDim = dim3(128);
   cfg.dynamicSmemBytes = 0;
   cfg.stream = st;
