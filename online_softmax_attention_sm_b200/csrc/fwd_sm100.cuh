@@ -349,36 +349,31 @@ __device__ __forceinline__ void fwd_softmax(const FwdParams& p, const FwdSmem<D>
       }
       tmem_wait_ld();
       const bool masked = (j >= mask_from);
-      // row max as 8 independent chains (a single 128-long chain is latency-bound)
-      float mx[8];
-      if (masked) {
-        const int kl = klim - j * 128;     // keys >= kl are invisible to this row
+      const bool fast = !masked && c2 >= 0.f;      // the common case: full tile, scale >= 0
+      float m_tile;
+      if (fast) {
+        // row max: 8 independent chains of 3-input max over 16 values each
+        float mx[8];
+#pragma unroll
+        for (int k = 0; k < 8; ++k) mx[k] = fmaxf(s[k], s[k + 8]);
+#pragma unroll
+        for (int i = 16; i < 128; i += 16)
+#pragma unroll
+          for (int k = 0; k < 8; ++k) mx[k] = max3f(mx[k], s[i + k], s[i + 8 + k]);
+        m_tile = fmaxf(max3f(mx[0], mx[1], mx[2]), max3f(max3f(mx[3], mx[4], mx[5]), mx[6], mx[7])) * c2;
+      } else {
+        // diagonal / ragged tiles (and negative scales): scale first, mask, then max
+        const int kl = masked ? klim - j * 128 : 128;   // keys >= kl are invisible to this row
 #pragma unroll
         for (int i = 0; i < 128; ++i) s[i] = (i < kl) ? s[i] * c2 : -INFINITY;
+        float mx[8];
 #pragma unroll
         for (int k = 0; k < 8; ++k) mx[k] = s[k];
 #pragma unroll
         for (int i = 8; i < 128; ++i) mx[i & 7] = fmaxf(mx[i & 7], s[i]);
-      } else if (c2 >= 0.f) {
-#pragma unroll
-        for (int k = 0; k < 8; ++k) mx[k] = s[k];
-#pragma unroll
-        for (int i = 8; i < 128; ++i) mx[i & 7] = fmaxf(mx[i & 7], s[i]);
-      } else {
-#pragma unroll
-        for (int k = 0; k < 8; ++k) mx[k] = s[k];
-#pragma unroll
-        for (int i = 8; i < 128; ++i) mx[i & 7] = fminf(mx[i & 7], s[i]);
-      }
-      float m_tile;
-      if (masked || c2 >= 0.f) {
         m_tile = fmaxf(fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])),
                        fmaxf(fmaxf(mx[4], mx[5]), fmaxf(mx[6], mx[7])));
-      } else {
-        m_tile = fminf(fminf(fminf(mx[0], mx[1]), fminf(mx[2], mx[3])),
-                       fminf(fminf(mx[4], mx[5]), fminf(mx[6], mx[7])));
       }
-      if (!masked) m_tile *= c2;
       // lazy rescale: move the reference max only when it grows by more than the threshold
       const bool need = m_tile > m_ref + kRescaleThresh;
       float alpha = 1.f;
@@ -389,38 +384,45 @@ __device__ __forceinline__ void fwd_softmax(const FwdParams& p, const FwdSmem<D>
         m_ref = m_tile;
       }
       const float m_use = (m_ref == -INFINITY) ? 0.f : m_ref;
-      float rs[4] = {0.f, 0.f, 0.f, 0.f}, rse[4] = {0.f, 0.f, 0.f, 0.f};   // 4 chains each
+      // p = 2^(c2 s - m) on pairs: one packed FMA per pair; both row sums packed
+      // (rse: fp32 weights for the LSE; rs: the 16-bit weights the MMA multiplies, so
+      // O / l is an exact weighted average of V)
+      const f32x2 scale2 = fast ? pack_f2(c2, c2) : pack_f2(1.f, 1.f);
+      const f32x2 negm2 = pack_f2(-m_use, -m_use);
+      f32x2 rs2[4] = {0ull, 0ull, 0ull, 0ull}, rse2[4] = {0ull, 0ull, 0ull, 0ull};
 #pragma unroll
       for (int c = 0; c < 4; ++c) {
         uint32_t pk[16];
 #pragma unroll
         for (int i = 0; i < 16; ++i) {
-          float a, b2;
-          if (masked) {
-            a = ex2(s[c * 32 + 2 * i] - m_use);
-            b2 = ex2(s[c * 32 + 2 * i + 1] - m_use);
-          } else {
-            a = ex2(fmaf(s[c * 32 + 2 * i], c2, -m_use));
-            b2 = ex2(fmaf(s[c * 32 + 2 * i + 1], c2, -m_use));
-          }
-          // the row sum adds the 16-bit weights the tensor core multiplies with, so
-          // O / l is an exact weighted average of V (no bias on one-key-dominated rows)
-          rse[i & 3] += a + b2;
+          float x0, x1;
+          unpack_f2(fma_f2(pack_f2(s[c * 32 + 2 * i], s[c * 32 + 2 * i + 1]), scale2, negm2), x0, x1);
+          const float a = ex2(x0), b2 = ex2(x1);
+          rse2[i & 3] = add_f2(rse2[i & 3], pack_f2(a, b2));
+          float lo, hi;
           if (BF16) {
             __nv_bfloat162 h2 = __floats2bfloat162_rn(a, b2);
             pk[i] = *reinterpret_cast<uint32_t*>(&h2);
-            rs[i & 3] += __uint_as_float(pk[i] << 16) + __uint_as_float(pk[i] & 0xffff0000u);
+            lo = __uint_as_float(pk[i] << 16);
+            hi = __uint_as_float(pk[i] & 0xffff0000u);
           } else {
             __half2 h2 = __floats2half2_rn(a, b2);
             pk[i] = *reinterpret_cast<uint32_t*>(&h2);
             const float2 f = __half22float2(h2);
-            rs[i & 3] += f.x + f.y;
+            lo = f.x;
+            hi = f.y;
           }
+          rs2[i & 3] = add_f2(rs2[i & 3], pack_f2(lo, hi));
         }
         tmem_st16(lane_addr + Cfg::P_COL(t) + c * 16, pk);
       }
-      l_sum += (rs[0] + rs[1]) + (rs[2] + rs[3]);
-      l_lse += (rse[0] + rse[1]) + (rse[2] + rse[3]);
+      {
+        float a0, a1, b0, b1;
+        unpack_f2(add_f2(add_f2(rs2[0], rs2[1]), add_f2(rs2[2], rs2[3])), a0, a1);
+        unpack_f2(add_f2(add_f2(rse2[0], rse2[1]), add_f2(rse2[2], rse2[3])), b0, b1);
+        l_sum += a0 + a1;
+        l_lse += b0 + b1;
+      }
       // O_t holds P V up to tile j-1, complete: S_t(j)'s commit covers every earlier MMA
       if (j > 0 && __any_sync(0xffffffffu, need)) {
 #pragma unroll 1
