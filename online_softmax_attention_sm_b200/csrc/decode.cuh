@@ -7,16 +7,18 @@
 // rescales every split's state to the common max and divides once.
 //
 // B200 design:
-//   * grid (split, KV head x head-group, batch); the G = Hq/Hkv query heads that share a
-//     KV head are packed as the rows of one 16-row mma.sync tile, so every K/V byte is
-//     read from HBM exactly once (never once per query head);
+//   * grid (split, KV head x head-group, batch), about three CTAs per SM; the
+//     G = Hq/Hkv query heads that share a KV head are packed as the rows of one 16-row
+//     mma.sync tile, so every K/V byte is read from HBM exactly once (never once per
+//     query head);
 //   * thread 0 streams 64-token K and V slices with TMA tensor loads (128-byte swizzle)
 //     into a ring of shared-memory stages; 4 warps each take 16 tokens of a stage;
 //   * S = Q K^T and O += P V on mma.sync.m16n8k16 (fp32 accumulate), fragments from
 //     ldmatrix; row max / sum by quad shuffles; the 4 warps merge through shared memory;
-//   * the split writes (unnormalised O, running max, running sum) in fp32; the combine
-//     kernel (one warp per (batch, query head)) is launched with programmatic dependent
-//     launch so its launch overlaps the split kernel's tail.
+//   * each split writes (unnormalised O, running max, two running sums) in fp32 to the
+//     workspace and arrives on its group's counter; the last CTA of the group merges all
+//     splits (one kernel, no second launch -- the page's two-kernel prototype lost to
+//     launch and merge overhead at small batch).
 #pragma once
 #include "ptx.cuh"
 #include <cuda_fp16.h>
@@ -33,12 +35,23 @@ struct DecCfg {
   static constexpr int KV_BYTES = KCH * CHUNK_BYTES;   // one K (or V) stage
   static constexpr int STAGES = (D == 64) ? 4 : 2;
   static constexpr int SMEM_STAGES = STAGES * 2 * KV_BYTES;
-  static constexpr int SMEM_MERGE = 4 * 16 * D * 4 + 3 * 4 * 16 * 4;
+  static constexpr int SMEM_MERGE_W = 4 * 16 * D * 4 + 3 * 4 * 16 * 4;   // write_partial
+  static constexpr int SMEM_MERGE_C = 4 * 1024 * 4;                       // decode_merge
+  static constexpr int SMEM_MERGE = SMEM_MERGE_W > SMEM_MERGE_C ? SMEM_MERGE_W : SMEM_MERGE_C;
   static constexpr int SMEM_TOTAL = 1024 + (SMEM_STAGES > SMEM_MERGE ? SMEM_STAGES : SMEM_MERGE) + 256;
 };
 
+// Workspace layout (caller-owned, zero-filled once when allocated):
+//   [0, kDecCounterBytes)   arrival counters, one per (b, kv head, head group); every
+//                           call leaves them at zero, and their place does not depend on
+//                           the problem size, so one workspace serves any shape
+//   then ws_ml [B, Hq, nsplit, 3] fp32, then ws_o [B, Hq, nsplit, D] fp32
+constexpr int kDecMaxGroups = 16384;
+constexpr size_t kDecCounterBytes = kDecMaxGroups * sizeof(unsigned int);
+
 struct DecParams {
   const void* q;       // [B, Hq, D]
+  unsigned int* counters;  // [B * Hkv * ngrp] arrival counters (see above)
   float* ws_o;         // [B, Hq, nsplit, D]
   float* ws_ml;        // [B, Hq, nsplit, 3]: max (log2 units of c2*s), 16-bit-weight sum, fp32 sum
   void* o;             // [B, Hq, D]
@@ -92,8 +105,131 @@ __device__ __forceinline__ uint32_t sw128(int row, int chunk16) {
   return (uint32_t)(row * 128 + ((chunk16 ^ (row & 7)) << 4));
 }
 
+// The 4 warps' states (each over its 16 tokens of every stage) are rescaled to the CTA
+// max through shared memory and written as this split's partial state.
+template <int D>
+__device__ __forceinline__ void write_partial(const DecParams& p, uint8_t* smem, int b, int h0, int nrows,
+                                              int split, int warp, int lane, const float (&o)[D / 8][4],
+                                              float m0, float m1, float l0, float l1, float e0, float e1) {
+  l0 += __shfl_xor_sync(0xffffffffu, l0, 1);
+  l0 += __shfl_xor_sync(0xffffffffu, l0, 2);
+  l1 += __shfl_xor_sync(0xffffffffu, l1, 1);
+  l1 += __shfl_xor_sync(0xffffffffu, l1, 2);
+  e0 += __shfl_xor_sync(0xffffffffu, e0, 1);
+  e0 += __shfl_xor_sync(0xffffffffu, e0, 2);
+  e1 += __shfl_xor_sync(0xffffffffu, e1, 1);
+  e1 += __shfl_xor_sync(0xffffffffu, e1, 2);
+  float* sm_o = reinterpret_cast<float*>(smem);              // [4][16][D] (stages are drained)
+  float* sm_m = sm_o + 4 * 16 * D;                           // [4][16]
+  float* sm_l = sm_m + 64;                                   // [4][16]
+  float* sm_e = sm_l + 64;                                   // [4][16]
+  const int r0 = lane >> 2, r1 = r0 + 8;
+  if ((lane & 3) == 0) {
+    sm_m[warp * 16 + r0] = m0; sm_m[warp * 16 + r1] = m1;
+    sm_l[warp * 16 + r0] = l0; sm_l[warp * 16 + r1] = l1;
+    sm_e[warp * 16 + r0] = e0; sm_e[warp * 16 + r1] = e1;
+  }
+  __syncthreads();
+  float M0 = -INFINITY, M1 = -INFINITY;
+#pragma unroll
+  for (int w = 0; w < 4; ++w) { M0 = fmaxf(M0, sm_m[w * 16 + r0]); M1 = fmaxf(M1, sm_m[w * 16 + r1]); }
+  const float w0 = (m0 == -INFINITY) ? 0.f : ex2(m0 - M0);
+  const float w1 = (m1 == -INFINITY) ? 0.f : ex2(m1 - M1);
+#pragma unroll
+  for (int n = 0; n < D / 8; ++n) {
+    const int c = n * 8 + (lane & 3) * 2;
+    sm_o[(warp * 16 + r0) * D + c] = o[n][0] * w0;
+    sm_o[(warp * 16 + r0) * D + c + 1] = o[n][1] * w0;
+    sm_o[(warp * 16 + r1) * D + c] = o[n][2] * w1;
+    sm_o[(warp * 16 + r1) * D + c + 1] = o[n][3] * w1;
+  }
+  __syncthreads();
+  const size_t ws_row0 = ((size_t)b * p.Hq + h0) * p.nsplit + split;   // row r -> + r * nsplit
+  for (int i = threadIdx.x; i < nrows * D; i += blockDim.x) {
+    const int r = i / D, d = i % D;
+    float acc = 0.f;
+#pragma unroll
+    for (int w = 0; w < 4; ++w) acc += sm_o[(w * 16 + r) * D + d];
+    p.ws_o[(ws_row0 + (size_t)r * p.nsplit) * D + d] = acc;
+  }
+  if (threadIdx.x < nrows) {
+    const int r = threadIdx.x;
+    float M = -INFINITY;
+#pragma unroll
+    for (int w = 0; w < 4; ++w) M = fmaxf(M, sm_m[w * 16 + r]);
+    float L = 0.f, E = 0.f;
+#pragma unroll
+    for (int w = 0; w < 4; ++w) {
+      const float mw = sm_m[w * 16 + r];
+      const float sc = (mw == -INFINITY) ? 0.f : ex2(mw - M);
+      L += sm_l[w * 16 + r] * sc;
+      E += sm_e[w * 16 + r] * sc;
+    }
+    float* ml = p.ws_ml + (ws_row0 + (size_t)r * p.nsplit) * 3;
+    ml[0] = M;
+    ml[1] = L;
+    ml[2] = E;
+  }
+}
+
+// LSE-weighted merge of every split's partial state, done by the last CTA of a
+// (batch, KV head, head group) to arrive.  Warp w merges rows w, w + 4, ...:
+//   M = max_s m_s,  w_s = 2^(m_s - M),  O = sum_s w_s O_s / sum_s w_s l_s,
+//   LSE = (M + log2 sum_s w_s e_s) * ln 2.
+constexpr int kCombineMaxSplits = 1024;
+
 template <int D, bool BF16>
-__global__ void __launch_bounds__(128)
+__device__ __forceinline__ void decode_merge(const DecParams& p, float* smem_f, int b, int h0, int nrows) {
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  float* sw = smem_f + warp * kCombineMaxSplits;      // this warp's split weights
+  const int ns = p.nsplit;
+  constexpr int NE = D / 32;                           // output columns per lane
+  for (int r = warp; r < nrows; r += 4) {
+    const size_t row = (size_t)b * p.Hq + h0 + r;
+    const float* ml = p.ws_ml + row * ns * 3;
+    const float* os = p.ws_o + row * ns * D;
+    float M = -INFINITY;
+    for (int s = lane; s < ns; s += 32) M = fmaxf(M, __ldcg(ml + 3 * s));
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
+    float L = 0.f, E = 0.f;
+    for (int s = lane; s < ns; s += 32) {
+      const float ms = __ldcg(ml + 3 * s);
+      const float w = (ms == -INFINITY) ? 0.f : ex2(ms - M);
+      sw[s] = w;
+      L += w * __ldcg(ml + 3 * s + 1);
+      E += w * __ldcg(ml + 3 * s + 2);
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+      L += __shfl_xor_sync(0xffffffffu, L, o);
+      E += __shfl_xor_sync(0xffffffffu, E, o);
+    }
+    __syncwarp();
+    float acc[NE];
+#pragma unroll
+    for (int e = 0; e < NE; ++e) acc[e] = 0.f;
+#pragma unroll 4
+    for (int s = 0; s < ns; ++s) {
+      const float w = sw[s];
+#pragma unroll
+      for (int e = 0; e < NE; ++e) acc[e] = fmaf(w, __ldcg(os + (size_t)s * D + e * 32 + lane), acc[e]);
+    }
+    const float inv = L > 0.f ? 1.f / L : 0.f;
+    using T = typename std::conditional<BF16, __nv_bfloat16, __half>::type;
+    T* out = reinterpret_cast<T*>(p.o) + row * D;
+#pragma unroll
+    for (int e = 0; e < NE; ++e) {
+      if (BF16) reinterpret_cast<__nv_bfloat16*>(out)[e * 32 + lane] = __float2bfloat16_rn(acc[e] * inv);
+      else reinterpret_cast<__half*>(out)[e * 32 + lane] = __float2half_rn(acc[e] * inv);
+    }
+    if (p.lse && lane == 0) p.lse[row] = E > 0.f ? (M + __log2f(E)) * 0.69314718055994531f : -INFINITY;
+    __syncwarp();
+  }
+}
+
+template <int D, bool BF16>
+__global__ void __launch_bounds__(128, 3)
 attn_decode_split(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
                   const DecParams p) {
   using Cfg = DecCfg<D>;
@@ -102,9 +238,6 @@ attn_decode_split(const __grid_constant__ CUtensorMap tm_k, const __grid_constan
   const int region = Cfg::SMEM_STAGES > Cfg::SMEM_MERGE ? Cfg::SMEM_STAGES : Cfg::SMEM_MERGE;
   uint64_t* full = (uint64_t*)(smem + region);
   volatile int* abort_flag = (volatile int*)(full + Cfg::STAGES);
-
-  // let the combine kernel get launched while this grid runs (it waits for our results)
-  asm volatile("griddepcontrol.launch_dependents;");
 
   const int split = blockIdx.x;
   const int kvh = blockIdx.y / p.ngrp;
@@ -258,140 +391,25 @@ attn_decode_split(const __grid_constant__ CUtensorMap tm_k, const __grid_constan
         mbar_wait(&full[st % Cfg::STAGES], (st / Cfg::STAGES) & 1, nullptr, 41);
     }
     __syncthreads();
-    return;
+    // still arrive below, so the group's counter completes and resets (the outputs of a
+    // call whose wait expired are undefined; the status word reports it)
+  } else {
+    write_partial<D>(p, smem, b, h0, nrows, split, warp, lane, o, m0, m1, l0, l1, e0, e1);
   }
-
-  // ---- merge the 4 warps: per row, rescale to the CTA max and add
-  l0 += __shfl_xor_sync(0xffffffffu, l0, 1);
-  l0 += __shfl_xor_sync(0xffffffffu, l0, 2);
-  l1 += __shfl_xor_sync(0xffffffffu, l1, 1);
-  l1 += __shfl_xor_sync(0xffffffffu, l1, 2);
-  e0 += __shfl_xor_sync(0xffffffffu, e0, 1);
-  e0 += __shfl_xor_sync(0xffffffffu, e0, 2);
-  e1 += __shfl_xor_sync(0xffffffffu, e1, 1);
-  e1 += __shfl_xor_sync(0xffffffffu, e1, 2);
-  float* sm_o = reinterpret_cast<float*>(smem);              // [4][16][D] (stages are drained)
-  float* sm_m = sm_o + 4 * 16 * D;                           // [4][16]
-  float* sm_l = sm_m + 64;                                   // [4][16]
-  float* sm_e = sm_l + 64;                                   // [4][16]
-  const int r0 = lane >> 2, r1 = r0 + 8;
-  if ((lane & 3) == 0) {
-    sm_m[warp * 16 + r0] = m0; sm_m[warp * 16 + r1] = m1;
-    sm_l[warp * 16 + r0] = l0; sm_l[warp * 16 + r1] = l1;
-    sm_e[warp * 16 + r0] = e0; sm_e[warp * 16 + r1] = e1;
+  __threadfence();                                            // partials visible device-wide
+  __shared__ int s_last;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    unsigned int* ctr = p.counters + ((size_t)b * p.Hkv + kvh) * p.ngrp + grp;
+    const unsigned int prev = atomicAdd(ctr, 1u);
+    s_last = (prev == (unsigned)p.nsplit - 1u);
+    if (s_last) *ctr = 0u;                                    // ready for the next call
   }
   __syncthreads();
-  float M0 = -INFINITY, M1 = -INFINITY;
-#pragma unroll
-  for (int w = 0; w < 4; ++w) { M0 = fmaxf(M0, sm_m[w * 16 + r0]); M1 = fmaxf(M1, sm_m[w * 16 + r1]); }
-  const float w0 = (m0 == -INFINITY) ? 0.f : ex2(m0 - M0);
-  const float w1 = (m1 == -INFINITY) ? 0.f : ex2(m1 - M1);
-#pragma unroll
-  for (int n = 0; n < D / 8; ++n) {
-    const int c = n * 8 + (lane & 3) * 2;
-    sm_o[(warp * 16 + r0) * D + c] = o[n][0] * w0;
-    sm_o[(warp * 16 + r0) * D + c + 1] = o[n][1] * w0;
-    sm_o[(warp * 16 + r1) * D + c] = o[n][2] * w1;
-    sm_o[(warp * 16 + r1) * D + c + 1] = o[n][3] * w1;
+  if (s_last) {
+    __threadfence();
+    decode_merge<D, BF16>(p, reinterpret_cast<float*>(smem), b, h0, nrows);
   }
-  __syncthreads();
-  const size_t ws_row0 = ((size_t)b * p.Hq + h0) * p.nsplit + split;   // row r -> + r * nsplit
-  for (int i = threadIdx.x; i < nrows * D; i += blockDim.x) {
-    const int r = i / D, d = i % D;
-    float acc = 0.f;
-#pragma unroll
-    for (int w = 0; w < 4; ++w) acc += sm_o[(w * 16 + r) * D + d];
-    p.ws_o[(ws_row0 + (size_t)r * p.nsplit) * D + d] = acc;
-  }
-  if (threadIdx.x < nrows) {
-    const int r = threadIdx.x;
-    float M = -INFINITY;
-#pragma unroll
-    for (int w = 0; w < 4; ++w) M = fmaxf(M, sm_m[w * 16 + r]);
-    float L = 0.f, E = 0.f;
-#pragma unroll
-    for (int w = 0; w < 4; ++w) {
-      const float mw = sm_m[w * 16 + r];
-      const float sc = (mw == -INFINITY) ? 0.f : ex2(mw - M);
-      L += sm_l[w * 16 + r] * sc;
-      E += sm_e[w * 16 + r] * sc;
-    }
-    float* ml = p.ws_ml + (ws_row0 + (size_t)r * p.nsplit) * 3;
-    ml[0] = M;
-    ml[1] = L;
-    ml[2] = E;
-  }
-}
-
-// One 128-thread block per (batch, query head):
-//   M = max_s m_s,  w_s = 2^(m_s - M),  O = sum_s w_s O_s / sum_s w_s l_s,
-//   LSE = (M + log2 sum_s w_s e_s) * ln 2.
-// Thread t owns column d = t % D and the splits s = t / D, t / D + 128 / D, ...; the
-// (128 / D) partial sums per column are added through shared memory.
-constexpr int kCombineMaxSplits = 1024;
-
-template <int D, bool BF16>
-__global__ void __launch_bounds__(128)
-attn_decode_combine(const DecParams p) {
-  asm volatile("griddepcontrol.wait;" ::: "memory");   // split results are complete
-  __shared__ float s_w[kCombineMaxSplits];
-  __shared__ float s_red[2][4];
-  __shared__ float s_acc[128];
-  const int gw = blockIdx.x;                           // (b, h)
-  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const float* ml = p.ws_ml + (size_t)gw * p.nsplit * 3;
-  const float* os = p.ws_o + (size_t)gw * p.nsplit * D;
-  const int ns = p.nsplit;
-  float M = -INFINITY;
-  for (int s = tid; s < ns; s += 128) M = fmaxf(M, ml[3 * s]);
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
-  if (lane == 0) s_red[0][warp] = M;
-  __syncthreads();
-  M = fmaxf(fmaxf(s_red[0][0], s_red[0][1]), fmaxf(s_red[0][2], s_red[0][3]));
-  float L = 0.f, E = 0.f;
-  for (int s = tid; s < ns; s += 128) {
-    const float ms = ml[3 * s];
-    const float w = (ms == -INFINITY) ? 0.f : ex2(ms - M);
-    s_w[s] = w;
-    L += w * ml[3 * s + 1];
-    E += w * ml[3 * s + 2];
-  }
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) {
-    L += __shfl_xor_sync(0xffffffffu, L, o);
-    E += __shfl_xor_sync(0xffffffffu, E, o);
-  }
-  __syncthreads();                                     // s_red[0] reads done, s_w written
-  if (lane == 0) { s_red[0][warp] = L; s_red[1][warp] = E; }
-  __syncthreads();
-  L = (s_red[0][0] + s_red[0][1]) + (s_red[0][2] + s_red[0][3]);
-  E = (s_red[1][0] + s_red[1][1]) + (s_red[1][2] + s_red[1][3]);
-  constexpr int GRP = 128 / D;                         // threads per column
-  const int d = tid % D, g = tid / D;
-  float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;        // independent chains
-  int s = g;
-  for (; s + 3 * GRP < ns; s += 4 * GRP) {
-    a0 += s_w[s] * os[(size_t)s * D + d];
-    a1 += s_w[s + GRP] * os[(size_t)(s + GRP) * D + d];
-    a2 += s_w[s + 2 * GRP] * os[(size_t)(s + 2 * GRP) * D + d];
-    a3 += s_w[s + 3 * GRP] * os[(size_t)(s + 3 * GRP) * D + d];
-  }
-  for (; s < ns; s += GRP) a0 += s_w[s] * os[(size_t)s * D + d];
-  s_acc[tid] = (a0 + a1) + (a2 + a3);
-  __syncthreads();
-  if (tid < D) {
-    float acc = 0.f;
-#pragma unroll
-    for (int k = 0; k < GRP; ++k) acc += s_acc[k * D + tid];
-    const float inv = L > 0.f ? 1.f / L : 0.f;
-    using T = typename std::conditional<BF16, __nv_bfloat16, __half>::type;
-    T* out = reinterpret_cast<T*>(p.o) + (size_t)gw * D + tid;
-    if (BF16) *reinterpret_cast<__nv_bfloat16*>(out) = __float2bfloat16_rn(acc * inv);
-    else *reinterpret_cast<__half*>(out) = __float2half_rn(acc * inv);
-  }
-  if (p.lse && tid == 0)
-    p.lse[gw] = E > 0.f ? (M + __log2f(E)) * 0.69314718055994531f : -INFINITY;
 }
 
 }  // namespace sa

@@ -72,12 +72,31 @@ def test_decode_workspace_contract():
     B, Sk, Hq, Hkv, D = 4, 32768, 14, 2, 64
     ns = sa_attn_decode_num_splits(B, Sk, Hq, Hkv, D)
     assert 1 <= ns <= Sk // 64
-    assert sa_attn_decode_workspace_size(B, Sk, Hq, Hkv, D) == B * Hq * ns * (D + 3) * 4
+    need = sa_attn_decode_workspace_size(B, Sk, Hq, Hkv, D)
+    assert need == 65536 + B * Hq * ns * (D + 3) * 4
     q, k, v = make_qkv(B, 1, Sk, Hq, Hkv, D, "fp16", seed=25, decode=True)
-    ws = torch.full((sa_attn_decode_workspace_size(B, Sk, Hq, Hkv, D) + 4096,), 0x5A,
-                    dtype=torch.uint8, device=dev())
+    # zeroed counter header, garbage scratch, canary past the declared size
+    ws = torch.full((need + 4096,), 0x5A, dtype=torch.uint8, device=dev())
+    ws[:65536] = 0
     o, l = sa_attn_decode(q.to(dev()), k.to(dev()), v.to(dev()), workspace=ws)
     sa_check_status()
     assert torch.all(ws[-4096:] == 0x5A), "wrote past the declared workspace size"
+    assert torch.all(ws[:65536] == 0), "arrival counters not left at zero"
     O, L = oracle.decode(f64(q), f64(k), f64(v), 1 / 8.0)
     assert_close(o, l, O, L, "fp16", "workspace contract")
+
+
+def test_decode_one_workspace_serves_many_shapes():
+    # a serving loop: the KV length grows and the batch changes between calls that reuse
+    # one workspace (zero-filled once, sized for the largest call)
+    ws = torch.zeros(sa_attn_decode_workspace_size(8, 9000, 16, 2, 128, 0) + 65536,
+                     dtype=torch.uint8, device=dev())
+    for i, (B, Sk, Hq, Hkv, D, dt) in enumerate([(2, 100, 14, 2, 64, "fp16"), (8, 9000, 16, 2, 128, "bf16"),
+                                               (1, 5000, 8, 8, 64, "fp16"), (3, 8191, 16, 1, 128, "bf16"),
+                                               (2, 101, 14, 2, 64, "fp16")]):
+        q, k, v = make_qkv(B, 1, Sk, Hq, Hkv, D, dt, seed=30 + i, decode=True)
+        o, l = sa_attn_decode(q.to(dev()), k.to(dev()), v.to(dev()), workspace=ws)
+        sa_check_status()
+        O, L = oracle.decode(f64(q), f64(k), f64(v), 1 / np.sqrt(D))
+        assert_close(o, l, O, L, dt, f"reuse #{i}")
+    assert torch.all(ws[:65536] == 0)
