@@ -89,11 +89,11 @@ def test_decode_workspace_contract():
 def test_decode_one_workspace_serves_many_shapes():
     # a serving loop: the KV length grows and the batch changes between calls that reuse
     # one workspace (zero-filled once, sized for the largest call)
-    ws = torch.zeros(sa_attn_decode_workspace_size(8, 9000, 16, 2, 128, 0) + 65536,
+    shapes = [(2, 100, 14, 2, 64, "fp16"), (8, 9000, 16, 2, 128, "bf16"), (1, 5000, 8, 8, 64, "fp16"),
+              (3, 8191, 16, 1, 128, "bf16"), (2, 101, 14, 2, 64, "fp16")]
+    ws = torch.zeros(max(sa_attn_decode_workspace_size(*sh[:5]) for sh in shapes),
                      dtype=torch.uint8, device=dev())
-    for i, (B, Sk, Hq, Hkv, D, dt) in enumerate([(2, 100, 14, 2, 64, "fp16"), (8, 9000, 16, 2, 128, "bf16"),
-                                               (1, 5000, 8, 8, 64, "fp16"), (3, 8191, 16, 1, 128, "bf16"),
-                                               (2, 101, 14, 2, 64, "fp16")]):
+    for i, (B, Sk, Hq, Hkv, D, dt) in enumerate(shapes):
         q, k, v = make_qkv(B, 1, Sk, Hq, Hkv, D, dt, seed=30 + i, decode=True)
         o, l = sa_attn_decode(q.to(dev()), k.to(dev()), v.to(dev()), workspace=ws)
         sa_check_status()
