@@ -73,11 +73,12 @@ int sa_attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse
 
 /*
  * Bytes of decode workspace needed for `num_splits` (0 = the automatic choice):
- * 65536 + B * Hq * splits * (D + 3) * 4.  Layout: a 64 KiB header of arrival counters
+ * 65536 + B * Hq * splits * (D + 4) * 4.  Layout: a 64 KiB header of arrival counters
  * (one per (b, kv head, group of up to 16 query heads)), then per (b, h, split) the
  * split's running max and two running sums (of the 16-bit weights the MMA used, and of
- * the fp32 weights for the LSE), then its unnormalised fp32 output row -- the partial
- * online-softmax states of the StreamAttention page, "Engine Direction".
+ * the fp32 weights for the LSE) padded to 4 floats, then its unnormalised fp32 output
+ * row -- the partial online-softmax states of the StreamAttention page, "Engine
+ * Direction".
  * Returns 0 for empty problems, invalid sizes or B * Hkv * ceil(Hq / Hkv / 16) > 16384.
  */
 size_t sa_attn_decode_workspace_size(int B, int Sk, int Hq, int Hkv, int D, int num_splits);
@@ -91,7 +92,8 @@ int sa_attn_decode_num_splits(int B, int Sk, int Hq, int Hkv, int D);
  * "Engine Direction" and "Distributed and Long-Context Variants": partial states merged
  * with log-sum-exp weights).
  *   q [B, Hq, D], k/v [B, Sk, Hkv, D], o [B, Hq, D]; lse [B, Hq] fp32 or NULL.
- *   num_splits : KV splits per (b, kv head); 0 = automatic; clamped to ceil(Sk / 64).
+ *   num_splits : KV splits per (b, kv head); 0 = automatic; clamped to ceil(Sk / 64) and
+ *                to 192 (D = 64) / 96 (D = 128).
  *   workspace  : device buffer of at least sa_attn_decode_workspace_size(...) bytes,
  *                16-byte aligned, owned by the caller.  ZERO-FILL IT ONCE after allocating
  *                it (e.g. cudaMemsetAsync): its first 64 KiB hold arrival counters that

@@ -35,9 +35,8 @@ struct DecCfg {
   static constexpr int KV_BYTES = KCH * CHUNK_BYTES;   // one K (or V) stage
   static constexpr int STAGES = (D == 64) ? 4 : 2;
   static constexpr int SMEM_STAGES = STAGES * 2 * KV_BYTES;
-  static constexpr int SMEM_MERGE_W = 4 * 16 * D * 4 + 3 * 4 * 16 * 4;   // write_partial
-  static constexpr int SMEM_MERGE_C = 4 * 1024 * 4;                       // decode_merge
-  static constexpr int SMEM_MERGE = SMEM_MERGE_W > SMEM_MERGE_C ? SMEM_MERGE_W : SMEM_MERGE_C;
+  // write_partial's buffers; decode_merge uses the SMEM_STAGES region
+  static constexpr int SMEM_MERGE = 4 * 16 * D * 4 + 3 * 4 * 16 * 4;
   static constexpr int SMEM_TOTAL = 1024 + (SMEM_STAGES > SMEM_MERGE ? SMEM_STAGES : SMEM_MERGE) + 256;
 };
 
@@ -45,7 +44,8 @@ struct DecCfg {
 //   [0, kDecCounterBytes)   arrival counters, one per (b, kv head, head group); every
 //                           call leaves them at zero, and their place does not depend on
 //                           the problem size, so one workspace serves any shape
-//   then ws_ml [B, Hq, nsplit, 3] fp32, then ws_o [B, Hq, nsplit, D] fp32
+//   then ws_ml [B, Hq, nsplit, 4] fp32 (max, 16-bit-weight sum, fp32 sum, pad),
+//   then ws_o [B, Hq, nsplit, D] fp32
 constexpr int kDecMaxGroups = 16384;
 constexpr size_t kDecCounterBytes = kDecMaxGroups * sizeof(unsigned int);
 
@@ -53,7 +53,7 @@ struct DecParams {
   const void* q;       // [B, Hq, D]
   unsigned int* counters;  // [B * Hkv * ngrp] arrival counters (see above)
   float* ws_o;         // [B, Hq, nsplit, D]
-  float* ws_ml;        // [B, Hq, nsplit, 3]: max (log2 units of c2*s), 16-bit-weight sum, fp32 sum
+  float* ws_ml;        // [B, Hq, nsplit, 4]: max (log2 units of c2*s), 16-bit-weight sum, fp32 sum, 0
   void* o;             // [B, Hq, D]
   float* lse;          // [B, Hq] or null
   int B, Sk, Hq, Hkv, G, ngrp, nsplit, chunk;
@@ -165,66 +165,96 @@ __device__ __forceinline__ void write_partial(const DecParams& p, uint8_t* smem,
       L += sm_l[w * 16 + r] * sc;
       E += sm_e[w * 16 + r] * sc;
     }
-    float* ml = p.ws_ml + (ws_row0 + (size_t)r * p.nsplit) * 3;
-    ml[0] = M;
-    ml[1] = L;
-    ml[2] = E;
+    *reinterpret_cast<float4*>(p.ws_ml + (ws_row0 + (size_t)r * p.nsplit) * 4) = make_float4(M, L, E, 0.f);
   }
 }
 
 // LSE-weighted merge of every split's partial state, done by the last CTA of a
-// (batch, KV head, head group) to arrive.  Warp w merges rows w, w + 4, ...:
+// (batch, KV head, head group) to arrive:
 //   M = max_s m_s,  w_s = 2^(m_s - M),  O = sum_s w_s O_s / sum_s w_s l_s,
 //   LSE = (M + log2 sum_s w_s e_s) * ln 2.
-constexpr int kCombineMaxSplits = 1024;
+// The group's partial states are contiguous in the workspace; they are pulled into
+// shared memory a batch of rows at a time with 16-byte cp.async copies (all in flight at
+// once), then merged from shared memory.
+template <int D>
+struct DecMerge {
+  // splits are capped so that one row's partial states fit the merge buffer
+  static constexpr int MAX_SPLITS = (D == 64) ? 192 : 96;
+  static constexpr int ROW_BYTES_PER_SPLIT = (D + 4) * 4;
+};
+
+__device__ __forceinline__ void cp_async16(void* smem_dst, const void* gmem_src) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_u32(smem_dst)), "l"(gmem_src) : "memory");
+}
+__device__ __forceinline__ void cp_async_wait_all() {
+  asm volatile("cp.async.wait_all;" ::: "memory");
+}
 
 template <int D, bool BF16>
-__device__ __forceinline__ void decode_merge(const DecParams& p, float* smem_f, int b, int h0, int nrows) {
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  float* sw = smem_f + warp * kCombineMaxSplits;      // this warp's split weights
+__device__ __forceinline__ void decode_merge(const DecParams& p, uint8_t* smem, int smem_bytes, int b, int h0,
+                                             int nrows) {
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int ns = p.nsplit;
-  constexpr int NE = D / 32;                           // output columns per lane
-  for (int r = warp; r < nrows; r += 4) {
-    const size_t row = (size_t)b * p.Hq + h0 + r;
-    const float* ml = p.ws_ml + row * ns * 3;
-    const float* os = p.ws_o + row * ns * D;
-    float M = -INFINITY;
-    for (int s = lane; s < ns; s += 32) M = fmaxf(M, __ldcg(ml + 3 * s));
+  const int rows_per_batch = max(1, smem_bytes / (ns * DecMerge<D>::ROW_BYTES_PER_SPLIT));
+  const size_t row0 = (size_t)b * p.Hq + h0;
+  for (int rb = 0; rb < nrows; rb += rows_per_batch) {
+    const int nr = min(rows_per_batch, nrows - rb);
+    float* s_ml = reinterpret_cast<float*>(smem);                 // [nr][ns][4]
+    float* s_o = s_ml + (size_t)nr * ns * 4;                       // [nr][ns][D]
+    const float4* g_ml = reinterpret_cast<const float4*>(p.ws_ml + (row0 + rb) * ns * 4);
+    const float4* g_o = reinterpret_cast<const float4*>(p.ws_o + (row0 + rb) * ns * D);
+    const int n_ml = nr * ns, n_o = nr * ns * (D / 4);
+    for (int i = tid; i < n_ml; i += 128) cp_async16(s_ml + 4 * i, g_ml + i);
+    for (int i = tid; i < n_o; i += 128) cp_async16(s_o + 4 * i, g_o + i);
+    cp_async_wait_all();
+    __syncthreads();
+    // per row: max, weights (kept in the pad slot), sums -- warp w takes rows w, w + 4, ...
+    __shared__ float s_LE[16][2];
+    for (int r = warp; r < nr; r += 4) {
+      float* ml = s_ml + (size_t)r * ns * 4;
+      float M = -INFINITY;
+      for (int s = lane; s < ns; s += 32) M = fmaxf(M, ml[4 * s]);
 #pragma unroll
-    for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
-    float L = 0.f, E = 0.f;
-    for (int s = lane; s < ns; s += 32) {
-      const float ms = __ldcg(ml + 3 * s);
-      const float w = (ms == -INFINITY) ? 0.f : ex2(ms - M);
-      sw[s] = w;
-      L += w * __ldcg(ml + 3 * s + 1);
-      E += w * __ldcg(ml + 3 * s + 2);
+      for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
+      float L = 0.f, E = 0.f;
+      for (int s = lane; s < ns; s += 32) {
+        const float ms = ml[4 * s];
+        const float w = (ms == -INFINITY) ? 0.f : ex2(ms - M);
+        ml[4 * s + 3] = w;
+        L += w * ml[4 * s + 1];
+        E += w * ml[4 * s + 2];
+      }
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) {
+        L += __shfl_xor_sync(0xffffffffu, L, o);
+        E += __shfl_xor_sync(0xffffffffu, E, o);
+      }
+      if (lane == 0) {
+        s_LE[r][0] = L;
+        if (p.lse) p.lse[row0 + rb + r] = E > 0.f ? (M + __log2f(E)) * 0.69314718055994531f : -INFINITY;
+      }
     }
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) {
-      L += __shfl_xor_sync(0xffffffffu, L, o);
-      E += __shfl_xor_sync(0xffffffffu, E, o);
-    }
-    __syncwarp();
-    float acc[NE];
-#pragma unroll
-    for (int e = 0; e < NE; ++e) acc[e] = 0.f;
-#pragma unroll 4
-    for (int s = 0; s < ns; ++s) {
-      const float w = sw[s];
-#pragma unroll
-      for (int e = 0; e < NE; ++e) acc[e] = fmaf(w, __ldcg(os + (size_t)s * D + e * 32 + lane), acc[e]);
-    }
-    const float inv = L > 0.f ? 1.f / L : 0.f;
+    __syncthreads();
+    // O[r][d] = sum_s w_s O_s[d] / L
     using T = typename std::conditional<BF16, __nv_bfloat16, __half>::type;
-    T* out = reinterpret_cast<T*>(p.o) + row * D;
-#pragma unroll
-    for (int e = 0; e < NE; ++e) {
-      if (BF16) reinterpret_cast<__nv_bfloat16*>(out)[e * 32 + lane] = __float2bfloat16_rn(acc[e] * inv);
-      else reinterpret_cast<__half*>(out)[e * 32 + lane] = __float2half_rn(acc[e] * inv);
+    for (int i = tid; i < nr * D; i += 128) {
+      const int r = i / D, d = i % D;
+      const float* ml = s_ml + (size_t)r * ns * 4;
+      const float* o = s_o + (size_t)r * ns * D + d;
+      float a0 = 0.f, a1 = 0.f;
+      int s = 0;
+      for (; s + 1 < ns; s += 2) {
+        a0 = fmaf(ml[4 * s + 3], o[(size_t)s * D], a0);
+        a1 = fmaf(ml[4 * s + 7], o[(size_t)(s + 1) * D], a1);
+      }
+      if (s < ns) a0 = fmaf(ml[4 * s + 3], o[(size_t)s * D], a0);
+      const float L = s_LE[r][0];
+      const float v = L > 0.f ? (a0 + a1) / L : 0.f;
+      T* out = reinterpret_cast<T*>(p.o) + (row0 + rb + r) * D + d;
+      if (BF16) *reinterpret_cast<__nv_bfloat16*>(out) = __float2bfloat16_rn(v);
+      else *reinterpret_cast<__half*>(out) = __float2half_rn(v);
     }
-    if (p.lse && lane == 0) p.lse[row] = E > 0.f ? (M + __log2f(E)) * 0.69314718055994531f : -INFINITY;
-    __syncwarp();
+    __syncthreads();                                            // buffer reused by the next batch
   }
 }
 
@@ -408,7 +438,7 @@ attn_decode_split(const __grid_constant__ CUtensorMap tm_k, const __grid_constan
   __syncthreads();
   if (s_last) {
     __threadfence();
-    decode_merge<D, BF16>(p, reinterpret_cast<float*>(smem), b, h0, nrows);
+    decode_merge<D, BF16>(p, smem, Cfg::SMEM_STAGES, b, h0, nrows);
   }
 }
 

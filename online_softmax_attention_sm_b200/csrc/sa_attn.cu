@@ -160,20 +160,21 @@ int launch_simple(const void* q, const void* k, const void* v, void* o, float* l
 
 // ---------------------------------------------------------------- decode planning
 size_t dec_ws_bytes(int B, int Hq, int nsplit, int D) {
-  return sa::kDecCounterBytes + (size_t)B * Hq * nsplit * (D + 3) * sizeof(float);
+  return sa::kDecCounterBytes + (size_t)B * Hq * nsplit * (D + 4) * sizeof(float);
 }
 
 struct DecPlan {
   int nsplit, chunk, ngrp;
 };
 
-DecPlan plan_decode(int B, int Sk, int Hq, int Hkv, int num_splits, int sms) {
+DecPlan plan_decode(int B, int Sk, int Hq, int Hkv, int D, int num_splits, int sms) {
   DecPlan pl;
   const int G = Hq / Hkv;
   pl.ngrp = (G + 15) / 16;
   const long long groups = (long long)B * Hkv * pl.ngrp;
   int max_split = (Sk + 63) / 64;
-  if (max_split > sa::kCombineMaxSplits) max_split = sa::kCombineMaxSplits;
+  const int cap = D == 64 ? sa::DecMerge<64>::MAX_SPLITS : sa::DecMerge<128>::MAX_SPLITS;
+  if (max_split > cap) max_split = cap;
   long long want = num_splits > 0 ? num_splits : (3LL * sms + groups - 1) / groups;
   if (want < 1) want = 1;
   if (want > max_split) want = max_split;
@@ -196,7 +197,7 @@ int launch_decode(const void* q, const void* k, const void* v, void* o, float* l
   p.q = q;
   p.counters = reinterpret_cast<unsigned int*>(ws);
   p.ws_ml = reinterpret_cast<float*>(reinterpret_cast<char*>(ws) + sa::kDecCounterBytes);
-  p.ws_o = p.ws_ml + (size_t)B * Hq * pl.nsplit * 3;
+  p.ws_o = p.ws_ml + (size_t)B * Hq * pl.nsplit * 4;
   p.o = o; p.lse = lse;
   p.B = B; p.Sk = Sk; p.Hq = Hq; p.Hkv = Hkv; p.G = Hq / Hkv; p.ngrp = pl.ngrp;
   p.nsplit = pl.nsplit; p.chunk = pl.chunk;
@@ -251,13 +252,13 @@ int sa_attn_fwd_simple(const void* q, const void* k, const void* v, void* o, flo
 int sa_attn_decode_num_splits(int B, int Sk, int Hq, int Hkv, int D) {
   if (check_dims(B, 1, Sk, Hq, Hkv, D, SA_FP16, 1.f) != SA_OK) return 0;
   if (B == 0 || Hq == 0 || Sk == 0) return 1;
-  return plan_decode(B, Sk, Hq, Hkv, 0, num_sms()).nsplit;
+  return plan_decode(B, Sk, Hq, Hkv, D, 0, num_sms()).nsplit;
 }
 
 size_t sa_attn_decode_workspace_size(int B, int Sk, int Hq, int Hkv, int D, int num_splits) {
   if (num_splits < 0 || check_dims(B, 1, Sk, Hq, Hkv, D, SA_FP16, 1.f) != SA_OK) return 0;
   if (B == 0 || Hq == 0 || Sk == 0) return 0;
-  DecPlan pl = plan_decode(B, Sk, Hq, Hkv, num_splits, num_sms());
+  DecPlan pl = plan_decode(B, Sk, Hq, Hkv, D, num_splits, num_sms());
   if ((long long)B * Hkv * pl.ngrp > sa::kDecMaxGroups) return 0;
   return dec_ws_bytes(B, Hq, pl.nsplit, D);
 }
@@ -272,7 +273,7 @@ int sa_attn_decode(const void* q, const void* k, const void* v, void* o, float* 
   if ((rc = check_ptrs(q, Sk ? k : q, Sk ? v : q, o, lse)) != SA_OK) return rc;
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   if (Sk == 0) return launch_fill(o, (size_t)B * Hq * D, lse, (size_t)B * Hq, st);
-  DecPlan pl = plan_decode(B, Sk, Hq, Hkv, num_splits, num_sms());
+  DecPlan pl = plan_decode(B, Sk, Hq, Hkv, D, num_splits, num_sms());
   if ((long long)B * Hkv * pl.ngrp > sa::kDecMaxGroups)
     return fail(SA_ERR_UNSUPPORTED, "B * Hkv * ceil(G / 16) = %lld exceeds %d", (long long)B * Hkv * pl.ngrp,
                 sa::kDecMaxGroups);

@@ -73,7 +73,7 @@ def test_decode_workspace_contract():
     ns = sa_attn_decode_num_splits(B, Sk, Hq, Hkv, D)
     assert 1 <= ns <= Sk // 64
     need = sa_attn_decode_workspace_size(B, Sk, Hq, Hkv, D)
-    assert need == 65536 + B * Hq * ns * (D + 3) * 4
+    assert need == 65536 + B * Hq * ns * (D + 4) * 4
     q, k, v = make_qkv(B, 1, Sk, Hq, Hkv, D, "fp16", seed=25, decode=True)
     # zeroed counter header, garbage scratch, canary past the declared size
     ws = torch.full((need + 4096,), 0x5A, dtype=torch.uint8, device=dev())
