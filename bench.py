@@ -277,10 +277,9 @@ def main():
     # for writing back up to an L2 of dirty lines)
     l2 = torch.cuda.get_device_properties(dev).L2_cache_size
     scrub = torch.ones(4 * l2 // 4, dtype=torch.float32, device=dev)
-    sink = torch.empty((), dtype=torch.float32, device=dev)
     cold = []
     for i in range(args.warmup + args.steps if run_dec else 0):
-        torch.sum(scrub, out=sink)
+        scrub.sum()
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         e0.record(stream)
         sa_attn_decode(dq, dk, dv, scale=wd.scale, workspace=ws, out=do, lse=dlse, stream=stream)
