@@ -5,7 +5,7 @@ One step = one pass of the whole hot path over one batch of synthetic input:
   * prefill: the 32768-token GQA causal forward (bf16, B=1, Hq=32, Hkv=8, D=128, K rows
     0..3 scaled x8), sa_attn_fwd -> persistent tcgen05 kernel;
   * decode: the 32768-token GQA split-KV decode (fp16, B=4, Hq=14, Hkv=2, D=64),
-    sa_attn_decode -> one split-KV kernel whose last CTA per group merges.
+    sa_attn_decode -> split-KV kernel + combine kernel (programmatic dependent launch).
 value = prefill FLOPs (4*B*Hq*Sq*Sk*D/2, causal) per second of whole step, TFLOP/s.
 The decode's KV bandwidth is reported beside it ("decode"), timed with its own events.
 
@@ -232,8 +232,7 @@ def main():
     lse = torch.empty((wp.B, wp.Hq, wp.Sq), dtype=torch.float32, device=dev)
     do = torch.empty_like(dq)
     dlse = torch.empty((wd.B, wd.Hq), dtype=torch.float32, device=dev)
-    # zero-filled once (its header holds arrival counters that every call leaves at zero)
-    ws = torch.zeros(sa_attn_decode_workspace_size(wd.B, wd.Sk, wd.Hq, wd.Hkv, wd.D), dtype=torch.uint8,
+    ws = torch.empty(sa_attn_decode_workspace_size(wd.B, wd.Sk, wd.Hq, wd.Hkv, wd.D), dtype=torch.uint8,
                      device=dev)
     stream = torch.cuda.current_stream(dev)
 
@@ -355,9 +354,9 @@ def main():
                          "traffic": traffic},
             "decode": {"value": dec_gbs_cold, "unit": "GB/s", "bound": "hbm", "peak": peaks["hbm_gbs"],
                        "frac": dec_gbs_cold / peaks["hbm_gbs"], "us": cold_avg * 1e3, "l2": "cold (4xL2 read scrub)",
-                       "in_step_gbs": dec_gbs_step, "kernels": "attn_decode_split (fused merge)"},
+                       "in_step_gbs": dec_gbs_step, "kernels": "attn_decode_split + attn_decode_combine (PDL)"},
             "prefill_ms": pre_avg,
-            "gpu_launches": (int(run_pre) + int(run_dec)) * args.steps,
+            "gpu_launches": (int(run_pre) + 2 * int(run_dec)) * args.steps,
             "clocks": clk.summary(),
         }
         if e2e_ms is not None:

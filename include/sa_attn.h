@@ -73,13 +73,11 @@ int sa_attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse
 
 /*
  * Bytes of decode workspace needed for `num_splits` (0 = the automatic choice):
- * 65536 + B * Hq * splits * (D + 4) * 4.  Layout: a 64 KiB header of arrival counters
- * (one per (b, kv head, group of up to 16 query heads)), then per (b, h, split) the
- * split's running max and two running sums (of the 16-bit weights the MMA used, and of
- * the fp32 weights for the LSE) padded to 4 floats, then its unnormalised fp32 output
- * row -- the partial online-softmax states of the StreamAttention page, "Engine
- * Direction".
- * Returns 0 for empty problems, invalid sizes or B * Hkv * ceil(Hq / Hkv / 16) > 16384.
+ * B * Hq * splits * (D + 4) * 4.  It holds, per (b, h, split), the split's running max
+ * and two running sums (of the 16-bit weights the MMA used, and of the fp32 weights for
+ * the LSE) padded to 4 floats, then its unnormalised fp32 output row -- the partial
+ * online-softmax states of the StreamAttention page, "Engine Direction".
+ * Returns 0 for empty problems or invalid sizes.
  */
 size_t sa_attn_decode_workspace_size(int B, int Sk, int Hq, int Hkv, int D, int num_splits);
 
@@ -95,14 +93,10 @@ int sa_attn_decode_num_splits(int B, int Sk, int Hq, int Hkv, int D);
  *   num_splits : KV splits per (b, kv head); 0 = automatic; clamped to ceil(Sk / 64) and
  *                to 192 (D = 64) / 96 (D = 128).
  *   workspace  : device buffer of at least sa_attn_decode_workspace_size(...) bytes,
- *                16-byte aligned, owned by the caller.  ZERO-FILL IT ONCE after allocating
- *                it (e.g. cudaMemsetAsync): its first 64 KiB hold arrival counters that
- *                every call leaves at zero, at a place independent of the problem size,
- *                so one workspace serves any later call that fits in it.  The rest is
- *                scratch.  Calls that may run concurrently must not share a workspace.
- * Launches one kernel: each split runs the online-softmax recurrence over its keys and
- * writes its partial state; the last split of each (b, kv head, head group) to finish
- * merges them with log-sum-exp weights and writes O and LSE.
+ *                16-byte aligned, owned by the caller; scratch (no initial contents
+ *                needed, overwritten); calls that may run concurrently must not share it.
+ * Launches the split kernel and, with programmatic dependent launch on the same stream,
+ * the combine kernel (one CTA per (b, h)) that merges the splits with log-sum-exp weights.
  */
 int sa_attn_decode(const void* q, const void* k, const void* v, void* o, float* lse,
                    int B, int Sk, int Hq, int Hkv, int D, float scale, int dtype,

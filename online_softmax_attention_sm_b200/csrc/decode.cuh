@@ -16,9 +16,9 @@
 //   * S = Q K^T and O += P V on mma.sync.m16n8k16 (fp32 accumulate), fragments from
 //     ldmatrix; row max / sum by quad shuffles; the 4 warps merge through shared memory;
 //   * each split writes (unnormalised O, running max, two running sums) in fp32 to the
-//     workspace and arrives on its group's counter; the last CTA of the group merges all
-//     splits (one kernel, no second launch -- the page's two-kernel prototype lost to
-//     launch and merge overhead at small batch).
+//     workspace; a combine kernel with one CTA per (batch, query head) merges them.  It
+//     is launched with programmatic dependent launch, so its launch overlaps the split
+//     grid (the page's two-kernel prototype lost to launch and merge overhead).
 #pragma once
 #include "ptx.cuh"
 #include <cuda_fp16.h>
@@ -36,22 +36,15 @@ struct DecCfg {
   static constexpr int STAGES = (D == 64) ? 4 : 2;
   static constexpr int SMEM_STAGES = STAGES * 2 * KV_BYTES;
   // write_partial's buffers; decode_merge uses the SMEM_STAGES region
-  static constexpr int SMEM_MERGE = 4 * 16 * D * 4 + 3 * 4 * 16 * 4;
+  static constexpr int SMEM_MERGE = 4 * 16 * (D + 4) * 4 + 3 * 4 * 16 * 4;
   static constexpr int SMEM_TOTAL = 1024 + (SMEM_STAGES > SMEM_MERGE ? SMEM_STAGES : SMEM_MERGE) + 256;
 };
 
-// Workspace layout (caller-owned, zero-filled once when allocated):
-//   [0, kDecCounterBytes)   arrival counters, one per (b, kv head, head group); every
-//                           call leaves them at zero, and their place does not depend on
-//                           the problem size, so one workspace serves any shape
-//   then ws_ml [B, Hq, nsplit, 4] fp32 (max, 16-bit-weight sum, fp32 sum, pad),
-//   then ws_o [B, Hq, nsplit, D] fp32
-constexpr int kDecMaxGroups = 16384;
-constexpr size_t kDecCounterBytes = kDecMaxGroups * sizeof(unsigned int);
-
+// Workspace layout (caller-owned scratch, contents irrelevant between calls):
+//   ws_ml [B, Hq, nsplit, 4] fp32 (max, 16-bit-weight sum, fp32 sum, pad),
+//   then ws_o [B, Hq, nsplit, D] fp32.
 struct DecParams {
   const void* q;       // [B, Hq, D]
-  unsigned int* counters;  // [B * Hkv * ngrp] arrival counters (see above)
   float* ws_o;         // [B, Hq, nsplit, D]
   float* ws_ml;        // [B, Hq, nsplit, 4]: max (log2 units of c2*s), 16-bit-weight sum, fp32 sum, 0
   void* o;             // [B, Hq, D]
@@ -119,8 +112,9 @@ __device__ __forceinline__ void write_partial(const DecParams& p, uint8_t* smem,
   e0 += __shfl_xor_sync(0xffffffffu, e0, 2);
   e1 += __shfl_xor_sync(0xffffffffu, e1, 1);
   e1 += __shfl_xor_sync(0xffffffffu, e1, 2);
-  float* sm_o = reinterpret_cast<float*>(smem);              // [4][16][D] (stages are drained)
-  float* sm_m = sm_o + 4 * 16 * D;                           // [4][16]
+  constexpr int LD = D + 4;                                  // padded row: no bank conflicts
+  float* sm_o = reinterpret_cast<float*>(smem);              // [4][16][LD] (stages are drained)
+  float* sm_m = sm_o + 4 * 16 * LD;                          // [4][16]
   float* sm_l = sm_m + 64;                                   // [4][16]
   float* sm_e = sm_l + 64;                                   // [4][16]
   const int r0 = lane >> 2, r1 = r0 + 8;
@@ -138,10 +132,8 @@ __device__ __forceinline__ void write_partial(const DecParams& p, uint8_t* smem,
 #pragma unroll
   for (int n = 0; n < D / 8; ++n) {
     const int c = n * 8 + (lane & 3) * 2;
-    sm_o[(warp * 16 + r0) * D + c] = o[n][0] * w0;
-    sm_o[(warp * 16 + r0) * D + c + 1] = o[n][1] * w0;
-    sm_o[(warp * 16 + r1) * D + c] = o[n][2] * w1;
-    sm_o[(warp * 16 + r1) * D + c + 1] = o[n][3] * w1;
+    *reinterpret_cast<float2*>(&sm_o[(warp * 16 + r0) * LD + c]) = make_float2(o[n][0] * w0, o[n][1] * w0);
+    *reinterpret_cast<float2*>(&sm_o[(warp * 16 + r1) * LD + c]) = make_float2(o[n][2] * w1, o[n][3] * w1);
   }
   __syncthreads();
   const size_t ws_row0 = ((size_t)b * p.Hq + h0) * p.nsplit + split;   // row r -> + r * nsplit
@@ -149,7 +141,7 @@ __device__ __forceinline__ void write_partial(const DecParams& p, uint8_t* smem,
     const int r = i / D, d = i % D;
     float acc = 0.f;
 #pragma unroll
-    for (int w = 0; w < 4; ++w) acc += sm_o[(w * 16 + r) * D + d];
+    for (int w = 0; w < 4; ++w) acc += sm_o[(w * 16 + r) * LD + d];
     p.ws_o[(ws_row0 + (size_t)r * p.nsplit) * D + d] = acc;
   }
   if (threadIdx.x < nrows) {
@@ -169,94 +161,11 @@ __device__ __forceinline__ void write_partial(const DecParams& p, uint8_t* smem,
   }
 }
 
-// LSE-weighted merge of every split's partial state, done by the last CTA of a
-// (batch, KV head, head group) to arrive:
-//   M = max_s m_s,  w_s = 2^(m_s - M),  O = sum_s w_s O_s / sum_s w_s l_s,
-//   LSE = (M + log2 sum_s w_s e_s) * ln 2.
-// The group's partial states are contiguous in the workspace; they are pulled into
-// shared memory a batch of rows at a time with 16-byte cp.async copies (all in flight at
-// once), then merged from shared memory.
+// Splits are capped so the combine's per-row weight table stays small.
 template <int D>
 struct DecMerge {
-  // splits are capped so that one row's partial states fit the merge buffer
   static constexpr int MAX_SPLITS = (D == 64) ? 192 : 96;
-  static constexpr int ROW_BYTES_PER_SPLIT = (D + 4) * 4;
 };
-
-__device__ __forceinline__ void cp_async16(void* smem_dst, const void* gmem_src) {
-  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_u32(smem_dst)), "l"(gmem_src) : "memory");
-}
-__device__ __forceinline__ void cp_async_wait_all() {
-  asm volatile("cp.async.wait_all;" ::: "memory");
-}
-
-template <int D, bool BF16>
-__device__ __forceinline__ void decode_merge(const DecParams& p, uint8_t* smem, int smem_bytes, int b, int h0,
-                                             int nrows) {
-  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int ns = p.nsplit;
-  const int rows_per_batch = max(1, smem_bytes / (ns * DecMerge<D>::ROW_BYTES_PER_SPLIT));
-  const size_t row0 = (size_t)b * p.Hq + h0;
-  for (int rb = 0; rb < nrows; rb += rows_per_batch) {
-    const int nr = min(rows_per_batch, nrows - rb);
-    float* s_ml = reinterpret_cast<float*>(smem);                 // [nr][ns][4]
-    float* s_o = s_ml + (size_t)nr * ns * 4;                       // [nr][ns][D]
-    const float4* g_ml = reinterpret_cast<const float4*>(p.ws_ml + (row0 + rb) * ns * 4);
-    const float4* g_o = reinterpret_cast<const float4*>(p.ws_o + (row0 + rb) * ns * D);
-    const int n_ml = nr * ns, n_o = nr * ns * (D / 4);
-    for (int i = tid; i < n_ml; i += 128) cp_async16(s_ml + 4 * i, g_ml + i);
-    for (int i = tid; i < n_o; i += 128) cp_async16(s_o + 4 * i, g_o + i);
-    cp_async_wait_all();
-    __syncthreads();
-    // per row: max, weights (kept in the pad slot), sums -- warp w takes rows w, w + 4, ...
-    __shared__ float s_LE[16][2];
-    for (int r = warp; r < nr; r += 4) {
-      float* ml = s_ml + (size_t)r * ns * 4;
-      float M = -INFINITY;
-      for (int s = lane; s < ns; s += 32) M = fmaxf(M, ml[4 * s]);
-#pragma unroll
-      for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
-      float L = 0.f, E = 0.f;
-      for (int s = lane; s < ns; s += 32) {
-        const float ms = ml[4 * s];
-        const float w = (ms == -INFINITY) ? 0.f : ex2(ms - M);
-        ml[4 * s + 3] = w;
-        L += w * ml[4 * s + 1];
-        E += w * ml[4 * s + 2];
-      }
-#pragma unroll
-      for (int o = 16; o > 0; o >>= 1) {
-        L += __shfl_xor_sync(0xffffffffu, L, o);
-        E += __shfl_xor_sync(0xffffffffu, E, o);
-      }
-      if (lane == 0) {
-        s_LE[r][0] = L;
-        if (p.lse) p.lse[row0 + rb + r] = E > 0.f ? (M + __log2f(E)) * 0.69314718055994531f : -INFINITY;
-      }
-    }
-    __syncthreads();
-    // O[r][d] = sum_s w_s O_s[d] / L
-    using T = typename std::conditional<BF16, __nv_bfloat16, __half>::type;
-    for (int i = tid; i < nr * D; i += 128) {
-      const int r = i / D, d = i % D;
-      const float* ml = s_ml + (size_t)r * ns * 4;
-      const float* o = s_o + (size_t)r * ns * D + d;
-      float a0 = 0.f, a1 = 0.f;
-      int s = 0;
-      for (; s + 1 < ns; s += 2) {
-        a0 = fmaf(ml[4 * s + 3], o[(size_t)s * D], a0);
-        a1 = fmaf(ml[4 * s + 7], o[(size_t)(s + 1) * D], a1);
-      }
-      if (s < ns) a0 = fmaf(ml[4 * s + 3], o[(size_t)s * D], a0);
-      const float L = s_LE[r][0];
-      const float v = L > 0.f ? (a0 + a1) / L : 0.f;
-      T* out = reinterpret_cast<T*>(p.o) + (row0 + rb + r) * D + d;
-      if (BF16) *reinterpret_cast<__nv_bfloat16*>(out) = __float2bfloat16_rn(v);
-      else *reinterpret_cast<__half*>(out) = __float2half_rn(v);
-    }
-    __syncthreads();                                            // buffer reused by the next batch
-  }
-}
 
 template <int D, bool BF16>
 __global__ void __launch_bounds__(128, 3)
@@ -269,6 +178,8 @@ attn_decode_split(const __grid_constant__ CUtensorMap tm_k, const __grid_constan
   uint64_t* full = (uint64_t*)(smem + region);
   volatile int* abort_flag = (volatile int*)(full + Cfg::STAGES);
 
+  // let the combine grid launch now (it waits for this grid's results before reading)
+  asm volatile("griddepcontrol.launch_dependents;");
   const int split = blockIdx.x;
   const int kvh = blockIdx.y / p.ngrp;
   const int grp = blockIdx.y % p.ngrp;
@@ -421,25 +332,95 @@ attn_decode_split(const __grid_constant__ CUtensorMap tm_k, const __grid_constan
         mbar_wait(&full[st % Cfg::STAGES], (st / Cfg::STAGES) & 1, nullptr, 41);
     }
     __syncthreads();
-    // still arrive below, so the group's counter completes and resets (the outputs of a
-    // call whose wait expired are undefined; the status word reports it)
-  } else {
-    write_partial<D>(p, smem, b, h0, nrows, split, warp, lane, o, m0, m1, l0, l1, e0, e1);
+    return;                                                   // outputs undefined; status word set
   }
-  __threadfence();                                            // partials visible device-wide
-  __shared__ int s_last;
+  write_partial<D>(p, smem, b, h0, nrows, split, warp, lane, o, m0, m1, l0, l1, e0, e1);
+}
+
+// Merge of every split's partial state for one (batch, query head) row per CTA:
+//   M = max_s m_s,  w_s = 2^(m_s - M),  O = sum_s w_s O_s / sum_s w_s l_s,
+//   LSE = (M + log2 sum_s w_s e_s) * ln 2.
+// Launched with programmatic dependent launch right behind the split kernel: its CTAs are
+// resident before the split grid ends and proceed the moment its results are visible.
+// Thread t owns float4 column c = t % (D/4) and the splits s = g, g + 128/(D/4), ... with
+// g = t / (D/4); the per-group partial sums are added through shared memory.
+template <int D, bool BF16>
+__global__ void __launch_bounds__(128)
+attn_decode_combine(const DecParams p) {
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+  constexpr int NC = D / 4, NG = 128 / NC;
+  __shared__ float s_w[DecMerge<D>::MAX_SPLITS];
+  __shared__ float s_red[3][4];
+  __shared__ float4 s_acc[128];
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const size_t row = blockIdx.x;                              // b * Hq + h
+  const int ns = p.nsplit;
+  const float4* ml = reinterpret_cast<const float4*>(p.ws_ml) + row * ns;
+  const float4* os = reinterpret_cast<const float4*>(p.ws_o) + row * ns * NC;
+  // 1. max over splits
+  float M = -INFINITY;
+  for (int s = tid; s < ns; s += 128) M = fmaxf(M, ml[s].x);
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
+  if (lane == 0) s_red[0][warp] = M;
   __syncthreads();
-  if (threadIdx.x == 0) {
-    unsigned int* ctr = p.counters + ((size_t)b * p.Hkv + kvh) * p.ngrp + grp;
-    const unsigned int prev = atomicAdd(ctr, 1u);
-    s_last = (prev == (unsigned)p.nsplit - 1u);
-    if (s_last) *ctr = 0u;                                    // ready for the next call
+  M = fmaxf(fmaxf(s_red[0][0], s_red[0][1]), fmaxf(s_red[0][2], s_red[0][3]));
+  // 2. weights and the two sums
+  float L = 0.f, E = 0.f;
+  for (int s = tid; s < ns; s += 128) {
+    const float4 v = ml[s];
+    const float w = (v.x == -INFINITY) ? 0.f : ex2(v.x - M);
+    s_w[s] = w;
+    L = fmaf(w, v.y, L);
+    E = fmaf(w, v.z, E);
   }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    L += __shfl_xor_sync(0xffffffffu, L, o);
+    E += __shfl_xor_sync(0xffffffffu, E, o);
+  }
+  __syncthreads();                                            // s_red[0] consumed, s_w written
+  if (lane == 0) { s_red[1][warp] = L; s_red[2][warp] = E; }
   __syncthreads();
-  if (s_last) {
-    __threadfence();
-    decode_merge<D, BF16>(p, smem, Cfg::SMEM_STAGES, b, h0, nrows);
+  L = (s_red[1][0] + s_red[1][1]) + (s_red[1][2] + s_red[1][3]);
+  E = (s_red[2][0] + s_red[2][1]) + (s_red[2][2] + s_red[2][3]);
+  // 3. weighted sum of the partial outputs; loads of 8 splits in flight per thread
+  const int c = tid % NC, g = tid / NC;
+  float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+  int s = g;
+  for (; s + 7 * NG < ns; s += 8 * NG) {
+    float4 v[8];
+#pragma unroll
+    for (int u = 0; u < 8; ++u) v[u] = os[(size_t)(s + u * NG) * NC + c];
+#pragma unroll
+    for (int u = 0; u < 8; ++u) {
+      const float w = s_w[s + u * NG];
+      acc.x = fmaf(w, v[u].x, acc.x); acc.y = fmaf(w, v[u].y, acc.y);
+      acc.z = fmaf(w, v[u].z, acc.z); acc.w = fmaf(w, v[u].w, acc.w);
+    }
   }
+  for (; s < ns; s += NG) {
+    const float4 v = os[(size_t)s * NC + c];
+    const float w = s_w[s];
+    acc.x = fmaf(w, v.x, acc.x); acc.y = fmaf(w, v.y, acc.y);
+    acc.z = fmaf(w, v.z, acc.z); acc.w = fmaf(w, v.w, acc.w);
+  }
+  s_acc[tid] = acc;
+  __syncthreads();
+  if (tid < NC) {
+    float4 a = s_acc[tid];
+#pragma unroll
+    for (int k = 1; k < NG; ++k) {
+      const float4 b2 = s_acc[k * NC + tid];
+      a.x += b2.x; a.y += b2.y; a.z += b2.z; a.w += b2.w;
+    }
+    const float inv = L > 0.f ? 1.f / L : 0.f;
+    uint2 packed;
+    packed.x = pack2<BF16>(a.x * inv, a.y * inv);
+    packed.y = pack2<BF16>(a.z * inv, a.w * inv);
+    reinterpret_cast<uint2*>(reinterpret_cast<uint16_t*>(p.o) + row * D)[tid] = packed;
+  }
+  if (p.lse && tid == 0) p.lse[row] = E > 0.f ? (M + __log2f(E)) * 0.69314718055994531f : -INFINITY;
 }
 
 }  // namespace sa

@@ -160,7 +160,7 @@ int launch_simple(const void* q, const void* k, const void* v, void* o, float* l
 
 // ---------------------------------------------------------------- decode planning
 size_t dec_ws_bytes(int B, int Hq, int nsplit, int D) {
-  return sa::kDecCounterBytes + (size_t)B * Hq * nsplit * (D + 4) * sizeof(float);
+  return (size_t)B * Hq * nsplit * (D + 4) * sizeof(float);
 }
 
 struct DecPlan {
@@ -195,8 +195,7 @@ int launch_decode(const void* q, const void* k, const void* v, void* o, float* l
   if ((rc = make_map(&mv, v, BF16, D, Hkv, Sk, B, 64)) != SA_OK) return rc;
   sa::DecParams p;
   p.q = q;
-  p.counters = reinterpret_cast<unsigned int*>(ws);
-  p.ws_ml = reinterpret_cast<float*>(reinterpret_cast<char*>(ws) + sa::kDecCounterBytes);
+  p.ws_ml = reinterpret_cast<float*>(ws);
   p.ws_o = p.ws_ml + (size_t)B * Hq * pl.nsplit * 4;
   p.o = o; p.lse = lse;
   p.B = B; p.Sk = Sk; p.Hq = Hq; p.Hkv = Hkv; p.G = Hq / Hkv; p.ngrp = pl.ngrp;
@@ -210,7 +209,20 @@ int launch_decode(const void* q, const void* k, const void* v, void* o, float* l
   if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(attn_decode_split)");
   ks<<<grid, 128, Cfg::SMEM_TOTAL, st>>>(mk, mv, p);
   e = cudaGetLastError();
-  return e == cudaSuccess ? SA_OK : cuda_fail(e, "attn_decode_split launch");
+  if (e != cudaSuccess) return cuda_fail(e, "attn_decode_split launch");
+  // combine: programmatic dependent launch, resident and waiting when the split grid ends
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)(B * Hq));
+  cfg.blockDim = dim3(128);
+  cfg.dynamicSmemBytes = 0;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  e = cudaLaunchKernelEx(&cfg, sa::attn_decode_combine<D, BF16>, p);
+  return e == cudaSuccess ? SA_OK : cuda_fail(e, "attn_decode_combine launch");
 }
 
 }  // namespace
@@ -259,7 +271,6 @@ size_t sa_attn_decode_workspace_size(int B, int Sk, int Hq, int Hkv, int D, int 
   if (num_splits < 0 || check_dims(B, 1, Sk, Hq, Hkv, D, SA_FP16, 1.f) != SA_OK) return 0;
   if (B == 0 || Hq == 0 || Sk == 0) return 0;
   DecPlan pl = plan_decode(B, Sk, Hq, Hkv, D, num_splits, num_sms());
-  if ((long long)B * Hkv * pl.ngrp > sa::kDecMaxGroups) return 0;
   return dec_ws_bytes(B, Hq, pl.nsplit, D);
 }
 
@@ -274,9 +285,6 @@ int sa_attn_decode(const void* q, const void* k, const void* v, void* o, float* 
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   if (Sk == 0) return launch_fill(o, (size_t)B * Hq * D, lse, (size_t)B * Hq, st);
   DecPlan pl = plan_decode(B, Sk, Hq, Hkv, D, num_splits, num_sms());
-  if ((long long)B * Hkv * pl.ngrp > sa::kDecMaxGroups)
-    return fail(SA_ERR_UNSUPPORTED, "B * Hkv * ceil(G / 16) = %lld exceeds %d", (long long)B * Hkv * pl.ngrp,
-                sa::kDecMaxGroups);
   const size_t need = dec_ws_bytes(B, Hq, pl.nsplit, D);
   if (!workspace || workspace_bytes < need)
     return fail(SA_ERR_WORKSPACE, "decode workspace of %zu bytes needed (got %zu)", need,

@@ -140,8 +140,7 @@ def sa_attn_decode(q, k, v, scale=None, num_splits=0, workspace=None, out=None, 
         lse = torch.empty((B, Hq), dtype=torch.float32, device=q.device)
     need = sa_attn_decode_workspace_size(B, Sk, Hq, Hkv, D, num_splits)
     if workspace is None:
-        # zero-filled once: the header of arrival counters must start at zero
-        workspace = torch.zeros(max(need, 16), dtype=torch.uint8, device=q.device)
+        workspace = torch.empty(max(need, 16), dtype=torch.uint8, device=q.device)
     _check(lib().sa_attn_decode(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse), B, Sk, Hq, Hkv, D,
                                 float(scale), _DT[q.dtype], int(num_splits), _ptr(workspace),
                                 workspace.numel() * workspace.element_size(), _stream(stream)))

@@ -1,4 +1,4 @@
-"""GPU parity of the split-KV decode (sa_attn_decode: split kernel + combine) against the
+"""GPU parity of the split-KV decode (sa_attn_decode: split kernel + PDL combine) against the
 fp64 oracle, and its invariants."""
 import numpy as np
 import pytest
@@ -73,30 +73,27 @@ def test_decode_workspace_contract():
     ns = sa_attn_decode_num_splits(B, Sk, Hq, Hkv, D)
     assert 1 <= ns <= Sk // 64
     need = sa_attn_decode_workspace_size(B, Sk, Hq, Hkv, D)
-    assert need == 65536 + B * Hq * ns * (D + 4) * 4
+    assert need == B * Hq * ns * (D + 4) * 4
     q, k, v = make_qkv(B, 1, Sk, Hq, Hkv, D, "fp16", seed=25, decode=True)
-    # zeroed counter header, garbage scratch, canary past the declared size
+    # garbage scratch, canary past the declared size
     ws = torch.full((need + 4096,), 0x5A, dtype=torch.uint8, device=dev())
-    ws[:65536] = 0
     o, l = sa_attn_decode(q.to(dev()), k.to(dev()), v.to(dev()), workspace=ws)
     sa_check_status()
     assert torch.all(ws[-4096:] == 0x5A), "wrote past the declared workspace size"
-    assert torch.all(ws[:65536] == 0), "arrival counters not left at zero"
     O, L = oracle.decode(f64(q), f64(k), f64(v), 1 / 8.0)
     assert_close(o, l, O, L, "fp16", "workspace contract")
 
 
 def test_decode_one_workspace_serves_many_shapes():
     # a serving loop: the KV length grows and the batch changes between calls that reuse
-    # one workspace (zero-filled once, sized for the largest call)
+    # one workspace sized for the largest call
     shapes = [(2, 100, 14, 2, 64, "fp16"), (8, 9000, 16, 2, 128, "bf16"), (1, 5000, 8, 8, 64, "fp16"),
               (3, 8191, 16, 1, 128, "bf16"), (2, 101, 14, 2, 64, "fp16")]
-    ws = torch.zeros(max(sa_attn_decode_workspace_size(*sh[:5]) for sh in shapes),
-                     dtype=torch.uint8, device=dev())
+    ws = torch.full((max(sa_attn_decode_workspace_size(*sh[:5]) for sh in shapes),), 0x77,
+                    dtype=torch.uint8, device=dev())
     for i, (B, Sk, Hq, Hkv, D, dt) in enumerate(shapes):
         q, k, v = make_qkv(B, 1, Sk, Hq, Hkv, D, dt, seed=30 + i, decode=True)
         o, l = sa_attn_decode(q.to(dev()), k.to(dev()), v.to(dev()), workspace=ws)
         sa_check_status()
         O, L = oracle.decode(f64(q), f64(k), f64(v), 1 / np.sqrt(D))
         assert_close(o, l, O, L, dt, f"reuse #{i}")
-    assert torch.all(ws[:65536] == 0)
