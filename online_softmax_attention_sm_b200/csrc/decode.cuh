@@ -342,14 +342,19 @@ attn_decode_split(const __grid_constant__ CUtensorMap tm_k, const __grid_constan
 //   LSE = (M + log2 sum_s w_s e_s) * ln 2.
 // Launched with programmatic dependent launch right behind the split kernel: its CTAs are
 // resident before the split grid ends and proceed the moment its results are visible.
-// Thread t owns float4 column c = t % (D/4) and the splits s = g, g + 128/(D/4), ... with
-// g = t / (D/4); the per-group partial sums are added through shared memory.
+// Every load (the split maxima/sums and the partial output rows) is issued up front, so
+// the merge costs one round trip to L2.  Thread t owns float4 column c = t % (D/4) and the
+// splits s = g, g + NG, ... with g = t / (D/4), NG = 128 / (D/4); the NG partial sums per
+// column are added through shared memory.
 template <int D, bool BF16>
 __global__ void __launch_bounds__(128)
 attn_decode_combine(const DecParams p) {
   asm volatile("griddepcontrol.wait;" ::: "memory");
   constexpr int NC = D / 4, NG = 128 / NC;
-  __shared__ float s_w[DecMerge<D>::MAX_SPLITS];
+  constexpr int MAXS = DecMerge<D>::MAX_SPLITS;
+  constexpr int PER = (MAXS + NG - 1) / NG;                   // splits per thread, at most
+  static_assert(MAXS <= 256, "two split maxima per thread");
+  __shared__ float s_w[MAXS];
   __shared__ float s_red[3][4];
   __shared__ float4 s_acc[128];
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
@@ -357,23 +362,30 @@ attn_decode_combine(const DecParams p) {
   const int ns = p.nsplit;
   const float4* ml = reinterpret_cast<const float4*>(p.ws_ml) + row * ns;
   const float4* os = reinterpret_cast<const float4*>(p.ws_o) + row * ns * NC;
-  // 1. max over splits
-  float M = -INFINITY;
-  for (int s = tid; s < ns; s += 128) M = fmaxf(M, ml[s].x);
+  const int c = tid % NC, g = tid / NC;
+  // all loads first
+  const float4 ninf = make_float4(-INFINITY, 0.f, 0.f, 0.f);
+  const float4 mlA = tid < ns ? ml[tid] : ninf;
+  const float4 mlB = tid + 128 < ns ? ml[tid + 128] : ninf;
+  float4 v[PER];
+#pragma unroll
+  for (int u = 0; u < PER; ++u) {
+    const int s = g + u * NG;
+    v[u] = s < ns ? os[(size_t)s * NC + c] : make_float4(0.f, 0.f, 0.f, 0.f);
+  }
+  // max over splits
+  float M = fmaxf(mlA.x, mlB.x);
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
   if (lane == 0) s_red[0][warp] = M;
   __syncthreads();
   M = fmaxf(fmaxf(s_red[0][0], s_red[0][1]), fmaxf(s_red[0][2], s_red[0][3]));
-  // 2. weights and the two sums
-  float L = 0.f, E = 0.f;
-  for (int s = tid; s < ns; s += 128) {
-    const float4 v = ml[s];
-    const float w = (v.x == -INFINITY) ? 0.f : ex2(v.x - M);
-    s_w[s] = w;
-    L = fmaf(w, v.y, L);
-    E = fmaf(w, v.z, E);
-  }
+  // weights and the two sums
+  const float wA = (mlA.x == -INFINITY) ? 0.f : ex2(mlA.x - M);
+  const float wB = (mlB.x == -INFINITY) ? 0.f : ex2(mlB.x - M);
+  if (tid < ns) s_w[tid] = wA;
+  if (tid + 128 < ns) s_w[tid + 128] = wB;
+  float L = wA * mlA.y + wB * mlB.y, E = wA * mlA.z + wB * mlB.z;
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) {
     L += __shfl_xor_sync(0xffffffffu, L, o);
@@ -384,26 +396,14 @@ attn_decode_combine(const DecParams p) {
   __syncthreads();
   L = (s_red[1][0] + s_red[1][1]) + (s_red[1][2] + s_red[1][3]);
   E = (s_red[2][0] + s_red[2][1]) + (s_red[2][2] + s_red[2][3]);
-  // 3. weighted sum of the partial outputs; loads of 8 splits in flight per thread
-  const int c = tid % NC, g = tid / NC;
+  // weighted sum of this thread's splits
   float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-  int s = g;
-  for (; s + 7 * NG < ns; s += 8 * NG) {
-    float4 v[8];
 #pragma unroll
-    for (int u = 0; u < 8; ++u) v[u] = os[(size_t)(s + u * NG) * NC + c];
-#pragma unroll
-    for (int u = 0; u < 8; ++u) {
-      const float w = s_w[s + u * NG];
-      acc.x = fmaf(w, v[u].x, acc.x); acc.y = fmaf(w, v[u].y, acc.y);
-      acc.z = fmaf(w, v[u].z, acc.z); acc.w = fmaf(w, v[u].w, acc.w);
-    }
-  }
-  for (; s < ns; s += NG) {
-    const float4 v = os[(size_t)s * NC + c];
-    const float w = s_w[s];
-    acc.x = fmaf(w, v.x, acc.x); acc.y = fmaf(w, v.y, acc.y);
-    acc.z = fmaf(w, v.z, acc.z); acc.w = fmaf(w, v.w, acc.w);
+  for (int u = 0; u < PER; ++u) {
+    const int s = g + u * NG;
+    const float w = s < ns ? s_w[s] : 0.f;
+    acc.x = fmaf(w, v[u].x, acc.x); acc.y = fmaf(w, v[u].y, acc.y);
+    acc.z = fmaf(w, v[u].z, acc.z); acc.w = fmaf(w, v[u].w, acc.w);
   }
   s_acc[tid] = acc;
   __syncthreads();

@@ -115,8 +115,12 @@ def test_workspace_size(L):
     assert L.sa_attn_decode_workspace_size(4, 32768, 14, 2, 64, 8) == 4 * 14 * 8 * 68 * 4
     # clamped to ceil(Sk / 64) splits, and to 192 (D = 64) / 96 (D = 128)
     assert L.sa_attn_decode_workspace_size(1, 100, 2, 1, 128, 50) == 1 * 2 * 2 * 132 * 4
-    assert L.sa_attn_decode_workspace_size(1, 1 << 20, 2, 1, 64, 5000) == 1 * 2 * 192 * 68 * 4
-    assert L.sa_attn_decode_workspace_size(1, 1 << 20, 2, 1, 128, 5000) == 1 * 2 * 96 * 132 * 4
+    def splits(Sk, cap):                      # chunk = ceil(Sk / cap) rounded up to 64 tokens
+        chunk = -(-(-(-Sk // cap)) // 64) * 64
+        return -(-Sk // chunk)
+    assert L.sa_attn_decode_workspace_size(1, 1 << 20, 2, 1, 64, 5000) == 1 * 2 * splits(1 << 20, 192) * 68 * 4
+    assert L.sa_attn_decode_workspace_size(1, 1 << 20, 2, 1, 128, 5000) == 1 * 2 * splits(1 << 20, 96) * 132 * 4
+    assert splits(1 << 20, 192) <= 192 and splits(1 << 20, 96) <= 96
     assert L.sa_attn_decode_workspace_size(1, 100, 3, 2, 64, 1) == 0      # invalid GQA
     assert L.sa_attn_decode_workspace_size(0, 100, 2, 2, 64, 1) == 0      # empty
     assert L.sa_attn_decode_num_splits(1, 100, 3, 2, 64) == 0
