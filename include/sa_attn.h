@@ -104,6 +104,28 @@ int sa_attn_decode(const void* q, const void* k, const void* v, void* o, float* 
                    sa_stream_t stream);
 
 /*
+ * The same decode as sa_attn_decode, for callers that cannot hand the library any device
+ * memory for scratch: runtimes that reserve all GPU memory up front and forbid further
+ * allocation, or hosts whose allocator is not reachable from the code that issues the
+ * call.  (The pages have no counterpart; this is a deployment convenience.)
+ *   Arguments as for sa_attn_decode, minus the workspace.  The scratch is a fixed 8 MiB
+ *   area inside the library's device image, present on every GPU that loads the library
+ *   until the process exits; this call allocates nothing (no cudaMalloc, cudaFree or
+ *   allocating library routine).
+ *   Limit: the split states must fit, B * Hq * splits * (D + 4) * 4 <= 8 MiB (splits as
+ *   chosen by num_splits, see sa_attn_decode_workspace_size); larger problems return
+ *   SA_ERR_UNSUPPORTED and leave the outputs untouched.
+ *   The first call on a device looks up the area's device address (with that device
+ *   current) and caches it; make that first call before any stream capture.
+ *   Every call uses the same area: calls whose work may overlap on the GPU (other
+ *   streams, other host threads) race and give undefined results.  Nothing in the area
+ *   needs to start at zero; each call writes every byte it reads.
+ */
+int sa_attn_decode_noalloc(const void* q, const void* k, const void* v, void* o, float* lse,
+                           int B, int Sk, int Hq, int Hkv, int D, float scale, int dtype,
+                           int num_splits, sa_stream_t stream);
+
+/*
  * Diagnostic only: the same forward as sa_attn_fwd computed by a plain CUDA-core kernel
  * (one thread per query row, fp32 online softmax).  Slow; used to cross-check the
  * tensor-core path.  Same arguments and conventions as sa_attn_fwd.

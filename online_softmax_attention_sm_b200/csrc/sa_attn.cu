@@ -225,6 +225,34 @@ int launch_decode(const void* q, const void* k, const void* v, void* o, float* l
   return e == cudaSuccess ? SA_OK : cuda_fail(e, "attn_decode_combine launch");
 }
 
+// ---------------------------------------------------------------- built-in decode scratch
+// Scratch for sa_attn_decode_noalloc: a fixed area in the library's own device image, so
+// that entry point needs no memory from the caller and allocates none.  Every GPU that
+// loads the library holds it until the process exits.  Host code must not use the
+// symbol's name as an address: the device address is looked up once per device.
+constexpr size_t kNoAllocScratchBytes = 8u << 20;
+static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
+
+// Device address of g_noalloc_scratch on the current device (looked up on the first call
+// per device, with that device current).  Returns SA_OK or SA_ERR_CUDA.
+int noalloc_scratch(void** out) {
+  static std::mutex mu;
+  static void* addr[64] = {nullptr};
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+  if (dev < 0 || dev >= 64) return fail(SA_ERR_UNSUPPORTED, "device ordinal %d out of range", dev);
+  std::lock_guard<std::mutex> lock(mu);
+  if (!addr[dev]) {
+    void* p = nullptr;
+    e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaGetSymbolAddress(built-in decode scratch)");
+    addr[dev] = p;
+  }
+  *out = addr[dev];
+  return SA_OK;
+}
+
 }  // namespace
 
 extern "C" {
@@ -295,6 +323,30 @@ int sa_attn_decode(const void* q, const void* k, const void* v, void* o, float* 
                          : launch_decode<64, false>(q, k, v, o, lse, B, Sk, Hq, Hkv, scale, pl, workspace, st);
   return bf ? launch_decode<128, true>(q, k, v, o, lse, B, Sk, Hq, Hkv, scale, pl, workspace, st)
             : launch_decode<128, false>(q, k, v, o, lse, B, Sk, Hq, Hkv, scale, pl, workspace, st);
+}
+
+int sa_attn_decode_noalloc(const void* q, const void* k, const void* v, void* o, float* lse, int B,
+                           int Sk, int Hq, int Hkv, int D, float scale, int dtype, int num_splits,
+                           sa_stream_t stream) {
+  int rc = check_dims(B, 1, Sk, Hq, Hkv, D, dtype, scale);
+  if (rc != SA_OK) return rc;
+  if (num_splits < 0) return fail(SA_ERR_INVALID, "num_splits must be >= 0");
+  if (B == 0 || Hq == 0) return SA_OK;
+  if ((rc = check_ptrs(q, Sk ? k : q, Sk ? v : q, o, lse)) != SA_OK) return rc;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  if (Sk == 0) return launch_fill(o, (size_t)B * Hq * D, lse, (size_t)B * Hq, st);
+  DecPlan pl = plan_decode(B, Sk, Hq, Hkv, D, num_splits, num_sms());
+  const size_t need = dec_ws_bytes(B, Hq, pl.nsplit, D);
+  if (need > kNoAllocScratchBytes)
+    return fail(SA_ERR_UNSUPPORTED, "this decode needs %zu bytes of scratch; the built-in area holds %zu "
+                "(use sa_attn_decode with a caller workspace, or fewer splits)", need, kNoAllocScratchBytes);
+  void* scratch = nullptr;
+  if ((rc = noalloc_scratch(&scratch)) != SA_OK) return rc;
+  const bool bf = dtype == SA_BF16;
+  if (D == 64) return bf ? launch_decode<64, true>(q, k, v, o, lse, B, Sk, Hq, Hkv, scale, pl, scratch, st)
+                         : launch_decode<64, false>(q, k, v, o, lse, B, Sk, Hq, Hkv, scale, pl, scratch, st);
+  return bf ? launch_decode<128, true>(q, k, v, o, lse, B, Sk, Hq, Hkv, scale, pl, scratch, st)
+            : launch_decode<128, false>(q, k, v, o, lse, B, Sk, Hq, Hkv, scale, pl, scratch, st);
 }
 
 const char* sa_last_error(void) { return g_err.c_str(); }

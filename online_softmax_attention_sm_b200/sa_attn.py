@@ -27,6 +27,7 @@ SIGNATURES = {
     "sa_attn_decode_workspace_size": (_Z, [_I, _I, _I, _I, _I, _I]),
     "sa_attn_decode_num_splits": (_I, [_I, _I, _I, _I, _I]),
     "sa_attn_decode": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _F, _I, _I, _P, _Z, _P]),
+    "sa_attn_decode_noalloc": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _F, _I, _I, _P]),
     "sa_last_error": (ctypes.c_char_p, []),
     "sa_check_status": (_I, [_P]),
     "sa_version": (ctypes.c_char_p, []),
