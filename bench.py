@@ -134,6 +134,14 @@ def oracle_prefill_sample(w, q, k, v, seconds, rng_seed=0, max_rows=None):
     return flops, el, f"{rows_done} random query rows (64 per head draw) of {w.name}"
 
 
+def kernel_source_hash():
+    import hashlib
+    h = hashlib.sha256()
+    for f in ("fwd_sm100.cuh", "ptx.cuh"):
+        h.update(open(os.path.join(ROOT, "online_softmax_attention_sm_b200", "csrc", f), "rb").read())
+    return h.hexdigest()
+
+
 def blas_threads():
     try:
         from threadpoolctl import threadpool_info
@@ -334,8 +342,11 @@ def main():
         dec_gbs_step = wd.kv_bytes / (dec_avg * 1e-3) / 1e9
         traffic = None
         prof = os.path.join(ROOT, "profiles", "traffic.json")
-        if os.path.exists(prof):
-            traffic = json.load(open(prof)).get("attn_fwd_sm100")
+        if os.path.exists(prof) and not args.prefill_seq:
+            rec = json.load(open(prof)).get("attn_fwd_sm100") or {}
+            # only while the kernel is the one the counters were taken from
+            if rec.get("kernel_source_sha256") == kernel_source_hash():
+                traffic = rec.get("bytes")
         line = {
             "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_step,
