@@ -349,10 +349,62 @@ __device__ __forceinline__ void fwd_softmax(const FwdParams& p, const FwdSmem<D>
       }
       tmem_wait_ld();
       const bool masked = (j >= mask_from);
-      const bool fast = !masked && c2 >= 0.f;      // the common case: full tile, scale >= 0
-      float m_tile;
-      if (fast) {
-        // row max: 8 independent chains of 3-input max over 16 values each
+      const bool plain = !masked && c2 >= 0.f;     // full tile, scale >= 0: s scaled in the FMA
+      if (!plain) {
+        // diagonal / ragged tiles (and negative scales): scale first, mask
+        const int kl = masked ? klim - j * 128 : 128;   // keys >= kl are invisible to this row
+#pragma unroll
+        for (int i = 0; i < 128; ++i) s[i] = (i < kl) ? s[i] * c2 : -INFINITY;
+      }
+      const f32x2 scale2 = plain ? pack_f2(c2, c2) : pack_f2(1.f, 1.f);
+      // One pass over the tile: p = 2^(scale2 * s - m_use) on pairs (one packed FMA per
+      // pair), P stored to tensor memory as 16-bit, both row sums (rse: fp32 weights for
+      // the LSE; rs: the 16-bit weights the MMA multiplies, so O / l is an exact weighted
+      // average of V), and optionally the row max of s as 8 chains of 3-input max.
+      float sum_r, sum_e, smax = -INFINITY;
+      auto exp_pass = [&](float m_use, bool track_max) {
+        const f32x2 negm2 = pack_f2(-m_use, -m_use);
+        f32x2 rs2[4] = {0ull, 0ull, 0ull, 0ull}, rse2[4] = {0ull, 0ull, 0ull, 0ull};
+        float mx[8];
+#pragma unroll
+        for (int k = 0; k < 8; ++k) mx[k] = -INFINITY;
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+          uint32_t pk[16];
+#pragma unroll
+          for (int i = 0; i < 16; ++i) {
+            const float s0 = s[c * 32 + 2 * i], s1 = s[c * 32 + 2 * i + 1];
+            if (track_max) mx[i & 7] = max3f(mx[i & 7], s0, s1);
+            float x0, x1;
+            unpack_f2(fma_f2(pack_f2(s0, s1), scale2, negm2), x0, x1);
+            const float a = ex2(x0), b2 = ex2(x1);
+            rse2[i & 3] = add_f2(rse2[i & 3], pack_f2(a, b2));
+            float lo, hi;
+            if (BF16) {
+              __nv_bfloat162 h2 = __floats2bfloat162_rn(a, b2);
+              pk[i] = *reinterpret_cast<uint32_t*>(&h2);
+              lo = __uint_as_float(pk[i] << 16);
+              hi = __uint_as_float(pk[i] & 0xffff0000u);
+            } else {
+              __half2 h2 = __floats2half2_rn(a, b2);
+              pk[i] = *reinterpret_cast<uint32_t*>(&h2);
+              const float2 f = __half22float2(h2);
+              lo = f.x;
+              hi = f.y;
+            }
+            rs2[i & 3] = add_f2(rs2[i & 3], pack_f2(lo, hi));
+          }
+          tmem_st16(lane_addr + Cfg::P_COL(t) + c * 16, pk);
+        }
+        float a0, a1, b0, b1;
+        unpack_f2(add_f2(add_f2(rs2[0], rs2[1]), add_f2(rs2[2], rs2[3])), a0, a1);
+        unpack_f2(add_f2(add_f2(rse2[0], rse2[1]), add_f2(rse2[2], rse2[3])), b0, b1);
+        sum_r = a0 + a1;
+        sum_e = b0 + b1;
+        if (track_max)
+          smax = fmaxf(max3f(mx[0], mx[1], mx[2]), max3f(max3f(mx[3], mx[4], mx[5]), mx[6], mx[7]));
+      };
+      auto row_max = [&]() {
         float mx[8];
 #pragma unroll
         for (int k = 0; k < 8; ++k) mx[k] = fmaxf(s[k], s[k + 8]);
@@ -360,69 +412,40 @@ __device__ __forceinline__ void fwd_softmax(const FwdParams& p, const FwdSmem<D>
         for (int i = 16; i < 128; i += 16)
 #pragma unroll
           for (int k = 0; k < 8; ++k) mx[k] = max3f(mx[k], s[i + k], s[i + 8 + k]);
-        m_tile = fmaxf(max3f(mx[0], mx[1], mx[2]), max3f(max3f(mx[3], mx[4], mx[5]), mx[6], mx[7])) * c2;
-      } else {
-        // diagonal / ragged tiles (and negative scales): scale first, mask, then max
-        const int kl = masked ? klim - j * 128 : 128;   // keys >= kl are invisible to this row
-#pragma unroll
-        for (int i = 0; i < 128; ++i) s[i] = (i < kl) ? s[i] * c2 : -INFINITY;
-        float mx[8];
-#pragma unroll
-        for (int k = 0; k < 8; ++k) mx[k] = s[k];
-#pragma unroll
-        for (int i = 8; i < 128; ++i) mx[i & 7] = fmaxf(mx[i & 7], s[i]);
-        m_tile = fmaxf(fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])),
-                       fmaxf(fmaxf(mx[4], mx[5]), fmaxf(mx[6], mx[7])));
-      }
-      // lazy rescale: move the reference max only when it grows by more than the threshold
-      const bool need = m_tile > m_ref + kRescaleThresh;
+        return fmaxf(max3f(mx[0], mx[1], mx[2]), max3f(max3f(mx[3], mx[4], mx[5]), mx[6], mx[7]));
+      };
+      bool need;
       float alpha = 1.f;
-      if (need) {
-        alpha = ex2(m_ref - m_tile);       // 0 when m_ref == -inf
-        l_sum *= alpha;
-        l_lse *= alpha;
-        m_ref = m_tile;
-      }
-      const float m_use = (m_ref == -INFINITY) ? 0.f : m_ref;
-      // p = 2^(c2 s - m) on pairs: one packed FMA per pair; both row sums packed
-      // (rse: fp32 weights for the LSE; rs: the 16-bit weights the MMA multiplies, so
-      // O / l is an exact weighted average of V)
-      const f32x2 scale2 = fast ? pack_f2(c2, c2) : pack_f2(1.f, 1.f);
-      const f32x2 negm2 = pack_f2(-m_use, -m_use);
-      f32x2 rs2[4] = {0ull, 0ull, 0ull, 0ull}, rse2[4] = {0ull, 0ull, 0ull, 0ull};
-#pragma unroll
-      for (int c = 0; c < 4; ++c) {
-        uint32_t pk[16];
-#pragma unroll
-        for (int i = 0; i < 16; ++i) {
-          float x0, x1;
-          unpack_f2(fma_f2(pack_f2(s[c * 32 + 2 * i], s[c * 32 + 2 * i + 1]), scale2, negm2), x0, x1);
-          const float a = ex2(x0), b2 = ex2(x1);
-          rse2[i & 3] = add_f2(rse2[i & 3], pack_f2(a, b2));
-          float lo, hi;
-          if (BF16) {
-            __nv_bfloat162 h2 = __floats2bfloat162_rn(a, b2);
-            pk[i] = *reinterpret_cast<uint32_t*>(&h2);
-            lo = __uint_as_float(pk[i] << 16);
-            hi = __uint_as_float(pk[i] & 0xffff0000u);
-          } else {
-            __half2 h2 = __floats2half2_rn(a, b2);
-            pk[i] = *reinterpret_cast<uint32_t*>(&h2);
-            const float2 f = __half22float2(h2);
-            lo = f.x;
-            hi = f.y;
+      if (plain && j > 0) {
+        // the reference is finite here (tile 0 of this Q tile was a full tile): exponentiate
+        // against it and find the tile max in the same pass; only if the max moved past the
+        // lazy threshold (rare) redo the tile against the new reference
+        exp_pass(m_ref, true);
+        const float m_tile = smax * c2;
+        need = m_tile > m_ref + kRescaleThresh;
+        if (__any_sync(0xffffffffu, need)) {
+          if (need) {
+            alpha = ex2(m_ref - m_tile);
+            l_sum *= alpha;
+            l_lse *= alpha;
+            m_ref = m_tile;
           }
-          rs2[i & 3] = add_f2(rs2[i & 3], pack_f2(lo, hi));
+          exp_pass(m_ref, false);
         }
-        tmem_st16(lane_addr + Cfg::P_COL(t) + c * 16, pk);
+      } else {
+        // first tile of a Q tile, masked tiles, negative scales: max first, then the pass
+        const float m_tile = plain ? row_max() * c2 : row_max();
+        need = m_tile > m_ref + kRescaleThresh;
+        if (need) {
+          alpha = ex2(m_ref - m_tile);       // 0 when m_ref == -inf
+          l_sum *= alpha;
+          l_lse *= alpha;
+          m_ref = m_tile;
+        }
+        exp_pass((m_ref == -INFINITY) ? 0.f : m_ref, false);
       }
-      {
-        float a0, a1, b0, b1;
-        unpack_f2(add_f2(add_f2(rs2[0], rs2[1]), add_f2(rs2[2], rs2[3])), a0, a1);
-        unpack_f2(add_f2(add_f2(rse2[0], rse2[1]), add_f2(rse2[2], rse2[3])), b0, b1);
-        l_sum += a0 + a1;
-        l_lse += b0 + b1;
-      }
+      l_sum += sum_r;
+      l_lse += sum_e;
       // O_t holds P V up to tile j-1, complete: S_t(j)'s commit covers every earlier MMA
       if (j > 0 && __any_sync(0xffffffffu, need)) {
 #pragma unroll 1
