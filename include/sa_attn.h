@@ -141,6 +141,13 @@ const char* sa_last_error(void);
  * wait expired since the last check, SA_ERR_CUDA on a CUDA error, else SA_OK. */
 int sa_check_status(sa_stream_t stream);
 
+/* Diagnostic: launches one kernel whose single bounded wait can never be satisfied, to
+ * exercise failure detection without a GPU fault: after about 2 s the wait gives up, the
+ * device status word records a timeout and the kernel returns.  The next
+ * sa_check_status(stream) then returns SA_ERR_TIMEOUT (and clears the word); the context
+ * stays usable.  Returns SA_OK once launched. */
+int sa_selftest_bounded_wait(sa_stream_t stream);
+
 /* Library version, "major.minor.patch". */
 const char* sa_version(void);
 

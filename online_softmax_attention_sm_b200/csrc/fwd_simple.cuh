@@ -67,4 +67,18 @@ __global__ void attn_fill_empty(uint16_t* o, size_t n_o, float* lse, size_t n_ls
     for (size_t i = blockIdx.x * (size_t)blockDim.x + threadIdx.x; i < n_lse; i += stride) lse[i] = -INFINITY;
 }
 
+// Self-test of the bounded-wait path: one thread waits on an mbarrier that nothing ever
+// completes.  The wait gives up after kWaitLimitNs, records a timeout in the status word
+// and the kernel returns normally -- no trap, no fault, the context stays usable.
+__global__ void selftest_bounded_wait() {
+  __shared__ uint64_t bar;
+  __shared__ int abort_flag;
+  if (threadIdx.x == 0) {
+    mbar_init(&bar, 1);          // expects one arrival that never comes
+    abort_flag = 0;
+    fence_barrier_init();
+    mbar_wait(&bar, 0, &abort_flag, 99);
+  }
+}
+
 }  // namespace sa

@@ -66,6 +66,7 @@ struct FwdParams {
   int B, Sq, Sk, Hq, Hkv, causal;
   int n_qblk;        // ceil(Sq / 256)
   int n_units;       // B * Hq * n_qblk
+  int kv_group;      // (batch, KV head) pairs per scheduling group (their K/V fit in L2)
   float c2;          // scale * log2(e)
 };
 
@@ -85,16 +86,25 @@ __device__ __forceinline__ int fwd_kv_tiles(const FwdParams& p, int r0) {
   return kend > 0 ? (kend + 127) / 128 : 0;
 }
 
-// Units are numbered longest-first: query block descending, then (b, h) with heads of
-// one KV head adjacent.
+// Units are numbered in groups of kv_group (batch, KV head) pairs, chosen on the host so
+// that a group's K and V fit in about half the L2 (the CTAs in flight then share their
+// K/V tiles through L2 instead of streaming them from HBM again); within a group,
+// longest first: query block descending, then the group's query heads.
 __device__ __forceinline__ UnitInfo fwd_unit(const FwdParams& p, int u) {
   UnitInfo x;
-  int bh = p.B * p.Hq;
-  int qb = p.n_qblk - 1 - u / bh;
-  int r = u % bh;
-  x.b = r / p.Hq;
-  x.h = r % p.Hq;
-  x.kvh = x.h / (p.Hq / p.Hkv);
+  const int G = p.Hq / p.Hkv;
+  const int n_bk = p.B * p.Hkv;
+  const int per_bk = G * p.n_qblk;                     // units of one (b, KV head)
+  const int full = p.kv_group * per_bk;                // units of a full group
+  const int grp = u / full;
+  const int gsize = min(p.kv_group, n_bk - grp * p.kv_group);
+  const int r = u - grp * full;
+  const int qb = p.n_qblk - 1 - r / (gsize * G);
+  const int rem = r % (gsize * G);
+  const int bk = grp * p.kv_group + rem / G;
+  x.b = bk / p.Hkv;
+  x.kvh = bk % p.Hkv;
+  x.h = x.kvh * G + rem % G;
   x.q0 = qb * 256;
   x.nkv[0] = fwd_kv_tiles(p, x.q0);
   x.nkv[1] = fwd_kv_tiles(p, x.q0 + 128);

@@ -131,6 +131,17 @@ int launch_fwd(const void* q, const void* k, const void* v, void* o, float* lse,
   if (units > 0x7fffffffLL) return fail(SA_ERR_UNSUPPORTED, "too many work units (%lld)", units);
   p.n_units = (int)units;
   p.c2 = scale * kLog2e;
+  {
+    // (batch, KV head) pairs per scheduling group: their K + V within about half the L2
+    int dev = 0, l2 = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || cudaDeviceGetAttribute(&l2, cudaDevAttrL2CacheSize, dev) != cudaSuccess)
+      l2 = 64 << 20;
+    const double kv_bytes = 2.0 * Sk * D * 2;          // K and V of one (b, KV head)
+    long long g = (long long)((l2 / 2) / kv_bytes);
+    if (g < 1) g = 1;
+    if (g > (long long)B * Hkv) g = (long long)B * Hkv;
+    p.kv_group = (int)g;
+  }
   auto kern = sa::attn_fwd_sm100<D, BF16>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::SMEM_TOTAL);
   if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(attn_fwd_sm100)");
@@ -364,6 +375,12 @@ int sa_check_status(sa_stream_t stream) {
   }
   g_err.clear();
   return SA_OK;
+}
+
+int sa_selftest_bounded_wait(sa_stream_t stream) {
+  sa::selftest_bounded_wait<<<1, 32, 0, reinterpret_cast<cudaStream_t>(stream)>>>();
+  cudaError_t e = cudaGetLastError();
+  return e == cudaSuccess ? SA_OK : cuda_fail(e, "selftest_bounded_wait launch");
 }
 
 const char* sa_version(void) { return "0.1.0"; }

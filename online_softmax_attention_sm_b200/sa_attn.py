@@ -31,6 +31,7 @@ SIGNATURES = {
     "sa_last_error": (ctypes.c_char_p, []),
     "sa_check_status": (_I, [_P]),
     "sa_version": (ctypes.c_char_p, []),
+    "sa_selftest_bounded_wait": (_I, [_P]),
 }
 
 _lib = None
