@@ -67,6 +67,7 @@ struct FwdParams {
   int n_qblk;        // ceil(Sq / 256)
   int n_units;       // B * Hq * n_qblk
   int kv_group;      // (batch, KV head) pairs per scheduling group (their K/V fit in L2)
+  int band;          // query blocks per band (a band of one group fills about one round)
   float c2;          // scale * log2(e)
 };
 
@@ -86,22 +87,27 @@ __device__ __forceinline__ int fwd_kv_tiles(const FwdParams& p, int r0) {
   return kend > 0 ? (kend + 127) / 128 : 0;
 }
 
-// Units are numbered in groups of kv_group (batch, KV head) pairs, chosen on the host so
-// that a group's K and V fit in about half the L2 (the CTAs in flight then share their
-// K/V tiles through L2 instead of streaming them from HBM again); within a group,
-// longest first: query block descending, then the group's query heads.
+// Unit order.  The query blocks are cut into bands of `band` blocks, longest first; within
+// a band, the (batch, KV head) pairs go in groups of kv_group, and within a group, query
+// block descending, then the group's query heads.  The host sizes a group so its K and V
+// fit in half the L2 and a (band, group) block fills about one round of the persistent
+// grid: the CTAs in flight then share K/V tiles through L2, and consecutive rounds hold
+// units of the same lengths (longest first overall, which the snake assignment needs).
 __device__ __forceinline__ UnitInfo fwd_unit(const FwdParams& p, int u) {
   UnitInfo x;
   const int G = p.Hq / p.Hkv;
   const int n_bk = p.B * p.Hkv;
-  const int per_bk = G * p.n_qblk;                     // units of one (b, KV head)
-  const int full = p.kv_group * per_bk;                // units of a full group
-  const int grp = u / full;
-  const int gsize = min(p.kv_group, n_bk - grp * p.kv_group);
-  const int r = u - grp * full;
-  const int qb = p.n_qblk - 1 - r / (gsize * G);
-  const int rem = r % (gsize * G);
-  const int bk = grp * p.kv_group + rem / G;
+  const int per_band = p.band * p.B * p.Hq;            // units of a full band
+  const int bi = u / per_band;
+  const int bs = min(p.band, p.n_qblk - bi * p.band);  // this band's query blocks
+  const int r = u - bi * per_band;
+  const int full_grp = p.kv_group * G * bs;            // units of a full group in this band
+  const int g = r / full_grp;
+  const int gsize = min(p.kv_group, n_bk - g * p.kv_group);
+  const int rr = r - g * full_grp;
+  const int qb = p.n_qblk - 1 - (bi * p.band + rr / (gsize * G));
+  const int rem = rr % (gsize * G);
+  const int bk = g * p.kv_group + rem / G;
   x.b = bk / p.Hkv;
   x.kvh = bk % p.Hkv;
   x.h = x.kvh * G + rem % G;

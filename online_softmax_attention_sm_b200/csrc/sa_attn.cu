@@ -132,15 +132,27 @@ int launch_fwd(const void* q, const void* k, const void* v, void* o, float* lse,
   p.n_units = (int)units;
   p.c2 = scale * kLog2e;
   {
-    // (batch, KV head) pairs per scheduling group: their K + V within about half the L2
+    // scheduling groups: (batch, KV head) pairs whose K + V fit in half the L2; among the
+    // admissible sizes take the one whose band (ceil(grid / (kv_group * G)) query blocks)
+    // fills whole rounds most exactly, then the smaller
     int dev = 0, l2 = 0;
     if (cudaGetDevice(&dev) != cudaSuccess || cudaDeviceGetAttribute(&l2, cudaDevAttrL2CacheSize, dev) != cudaSuccess)
       l2 = 64 << 20;
+    const int G = Hq / Hkv, n_bk = B * Hkv;
+    const int ncta = p.n_units < num_sms() ? p.n_units : num_sms();
     const double kv_bytes = 2.0 * Sk * D * 2;          // K and V of one (b, KV head)
-    long long g = (long long)((l2 / 2) / kv_bytes);
-    if (g < 1) g = 1;
-    if (g > (long long)B * Hkv) g = (long long)B * Hkv;
-    p.kv_group = (int)g;
+    long long gmax = (long long)((l2 / 2) / kv_bytes);
+    if (gmax < 1) gmax = 1;
+    if (gmax > n_bk) gmax = n_bk;
+    int best_g = 1, best_band = 1;
+    double best_waste = 1e30;
+    for (int g = 1; g <= gmax; ++g) {
+      const int band = (ncta + g * G - 1) / (g * G);
+      const double waste = (double)((long long)band * g * G % ncta) / ncta;   // partial round
+      if (waste < best_waste - 1e-9) { best_waste = waste; best_g = g; best_band = band; }
+    }
+    p.kv_group = best_g;
+    p.band = best_band < p.n_qblk ? best_band : p.n_qblk;
   }
   auto kern = sa::attn_fwd_sm100<D, BF16>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::SMEM_TOTAL);
