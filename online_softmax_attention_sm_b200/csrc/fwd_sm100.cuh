@@ -137,6 +137,7 @@ struct FwdSmem {
   uint64_t* p_full;    // [2]  P_t written and O_t rescaled (128 softmax threads)
   uint64_t* o_done;    // [2]  P_t V complete (tcgen05.commit)
   uint64_t* fin;       // [1]  every MMA of this CTA complete
+  uint64_t* p_part;    // [2]  first 96 keys of P_t written, O_t rescaled (128 threads)
   uint32_t* tmem_holder;
   volatile int* abort_flag;
   __device__ explicit FwdSmem(uint8_t* s) {
@@ -151,7 +152,8 @@ struct FwdSmem {
     p_full = q_full + 6;
     o_done = q_full + 8;
     fin = q_full + 10;
-    tmem_holder = (uint32_t*)(q_full + 12);
+    p_part = q_full + 11;
+    tmem_holder = (uint32_t*)(q_full + 13);
     abort_flag = (volatile int*)(tmem_holder + 1);
   }
 };
@@ -277,15 +279,23 @@ __device__ __forceinline__ void fwd_mma(const FwdParams& p, const FwdSmem<D>& sm
         bool k_ready = false;
         for (int t = 0; t < 2; ++t) {
           if (j >= x.nkv[t]) continue;
-          // ---- O_t += P_t V_j
+          // ---- O_t += P_t V_j: keys 0-95 as soon as their P is written, then 96-127
+          ok = mbar_wait(&sm.p_part[t], (t ? pv1 : pv0) & 1, sm.abort_flag, 17);
+          if (!ok) break;
+          tc_fence_after();
+#pragma unroll
+          for (int kk = 0; kk < 6; ++kk) {
+            mma_ts(tmem_base + Cfg::O_COL(t), tmem_base + Cfg::P_COL(t) + kk * 8,
+                   smem_desc_sw128(v_addr + kk * 2048, Cfg::CHUNK_BYTES, 1024), IDESC_PV,
+                   (j > 0 || kk > 0) ? 1u : 0u);
+          }
           ok = mbar_wait(&sm.p_full[t], (t ? pv1 : pv0) & 1, sm.abort_flag, 14);
           if (!ok) break;
           tc_fence_after();
 #pragma unroll
-          for (int kk = 0; kk < 128 / 16; ++kk) {
+          for (int kk = 6; kk < 8; ++kk) {
             mma_ts(tmem_base + Cfg::O_COL(t), tmem_base + Cfg::P_COL(t) + kk * 8,
-                   smem_desc_sw128(v_addr + kk * 2048, Cfg::CHUNK_BYTES, 1024), IDESC_PV,
-                   (j > 0 || kk > 0) ? 1u : 0u);
+                   smem_desc_sw128(v_addr + kk * 2048, Cfg::CHUNK_BYTES, 1024), IDESC_PV, 1u);
           }
           mma_commit(&sm.o_done[t]);
           if (t) ++pv1; else ++pv0;
@@ -372,27 +382,53 @@ __device__ __forceinline__ void fwd_softmax(const FwdParams& p, const FwdSmem<D>
 #pragma unroll
         for (int i = 0; i < 128; ++i) s[i] = (i < kl) ? s[i] * c2 : -INFINITY;
       }
-      const f32x2 scale2 = plain ? pack_f2(c2, c2) : pack_f2(1.f, 1.f);
-      // One pass over the tile: p = 2^(scale2 * s - m_use) on pairs (one packed FMA per
-      // pair), P stored to tensor memory as 16-bit, both row sums (rse: fp32 weights for
-      // the LSE; rs: the 16-bit weights the MMA multiplies, so O / l is an exact weighted
-      // average of V), and optionally the row max of s as 8 chains of 3-input max.
-      float sum_r, sum_e, smax = -INFINITY;
-      auto exp_pass = [&](float m_use, bool track_max) {
+      // the row max, the reference (moved only past the lazy threshold), alpha
+      float mx[8];
+#pragma unroll
+      for (int k = 0; k < 8; ++k) mx[k] = fmaxf(s[k], s[k + 8]);
+#pragma unroll
+      for (int i = 16; i < 128; i += 16)
+#pragma unroll
+        for (int k = 0; k < 8; ++k) mx[k] = max3f(mx[k], s[i + k], s[i + 8 + k]);
+      float m_tile = fmaxf(max3f(mx[0], mx[1], mx[2]), max3f(max3f(mx[3], mx[4], mx[5]), mx[6], mx[7]));
+      if (plain) m_tile *= c2;
+      const bool need = m_tile > m_ref + kRescaleThresh;
+      float alpha = 1.f;
+      if (need) {
+        alpha = ex2(m_ref - m_tile);       // 0 when m_ref == -inf
+        l_sum *= alpha;
+        l_lse *= alpha;
+        m_ref = m_tile;
+      }
+      // O_t holds P V up to tile j-1, complete: S_t(j)'s commit covers every earlier MMA.
+      // Rescale it before any of this tile's P is handed to the MMA warp.
+      if (j > 0 && __any_sync(0xffffffffu, need)) {
+#pragma unroll 1
+        for (int c = 0; c < D / 32; ++c) {
+          uint32_t r[32];
+          tmem_ld32(lane_addr + Cfg::O_COL(t) + c * 32, r);
+          tmem_wait_ld();
+#pragma unroll
+          for (int i = 0; i < 32; ++i) r[i] = __float_as_uint(__uint_as_float(r[i]) * alpha);
+          tmem_st32(lane_addr + Cfg::O_COL(t) + c * 32, r);
+        }
+      }
+      // p = 2^(scale2 * s - m_use) on pairs (one packed FMA per pair), P stored to tensor
+      // memory as 16-bit, both row sums (rse: fp32 weights for the LSE; rs: the 16-bit
+      // weights the MMA multiplies, so O / l is an exact weighted average of V).  After the
+      // first 96 keys the MMA warp may start on them.
+      {
+        const float m_use = (m_ref == -INFINITY) ? 0.f : m_ref;
+        const f32x2 scale2 = plain ? pack_f2(c2, c2) : pack_f2(1.f, 1.f);
         const f32x2 negm2 = pack_f2(-m_use, -m_use);
         f32x2 rs2[4] = {0ull, 0ull, 0ull, 0ull}, rse2[4] = {0ull, 0ull, 0ull, 0ull};
-        float mx[8];
-#pragma unroll
-        for (int k = 0; k < 8; ++k) mx[k] = -INFINITY;
 #pragma unroll
         for (int c = 0; c < 4; ++c) {
           uint32_t pk[16];
 #pragma unroll
           for (int i = 0; i < 16; ++i) {
-            const float s0 = s[c * 32 + 2 * i], s1 = s[c * 32 + 2 * i + 1];
-            if (track_max) mx[i & 7] = max3f(mx[i & 7], s0, s1);
             float x0, x1;
-            unpack_f2(fma_f2(pack_f2(s0, s1), scale2, negm2), x0, x1);
+            unpack_f2(fma_f2(pack_f2(s[c * 32 + 2 * i], s[c * 32 + 2 * i + 1]), scale2, negm2), x0, x1);
             const float a = ex2(x0), b2 = ex2(x1);
             rse2[i & 3] = add_f2(rse2[i & 3], pack_f2(a, b2));
             float lo, hi;
@@ -411,68 +447,17 @@ __device__ __forceinline__ void fwd_softmax(const FwdParams& p, const FwdSmem<D>
             rs2[i & 3] = add_f2(rs2[i & 3], pack_f2(lo, hi));
           }
           tmem_st16(lane_addr + Cfg::P_COL(t) + c * 16, pk);
+          if (c == 2) {
+            tmem_wait_st();
+            tc_fence_before();
+            mbar_arrive(&sm.p_part[t]);
+          }
         }
         float a0, a1, b0, b1;
         unpack_f2(add_f2(add_f2(rs2[0], rs2[1]), add_f2(rs2[2], rs2[3])), a0, a1);
         unpack_f2(add_f2(add_f2(rse2[0], rse2[1]), add_f2(rse2[2], rse2[3])), b0, b1);
-        sum_r = a0 + a1;
-        sum_e = b0 + b1;
-        if (track_max)
-          smax = fmaxf(max3f(mx[0], mx[1], mx[2]), max3f(max3f(mx[3], mx[4], mx[5]), mx[6], mx[7]));
-      };
-      auto row_max = [&]() {
-        float mx[8];
-#pragma unroll
-        for (int k = 0; k < 8; ++k) mx[k] = fmaxf(s[k], s[k + 8]);
-#pragma unroll
-        for (int i = 16; i < 128; i += 16)
-#pragma unroll
-          for (int k = 0; k < 8; ++k) mx[k] = max3f(mx[k], s[i + k], s[i + 8 + k]);
-        return fmaxf(max3f(mx[0], mx[1], mx[2]), max3f(max3f(mx[3], mx[4], mx[5]), mx[6], mx[7]));
-      };
-      bool need;
-      float alpha = 1.f;
-      if (plain && j > 0) {
-        // the reference is finite here (tile 0 of this Q tile was a full tile): exponentiate
-        // against it and find the tile max in the same pass; only if the max moved past the
-        // lazy threshold (rare) redo the tile against the new reference
-        exp_pass(m_ref, true);
-        const float m_tile = smax * c2;
-        need = m_tile > m_ref + kRescaleThresh;
-        if (__any_sync(0xffffffffu, need)) {
-          if (need) {
-            alpha = ex2(m_ref - m_tile);
-            l_sum *= alpha;
-            l_lse *= alpha;
-            m_ref = m_tile;
-          }
-          exp_pass(m_ref, false);
-        }
-      } else {
-        // first tile of a Q tile, masked tiles, negative scales: max first, then the pass
-        const float m_tile = plain ? row_max() * c2 : row_max();
-        need = m_tile > m_ref + kRescaleThresh;
-        if (need) {
-          alpha = ex2(m_ref - m_tile);       // 0 when m_ref == -inf
-          l_sum *= alpha;
-          l_lse *= alpha;
-          m_ref = m_tile;
-        }
-        exp_pass((m_ref == -INFINITY) ? 0.f : m_ref, false);
-      }
-      l_sum += sum_r;
-      l_lse += sum_e;
-      // O_t holds P V up to tile j-1, complete: S_t(j)'s commit covers every earlier MMA
-      if (j > 0 && __any_sync(0xffffffffu, need)) {
-#pragma unroll 1
-        for (int c = 0; c < D / 32; ++c) {
-          uint32_t r[32];
-          tmem_ld32(lane_addr + Cfg::O_COL(t) + c * 32, r);
-          tmem_wait_ld();
-#pragma unroll
-          for (int i = 0; i < 32; ++i) r[i] = __float_as_uint(__uint_as_float(r[i]) * alpha);
-          tmem_st32(lane_addr + Cfg::O_COL(t) + c * 32, r);
-        }
+        l_sum += a0 + a1;
+        l_lse += b0 + b1;
       }
       tmem_wait_st();
       tc_fence_before();
@@ -555,6 +540,7 @@ attn_fwd_sm100(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
     for (int t = 0; t < 2; ++t) {
       mbar_init(&sm.q_full[t], 1); mbar_init(&sm.q_empty[t], 1);
       mbar_init(&sm.s_full[t], 1); mbar_init(&sm.p_full[t], 128); mbar_init(&sm.o_done[t], 1);
+      mbar_init(&sm.p_part[t], 128);
     }
     mbar_init(sm.fin, 1);
     *sm.abort_flag = 0;
