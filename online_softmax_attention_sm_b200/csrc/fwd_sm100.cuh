@@ -10,13 +10,14 @@
 //   * unit of work = (batch, query head, 256 query rows) = two 128-row Q tiles that
 //     share every K/V tile; a persistent grid of one CTA per SM walks the units in
 //     longest-first order (causal units with more K/V tiles first);
-//   * warp 8 (one lane) issues TMA tensor loads: the two Q tiles once per unit, then
+//   * warp 1 (one lane) issues TMA tensor loads: the two Q tiles once per unit, then
 //     K and V tiles into a ring of shared-memory slots (full/empty mbarriers);
-//   * warp 9 (one lane) issues tcgen05.mma: S_t = Q_t K^T (128x128, fp32 in tensor
+//   * warp 0 issues tcgen05.mma (warp-uniform code, one elected lane per instruction):
+//     S_t = Q_t K^T (128x128, fp32 in tensor
 //     memory) and O_t += P_t V (P_t read from tensor memory, O_t fp32 in tensor memory),
 //     in the order PV_0(j), QK_0(j+1), PV_1(j), QK_1(j+1) so that each softmax
 //     warpgroup works while the tensor core serves the other Q tile;
-//   * warpgroups 0 and 1 run the softmax of Q tile 0 and 1: each thread owns one row of
+//   * warpgroups 1 and 2 run the softmax of Q tile 0 and 1: each thread owns one row of
 //     S (tcgen05.ld 32x32b), computes the row max, p = 2^(c*s - m) with c = scale*log2(e),
 //     the row sums, writes P as 16-bit into tensor memory over S, and rescales its O row
 //     only when the reference max moves by more than kRescaleThresh (exact after the
@@ -58,7 +59,15 @@ struct FwdCfg {
   __host__ __device__ static constexpr uint32_t P_COL(int t) { return 128u * t; }
 };
 
-constexpr float kRescaleThresh = 8.0f;   // log2 units
+// Warp roles.  The MMA issuer is warp 0: it shares a scheduler with two softmax warps
+// that issue nearly every cycle, and the lowest warp index keeps its few instructions
+// from waiting behind theirs.  Warps 4-11 are the two softmax warpgroups.
+constexpr int kWarpMma = 0;
+constexpr int kWarpLoad = 1;
+
+constexpr float kRescaleThresh = 8.0f;   // log2 units: the reference moves past this
+constexpr float kHardThresh = 15.0f;     // log2 units: p < 2^15 fits fp16 and bf16
+constexpr int kPolyEvery = 0;            // full tiles: one exponential pair in kPolyEvery on the FMA pipe (0: none)
 
 struct FwdParams {
   void* o;
@@ -224,7 +233,8 @@ template <int D, bool BF16>
 __device__ __forceinline__ void fwd_mma(const FwdParams& p, const FwdSmem<D>& sm, uint32_t tmem_base,
                                         int lane, int cta, int ncta) {
   using Cfg = FwdCfg<D>;
-  if (lane == 0) {
+  (void)lane;
+  {
     constexpr uint32_t IDESC_QK = idesc_f16(BF16 ? 1 : 0, 128, 128, 0, 0);
     constexpr uint32_t IDESC_PV = idesc_f16(BF16 ? 1 : 0, 128, D, 0, 1);
     const uint32_t sQ_addr = smem_u32(sm.q);
@@ -238,10 +248,10 @@ __device__ __forceinline__ void fwd_mma(const FwdParams& p, const FwdSmem<D>& sm
 #pragma unroll
       for (int kk = 0; kk < D / 16; ++kk) {
         const uint32_t off = (kk >> 2) * Cfg::CHUNK_BYTES + (kk & 3) * 32;
-        mma_ss(tmem_base + Cfg::S_COL(t), smem_desc_sw128(q_addr + off, 16, 1024),
+        mma_ss_warp(tmem_base + Cfg::S_COL(t), smem_desc_sw128(q_addr + off, 16, 1024),
                smem_desc_sw128(k_addr + off, 16, 1024), IDESC_QK, kk > 0);
       }
-      mma_commit(&sm.s_full[t]);
+      mma_commit_warp(&sm.s_full[t]);
     };
     // Issue order per K/V step j:  PV_0(j), QK_0(j+1), PV_1(j), QK_1(j+1).
     // P_t lives in S_t's tensor-memory columns; QK_t(j+1) overwrites them right after
@@ -257,22 +267,22 @@ __device__ __forceinline__ void fwd_mma(const FwdParams& p, const FwdSmem<D>& sm
       // ---- prologue: S_t = Q_t K_0^T
       {
         const int pos = base;
-        ok = mbar_wait(&sm.kv_full[pos % Cfg::STAGES], (pos / Cfg::STAGES) & 1, sm.abort_flag, 10);
+        ok = mbar_wait_warp(&sm.kv_full[pos % Cfg::STAGES], (pos / Cfg::STAGES) & 1, sm.abort_flag, 10);
         if (!ok) break;
         const uint32_t k_addr = sRing_addr + (pos % Cfg::STAGES) * Cfg::TILE_BYTES;
         for (int t = 0; t < 2 && ok; ++t) {
           if (x.nkv[t] == 0) continue;
-          ok = mbar_wait(&sm.q_full[t], (t ? q_use1 : q_use0) & 1, sm.abort_flag, 11);
+          ok = mbar_wait_warp(&sm.q_full[t], (t ? q_use1 : q_use0) & 1, sm.abort_flag, 11);
           if (!ok) break;
           tc_fence_after();
           issue_qk(t, k_addr);
         }
         if (!ok) break;
-        mma_commit(&sm.kv_empty[pos % Cfg::STAGES]);
+        mma_commit_warp(&sm.kv_empty[pos % Cfg::STAGES]);
       }
       for (int j = 0; j < x.nkv_max && ok; ++j) {
         const int vpos = base + 2 * j + 1, kpos = base + 2 * j + 2;
-        ok = mbar_wait(&sm.kv_full[vpos % Cfg::STAGES], (vpos / Cfg::STAGES) & 1, sm.abort_flag, 13);
+        ok = mbar_wait_warp(&sm.kv_full[vpos % Cfg::STAGES], (vpos / Cfg::STAGES) & 1, sm.abort_flag, 13);
         if (!ok) break;
         const uint32_t v_addr = sRing_addr + (vpos % Cfg::STAGES) * Cfg::TILE_BYTES;
         const uint32_t k_addr = sRing_addr + (kpos % Cfg::STAGES) * Cfg::TILE_BYTES;
@@ -280,29 +290,29 @@ __device__ __forceinline__ void fwd_mma(const FwdParams& p, const FwdSmem<D>& sm
         for (int t = 0; t < 2; ++t) {
           if (j >= x.nkv[t]) continue;
           // ---- O_t += P_t V_j: keys 0-95 as soon as their P is written, then 96-127
-          ok = mbar_wait(&sm.p_part[t], (t ? pv1 : pv0) & 1, sm.abort_flag, 17);
+          ok = mbar_wait_warp(&sm.p_part[t], (t ? pv1 : pv0) & 1, sm.abort_flag, 17);
           if (!ok) break;
           tc_fence_after();
 #pragma unroll
           for (int kk = 0; kk < 6; ++kk) {
-            mma_ts(tmem_base + Cfg::O_COL(t), tmem_base + Cfg::P_COL(t) + kk * 8,
+            mma_ts_warp(tmem_base + Cfg::O_COL(t), tmem_base + Cfg::P_COL(t) + kk * 8,
                    smem_desc_sw128(v_addr + kk * 2048, Cfg::CHUNK_BYTES, 1024), IDESC_PV,
                    (j > 0 || kk > 0) ? 1u : 0u);
           }
-          ok = mbar_wait(&sm.p_full[t], (t ? pv1 : pv0) & 1, sm.abort_flag, 14);
+          ok = mbar_wait_warp(&sm.p_full[t], (t ? pv1 : pv0) & 1, sm.abort_flag, 14);
           if (!ok) break;
           tc_fence_after();
 #pragma unroll
           for (int kk = 6; kk < 8; ++kk) {
-            mma_ts(tmem_base + Cfg::O_COL(t), tmem_base + Cfg::P_COL(t) + kk * 8,
+            mma_ts_warp(tmem_base + Cfg::O_COL(t), tmem_base + Cfg::P_COL(t) + kk * 8,
                    smem_desc_sw128(v_addr + kk * 2048, Cfg::CHUNK_BYTES, 1024), IDESC_PV, 1u);
           }
-          mma_commit(&sm.o_done[t]);
+          mma_commit_warp(&sm.o_done[t]);
           if (t) ++pv1; else ++pv0;
           // ---- S_t = Q_t K_{j+1}^T
           if (j + 1 < x.nkv[t]) {
             if (!k_ready) {
-              ok = mbar_wait(&sm.kv_full[kpos % Cfg::STAGES], (kpos / Cfg::STAGES) & 1, sm.abort_flag, 10);
+              ok = mbar_wait_warp(&sm.kv_full[kpos % Cfg::STAGES], (kpos / Cfg::STAGES) & 1, sm.abort_flag, 10);
               if (!ok) break;
               k_ready = true;
             }
@@ -310,35 +320,118 @@ __device__ __forceinline__ void fwd_mma(const FwdParams& p, const FwdSmem<D>& sm
           }
         }
         if (!ok) break;
-        mma_commit(&sm.kv_empty[vpos % Cfg::STAGES]);
+        mma_commit_warp(&sm.kv_empty[vpos % Cfg::STAGES]);
         if (j + 1 < x.nkv_max) {
           if (!k_ready) {
             // (cannot happen: the Q tile with the most K/V tiles needs K(j+1))
-            ok = mbar_wait(&sm.kv_full[kpos % Cfg::STAGES], (kpos / Cfg::STAGES) & 1, sm.abort_flag, 16);
+            ok = mbar_wait_warp(&sm.kv_full[kpos % Cfg::STAGES], (kpos / Cfg::STAGES) & 1, sm.abort_flag, 16);
             if (!ok) break;
           }
-          mma_commit(&sm.kv_empty[kpos % Cfg::STAGES]);
+          mma_commit_warp(&sm.kv_empty[kpos % Cfg::STAGES]);
         }
       }
       if (!ok) break;
       ring_n = base + 2 * x.nkv_max;
-      if (x.nkv[0] > 0) { mma_commit(&sm.q_empty[0]); ++q_use0; }
-      if (x.nkv[1] > 0) { mma_commit(&sm.q_empty[1]); ++q_use1; }
+      if (x.nkv[0] > 0) { mma_commit_warp(&sm.q_empty[0]); ++q_use0; }
+      if (x.nkv[1] > 0) { mma_commit_warp(&sm.q_empty[1]); ++q_use1; }
     }
     // every MMA issued above completes before tensor memory is released
-    mma_commit(sm.fin);
-    mbar_wait(sm.fin, 0, nullptr, 15);
+    mma_commit_warp(sm.fin);
+    mbar_wait_warp(sm.fin, 0, nullptr, 15);
   }
   __syncwarp();
 }
 
 // ------------------------------------------------------------------ softmax + epilogue
+// 2^x for a pair of finite x on the FMA pipe (the MUFU ex2 unit is the softmax's
+// bottleneck: 16 results per clock per SM).  x = n + f with n = round(x) taken from the
+// low mantissa bits of x + 1.5 * 2^23 and f in [-1/2, 1/2]; 2^f by a cubic fitted for
+// minimum relative error on that interval (max 7.6e-5, below the 16-bit rounding of P);
+// 2^n enters through the exponent field.  x is clamped at -126 so 2^n stays normal
+// (the result is then within 2^-126 of the true, smaller value).
+__device__ __forceinline__ void exp2_poly_pair(float x0, float x1, float& a, float& b) {
+  const f32x2 x = pack_f2(fmaxf(x0, -126.f), fmaxf(x1, -126.f));
+  const f32x2 t = add_f2(x, pack_f2(12582912.f, 12582912.f));       // 1.5 * 2^23 + n
+  const f32x2 f = fma_f2(add_f2(t, pack_f2(-12582912.f, -12582912.f)), pack_f2(-1.f, -1.f), x);
+  f32x2 q = fma_f2(pack_f2(0.055174146f, 0.055174146f), f, pack_f2(0.24261758f, 0.24261758f));
+  q = fma_f2(q, f, pack_f2(0.69326109f, 0.69326109f));
+  q = fma_f2(q, f, pack_f2(0.99992758f, 0.99992758f));
+  float q0, q1, t0, t1;
+  unpack_f2(q, q0, q1);
+  unpack_f2(t, t0, t1);
+  // n sits in the low bits of t; n << 23 added to the bits of 2^f scales it by 2^n
+  a = __uint_as_float(__float_as_uint(q0) + (__float_as_uint(t0) << 23));
+  b = __uint_as_float(__float_as_uint(q1) + (__float_as_uint(t1) << 23));
+}
+
+// One 32-key chunk of a row: p = 2^(scale2 * s - m) on pairs (one packed FMA per pair),
+// P stored to tensor memory as 16-bit at taddr, both row sums (rse2: the fp32 weights,
+// for the LSE; rs2: the 16-bit weights the MMA multiplies, so O / l is an exact weighted
+// average of V).  With TRACK the chunk's scores also enter the running max mx.  With
+// POLY > 0, one pair in POLY is exponentiated by exp2_poly_pair (finite x only).
+template <bool BF16, bool TRACK, int POLY>
+__device__ __forceinline__ void softmax_chunk(const float (&s)[128], const int c, const f32x2 scale2,
+                                              const f32x2 negm2, f32x2 (&rs2)[2], f32x2 (&rse2)[2],
+                                              float (&mx)[8], const uint32_t taddr) {
+  uint32_t pk[16];
+#pragma unroll
+  for (int i = 0; i < 16; ++i) {
+    const float s0 = s[c * 32 + 2 * i], s1 = s[c * 32 + 2 * i + 1];
+    if (TRACK) mx[i & 7] = max3f(mx[i & 7], s0, s1);
+    float x0, x1;
+    unpack_f2(fma_f2(pack_f2(s0, s1), scale2, negm2), x0, x1);
+    float a, b2;
+    if (POLY > 0 && (i % (POLY > 0 ? POLY : 1)) == POLY - 1) {
+      exp2_poly_pair(x0, x1, a, b2);          // on the FMA pipe, sparing the MUFU
+    } else {
+      a = ex2(x0);
+      b2 = ex2(x1);
+    }
+    rse2[i & 1] = add_f2(rse2[i & 1], pack_f2(a, b2));
+    float lo, hi;
+    if (BF16) {
+      __nv_bfloat162 h2 = __floats2bfloat162_rn(a, b2);
+      pk[i] = *reinterpret_cast<uint32_t*>(&h2);
+      lo = __uint_as_float(pk[i] << 16);
+      hi = __uint_as_float(pk[i] & 0xffff0000u);
+    } else {
+      __half2 h2 = __floats2half2_rn(a, b2);
+      pk[i] = *reinterpret_cast<uint32_t*>(&h2);
+      const float2 f = __half22float2(h2);
+      lo = f.x;
+      hi = f.y;
+    }
+    rs2[i & 1] = add_f2(rs2[i & 1], pack_f2(lo, hi));
+  }
+  tmem_st16(taddr, pk);
+}
+
+// O_t row *= alpha, in place in tensor memory (32 columns at a time).
+template <int D>
+__device__ __forceinline__ void rescale_o_row(const uint32_t taddr, const float alpha) {
+#pragma unroll 1
+  for (int c = 0; c < D / 32; ++c) {
+    uint32_t r[32];
+    tmem_ld32(taddr + c * 32, r);
+    tmem_wait_ld();
+#pragma unroll
+    for (int i = 0; i < 32; ++i) r[i] = __float_as_uint(__uint_as_float(r[i]) * alpha);
+    tmem_st32(taddr + c * 32, r);
+  }
+}
+
+__device__ __forceinline__ void sum_f2x2(const f32x2 (&v)[2], float& acc) {
+  float a0, a1;
+  unpack_f2(add_f2(v[0], v[1]), a0, a1);
+  acc += a0 + a1;
+}
+
 template <int D, bool BF16>
 __device__ __forceinline__ void fwd_softmax(const FwdParams& p, const FwdSmem<D>& sm, uint32_t tmem_base,
                                             int warp, int lane, int cta, int ncta) {
   using Cfg = FwdCfg<D>;
-  const int t = warp >> 2;                  // Q tile of this warpgroup
-  const int wl = warp & 3;                  // TMEM lane quarter
+  const int t = warp >> 2;                  // Q tile of this warpgroup (warp: 0-7 here)
+  const int wl = warp & 3;                  // TMEM lane quarter (physical warp index % 4)
   const int row_in_tile = wl * 32 + lane;
   const uint32_t lane_addr = tmem_base + ((uint32_t)(wl * 32) << 16);
   const float c2 = p.c2;
@@ -360,6 +453,8 @@ __device__ __forceinline__ void fwd_softmax(const FwdParams& p, const FwdSmem<D>
     // l_sum: sum of the 16-bit weights (normalises O, matching what the MMA multiplied);
     // l_lse: sum of the fp32 weights (gives the LSE without the 16-bit rounding bias)
     float m_ref = -INFINITY, l_sum = 0.f, l_lse = 0.f;
+    float m_next = -INFINITY;               // a reference chosen on one tile, applied on the next
+    const uint32_t p_addr = lane_addr + Cfg::P_COL(t);
     for (int j = 0; j < nkv; ++j) {
       ok = __all_sync(0xffffffffu, mbar_wait(&sm.s_full[t], s_n & 1, sm.abort_flag, 20 + t));
       if (!ok) break;
@@ -376,88 +471,91 @@ __device__ __forceinline__ void fwd_softmax(const FwdParams& p, const FwdSmem<D>
       tmem_wait_ld();
       const bool masked = (j >= mask_from);
       const bool plain = !masked && c2 >= 0.f;     // full tile, scale >= 0: s scaled in the FMA
-      if (!plain) {
-        // diagonal / ragged tiles (and negative scales): scale first, mask
-        const int kl = masked ? klim - j * 128 : 128;   // keys >= kl are invisible to this row
-#pragma unroll
-        for (int i = 0; i < 128; ++i) s[i] = (i < kl) ? s[i] * c2 : -INFINITY;
-      }
-      // the row max, the reference (moved only past the lazy threshold), alpha
-      float mx[8];
-#pragma unroll
-      for (int k = 0; k < 8; ++k) mx[k] = fmaxf(s[k], s[k + 8]);
-#pragma unroll
-      for (int i = 16; i < 128; i += 16)
-#pragma unroll
-        for (int k = 0; k < 8; ++k) mx[k] = max3f(mx[k], s[i + k], s[i + 8 + k]);
-      float m_tile = fmaxf(max3f(mx[0], mx[1], mx[2]), max3f(max3f(mx[3], mx[4], mx[5]), mx[6], mx[7]));
-      if (plain) m_tile *= c2;
-      const bool need = m_tile > m_ref + kRescaleThresh;
-      float alpha = 1.f;
-      if (need) {
-        alpha = ex2(m_ref - m_tile);       // 0 when m_ref == -inf
-        l_sum *= alpha;
-        l_lse *= alpha;
-        m_ref = m_tile;
-      }
       // O_t holds P V up to tile j-1, complete: S_t(j)'s commit covers every earlier MMA.
-      // Rescale it before any of this tile's P is handed to the MMA warp.
-      if (j > 0 && __any_sync(0xffffffffu, need)) {
-#pragma unroll 1
-        for (int c = 0; c < D / 32; ++c) {
-          uint32_t r[32];
-          tmem_ld32(lane_addr + Cfg::O_COL(t) + c * 32, r);
-          tmem_wait_ld();
+      // A move of the reference chosen on tile j-1 is applied to it now, before any of
+      // this tile's P is handed to the MMA warp.
+      {
+        const bool moved = m_next > m_ref;
+        float alpha = 1.f;
+        if (moved) {
+          alpha = ex2(m_ref - m_next);
+          l_sum *= alpha;
+          l_lse *= alpha;
+          m_ref = m_next;
+        }
+        if (__any_sync(0xffffffffu, moved)) rescale_o_row<D>(lane_addr + Cfg::O_COL(t), alpha);
+      }
+      bool done = false;
+      if (__all_sync(0xffffffffu, plain && m_ref > -INFINITY)) {
+        // Full tile after the first: exponentiate against the current reference while
+        // taking the tile max in the same pass (the last chunk's max first, so that the
+        // whole max is known before the first 96 keys are handed over).  A tile max up
+        // to kHardThresh above the reference is accepted (p < 2^kHardThresh stays finite
+        // and exact to the 16-bit rounding) and moves the reference for the next tile;
+        // a larger one redoes the tile below with the moved reference.
+        float mx[8];
 #pragma unroll
-          for (int i = 0; i < 32; ++i) r[i] = __float_as_uint(__uint_as_float(r[i]) * alpha);
-          tmem_st32(lane_addr + Cfg::O_COL(t) + c * 32, r);
+        for (int k = 0; k < 8; ++k) mx[k] = max3f(s[96 + k], s[104 + k], fmaxf(s[112 + k], s[120 + k]));
+        const f32x2 scale2 = pack_f2(c2, c2), negm2 = pack_f2(-m_ref, -m_ref);
+        f32x2 rs2[2] = {0ull, 0ull}, rse2[2] = {0ull, 0ull};
+#pragma unroll
+        for (int c = 0; c < 3; ++c) softmax_chunk<BF16, true, kPolyEvery>(s, c, scale2, negm2, rs2, rse2, mx, p_addr + c * 16);
+        const float m_tile =
+            fmaxf(max3f(mx[0], mx[1], mx[2]), max3f(max3f(mx[3], mx[4], mx[5]), mx[6], mx[7])) * c2;
+        if (!__any_sync(0xffffffffu, m_tile > m_ref + kHardThresh)) {
+          tmem_wait_st();
+          tc_fence_before();
+          mbar_arrive(&sm.p_part[t]);
+          softmax_chunk<BF16, false, kPolyEvery>(s, 3, scale2, negm2, rs2, rse2, mx, p_addr + 48);
+          sum_f2x2(rs2, l_sum);
+          sum_f2x2(rse2, l_lse);
+          if (m_tile > m_ref + kRescaleThresh) m_next = m_tile;
+          done = true;
+        } else {
+          tmem_wait_st();                          // the redo below rewrites these columns
         }
       }
-      // p = 2^(scale2 * s - m_use) on pairs (one packed FMA per pair), P stored to tensor
-      // memory as 16-bit, both row sums (rse: fp32 weights for the LSE; rs: the 16-bit
-      // weights the MMA multiplies, so O / l is an exact weighted average of V).  After the
-      // first 96 keys the MMA warp may start on them.
-      {
+      if (!done) {
+        if (!plain) {
+          // diagonal / ragged tiles (and negative scales): scale first, mask
+          const int kl = masked ? klim - j * 128 : 128;   // keys >= kl are invisible to this row
+#pragma unroll
+          for (int i = 0; i < 128; ++i) s[i] = (i < kl) ? s[i] * c2 : -INFINITY;
+        }
+        // the row max, the reference (moved only past the lazy threshold), alpha
+        float mx[8];
+#pragma unroll
+        for (int k = 0; k < 8; ++k) mx[k] = fmaxf(s[k], s[k + 8]);
+#pragma unroll
+        for (int i = 16; i < 128; i += 16)
+#pragma unroll
+          for (int k = 0; k < 8; ++k) mx[k] = max3f(mx[k], s[i + k], s[i + 8 + k]);
+        float m_tile = fmaxf(max3f(mx[0], mx[1], mx[2]), max3f(max3f(mx[3], mx[4], mx[5]), mx[6], mx[7]));
+        if (plain) m_tile *= c2;
+        const bool need = m_tile > m_ref + kRescaleThresh;
+        float alpha = 1.f;
+        if (need) {
+          alpha = ex2(m_ref - m_tile);       // 0 when m_ref == -inf
+          l_sum *= alpha;
+          l_lse *= alpha;
+          m_ref = m_tile;
+        }
+        if (j > 0 && __any_sync(0xffffffffu, need)) rescale_o_row<D>(lane_addr + Cfg::O_COL(t), alpha);
         const float m_use = (m_ref == -INFINITY) ? 0.f : m_ref;
         const f32x2 scale2 = plain ? pack_f2(c2, c2) : pack_f2(1.f, 1.f);
         const f32x2 negm2 = pack_f2(-m_use, -m_use);
-        f32x2 rs2[4] = {0ull, 0ull, 0ull, 0ull}, rse2[4] = {0ull, 0ull, 0ull, 0ull};
+        f32x2 rs2[2] = {0ull, 0ull}, rse2[2] = {0ull, 0ull};
 #pragma unroll
         for (int c = 0; c < 4; ++c) {
-          uint32_t pk[16];
-#pragma unroll
-          for (int i = 0; i < 16; ++i) {
-            float x0, x1;
-            unpack_f2(fma_f2(pack_f2(s[c * 32 + 2 * i], s[c * 32 + 2 * i + 1]), scale2, negm2), x0, x1);
-            const float a = ex2(x0), b2 = ex2(x1);
-            rse2[i & 3] = add_f2(rse2[i & 3], pack_f2(a, b2));
-            float lo, hi;
-            if (BF16) {
-              __nv_bfloat162 h2 = __floats2bfloat162_rn(a, b2);
-              pk[i] = *reinterpret_cast<uint32_t*>(&h2);
-              lo = __uint_as_float(pk[i] << 16);
-              hi = __uint_as_float(pk[i] & 0xffff0000u);
-            } else {
-              __half2 h2 = __floats2half2_rn(a, b2);
-              pk[i] = *reinterpret_cast<uint32_t*>(&h2);
-              const float2 f = __half22float2(h2);
-              lo = f.x;
-              hi = f.y;
-            }
-            rs2[i & 3] = add_f2(rs2[i & 3], pack_f2(lo, hi));
-          }
-          tmem_st16(lane_addr + Cfg::P_COL(t) + c * 16, pk);
-          if (c == 2) {
+          softmax_chunk<BF16, false, 0>(s, c, scale2, negm2, rs2, rse2, mx, p_addr + c * 16);
+          if (c == 2) {                       // the MMA warp may start on the first 96 keys
             tmem_wait_st();
             tc_fence_before();
             mbar_arrive(&sm.p_part[t]);
           }
         }
-        float a0, a1, b0, b1;
-        unpack_f2(add_f2(add_f2(rs2[0], rs2[1]), add_f2(rs2[2], rs2[3])), a0, a1);
-        unpack_f2(add_f2(add_f2(rse2[0], rse2[1]), add_f2(rse2[2], rse2[3])), b0, b1);
-        l_sum += a0 + a1;
-        l_lse += b0 + b1;
+        sum_f2x2(rs2, l_sum);
+        sum_f2x2(rse2, l_lse);
       }
       tmem_wait_st();
       tc_fence_before();
@@ -546,11 +644,11 @@ attn_fwd_sm100(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
     *sm.abort_flag = 0;
     fence_barrier_init();
   }
-  if (warp == 9) {
+  if (warp == kWarpMma) {
     tmem_alloc(sm.tmem_holder, Cfg::TMEM_COLS);
     tmem_relinquish();
   }
-  if (warp == 8 && lane == 0) {
+  if (warp == kWarpLoad && lane == 0) {
     tma_prefetch_desc(&tm_q); tma_prefetch_desc(&tm_k); tma_prefetch_desc(&tm_v);
   }
   tc_fence_before();
@@ -558,15 +656,15 @@ attn_fwd_sm100(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
   tc_fence_after();
   const uint32_t tmem_base = *sm.tmem_holder;
 
-  if (warp >= 8) {
-    // load / MMA warpgroup (warps 10 and 11 have no role) gives registers away
+  if (warp < 4) {
+    // load / MMA warpgroup (warps 2 and 3 have no role) gives registers away
     regs_dec<Cfg::REGS_OTHER>();
-    if (warp == 8) fwd_producer<D, BF16>(&tm_q, &tm_k, &tm_v, p, sm, lane, cta, ncta);
-    else if (warp == 9) fwd_mma<D, BF16>(p, sm, tmem_base, lane, cta, ncta);
-    fwd_teardown(warp == 9, tmem_base, Cfg::TMEM_COLS);
+    if (warp == kWarpLoad) fwd_producer<D, BF16>(&tm_q, &tm_k, &tm_v, p, sm, lane, cta, ncta);
+    else if (warp == kWarpMma) fwd_mma<D, BF16>(p, sm, tmem_base, lane, cta, ncta);
+    fwd_teardown(warp == kWarpMma, tmem_base, Cfg::TMEM_COLS);
   } else {
     regs_inc<Cfg::REGS_SOFTMAX>();
-    fwd_softmax<D, BF16>(p, sm, tmem_base, warp, lane, cta, ncta);
+    fwd_softmax<D, BF16>(p, sm, tmem_base, warp - 4, lane, cta, ncta);
     fwd_teardown(false, tmem_base, Cfg::TMEM_COLS);
   }
 }
