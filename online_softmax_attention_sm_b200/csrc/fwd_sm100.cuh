@@ -13,10 +13,10 @@
 //   * warp 1 (one lane) issues TMA tensor loads: the two Q tiles once per unit, then
 //     K and V tiles into a ring of shared-memory slots (full/empty mbarriers);
 //   * warp 0 issues tcgen05.mma (warp-uniform code, one elected lane per instruction):
-//     S_t = Q_t K^T (128x128, fp32 in tensor
-//     memory) and O_t += P_t V (P_t read from tensor memory, O_t fp32 in tensor memory),
-//     in the order PV_0(j), QK_0(j+1), PV_1(j), QK_1(j+1) so that each softmax
-//     warpgroup works while the tensor core serves the other Q tile;
+//     S_t = Q_t K^T (128x128, fp32 in tensor memory) and O_t += P_t V (P_t read from
+//     tensor memory, O_t fp32 in tensor memory), in the order PV_0(j), QK_0(j+1), PV_1(j),
+//     QK_1(j+1) so that each softmax warpgroup works while the tensor core serves the
+//     other Q tile;
 //   * warpgroups 1 and 2 run the softmax of Q tile 0 and 1: each thread owns one row of
 //     S (tcgen05.ld 32x32b), computes the row max, p = 2^(c*s - m) with c = scale*log2(e),
 //     the row sums, writes P as 16-bit into tensor memory over S, and rescales its O row
@@ -59,15 +59,13 @@ struct FwdCfg {
   __host__ __device__ static constexpr uint32_t P_COL(int t) { return 128u * t; }
 };
 
-// Warp roles.  The MMA issuer is warp 0: it shares a scheduler with two softmax warps
-// that issue nearly every cycle, and the lowest warp index keeps its few instructions
-// from waiting behind theirs.  Warps 4-11 are the two softmax warpgroups.
+// Warp roles: warp 0 issues the MMAs, warp 1 the TMA loads, warps 4-11 are the two
+// softmax warpgroups.
 constexpr int kWarpMma = 0;
 constexpr int kWarpLoad = 1;
 
 constexpr float kRescaleThresh = 8.0f;   // log2 units: the reference moves past this
-constexpr float kHardThresh = 15.0f;     // log2 units: p < 2^15 fits fp16 and bf16
-constexpr int kPolyEvery = 0;            // full tiles: one exponential pair in kPolyEvery on the FMA pipe (0: none)
+constexpr int kPolyEvery = 4;            // full tiles: one exponential pair in kPolyEvery on the FMA pipe (0: none)
 
 struct FwdParams {
   void* o;
@@ -245,12 +243,11 @@ __device__ __forceinline__ void fwd_mma(const FwdParams& p, const FwdSmem<D>& sm
     bool ok = true;
     auto issue_qk = [&](int t, uint32_t k_addr) {
       const uint32_t q_addr = sQ_addr + t * Cfg::TILE_BYTES;
+      // D / 16 k-steps: 4 per 64-element (128-byte) chunk of the head dimension
 #pragma unroll
-      for (int kk = 0; kk < D / 16; ++kk) {
-        const uint32_t off = (kk >> 2) * Cfg::CHUNK_BYTES + (kk & 3) * 32;
-        mma_ss_warp(tmem_base + Cfg::S_COL(t), smem_desc_sw128(q_addr + off, 16, 1024),
-               smem_desc_sw128(k_addr + off, 16, 1024), IDESC_QK, kk > 0);
-      }
+      for (int c = 0; c < Cfg::KCH; ++c)
+        mma_ss_x4(tmem_base + Cfg::S_COL(t), smem_desc_sw128(q_addr + c * Cfg::CHUNK_BYTES, 16, 1024),
+                  smem_desc_sw128(k_addr + c * Cfg::CHUNK_BYTES, 16, 1024), IDESC_QK, c > 0);
       mma_commit_warp(&sm.s_full[t]);
     };
     // Issue order per K/V step j:  PV_0(j), QK_0(j+1), PV_1(j), QK_1(j+1).
@@ -293,21 +290,14 @@ __device__ __forceinline__ void fwd_mma(const FwdParams& p, const FwdSmem<D>& sm
           ok = mbar_wait_warp(&sm.p_part[t], (t ? pv1 : pv0) & 1, sm.abort_flag, 17);
           if (!ok) break;
           tc_fence_after();
-#pragma unroll
-          for (int kk = 0; kk < 6; ++kk) {
-            mma_ts_warp(tmem_base + Cfg::O_COL(t), tmem_base + Cfg::P_COL(t) + kk * 8,
-                   smem_desc_sw128(v_addr + kk * 2048, Cfg::CHUNK_BYTES, 1024), IDESC_PV,
-                   (j > 0 || kk > 0) ? 1u : 0u);
-          }
+          mma_ts_x6(tmem_base + Cfg::O_COL(t), tmem_base + Cfg::P_COL(t),
+                    smem_desc_sw128(v_addr, Cfg::CHUNK_BYTES, 1024), IDESC_PV, j > 0 ? 1u : 0u);
           ok = mbar_wait_warp(&sm.p_full[t], (t ? pv1 : pv0) & 1, sm.abort_flag, 14);
           if (!ok) break;
           tc_fence_after();
-#pragma unroll
-          for (int kk = 6; kk < 8; ++kk) {
-            mma_ts_warp(tmem_base + Cfg::O_COL(t), tmem_base + Cfg::P_COL(t) + kk * 8,
-                   smem_desc_sw128(v_addr + kk * 2048, Cfg::CHUNK_BYTES, 1024), IDESC_PV, 1u);
-          }
-          mma_commit_warp(&sm.o_done[t]);
+          mma_ts_x2(tmem_base + Cfg::O_COL(t), tmem_base + Cfg::P_COL(t) + 6 * 8,
+                    smem_desc_sw128(v_addr + 6 * 2048, Cfg::CHUNK_BYTES, 1024), IDESC_PV, 1u);
+          if (j + 1 == x.nkv[t]) mma_commit_warp(&sm.o_done[t]);   // O_t complete for the epilogue
           if (t) ++pv1; else ++pv0;
           // ---- S_t = Q_t K_{j+1}^T
           if (j + 1 < x.nkv[t]) {
@@ -364,22 +354,20 @@ __device__ __forceinline__ void exp2_poly_pair(float x0, float x1, float& a, flo
   b = __uint_as_float(__float_as_uint(q1) + (__float_as_uint(t1) << 23));
 }
 
-// One 32-key chunk of a row: p = 2^(scale2 * s - m) on pairs (one packed FMA per pair),
-// P stored to tensor memory as 16-bit at taddr, both row sums (rse2: the fp32 weights,
-// for the LSE; rs2: the 16-bit weights the MMA multiplies, so O / l is an exact weighted
-// average of V).  With TRACK the chunk's scores also enter the running max mx.  With
-// POLY > 0, one pair in POLY is exponentiated by exp2_poly_pair (finite x only).
-template <bool BF16, bool TRACK, int POLY>
-__device__ __forceinline__ void softmax_chunk(const float (&s)[128], const int c, const f32x2 scale2,
+// One 32-key chunk of a row (v: the 32 scores as raw fp32 bits): p = 2^(scale2 * s - m) on
+// pairs (one packed FMA per pair), P stored to tensor memory as 16-bit at taddr, both row
+// sums (rse2: the fp32 weights, for the LSE; rs2: the 16-bit weights the MMA multiplies,
+// so O / l is an exact weighted average of V).  With POLY > 0, one pair in POLY is
+// exponentiated by exp2_poly_pair (finite scores only).
+template <bool BF16, int POLY>
+__device__ __forceinline__ void softmax_chunk(const uint32_t (&v)[32], const f32x2 scale2,
                                               const f32x2 negm2, f32x2 (&rs2)[2], f32x2 (&rse2)[2],
-                                              float (&mx)[8], const uint32_t taddr) {
+                                              const uint32_t taddr) {
   uint32_t pk[16];
 #pragma unroll
   for (int i = 0; i < 16; ++i) {
-    const float s0 = s[c * 32 + 2 * i], s1 = s[c * 32 + 2 * i + 1];
-    if (TRACK) mx[i & 7] = max3f(mx[i & 7], s0, s1);
     float x0, x1;
-    unpack_f2(fma_f2(pack_f2(s0, s1), scale2, negm2), x0, x1);
+    unpack_f2(fma_f2(pack_f2(__uint_as_float(v[2 * i]), __uint_as_float(v[2 * i + 1])), scale2, negm2), x0, x1);
     float a, b2;
     if (POLY > 0 && (i % (POLY > 0 ? POLY : 1)) == POLY - 1) {
       exp2_poly_pair(x0, x1, a, b2);          // on the FMA pipe, sparing the MUFU
@@ -406,6 +394,18 @@ __device__ __forceinline__ void softmax_chunk(const float (&s)[128], const int c
   tmem_st16(taddr, pk);
 }
 
+// Running max over a 32-score chunk on 8 chains.
+__device__ __forceinline__ void chunk_max(const uint32_t (&v)[32], float (&mx)[8]) {
+#pragma unroll
+  for (int k = 0; k < 8; ++k)
+    mx[k] = max3f(mx[k], max3f(__uint_as_float(v[k]), __uint_as_float(v[k + 8]), __uint_as_float(v[k + 16])),
+                  __uint_as_float(v[k + 24]));
+}
+
+__device__ __forceinline__ float max_of8(const float (&mx)[8]) {
+  return fmaxf(max3f(mx[0], mx[1], mx[2]), max3f(max3f(mx[3], mx[4], mx[5]), mx[6], mx[7]));
+}
+
 // O_t row *= alpha, in place in tensor memory (32 columns at a time).
 template <int D>
 __device__ __forceinline__ void rescale_o_row(const uint32_t taddr, const float alpha) {
@@ -426,6 +426,112 @@ __device__ __forceinline__ void sum_f2x2(const f32x2 (&v)[2], float& acc) {
   acc += a0 + a1;
 }
 
+// Move the row's reference max to m_tile when it exceeds the reference by more than
+// kRescaleThresh, rescaling both sums and (after the first tile) the O_t row by
+// 2^(m_ref - m_tile).  O_t holds P V up to the previous tile, complete: the commit that
+// signalled this tile's S covers every earlier MMA.
+template <int D>
+__device__ __forceinline__ void move_reference(const float m_tile, const bool first, float& m_ref,
+                                               float& l_sum, float& l_lse, const uint32_t o_addr) {
+  const bool need = m_tile > m_ref + kRescaleThresh;
+  float alpha = 1.f;
+  if (need) {
+    alpha = ex2(m_ref - m_tile);       // 0 when m_ref == -inf
+    l_sum *= alpha;
+    l_lse *= alpha;
+    m_ref = m_tile;
+  }
+  if (!first && __any_sync(0xffffffffu, need)) rescale_o_row<D>(o_addr, alpha);
+}
+
+// A K/V tile every row of the Q tile sees in full, with scale >= 0 (the scale goes into
+// the exponent's FMA).  Two passes over S: the row max from all 128 scores, then the
+// exponentials.  P overwrites S columns 0-63 only, so the second pass holds chunks 0-1
+// from the first and loads chunks 2-3 again, which keeps a quarter fewer registers live
+// through the exponentials.  The MMA warp may start on keys 0-95 at p_part.
+template <int D, bool BF16>
+__device__ __forceinline__ void softmax_tile_full(const uint32_t s_addr, const uint32_t o_addr,
+                                                  const uint32_t p_addr, const float c2, const bool first,
+                                                  float& m_ref, float& l_sum, float& l_lse,
+                                                  uint64_t* p_part) {
+  uint32_t v0[32], v1[32];
+  float mx[8];
+#pragma unroll
+  for (int k = 0; k < 8; ++k) mx[k] = -INFINITY;
+  {
+    uint32_t v2[32], v3[32];
+    tmem_ld32(s_addr, v0);
+    tmem_ld32(s_addr + 32, v1);
+    tmem_ld32(s_addr + 64, v2);
+    tmem_ld32(s_addr + 96, v3);
+    tmem_wait_ld_regs(v0);
+    tmem_wait_ld_regs(v1);
+    tmem_wait_ld_regs(v2);
+    tmem_wait_ld_regs(v3);
+    chunk_max(v0, mx);
+    chunk_max(v1, mx);
+    chunk_max(v2, mx);
+    chunk_max(v3, mx);
+  }
+  move_reference<D>(max_of8(mx) * c2, first, m_ref, l_sum, l_lse, o_addr);
+  const float m_use = (m_ref == -INFINITY) ? 0.f : m_ref;
+  const f32x2 scale2 = pack_f2(c2, c2), negm2 = pack_f2(-m_use, -m_use);
+  f32x2 rs2[2] = {0ull, 0ull}, rse2[2] = {0ull, 0ull};
+  uint32_t v2[32], v3[32];
+  tmem_ld32(s_addr + 64, v2);
+  softmax_chunk<BF16, kPolyEvery>(v0, scale2, negm2, rs2, rse2, p_addr);
+  softmax_chunk<BF16, kPolyEvery>(v1, scale2, negm2, rs2, rse2, p_addr + 16);
+  tmem_wait_ld_regs(v2);
+  tmem_ld32(s_addr + 96, v3);
+  softmax_chunk<BF16, kPolyEvery>(v2, scale2, negm2, rs2, rse2, p_addr + 32);
+  tmem_wait_st();
+  tc_fence_before();
+  mbar_arrive(p_part);
+  tmem_wait_ld_regs(v3);
+  softmax_chunk<BF16, kPolyEvery>(v3, scale2, negm2, rs2, rse2, p_addr + 48);
+  sum_f2x2(rs2, l_sum);
+  sum_f2x2(rse2, l_lse);
+}
+
+// A tile that crosses the causal diagonal or the ragged end of K (or a negative scale):
+// scores are scaled first and keys >= kl set to -inf, then max and exponentials.
+template <int D, bool BF16>
+__device__ __forceinline__ void softmax_tile_masked(const uint32_t s_addr, const uint32_t o_addr,
+                                                    const uint32_t p_addr, const float c2, const int kl,
+                                                    const bool first, float& m_ref, float& l_sum,
+                                                    float& l_lse, uint64_t* p_part) {
+  uint32_t v[4][32];
+#pragma unroll
+  for (int c = 0; c < 4; ++c) tmem_ld32(s_addr + c * 32, v[c]);
+#pragma unroll
+  for (int c = 0; c < 4; ++c) tmem_wait_ld_regs(v[c]);
+  float mx[8];
+#pragma unroll
+  for (int k = 0; k < 8; ++k) mx[k] = -INFINITY;
+#pragma unroll
+  for (int c = 0; c < 4; ++c) {
+#pragma unroll
+    for (int i = 0; i < 32; ++i)
+      v[c][i] = __float_as_uint((c * 32 + i < kl) ? __uint_as_float(v[c][i]) * c2 : -INFINITY);
+    chunk_max(v[c], mx);
+  }
+  move_reference<D>(max_of8(mx), first, m_ref, l_sum, l_lse, o_addr);
+  const float m_use = (m_ref == -INFINITY) ? 0.f : m_ref;
+  const f32x2 scale2 = pack_f2(1.f, 1.f), negm2 = pack_f2(-m_use, -m_use);
+  f32x2 rs2[2] = {0ull, 0ull}, rse2[2] = {0ull, 0ull};
+#pragma unroll
+  for (int c = 0; c < 4; ++c) {
+    softmax_chunk<BF16, 0>(v[c], scale2, negm2, rs2, rse2, p_addr + c * 16);
+    if (c == 2) {
+      tmem_wait_st();
+      tc_fence_before();
+      mbar_arrive(p_part);
+    }
+  }
+  sum_f2x2(rs2, l_sum);
+  sum_f2x2(rse2, l_lse);
+}
+
 template <int D, bool BF16>
 __device__ __forceinline__ void fwd_softmax(const FwdParams& p, const FwdSmem<D>& sm, uint32_t tmem_base,
                                             int warp, int lane, int cta, int ncta) {
@@ -435,7 +541,7 @@ __device__ __forceinline__ void fwd_softmax(const FwdParams& p, const FwdSmem<D>
   const int row_in_tile = wl * 32 + lane;
   const uint32_t lane_addr = tmem_base + ((uint32_t)(wl * 32) << 16);
   const float c2 = p.c2;
-  int s_n = 0, o_n = 0;                     // s_full / o_done phases consumed
+  int s_n = 0, o_n = 0;                     // s_full / o_done phases consumed (o_done: one per unit)
   bool ok = true;
   for (int round = 0; ok; ++round) {
     int u = fwd_unit_of(round, cta, ncta);
@@ -453,109 +559,19 @@ __device__ __forceinline__ void fwd_softmax(const FwdParams& p, const FwdSmem<D>
     // l_sum: sum of the 16-bit weights (normalises O, matching what the MMA multiplied);
     // l_lse: sum of the fp32 weights (gives the LSE without the 16-bit rounding bias)
     float m_ref = -INFINITY, l_sum = 0.f, l_lse = 0.f;
-    float m_next = -INFINITY;               // a reference chosen on one tile, applied on the next
+    const uint32_t s_addr = lane_addr + Cfg::S_COL(t), o_addr = lane_addr + Cfg::O_COL(t);
     const uint32_t p_addr = lane_addr + Cfg::P_COL(t);
     for (int j = 0; j < nkv; ++j) {
-      ok = __all_sync(0xffffffffu, mbar_wait(&sm.s_full[t], s_n & 1, sm.abort_flag, 20 + t));
+      ok = mbar_wait_warp(&sm.s_full[t], s_n & 1, sm.abort_flag, 20 + t);
       if (!ok) break;
       ++s_n;
       tc_fence_after();
-      float s[128];
-#pragma unroll
-      for (int c = 0; c < 4; ++c) {
-        uint32_t r[32];
-        tmem_ld32(lane_addr + Cfg::S_COL(t) + c * 32, r);
-#pragma unroll
-        for (int i = 0; i < 32; ++i) s[c * 32 + i] = __uint_as_float(r[i]);
-      }
-      tmem_wait_ld();
-      const bool masked = (j >= mask_from);
-      const bool plain = !masked && c2 >= 0.f;     // full tile, scale >= 0: s scaled in the FMA
-      // O_t holds P V up to tile j-1, complete: S_t(j)'s commit covers every earlier MMA.
-      // A move of the reference chosen on tile j-1 is applied to it now, before any of
-      // this tile's P is handed to the MMA warp.
-      {
-        const bool moved = m_next > m_ref;
-        float alpha = 1.f;
-        if (moved) {
-          alpha = ex2(m_ref - m_next);
-          l_sum *= alpha;
-          l_lse *= alpha;
-          m_ref = m_next;
-        }
-        if (__any_sync(0xffffffffu, moved)) rescale_o_row<D>(lane_addr + Cfg::O_COL(t), alpha);
-      }
-      bool done = false;
-      if (__all_sync(0xffffffffu, plain && m_ref > -INFINITY)) {
-        // Full tile after the first: exponentiate against the current reference while
-        // taking the tile max in the same pass (the last chunk's max first, so that the
-        // whole max is known before the first 96 keys are handed over).  A tile max up
-        // to kHardThresh above the reference is accepted (p < 2^kHardThresh stays finite
-        // and exact to the 16-bit rounding) and moves the reference for the next tile;
-        // a larger one redoes the tile below with the moved reference.
-        float mx[8];
-#pragma unroll
-        for (int k = 0; k < 8; ++k) mx[k] = max3f(s[96 + k], s[104 + k], fmaxf(s[112 + k], s[120 + k]));
-        const f32x2 scale2 = pack_f2(c2, c2), negm2 = pack_f2(-m_ref, -m_ref);
-        f32x2 rs2[2] = {0ull, 0ull}, rse2[2] = {0ull, 0ull};
-#pragma unroll
-        for (int c = 0; c < 3; ++c) softmax_chunk<BF16, true, kPolyEvery>(s, c, scale2, negm2, rs2, rse2, mx, p_addr + c * 16);
-        const float m_tile =
-            fmaxf(max3f(mx[0], mx[1], mx[2]), max3f(max3f(mx[3], mx[4], mx[5]), mx[6], mx[7])) * c2;
-        if (!__any_sync(0xffffffffu, m_tile > m_ref + kHardThresh)) {
-          tmem_wait_st();
-          tc_fence_before();
-          mbar_arrive(&sm.p_part[t]);
-          softmax_chunk<BF16, false, kPolyEvery>(s, 3, scale2, negm2, rs2, rse2, mx, p_addr + 48);
-          sum_f2x2(rs2, l_sum);
-          sum_f2x2(rse2, l_lse);
-          if (m_tile > m_ref + kRescaleThresh) m_next = m_tile;
-          done = true;
-        } else {
-          tmem_wait_st();                          // the redo below rewrites these columns
-        }
-      }
-      if (!done) {
-        if (!plain) {
-          // diagonal / ragged tiles (and negative scales): scale first, mask
-          const int kl = masked ? klim - j * 128 : 128;   // keys >= kl are invisible to this row
-#pragma unroll
-          for (int i = 0; i < 128; ++i) s[i] = (i < kl) ? s[i] * c2 : -INFINITY;
-        }
-        // the row max, the reference (moved only past the lazy threshold), alpha
-        float mx[8];
-#pragma unroll
-        for (int k = 0; k < 8; ++k) mx[k] = fmaxf(s[k], s[k + 8]);
-#pragma unroll
-        for (int i = 16; i < 128; i += 16)
-#pragma unroll
-          for (int k = 0; k < 8; ++k) mx[k] = max3f(mx[k], s[i + k], s[i + 8 + k]);
-        float m_tile = fmaxf(max3f(mx[0], mx[1], mx[2]), max3f(max3f(mx[3], mx[4], mx[5]), mx[6], mx[7]));
-        if (plain) m_tile *= c2;
-        const bool need = m_tile > m_ref + kRescaleThresh;
-        float alpha = 1.f;
-        if (need) {
-          alpha = ex2(m_ref - m_tile);       // 0 when m_ref == -inf
-          l_sum *= alpha;
-          l_lse *= alpha;
-          m_ref = m_tile;
-        }
-        if (j > 0 && __any_sync(0xffffffffu, need)) rescale_o_row<D>(lane_addr + Cfg::O_COL(t), alpha);
-        const float m_use = (m_ref == -INFINITY) ? 0.f : m_ref;
-        const f32x2 scale2 = plain ? pack_f2(c2, c2) : pack_f2(1.f, 1.f);
-        const f32x2 negm2 = pack_f2(-m_use, -m_use);
-        f32x2 rs2[2] = {0ull, 0ull}, rse2[2] = {0ull, 0ull};
-#pragma unroll
-        for (int c = 0; c < 4; ++c) {
-          softmax_chunk<BF16, false, 0>(s, c, scale2, negm2, rs2, rse2, mx, p_addr + c * 16);
-          if (c == 2) {                       // the MMA warp may start on the first 96 keys
-            tmem_wait_st();
-            tc_fence_before();
-            mbar_arrive(&sm.p_part[t]);
-          }
-        }
-        sum_f2x2(rs2, l_sum);
-        sum_f2x2(rse2, l_lse);
+      if (j < mask_from && c2 >= 0.f) {
+        softmax_tile_full<D, BF16>(s_addr, o_addr, p_addr, c2, j == 0, m_ref, l_sum, l_lse, &sm.p_part[t]);
+      } else {
+        const int kl = (j >= mask_from) ? klim - j * 128 : 128;   // keys >= kl: invisible to this row
+        softmax_tile_masked<D, BF16>(s_addr, o_addr, p_addr, c2, kl, j == 0, m_ref, l_sum, l_lse,
+                                     &sm.p_part[t]);
       }
       tmem_wait_st();
       tc_fence_before();
@@ -564,9 +580,9 @@ __device__ __forceinline__ void fwd_softmax(const FwdParams& p, const FwdSmem<D>
     if (!ok) break;
     // ---------------- epilogue: O / l, LSE
     if (nkv > 0) {
-      ok = __all_sync(0xffffffffu, mbar_wait(&sm.o_done[t], (o_n + nkv - 1) & 1, sm.abort_flag, 22 + t));
+      ok = mbar_wait_warp(&sm.o_done[t], o_n & 1, sm.abort_flag, 22 + t);
       if (!ok) break;
-      o_n += nkv;
+      ++o_n;
       tc_fence_after();
     }
     const bool store = row < p.Sq;

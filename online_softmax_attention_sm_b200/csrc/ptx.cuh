@@ -83,10 +83,27 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity,
   }
 }
 
-// mbar_wait by every lane of a warp, with one answer for the whole warp.
+// Bounded wait by every lane of a warp, with one answer for the whole warp.  Each poll
+// is a warp vote and every branch depends only on votes, so the warp never diverges:
+// an already-completed phase costs one poll and one vote (a per-lane early return
+// would make the compiler split and re-converge the warp around every wait).
 __device__ __forceinline__ bool mbar_wait_warp(uint64_t* bar, uint32_t parity,
                                                volatile int* abort, int where) {
-  return __all_sync(0xffffffffu, mbar_wait(bar, parity, abort, where));
+  if (__all_sync(0xffffffffu, mbar_try_wait(bar, parity))) return true;
+  const uint64_t t0 = globaltimer_ns();
+  for (uint32_t it = 1;; ++it) {
+    if (__all_sync(0xffffffffu, mbar_try_wait(bar, parity))) return true;
+    if ((it & 255u) == 0) {
+      if (__any_sync(0xffffffffu, abort != nullptr && *abort != 0)) return false;
+      if (__any_sync(0xffffffffu, globaltimer_ns() - t0 > kWaitLimitNs)) {
+        if ((threadIdx.x & 31) == 0) {
+          record_timeout(where);
+          if (abort) *abort = 1;
+        }
+        return false;
+      }
+    }
+  }
 }
 
 // ----------------------------------------------------------------------------------
@@ -133,24 +150,61 @@ __device__ __forceinline__ void tc_fence_after() {
 // tcgen05.mma (D[tmem] (+)= A * B, A from a shared-memory descriptor or tensor memory, B
 // from a shared-memory descriptor) and tcgen05.commit (arrive once on `bar` when every
 // tcgen05 op issued so far has completed), in warp-wide form: all 32 lanes execute them
-// with the same operands and elect.sync picks the one lane that issues.  Keeping the issuing code warp-uniform (no lane-0 branch)
-// lets the operands stay on the uniform datapath, so an MMA costs a few issue slots even
-// while the softmax warps on the same scheduler issue every cycle.
-__device__ __forceinline__ void mma_ss_warp(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
-                                            uint32_t idesc, uint32_t accumulate) {
+// with the same operands and elect.sync picks the one lane that issues.  Keeping the
+// issuing code warp-uniform (no lane-0 branch) lets the operands stay on the uniform
+// datapath, so an MMA costs a few issue slots even while the softmax warps on the same
+// scheduler issue every cycle.
+//
+// Batches of k-steps in one asm block, one elect.sync per batch (fewer instructions for
+// the issuing warp, whose scheduler it shares with two busy softmax warps).  A descriptor
+// holds the shared-memory address >> 4 in its low 14 bits; addresses stay below 256 KB, so
+// stepping a descriptor is a plain add on it.
+//   mma_ss_x4: 4 k-steps of 16 elements along a 128-byte swizzled row: both descriptors
+//              advance 32 bytes per step; the first step accumulates iff acc_first.
+__device__ __forceinline__ void mma_ss_x4(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
+                                          uint32_t idesc, uint32_t acc_first) {
   asm volatile(
-      "{\n .reg .pred p, e;\n .reg .b32 r;\n elect.sync r|e, 0xffffffff;\n"
-      " setp.ne.b32 p, %4, 0;\n"
-      " @e tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n}\n"
-      ::"r"(d_tmem), "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate) : "memory");
+      "{\n .reg .pred e, p, q;\n .reg .b32 r;\n .reg .b64 a, b;\n"
+      " elect.sync r|e, 0xffffffff;\n setp.ne.b32 p, %4, 0;\n setp.ne.b32 q, %5, 0;\n"
+      " @e tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n"
+      " add.s64 a, %1, 2;\n add.s64 b, %2, 2;\n"
+      " @e tcgen05.mma.cta_group::1.kind::f16 [%0], a, b, %3, q;\n"
+      " add.s64 a, %1, 4;\n add.s64 b, %2, 4;\n"
+      " @e tcgen05.mma.cta_group::1.kind::f16 [%0], a, b, %3, q;\n"
+      " add.s64 a, %1, 6;\n add.s64 b, %2, 6;\n"
+      " @e tcgen05.mma.cta_group::1.kind::f16 [%0], a, b, %3, q;\n}\n"
+      ::"r"(d_tmem), "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(acc_first), "r"(1u) : "memory");
 }
-__device__ __forceinline__ void mma_ts_warp(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc,
-                                            uint32_t idesc, uint32_t accumulate) {
+//   mma_ts_x2: 2 k-steps with A in tensor memory (16 keys = 8 columns of 16-bit pairs per
+//              step) and B stepping 16 rows of 128 bytes (2048 bytes) per step.
+__device__ __forceinline__ void mma_ts_x2(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc,
+                                          uint32_t idesc, uint32_t acc_first) {
   asm volatile(
-      "{\n .reg .pred p, e;\n .reg .b32 r;\n elect.sync r|e, 0xffffffff;\n"
-      " setp.ne.b32 p, %4, 0;\n"
-      " @e tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n}\n"
-      ::"r"(d_tmem), "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate) : "memory");
+      "{\n .reg .pred e, p, q;\n .reg .b32 r, a;\n .reg .b64 b;\n"
+      " elect.sync r|e, 0xffffffff;\n setp.ne.b32 p, %4, 0;\n setp.ne.b32 q, %5, 0;\n"
+      " @e tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n"
+      " add.u32 a, %1, 8;\n add.s64 b, %2, 128;\n"
+      " @e tcgen05.mma.cta_group::1.kind::f16 [%0], [a], b, %3, q;\n}\n"
+      ::"r"(d_tmem), "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(acc_first), "r"(1u) : "memory");
+}
+//   mma_ts_x6: 6 such k-steps.
+__device__ __forceinline__ void mma_ts_x6(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc,
+                                          uint32_t idesc, uint32_t acc_first) {
+  asm volatile(
+      "{\n .reg .pred e, p, q;\n .reg .b32 r, a;\n .reg .b64 b;\n"
+      " elect.sync r|e, 0xffffffff;\n setp.ne.b32 p, %4, 0;\n setp.ne.b32 q, %5, 0;\n"
+      " @e tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n"
+      " add.u32 a, %1, 8;\n add.s64 b, %2, 128;\n"
+      " @e tcgen05.mma.cta_group::1.kind::f16 [%0], [a], b, %3, q;\n"
+      " add.u32 a, %1, 16;\n add.s64 b, %2, 256;\n"
+      " @e tcgen05.mma.cta_group::1.kind::f16 [%0], [a], b, %3, q;\n"
+      " add.u32 a, %1, 24;\n add.s64 b, %2, 384;\n"
+      " @e tcgen05.mma.cta_group::1.kind::f16 [%0], [a], b, %3, q;\n"
+      " add.u32 a, %1, 32;\n add.s64 b, %2, 512;\n"
+      " @e tcgen05.mma.cta_group::1.kind::f16 [%0], [a], b, %3, q;\n"
+      " add.u32 a, %1, 40;\n add.s64 b, %2, 640;\n"
+      " @e tcgen05.mma.cta_group::1.kind::f16 [%0], [a], b, %3, q;\n}\n"
+      ::"r"(d_tmem), "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(acc_first), "r"(1u) : "memory");
 }
 __device__ __forceinline__ void mma_commit_warp(uint64_t* bar) {
   asm volatile(
@@ -200,6 +254,18 @@ __device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t* r) {
 
 __device__ __forceinline__ void tmem_wait_ld() {
   asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+}
+// tcgen05.wait::ld that also names the 32 registers a preceding tmem_ld32 filled, so no
+// use of them can be scheduled above the wait (the load writes them asynchronously).
+__device__ __forceinline__ void tmem_wait_ld_regs(uint32_t (&r)[32]) {
+  asm volatile("tcgen05.wait::ld.sync.aligned;"
+               : "+r"(r[0]), "+r"(r[1]), "+r"(r[2]), "+r"(r[3]), "+r"(r[4]), "+r"(r[5]), "+r"(r[6]),
+                 "+r"(r[7]), "+r"(r[8]), "+r"(r[9]), "+r"(r[10]), "+r"(r[11]), "+r"(r[12]),
+                 "+r"(r[13]), "+r"(r[14]), "+r"(r[15]), "+r"(r[16]), "+r"(r[17]), "+r"(r[18]),
+                 "+r"(r[19]), "+r"(r[20]), "+r"(r[21]), "+r"(r[22]), "+r"(r[23]), "+r"(r[24]),
+                 "+r"(r[25]), "+r"(r[26]), "+r"(r[27]), "+r"(r[28]), "+r"(r[29]), "+r"(r[30]),
+                 "+r"(r[31])
+               :: "memory");
 }
 __device__ __forceinline__ void tmem_wait_st() {
   asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
