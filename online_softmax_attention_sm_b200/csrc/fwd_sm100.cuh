@@ -8,8 +8,9 @@
 //
 // B200 design:
 //   * unit of work = (batch, query head, 256 query rows) = two 128-row Q tiles that
-//     share every K/V tile; a persistent grid of one CTA per SM walks the units in
-//     longest-first order (causal units with more K/V tiles first);
+//     share every K/V tile; a persistent grid of one CTA per SM takes the units in
+//     longest-first order (causal units with more K/V tiles first), each CTA fetching its
+//     next unit from a global counter when it is ready for one;
 //   * warp 1 (one lane) issues TMA tensor loads: the two Q tiles once per unit, then
 //     K and V tiles into a ring of shared-memory slots (full/empty mbarriers);
 //   * warp 0 issues tcgen05.mma (warp-uniform code, one elected lane per instruction):
@@ -76,7 +77,12 @@ struct FwdParams {
   int kv_group;      // (batch, KV head) pairs per scheduling group (their K/V fit in L2)
   int band;          // query blocks per band (a band of one group fills about one round)
   float c2;          // scale * log2(e)
+  unsigned int* work;  // [2] dynamic scheduling (the kernel's DYN instance): next unit to
+                       // hand out past the first round, CTAs done fetching; zero at launch,
+                       // zeroed again by the launch's last CTA
 };
+
+constexpr int kUnitQueue = 4;    // unit indices the load warp may hand out ahead
 
 struct UnitInfo {
   int b, h, kvh, q0;         // q0: first query row of the unit
@@ -99,7 +105,7 @@ __device__ __forceinline__ int fwd_kv_tiles(const FwdParams& p, int r0) {
 // block descending, then the group's query heads.  The host sizes a group so its K and V
 // fit in half the L2 and a (band, group) block fills about one round of the persistent
 // grid: the CTAs in flight then share K/V tiles through L2, and consecutive rounds hold
-// units of the same lengths (longest first overall, which the snake assignment needs).
+// units of similar lengths (longest first overall, so the last units handed out are short).
 __device__ __forceinline__ UnitInfo fwd_unit(const FwdParams& p, int u) {
   UnitInfo x;
   const int G = p.Hq / p.Hkv;
@@ -125,11 +131,15 @@ __device__ __forceinline__ UnitInfo fwd_unit(const FwdParams& p, int u) {
   return x;
 }
 
-// Snake assignment of the longest-first unit list over the persistent CTAs.
+// Units are handed out in list order (longest first).  Static: round r gives CTA c unit
+// r * ncta + c, reversed on odd rounds (a snake, so a CTA's long and short units pair up).
+// Dynamic: CTA c starts with unit c, then its load warp takes the next unit from a global
+// counter when it is ready for one (the kernel's DYN instance).  The host picks dynamic when
+// its estimate of the static order's imbalance is large (few rounds of very different
+// lengths); where the static order balances, the static instance measured faster.
 __device__ __forceinline__ int fwd_unit_of(int round, int cta, int ncta) {
   return round * ncta + ((round & 1) ? (ncta - 1 - cta) : cta);
 }
-
 // Shared-memory map: Q tiles, K/V ring, then the barriers and two words.
 template <int D>
 struct FwdSmem {
@@ -147,6 +157,9 @@ struct FwdSmem {
   uint64_t* p_part;    // [2]  first 96 keys of P_t written, O_t rescaled (128 threads)
   uint32_t* tmem_holder;
   volatile int* abort_flag;
+  uint64_t* unit_full;   // [kUnitQueue]  unit index written by the load warp
+  uint64_t* unit_empty;  // [kUnitQueue]  read by the MMA warp and the 8 softmax warps
+  volatile int* uq;      // [kUnitQueue]  the unit indices
   __device__ explicit FwdSmem(uint8_t* s) {
     q = s;
     ring = s + Cfg::SMEM_Q;
@@ -162,11 +175,25 @@ struct FwdSmem {
     p_part = q_full + 11;
     tmem_holder = (uint32_t*)(q_full + 13);
     abort_flag = (volatile int*)(tmem_holder + 1);
+    unit_full = q_full + 14;
+    unit_empty = unit_full + kUnitQueue;
+    uq = (volatile int*)(unit_empty + kUnitQueue);
   }
 };
 
+// The n-th unit of this CTA, for a consuming warp: wait for the load warp to post it, read
+// it, release the queue slot (one arrival per warp).  Returns -1 if the wait gave up.
+template <int D>
+__device__ __forceinline__ int fwd_next_unit(const FwdSmem<D>& sm, int n, int where) {
+  const int slot = n % kUnitQueue;
+  if (!mbar_wait_warp(&sm.unit_full[slot], (n / kUnitQueue) & 1, sm.abort_flag, where)) return -1;
+  const int u = sm.uq[slot];
+  mbar_arrive_warp(&sm.unit_empty[slot]);
+  return u;
+}
+
 // ------------------------------------------------------------------ TMA producer
-template <int D, bool BF16>
+template <int D, bool BF16, bool DYN>
 __device__ __forceinline__ void fwd_producer(const CUtensorMap* tm_q, const CUtensorMap* tm_k,
                                              const CUtensorMap* tm_v, const FwdParams& p,
                                              const FwdSmem<D>& sm, int lane, int cta, int ncta) {
@@ -175,8 +202,21 @@ __device__ __forceinline__ void fwd_producer(const CUtensorMap* tm_q, const CUte
     int slot = 0, ring_n = 0;            // ring position and total loads issued
     int q_load0 = 0, q_load1 = 0;        // Q tile loads issued
     bool ok = true;
-    for (int round = 0; ok; ++round) {
-      int u = fwd_unit_of(round, cta, ncta);
+    for (int n = 0; ok; ++n) {
+      // ---- the next unit (an index past the list ends the CTA), posted to the other roles
+      int u;
+      if (!DYN) {
+        u = fwd_unit_of(n, cta, ncta);       // every role computes the same index
+      } else {
+        const int us = n % kUnitQueue;
+        u = n == 0 ? cta : ncta + (int)atomicAdd(p.work, 1u);
+        if (n >= kUnitQueue) {
+          ok = mbar_wait(&sm.unit_empty[us], ((n / kUnitQueue) - 1) & 1, sm.abort_flag, 5);
+          if (!ok) break;
+        }
+        sm.uq[us] = u;
+        mbar_arrive(&sm.unit_full[us]);
+      }
       if (u >= p.n_units) break;
       UnitInfo x = fwd_unit(p, u);
       for (int j = 0; j < x.nkv_max && ok; ++j) {
@@ -222,12 +262,18 @@ __device__ __forceinline__ void fwd_producer(const CUtensorMap* tm_q, const CUte
       if (q_load0 > 0) mbar_wait(&sm.q_full[0], (q_load0 - 1) & 1, nullptr, 4);
       if (q_load1 > 0) mbar_wait(&sm.q_full[1], (q_load1 - 1) & 1, nullptr, 4);
     }
+    // this CTA takes no more units; the last CTA to get here zeroes the launch's counters
+    // for the next launch that uses them (nothing reads them after this point)
+    if (DYN && atomicAdd(p.work + 1, 1u) == (unsigned)ncta - 1) {
+      atomicExch(p.work, 0u);
+      atomicExch(p.work + 1, 0u);
+    }
   }
   __syncwarp();
 }
 
 // ------------------------------------------------------------------ MMA issuer
-template <int D, bool BF16>
+template <int D, bool BF16, bool DYN>
 __device__ __forceinline__ void fwd_mma(const FwdParams& p, const FwdSmem<D>& sm, uint32_t tmem_base,
                                         int lane, int cta, int ncta) {
   using Cfg = FwdCfg<D>;
@@ -255,8 +301,9 @@ __device__ __forceinline__ void fwd_mma(const FwdParams& p, const FwdSmem<D>& sm
     // PV_t(j) read them.  tcgen05.mma instructions issued by one thread execute in
     // issue order, so the overwrite cannot overtake the read, and each softmax
     // warpgroup gets the other tile's PV + QK as cover for its exponentials.
-    for (int round = 0; ok; ++round) {
-      int u = fwd_unit_of(round, cta, ncta);
+    for (int n = 0; ok; ++n) {
+      const int u = DYN ? fwd_next_unit(sm, n, 12) : fwd_unit_of(n, cta, ncta);
+      if (u < 0) { ok = false; break; }
       if (u >= p.n_units) break;
       UnitInfo x = fwd_unit(p, u);
       if (x.nkv_max == 0) continue;
@@ -532,7 +579,7 @@ __device__ __forceinline__ void softmax_tile_masked(const uint32_t s_addr, const
   sum_f2x2(rse2, l_lse);
 }
 
-template <int D, bool BF16>
+template <int D, bool BF16, bool DYN>
 __device__ __forceinline__ void fwd_softmax(const FwdParams& p, const FwdSmem<D>& sm, uint32_t tmem_base,
                                             int warp, int lane, int cta, int ncta) {
   using Cfg = FwdCfg<D>;
@@ -543,8 +590,9 @@ __device__ __forceinline__ void fwd_softmax(const FwdParams& p, const FwdSmem<D>
   const float c2 = p.c2;
   int s_n = 0, o_n = 0;                     // s_full / o_done phases consumed (o_done: one per unit)
   bool ok = true;
-  for (int round = 0; ok; ++round) {
-    int u = fwd_unit_of(round, cta, ncta);
+  for (int n = 0; ok; ++n) {
+    const int u = DYN ? fwd_next_unit(sm, n, 23) : fwd_unit_of(n, cta, ncta);
+    if (u < 0) { ok = false; break; }
     if (u >= p.n_units) break;
     UnitInfo x = fwd_unit(p, u);
     const int nkv = x.nkv[t];
@@ -636,7 +684,7 @@ __device__ __forceinline__ void fwd_teardown(bool owner, uint32_t tmem_base, uin
   }
 }
 
-template <int D, bool BF16>
+template <int D, bool BF16, bool DYN>
 __global__ void __launch_bounds__(384, 1)
 attn_fwd_sm100(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                const __grid_constant__ CUtensorMap tm_v, const FwdParams p) {
@@ -657,6 +705,8 @@ attn_fwd_sm100(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
       mbar_init(&sm.p_part[t], 128);
     }
     mbar_init(sm.fin, 1);
+    // unit queue: the load warp posts, the MMA warp and the 8 softmax warps each release
+    for (int i = 0; i < kUnitQueue; ++i) { mbar_init(&sm.unit_full[i], 1); mbar_init(&sm.unit_empty[i], 9); }
     *sm.abort_flag = 0;
     fence_barrier_init();
   }
@@ -675,12 +725,12 @@ attn_fwd_sm100(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
   if (warp < 4) {
     // load / MMA warpgroup (warps 2 and 3 have no role) gives registers away
     regs_dec<Cfg::REGS_OTHER>();
-    if (warp == kWarpLoad) fwd_producer<D, BF16>(&tm_q, &tm_k, &tm_v, p, sm, lane, cta, ncta);
-    else if (warp == kWarpMma) fwd_mma<D, BF16>(p, sm, tmem_base, lane, cta, ncta);
+    if (warp == kWarpLoad) fwd_producer<D, BF16, DYN>(&tm_q, &tm_k, &tm_v, p, sm, lane, cta, ncta);
+    else if (warp == kWarpMma) fwd_mma<D, BF16, DYN>(p, sm, tmem_base, lane, cta, ncta);
     fwd_teardown(warp == kWarpMma, tmem_base, Cfg::TMEM_COLS);
   } else {
     regs_inc<Cfg::REGS_SOFTMAX>();
-    fwd_softmax<D, BF16>(p, sm, tmem_base, warp - 4, lane, cta, ncta);
+    fwd_softmax<D, BF16, DYN>(p, sm, tmem_base, warp - 4, lane, cta, ncta);
     fwd_teardown(false, tmem_base, Cfg::TMEM_COLS);
   }
 }

@@ -83,6 +83,13 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity,
   }
 }
 
+// One arrival for the whole warp (all 32 lanes execute it; elect.sync picks the lane).
+__device__ __forceinline__ void mbar_arrive_warp(uint64_t* bar) {
+  asm volatile(
+      "{\n .reg .pred e;\n .reg .b32 r;\n elect.sync r|e, 0xffffffff;\n"
+      " @e mbarrier.arrive.shared::cta.b64 _, [%0];\n}\n" ::"r"(smem_u32(bar)) : "memory");
+}
+
 // Bounded wait by every lane of a warp, with one answer for the whole warp.  Each poll
 // is a warp vote and every branch depends only on votes, so the warp never diverges:
 // an already-completed phase costs one poll and one vote (a per-lane early return

@@ -11,7 +11,10 @@
 #include <cstdarg>
 #include <cstdio>
 #include <cstring>
+#include <map>
 #include <mutex>
+#include <vector>
+#include <algorithm>
 #include <string>
 
 namespace {
@@ -114,6 +117,80 @@ int launch_fill(void* o, size_t n_o, float* lse, size_t n_lse, cudaStream_t st) 
   return e == cudaSuccess ? SA_OK : cuda_fail(e, "fill launch");
 }
 
+// Static-order imbalance of the forward kernel's unit list over ncta CTAs: the snake order
+// (fwd_unit_of) with each unit costing its K/V tiles plus two tiles of per-unit overhead,
+// max over CTAs / mean.  Mirrors fwd_unit (query block of a unit) and fwd_kv_tiles.
+double static_imbalance(const sa::FwdParams& p, int ncta) {
+  const int G = p.Hq / p.Hkv, n_bk = p.B * p.Hkv;
+  auto tiles = [&](int r0) -> int {
+    if (r0 >= p.Sq) return 0;
+    int kend = p.Sk;
+    if (p.causal) {
+      const int rmax = std::min(r0 + 127, p.Sq - 1);
+      kend = std::min(p.Sk, rmax + p.Sk - p.Sq + 1);
+    }
+    return kend > 0 ? (kend + 127) / 128 : 0;
+  };
+  std::vector<double> load(ncta, 0.0);
+  const long long per_band = (long long)p.band * p.B * p.Hq;
+  for (int u = 0; u < p.n_units; ++u) {
+    const long long bi = u / per_band;
+    const int bs = std::min<long long>(p.band, p.n_qblk - bi * p.band);
+    const long long r = u - bi * per_band;
+    const long long full_grp = (long long)p.kv_group * G * bs;
+    const long long g = r / full_grp;
+    const int gsize = (int)std::min<long long>(p.kv_group, n_bk - g * p.kv_group);
+    const long long rr = r - g * full_grp;
+    const int qb = p.n_qblk - 1 - (int)(bi * p.band + rr / ((long long)gsize * G));
+    const int cost = std::max(tiles(qb * 256), tiles(qb * 256 + 128)) + 2;
+    const int round = u / ncta, c = u % ncta;
+    load[(round & 1) ? ncta - 1 - c : c] += cost;
+  }
+  double mx = 0, sum = 0;
+  for (double l : load) { mx = std::max(mx, l); sum += l; }
+  return sum > 0 ? mx * ncta / sum : 1.0;
+}
+
+// Whether the forward kernel should take its units dynamically, decided once per shape.
+bool fwd_use_dynamic(const sa::FwdParams& p, int D, int ncta) {
+  static std::mutex mu;
+  static std::map<std::vector<long long>, bool> memo;
+  const std::vector<long long> key = {p.B, p.Sq, p.Sk, p.Hq, p.Hkv, D, p.causal, ncta};
+  std::lock_guard<std::mutex> lock(mu);
+  auto it = memo.find(key);
+  if (it != memo.end()) return it->second;
+  // many rounds balance on their own; counting them would only cost host time
+  const bool dyn = p.n_units <= 64 * ncta && static_imbalance(p, ncta) > 1.05;
+  if (memo.size() < 4096) memo[key] = dyn;
+  return dyn;
+}
+
+// Dynamic-scheduling counters of the forward kernel: kFwdWorkSlots pairs (next unit, CTAs
+// done), zero-initialised with the module; launches take slots in turn and the last CTA of
+// a launch zeroes its pair, so up to kFwdWorkSlots forward launches may be in flight at once
+// (on any streams) without sharing a counter.
+constexpr int kFwdWorkSlots = 64;
+static __device__ unsigned int g_fwd_work[2 * kFwdWorkSlots];
+
+int fwd_work_slot(unsigned int** out) {
+  static std::mutex mu;
+  static unsigned int* addr[64] = {nullptr};
+  static unsigned int next[64] = {0};
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+  if (dev < 0 || dev >= 64) return fail(SA_ERR_UNSUPPORTED, "device ordinal %d out of range", dev);
+  std::lock_guard<std::mutex> lock(mu);
+  if (!addr[dev]) {
+    void* p = nullptr;
+    e = cudaGetSymbolAddress(&p, g_fwd_work);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaGetSymbolAddress(forward work counters)");
+    addr[dev] = static_cast<unsigned int*>(p);
+  }
+  *out = addr[dev] + 2 * (next[dev]++ % kFwdWorkSlots);
+  return SA_OK;
+}
+
 template <int D, bool BF16>
 int launch_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Sq,
                int Sk, int Hq, int Hkv, int causal, float scale, cudaStream_t st) {
@@ -131,6 +208,7 @@ int launch_fwd(const void* q, const void* k, const void* v, void* o, float* lse,
   if (units > 0x7fffffffLL) return fail(SA_ERR_UNSUPPORTED, "too many work units (%lld)", units);
   p.n_units = (int)units;
   p.c2 = scale * kLog2e;
+  if ((rc = fwd_work_slot(&p.work)) != SA_OK) return rc;
   {
     // scheduling groups: (batch, KV head) pairs whose K + V fit in half the L2; among the
     // admissible sizes take the one whose band (ceil(grid / (kv_group * G)) query blocks)
@@ -154,7 +232,8 @@ int launch_fwd(const void* q, const void* k, const void* v, void* o, float* lse,
     p.kv_group = best_g;
     p.band = best_band < p.n_qblk ? best_band : p.n_qblk;
   }
-  auto kern = sa::attn_fwd_sm100<D, BF16>;
+  const int grid = p.n_units < num_sms() ? p.n_units : num_sms();
+  auto kern = fwd_use_dynamic(p, D, grid) ? sa::attn_fwd_sm100<D, BF16, true> : sa::attn_fwd_sm100<D, BF16, false>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::SMEM_TOTAL);
   if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(attn_fwd_sm100)");
   // the in-kernel register reallocation must fit in what the block is launched with,
@@ -165,7 +244,6 @@ int launch_fwd(const void* q, const void* k, const void* v, void* o, float* lse,
   if ((long long)fa.numRegs * Cfg::THREADS < 256LL * Cfg::REGS_SOFTMAX + 128LL * Cfg::REGS_OTHER)
     return fail(SA_ERR_UNSUPPORTED, "attn_fwd_sm100 launches with %d registers per thread, too few for "
                 "its register split", fa.numRegs);
-  int grid = p.n_units < num_sms() ? p.n_units : num_sms();
   kern<<<grid, Cfg::THREADS, Cfg::SMEM_TOTAL, st>>>(mq, mk, mv, p);
   e = cudaGetLastError();
   return e == cudaSuccess ? SA_OK : cuda_fail(e, "attn_fwd_sm100 launch");
