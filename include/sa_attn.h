@@ -126,6 +126,40 @@ int sa_attn_decode_noalloc(const void* q, const void* k, const void* v, void* o,
                            int num_splits, sa_stream_t stream);
 
 /*
+ * Single-token decode over a paged K/V cache, sequences of their own lengths: the paged
+ * layout of the Stem (AngelSlim sparse attention) page's serving backend (section 2: its
+ * prefill has "varlen" and "paged" paths) applied to the split-KV decode above; the
+ * flash-attn-volta page ("What's NOT here") lists variable-length sequences as missing.
+ * For sequence b the keys are tokens 0 .. seqlens[b]-1; token t lives in cache page
+ * block_table[b * max_blocks + t / page_size] at row t % page_size.  The result is the
+ * attention of q[b] over those keys, as sa_attn_decode computes it over a dense K/V.
+ *   q [B, Hq, D], o [B, Hq, D] (dtype); lse [B, Hq] fp32 or NULL.
+ *   k_cache, v_cache : [num_pages, page_size, Hkv, D] (dtype), 16-byte aligned.
+ *   block_table : [B, max_blocks] int32, device memory; entries for the tokens in use must
+ *                 be in [0, num_pages) (others are never read).
+ *   seqlens     : [B] int32, device memory; values are clamped to [0, page_size * max_blocks].
+ *                 A sequence of length 0 gives O = 0, LSE = -inf.
+ *   page_size   : a positive multiple of 64 (SA_ERR_UNSUPPORTED otherwise).
+ *   num_splits  : as for sa_attn_decode, planned for page_size * max_blocks tokens; a split
+ *                 covers at most 16384 tokens, so the longest sequence may hold up to
+ *                 192 * 16384 (D = 64) / 96 * 16384 (D = 128) tokens.
+ *   workspace   : at least sa_attn_decode_paged_workspace_size(...) bytes, rules as for
+ *                 sa_attn_decode.
+ * Errors as for sa_attn_decode, plus SA_ERR_INVALID for a null block_table or seqlens or
+ * non-positive max_blocks / num_pages.
+ */
+int sa_attn_decode_paged(const void* q, const void* k_cache, const void* v_cache,
+                         const int* block_table, const int* seqlens, void* o, float* lse,
+                         int B, int Hq, int Hkv, int D, int page_size, int max_blocks,
+                         int num_pages, float scale, int dtype, int num_splits,
+                         void* workspace, size_t workspace_bytes, sa_stream_t stream);
+
+/* Bytes of workspace sa_attn_decode_paged needs for these sizes and num_splits (0 for
+ * invalid sizes or B * Hq == 0). */
+size_t sa_attn_decode_paged_workspace_size(int B, int Hq, int Hkv, int D, int page_size,
+                                           int max_blocks, int num_splits);
+
+/*
  * Diagnostic only: the same forward as sa_attn_fwd computed by a plain CUDA-core kernel
  * (one thread per query row, fp32 online softmax).  Slow; used to cross-check the
  * tensor-core path.  Same arguments and conventions as sa_attn_fwd.

@@ -15,6 +15,9 @@
 //     into a ring of shared-memory stages; 4 warps each take 16 tokens of a stage;
 //   * S = Q K^T and O += P V on mma.sync.m16n8k16 (fp32 accumulate), fragments from
 //     ldmatrix; row max / sum by quad shuffles; the 4 warps merge through shared memory;
+//   * paged K/V caches (the `PAGED` instance): a split looks up the cache page of each of
+//     its 64-token stages in the block table once, and TMA reads (row in page, page)
+//     instead of (token, batch); sequences have their own lengths;
 //   * each split writes (unnormalised O, running max, two running sums) in fp32 to the
 //     workspace; a combine kernel with one CTA per (batch, query head) merges them.  It
 //     is launched with programmatic dependent launch, so its launch overlaps the split
@@ -37,7 +40,10 @@ struct DecCfg {
   static constexpr int SMEM_STAGES = STAGES * 2 * KV_BYTES;
   // write_partial's buffers; decode_merge uses the SMEM_STAGES region
   static constexpr int SMEM_MERGE = 4 * 16 * (D + 4) * 4 + 3 * 4 * 16 * 4;
-  static constexpr int SMEM_TOTAL = 1024 + (SMEM_STAGES > SMEM_MERGE ? SMEM_STAGES : SMEM_MERGE) + 256;
+  // paged K/V: the cache page of each stage of a split, looked up once at the start
+  static constexpr int MAX_PAGED_STAGES = 256;         // a split covers at most 16384 tokens
+  static constexpr int SMEM_TOTAL = 1024 + (SMEM_STAGES > SMEM_MERGE ? SMEM_STAGES : SMEM_MERGE) + 256 +
+                                    MAX_PAGED_STAGES * 4;
 };
 
 // Workspace layout (caller-owned scratch, contents irrelevant between calls):
@@ -51,6 +57,12 @@ struct DecParams {
   float* lse;          // [B, Hq] or null
   int B, Sk, Hq, Hkv, G, ngrp, nsplit, chunk;
   float c2;
+  // paged K/V (attn_decode_split<.., PAGED = true>): caches [num_pages, page_size, Hkv, D];
+  // the keys of sequence b are tokens 0 .. seqlens[b]-1, token t in page
+  // block_table[b * max_blocks + t / page_size] at row t % page_size
+  const int* block_table;   // [B, max_blocks]
+  const int* seqlens;       // [B]
+  int max_blocks, page_size;
 };
 
 __device__ __forceinline__ void ldsm_x4(uint32_t addr, uint32_t& r0, uint32_t& r1, uint32_t& r2, uint32_t& r3) {
@@ -167,7 +179,7 @@ struct DecMerge {
   static constexpr int MAX_SPLITS = (D == 64) ? 192 : 96;
 };
 
-template <int D, bool BF16>
+template <int D, bool BF16, bool PAGED>
 __global__ void __launch_bounds__(128, 3)
 attn_decode_split(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
                   const DecParams p) {
@@ -177,6 +189,7 @@ attn_decode_split(const __grid_constant__ CUtensorMap tm_k, const __grid_constan
   const int region = Cfg::SMEM_STAGES > Cfg::SMEM_MERGE ? Cfg::SMEM_STAGES : Cfg::SMEM_MERGE;
   uint64_t* full = (uint64_t*)(smem + region);
   volatile int* abort_flag = (volatile int*)(full + Cfg::STAGES);
+  int* s_page = (int*)(smem + region + 256);            // PAGED: cache page of each stage
 
   // let the combine grid launch now (it waits for this grid's results before reading)
   asm volatile("griddepcontrol.launch_dependents;");
@@ -186,10 +199,21 @@ attn_decode_split(const __grid_constant__ CUtensorMap tm_k, const __grid_constan
   const int b = blockIdx.z;
   const int h0 = kvh * p.G + grp * 16;                  // first query head of this tile
   const int nrows = min(16, p.G - grp * 16);            // valid rows of the tile
+  // keys of this sequence: Sk, or (paged) its own length, clamped to what its block table holds
+  const int seqlen = PAGED ? max(0, min(__ldg(p.seqlens + b), p.max_blocks * p.page_size)) : p.Sk;
   const int tok0 = split * p.chunk;
-  const int tok1 = min(p.Sk, tok0 + p.chunk);
-  const int nstage = (tok1 - tok0 + Cfg::TOK - 1) / Cfg::TOK;
+  const int tok1 = min(seqlen, tok0 + p.chunk);
+  const int nstage = tok1 > tok0 ? (tok1 - tok0 + Cfg::TOK - 1) / Cfg::TOK : 0;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (PAGED) {
+    // a 64-token stage never crosses a page (pages are multiples of 64 tokens, stages start
+    // on multiples of 64); the host keeps nstage <= MAX_PAGED_STAGES
+    const int* bt = p.block_table + (size_t)b * p.max_blocks;
+    for (int i = threadIdx.x; i < nstage; i += blockDim.x) s_page[i] = __ldg(bt + (tok0 + i * Cfg::TOK) / p.page_size);
+  }
+  // TMA coordinates (token row, batch or page) of stage st
+  auto stage_row = [&](int st) { const int t = tok0 + st * Cfg::TOK; return PAGED ? t % p.page_size : t; };
+  auto stage_outer = [&](int st) { return PAGED ? s_page[st] : b; };
 
   if (threadIdx.x == 0) {
     for (int i = 0; i < Cfg::STAGES; ++i) mbar_init(&full[i], 1);
@@ -203,8 +227,8 @@ attn_decode_split(const __grid_constant__ CUtensorMap tm_k, const __grid_constan
       uint8_t* dk = smem + s * 2 * Cfg::KV_BYTES;
       mbar_arrive_expect_tx(&full[s], 2 * Cfg::KV_BYTES);
       for (int c = 0; c < Cfg::KCH; ++c) {
-        tma_load_4d(dk + c * Cfg::CHUNK_BYTES, &tm_k, &full[s], c * 64, kvh, tok0 + s * Cfg::TOK, b);
-        tma_load_4d(dk + Cfg::KV_BYTES + c * Cfg::CHUNK_BYTES, &tm_v, &full[s], c * 64, kvh, tok0 + s * Cfg::TOK, b);
+        tma_load_4d(dk + c * Cfg::CHUNK_BYTES, &tm_k, &full[s], c * 64, kvh, stage_row(s), stage_outer(s));
+        tma_load_4d(dk + Cfg::KV_BYTES + c * Cfg::CHUNK_BYTES, &tm_v, &full[s], c * 64, kvh, stage_row(s), stage_outer(s));
       }
     }
   }
@@ -318,8 +342,8 @@ attn_decode_split(const __grid_constant__ CUtensorMap tm_k, const __grid_constan
       uint8_t* dk = smem + slot * 2 * Cfg::KV_BYTES;
       mbar_arrive_expect_tx(&full[slot], 2 * Cfg::KV_BYTES);
       for (int c = 0; c < Cfg::KCH; ++c) {
-        tma_load_4d(dk + c * Cfg::CHUNK_BYTES, &tm_k, &full[slot], c * 64, kvh, tok0 + ns * Cfg::TOK, b);
-        tma_load_4d(dk + Cfg::KV_BYTES + c * Cfg::CHUNK_BYTES, &tm_v, &full[slot], c * 64, kvh, tok0 + ns * Cfg::TOK, b);
+        tma_load_4d(dk + c * Cfg::CHUNK_BYTES, &tm_k, &full[slot], c * 64, kvh, stage_row(ns), stage_outer(ns));
+        tma_load_4d(dk + Cfg::KV_BYTES + c * Cfg::CHUNK_BYTES, &tm_v, &full[slot], c * 64, kvh, stage_row(ns), stage_outer(ns));
       }
     }
   }

@@ -268,7 +268,9 @@ struct DecPlan {
   int nsplit, chunk, ngrp;
 };
 
-DecPlan plan_decode(int B, int Sk, int Hq, int Hkv, int D, int num_splits, int sms) {
+// max_chunk: the most tokens one split may take (paged decode: its stage table's size).
+DecPlan plan_decode(int B, int Sk, int Hq, int Hkv, int D, int num_splits, int sms,
+                    int max_chunk = 0x7fffffff) {
   DecPlan pl;
   const int G = Hq / Hkv;
   pl.ngrp = (G + 15) / 16;
@@ -281,20 +283,34 @@ DecPlan plan_decode(int B, int Sk, int Hq, int Hkv, int D, int num_splits, int s
   if (want > max_split) want = max_split;
   int chunk = (int)((Sk + want - 1) / want);
   chunk = (chunk + 63) / 64 * 64;
+  if (chunk > max_chunk) chunk = max_chunk;     // more splits than the cap above: caller checks
   pl.chunk = chunk;
   pl.nsplit = (Sk + chunk - 1) / chunk;
   return pl;
 }
 
-template <int D, bool BF16>
+// Paged K/V caches for launch_decode: [num_pages, page_size, Hkv, D], block table
+// [B, max_blocks], sequence lengths [B] (all device memory).
+struct DecPaged {
+  const int* block_table = nullptr;
+  const int* seqlens = nullptr;
+  int max_blocks = 0, page_size = 0, num_pages = 0;
+};
+
+template <int D, bool BF16, bool PAGED>
 int launch_decode(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Sk,
-                  int Hq, int Hkv, float scale, const DecPlan& pl, void* ws, cudaStream_t st) {
+                  int Hq, int Hkv, float scale, const DecPlan& pl, void* ws, cudaStream_t st,
+                  const DecPaged& pg = DecPaged()) {
   using Cfg = sa::DecCfg<D>;
   CUtensorMap mk, mv;
   int rc;
-  if ((rc = make_map(&mk, k, BF16, D, Hkv, Sk, B, 64)) != SA_OK) return rc;
-  if ((rc = make_map(&mv, v, BF16, D, Hkv, Sk, B, 64)) != SA_OK) return rc;
+  // TMA views: (D, Hkv, token, batch), or for a paged cache (D, Hkv, row in page, page)
+  const int rows = PAGED ? pg.page_size : Sk, outer = PAGED ? pg.num_pages : B;
+  if ((rc = make_map(&mk, k, BF16, D, Hkv, rows, outer, 64)) != SA_OK) return rc;
+  if ((rc = make_map(&mv, v, BF16, D, Hkv, rows, outer, 64)) != SA_OK) return rc;
   sa::DecParams p;
+  p.block_table = pg.block_table; p.seqlens = pg.seqlens;
+  p.max_blocks = pg.max_blocks; p.page_size = pg.page_size;
   p.q = q;
   p.ws_ml = reinterpret_cast<float*>(ws);
   p.ws_o = p.ws_ml + (size_t)B * Hq * pl.nsplit * 4;
@@ -305,7 +321,7 @@ int launch_decode(const void* q, const void* k, const void* v, void* o, float* l
   dim3 grid(pl.nsplit, Hkv * pl.ngrp, B);
   if ((long long)B * Hq > 0x7fffffffLL || grid.y > 65535 || grid.z > 65535)
     return fail(SA_ERR_UNSUPPORTED, "decode grid too large");
-  auto ks = sa::attn_decode_split<D, BF16>;
+  auto ks = sa::attn_decode_split<D, BF16, PAGED>;
   cudaError_t e = cudaFuncSetAttribute(ks, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::SMEM_TOTAL);
   if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(attn_decode_split)");
   ks<<<grid, 128, Cfg::SMEM_TOTAL, st>>>(mk, mv, p);
@@ -420,10 +436,10 @@ int sa_attn_decode(const void* q, const void* k, const void* v, void* o, float* 
                 workspace ? workspace_bytes : (size_t)0);
   if (!aligned16(workspace)) return fail(SA_ERR_INVALID, "workspace must be 16-byte aligned");
   const bool bf = dtype == SA_BF16;
-  if (D == 64) return bf ? launch_decode<64, true>(q, k, v, o, lse, B, Sk, Hq, Hkv, scale, pl, workspace, st)
-                         : launch_decode<64, false>(q, k, v, o, lse, B, Sk, Hq, Hkv, scale, pl, workspace, st);
-  return bf ? launch_decode<128, true>(q, k, v, o, lse, B, Sk, Hq, Hkv, scale, pl, workspace, st)
-            : launch_decode<128, false>(q, k, v, o, lse, B, Sk, Hq, Hkv, scale, pl, workspace, st);
+  if (D == 64) return bf ? launch_decode<64, true, false>(q, k, v, o, lse, B, Sk, Hq, Hkv, scale, pl, workspace, st)
+                         : launch_decode<64, false, false>(q, k, v, o, lse, B, Sk, Hq, Hkv, scale, pl, workspace, st);
+  return bf ? launch_decode<128, true, false>(q, k, v, o, lse, B, Sk, Hq, Hkv, scale, pl, workspace, st)
+            : launch_decode<128, false, false>(q, k, v, o, lse, B, Sk, Hq, Hkv, scale, pl, workspace, st);
 }
 
 int sa_attn_decode_noalloc(const void* q, const void* k, const void* v, void* o, float* lse, int B,
@@ -444,10 +460,75 @@ int sa_attn_decode_noalloc(const void* q, const void* k, const void* v, void* o,
   void* scratch = nullptr;
   if ((rc = noalloc_scratch(&scratch)) != SA_OK) return rc;
   const bool bf = dtype == SA_BF16;
-  if (D == 64) return bf ? launch_decode<64, true>(q, k, v, o, lse, B, Sk, Hq, Hkv, scale, pl, scratch, st)
-                         : launch_decode<64, false>(q, k, v, o, lse, B, Sk, Hq, Hkv, scale, pl, scratch, st);
-  return bf ? launch_decode<128, true>(q, k, v, o, lse, B, Sk, Hq, Hkv, scale, pl, scratch, st)
-            : launch_decode<128, false>(q, k, v, o, lse, B, Sk, Hq, Hkv, scale, pl, scratch, st);
+  if (D == 64) return bf ? launch_decode<64, true, false>(q, k, v, o, lse, B, Sk, Hq, Hkv, scale, pl, scratch, st)
+                         : launch_decode<64, false, false>(q, k, v, o, lse, B, Sk, Hq, Hkv, scale, pl, scratch, st);
+  return bf ? launch_decode<128, true, false>(q, k, v, o, lse, B, Sk, Hq, Hkv, scale, pl, scratch, st)
+            : launch_decode<128, false, false>(q, k, v, o, lse, B, Sk, Hq, Hkv, scale, pl, scratch, st);
+}
+
+// Checks and plan shared by the paged-decode entry points.  Returns SA_OK and fills
+// *max_seqlen and *pl, or an error code.
+static int paged_plan(int B, int Hq, int Hkv, int D, int dtype, float scale, int page_size, int max_blocks,
+                      int num_pages, int num_splits, int* max_seqlen, DecPlan* pl) {
+  int rc = check_dims(B, 1, 0, Hq, Hkv, D, dtype, scale);
+  if (rc != SA_OK) return rc;
+  if (num_splits < 0) return fail(SA_ERR_INVALID, "num_splits must be >= 0");
+  if (page_size <= 0 || page_size % 64 != 0)
+    return fail(SA_ERR_UNSUPPORTED, "page_size must be a positive multiple of 64 (got %d)", page_size);
+  if (max_blocks <= 0 || num_pages <= 0)
+    return fail(SA_ERR_INVALID, "max_blocks (%d) and num_pages (%d) must be positive", max_blocks, num_pages);
+  const long long msl = (long long)page_size * max_blocks;
+  if (msl > 0x7fffffffLL) return fail(SA_ERR_UNSUPPORTED, "page_size * max_blocks too large");
+  *max_seqlen = (int)msl;
+  pl->nsplit = pl->chunk = pl->ngrp = 0;
+  if (B == 0 || Hq == 0) return SA_OK;                       // nothing to plan
+  // one split's stage table holds MAX_PAGED_STAGES 64-token stages
+  constexpr int max_chunk = sa::DecCfg<64>::MAX_PAGED_STAGES * 64;
+  *pl = plan_decode(B, *max_seqlen, Hq, Hkv, D, num_splits, num_sms(), max_chunk);
+  const int cap = D == 64 ? sa::DecMerge<64>::MAX_SPLITS : sa::DecMerge<128>::MAX_SPLITS;
+  if (pl->nsplit > cap)
+    return fail(SA_ERR_UNSUPPORTED, "paged decode of up to %d tokens needs %d splits (at most %d)", *max_seqlen,
+                pl->nsplit, cap);
+  return SA_OK;
+}
+
+size_t sa_attn_decode_paged_workspace_size(int B, int Hq, int Hkv, int D, int page_size, int max_blocks,
+                                           int num_splits) {
+  int msl = 0;
+  DecPlan pl;
+  if (B <= 0 || Hq <= 0) return 0;
+  if (paged_plan(B, Hq, Hkv, D, SA_FP16, 1.f, page_size, max_blocks, 1, num_splits, &msl, &pl) != SA_OK) return 0;
+  return dec_ws_bytes(B, Hq, pl.nsplit, D);
+}
+
+int sa_attn_decode_paged(const void* q, const void* k_cache, const void* v_cache, const int* block_table,
+                         const int* seqlens, void* o, float* lse, int B, int Hq, int Hkv, int D, int page_size,
+                         int max_blocks, int num_pages, float scale, int dtype, int num_splits, void* workspace,
+                         size_t workspace_bytes, sa_stream_t stream) {
+  int msl = 0;
+  DecPlan pl;
+  int rc = paged_plan(B, Hq, Hkv, D, dtype, scale, page_size, max_blocks, num_pages, num_splits, &msl, &pl);
+  if (rc != SA_OK) return rc;
+  if (B == 0 || Hq == 0) return SA_OK;                       // (after the argument checks)
+  if ((rc = check_ptrs(q, k_cache, v_cache, o, lse)) != SA_OK) return rc;
+  if (!block_table || !seqlens) return fail(SA_ERR_INVALID, "block_table and seqlens must be non-null");
+  if ((long long)num_pages * page_size * Hkv * D > (1LL << 40))
+    return fail(SA_ERR_UNSUPPORTED, "K/V cache too large");
+  const size_t need = dec_ws_bytes(B, Hq, pl.nsplit, D);
+  if (!workspace || workspace_bytes < need)
+    return fail(SA_ERR_WORKSPACE, "decode workspace of %zu bytes needed (got %zu)", need,
+                workspace ? workspace_bytes : (size_t)0);
+  if (!aligned16(workspace)) return fail(SA_ERR_INVALID, "workspace must be 16-byte aligned");
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  DecPaged pg;
+  pg.block_table = block_table; pg.seqlens = seqlens;
+  pg.max_blocks = max_blocks; pg.page_size = page_size; pg.num_pages = num_pages;
+  const bool bf = dtype == SA_BF16;
+  if (D == 64)
+    return bf ? launch_decode<64, true, true>(q, k_cache, v_cache, o, lse, B, msl, Hq, Hkv, scale, pl, workspace, st, pg)
+              : launch_decode<64, false, true>(q, k_cache, v_cache, o, lse, B, msl, Hq, Hkv, scale, pl, workspace, st, pg);
+  return bf ? launch_decode<128, true, true>(q, k_cache, v_cache, o, lse, B, msl, Hq, Hkv, scale, pl, workspace, st, pg)
+            : launch_decode<128, false, true>(q, k_cache, v_cache, o, lse, B, msl, Hq, Hkv, scale, pl, workspace, st, pg);
 }
 
 const char* sa_last_error(void) { return g_err.c_str(); }

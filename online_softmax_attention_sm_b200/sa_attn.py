@@ -28,6 +28,8 @@ SIGNATURES = {
     "sa_attn_decode_num_splits": (_I, [_I, _I, _I, _I, _I]),
     "sa_attn_decode": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _F, _I, _I, _P, _Z, _P]),
     "sa_attn_decode_noalloc": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _F, _I, _I, _P]),
+    "sa_attn_decode_paged": (_I, [_P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _F, _I, _I, _P, _Z, _P]),
+    "sa_attn_decode_paged_workspace_size": (_Z, [_I, _I, _I, _I, _I, _I, _I]),
     "sa_last_error": (ctypes.c_char_p, []),
     "sa_check_status": (_I, [_P]),
     "sa_version": (ctypes.c_char_p, []),
@@ -146,6 +148,46 @@ def sa_attn_decode(q, k, v, scale=None, num_splits=0, workspace=None, out=None, 
     _check(lib().sa_attn_decode(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse), B, Sk, Hq, Hkv, D,
                                 float(scale), _DT[q.dtype], int(num_splits), _ptr(workspace),
                                 workspace.numel() * workspace.element_size(), _stream(stream)))
+    return out, lse
+
+
+def sa_attn_decode_paged_workspace_size(B, Hq, Hkv, D, page_size, max_blocks, num_splits=0):
+    return int(lib().sa_attn_decode_paged_workspace_size(B, Hq, Hkv, D, page_size, max_blocks, num_splits))
+
+
+def sa_attn_decode_paged(q, k_cache, v_cache, block_table, seqlens, scale=None, num_splits=0,
+                         workspace=None, out=None, lse=None, return_lse=True, stream=None):
+    """Decode over a paged K/V cache.  q [B,Hq,D]; k_cache/v_cache [num_pages, page_size, Hkv, D];
+    block_table [B, max_blocks] int32; seqlens [B] int32 (all CUDA, contiguous).
+    Returns (o [B,Hq,D], lse [B,Hq])."""
+    B, Hq, D = q.shape
+    num_pages, page_size, Hkv = k_cache.shape[0], k_cache.shape[1], k_cache.shape[2]
+    if k_cache.shape != (num_pages, page_size, Hkv, D) or v_cache.shape != k_cache.shape:
+        raise ValueError(f"shape mismatch q{tuple(q.shape)} k{tuple(k_cache.shape)} v{tuple(v_cache.shape)}")
+    if q.dtype not in _DT:
+        raise TypeError(f"unsupported dtype {q.dtype}")
+    for n, t in (("q", q), ("k_cache", k_cache), ("v_cache", v_cache)):
+        _check_tensor(n, t, q.dtype, q.device)
+    if block_table.dim() != 2 or block_table.shape[0] != B:
+        raise ValueError(f"block_table must be [B, max_blocks], got {tuple(block_table.shape)}")
+    _check_tensor("block_table", block_table, torch.int32, q.device)
+    _check_tensor("seqlens", seqlens, torch.int32, q.device)
+    if seqlens.shape != (B,):
+        raise ValueError(f"seqlens must be [B], got {tuple(seqlens.shape)}")
+    max_blocks = block_table.shape[1]
+    if scale is None:
+        scale = 1.0 / math.sqrt(D)
+    if out is None:
+        out = torch.empty_like(q)
+    if return_lse and lse is None:
+        lse = torch.empty((B, Hq), dtype=torch.float32, device=q.device)
+    need = sa_attn_decode_paged_workspace_size(B, Hq, Hkv, D, page_size, max_blocks, num_splits)
+    if workspace is None:
+        workspace = torch.empty(max(need, 16), dtype=torch.uint8, device=q.device)
+    _check(lib().sa_attn_decode_paged(_ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(block_table), _ptr(seqlens),
+                                      _ptr(out), _ptr(lse), B, Hq, Hkv, D, page_size, max_blocks, num_pages,
+                                      float(scale), _DT[q.dtype], int(num_splits), _ptr(workspace),
+                                      workspace.numel() * workspace.element_size(), _stream(stream)))
     return out, lse
 
 

@@ -7,6 +7,7 @@ It shares no code with the CUDA path.  Every function here is pinned by
 "parity unpinned".
 """
 from .attention import (attention, attention_rows, attention_blockwise, decode,
-                        combine_lse)
+                        decode_paged, combine_lse)
 
-__all__ = ["attention", "attention_rows", "attention_blockwise", "decode", "combine_lse"]
+__all__ = ["attention", "attention_rows", "attention_blockwise", "decode", "decode_paged",
+           "combine_lse"]

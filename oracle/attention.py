@@ -111,6 +111,34 @@ def decode(q, k, v, scale):
     return O[:, 0], LSE[:, :, 0]
 
 
+def decode_paged(q, k_cache, v_cache, block_table, seqlens, scale):
+    """Single-token decode over a paged K/V cache (the Stem / AngelSlim page, section 2:
+    the serving backend's "paged" path; the flash-attn-volta page lists variable-length
+    sequences among what it lacks).  q [B,Hq,D]; k_cache/v_cache [num_pages, page_size,
+    Hkv, D]; block_table [B, max_blocks]; seqlens [B].  Sequence b's keys are tokens
+    0 .. seqlens[b]-1, token t stored in page block_table[b, t // page_size] at row
+    t % page_size; the result is :func:`decode` of q[b] over exactly those keys (a length
+    of 0 gives O = 0, LSE = -inf).  Lengths are clamped to [0, page_size * max_blocks].
+    Returns O [B,Hq,D] and LSE [B,Hq]."""
+    q = _f64(q)
+    B, Hq, D = q.shape
+    page_size = k_cache.shape[1]
+    bt = np.asarray(block_table)
+    O = np.zeros((B, Hq, D))
+    LSE = np.full((B, Hq), NEG_INF)
+    for b in range(B):
+        n = int(min(max(int(seqlens[b]), 0), page_size * bt.shape[1]))
+        if n == 0:
+            continue
+        t = np.arange(n)
+        pages = bt[b, t // page_size]
+        kb = _f64(k_cache)[pages, t % page_size]          # [n, Hkv, D] in token order
+        vb = _f64(v_cache)[pages, t % page_size]
+        o, lse = decode(q[b:b + 1], kb[None], vb[None], scale)
+        O[b], LSE[b] = o[0], lse[0]
+    return O, LSE
+
+
 def attention_blockwise(q, k, v, scale, causal=False, block=64):
     """The online-softmax recurrence, restated in float64 (TurboQuant page,
     ``online_softmax_attention``; StreamAttention page, "Kernel Design"): walk the

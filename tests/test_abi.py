@@ -127,6 +127,47 @@ def test_workspace_size(L):
     assert L.sa_attn_decode_num_splits(4, 32768, 14, 2, 64) >= 1
 
 
+def dec_paged(L, q=FAKE, kc=FAKE, vc=FAKE, bt=FAKE, sl=FAKE, o=FAKE, lse=NULL, B=1, Hq=2, Hkv=1, D=64,
+              page=64, mb=4, npg=8, scale=0.125, dtype=0, ns=0, ws=FAKE, wsb=1 << 30):
+    return L.sa_attn_decode_paged(q, kc, vc, bt, sl, o, lse, B, Hq, Hkv, D, page, mb, npg, scale, dtype, ns,
+                                  ws, wsb, None)
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(q=NULL), sa.SA_ERR_INVALID),
+    (dict(bt=NULL), sa.SA_ERR_INVALID),
+    (dict(sl=NULL), sa.SA_ERR_INVALID),
+    (dict(Hq=3, Hkv=2), sa.SA_ERR_INVALID),
+    (dict(D=96), sa.SA_ERR_UNSUPPORTED),
+    (dict(page=32), sa.SA_ERR_UNSUPPORTED),
+    (dict(page=100), sa.SA_ERR_UNSUPPORTED),
+    (dict(mb=0), sa.SA_ERR_INVALID),
+    (dict(npg=0), sa.SA_ERR_INVALID),
+    (dict(ns=-2), sa.SA_ERR_INVALID),
+    (dict(ws=NULL), sa.SA_ERR_WORKSPACE),
+    (dict(wsb=16), sa.SA_ERR_WORKSPACE),
+    # 192 splits of at most 16384 tokens hold 3145728 tokens (D = 64)
+    (dict(page=64, mb=3145728 // 64 + 1), sa.SA_ERR_UNSUPPORTED),
+])
+def test_paged_decode_rejects_invalid_arguments(L, kw, code):
+    assert dec_paged(L, **kw) == code
+
+
+def test_paged_decode_empty_is_a_no_op(L):
+    assert dec_paged(L, q=NULL, kc=NULL, vc=NULL, bt=NULL, sl=NULL, o=NULL, B=0) == sa.SA_OK
+
+
+def test_paged_workspace_size(L):
+    # planned for page_size * max_blocks tokens, like the dense decode of that length ...
+    assert (L.sa_attn_decode_paged_workspace_size(4, 14, 2, 64, 64, 512, 0)
+            == L.sa_attn_decode_workspace_size(4, 32768, 14, 2, 64, 0))
+    assert L.sa_attn_decode_paged_workspace_size(2, 8, 8, 128, 128, 10, 3) == 2 * 8 * 3 * 132 * 4
+    # ... but a split takes at most 16384 tokens: one requested split becomes two
+    assert L.sa_attn_decode_paged_workspace_size(1, 2, 1, 64, 64, 512, 1) == 1 * 2 * 2 * 68 * 4
+    assert L.sa_attn_decode_paged_workspace_size(1, 2, 1, 64, 32, 512, 1) == 0      # bad page size
+    assert L.sa_attn_decode_paged_workspace_size(0, 2, 1, 64, 64, 512, 1) == 0      # empty
+
+
 def test_version(L):
     assert re.fullmatch(r"\d+\.\d+\.\d+", sa.sa_version())
 

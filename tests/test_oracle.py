@@ -11,7 +11,7 @@ import os
 import numpy as np
 import pytest
 
-from oracle import attention, attention_rows, attention_blockwise, decode, combine_lse
+from oracle import attention, attention_rows, attention_blockwise, decode, decode_paged, combine_lse
 
 GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
 TOL = 1e-12
@@ -260,3 +260,60 @@ def test_large_scores_stay_finite():
     O, L = attention(q, k, v, 1.0, True)
     assert np.all(np.isfinite(O)) and np.all(np.isfinite(L))
     assert np.all(np.abs(O) <= np.abs(v).max() + 1e-9)
+
+
+# ---- paged decode: a gather by the block table, then the plain decode
+
+def paged_from_dense(k, v, page_size, perm_seed=None):
+    """Cut dense [B,Sk,Hkv,D] K/V into pages of page_size rows (Sk a multiple), optionally
+    shuffle the pages in the cache, and return (k_cache, v_cache, block_table)."""
+    B, Sk, Hkv, D = k.shape
+    nb = Sk // page_size
+    kc = k.reshape(B * nb, page_size, Hkv, D)
+    vc = v.reshape(B * nb, page_size, Hkv, D)
+    table = np.arange(B * nb).reshape(B, nb)
+    if perm_seed is not None:
+        perm = np.random.default_rng(perm_seed).permutation(B * nb)   # page i moves to slot perm[i]
+        kc2, vc2 = np.empty_like(kc), np.empty_like(vc)
+        kc2[perm], vc2[perm] = kc, vc
+        kc, vc, table = kc2, vc2, perm[table]
+    return kc, vc, table
+
+
+def test_paged_decode_identity_layout_is_dense_decode():
+    q, k, v = qkv(B=3, Sq=1, Sk=12, Hq=4, Hkv=2)
+    kc, vc, table = paged_from_dense(k, v, 4)
+    O, L = decode_paged(q[:, 0], kc, vc, table, np.full(3, 12), 0.5)
+    Od, Ld = decode(q[:, 0], k, v, 0.5)
+    np.testing.assert_allclose(O, Od, atol=TOL)
+    np.testing.assert_allclose(L, Ld, atol=TOL)
+
+
+def test_paged_decode_ignores_where_pages_sit():
+    q, k, v = qkv(B=2, Sq=1, Sk=16, Hq=6, Hkv=3, seed=5)
+    kc, vc, table = paged_from_dense(k, v, 4, perm_seed=11)
+    O, L = decode_paged(q[:, 0], kc, vc, table, np.array([16, 16]), 0.7)
+    Od, Ld = decode(q[:, 0], k, v, 0.7)
+    np.testing.assert_allclose(O, Od, atol=TOL)
+    np.testing.assert_allclose(L, Ld, atol=TOL)
+
+
+def test_paged_decode_lengths_truncate_and_empty():
+    q, k, v = qkv(B=4, Sq=1, Sk=12, Hq=2, Hkv=1, seed=9)
+    kc, vc, table = paged_from_dense(k, v, 4, perm_seed=3)
+    lens = np.array([12, 5, 0, 1])
+    O, L = decode_paged(q[:, 0], kc, vc, table, lens, 0.5)
+    for b, n in enumerate(lens):
+        if n == 0:
+            assert np.all(O[b] == 0) and np.all(np.isneginf(L[b]))
+            continue
+        Od, Ld = decode(q[b:b + 1, 0], k[b:b + 1, :n], v[b:b + 1, :n], 0.5)
+        np.testing.assert_allclose(O[b], Od[0], atol=TOL)
+        np.testing.assert_allclose(L[b], Ld[0], atol=TOL)
+    # one visible key: the output is that key's V row, the LSE its score
+    np.testing.assert_allclose(O[3], v[3, 0, [0, 0]], atol=TOL)
+    np.testing.assert_allclose(L[3], 0.5 * (q[3, 0] @ k[3, 0, 0]), atol=TOL)
+    # lengths beyond the table are clamped to it
+    O2, L2 = decode_paged(q[:, 0], kc, vc, table, np.array([99, 5, -3, 1]), 0.5)
+    np.testing.assert_allclose(O2[0], O[0], atol=TOL)
+    assert np.all(O2[2] == 0) and np.all(np.isneginf(L2[2]))
