@@ -212,8 +212,9 @@ def main():
     import numpy as np
     import torch
     import torch.distributed as dist
-    from online_softmax_attention_sm_b200 import (sa_attn_decode, sa_attn_decode_workspace_size,
-                                                   sa_attn_fwd, sa_check_status)
+    from online_softmax_attention_sm_b200 import (sa_attn_decode, sa_attn_decode_paged,
+                                                   sa_attn_decode_paged_workspace_size,
+                                                   sa_attn_decode_workspace_size, sa_attn_fwd, sa_check_status)
     from online_softmax_attention_sm_b200.dist import aggregate_throughput, max_over_ranks, rank_seed
     from online_softmax_attention_sm_b200.inputs import make_workload_inputs
     from online_softmax_attention_sm_b200.workloads import WORKLOADS
@@ -295,6 +296,36 @@ def main():
             cold.append((e0, e1))
     torch.cuda.synchronize(dev)
     cold_ms = [a.elapsed_time(b) for a, b in cold] or [float("nan")]
+
+    # the same decode over a paged cache: the K/V cut into 64-token pages, the pages
+    # shuffled (a fixed permutation), every sequence at full length; same cold-L2 protocol
+    paged_ms = [float("nan")]
+    if run_dec:
+        ps = 64
+        nb = wd.Sk // ps
+        perm = torch.randperm(wd.B * nb, generator=torch.Generator().manual_seed(wd.seed)).to(dev)
+        kc = torch.empty((wd.B * nb, ps, wd.Hkv, wd.D), dtype=dk.dtype, device=dev)
+        vc = torch.empty_like(kc)
+        kc[perm] = dk.reshape(wd.B * nb, ps, wd.Hkv, wd.D)
+        vc[perm] = dv.reshape(wd.B * nb, ps, wd.Hkv, wd.D)
+        table = perm.view(wd.B, nb).to(torch.int32)
+        seqlens = torch.full((wd.B,), wd.Sk, dtype=torch.int32, device=dev)
+        pws = torch.empty(max(16, sa_attn_decode_paged_workspace_size(wd.B, wd.Hq, wd.Hkv, wd.D, ps, nb)),
+                          dtype=torch.uint8, device=dev)
+        pev = []
+        for i in range(args.warmup + args.steps):
+            scrub.sum()
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            sa_attn_decode_paged(dq, kc, vc, table, seqlens, scale=wd.scale, workspace=pws, out=do, lse=dlse,
+                                 stream=stream)
+            e1.record(stream)
+            if i >= args.warmup:
+                pev.append((e0, e1))
+        torch.cuda.synchronize(dev)
+        sa_check_status(stream)
+        paged_ms = [a.elapsed_time(b) for a, b in pev]
+        del kc, vc
     del scrub
 
     # e2e through the public API with host buffers: H2D of the step's inputs, D2H of outputs
@@ -329,6 +360,7 @@ def main():
     pre_avg = max_over_ranks(sum(pre_ms) / len(pre_ms), dev)
     dec_avg = max_over_ranks(sum(dec_ms) / len(dec_ms), dev)
     cold_avg = max_over_ranks(sum(cold_ms) / len(cold_ms), dev)
+    paged_avg = max_over_ranks(sum(paged_ms) / len(paged_ms), dev)
     e2e_ms = max_over_ranks(e2e_ms, dev) if e2e_ms is not None else None
 
     if rank == 0:
@@ -339,7 +371,7 @@ def main():
         # (cuBLAS timed alone) is the comparable -- and the stricter -- denominator
         peak = peaks["bf16_tflops"]
         dec_gbs_cold = wd.kv_bytes / (cold_avg * 1e-3) / 1e9
-        dec_gbs_step = wd.kv_bytes / (dec_avg * 1e-3) / 1e9
+        dec_gbs_step = wd.kv_bytes / (dec_avg * 1e-3) / 1e9 if run_dec else float("nan")
         traffic = None
         prof = os.path.join(ROOT, "profiles", "traffic.json")
         if os.path.exists(prof) and not args.prefill_seq:
@@ -365,7 +397,12 @@ def main():
                          "traffic": traffic},
             "decode": {"value": dec_gbs_cold, "unit": "GB/s", "bound": "hbm", "peak": peaks["hbm_gbs"],
                        "frac": dec_gbs_cold / peaks["hbm_gbs"], "us": cold_avg * 1e3, "l2": "cold (4xL2 read scrub)",
-                       "in_step_gbs": dec_gbs_step, "kernels": "attn_decode_split + attn_decode_combine (PDL)"},
+                       "in_step_gbs": dec_gbs_step, "kernels": "attn_decode_split + attn_decode_combine (PDL)",
+                       "paged": {"value": wd.kv_bytes / (paged_avg * 1e-3) / 1e9, "unit": "GB/s",
+                                 "frac": wd.kv_bytes / (paged_avg * 1e-3) / 1e9 / peaks["hbm_gbs"],
+                                 "us": paged_avg * 1e3, "page_size": 64,
+                                 "layout": "the same K/V in shuffled 64-token pages, full-length sequences",
+                                 "l2": "cold (4xL2 read scrub)"}},
             "prefill_ms": pre_avg,
             "gpu_launches": (int(run_pre) + 2 * int(run_dec)) * args.steps,
             "clocks": clk.summary(),
