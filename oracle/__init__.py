@@ -6,8 +6,8 @@ It shares no code with the CUDA path.  Every function here is pinned by
 ``tests/test_oracle.py`` to closed forms, invariants and brute force; none is
 "parity unpinned".
 """
-from .attention import (attention, attention_rows, attention_blockwise, decode,
-                        decode_paged, combine_lse)
+from .attention import (attention, attention_rows, attention_blockwise, attention_varlen,
+                        decode, decode_paged, combine_lse)
 
-__all__ = ["attention", "attention_rows", "attention_blockwise", "decode", "decode_paged",
-           "combine_lse"]
+__all__ = ["attention", "attention_rows", "attention_blockwise", "attention_varlen", "decode",
+           "decode_paged", "combine_lse"]

@@ -139,6 +139,32 @@ def decode_paged(q, k_cache, v_cache, block_table, seqlens, scale):
     return O, LSE
 
 
+def attention_varlen(q, k, v, cu_seqlens_q, cu_seqlens_k, scale, causal=False):
+    """Attention over sequences of different lengths packed back to back (the Stem /
+    AngelSlim page, section 2: the serving backend's "varlen" path; the flash-attn-volta
+    page lists variable-length sequences among what it lacks).  q [total_q, Hq, D],
+    k/v [total_k, Hkv, D]; sequence b owns query rows cu_seqlens_q[b] .. cu_seqlens_q[b+1]-1
+    and key rows cu_seqlens_k[b] .. cu_seqlens_k[b+1]-1, and is :func:`attention` of those
+    rows alone (batch of one; causal alignment bottom-right within the sequence).
+    Returns O [total_q, Hq, D] and LSE [Hq, total_q]; rows outside every sequence stay
+    O = 0, LSE = -inf."""
+    q, k, v = _f64(q), _f64(k), _f64(v)
+    cq = [int(x) for x in np.asarray(cu_seqlens_q)]
+    ck = [int(x) for x in np.asarray(cu_seqlens_k)]
+    if len(cq) != len(ck):
+        raise ValueError("cu_seqlens_q and cu_seqlens_k must have the same length")
+    total_q, Hq, D = q.shape
+    O = np.zeros((total_q, Hq, D))
+    LSE = np.full((Hq, total_q), NEG_INF)
+    for b in range(len(cq) - 1):
+        q0, q1, k0, k1 = cq[b], cq[b + 1], ck[b], ck[b + 1]
+        if q1 <= q0:
+            continue
+        o, lse = attention(q[None, q0:q1], k[None, k0:k1], v[None, k0:k1], scale, causal)
+        O[q0:q1], LSE[:, q0:q1] = o[0], lse[0]
+    return O, LSE
+
+
 def attention_blockwise(q, k, v, scale, causal=False, block=64):
     """The online-softmax recurrence, restated in float64 (TurboQuant page,
     ``online_softmax_attention``; StreamAttention page, "Kernel Design"): walk the

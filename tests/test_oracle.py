@@ -11,7 +11,8 @@ import os
 import numpy as np
 import pytest
 
-from oracle import attention, attention_rows, attention_blockwise, decode, decode_paged, combine_lse
+from oracle import (attention, attention_rows, attention_blockwise, attention_varlen, decode, decode_paged,
+                    combine_lse)
 
 GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
 TOL = 1e-12
@@ -317,3 +318,94 @@ def test_paged_decode_lengths_truncate_and_empty():
     O2, L2 = decode_paged(q[:, 0], kc, vc, table, np.array([99, 5, -3, 1]), 0.5)
     np.testing.assert_allclose(O2[0], O[0], atol=TOL)
     assert np.all(O2[2] == 0) and np.all(np.isneginf(L2[2]))
+
+
+# ---- variable-length sequences packed back to back
+
+def packed(lens_q, lens_k, Hq=4, Hkv=2, D=8, seed=0, lead=0, tail=0):
+    """Random packed q [lead + sum(lens_q) + tail, Hq, D] and k/v [sum(lens_k) + tail, Hkv, D]
+    with the cumulative offsets (sequence 0 starting at row `lead` of q)."""
+    cq = np.concatenate([[0], np.cumsum(lens_q)]) + lead
+    ck = np.concatenate([[0], np.cumsum(lens_k)])
+    q = rnd((cq[-1] + tail, Hq, D), seed)
+    k = rnd((ck[-1] + tail, Hkv, D), seed + 1)
+    v = rnd((ck[-1] + tail, Hkv, D), seed + 2)
+    return q, k, v, cq, ck
+
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_varlen_zero_query_is_mean_of_own_sequence(causal):
+    # Q = 0: every visible score is 0, so O = mean of V over the row's visible keys of its
+    # own sequence and LSE = log(count) -- fails on a wrong offset, a key leaking across a
+    # sequence boundary, or a causal offset taken from the pack instead of the sequence
+    lens_q, lens_k = [3, 5, 1, 4], [3, 7, 2, 4]
+    q, k, v, cq, ck = packed(lens_q, lens_k, seed=4)
+    q[:] = 0
+    O, L = attention_varlen(q, k, v, cq, ck, 0.9, causal)
+    G = 2
+    for b in range(4):
+        for i in range(lens_q[b]):
+            n = visible_count(i, lens_q[b], lens_k[b], causal)
+            r = cq[b] + i
+            for h in range(4):
+                np.testing.assert_allclose(O[r, h], v[ck[b]:ck[b] + n, h // G].mean(axis=0), atol=TOL)
+                np.testing.assert_allclose(L[h, r], math.log(n), atol=TOL)
+
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_varlen_equal_lengths_is_batched_attention(causal):
+    B, S = 3, 6
+    q, k, v, cq, ck = packed([S] * B, [S] * B, seed=8)
+    O, L = attention_varlen(q, k, v, cq, ck, 0.6, causal)
+    Ob, Lb = attention(q.reshape(B, S, 4, 8), k.reshape(B, S, 2, 8), v.reshape(B, S, 2, 8), 0.6, causal)
+    np.testing.assert_allclose(O, Ob.reshape(B * S, 4, 8), atol=TOL)
+    np.testing.assert_allclose(L, Lb.transpose(1, 0, 2).reshape(4, B * S), atol=TOL)
+
+
+def test_varlen_sequence_order_does_not_matter():
+    # packing the same sequences in the opposite order moves their outputs with them
+    lens = [4, 1, 6]
+    q, k, v, cq, ck = packed(lens, lens, seed=13)
+    O, L = attention_varlen(q, k, v, cq, ck, 0.5, True)
+    order = [2, 1, 0]
+    qs = np.concatenate([q[cq[b]:cq[b + 1]] for b in order])
+    ks = np.concatenate([k[ck[b]:ck[b + 1]] for b in order])
+    vs = np.concatenate([v[ck[b]:ck[b + 1]] for b in order])
+    c2 = np.concatenate([[0], np.cumsum([lens[b] for b in order])])
+    O2, L2 = attention_varlen(qs, ks, vs, c2, c2, 0.5, True)
+    for n, b in enumerate(order):
+        np.testing.assert_allclose(O2[c2[n]:c2[n + 1]], O[cq[b]:cq[b + 1]], atol=TOL)
+        np.testing.assert_allclose(L2[:, c2[n]:c2[n + 1]], L[:, cq[b]:cq[b + 1]], atol=TOL)
+
+
+def test_varlen_empty_single_key_and_uncovered_rows():
+    # sequence 0: no keys (O = 0, LSE = -inf); 1: no queries; 2: one key (O = its V row,
+    # LSE = its score); rows before the first and after the last sequence untouched
+    lens_q, lens_k = [2, 0, 3], [0, 5, 1]
+    q, k, v, cq, ck = packed(lens_q, lens_k, seed=21, lead=2, tail=3)
+    O, L = attention_varlen(q, k, v, cq, ck, 0.7, False)
+    assert np.all(O[cq[0]:cq[1]] == 0) and np.all(np.isneginf(L[:, cq[0]:cq[1]]))
+    for r in range(cq[2], cq[3]):
+        for h in range(4):
+            np.testing.assert_allclose(O[r, h], v[ck[2], h // 2], atol=TOL)
+            np.testing.assert_allclose(L[h, r], 0.7 * (q[r, h] @ k[ck[2], h // 2]), atol=TOL)
+    for r in list(range(cq[0])) + list(range(cq[-1], q.shape[0])):
+        assert np.all(O[r] == 0) and np.all(np.isneginf(L[:, r]))
+
+
+def test_varlen_chunked_prefill_last_row_is_decode():
+    # queries fewer than keys (a chunk appended to a cached prefix): with bottom-right
+    # alignment the chunk's last row sees every key of its sequence, the first row
+    # Sk - Sq + 1 of them
+    lens_q, lens_k = [3, 2], [9, 5]
+    q, k, v, cq, ck = packed(lens_q, lens_k, seed=30)
+    O, L = attention_varlen(q, k, v, cq, ck, 0.4, True)
+    for b in range(2):
+        r = cq[b + 1] - 1
+        Od, Ld = decode(q[None, r], k[None, ck[b]:ck[b + 1]], v[None, ck[b]:ck[b + 1]], 0.4)
+        np.testing.assert_allclose(O[r], Od[0], atol=TOL)
+        np.testing.assert_allclose(L[:, r], Ld[0], atol=TOL)
+        n = lens_k[b] - lens_q[b] + 1
+        Od, Ld = decode(q[None, cq[b]], k[None, ck[b]:ck[b] + n], v[None, ck[b]:ck[b] + n], 0.4)
+        np.testing.assert_allclose(O[cq[b]], Od[0], atol=TOL)
+        np.testing.assert_allclose(L[:, cq[b]], Ld[0], atol=TOL)
