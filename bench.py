@@ -32,6 +32,7 @@ sys.path.insert(0, ROOT)
 
 PREFILL = "gqa_causal_s32768_d128_bf16_sinks"
 DECODE = "gqa_decode_sk32768_d64_fp16"
+VARLEN = "gqa_causal_varlen16_t32768_d128_bf16"
 METRIC = "attn fwd TFLOP/s (prefill) and KV GB/s (decode) vs B200 roofline, 1 GPU"
 
 
@@ -199,7 +200,7 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
     ap.add_argument("--no-e2e", action="store_true")
-    ap.add_argument("--only", default="all", choices=["all", "prefill", "decode"],
+    ap.add_argument("--only", default="all", choices=["all", "prefill", "decode", "varlen"],
                     help="profiling aid: run only one half of the step (the JSON line is then partial)")
     ap.add_argument("--prefill-seq", type=int, default=0,
                     help="profiling aid: shorter prefill sequence (same heads, dtype, sinks)")
@@ -214,9 +215,10 @@ def main():
     import torch.distributed as dist
     from online_softmax_attention_sm_b200 import (sa_attn_decode, sa_attn_decode_paged,
                                                    sa_attn_decode_paged_workspace_size,
-                                                   sa_attn_decode_workspace_size, sa_attn_fwd, sa_check_status)
+                                                   sa_attn_decode_workspace_size, sa_attn_fwd, sa_attn_fwd_varlen,
+                                                   sa_check_status)
     from online_softmax_attention_sm_b200.dist import aggregate_throughput, max_over_ranks, rank_seed
-    from online_softmax_attention_sm_b200.inputs import make_workload_inputs
+    from online_softmax_attention_sm_b200.inputs import make_qkv, make_workload_inputs
     from online_softmax_attention_sm_b200.workloads import WORKLOADS
 
     rank, world, local = dist_env()
@@ -227,12 +229,13 @@ def main():
     dev = torch.device("cuda", local if world > 1 else 0)
     torch.cuda.set_device(dev)
 
-    wp, wd = WORKLOADS[PREFILL], WORKLOADS[DECODE]
+    wp, wd, wv = WORKLOADS[PREFILL], WORKLOADS[DECODE], WORKLOADS[VARLEN]
     if args.prefill_seq:
         import dataclasses
         wp = dataclasses.replace(wp, name=f"{wp.name}_seq{args.prefill_seq}", Sq=args.prefill_seq,
                                  Sk=args.prefill_seq)
     run_pre, run_dec = args.only in ("all", "prefill"), args.only in ("all", "decode")
+    run_var = args.only in ("all", "varlen")
     q_h, k_h, v_h = make_workload_inputs(wp, seed=rank_seed(wp.seed, rank))
     dq_h, dk_h, dv_h = make_workload_inputs(wd, seed=rank_seed(wd.seed, rank))
     q, k, v = q_h.to(dev), k_h.to(dev), v_h.to(dev)
@@ -328,6 +331,30 @@ def main():
         del kc, vc
     del scrub
 
+    # packed variable-length prefill: the long prefill's heads over 16 sequences of 32768
+    # tokens in all (inputs and outputs exceed the L2)
+    var_ms = [float("nan")]
+    lens = wv.lengths
+    if run_var:
+        vq, vk, vv = (t[0].to(dev) for t in make_qkv(1, wv.Sq, wv.Sk, wv.Hq, wv.Hkv, wv.D, wv.dtype,
+                                                       seed=rank_seed(wv.seed, rank)))
+        cu = torch.tensor(np.concatenate([[0], np.cumsum(lens)]), dtype=torch.int32, device=dev)
+        vo = torch.empty_like(vq)
+        vlse = torch.empty((wv.Hq, wv.Sq), dtype=torch.float32, device=dev)
+        vev = []
+        for i in range(args.warmup + args.steps):
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            sa_attn_fwd_varlen(vq, vk, vv, cu, cu, max(lens), max(lens), causal=wv.causal, scale=wv.scale,
+                               out=vo, lse=vlse, stream=stream)
+            e1.record(stream)
+            if i >= args.warmup:
+                vev.append((e0, e1))
+        torch.cuda.synchronize(dev)
+        sa_check_status(stream)
+        var_ms = [a.elapsed_time(b) for a, b in vev]
+        del vq, vk, vv, vo, vlse
+
     # e2e through the public API with host buffers: H2D of the step's inputs, D2H of outputs
     e2e_ms = None
     h2d = sum(t.numel() * t.element_size() for t in (q_h, k_h, v_h, dq_h, dk_h, dv_h))
@@ -361,6 +388,7 @@ def main():
     dec_avg = max_over_ranks(sum(dec_ms) / len(dec_ms), dev)
     cold_avg = max_over_ranks(sum(cold_ms) / len(cold_ms), dev)
     paged_avg = max_over_ranks(sum(paged_ms) / len(paged_ms), dev)
+    var_avg = max_over_ranks(sum(var_ms) / len(var_ms), dev)
     e2e_ms = max_over_ranks(e2e_ms, dev) if e2e_ms is not None else None
 
     if rank == 0:
@@ -403,6 +431,11 @@ def main():
                                  "us": paged_avg * 1e3, "page_size": 64,
                                  "layout": "the same K/V in shuffled 64-token pages, full-length sequences",
                                  "l2": "cold (4xL2 read scrub)"}},
+            "prefill_varlen": {"workload": VARLEN, "value": wv.flops / (var_avg * 1e-3) / 1e12,
+                               "unit": "TFLOP/s", "bound": "tensor", "peak": peak,
+                               "frac": wv.flops / (var_avg * 1e-3) / 1e12 / peak, "ms": var_avg,
+                               "sequences": len(lens), "lengths": f"{min(lens)}-{max(lens)}",
+                               "kernel": "attn_fwd_sm100 (dynamic unit order)"},
             "prefill_ms": pre_avg,
             "gpu_launches": (int(run_pre) + 2 * int(run_dec)) * args.steps,
             "clocks": clk.summary(),

@@ -72,6 +72,33 @@ int sa_attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse
                 float scale, int dtype, sa_stream_t stream);
 
 /*
+ * The same forward over B sequences of different lengths packed back to back (Stem /
+ * AngelSlim page, section 2: the serving backend's "varlen" path; the flash-attn-volta
+ * page lists variable-length sequences among what it lacks).
+ *   q, o         : device [total_q, Hq, D]; k, v : device [total_k, Hkv, D] (dtype).
+ *   lse          : device fp32 [Hq, total_q], or NULL.
+ *   cu_seqlens_q : device int32 [B + 1]; sequence b owns query rows
+ *                  cu_seqlens_q[b] .. cu_seqlens_q[b+1]-1 (4-byte aligned).
+ *   cu_seqlens_k : device int32 [B + 1]; its key rows likewise.
+ *   max_seqlen_q : an upper bound on every cu_seqlens_q[b+1] - cu_seqlens_q[b] (sizes
+ *                  the work list); max_seqlen_k likewise for keys (a scheduling hint).
+ *   causal       : 0 or 1, bottom-right aligned within each sequence (a query chunk
+ *                  shorter than its keys sees the whole prefix).
+ * Each sequence gets exactly sa_attn_fwd of its own rows.  Rows of o/lse outside every
+ * sequence are not written.  The offsets stay on the device: the kernel clamps them into
+ * the buffers (never reading or writing outside q/k/v/o/lse), and if they run backwards,
+ * leave the buffers or give a query length above max_seqlen_q it records that in the
+ * device status word, so the next sa_check_status() returns SA_ERR_INVALID (outputs of the
+ * offending sequences are then undefined).  B, total_q, Hq or max_seqlen_q == 0: SA_OK,
+ * nothing launched; total_k == 0: O = 0, LSE = -inf for every row.
+ */
+int sa_attn_fwd_varlen(const void* q, const void* k, const void* v, void* o, float* lse,
+                       const int* cu_seqlens_q, const int* cu_seqlens_k, int B,
+                       int max_seqlen_q, int max_seqlen_k, int total_q, int total_k,
+                       int Hq, int Hkv, int D, int causal, float scale, int dtype,
+                       sa_stream_t stream);
+
+/*
  * Bytes of decode workspace needed for `num_splits` (0 = the automatic choice):
  * B * Hq * splits * (D + 4) * 4.  It holds, per (b, h, split), the split's running max
  * and two running sums (of the 16-bit weights the MMA used, and of the fp32 weights for
@@ -171,8 +198,9 @@ int sa_attn_fwd_simple(const void* q, const void* k, const void* v, void* o, flo
 /* Thread-local description of the last non-OK return of this thread ("" if none). */
 const char* sa_last_error(void);
 
-/* Synchronises `stream`, then returns SA_ERR_TIMEOUT (and clears the word) if a device
- * wait expired since the last check, SA_ERR_CUDA on a CUDA error, else SA_OK. */
+/* Synchronises `stream`, then reads and clears the device status word: SA_ERR_TIMEOUT if a
+ * device wait expired since the last check, SA_ERR_INVALID if a kernel found invalid
+ * packed sequence offsets (sa_attn_fwd_varlen), SA_ERR_CUDA on a CUDA error, else SA_OK. */
 int sa_check_status(sa_stream_t stream);
 
 /* Diagnostic: launches one kernel whose single bounded wait can never be satisfied, to

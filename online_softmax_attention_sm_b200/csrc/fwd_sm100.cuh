@@ -80,24 +80,46 @@ struct FwdParams {
   unsigned int* work;  // [2] dynamic scheduling (the kernel's DYN instance): next unit to
                        // hand out past the first round, CTAs done fetching; zero at launch,
                        // zeroed again by the launch's last CTA
+  // Packed variable-length sequences (null: the dense [B, S, H, D] layout).  Sequence b owns
+  // query rows cu_q[b] .. cu_q[b+1]-1 of q/o [Sq, Hq, D] and key rows cu_k[b] .. cu_k[b+1]-1
+  // of k/v [Sk, Hkv, D] (Sq, Sk: the packed totals); LSE is [Hq, Sq].  n_qblk covers
+  // max_sq query rows per sequence.
+  const int* cu_q;
+  const int* cu_k;
+  int max_sq;
 };
 
 constexpr int kUnitQueue = 4;    // unit indices the load warp may hand out ahead
 
 struct UnitInfo {
-  int b, h, kvh, q0;         // q0: first query row of the unit
+  int b, h, kvh, q0;         // q0: first query row of the unit within its sequence
+  int sq, sk;                // the sequence's query and key lengths
+  int qbase, kbase, mb;      // its first query / key row and batch index in the TMA maps
   int nkv[2];                // K/V tiles needed by Q tile 0 / 1 (0: tile has no work)
   int nkv_max;
 };
 
-__device__ __forceinline__ int fwd_kv_tiles(const FwdParams& p, int r0) {
-  if (r0 >= p.Sq) return 0;
-  int kend = p.Sk;
-  if (p.causal) {
-    int rmax = min(r0 + 127, p.Sq - 1);
-    kend = min(p.Sk, rmax + p.Sk - p.Sq + 1);
+__device__ __forceinline__ int fwd_kv_tiles(int sq, int sk, int causal, int r0) {
+  if (r0 >= sq) return 0;
+  int kend = sk;
+  if (causal) {
+    int rmax = min(r0 + 127, sq - 1);
+    kend = min(sk, rmax + sk - sq + 1);
   }
   return kend > 0 ? (kend + 127) / 128 : 0;
+}
+
+// Packed sequences: the offsets must run forward inside the buffers and no sequence may
+// be longer than max_sq.  The producer warps check them (each CTA a share) and record a
+// status code for the first violation; the kernel itself clamps (fwd_unit), so bad offsets
+// only shorten or empty a sequence.
+__device__ __forceinline__ void fwd_check_lengths(const FwdParams& p, int lane, int cta, int ncta) {
+  for (int b = cta * 32 + lane; b < p.B; b += ncta * 32) {
+    const int q0 = __ldg(p.cu_q + b), q1 = __ldg(p.cu_q + b + 1);
+    const int k0 = __ldg(p.cu_k + b), k1 = __ldg(p.cu_k + b + 1);
+    if (q0 < 0 || q1 < q0 || q1 > p.Sq || q1 - q0 > p.max_sq || k0 < 0 || k1 < k0 || k1 > p.Sk)
+      record_status(kStatusBadLengths, b);
+  }
 }
 
 // Unit order.  The query blocks are cut into bands of `band` blocks, longest first; within
@@ -125,8 +147,21 @@ __device__ __forceinline__ UnitInfo fwd_unit(const FwdParams& p, int u) {
   x.kvh = bk % p.Hkv;
   x.h = x.kvh * G + rem % G;
   x.q0 = qb * 256;
-  x.nkv[0] = fwd_kv_tiles(p, x.q0);
-  x.nkv[1] = fwd_kv_tiles(p, x.q0 + 128);
+  if (p.cu_q) {
+    // clamped into the buffers: offsets that run backwards or past the end give an empty
+    // or shortened sequence, never an access outside q/k/v/o
+    const int q_lo = min(max(__ldg(p.cu_q + x.b), 0), p.Sq);
+    const int q_hi = min(max(__ldg(p.cu_q + x.b + 1), q_lo), p.Sq);
+    const int k_lo = min(max(__ldg(p.cu_k + x.b), 0), p.Sk);
+    const int k_hi = min(max(__ldg(p.cu_k + x.b + 1), k_lo), p.Sk);
+    x.sq = q_hi - q_lo; x.sk = k_hi - k_lo;
+    x.qbase = q_lo; x.kbase = k_lo; x.mb = 0;
+  } else {
+    x.sq = p.Sq; x.sk = p.Sk;
+    x.qbase = 0; x.kbase = 0; x.mb = x.b;
+  }
+  x.nkv[0] = fwd_kv_tiles(x.sq, x.sk, p.causal, x.q0);
+  x.nkv[1] = fwd_kv_tiles(x.sq, x.sk, p.causal, x.q0 + 128);
   x.nkv_max = max(x.nkv[0], x.nkv[1]);
   return x;
 }
@@ -230,7 +265,7 @@ __device__ __forceinline__ void fwd_producer(const CUtensorMap* tm_q, const CUte
           const CUtensorMap* tm = kv ? tm_v : tm_k;
 #pragma unroll
           for (int c = 0; c < Cfg::KCH; ++c)
-            tma_load_4d(dst + c * Cfg::CHUNK_BYTES, tm, &sm.kv_full[slot], c * 64, x.kvh, j * 128, x.b);
+            tma_load_4d(dst + c * Cfg::CHUNK_BYTES, tm, &sm.kv_full[slot], c * 64, x.kvh, x.kbase + j * 128, x.mb);
           ++ring_n;
           slot = (slot + 1 == Cfg::STAGES) ? 0 : slot + 1;
           if (j == 0 && kv == 0) {
@@ -246,7 +281,8 @@ __device__ __forceinline__ void fwd_producer(const CUtensorMap* tm_q, const CUte
               mbar_arrive_expect_tx(&sm.q_full[t], Cfg::TILE_BYTES);
 #pragma unroll
               for (int c = 0; c < Cfg::KCH; ++c)
-                tma_load_4d(qd + c * Cfg::CHUNK_BYTES, tm_q, &sm.q_full[t], c * 64, x.h, x.q0 + t * 128, x.b);
+                tma_load_4d(qd + c * Cfg::CHUNK_BYTES, tm_q, &sm.q_full[t], c * 64, x.h,
+                            x.qbase + x.q0 + t * 128, x.mb);
               ++ql;
             }
           }
@@ -597,12 +633,12 @@ __device__ __forceinline__ void fwd_softmax(const FwdParams& p, const FwdSmem<D>
     UnitInfo x = fwd_unit(p, u);
     const int nkv = x.nkv[t];
     const int row = x.q0 + t * 128 + row_in_tile;
-    int klim = p.Sk;
-    if (p.causal) klim = min(p.Sk, row + p.Sk - p.Sq + 1);
+    int klim = x.sk;
+    if (p.causal) klim = min(x.sk, row + x.sk - x.sq + 1);
     // the first key tile that any row of this Q tile must mask
     const int r0 = x.q0 + t * 128;
-    int kvis = p.Sk;                        // keys every row of the tile can see
-    if (p.causal) kvis = min(kvis, max(0, r0 + p.Sk - p.Sq + 1));
+    int kvis = x.sk;                        // keys every row of the tile can see
+    if (p.causal) kvis = min(kvis, max(0, r0 + x.sk - x.sq + 1));
     const int mask_from = kvis / 128;
     // l_sum: sum of the 16-bit weights (normalises O, matching what the MMA multiplied);
     // l_lse: sum of the fp32 weights (gives the LSE without the 16-bit rounding bias)
@@ -633,10 +669,10 @@ __device__ __forceinline__ void fwd_softmax(const FwdParams& p, const FwdSmem<D>
       ++o_n;
       tc_fence_after();
     }
-    const bool store = row < p.Sq;
+    const bool store = row < x.sq;
     const float inv_l = l_sum > 0.f ? 1.f / l_sum : 0.f;
     using T = typename std::conditional<BF16, __nv_bfloat16, __half>::type;
-    T* orow = reinterpret_cast<T*>(p.o) + (((size_t)x.b * p.Sq + row) * p.Hq + x.h) * D;
+    T* orow = reinterpret_cast<T*>(p.o) + (((size_t)x.mb * p.Sq + x.qbase + row) * p.Hq + x.h) * D;
 #pragma unroll 1
     for (int c = 0; c < D / 32; ++c) {
       uint32_t r[32];
@@ -667,7 +703,7 @@ __device__ __forceinline__ void fwd_softmax(const FwdParams& p, const FwdSmem<D>
     }
     if (store && p.lse) {
       float lse = l_lse > 0.f ? (m_ref + __log2f(l_lse)) * 0.69314718055994531f : -INFINITY;
-      p.lse[((size_t)x.b * p.Hq + x.h) * p.Sq + row] = lse;
+      p.lse[((size_t)x.mb * p.Hq + x.h) * p.Sq + x.qbase + row] = lse;
     }
     tc_fence_before();
   }
@@ -723,10 +759,12 @@ attn_fwd_sm100(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
   const uint32_t tmem_base = *sm.tmem_holder;
 
   if (warp < 4) {
-    // load / MMA warpgroup (warps 2 and 3 have no role) gives registers away
+    // load / MMA warpgroup gives registers away; warp 2 checks packed sequence offsets,
+    // warp 3 has no role
     regs_dec<Cfg::REGS_OTHER>();
     if (warp == kWarpLoad) fwd_producer<D, BF16, DYN>(&tm_q, &tm_k, &tm_v, p, sm, lane, cta, ncta);
     else if (warp == kWarpMma) fwd_mma<D, BF16, DYN>(p, sm, tmem_base, lane, cta, ncta);
+    else if (warp == 2 && p.cu_q) fwd_check_lengths(p, lane, cta, ncta);
     fwd_teardown(warp == kWarpMma, tmem_base, Cfg::TMEM_COLS);
   } else {
     regs_inc<Cfg::REGS_SOFTMAX>();

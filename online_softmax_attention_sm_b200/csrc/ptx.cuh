@@ -14,11 +14,13 @@ namespace sa {
 // ----------------------------------------------------------------------------------
 __device__ int g_status;
 
-enum : int { kStatusTimeout = 1 };
+enum : int { kStatusTimeout = 1, kStatusBadLengths = 2 };
 
-__device__ __forceinline__ void record_timeout(int where) {
-  atomicCAS(&g_status, 0, (kStatusTimeout << 16) | (where & 0xffff));
+__device__ __forceinline__ void record_status(int code, int where) {
+  atomicCAS(&g_status, 0, (code << 16) | (where & 0xffff));
 }
+
+__device__ __forceinline__ void record_timeout(int where) { record_status(kStatusTimeout, where); }
 
 __device__ __forceinline__ uint64_t globaltimer_ns() {
   uint64_t t;

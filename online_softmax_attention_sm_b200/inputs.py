@@ -13,6 +13,9 @@ identical bits):
 
 Layouts: prefill Q [B, Sq, Hq, D], K/V [B, Sk, Hkv, D]; decode Q [B, Hq, D].
 All tensors are contiguous CPU tensors of the storage dtype.
+
+Packed variable-length batches draw their sequence lengths with :func:`varlen_lengths`
+and their tokens with ``make_qkv(1, total, total, ...)`` (sequence after sequence).
 """
 from __future__ import annotations
 
@@ -55,3 +58,24 @@ def sample_rows(Sq, n_random, seed, extra=()):
     fixed = [0, 1, 2, 3, 127, 128, 129, 255, 256, 257, Sq - 1] + list(extra)
     rnd = torch.randint(0, Sq, (n_random,), generator=g).tolist() if n_random else []
     return sorted({r for r in fixed + rnd if 0 <= r < Sq})
+
+
+def varlen_lengths(total, n, seed):
+    """A seeded mix of n sequence lengths (each >= 1) summing to `total`: weights
+    2^(4u), u ~ U(0, 1) (a 16x spread between the shortest and the longest), scaled to
+    the total and floored, the remainder given one token at a time to the first
+    sequences."""
+    if n <= 0 or total < n:
+        raise ValueError("need 1 <= n <= total")
+    g = torch.Generator(device="cpu")
+    g.manual_seed(int(seed) + 104729)
+    w = torch.pow(2.0, 4.0 * torch.rand(n, generator=g, dtype=torch.float64))
+    lens = [max(1, int(x)) for x in (w / w.sum() * total).floor().tolist()]
+    i = 0
+    while sum(lens) < total:
+        lens[i % n] += 1
+        i += 1
+    while sum(lens) > total:                  # only if flooring to >= 1 overshot
+        j = max(range(n), key=lambda t: lens[t])
+        lens[j] -= 1
+    return lens

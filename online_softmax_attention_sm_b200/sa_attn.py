@@ -24,6 +24,7 @@ _P, _I, _F, _Z = ctypes.c_void_p, ctypes.c_int, ctypes.c_float, ctypes.c_size_t
 SIGNATURES = {
     "sa_attn_fwd": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _F, _I, _P]),
     "sa_attn_fwd_simple": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _F, _I, _P]),
+    "sa_attn_fwd_varlen": (_I, [_P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _I, _I, _F, _I, _P]),
     "sa_attn_decode_workspace_size": (_Z, [_I, _I, _I, _I, _I, _I]),
     "sa_attn_decode_num_splits": (_I, [_I, _I, _I, _I, _I]),
     "sa_attn_decode": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _F, _I, _I, _P, _Z, _P]),
@@ -109,6 +110,42 @@ def sa_attn_fwd(q, k, v, causal=False, scale=None, out=None, lse=None, return_ls
     fn = lib().sa_attn_fwd_simple if simple else lib().sa_attn_fwd
     _check(fn(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse), B, Sq, Sk, Hq, Hkv, D,
               int(bool(causal)), float(scale), _DT[q.dtype], _stream(stream)))
+    return out, lse
+
+
+def sa_attn_fwd_varlen(q, k, v, cu_seqlens_q, cu_seqlens_k, max_seqlen_q, max_seqlen_k, causal=False,
+                       scale=None, out=None, lse=None, return_lse=True, stream=None):
+    """Attention forward over sequences packed back to back.  q [total_q,Hq,D], k/v
+    [total_k,Hkv,D] (fp16/bf16, CUDA, contiguous); cu_seqlens_q/k int32 [B+1] on the same
+    device; max_seqlen_q/k host ints bounding every sequence's length.
+    Returns (o [total_q,Hq,D], lse [Hq,total_q] fp32 or None)."""
+    total_q, Hq, D = q.shape
+    total_k, Hkv = k.shape[0], k.shape[1]
+    if k.shape != (total_k, Hkv, D) or v.shape != k.shape:
+        raise ValueError(f"shape mismatch q{tuple(q.shape)} k{tuple(k.shape)} v{tuple(v.shape)}")
+    if q.dtype not in _DT:
+        raise TypeError(f"unsupported dtype {q.dtype}")
+    for n, t in (("q", q), ("k", k), ("v", v)):
+        _check_tensor(n, t, q.dtype, q.device)
+    for n, t in (("cu_seqlens_q", cu_seqlens_q), ("cu_seqlens_k", cu_seqlens_k)):
+        _check_tensor(n, t, torch.int32, q.device)
+    if cu_seqlens_q.dim() != 1 or cu_seqlens_q.shape != cu_seqlens_k.shape or cu_seqlens_q.numel() < 1:
+        raise ValueError(f"cu_seqlens must both be [B+1], got {tuple(cu_seqlens_q.shape)} "
+                         f"and {tuple(cu_seqlens_k.shape)}")
+    B = cu_seqlens_q.numel() - 1
+    if scale is None:
+        scale = 1.0 / math.sqrt(D)
+    if out is None:
+        out = torch.empty_like(q)
+    _check_tensor("out", out, q.dtype, q.device)
+    if return_lse and lse is None:
+        lse = torch.empty((Hq, total_q), dtype=torch.float32, device=q.device)
+    if lse is not None:
+        _check_tensor("lse", lse, torch.float32, q.device)
+    _check(lib().sa_attn_fwd_varlen(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse), _ptr(cu_seqlens_q),
+                                    _ptr(cu_seqlens_k), B, int(max_seqlen_q), int(max_seqlen_k), total_q,
+                                    total_k, Hq, Hkv, D, int(bool(causal)), float(scale), _DT[q.dtype],
+                                    _stream(stream)))
     return out, lse
 
 

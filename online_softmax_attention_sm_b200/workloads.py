@@ -38,10 +38,22 @@ class Workload:
         return 1.0 / math.sqrt(self.D)
 
     @property
+    def lengths(self):
+        """Packed variable-length workloads ("prefill_varlen": B sequences, Sq = Sk = the
+        total tokens): the seeded sequence lengths; None otherwise."""
+        if self.kind != "prefill_varlen":
+            return None
+        from .inputs import varlen_lengths
+        return varlen_lengths(self.Sq, self.B, self.seed)
+
+    @property
     def flops(self) -> float:
         """Forward FLOPs under the flash-attn-volta convention 4*B*H*Sq*Sk*D,
-        halved for causal."""
-        f = 4.0 * self.B * self.Hq * self.Sq * self.Sk * self.D
+        halved for causal (summed over the sequences of a packed workload)."""
+        if self.kind == "prefill_varlen":
+            f = sum(4.0 * self.Hq * n * n * self.D for n in self.lengths)
+        else:
+            f = 4.0 * self.B * self.Hq * self.Sq * self.Sk * self.D
         return f / 2 if self.causal else f
 
     @property
@@ -65,5 +77,9 @@ WORKLOADS = {
                  True, k_sink_rows=4, k_sink_factor=8.0, seed=20261202 + 3),
         Workload("gqa_decode_sk32768_d64_fp16", "decode", "fp16", 4, 1, 32768, 14, 2, 64, False,
                  seed=20261202 + 4),
+        # the long prefill's heads over 16 packed sequences of 32768 tokens in all
+        Workload("gqa_causal_varlen16_t32768_d128_bf16", "prefill_varlen", "bf16", 16, 32768, 32768,
+                 32, 8, 128, True, seed=20261202 + 6,
+                 notes="packed sequences, lengths from inputs.varlen_lengths"),
     ]
 }

@@ -168,6 +168,40 @@ def test_paged_workspace_size(L):
     assert L.sa_attn_decode_paged_workspace_size(0, 2, 1, 64, 64, 512, 1) == 0      # empty
 
 
+def fwd_varlen(L, q=FAKE, k=FAKE, v=FAKE, o=FAKE, lse=NULL, cq=FAKE, ck=FAKE, B=2, mq=64, mk=64, tq=100,
+               tk=100, Hq=2, Hkv=1, D=64, causal=1, scale=0.125, dtype=1):
+    return L.sa_attn_fwd_varlen(q, k, v, o, lse, cq, ck, B, mq, mk, tq, tk, Hq, Hkv, D, causal, scale, dtype,
+                                None)
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(q=NULL), sa.SA_ERR_INVALID),
+    (dict(o=NULL), sa.SA_ERR_INVALID),
+    (dict(cq=NULL), sa.SA_ERR_INVALID),
+    (dict(ck=NULL), sa.SA_ERR_INVALID),
+    (dict(cq=ctypes.c_void_p((1 << 20) + 2)), sa.SA_ERR_INVALID),
+    (dict(B=-1), sa.SA_ERR_INVALID),
+    (dict(tq=-5), sa.SA_ERR_INVALID),
+    (dict(mq=-1), sa.SA_ERR_INVALID),
+    (dict(mk=-1), sa.SA_ERR_INVALID),
+    (dict(Hq=3, Hkv=2), sa.SA_ERR_INVALID),
+    (dict(D=96), sa.SA_ERR_UNSUPPORTED),
+    (dict(dtype=5), sa.SA_ERR_UNSUPPORTED),
+    (dict(causal=3), sa.SA_ERR_INVALID),
+    (dict(scale=math.nan), sa.SA_ERR_INVALID),
+    (dict(k=ctypes.c_void_p((1 << 20) + 8)), sa.SA_ERR_INVALID),
+])
+def test_fwd_varlen_rejects_invalid_arguments(L, kw, code):
+    assert fwd_varlen(L, **kw) == code
+
+
+@pytest.mark.parametrize("kw", [dict(B=0), dict(tq=0), dict(Hq=0, Hkv=0), dict(mq=0)])
+def test_fwd_varlen_empty_problem_is_a_no_op(L, kw):
+    args = dict(q=NULL, k=NULL, v=NULL, o=NULL, cq=NULL, ck=NULL)
+    args.update(kw)
+    assert fwd_varlen(L, **args) == sa.SA_OK
+
+
 def test_version(L):
     assert re.fullmatch(r"\d+\.\d+\.\d+", sa.sa_version())
 
