@@ -79,3 +79,33 @@ def varlen_lengths(total, n, seed):
         j = max(range(n), key=lambda t: lens[t])
         lens[j] -= 1
     return lens
+
+
+def stem_block_mask(B, Hq, Sq, Sk, causal, seed, initial_blocks=4, window_blocks=4, keep_ratio=0.1,
+                    block=128):
+    """A seeded block mask [B, Hq, ceil(Sq/block), ceil(Sk/block)] (uint8, 1 = keep) shaped like
+    the selection of the Stem page's block-sparse prefill: for every query block, the first
+    `initial_blocks` key blocks (sinks) and the last `window_blocks` key blocks it can see
+    (sliding window) are kept, and of the key blocks in between a fraction `keep_ratio`
+    (rounded) is drawn uniformly at random -- a stand-in for the page's top-k by block score.
+    "Can see": with causal, up to the block holding key (last row of the query block) +
+    Sk - Sq; otherwise every key block."""
+    nq, nk = -(-Sq // block), -(-Sk // block)
+    g = torch.Generator(device="cpu")
+    g.manual_seed(int(seed) + 611953)
+    mask = torch.zeros((B, Hq, nq, nk), dtype=torch.uint8)
+    for qi in range(nq):
+        last_row = min(Sq, (qi + 1) * block) - 1
+        kmax = min(nk - 1, (last_row + Sk - Sq) // block) if causal else nk - 1
+        if kmax < 0:
+            continue
+        lo, hi = min(initial_blocks, kmax + 1), max(0, kmax + 1 - window_blocks)
+        mask[:, :, qi, :lo] = 1
+        mask[:, :, qi, hi:kmax + 1] = 1
+        mid = hi - lo
+        take = int(round(keep_ratio * mid)) if mid > 0 else 0
+        if take:
+            r = torch.rand((B, Hq, mid), generator=g)
+            idx = r.topk(take, dim=-1).indices + lo
+            mask[:, :, qi].scatter_(-1, idx, 1)
+    return mask

@@ -7,7 +7,9 @@ It shares no code with the CUDA path.  Every function here is pinned by
 "parity unpinned".
 """
 from .attention import (attention, attention_rows, attention_blockwise, attention_varlen,
+                        attention_block_sparse, attention_block_sparse_rows, block_sparse_pairs,
                         decode, decode_paged, combine_lse)
 
-__all__ = ["attention", "attention_rows", "attention_blockwise", "attention_varlen", "decode",
+__all__ = ["attention", "attention_rows", "attention_blockwise", "attention_varlen",
+           "attention_block_sparse", "attention_block_sparse_rows", "block_sparse_pairs", "decode",
            "decode_paged", "combine_lse"]

@@ -165,6 +165,74 @@ def attention_varlen(q, k, v, cu_seqlens_q, cu_seqlens_k, scale, causal=False):
     return O, LSE
 
 
+def attention_block_sparse(q, k, v, block_mask, scale, causal=False, block=128):
+    """Block-sparse attention (the Stem / AngelSlim page, section 2.3: attention over
+    the key blocks the top-k mask keeps, block_size 128; initial "sink" blocks and the
+    sliding-window blocks are among them).  q [B,Sq,Hq,D], k/v [B,Sk,Hkv,D];
+    block_mask [B, Hq, ceil(Sq/block), ceil(Sk/block)], nonzero = keep.  Key j is visible
+    to query row i of head h iff the dense rule allows it (bottom-right causal alignment
+    when causal) AND block_mask[b, h, i // block, j // block] is nonzero; the rest is
+    :func:`attention`'s definition (no visible key: O = 0, LSE = -inf).
+    Returns O [B,Sq,Hq,D], LSE [B,Hq,Sq]."""
+    q, k, v = _f64(q), _f64(k), _f64(v)
+    B, Sq, Hq, D = q.shape
+    Sk, Hkv = k.shape[1], k.shape[2]
+    if Hkv == 0 or Hq % Hkv:
+        raise ValueError("Hq must be a positive multiple of Hkv")
+    bm = np.asarray(block_mask) != 0
+    nq, nk = -(-Sq // block), -(-Sk // block)
+    if bm.shape != (B, Hq, nq, nk):
+        raise ValueError(f"block_mask must be [{B}, {Hq}, {nq}, {nk}], got {bm.shape}")
+    G = Hq // Hkv
+    O = np.zeros((B, Sq, Hq, D))
+    LSE = np.full((B, Hq, Sq), NEG_INF)
+    if Sq == 0 or Sk == 0:
+        return O, LSE
+    base = _visible(Sq, Sk, causal)
+    rows, cols = np.arange(Sq) // block, np.arange(Sk) // block
+    for b in range(B):
+        for h in range(Hq):
+            vis = base & bm[b, h][rows[:, None], cols[None, :]]
+            kvh = h // G
+            O[b, :, h, :], LSE[b, h, :] = _softmax_attend(
+                q[b, :, h, :], k[b, :, kvh, :], v[b, :, kvh, :], scale, vis)
+    return O, LSE
+
+
+def attention_block_sparse_rows(q, k, v, block_mask, scale, causal, b, h, rows, block=128):
+    """:func:`attention_block_sparse` for selected query rows of one (batch, head):
+    O [n, D], LSE [n].  For sizes whose full score matrix would not fit."""
+    rows = np.asarray(rows, dtype=np.int64)
+    Sq, Hq = q.shape[1], q.shape[2]
+    Sk, Hkv = k.shape[1], k.shape[2]
+    kvh = h // (Hq // Hkv)
+    if Sk == 0:
+        return np.zeros((rows.size, q.shape[3])), np.full(rows.size, NEG_INF)
+    bm = np.asarray(block_mask[b, h]) != 0
+    vis = _visible(Sq, Sk, causal, rows) & bm[(rows // block)[:, None], (np.arange(Sk) // block)[None, :]]
+    return _softmax_attend(_f64(q[b, rows, h, :]), _f64(k[b, :, kvh, :]), _f64(v[b, :, kvh, :]), scale, vis)
+
+
+def block_sparse_pairs(Sq, Sk, block_mask, causal, block=128):
+    """Number of visible (query row, key) pairs under a block mask [.., nq, nk] summed
+    over its leading dimensions: the work a block-sparse forward does (4*D FLOP per
+    pair).  Counted per kept block from the dense visibility rule."""
+    bm = np.asarray(block_mask) != 0
+    nq, nk = bm.shape[-2], bm.shape[-1]
+    per_block = np.zeros((nq, nk), dtype=np.int64)
+    for qi in range(nq):
+        r0, r1 = qi * block, min(Sq, (qi + 1) * block)
+        for ki in range(nk):
+            c0, c1 = ki * block, min(Sk, (ki + 1) * block)
+            if not causal:
+                per_block[qi, ki] = (r1 - r0) * (c1 - c0)
+            else:
+                # row i sees keys j <= i + Sk - Sq: clip that bound into the block's columns
+                hi = np.clip(np.arange(r0, r1) + Sk - Sq + 1, c0, c1)
+                per_block[qi, ki] = int((hi - c0).sum())
+    return int((bm.reshape(-1, nq, nk) * per_block[None]).sum())
+
+
 def attention_blockwise(q, k, v, scale, causal=False, block=64):
     """The online-softmax recurrence, restated in float64 (TurboQuant page,
     ``online_softmax_attention``; StreamAttention page, "Kernel Design"): walk the

@@ -11,7 +11,8 @@ import os
 import numpy as np
 import pytest
 
-from oracle import (attention, attention_rows, attention_blockwise, attention_varlen, decode, decode_paged,
+from oracle import (attention, attention_rows, attention_blockwise, attention_varlen, attention_block_sparse,
+                    attention_block_sparse_rows, block_sparse_pairs, decode, decode_paged,
                     combine_lse)
 
 GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
@@ -409,3 +410,104 @@ def test_varlen_chunked_prefill_last_row_is_decode():
         Od, Ld = decode(q[None, cq[b]], k[None, ck[b]:ck[b] + n], v[None, ck[b]:ck[b] + n], 0.4)
         np.testing.assert_allclose(O[cq[b]], Od[0], atol=TOL)
         np.testing.assert_allclose(L[:, cq[b]], Ld[0], atol=TOL)
+
+
+# ---- block-sparse attention: a 0/1 mask over (query block, key block) on top of the
+#      dense rule (tiny blocks so the pins stay small)
+
+def rand_mask(B, Hq, nq, nk, density, seed):
+    return (np.random.default_rng(seed).random((B, Hq, nq, nk)) < density).astype(np.uint8)
+
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_block_sparse_all_kept_is_dense(causal):
+    q, k, v = qkv(B=2, Sq=10, Sk=10, Hq=4, Hkv=2, seed=51)
+    m = np.ones((2, 4, 3, 3), np.uint8)
+    O, L = attention_block_sparse(q, k, v, m, 0.3, causal, block=4)
+    Od, Ld = attention(q, k, v, 0.3, causal)
+    np.testing.assert_allclose(O, Od, atol=TOL)
+    np.testing.assert_allclose(L, Ld, atol=TOL)
+
+
+def test_block_sparse_lower_block_triangle_with_causal_is_causal():
+    # blocks above the diagonal are causally invisible anyway
+    q, k, v = qkv(B=1, Sq=12, Sk=12, Hq=2, Hkv=1, seed=52)
+    m = np.tril(np.ones((3, 3), np.uint8))[None, None].repeat(2, axis=1)
+    O, L = attention_block_sparse(q, k, v, m, 0.3, True, block=4)
+    Od, Ld = attention(q, k, v, 0.3, True)
+    np.testing.assert_allclose(O, Od, atol=TOL)
+    np.testing.assert_allclose(L, Ld, atol=TOL)
+
+
+def test_block_sparse_diagonal_blocks_are_independent_attentions():
+    q, k, v = qkv(B=1, Sq=12, Sk=12, Hq=2, Hkv=2, seed=53)
+    m = np.eye(3, dtype=np.uint8)[None, None].repeat(2, axis=1)
+    O, L = attention_block_sparse(q, k, v, m, 0.5, False, block=4)
+    for i in range(3):
+        sl = slice(4 * i, 4 * i + 4)
+        Ob, Lb = attention(q[:, sl], k[:, sl], v[:, sl], 0.5, False)
+        np.testing.assert_allclose(O[:, sl], Ob, atol=TOL)
+        np.testing.assert_allclose(L[:, :, sl], Lb, atol=TOL)
+
+
+def test_block_sparse_equals_attention_over_the_gathered_keys():
+    # non-causal: each query block attends exactly the concatenation of its kept key blocks
+    B, Sq, Sk, Hq, Hkv, blk = 1, 11, 14, 4, 2, 4
+    q, k, v = qkv(B=B, Sq=Sq, Sk=Sk, Hq=Hq, Hkv=Hkv, seed=54)
+    m = rand_mask(B, Hq, 3, 4, 0.5, seed=9)
+    O, L = attention_block_sparse(q, k, v, m, 0.4, False, block=blk)
+    for h in range(Hq):
+        for qi in range(3):
+            keys = [j for ki in range(4) if m[0, h, qi, ki] for j in range(ki * blk, min(Sk, ki * blk + blk))]
+            rows = slice(qi * blk, min(Sq, qi * blk + blk))
+            if not keys:
+                assert np.all(O[0, rows, h] == 0) and np.all(np.isneginf(L[0, h, rows]))
+                continue
+            kk = k[:, keys][:, :, [h // 2]]
+            vv = v[:, keys][:, :, [h // 2]]
+            Og, Lg = attention(q[:, rows][:, :, [h]], kk, vv, 0.4, False)
+            np.testing.assert_allclose(O[0, rows, h], Og[0, :, 0], atol=TOL)
+            np.testing.assert_allclose(L[0, h, rows], Lg[0, 0], atol=TOL)
+
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_block_sparse_zero_query_is_mean_over_kept_visible_keys(causal):
+    Sq, Sk, blk = 9, 13, 4
+    q, k, v = qkv(B=1, Sq=Sq, Sk=Sk, Hq=2, Hkv=1, seed=55)
+    q[:] = 0
+    m = rand_mask(1, 2, 3, 4, 0.6, seed=4)
+    O, L = attention_block_sparse(q, k, v, m, 1.0, causal, block=blk)
+    for h in range(2):
+        for i in range(Sq):
+            keys = [j for j in range(Sk) if m[0, h, i // blk, j // blk] and (not causal or j <= i + Sk - Sq)]
+            if not keys:
+                assert np.all(O[0, i, h] == 0) and np.isneginf(L[0, h, i])
+            else:
+                np.testing.assert_allclose(O[0, i, h], v[0, keys, 0].mean(axis=0), atol=TOL)
+                np.testing.assert_allclose(L[0, h, i], math.log(len(keys)), atol=TOL)
+
+
+def test_block_sparse_rows_match_full():
+    q, k, v = qkv(B=2, Sq=13, Sk=17, Hq=4, Hkv=2, seed=56)
+    m = rand_mask(2, 4, 4, 5, 0.5, seed=5)
+    O, L = attention_block_sparse(q, k, v, m, 0.3, True, block=4)
+    rows = [0, 3, 4, 12]
+    Or, Lr = attention_block_sparse_rows(q, k, v, m, 0.3, True, 1, 3, rows, block=4)
+    np.testing.assert_allclose(Or, O[1, rows, 3], atol=TOL)
+    np.testing.assert_allclose(Lr, L[1, 3, rows], atol=TOL)
+
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_block_sparse_pair_count_by_brute_force(causal):
+    Sq, Sk, blk = 10, 14, 4
+    m = rand_mask(2, 3, 3, 4, 0.5, seed=6)
+    n = 0
+    for b in range(2):
+        for h in range(3):
+            for i in range(Sq):
+                for j in range(Sk):
+                    n += bool(m[b, h, i // blk, j // blk]) and (not causal or j <= i + Sk - Sq)
+    assert block_sparse_pairs(Sq, Sk, m, causal, block=blk) == n
+    ones = np.ones((1, 1, 3, 3), np.uint8)
+    assert block_sparse_pairs(12, 12, ones, True, block=4) == 12 * 13 // 2
+    assert block_sparse_pairs(12, 12, ones, False, block=4) == 144
