@@ -200,7 +200,7 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
     ap.add_argument("--no-e2e", action="store_true")
-    ap.add_argument("--only", default="all", choices=["all", "prefill", "decode", "varlen"],
+    ap.add_argument("--only", default="all", choices=["all", "prefill", "decode", "varlen", "sparse"],
                     help="profiling aid: run only one half of the step (the JSON line is then partial)")
     ap.add_argument("--prefill-seq", type=int, default=0,
                     help="profiling aid: shorter prefill sequence (same heads, dtype, sinks)")
@@ -215,11 +215,12 @@ def main():
     import torch.distributed as dist
     from online_softmax_attention_sm_b200 import (sa_attn_decode, sa_attn_decode_paged,
                                                    sa_attn_decode_paged_workspace_size,
-                                                   sa_attn_decode_workspace_size, sa_attn_fwd, sa_attn_fwd_varlen,
-                                                   sa_check_status)
+                                                   sa_attn_decode_workspace_size, sa_attn_fwd,
+                                                   sa_attn_fwd_block_sparse, sa_attn_fwd_block_sparse_workspace_size,
+                                                   sa_attn_fwd_varlen, sa_check_status)
     from online_softmax_attention_sm_b200.dist import aggregate_throughput, max_over_ranks, rank_seed
-    from online_softmax_attention_sm_b200.inputs import make_qkv, make_workload_inputs
-    from online_softmax_attention_sm_b200.workloads import WORKLOADS
+    from online_softmax_attention_sm_b200.inputs import make_qkv, make_workload_inputs, stem_block_mask
+    from online_softmax_attention_sm_b200.workloads import WORKLOADS, block_sparse_flops
 
     rank, world, local = dist_env()
     if world > 1:
@@ -236,6 +237,7 @@ def main():
                                  Sk=args.prefill_seq)
     run_pre, run_dec = args.only in ("all", "prefill"), args.only in ("all", "decode")
     run_var = args.only in ("all", "varlen")
+    run_sparse = args.only in ("all", "sparse")
     q_h, k_h, v_h = make_workload_inputs(wp, seed=rank_seed(wp.seed, rank))
     dq_h, dk_h, dv_h = make_workload_inputs(wd, seed=rank_seed(wd.seed, rank))
     q, k, v = q_h.to(dev), k_h.to(dev), v_h.to(dev)
@@ -355,6 +357,30 @@ def main():
         var_ms = [a.elapsed_time(b) for a, b in vev]
         del vq, vk, vv, vo, vlse
 
+    # block-sparse prefill: the prefill workload's tensors under a Stem-shaped block mask
+    # (4 sink blocks, 4 window blocks, 10 % of the blocks between drawn at random); one API
+    # call = the list-building kernel + the block-sparse forward
+    sp_ms, sp_flops = [float("nan")], float("nan")
+    if run_sparse:
+        bmask = stem_block_mask(wp.B, wp.Hq, wp.Sq, wp.Sk, wp.causal, seed=wp.seed + 4)
+        sp_flops = block_sparse_flops(bmask.numpy(), wp.Sq, wp.Sk, wp.D, wp.causal)
+        bmask = bmask.to(dev)
+        sws = torch.empty(max(16, sa_attn_fwd_block_sparse_workspace_size(wp.B, wp.Sq, wp.Sk, wp.Hq)),
+                          dtype=torch.uint8, device=dev)
+        sev = []
+        for i in range(args.warmup + args.steps):
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            sa_attn_fwd_block_sparse(q, k, v, bmask, causal=wp.causal, scale=wp.scale, workspace=sws, out=o,
+                                     lse=lse, stream=stream)
+            e1.record(stream)
+            if i >= args.warmup:
+                sev.append((e0, e1))
+        torch.cuda.synchronize(dev)
+        sa_check_status(stream)
+        sp_ms = [a.elapsed_time(b) for a, b in sev]
+        del bmask, sws
+
     # e2e through the public API with host buffers: H2D of the step's inputs, D2H of outputs
     e2e_ms = None
     h2d = sum(t.numel() * t.element_size() for t in (q_h, k_h, v_h, dq_h, dk_h, dv_h))
@@ -389,6 +415,7 @@ def main():
     cold_avg = max_over_ranks(sum(cold_ms) / len(cold_ms), dev)
     paged_avg = max_over_ranks(sum(paged_ms) / len(paged_ms), dev)
     var_avg = max_over_ranks(sum(var_ms) / len(var_ms), dev)
+    sp_avg = max_over_ranks(sum(sp_ms) / len(sp_ms), dev)
     e2e_ms = max_over_ranks(e2e_ms, dev) if e2e_ms is not None else None
 
     if rank == 0:
@@ -436,6 +463,13 @@ def main():
                                "frac": wv.flops / (var_avg * 1e-3) / 1e12 / peak, "ms": var_avg,
                                "sequences": len(lens), "lengths": f"{min(lens)}-{max(lens)}",
                                "kernel": "attn_fwd_sm100 (dynamic unit order)"},
+            "prefill_block_sparse": {"workload": f"{PREFILL} + Stem-shaped block mask (4 sink, 4 window, "
+                                                 "10 % of the blocks between)",
+                                     "value": sp_flops / (sp_avg * 1e-3) / 1e12, "unit": "TFLOP/s",
+                                     "bound": "tensor", "peak": peak,
+                                     "frac": sp_flops / (sp_avg * 1e-3) / 1e12 / peak, "ms": sp_avg,
+                                     "work_vs_dense_causal": sp_flops / wp.flops,
+                                     "kernels": "sparse_unit_lists + attn_fwd_sm100 (block-sparse instance)"},
             "prefill_ms": pre_avg,
             "gpu_launches": (int(run_pre) + 2 * int(run_dec)) * args.steps,
             "clocks": clk.summary(),

@@ -99,6 +99,26 @@ int sa_attn_fwd_varlen(const void* q, const void* k, const void* v, void* o, flo
                        sa_stream_t stream);
 
 /*
+ * Block-sparse forward (Stem / AngelSlim page, section 2.3: attention over the 128 x 128
+ * blocks a top-k mask keeps, with the initial "sink" blocks and a sliding window of blocks
+ * among them).  Same tensors, layouts and rules as sa_attn_fwd, plus:
+ *   block_mask : device uint8 [B, Hq, ceil(Sq/128), ceil(Sk/128)], row-major; nonzero =
+ *                query block i attends key block j.  Key j is visible to query row i iff
+ *                sa_attn_fwd's rule allows it (causal: bottom-right) AND the mask keeps
+ *                block (i / 128, j / 128).  A row with no visible key: O = 0, LSE = -inf.
+ *   workspace  : device scratch of sa_attn_fwd_block_sparse_workspace_size() bytes,
+ *                16-byte aligned, no initial contents; it receives each work unit's list
+ *                of kept key blocks (a first kernel builds it from the mask).
+ * Kept blocks wholly past the causal diagonal cost nothing.  Sk <= 131072 (else
+ * SA_ERR_UNSUPPORTED); workspace missing or short: SA_ERR_WORKSPACE.
+ */
+size_t sa_attn_fwd_block_sparse_workspace_size(int B, int Sq, int Sk, int Hq);
+int sa_attn_fwd_block_sparse(const void* q, const void* k, const void* v, void* o, float* lse,
+                             const unsigned char* block_mask, int B, int Sq, int Sk, int Hq,
+                             int Hkv, int D, int causal, float scale, int dtype,
+                             void* workspace, size_t workspace_bytes, sa_stream_t stream);
+
+/*
  * Bytes of decode workspace needed for `num_splits` (0 = the automatic choice):
  * B * Hq * splits * (D + 4) * 4.  It holds, per (b, h, split), the split's running max
  * and two running sums (of the 16-bit weights the MMA used, and of the fp32 weights for

@@ -35,6 +35,16 @@
 
 namespace sa {
 
+constexpr int kUnitQueue = 4;    // unit indices the load warp may hand out ahead
+
+// Block-sparse forward: each unit's K/V tile list, one record per (batch, head, 256-row query
+// block), built by sparse_unit_lists from the caller's block mask.  A record is uint16:
+// [0] list length, [1] / [2] tiles of Q tile 0 / 1, [3..7] zero, then the list (order: see
+// sparse_unit_lists), each entry key tile | (Q tile 0 uses it) << 14 | (Q tile 1 uses it) << 15.
+// The load warp copies a unit's record into one of kUnitQueue shared-memory slots.
+constexpr int kSparseMaxKTiles = 1024;                       // keys <= 131072
+constexpr int kSparseSlotBytes = 16 + 2 * kSparseMaxKTiles;  // header + longest list
+
 template <int D>
 struct FwdCfg {
   static constexpr int BM = 128;                     // query rows per Q tile
@@ -47,6 +57,7 @@ struct FwdCfg {
   static constexpr int SMEM_RING = STAGES * TILE_BYTES;
   static constexpr int SMEM_BARS = 1024;
   static constexpr int SMEM_TOTAL = 1024 /*align slack*/ + SMEM_Q + SMEM_RING + SMEM_BARS;
+  static constexpr int SMEM_SPARSE = kUnitQueue * kSparseSlotBytes;   // block-sparse instance only
   static constexpr int THREADS = 384;                // 2 softmax WGs + load/MMA WG
   // per-thread registers after reallocation: softmax warpgroups / load+MMA warpgroup.
   // 2*128*REGS_SOFTMAX + 128*REGS_OTHER must not exceed the block's launch registers
@@ -87,16 +98,19 @@ struct FwdParams {
   const int* cu_q;
   const int* cu_k;
   int max_sq;
+  // Block-sparse (the kernel's SPARSE instance): unit records of sp_stride uint16 each,
+  // record (b * Hq + h) * n_qblk + query block.
+  const uint16_t* sp;
+  int sp_stride;
 };
-
-constexpr int kUnitQueue = 4;    // unit indices the load warp may hand out ahead
 
 struct UnitInfo {
   int b, h, kvh, q0;         // q0: first query row of the unit within its sequence
   int sq, sk;                // the sequence's query and key lengths
   int qbase, kbase, mb;      // its first query / key row and batch index in the TMA maps
   int nkv[2];                // K/V tiles needed by Q tile 0 / 1 (0: tile has no work)
-  int nkv_max;
+  int nkv_max;               // K/V steps of the unit (block-sparse: its list length)
+  const uint16_t* ent;       // block-sparse: the unit's list in shared memory
 };
 
 __device__ __forceinline__ int fwd_kv_tiles(int sq, int sk, int causal, int r0) {
@@ -195,6 +209,7 @@ struct FwdSmem {
   uint64_t* unit_full;   // [kUnitQueue]  unit index written by the load warp
   uint64_t* unit_empty;  // [kUnitQueue]  read by the MMA warp and the 8 softmax warps
   volatile int* uq;      // [kUnitQueue]  the unit indices
+  uint8_t* lists;        // [kUnitQueue][kSparseSlotBytes]  block-sparse unit records
   __device__ explicit FwdSmem(uint8_t* s) {
     q = s;
     ring = s + Cfg::SMEM_Q;
@@ -213,22 +228,44 @@ struct FwdSmem {
     unit_full = q_full + 14;
     unit_empty = unit_full + kUnitQueue;
     uq = (volatile int*)(unit_empty + kUnitQueue);
+    lists = s + Cfg::SMEM_Q + Cfg::SMEM_RING + Cfg::SMEM_BARS;
   }
 };
 
 // The n-th unit of this CTA, for a consuming warp: wait for the load warp to post it, read
-// it, release the queue slot (one arrival per warp).  Returns -1 if the wait gave up.
+// it, release the queue slot (one arrival per warp) unless the unit's shared-memory record
+// is still needed (block-sparse: released by fwd_release_unit at the unit's end).
+// Returns -1 if the wait gave up.
 template <int D>
-__device__ __forceinline__ int fwd_next_unit(const FwdSmem<D>& sm, int n, int where) {
+__device__ __forceinline__ int fwd_next_unit(const FwdSmem<D>& sm, int n, int where, bool release = true) {
   const int slot = n % kUnitQueue;
   if (!mbar_wait_warp(&sm.unit_full[slot], (n / kUnitQueue) & 1, sm.abort_flag, where)) return -1;
   const int u = sm.uq[slot];
-  mbar_arrive_warp(&sm.unit_empty[slot]);
+  if (release) mbar_arrive_warp(&sm.unit_empty[slot]);
   return u;
 }
 
+template <int D>
+__device__ __forceinline__ void fwd_release_unit(const FwdSmem<D>& sm, int n) {
+  mbar_arrive_warp(&sm.unit_empty[n % kUnitQueue]);
+}
+
+// Block-sparse: the record of unit x (global, in the caller's workspace) and its copy in
+// queue slot `slot` (shared memory), which sets the unit's step counts and list.
+__device__ __forceinline__ const uint16_t* fwd_sparse_record(const FwdParams& p, const UnitInfo& x) {
+  return p.sp + ((size_t)(x.b * p.Hq + x.h) * p.n_qblk + x.q0 / 256) * p.sp_stride;
+}
+template <int D>
+__device__ __forceinline__ void fwd_sparse_attach(const FwdSmem<D>& sm, int slot, UnitInfo& x) {
+  const uint16_t* rec = reinterpret_cast<const uint16_t*>(sm.lists + slot * kSparseSlotBytes);
+  x.nkv_max = rec[0];
+  x.nkv[0] = rec[1];
+  x.nkv[1] = rec[2];
+  x.ent = rec + 8;
+}
+
 // ------------------------------------------------------------------ TMA producer
-template <int D, bool BF16, bool DYN>
+template <int D, bool BF16, bool DYN, bool SPARSE>
 __device__ __forceinline__ void fwd_producer(const CUtensorMap* tm_q, const CUtensorMap* tm_k,
                                              const CUtensorMap* tm_v, const FwdParams& p,
                                              const FwdSmem<D>& sm, int lane, int cta, int ncta) {
@@ -236,10 +273,12 @@ __device__ __forceinline__ void fwd_producer(const CUtensorMap* tm_q, const CUte
   if (lane == 0) {
     int slot = 0, ring_n = 0;            // ring position and total loads issued
     int q_load0 = 0, q_load1 = 0;        // Q tile loads issued
+    int copy_n = -1;                     // block-sparse: unit whose record copy is in flight
     bool ok = true;
     for (int n = 0; ok; ++n) {
       // ---- the next unit (an index past the list ends the CTA), posted to the other roles
       int u;
+      UnitInfo x;
       if (!DYN) {
         u = fwd_unit_of(n, cta, ncta);       // every role computes the same index
       } else {
@@ -250,11 +289,25 @@ __device__ __forceinline__ void fwd_producer(const CUtensorMap* tm_q, const CUte
           if (!ok) break;
         }
         sm.uq[us] = u;
-        mbar_arrive(&sm.unit_full[us]);
+        if (SPARSE && u < p.n_units) {
+          // the unit's K/V tile list lands in the queue slot with the posting itself
+          x = fwd_unit(p, u);
+          const uint32_t bytes = (uint32_t)p.sp_stride * 2u;
+          mbar_arrive_expect_tx(&sm.unit_full[us], bytes);
+          bulk_copy_g2s(sm.lists + us * kSparseSlotBytes, fwd_sparse_record(p, x), bytes, &sm.unit_full[us]);
+          copy_n = n;
+          ok = mbar_wait(&sm.unit_full[us], (n / kUnitQueue) & 1, sm.abort_flag, 6);
+          if (!ok) break;
+          copy_n = -1;
+          fwd_sparse_attach(sm, us, x);
+        } else {
+          mbar_arrive(&sm.unit_full[us]);
+        }
       }
       if (u >= p.n_units) break;
-      UnitInfo x = fwd_unit(p, u);
+      if (!SPARSE) x = fwd_unit(p, u);
       for (int j = 0; j < x.nkv_max && ok; ++j) {
+        const int kt = SPARSE ? (int)(x.ent[j] & 0x3fffu) : j;   // key tile of this step
         for (int kv = 0; kv < 2 && ok; ++kv) {
           if (ring_n >= Cfg::STAGES) {
             ok = mbar_wait(&sm.kv_empty[slot], ((ring_n / Cfg::STAGES) - 1) & 1, sm.abort_flag, 1);
@@ -265,7 +318,7 @@ __device__ __forceinline__ void fwd_producer(const CUtensorMap* tm_q, const CUte
           const CUtensorMap* tm = kv ? tm_v : tm_k;
 #pragma unroll
           for (int c = 0; c < Cfg::KCH; ++c)
-            tma_load_4d(dst + c * Cfg::CHUNK_BYTES, tm, &sm.kv_full[slot], c * 64, x.kvh, x.kbase + j * 128, x.mb);
+            tma_load_4d(dst + c * Cfg::CHUNK_BYTES, tm, &sm.kv_full[slot], c * 64, x.kvh, x.kbase + kt * 128, x.mb);
           ++ring_n;
           slot = (slot + 1 == Cfg::STAGES) ? 0 : slot + 1;
           if (j == 0 && kv == 0) {
@@ -297,6 +350,8 @@ __device__ __forceinline__ void fwd_producer(const CUtensorMap* tm_q, const CUte
         mbar_wait(&sm.kv_full[n % Cfg::STAGES], (n / Cfg::STAGES) & 1, nullptr, 3);
       if (q_load0 > 0) mbar_wait(&sm.q_full[0], (q_load0 - 1) & 1, nullptr, 4);
       if (q_load1 > 0) mbar_wait(&sm.q_full[1], (q_load1 - 1) & 1, nullptr, 4);
+      if (SPARSE && copy_n >= 0)
+        mbar_wait(&sm.unit_full[copy_n % kUnitQueue], (copy_n / kUnitQueue) & 1, nullptr, 7);
     }
     // this CTA takes no more units; the last CTA to get here zeroes the launch's counters
     // for the next launch that uses them (nothing reads them after this point)
@@ -309,7 +364,7 @@ __device__ __forceinline__ void fwd_producer(const CUtensorMap* tm_q, const CUte
 }
 
 // ------------------------------------------------------------------ MMA issuer
-template <int D, bool BF16, bool DYN>
+template <int D, bool BF16, bool DYN, bool SPARSE>
 __device__ __forceinline__ void fwd_mma(const FwdParams& p, const FwdSmem<D>& sm, uint32_t tmem_base,
                                         int lane, int cta, int ncta) {
   using Cfg = FwdCfg<D>;
@@ -338,11 +393,23 @@ __device__ __forceinline__ void fwd_mma(const FwdParams& p, const FwdSmem<D>& sm
     // issue order, so the overwrite cannot overtake the read, and each softmax
     // warpgroup gets the other tile's PV + QK as cover for its exponentials.
     for (int n = 0; ok; ++n) {
-      const int u = DYN ? fwd_next_unit(sm, n, 12) : fwd_unit_of(n, cta, ncta);
+      const int u = DYN ? fwd_next_unit(sm, n, 12, !SPARSE) : fwd_unit_of(n, cta, ncta);
       if (u < 0) { ok = false; break; }
       if (u >= p.n_units) break;
       UnitInfo x = fwd_unit(p, u);
-      if (x.nkv_max == 0) continue;
+      if (SPARSE) fwd_sparse_attach(sm, n % kUnitQueue, x);
+      if (x.nkv_max == 0) {
+        if (SPARSE) fwd_release_unit(sm, n);
+        continue;
+      }
+      // whether Q tile t multiplies the K/V of step j: every step below its count (dense),
+      // the steps whose list entry carries its bit (block-sparse)
+      auto act = [&](int t, int j) -> bool {
+        if constexpr (SPARSE) return j < x.nkv_max && ((x.ent[j] >> (14 + t)) & 1u);
+        else return j < x.nkv[t];
+      };
+      int npv[2] = {0, 0};                     // block-sparse: P_t V products of this unit
+      bool q_wait[2] = {true, true};           // block-sparse: Q_t not yet waited for
       const int base = ring_n;                 // K(j) at base + 2j, V(j) at base + 2j + 1
       // ---- prologue: S_t = Q_t K_0^T
       {
@@ -351,9 +418,10 @@ __device__ __forceinline__ void fwd_mma(const FwdParams& p, const FwdSmem<D>& sm
         if (!ok) break;
         const uint32_t k_addr = sRing_addr + (pos % Cfg::STAGES) * Cfg::TILE_BYTES;
         for (int t = 0; t < 2 && ok; ++t) {
-          if (x.nkv[t] == 0) continue;
+          if (!act(t, 0)) continue;
           ok = mbar_wait_warp(&sm.q_full[t], (t ? q_use1 : q_use0) & 1, sm.abort_flag, 11);
           if (!ok) break;
+          q_wait[t] = false;
           tc_fence_after();
           issue_qk(t, k_addr);
         }
@@ -368,26 +436,37 @@ __device__ __forceinline__ void fwd_mma(const FwdParams& p, const FwdSmem<D>& sm
         const uint32_t k_addr = sRing_addr + (kpos % Cfg::STAGES) * Cfg::TILE_BYTES;
         bool k_ready = false;
         for (int t = 0; t < 2; ++t) {
-          if (j >= x.nkv[t]) continue;
-          // ---- O_t += P_t V_j: keys 0-95 as soon as their P is written, then 96-127
-          ok = mbar_wait_warp(&sm.p_part[t], (t ? pv1 : pv0) & 1, sm.abort_flag, 17);
-          if (!ok) break;
-          tc_fence_after();
-          mma_ts_x6(tmem_base + Cfg::O_COL(t), tmem_base + Cfg::P_COL(t),
-                    smem_desc_sw128(v_addr, Cfg::CHUNK_BYTES, 1024), IDESC_PV, j > 0 ? 1u : 0u);
-          ok = mbar_wait_warp(&sm.p_full[t], (t ? pv1 : pv0) & 1, sm.abort_flag, 14);
-          if (!ok) break;
-          tc_fence_after();
-          mma_ts_x2(tmem_base + Cfg::O_COL(t), tmem_base + Cfg::P_COL(t) + 6 * 8,
-                    smem_desc_sw128(v_addr + 6 * 2048, Cfg::CHUNK_BYTES, 1024), IDESC_PV, 1u);
-          if (j + 1 == x.nkv[t]) mma_commit_warp(&sm.o_done[t]);   // O_t complete for the epilogue
-          if (t) ++pv1; else ++pv0;
+          if (!SPARSE && j >= x.nkv[t]) continue;
+          if (act(t, j)) {
+            // ---- O_t += P_t V_j: keys 0-95 as soon as their P is written, then 96-127
+            ok = mbar_wait_warp(&sm.p_part[t], (t ? pv1 : pv0) & 1, sm.abort_flag, 17);
+            if (!ok) break;
+            tc_fence_after();
+            const uint32_t acc = SPARSE ? (npv[t] > 0 ? 1u : 0u) : (j > 0 ? 1u : 0u);
+            mma_ts_x6(tmem_base + Cfg::O_COL(t), tmem_base + Cfg::P_COL(t),
+                      smem_desc_sw128(v_addr, Cfg::CHUNK_BYTES, 1024), IDESC_PV, acc);
+            ok = mbar_wait_warp(&sm.p_full[t], (t ? pv1 : pv0) & 1, sm.abort_flag, 14);
+            if (!ok) break;
+            tc_fence_after();
+            mma_ts_x2(tmem_base + Cfg::O_COL(t), tmem_base + Cfg::P_COL(t) + 6 * 8,
+                      smem_desc_sw128(v_addr + 6 * 2048, Cfg::CHUNK_BYTES, 1024), IDESC_PV, 1u);
+            const bool last = SPARSE ? (++npv[t] == x.nkv[t]) : (j + 1 == x.nkv[t]);
+            if (last) mma_commit_warp(&sm.o_done[t]);   // O_t complete for the epilogue
+            if (t) ++pv1; else ++pv0;
+          }
           // ---- S_t = Q_t K_{j+1}^T
-          if (j + 1 < x.nkv[t]) {
+          if (act(t, j + 1)) {
             if (!k_ready) {
               ok = mbar_wait_warp(&sm.kv_full[kpos % Cfg::STAGES], (kpos / Cfg::STAGES) & 1, sm.abort_flag, 10);
               if (!ok) break;
               k_ready = true;
+            }
+            if (SPARSE && q_wait[t]) {
+              // block-sparse: a Q tile whose first K/V step is not the unit's first
+              ok = mbar_wait_warp(&sm.q_full[t], (t ? q_use1 : q_use0) & 1, sm.abort_flag, 11);
+              if (!ok) break;
+              q_wait[t] = false;
+              tc_fence_after();
             }
             issue_qk(t, k_addr);
           }
@@ -407,6 +486,7 @@ __device__ __forceinline__ void fwd_mma(const FwdParams& p, const FwdSmem<D>& sm
       ring_n = base + 2 * x.nkv_max;
       if (x.nkv[0] > 0) { mma_commit_warp(&sm.q_empty[0]); ++q_use0; }
       if (x.nkv[1] > 0) { mma_commit_warp(&sm.q_empty[1]); ++q_use1; }
+      if (SPARSE) fwd_release_unit(sm, n);
     }
     // every MMA issued above completes before tensor memory is released
     mma_commit_warp(sm.fin);
@@ -615,7 +695,7 @@ __device__ __forceinline__ void softmax_tile_masked(const uint32_t s_addr, const
   sum_f2x2(rse2, l_lse);
 }
 
-template <int D, bool BF16, bool DYN>
+template <int D, bool BF16, bool DYN, bool SPARSE>
 __device__ __forceinline__ void fwd_softmax(const FwdParams& p, const FwdSmem<D>& sm, uint32_t tmem_base,
                                             int warp, int lane, int cta, int ncta) {
   using Cfg = FwdCfg<D>;
@@ -627,10 +707,11 @@ __device__ __forceinline__ void fwd_softmax(const FwdParams& p, const FwdSmem<D>
   int s_n = 0, o_n = 0;                     // s_full / o_done phases consumed (o_done: one per unit)
   bool ok = true;
   for (int n = 0; ok; ++n) {
-    const int u = DYN ? fwd_next_unit(sm, n, 23) : fwd_unit_of(n, cta, ncta);
+    const int u = DYN ? fwd_next_unit(sm, n, 23, !SPARSE) : fwd_unit_of(n, cta, ncta);
     if (u < 0) { ok = false; break; }
     if (u >= p.n_units) break;
     UnitInfo x = fwd_unit(p, u);
+    if (SPARSE) fwd_sparse_attach(sm, n % kUnitQueue, x);
     const int nkv = x.nkv[t];
     const int row = x.q0 + t * 128 + row_in_tile;
     int klim = x.sk;
@@ -645,21 +726,30 @@ __device__ __forceinline__ void fwd_softmax(const FwdParams& p, const FwdSmem<D>
     float m_ref = -INFINITY, l_sum = 0.f, l_lse = 0.f;
     const uint32_t s_addr = lane_addr + Cfg::S_COL(t), o_addr = lane_addr + Cfg::O_COL(t);
     const uint32_t p_addr = lane_addr + Cfg::P_COL(t);
-    for (int j = 0; j < nkv; ++j) {
+    int i = 0;                              // block-sparse: this tile's K/V steps so far
+    for (int j = 0; j < (SPARSE ? x.nkv_max : nkv); ++j) {
+      int kt = j;                           // key tile of the step
+      if constexpr (SPARSE) {
+        const uint32_t e = x.ent[j];
+        if (!((e >> (14 + t)) & 1u)) continue;
+        kt = (int)(e & 0x3fffu);
+      }
+      const bool first = SPARSE ? (i == 0) : (j == 0);
       ok = mbar_wait_warp(&sm.s_full[t], s_n & 1, sm.abort_flag, 20 + t);
       if (!ok) break;
       ++s_n;
       tc_fence_after();
-      if (j < mask_from && c2 >= 0.f) {
-        softmax_tile_full<D, BF16>(s_addr, o_addr, p_addr, c2, j == 0, m_ref, l_sum, l_lse, &sm.p_part[t]);
+      if (kt < mask_from && c2 >= 0.f) {
+        softmax_tile_full<D, BF16>(s_addr, o_addr, p_addr, c2, first, m_ref, l_sum, l_lse, &sm.p_part[t]);
       } else {
-        const int kl = (j >= mask_from) ? klim - j * 128 : 128;   // keys >= kl: invisible to this row
-        softmax_tile_masked<D, BF16>(s_addr, o_addr, p_addr, c2, kl, j == 0, m_ref, l_sum, l_lse,
+        const int kl = (kt >= mask_from) ? klim - kt * 128 : 128;   // keys >= kl: invisible to this row
+        softmax_tile_masked<D, BF16>(s_addr, o_addr, p_addr, c2, kl, first, m_ref, l_sum, l_lse,
                                      &sm.p_part[t]);
       }
       tmem_wait_st();
       tc_fence_before();
       mbar_arrive(&sm.p_full[t]);
+      if (SPARSE) ++i;
     }
     if (!ok) break;
     // ---------------- epilogue: O / l, LSE
@@ -706,6 +796,7 @@ __device__ __forceinline__ void fwd_softmax(const FwdParams& p, const FwdSmem<D>
       p.lse[((size_t)x.mb * p.Hq + x.h) * p.Sq + x.qbase + row] = lse;
     }
     tc_fence_before();
+    if (SPARSE) fwd_release_unit(sm, n);
   }
 }
 
@@ -720,11 +811,12 @@ __device__ __forceinline__ void fwd_teardown(bool owner, uint32_t tmem_base, uin
   }
 }
 
-template <int D, bool BF16, bool DYN>
+template <int D, bool BF16, bool DYN, bool SPARSE>
 __global__ void __launch_bounds__(384, 1)
 attn_fwd_sm100(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                const __grid_constant__ CUtensorMap tm_v, const FwdParams p) {
   using Cfg = FwdCfg<D>;
+  static_assert(DYN || !SPARSE, "the block-sparse units go through the dynamic unit queue");
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
   const FwdSmem<D> sm(smem);
@@ -762,15 +854,16 @@ attn_fwd_sm100(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
     // load / MMA warpgroup gives registers away; warp 2 checks packed sequence offsets,
     // warp 3 has no role
     regs_dec<Cfg::REGS_OTHER>();
-    if (warp == kWarpLoad) fwd_producer<D, BF16, DYN>(&tm_q, &tm_k, &tm_v, p, sm, lane, cta, ncta);
-    else if (warp == kWarpMma) fwd_mma<D, BF16, DYN>(p, sm, tmem_base, lane, cta, ncta);
+    if (warp == kWarpLoad) fwd_producer<D, BF16, DYN, SPARSE>(&tm_q, &tm_k, &tm_v, p, sm, lane, cta, ncta);
+    else if (warp == kWarpMma) fwd_mma<D, BF16, DYN, SPARSE>(p, sm, tmem_base, lane, cta, ncta);
     else if (warp == 2 && p.cu_q) fwd_check_lengths(p, lane, cta, ncta);
     fwd_teardown(warp == kWarpMma, tmem_base, Cfg::TMEM_COLS);
   } else {
     regs_inc<Cfg::REGS_SOFTMAX>();
-    fwd_softmax<D, BF16, DYN>(p, sm, tmem_base, warp - 4, lane, cta, ncta);
+    fwd_softmax<D, BF16, DYN, SPARSE>(p, sm, tmem_base, warp - 4, lane, cta, ncta);
     fwd_teardown(false, tmem_base, Cfg::TMEM_COLS);
   }
 }
 
 }  // namespace sa
+

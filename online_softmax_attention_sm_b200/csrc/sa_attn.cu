@@ -4,6 +4,7 @@
 #include "../../include/sa_attn.h"
 #include "ptx.cuh"
 #include "fwd_sm100.cuh"
+#include "sparse_lists.cuh"
 #include "fwd_simple.cuh"
 #include "decode.cuh"
 
@@ -198,12 +199,23 @@ struct FwdVarlen {
   int max_sq = 0, max_sk = 0;
 };
 
+// Block-sparse unit records for launch_fwd (sp null: every key tile up to the diagonal).
+struct FwdSparse {
+  const uint16_t* sp = nullptr;
+  int stride = 0;   // uint16 per record
+};
+
+// uint16 per block-sparse unit record for Sk keys: 8 header slots + the longest list,
+// rounded up to 16 bytes.
+int sparse_stride(int Sk) { return 8 + (((Sk + 127) / 128 + 7) / 8) * 8; }
+
 // Dense: q/o [B, Sq, Hq, D], k/v [B, Sk, Hkv, D].  Packed (vl.cu_q set): B sequences,
 // q/o [Sq, Hq, D] and k/v [Sk, Hkv, D] with Sq, Sk the totals, LSE [Hq, Sq].
+// Block-sparse (sparse.sp set, dense layout): the unit records built by sparse_unit_lists.
 template <int D, bool BF16>
 int launch_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Sq,
                int Sk, int Hq, int Hkv, int causal, float scale, cudaStream_t st,
-               const FwdVarlen& vl = FwdVarlen()) {
+               const FwdVarlen& vl = FwdVarlen(), const FwdSparse& sparse = FwdSparse()) {
   using Cfg = sa::FwdCfg<D>;
   const bool packed = vl.cu_q != nullptr;
   const int map_b = packed ? 1 : B;
@@ -217,6 +229,7 @@ int launch_fwd(const void* q, const void* k, const void* v, void* o, float* lse,
   p.B = B; p.Sq = Sq; p.Sk = Sk; p.Hq = Hq; p.Hkv = Hkv; p.causal = causal;
   p.cu_q = vl.cu_q; p.cu_k = vl.cu_k;
   p.max_sq = packed ? vl.max_sq : Sq;
+  p.sp = sparse.sp; p.sp_stride = sparse.stride;
   const int seq_k = packed ? (vl.max_sk > 0 ? vl.max_sk : 1) : Sk;   // one sequence's keys, for L2 grouping
   p.n_qblk = (p.max_sq + 255) / 256;
   long long units = (long long)B * Hq * p.n_qblk;
@@ -259,10 +272,13 @@ int launch_fwd(const void* q, const void* k, const void* v, void* o, float* lse,
     }
   }
   const int grid = p.n_units < num_sms() ? p.n_units : num_sms();
-  // packed lengths live on the device, so the static order's balance is unknown: dynamic
-  auto kern = (packed || fwd_use_dynamic(p, D, grid)) ? sa::attn_fwd_sm100<D, BF16, true>
-                                                      : sa::attn_fwd_sm100<D, BF16, false>;
-  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::SMEM_TOTAL);
+  // packed lengths and block-sparse lists live on the device, so the static order's
+  // balance is unknown: dynamic
+  auto kern = sparse.sp ? sa::attn_fwd_sm100<D, BF16, true, true>
+            : (packed || fwd_use_dynamic(p, D, grid)) ? sa::attn_fwd_sm100<D, BF16, true, false>
+                                                      : sa::attn_fwd_sm100<D, BF16, false, false>;
+  const int smem = Cfg::SMEM_TOTAL + (sparse.sp ? Cfg::SMEM_SPARSE : 0);
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(attn_fwd_sm100)");
   // the in-kernel register reallocation must fit in what the block is launched with,
   // otherwise the increasing warpgroups would wait forever
@@ -272,7 +288,7 @@ int launch_fwd(const void* q, const void* k, const void* v, void* o, float* lse,
   if ((long long)fa.numRegs * Cfg::THREADS < 256LL * Cfg::REGS_SOFTMAX + 128LL * Cfg::REGS_OTHER)
     return fail(SA_ERR_UNSUPPORTED, "attn_fwd_sm100 launches with %d registers per thread, too few for "
                 "its register split", fa.numRegs);
-  kern<<<grid, Cfg::THREADS, Cfg::SMEM_TOTAL, st>>>(mq, mk, mv, p);
+  kern<<<grid, Cfg::THREADS, smem, st>>>(mq, mk, mv, p);
   e = cudaGetLastError();
   return e == cudaSuccess ? SA_OK : cuda_fail(e, "attn_fwd_sm100 launch");
 }
@@ -443,6 +459,51 @@ int sa_attn_fwd_varlen(const void* q, const void* k, const void* v, void* o, flo
               : launch_fwd<64, false>(q, k, v, o, lse, B, total_q, total_k, Hq, Hkv, causal, scale, st, vl);
   return bf ? launch_fwd<128, true>(q, k, v, o, lse, B, total_q, total_k, Hq, Hkv, causal, scale, st, vl)
             : launch_fwd<128, false>(q, k, v, o, lse, B, total_q, total_k, Hq, Hkv, causal, scale, st, vl);
+}
+
+size_t sa_attn_fwd_block_sparse_workspace_size(int B, int Sq, int Sk, int Hq) {
+  if (B <= 0 || Sq <= 0 || Sk <= 0 || Hq <= 0) return 0;
+  if ((Sk + 127) / 128 > sa::kSparseMaxKTiles) return 0;
+  return (size_t)B * Hq * ((Sq + 255) / 256) * sparse_stride(Sk) * sizeof(uint16_t);
+}
+
+int sa_attn_fwd_block_sparse(const void* q, const void* k, const void* v, void* o, float* lse,
+                             const unsigned char* block_mask, int B, int Sq, int Sk, int Hq, int Hkv,
+                             int D, int causal, float scale, int dtype, void* workspace,
+                             size_t workspace_bytes, sa_stream_t stream) {
+  int rc = check_dims(B, Sq, Sk, Hq, Hkv, D, dtype, scale);
+  if (rc != SA_OK) return rc;
+  if (causal != 0 && causal != 1) return fail(SA_ERR_INVALID, "causal must be 0 or 1");
+  if (B == 0 || Sq == 0 || Hq == 0) return SA_OK;
+  if ((rc = check_ptrs(q, Sk ? k : q, Sk ? v : q, o, lse)) != SA_OK) return rc;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  if (Sk == 0) return launch_fill(o, (size_t)B * Sq * Hq * D, lse, (size_t)B * Hq * Sq, st);
+  if (!block_mask) return fail(SA_ERR_INVALID, "block_mask must be non-null");
+  if ((Sk + 127) / 128 > sa::kSparseMaxKTiles)
+    return fail(SA_ERR_UNSUPPORTED, "block-sparse forward supports at most %d keys (Sk=%d)",
+                sa::kSparseMaxKTiles * 128, Sk);
+  const size_t need = sa_attn_fwd_block_sparse_workspace_size(B, Sq, Sk, Hq);
+  if (!workspace || workspace_bytes < need)
+    return fail(SA_ERR_WORKSPACE, "block-sparse workspace of %zu bytes needed, %zu given", need,
+                workspace ? workspace_bytes : (size_t)0);
+  if (!aligned16(workspace)) return fail(SA_ERR_INVALID, "workspace must be 16-byte aligned");
+  const int n_qblk = (Sq + 255) / 256;
+  const long long n_rec = (long long)B * Hq * n_qblk;
+  if (n_rec > 0x7fffffffLL) return fail(SA_ERR_UNSUPPORTED, "too many work units (%lld)", n_rec);
+  FwdSparse sp;
+  sp.sp = static_cast<const uint16_t*>(workspace);
+  sp.stride = sparse_stride(Sk);
+  sa::sparse_unit_lists<<<(unsigned)((n_rec + 7) / 8), 256, 0, st>>>(
+      block_mask, static_cast<uint16_t*>(workspace), B, Hq, Sq, Sk, causal, n_qblk, sp.stride);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return cuda_fail(e, "sparse_unit_lists launch");
+  const bool bf = dtype == SA_BF16;
+  const FwdVarlen none;
+  if (D == 64)
+    return bf ? launch_fwd<64, true>(q, k, v, o, lse, B, Sq, Sk, Hq, Hkv, causal, scale, st, none, sp)
+              : launch_fwd<64, false>(q, k, v, o, lse, B, Sq, Sk, Hq, Hkv, causal, scale, st, none, sp);
+  return bf ? launch_fwd<128, true>(q, k, v, o, lse, B, Sq, Sk, Hq, Hkv, causal, scale, st, none, sp)
+            : launch_fwd<128, false>(q, k, v, o, lse, B, Sq, Sk, Hq, Hkv, causal, scale, st, none, sp);
 }
 
 int sa_attn_fwd_simple(const void* q, const void* k, const void* v, void* o, float* lse, int B,

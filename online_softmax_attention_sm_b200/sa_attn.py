@@ -25,6 +25,8 @@ SIGNATURES = {
     "sa_attn_fwd": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _F, _I, _P]),
     "sa_attn_fwd_simple": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _F, _I, _P]),
     "sa_attn_fwd_varlen": (_I, [_P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _I, _I, _F, _I, _P]),
+    "sa_attn_fwd_block_sparse_workspace_size": (_Z, [_I, _I, _I, _I]),
+    "sa_attn_fwd_block_sparse": (_I, [_P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _F, _I, _P, _Z, _P]),
     "sa_attn_decode_workspace_size": (_Z, [_I, _I, _I, _I, _I, _I]),
     "sa_attn_decode_num_splits": (_I, [_I, _I, _I, _I, _I]),
     "sa_attn_decode": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _F, _I, _I, _P, _Z, _P]),
@@ -146,6 +148,46 @@ def sa_attn_fwd_varlen(q, k, v, cu_seqlens_q, cu_seqlens_k, max_seqlen_q, max_se
                                     _ptr(cu_seqlens_k), B, int(max_seqlen_q), int(max_seqlen_k), total_q,
                                     total_k, Hq, Hkv, D, int(bool(causal)), float(scale), _DT[q.dtype],
                                     _stream(stream)))
+    return out, lse
+
+
+def sa_attn_fwd_block_sparse_workspace_size(B, Sq, Sk, Hq):
+    return int(lib().sa_attn_fwd_block_sparse_workspace_size(B, Sq, Sk, Hq))
+
+
+def sa_attn_fwd_block_sparse(q, k, v, block_mask, causal=False, scale=None, workspace=None, out=None,
+                             lse=None, return_lse=True, stream=None):
+    """Block-sparse attention forward.  q [B,Sq,Hq,D], k/v [B,Sk,Hkv,D] (fp16/bf16, CUDA,
+    contiguous); block_mask uint8 [B,Hq,ceil(Sq/128),ceil(Sk/128)] on the same device
+    (nonzero = keep).  Returns (o [B,Sq,Hq,D], lse [B,Hq,Sq] fp32 or None)."""
+    B, Sq, Hq, D = q.shape
+    Sk, Hkv = k.shape[1], k.shape[2]
+    if k.shape != (B, Sk, Hkv, D) or v.shape != k.shape:
+        raise ValueError(f"shape mismatch q{tuple(q.shape)} k{tuple(k.shape)} v{tuple(v.shape)}")
+    if q.dtype not in _DT:
+        raise TypeError(f"unsupported dtype {q.dtype}")
+    for n, t in (("q", q), ("k", k), ("v", v)):
+        _check_tensor(n, t, q.dtype, q.device)
+    _check_tensor("block_mask", block_mask, torch.uint8, q.device)
+    want = (B, Hq, -(-Sq // 128), -(-Sk // 128))
+    if tuple(block_mask.shape) != want:
+        raise ValueError(f"block_mask must be {want}, got {tuple(block_mask.shape)}")
+    if scale is None:
+        scale = 1.0 / math.sqrt(D)
+    if out is None:
+        out = torch.empty_like(q)
+    _check_tensor("out", out, q.dtype, q.device)
+    if return_lse and lse is None:
+        lse = torch.empty((B, Hq, Sq), dtype=torch.float32, device=q.device)
+    if lse is not None:
+        _check_tensor("lse", lse, torch.float32, q.device)
+    need = sa_attn_fwd_block_sparse_workspace_size(B, Sq, Sk, Hq)
+    if workspace is None:
+        workspace = torch.empty(max(need, 16), dtype=torch.uint8, device=q.device)
+    _check(lib().sa_attn_fwd_block_sparse(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse), _ptr(block_mask),
+                                          B, Sq, Sk, Hq, Hkv, D, int(bool(causal)), float(scale), _DT[q.dtype],
+                                          _ptr(workspace), workspace.numel() * workspace.element_size(),
+                                          _stream(stream)))
     return out, lse
 
 

@@ -62,6 +62,25 @@ class Workload:
         return 2 * self.B * self.Sk * self.Hkv * self.D * 2
 
 
+def block_sparse_flops(mask, Sq, Sk, D, causal, block=128):
+    """Forward FLOPs of a block-sparse launch: 4*D per visible (row, key) pair, pairs
+    counted per kept block of `mask` [..., ceil(Sq/block), ceil(Sk/block)] under the dense
+    visibility rule (causal: key j <= row + Sk - Sq).  Unlike the dense causal convention
+    (S*S/2), the diagonal blocks count exactly."""
+    import numpy as np
+    m = np.asarray(mask) != 0
+    nq, nk = m.shape[-2], m.shape[-1]
+    rows = np.arange(Sq)
+    limit = np.clip(rows + Sk - Sq + 1, 0, Sk) if causal else np.full(Sq, Sk)
+    per_block = np.zeros((nq, nk), dtype=np.int64)
+    for ki in range(nk):
+        c0 = ki * block
+        width = min(block, Sk - c0)
+        seen = np.clip(limit - c0, 0, width)                   # keys of this block each row sees
+        per_block[:, ki] = np.add.reduceat(seen, np.arange(0, Sq, block))
+    return 4.0 * D * float((m.reshape(-1, nq, nk).sum(axis=0) * per_block).sum())
+
+
 WORKLOADS = {
     w.name: w
     for w in [

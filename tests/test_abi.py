@@ -202,6 +202,42 @@ def test_fwd_varlen_empty_problem_is_a_no_op(L, kw):
     assert fwd_varlen(L, **args) == sa.SA_OK
 
 
+def fwd_sparse(L, q=FAKE, k=FAKE, v=FAKE, o=FAKE, lse=NULL, m=FAKE, B=1, Sq=256, Sk=256, Hq=2, Hkv=1, D=64,
+               causal=1, scale=0.125, dtype=0, ws=FAKE, wsb=1 << 20):
+    return L.sa_attn_fwd_block_sparse(q, k, v, o, lse, m, B, Sq, Sk, Hq, Hkv, D, causal, scale, dtype, ws, wsb,
+                                      None)
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(q=NULL), sa.SA_ERR_INVALID),
+    (dict(m=NULL), sa.SA_ERR_INVALID),
+    (dict(Hq=3, Hkv=2), sa.SA_ERR_INVALID),
+    (dict(D=80), sa.SA_ERR_UNSUPPORTED),
+    (dict(causal=2), sa.SA_ERR_INVALID),
+    (dict(scale=math.inf), sa.SA_ERR_INVALID),
+    (dict(ws=NULL), sa.SA_ERR_WORKSPACE),
+    (dict(wsb=32), sa.SA_ERR_WORKSPACE),
+    (dict(ws=ctypes.c_void_p((1 << 20) + 8)), sa.SA_ERR_INVALID),
+    (dict(Sk=131072 + 1), sa.SA_ERR_UNSUPPORTED),
+])
+def test_fwd_block_sparse_rejects_invalid_arguments(L, kw, code):
+    assert fwd_sparse(L, **kw) == code
+
+
+def test_fwd_block_sparse_empty_is_a_no_op(L):
+    assert fwd_sparse(L, q=NULL, k=NULL, v=NULL, o=NULL, m=NULL, ws=NULL, B=0) == sa.SA_OK
+
+
+def test_block_sparse_workspace_size(L):
+    # one record per (batch, head, 256-row query block): 8 header slots + the longest list,
+    # rounded up to 16 bytes, in uint16
+    assert L.sa_attn_fwd_block_sparse_workspace_size(1, 256, 256, 2) == 2 * (8 + 8) * 2
+    assert L.sa_attn_fwd_block_sparse_workspace_size(2, 32768, 32768, 32) == 2 * 32 * 128 * (8 + 256) * 2
+    assert L.sa_attn_fwd_block_sparse_workspace_size(1, 300, 1300, 3) == 3 * 2 * (8 + 16) * 2
+    assert L.sa_attn_fwd_block_sparse_workspace_size(1, 256, 131072 + 1, 2) == 0
+    assert L.sa_attn_fwd_block_sparse_workspace_size(0, 256, 256, 2) == 0
+
+
 def test_version(L):
     assert re.fullmatch(r"\d+\.\d+\.\d+", sa.sa_version())
 

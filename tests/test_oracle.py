@@ -511,3 +511,11 @@ def test_block_sparse_pair_count_by_brute_force(causal):
     ones = np.ones((1, 1, 3, 3), np.uint8)
     assert block_sparse_pairs(12, 12, ones, True, block=4) == 12 * 13 // 2
     assert block_sparse_pairs(12, 12, ones, False, block=4) == 144
+
+
+def test_bench_block_sparse_flop_count_matches_the_oracle_count():
+    from online_softmax_attention_sm_b200.workloads import block_sparse_flops
+    for Sq, Sk, causal, seed in ((10, 14, True, 1), (13, 9, True, 2), (12, 12, False, 3), (7, 20, True, 4)):
+        m = rand_mask(2, 3, -(-Sq // 4), -(-Sk // 4), 0.5, seed)
+        assert block_sparse_flops(m, Sq, Sk, 8, causal, block=4) == 4 * 8 * block_sparse_pairs(Sq, Sk, m, causal,
+                                                                                               block=4)
