@@ -233,6 +233,48 @@ def block_sparse_pairs(Sq, Sk, block_mask, causal, block=128):
     return int((bm.reshape(-1, nq, nk) * per_block[None]).sum())
 
 
+def attention_backward(q, k, v, do, scale, causal=False):
+    """Gradients of the forward's output O with respect to q, k, v for an upstream
+    gradient dO (the StreamAttention page, "Backward": recompute the probabilities from the
+    saved LSE and stream dQ/dK/dV; the flash-attn-volta page's backward follows the same
+    algorithm).  With P = softmax over the visible keys (the forward's rule) and O = P V:
+        dV    = P^T dO                       (summed over the query heads of a KV head)
+        dP    = dO V^T
+        Delta = rowsum(dO * O)  (= rowsum(P * dP))
+        dS    = P * (dP - Delta)             (zero at invisible keys)
+        dQ    = scale * dS K,   dK = scale * dS^T Q   (dK summed like dV)
+    q [B,Sq,Hq,D], k/v [B,Sk,Hkv,D], do [B,Sq,Hq,D].  Returns dQ, dK, dV in float64 with the
+    shapes of q, k, v.  Rows without a visible key have P = 0 and contribute nothing."""
+    q, k, v, do = _f64(q), _f64(k), _f64(v), _f64(do)
+    B, Sq, Hq, D = q.shape
+    Sk, Hkv = k.shape[1], k.shape[2]
+    if Hkv == 0 or Hq % Hkv:
+        raise ValueError("Hq must be a positive multiple of Hkv")
+    G = Hq // Hkv
+    dq, dk, dv = np.zeros_like(q), np.zeros_like(k), np.zeros_like(v)
+    if Sq == 0 or Sk == 0:
+        return dq, dk, dv
+    vis = _visible(Sq, Sk, causal)
+    has = vis.any(axis=1)
+    for b in range(B):
+        for h in range(Hq):
+            kvh = h // G
+            qm, km, vm, dom = q[b, :, h, :], k[b, :, kvh, :], v[b, :, kvh, :], do[b, :, h, :]
+            s = np.where(vis, scale * (qm @ km.T), NEG_INF)
+            p = np.zeros_like(s)
+            m = s[has].max(axis=1)
+            e = np.exp(s[has] - m[:, None])
+            p[has] = e / e.sum(axis=1, keepdims=True)
+            o = p @ vm
+            dv[b, :, kvh, :] += p.T @ dom
+            dp = dom @ vm.T
+            delta = (dom * o).sum(axis=1)
+            ds = p * (dp - delta[:, None])
+            dq[b, :, h, :] = scale * (ds @ km)
+            dk[b, :, kvh, :] += scale * (ds.T @ qm)
+    return dq, dk, dv
+
+
 def attention_blockwise(q, k, v, scale, causal=False, block=64):
     """The online-softmax recurrence, restated in float64 (TurboQuant page,
     ``online_softmax_attention``; StreamAttention page, "Kernel Design"): walk the

@@ -12,7 +12,7 @@ import numpy as np
 import pytest
 
 from oracle import (attention, attention_rows, attention_blockwise, attention_varlen, attention_block_sparse,
-                    attention_block_sparse_rows, block_sparse_pairs, decode, decode_paged,
+                    attention_block_sparse_rows, block_sparse_pairs, attention_backward, decode, decode_paged,
                     combine_lse)
 
 GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
@@ -519,3 +519,78 @@ def test_bench_block_sparse_flop_count_matches_the_oracle_count():
         m = rand_mask(2, 3, -(-Sq // 4), -(-Sk // 4), 0.5, seed)
         assert block_sparse_flops(m, Sq, Sk, 8, causal, block=4) == 4 * 8 * block_sparse_pairs(Sq, Sk, m, causal,
                                                                                                block=4)
+
+
+# ---- backward: gradients of L = sum(O * dO)
+
+def loss(q, k, v, do, scale, causal):
+    O, _ = attention(q, k, v, scale, causal)
+    return float((O * do).sum())
+
+
+@pytest.mark.parametrize("causal,Sq,Sk", [(False, 3, 4), (True, 4, 4), (True, 3, 5)])
+def test_backward_matches_central_differences(causal, Sq, Sk):
+    # brute force: every input element perturbed by +-eps, the loss re-evaluated
+    q, k, v = qkv(B=1, Sq=Sq, Sk=Sk, Hq=2, Hkv=1, D=3, seed=71)
+    do = rnd(q.shape, 72)
+    dq, dk, dv = attention_backward(q, k, v, do, 0.7, causal)
+    eps = 1e-6
+    for x, g in ((q, dq), (k, dk), (v, dv)):
+        num = np.zeros_like(x)
+        for idx in np.ndindex(*x.shape):
+            old = x[idx]
+            x[idx] = old + eps
+            lp = loss(q, k, v, do, 0.7, causal)
+            x[idx] = old - eps
+            lm = loss(q, k, v, do, 0.7, causal)
+            x[idx] = old
+            num[idx] = (lp - lm) / (2 * eps)
+        np.testing.assert_allclose(g, num, atol=1e-7)
+
+
+def test_backward_zero_query_dv_is_the_mean_of_do():
+    # Q = 0: uniform weights over the visible keys, so dV_j = sum over rows i that see j
+    # of dO_i / |V_i|
+    Sq, Sk = 5, 5
+    q, k, v = qkv(B=1, Sq=Sq, Sk=Sk, Hq=1, Hkv=1, D=4, seed=73)
+    q[:] = 0
+    do = rnd(q.shape, 74)
+    _, _, dv = attention_backward(q, k, v, do, 1.0, True)
+    want = np.zeros((Sk, 4))
+    for i in range(Sq):
+        n = visible_count(i, Sq, Sk, True)
+        want[:n] += do[0, i, 0] / n
+    np.testing.assert_allclose(dv[0, :, 0], want, atol=TOL)
+
+
+def test_backward_equal_keys_give_zero_dq():
+    # all keys equal: every score of a row is the same, so moving q changes nothing
+    q, k, v = qkv(B=1, Sq=4, Sk=6, Hq=2, Hkv=2, D=5, seed=75)
+    k[:] = k[:, :1]
+    do = rnd(q.shape, 76)
+    dq, _, _ = attention_backward(q, k, v, do, 0.9, False)
+    np.testing.assert_allclose(dq, 0, atol=TOL)
+
+
+def test_backward_gqa_is_mha_on_repeated_kv_summed():
+    q, k, v = qkv(B=2, Sq=5, Sk=6, Hq=4, Hkv=2, D=3, seed=77)
+    do = rnd(q.shape, 78)
+    dq, dk, dv = attention_backward(q, k, v, do, 0.5, True)
+    kr, vr = np.repeat(k, 2, axis=2), np.repeat(v, 2, axis=2)
+    dq2, dk2, dv2 = attention_backward(q, kr, vr, do, 0.5, True)
+    np.testing.assert_allclose(dq, dq2, atol=TOL)
+    np.testing.assert_allclose(dk, dk2.reshape(2, 6, 2, 2, 3).sum(axis=3), atol=TOL)
+    np.testing.assert_allclose(dv, dv2.reshape(2, 6, 2, 2, 3).sum(axis=3), atol=TOL)
+
+
+def test_backward_rows_without_keys_contribute_nothing():
+    # causal with Sq > Sk: the first Sq - Sk rows see no key
+    q, k, v = qkv(B=1, Sq=6, Sk=3, Hq=1, Hkv=1, D=2, seed=79)
+    do = rnd(q.shape, 80)
+    dq, dk, dv = attention_backward(q, k, v, do, 0.8, True)
+    assert np.all(dq[0, :3] == 0)
+    do2 = do.copy()
+    do2[0, :3] = 123.0                       # upstream gradient of those rows is irrelevant
+    dq2, dk2, dv2 = attention_backward(q, k, v, do2, 0.8, True)
+    np.testing.assert_allclose(dk2, dk, atol=TOL)
+    np.testing.assert_allclose(dv2, dv, atol=TOL)
