@@ -200,7 +200,7 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
     ap.add_argument("--no-e2e", action="store_true")
-    ap.add_argument("--only", default="all", choices=["all", "prefill", "decode", "varlen", "sparse"],
+    ap.add_argument("--only", default="all", choices=["all", "prefill", "decode", "varlen", "sparse", "backward"],
                     help="profiling aid: run only one half of the step (the JSON line is then partial)")
     ap.add_argument("--prefill-seq", type=int, default=0,
                     help="profiling aid: shorter prefill sequence (same heads, dtype, sinks)")
@@ -217,9 +217,10 @@ def main():
                                                    sa_attn_decode_paged_workspace_size,
                                                    sa_attn_decode_workspace_size, sa_attn_fwd,
                                                    sa_attn_fwd_block_sparse, sa_attn_fwd_block_sparse_workspace_size,
+                                                   sa_attn_bwd, sa_attn_bwd_workspace_size,
                                                    sa_attn_fwd_varlen, sa_check_status)
     from online_softmax_attention_sm_b200.dist import aggregate_throughput, max_over_ranks, rank_seed
-    from online_softmax_attention_sm_b200.inputs import make_qkv, make_workload_inputs, stem_block_mask
+    from online_softmax_attention_sm_b200.inputs import make_dout, make_qkv, make_workload_inputs, stem_block_mask
     from online_softmax_attention_sm_b200.workloads import WORKLOADS, block_sparse_flops
 
     rank, world, local = dist_env()
@@ -238,6 +239,7 @@ def main():
     run_pre, run_dec = args.only in ("all", "prefill"), args.only in ("all", "decode")
     run_var = args.only in ("all", "varlen")
     run_sparse = args.only in ("all", "sparse")
+    run_bwd = args.only in ("all", "backward")
     q_h, k_h, v_h = make_workload_inputs(wp, seed=rank_seed(wp.seed, rank))
     dq_h, dk_h, dv_h = make_workload_inputs(wd, seed=rank_seed(wd.seed, rank))
     q, k, v = q_h.to(dev), k_h.to(dev), v_h.to(dev)
@@ -381,6 +383,28 @@ def main():
         sp_ms = [a.elapsed_time(b) for a, b in sev]
         del bmask, sws
 
+    # backward of the prefill workload: dQ, dK, dV for a seeded dO (three kernels: prep,
+    # dK/dV, dQ); the forward's O and LSE are made once, outside the events
+    bwd_ms = [float("nan")]
+    if run_bwd:
+        dout = make_dout(wp.B, wp.Sq, wp.Hq, wp.D, wp.dtype, seed=rank_seed(wp.seed, rank)).to(dev)
+        sa_attn_fwd(q, k, v, causal=wp.causal, scale=wp.scale, out=o, lse=lse, stream=stream)
+        gq, gk, gv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+        bws = torch.empty(max(16, sa_attn_bwd_workspace_size(wp.B, wp.Sq, wp.Hq)), dtype=torch.uint8, device=dev)
+        bev = []
+        for i in range(args.warmup + args.steps):
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            sa_attn_bwd(q, k, v, o, lse, dout, causal=wp.causal, scale=wp.scale, workspace=bws, dq=gq, dk=gk,
+                        dv=gv, stream=stream)
+            e1.record(stream)
+            if i >= args.warmup:
+                bev.append((e0, e1))
+        torch.cuda.synchronize(dev)
+        sa_check_status(stream)
+        bwd_ms = [a.elapsed_time(b) for a, b in bev]
+        del dout, gq, gk, gv, bws
+
     # e2e through the public API with host buffers: H2D of the step's inputs, D2H of outputs
     e2e_ms = None
     h2d = sum(t.numel() * t.element_size() for t in (q_h, k_h, v_h, dq_h, dk_h, dv_h))
@@ -416,6 +440,7 @@ def main():
     paged_avg = max_over_ranks(sum(paged_ms) / len(paged_ms), dev)
     var_avg = max_over_ranks(sum(var_ms) / len(var_ms), dev)
     sp_avg = max_over_ranks(sum(sp_ms) / len(sp_ms), dev)
+    bwd_avg = max_over_ranks(sum(bwd_ms) / len(bwd_ms), dev)
     e2e_ms = max_over_ranks(e2e_ms, dev) if e2e_ms is not None else None
 
     if rank == 0:
@@ -470,6 +495,12 @@ def main():
                                      "frac": sp_flops / (sp_avg * 1e-3) / 1e12 / peak, "ms": sp_avg,
                                      "work_vs_dense_causal": sp_flops / wp.flops,
                                      "kernels": "sparse_unit_lists + attn_fwd_sm100 (block-sparse instance)"},
+            "backward": {"workload": PREFILL, "value": 2.5 * wp.flops / (bwd_avg * 1e-3) / 1e12,
+                         "unit": "TFLOP/s", "bound": "tensor", "peak": peak,
+                         "frac": 2.5 * wp.flops / (bwd_avg * 1e-3) / 1e12 / peak, "ms": bwd_avg,
+                         "flops": "2.5 x the forward's (5 tile products against 2; the dQ kernel's "
+                                  "recomputed S and dP are not credited)",
+                         "kernels": "bwd_prep + attn_bwd_kv + attn_bwd_q"},
             "prefill_ms": pre_avg,
             "gpu_launches": (int(run_pre) + 2 * int(run_dec)) * args.steps,
             "clocks": clk.summary(),

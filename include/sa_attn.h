@@ -119,6 +119,26 @@ int sa_attn_fwd_block_sparse(const void* q, const void* k, const void* v, void* 
                              void* workspace, size_t workspace_bytes, sa_stream_t stream);
 
 /*
+ * Attention backward: dQ, dK, dV of the forward's O for an upstream gradient dO
+ * (StreamAttention page, "Backward": the QK tiles are recomputed from the saved LSE and
+ * dQ/dK/dV are streamed, never the attention matrix; flash-attn-volta page, backward).
+ *   q, k, v, causal, scale, dtype : as given to sa_attn_fwd;
+ *   o, lse     : that forward's output [B, Sq, Hq, D] and LSE [B, Hq, Sq] (fp32, required);
+ *   dout       : [B, Sq, Hq, D] upstream gradient (dtype);
+ *   dq         : out [B, Sq, Hq, D]; dk, dv : out [B, Sk, Hkv, D] (dtype; dk and dv summed
+ *                over the query heads that share a KV head);
+ *   workspace  : device scratch of sa_attn_bwd_workspace_size() bytes, 16-byte aligned,
+ *                no initial contents (per-row Delta = rowsum(dout * o) and LSE * log2 e).
+ * Rows without a visible key contribute nothing.  Sq == 0 or Sk == 0: the gradients are
+ * zero-filled.  Three kernels on `stream`; no atomics, deterministic.
+ */
+size_t sa_attn_bwd_workspace_size(int B, int Sq, int Hq);
+int sa_attn_bwd(const void* q, const void* k, const void* v, const void* o, const float* lse,
+                const void* dout, void* dq, void* dk, void* dv, int B, int Sq, int Sk, int Hq,
+                int Hkv, int D, int causal, float scale, int dtype, void* workspace,
+                size_t workspace_bytes, sa_stream_t stream);
+
+/*
  * Bytes of decode workspace needed for `num_splits` (0 = the automatic choice):
  * B * Hq * splits * (D + 4) * 4.  It holds, per (b, h, split), the split's running max
  * and two running sums (of the 16-bit weights the MMA used, and of the fp32 weights for

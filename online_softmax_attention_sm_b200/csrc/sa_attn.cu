@@ -5,6 +5,7 @@
 #include "ptx.cuh"
 #include "fwd_sm100.cuh"
 #include "sparse_lists.cuh"
+#include "bwd_sm100.cuh"
 #include "fwd_simple.cuh"
 #include "decode.cuh"
 
@@ -293,6 +294,50 @@ int launch_fwd(const void* q, const void* k, const void* v, void* o, float* lse,
   return e == cudaSuccess ? SA_OK : cuda_fail(e, "attn_fwd_sm100 launch");
 }
 
+// Backward: prep (Delta, lse2), then the dK/dV and dQ kernels, all on `st`.
+template <int D, bool BF16>
+int launch_bwd(const void* q, const void* k, const void* v, const void* o, const float* lse, const void* dout,
+               void* dq, void* dk, void* dv, int B, int Sq, int Sk, int Hq, int Hkv, int causal, float scale,
+               float* ws, cudaStream_t st) {
+  using Cfg = sa::BwdCfg<D>;
+  CUtensorMap mq, mdo, mk, mv;
+  int rc;
+  if ((rc = make_map(&mq, q, BF16, D, Hq, Sq, B, 128)) != SA_OK) return rc;
+  if ((rc = make_map(&mdo, dout, BF16, D, Hq, Sq, B, 128)) != SA_OK) return rc;
+  if ((rc = make_map(&mk, k, BF16, D, Hkv, Sk, B, 128)) != SA_OK) return rc;
+  if ((rc = make_map(&mv, v, BF16, D, Hkv, Sk, B, 128)) != SA_OK) return rc;
+  sa::BwdParams p;
+  p.o = o; p.dout = dout; p.lse = lse;
+  p.sq_pad = (Sq + 127) / 128 * 128;
+  p.lse2 = ws;
+  p.delta = ws + (size_t)B * Hq * p.sq_pad;
+  p.dq = dq; p.dk = dk; p.dv = dv;
+  p.B = B; p.Sq = Sq; p.Sk = Sk; p.Hq = Hq; p.Hkv = Hkv; p.G = Hq / Hkv; p.causal = causal;
+  p.n_qt = p.sq_pad / 128;
+  p.n_kt = (Sk + 127) / 128;
+  p.c2 = scale * kLog2e;
+  p.scale = scale;
+  if (Hq > 65535 || B > 65535) return fail(SA_ERR_UNSUPPORTED, "backward supports Hq, B <= 65535");
+  const long long prep_threads = (long long)B * p.sq_pad * Hq;
+  sa::bwd_prep<D, BF16><<<(unsigned)((prep_threads + 255) / 256), 256, 0, st>>>(p);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return cuda_fail(e, "bwd_prep launch");
+  // D = 64 would fit two CTAs per SM in shared memory, but each holds all 512 tensor-memory
+  // columns: ask for enough shared memory to keep one
+  const int smem = Cfg::SMEM_TOTAL > 120 * 1024 ? Cfg::SMEM_TOTAL : 120 * 1024;
+  auto kv = sa::attn_bwd_kv<D, BF16>;
+  auto kq = sa::attn_bwd_q<D, BF16>;
+  if ((e = cudaFuncSetAttribute(kv, cudaFuncAttributeMaxDynamicSharedMemorySize, smem)) != cudaSuccess)
+    return cuda_fail(e, "cudaFuncSetAttribute(attn_bwd_kv)");
+  if ((e = cudaFuncSetAttribute(kq, cudaFuncAttributeMaxDynamicSharedMemorySize, smem)) != cudaSuccess)
+    return cuda_fail(e, "cudaFuncSetAttribute(attn_bwd_q)");
+  kv<<<dim3(p.n_kt, Hkv, B), Cfg::THREADS, smem, st>>>(mq, mdo, mk, mv, p);
+  if ((e = cudaGetLastError()) != cudaSuccess) return cuda_fail(e, "attn_bwd_kv launch");
+  kq<<<dim3(p.n_qt, Hq, B), Cfg::THREADS, smem, st>>>(mq, mdo, mk, mv, p);
+  if ((e = cudaGetLastError()) != cudaSuccess) return cuda_fail(e, "attn_bwd_q launch");
+  return SA_OK;
+}
+
 template <int D, bool BF16>
 int launch_simple(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Sq,
                   int Sk, int Hq, int Hkv, int causal, float scale, cudaStream_t st) {
@@ -504,6 +549,49 @@ int sa_attn_fwd_block_sparse(const void* q, const void* k, const void* v, void* 
               : launch_fwd<64, false>(q, k, v, o, lse, B, Sq, Sk, Hq, Hkv, causal, scale, st, none, sp);
   return bf ? launch_fwd<128, true>(q, k, v, o, lse, B, Sq, Sk, Hq, Hkv, causal, scale, st, none, sp)
             : launch_fwd<128, false>(q, k, v, o, lse, B, Sq, Sk, Hq, Hkv, causal, scale, st, none, sp);
+}
+
+size_t sa_attn_bwd_workspace_size(int B, int Sq, int Hq) {
+  if (B <= 0 || Sq <= 0 || Hq <= 0) return 0;
+  return 2 * (size_t)B * Hq * (((size_t)Sq + 127) / 128 * 128) * sizeof(float);
+}
+
+int sa_attn_bwd(const void* q, const void* k, const void* v, const void* o, const float* lse, const void* dout,
+                void* dq, void* dk, void* dv, int B, int Sq, int Sk, int Hq, int Hkv, int D, int causal,
+                float scale, int dtype, void* workspace, size_t workspace_bytes, sa_stream_t stream) {
+  int rc = check_dims(B, Sq, Sk, Hq, Hkv, D, dtype, scale);
+  if (rc != SA_OK) return rc;
+  if (causal != 0 && causal != 1) return fail(SA_ERR_INVALID, "causal must be 0 or 1");
+  if (B == 0 || Hq == 0) return SA_OK;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  const size_t kv_bytes = (size_t)B * Sk * Hkv * D * 2;
+  if (Sq == 0 || Sk == 0) {
+    // no (query, key) pair: every gradient is zero
+    if (Sk > 0 && (!dk || !dv)) return fail(SA_ERR_INVALID, "dk and dv must be non-null");
+    if (Sq > 0 && !dq) return fail(SA_ERR_INVALID, "dq must be non-null");
+    cudaError_t e = cudaSuccess;
+    if (Sk > 0 && e == cudaSuccess) e = cudaMemsetAsync(dk, 0, kv_bytes, st);
+    if (Sk > 0 && e == cudaSuccess) e = cudaMemsetAsync(dv, 0, kv_bytes, st);
+    if (Sq > 0 && e == cudaSuccess) e = cudaMemsetAsync(dq, 0, (size_t)B * Sq * Hq * D * 2, st);
+    return e == cudaSuccess ? SA_OK : cuda_fail(e, "zero fill of the gradients");
+  }
+  if (!q || !k || !v || !o || !lse || !dout || !dq || !dk || !dv)
+    return fail(SA_ERR_INVALID, "q, k, v, o, lse, dout, dq, dk and dv must be non-null");
+  const void* ptrs[] = {q, k, v, o, lse, dout, dq, dk, dv};
+  for (const void* ptr : ptrs)
+    if (!aligned16(ptr)) return fail(SA_ERR_INVALID, "tensor pointers must be 16-byte aligned");
+  const size_t need = sa_attn_bwd_workspace_size(B, Sq, Hq);
+  if (!workspace || workspace_bytes < need)
+    return fail(SA_ERR_WORKSPACE, "backward workspace of %zu bytes needed, %zu given", need,
+                workspace ? workspace_bytes : (size_t)0);
+  if (!aligned16(workspace)) return fail(SA_ERR_INVALID, "workspace must be 16-byte aligned");
+  float* ws = static_cast<float*>(workspace);
+  const bool bf = dtype == SA_BF16;
+  if (D == 64)
+    return bf ? launch_bwd<64, true>(q, k, v, o, lse, dout, dq, dk, dv, B, Sq, Sk, Hq, Hkv, causal, scale, ws, st)
+              : launch_bwd<64, false>(q, k, v, o, lse, dout, dq, dk, dv, B, Sq, Sk, Hq, Hkv, causal, scale, ws, st);
+  return bf ? launch_bwd<128, true>(q, k, v, o, lse, dout, dq, dk, dv, B, Sq, Sk, Hq, Hkv, causal, scale, ws, st)
+            : launch_bwd<128, false>(q, k, v, o, lse, dout, dq, dk, dv, B, Sq, Sk, Hq, Hkv, causal, scale, ws, st);
 }
 
 int sa_attn_fwd_simple(const void* q, const void* k, const void* v, void* o, float* lse, int B,

@@ -109,3 +109,11 @@ def stem_block_mask(B, Hq, Sq, Sk, causal, seed, initial_blocks=4, window_blocks
             idx = r.topk(take, dim=-1).indices + lo
             mask[:, :, qi].scatter_(-1, idx, 1)
     return mask
+
+
+def make_dout(B, Sq, Hq, D, dtype="fp16", seed=0):
+    """Upstream gradient dO [B, Sq, Hq, D] for the backward: float32 N(0,1) from a generator
+    seeded with seed + 7777, rounded to the storage dtype."""
+    g = torch.Generator(device="cpu")
+    g.manual_seed(int(seed) + 7777)
+    return torch.randn((B, Sq, Hq, D), generator=g, dtype=torch.float32).to(DTYPES[dtype]).contiguous()

@@ -26,6 +26,8 @@ SIGNATURES = {
     "sa_attn_fwd_simple": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _F, _I, _P]),
     "sa_attn_fwd_varlen": (_I, [_P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _I, _I, _F, _I, _P]),
     "sa_attn_fwd_block_sparse_workspace_size": (_Z, [_I, _I, _I, _I]),
+    "sa_attn_bwd_workspace_size": (_Z, [_I, _I, _I]),
+    "sa_attn_bwd": (_I, [_P] * 9 + [_I] * 7 + [_F, _I, _P, _Z, _P]),
     "sa_attn_fwd_block_sparse": (_I, [_P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _F, _I, _P, _Z, _P]),
     "sa_attn_decode_workspace_size": (_Z, [_I, _I, _I, _I, _I, _I]),
     "sa_attn_decode_num_splits": (_I, [_I, _I, _I, _I, _I]),
@@ -189,6 +191,44 @@ def sa_attn_fwd_block_sparse(q, k, v, block_mask, causal=False, scale=None, work
                                           _ptr(workspace), workspace.numel() * workspace.element_size(),
                                           _stream(stream)))
     return out, lse
+
+
+def sa_attn_bwd_workspace_size(B, Sq, Hq):
+    return int(lib().sa_attn_bwd_workspace_size(B, Sq, Hq))
+
+
+def sa_attn_bwd(q, k, v, o, lse, dout, causal=False, scale=None, workspace=None, dq=None, dk=None, dv=None,
+                stream=None):
+    """Attention backward.  q/o/dout [B,Sq,Hq,D], k/v [B,Sk,Hkv,D] (fp16/bf16, CUDA, contiguous),
+    lse [B,Hq,Sq] fp32 from the forward.  Returns (dq, dk, dv) shaped like q, k, v."""
+    B, Sq, Hq, D = q.shape
+    Sk, Hkv = k.shape[1], k.shape[2]
+    if k.shape != (B, Sk, Hkv, D) or v.shape != k.shape or o.shape != q.shape or dout.shape != q.shape:
+        raise ValueError(f"shape mismatch q{tuple(q.shape)} k{tuple(k.shape)} v{tuple(v.shape)} "
+                         f"o{tuple(o.shape)} dout{tuple(dout.shape)}")
+    if q.dtype not in _DT:
+        raise TypeError(f"unsupported dtype {q.dtype}")
+    for n, t in (("q", q), ("k", k), ("v", v), ("o", o), ("dout", dout)):
+        _check_tensor(n, t, q.dtype, q.device)
+    _check_tensor("lse", lse, torch.float32, q.device)
+    if lse.shape != (B, Hq, Sq):
+        raise ValueError(f"lse must be [B, Hq, Sq], got {tuple(lse.shape)}")
+    if scale is None:
+        scale = 1.0 / math.sqrt(D)
+    dq = torch.empty_like(q) if dq is None else dq
+    dk = torch.empty_like(k) if dk is None else dk
+    dv = torch.empty_like(v) if dv is None else dv
+    for n, t, like in (("dq", dq, q), ("dk", dk, k), ("dv", dv, v)):
+        _check_tensor(n, t, q.dtype, q.device)
+        if t.shape != like.shape:
+            raise ValueError(f"{n} must have shape {tuple(like.shape)}")
+    need = sa_attn_bwd_workspace_size(B, Sq, Hq)
+    if workspace is None:
+        workspace = torch.empty(max(need, 16), dtype=torch.uint8, device=q.device)
+    _check(lib().sa_attn_bwd(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), _ptr(dout), _ptr(dq), _ptr(dk),
+                             _ptr(dv), B, Sq, Sk, Hq, Hkv, D, int(bool(causal)), float(scale), _DT[q.dtype],
+                             _ptr(workspace), workspace.numel() * workspace.element_size(), _stream(stream)))
+    return dq, dk, dv
 
 
 def sa_attn_fwd_simple(q, k, v, causal=False, scale=None, **kw):

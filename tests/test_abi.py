@@ -238,6 +238,40 @@ def test_block_sparse_workspace_size(L):
     assert L.sa_attn_fwd_block_sparse_workspace_size(0, 256, 256, 2) == 0
 
 
+def bwd(L, q=FAKE, k=FAKE, v=FAKE, o=FAKE, lse=FAKE, do=FAKE, dq=FAKE, dk=FAKE, dv=FAKE, B=1, Sq=128, Sk=128, Hq=2,
+        Hkv=1, D=64, causal=1, scale=0.125, dtype=1, ws=FAKE, wsb=1 << 20):
+    return L.sa_attn_bwd(q, k, v, o, lse, do, dq, dk, dv, B, Sq, Sk, Hq, Hkv, D, causal, scale, dtype, ws, wsb,
+                         None)
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(q=NULL), sa.SA_ERR_INVALID),
+    (dict(lse=NULL), sa.SA_ERR_INVALID),
+    (dict(do=NULL), sa.SA_ERR_INVALID),
+    (dict(dk=NULL), sa.SA_ERR_INVALID),
+    (dict(Hq=3, Hkv=2), sa.SA_ERR_INVALID),
+    (dict(D=96), sa.SA_ERR_UNSUPPORTED),
+    (dict(causal=4), sa.SA_ERR_INVALID),
+    (dict(scale=math.nan), sa.SA_ERR_INVALID),
+    (dict(dv=ctypes.c_void_p((1 << 20) + 4)), sa.SA_ERR_INVALID),
+    (dict(ws=NULL), sa.SA_ERR_WORKSPACE),
+    (dict(wsb=64), sa.SA_ERR_WORKSPACE),
+])
+def test_bwd_rejects_invalid_arguments(L, kw, code):
+    assert bwd(L, **kw) == code
+
+
+def test_bwd_empty_is_a_no_op(L):
+    assert bwd(L, q=NULL, k=NULL, v=NULL, o=NULL, lse=NULL, do=NULL, dq=NULL, dk=NULL, dv=NULL, ws=NULL, B=0) == sa.SA_OK
+
+
+def test_bwd_workspace_size(L):
+    # two fp32 rows (lse2, Delta) per (batch, query head), padded to 128 queries
+    assert L.sa_attn_bwd_workspace_size(1, 300, 4) == 2 * 4 * 384 * 4
+    assert L.sa_attn_bwd_workspace_size(2, 32768, 32) == 2 * 2 * 32 * 32768 * 4
+    assert L.sa_attn_bwd_workspace_size(0, 300, 4) == 0
+
+
 def test_version(L):
     assert re.fullmatch(r"\d+\.\d+\.\d+", sa.sa_version())
 
