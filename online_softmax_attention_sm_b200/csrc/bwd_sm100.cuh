@@ -7,9 +7,10 @@
 //   dV = P^T dO,  dP = dO V^T,  dS = P * (dP - Delta),  dQ = scale dS K,  dK = scale dS^T Q.
 //
 // B200 design: three kernels, no atomics.
-//   * bwd_prep: Delta and lse2 per query row into the caller's workspace ([B, Hq, Sq_pad],
-//     Sq_pad = Sq rounded up to 128; padding rows get lse2 = -inf, Delta = 0, so a whole
-//     128-row slice can always be copied);
+//   * bwd_prep: -lse2 and -Delta per query row into the caller's workspace ([B, Hq, Sq_pad],
+//     Sq_pad = Sq rounded up to 128; padding rows get -lse2 = -inf (P = 0) and -Delta = 0,
+//     so a whole 128-row slice can always be copied); stored negated so that
+//     c2 S - lse2 and dP - Delta are one packed FMA / ADD each;
 //   * attn_bwd_kv<D>: one CTA per (128-key tile, KV head, batch) keeps K and V in shared
 //     memory and walks every (query head of the group, 128-row Q tile) that sees the tile:
 //     S^T = K Q^T and dP^T = V dO^T (tcgen05, both operands K-major from shared memory),
@@ -59,8 +60,8 @@ struct BwdParams {
   const void* o;        // [B, Sq, Hq, D] forward output (prep)
   const void* dout;     // [B, Sq, Hq, D]
   const float* lse;     // [B, Hq, Sq] forward LSE (natural log)
-  float* lse2;          // [B, Hq, Sq_pad] workspace: LSE * log2(e)
-  float* delta;         // [B, Hq, Sq_pad] workspace: rowsum(dO * O)
+  float* nlse2;         // [B, Hq, Sq_pad] workspace: -LSE * log2(e)
+  float* ndelta;        // [B, Hq, Sq_pad] workspace: -rowsum(dO * O)
   void* dq;             // [B, Sq, Hq, D]
   void* dk;             // [B, Sk, Hkv, D]
   void* dv;             // [B, Sk, Hkv, D]
@@ -81,8 +82,8 @@ __global__ void __launch_bounds__(256) bwd_prep(const BwdParams p) {
   const int q = (int)(bq % p.sq_pad), b = (int)(bq / p.sq_pad);
   const size_t out = ((size_t)b * p.Hq + h) * p.sq_pad + q;
   if (q >= p.Sq) {
-    p.lse2[out] = -INFINITY;
-    p.delta[out] = 0.f;
+    p.nlse2[out] = -INFINITY;
+    p.ndelta[out] = 0.f;
     return;
   }
   const size_t row = (((size_t)b * p.Sq + q) * p.Hq + h) * D;
@@ -112,8 +113,8 @@ __global__ void __launch_bounds__(256) bwd_prep(const BwdParams p) {
     }
   }
   const float l = p.lse[((size_t)b * p.Hq + h) * p.Sq + q];
-  p.lse2[out] = l * 1.4426950408889634f;      // -inf stays -inf (row without keys)
-  p.delta[out] = acc;
+  p.nlse2[out] = -l * 1.4426950408889634f;    // row without keys: +inf, never unmasked
+  p.ndelta[out] = -acc;
 }
 
 // ---------------------------------------------------------------- shared helpers
@@ -146,27 +147,30 @@ __device__ __forceinline__ uint32_t bwd_pack(float lo, float hi) {
 }
 
 // One 32-column chunk of a P / dS half for the calling thread's row: s, dp = 32 fp32
-// columns of S and dP; lse2 / delta per column (KV kernel: per query) or per row (Q
-// kernel, the same value 32 times); vis(i) says whether column i is visible.  Writes the
-// 16 packed P pairs and 16 packed dS pairs.
-template <bool BF16, typename Lse, typename Delta, typename Vis>
-__device__ __forceinline__ void bwd_chunk(const uint32_t (&s)[32], const uint32_t (&dp)[32], float c2,
-                                          Lse lse2, Delta delta, Vis vis, uint32_t (&pp)[16],
-                                          uint32_t (&dsp)[16]) {
+// columns of S and dP; nl, nd = -lse2 and -Delta of each column (pairs); columns
+// lo <= i < hi are visible (the rest get P = dS = 0; lo <= 0, hi >= 32 takes the unmasked
+// path).  P = 2^(c2 s - lse2), dS = P (dP - Delta) on packed f32x2 pairs, written as 16
+// packed 16-bit pairs each.
+template <bool BF16>
+__device__ __forceinline__ void bwd_chunk(const uint32_t (&s)[32], const uint32_t (&dp)[32], f32x2 c2,
+                                          const f32x2 (&nl)[16], const f32x2 (&nd)[16], int lo, int hi,
+                                          uint32_t (&pp)[16], uint32_t (&dsp)[16]) {
+  const bool full = lo <= 0 && hi >= 32;
 #pragma unroll
   for (int i = 0; i < 16; ++i) {
-    float pv[2], dsv[2];
-#pragma unroll
-    for (int e = 0; e < 2; ++e) {
-      const int c = 2 * i + e;
-      const float l = lse2(c);
-      const bool on = vis(c) && l != -INFINITY;
-      const float pr = on ? ex2(fmaf(__uint_as_float(s[c]), c2, -l)) : 0.f;
-      pv[e] = pr;
-      dsv[e] = pr * (__uint_as_float(dp[c]) - delta(c));
+    float x0, x1;
+    unpack_f2(fma_f2(pack_f2(__uint_as_float(s[2 * i]), __uint_as_float(s[2 * i + 1])), c2, nl[i]), x0, x1);
+    float p0 = ex2(x0), p1 = ex2(x1);
+    if (!full) {
+      p0 = (2 * i >= lo && 2 * i < hi) ? p0 : 0.f;
+      p1 = (2 * i + 1 >= lo && 2 * i + 1 < hi) ? p1 : 0.f;
     }
-    pp[i] = bwd_pack<BF16>(pv[0], pv[1]);
-    dsp[i] = bwd_pack<BF16>(dsv[0], dsv[1]);
+    const f32x2 d2 = mul_f2(pack_f2(p0, p1),
+                            add_f2(pack_f2(__uint_as_float(dp[2 * i]), __uint_as_float(dp[2 * i + 1])), nd[i]));
+    float d0, d1;
+    unpack_f2(d2, d0, d1);
+    pp[i] = bwd_pack<BF16>(p0, p1);
+    dsp[i] = bwd_pack<BF16>(d0, d1);
   }
 }
 
@@ -303,7 +307,10 @@ attn_bwd_kv(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
   uint8_t* smem = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
   const BwdSmem<D> sm(smem);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int kt = blockIdx.x, kvh = blockIdx.y, b = blockIdx.z;
+  // one flat grid, longest first: key tile major (causal: the first tiles see the most
+  // queries), then batch, then KV head
+  const int per_tile = p.Hkv * p.B;
+  const int kt = (int)blockIdx.x / per_tile, b = ((int)blockIdx.x % per_tile) / p.Hkv, kvh = (int)blockIdx.x % p.Hkv;
   // query tiles that see this key tile: all, or (causal) from the first row whose
   // bottom-right-aligned diagonal reaches the tile's first key
   int qt0 = 0;
@@ -349,8 +356,8 @@ attn_bwd_kv(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
           tma_load_4d(dst + Cfg::TILE + c * Cfg::CHUNK, &tm_do, &sm.full[s], c * 64, h, qt * 128, b);
         }
         const size_t vrow = ((size_t)b * p.Hq + h) * p.sq_pad + (size_t)qt * 128;
-        bulk_copy_g2s(dst + 2 * Cfg::TILE, p.lse2 + vrow, 512, &sm.full[s]);
-        bulk_copy_g2s(dst + 2 * Cfg::TILE + 512, p.delta + vrow, 512, &sm.full[s]);
+        bulk_copy_g2s(dst + 2 * Cfg::TILE, p.nlse2 + vrow, 512, &sm.full[s]);
+        bulk_copy_g2s(dst + 2 * Cfg::TILE + 512, p.ndelta + vrow, 512, &sm.full[s]);
         issued = n + 1;
       }
       if (!ok) bwd_drain(sm, nsteps > 0, issued);
@@ -399,6 +406,7 @@ attn_bwd_kv(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
     const int kr = wl * 32 + lane, key = kt * 128 + kr;
     const uint32_t lane_addr = tmem + ((uint32_t)(wl * 32) << 16);
     const int shift = p.Sk - p.Sq;
+    const f32x2 c2x2 = pack_f2(p.c2, p.c2);
     bool ok = true;
     for (int n = 0; n < nsteps; ++n) {
       ok = mbar_wait_warp(&sm.s_ready[c], n & 1, sm.abort_flag, 67 + c);
@@ -417,13 +425,15 @@ attn_bwd_kv(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
         tmem_wait_ld_regs(sv);
         tmem_wait_ld_regs(dp);
         const int col0 = 64 * c + 32 * ch, q0 = qbase + 32 * ch;
-        bwd_chunk<BF16>(sv, dp, p.c2, [&](int i) { return vec[col0 + i]; },
-                        [&](int i) { return vec[128 + col0 + i]; },
-                        [&](int i) {
-                          const int q = q0 + i;
-                          return q < p.Sq && key < p.Sk && (!p.causal || key <= q + shift);
-                        },
-                        pp, dsp);
+        // visible queries of this key row: q >= key - shift (causal), q < Sq; none past Sk
+        const int lo = p.causal ? key - shift - q0 : 0;
+        const int hi = key < p.Sk ? min(32, p.Sq - q0) : 0;
+        const f32x2* nl2 = reinterpret_cast<const f32x2*>(vec + col0);
+        const f32x2* nd2 = reinterpret_cast<const f32x2*>(vec + 128 + col0);
+        f32x2 nl[16], nd[16];
+#pragma unroll
+        for (int i = 0; i < 16; ++i) { nl[i] = nl2[i]; nd[i] = nd2[i]; }
+        bwd_chunk<BF16>(sv, dp, c2x2, nl, nd, lo, hi, pp, dsp);
         tmem_st16(lane_addr + Cfg::S_COL + 64 * c + 16 * ch, pp);
         tmem_st16(lane_addr + Cfg::DP_COL + 64 * c + 16 * ch, dsp);
       }
@@ -457,8 +467,11 @@ attn_bwd_q(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUt
   uint8_t* smem = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
   const BwdSmem<D> sm(smem);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  // longest first: causal Q tiles near the end see the most keys
-  const int qt = p.n_qt - 1 - (int)blockIdx.x, h = blockIdx.y, b = blockIdx.z;
+  // one flat grid, longest first: Q tile major from the last (causal: it sees the most
+  // keys), then batch, then query head
+  const int per_tile = p.Hq * p.B;
+  const int qt = p.n_qt - 1 - (int)blockIdx.x / per_tile;
+  const int b = ((int)blockIdx.x % per_tile) / p.Hq, h = (int)blockIdx.x % p.Hq;
   const int kvh = h / p.G;
   int kend = p.Sk;                                   // keys any row of the tile sees
   if (p.causal) kend = min(p.Sk, min(qt * 128 + 127, p.Sq - 1) + p.Sk - p.Sq + 1);
@@ -540,8 +553,12 @@ attn_bwd_q(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUt
     const int qr = wl * 32 + lane, q = qt * 128 + qr;
     const uint32_t lane_addr = tmem + ((uint32_t)(wl * 32) << 16);
     const size_t vrow = ((size_t)b * p.Hq + h) * p.sq_pad + q;     // q < sq_pad always
-    const float l2 = p.lse2[vrow], dl = p.delta[vrow];
+    const float nl1 = p.nlse2[vrow], nd1 = p.ndelta[vrow];
     const int klim = p.causal ? q + p.Sk - p.Sq : p.Sk - 1;          // last key this row sees
+    const f32x2 c2x2 = pack_f2(p.c2, p.c2);
+    f32x2 nl[16], nd[16];
+#pragma unroll
+    for (int i = 0; i < 16; ++i) { nl[i] = pack_f2(nl1, nl1); nd[i] = pack_f2(nd1, nd1); }
     bool ok = true;
     for (int n = 0; n < nsteps; ++n) {
       ok = mbar_wait_warp(&sm.s_ready[c], n & 1, sm.abort_flag, 77 + c);
@@ -556,8 +573,9 @@ attn_bwd_q(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUt
         tmem_wait_ld_regs(sv);
         tmem_wait_ld_regs(dp);
         const int k0 = kbase + 32 * ch;
-        bwd_chunk<BF16>(sv, dp, p.c2, [&](int) { return l2; }, [&](int) { return dl; },
-                        [&](int i) { return q < p.Sq && k0 + i < p.Sk && k0 + i <= klim; }, pp, dsp);
+        // visible keys of this row: k <= klim, k < Sk; none for padding rows
+        const int hi = q < p.Sq ? min(p.Sk, klim + 1) - k0 : 0;
+        bwd_chunk<BF16>(sv, dp, c2x2, nl, nd, 0, hi, pp, dsp);
         tmem_st16(lane_addr + Cfg::DP_COL + 64 * c + 16 * ch, dsp);
       }
       tmem_wait_st();

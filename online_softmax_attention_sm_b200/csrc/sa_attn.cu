@@ -309,15 +309,16 @@ int launch_bwd(const void* q, const void* k, const void* v, const void* o, const
   sa::BwdParams p;
   p.o = o; p.dout = dout; p.lse = lse;
   p.sq_pad = (Sq + 127) / 128 * 128;
-  p.lse2 = ws;
-  p.delta = ws + (size_t)B * Hq * p.sq_pad;
+  p.nlse2 = ws;
+  p.ndelta = ws + (size_t)B * Hq * p.sq_pad;
   p.dq = dq; p.dk = dk; p.dv = dv;
   p.B = B; p.Sq = Sq; p.Sk = Sk; p.Hq = Hq; p.Hkv = Hkv; p.G = Hq / Hkv; p.causal = causal;
   p.n_qt = p.sq_pad / 128;
   p.n_kt = (Sk + 127) / 128;
   p.c2 = scale * kLog2e;
   p.scale = scale;
-  if (Hq > 65535 || B > 65535) return fail(SA_ERR_UNSUPPORTED, "backward supports Hq, B <= 65535");
+  if ((long long)p.n_qt * Hq * B > 0x7fffffffLL || (long long)p.n_kt * Hkv * B > 0x7fffffffLL)
+    return fail(SA_ERR_UNSUPPORTED, "backward grid too large");
   const long long prep_threads = (long long)B * p.sq_pad * Hq;
   sa::bwd_prep<D, BF16><<<(unsigned)((prep_threads + 255) / 256), 256, 0, st>>>(p);
   cudaError_t e = cudaGetLastError();
@@ -331,9 +332,9 @@ int launch_bwd(const void* q, const void* k, const void* v, const void* o, const
     return cuda_fail(e, "cudaFuncSetAttribute(attn_bwd_kv)");
   if ((e = cudaFuncSetAttribute(kq, cudaFuncAttributeMaxDynamicSharedMemorySize, smem)) != cudaSuccess)
     return cuda_fail(e, "cudaFuncSetAttribute(attn_bwd_q)");
-  kv<<<dim3(p.n_kt, Hkv, B), Cfg::THREADS, smem, st>>>(mq, mdo, mk, mv, p);
+  kv<<<p.n_kt * Hkv * B, Cfg::THREADS, smem, st>>>(mq, mdo, mk, mv, p);
   if ((e = cudaGetLastError()) != cudaSuccess) return cuda_fail(e, "attn_bwd_kv launch");
-  kq<<<dim3(p.n_qt, Hq, B), Cfg::THREADS, smem, st>>>(mq, mdo, mk, mv, p);
+  kq<<<p.n_qt * Hq * B, Cfg::THREADS, smem, st>>>(mq, mdo, mk, mv, p);
   if ((e = cudaGetLastError()) != cudaSuccess) return cuda_fail(e, "attn_bwd_q launch");
   return SA_OK;
 }
