@@ -146,31 +146,77 @@ __device__ __forceinline__ uint32_t bwd_pack(float lo, float hi) {
   return *reinterpret_cast<uint32_t*>(&h);
 }
 
-// One 32-column chunk of a P / dS half for the calling thread's row: s, dp = 32 fp32
-// columns of S and dP; nl, nd = -lse2 and -Delta of each column (pairs); columns
-// lo <= i < hi are visible (the rest get P = dS = 0; lo <= 0, hi >= 32 takes the unmasked
-// path).  P = 2^(c2 s - lse2), dS = P (dP - Delta) on packed f32x2 pairs, written as 16
-// packed 16-bit pairs each.
-template <bool BF16>
-__device__ __forceinline__ void bwd_chunk(const uint32_t (&s)[32], const uint32_t (&dp)[32], f32x2 c2,
-                                          const f32x2 (&nl)[16], const f32x2 (&nd)[16], int lo, int hi,
-                                          uint32_t (&pp)[16], uint32_t (&dsp)[16]) {
-  const bool full = lo <= 0 && hi >= 32;
+// Tensor-memory loads / stores of 16 and 8 columns (32 lanes x 32-bit, one lane per thread).
+__device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t (&r)[16]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x16.b32 "
+      "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+        "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
+      : "r"(taddr));
+}
+__device__ __forceinline__ void tmem_st8(uint32_t taddr, const uint32_t (&r)[8]) {
+  asm volatile("tcgen05.st.sync.aligned.32x32b.x8.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8};"
+               ::"r"(taddr), "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]),
+                 "r"(r[6]), "r"(r[7])
+               : "memory");
+}
+// tcgen05.wait::ld naming the 32 registers of the loads it waits for (no use of them can be
+// scheduled above it)
+__device__ __forceinline__ void tmem_wait_ld_2x16(uint32_t (&a)[16], uint32_t (&b)[16]) {
+  asm volatile("tcgen05.wait::ld.sync.aligned;"
+               : "+r"(a[0]), "+r"(a[1]), "+r"(a[2]), "+r"(a[3]), "+r"(a[4]), "+r"(a[5]), "+r"(a[6]),
+                 "+r"(a[7]), "+r"(a[8]), "+r"(a[9]), "+r"(a[10]), "+r"(a[11]), "+r"(a[12]), "+r"(a[13]),
+                 "+r"(a[14]), "+r"(a[15]), "+r"(b[0]), "+r"(b[1]), "+r"(b[2]), "+r"(b[3]), "+r"(b[4]),
+                 "+r"(b[5]), "+r"(b[6]), "+r"(b[7]), "+r"(b[8]), "+r"(b[9]), "+r"(b[10]), "+r"(b[11]),
+                 "+r"(b[12]), "+r"(b[13]), "+r"(b[14]), "+r"(b[15])
+               :: "memory");
+}
+
+// P and dS of one 64-column half for the calling thread's row (S at s_addr, dP at dp_addr,
+// fp32 columns).  nl(j), nd(j) = -lse2 and -Delta of columns (2j, 2j+1) as a packed pair;
+// columns lo <= c < hi are visible (the rest get P = dS = 0).  P = 2^(c2 s - lse2) and
+// dS = P (dP - Delta) on packed f32x2 pairs; dS (and, if STORE_P, P) go back as 16-bit pairs
+// over the half's first 32 columns (pair j at column j).  Four 16-column pieces; the loads
+// of a piece are issued before the arithmetic of the previous one.  A piece's 16-bit pairs
+// land on columns whose fp32 values earlier pieces have already read.
+template <bool BF16, bool STORE_P, typename NL, typename ND>
+__device__ __forceinline__ void bwd_half(uint32_t s_addr, uint32_t dp_addr, f32x2 c2, NL nl, ND nd, int lo, int hi) {
+  const bool full = lo <= 0 && hi >= 64;
+  uint32_t sv[2][16], dv[2][16];
+  tmem_ld16(s_addr, sv[0]);
+  tmem_ld16(dp_addr, dv[0]);
+  tmem_wait_ld_2x16(sv[0], dv[0]);
 #pragma unroll
-  for (int i = 0; i < 16; ++i) {
-    float x0, x1;
-    unpack_f2(fma_f2(pack_f2(__uint_as_float(s[2 * i]), __uint_as_float(s[2 * i + 1])), c2, nl[i]), x0, x1);
-    float p0 = ex2(x0), p1 = ex2(x1);
-    if (!full) {
-      p0 = (2 * i >= lo && 2 * i < hi) ? p0 : 0.f;
-      p1 = (2 * i + 1 >= lo && 2 * i + 1 < hi) ? p1 : 0.f;
+  for (int pc = 0; pc < 4; ++pc) {
+    const int cur = pc & 1;
+    if (pc + 1 < 4) {
+      tmem_ld16(s_addr + 16 * (pc + 1), sv[cur ^ 1]);
+      tmem_ld16(dp_addr + 16 * (pc + 1), dv[cur ^ 1]);
     }
-    const f32x2 d2 = mul_f2(pack_f2(p0, p1),
-                            add_f2(pack_f2(__uint_as_float(dp[2 * i]), __uint_as_float(dp[2 * i + 1])), nd[i]));
-    float d0, d1;
-    unpack_f2(d2, d0, d1);
-    pp[i] = bwd_pack<BF16>(p0, p1);
-    dsp[i] = bwd_pack<BF16>(d0, d1);
+    uint32_t pp[8], dsp[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      const int j = 8 * pc + i, c = 2 * j;        // pair j: columns c, c + 1 of the half
+      float x0, x1;
+      unpack_f2(fma_f2(pack_f2(__uint_as_float(sv[cur][2 * i]), __uint_as_float(sv[cur][2 * i + 1])), c2, nl(j)),
+                x0, x1);
+      float p0 = ex2(x0), p1 = ex2(x1);
+      if (!full) {
+        p0 = (c >= lo && c < hi) ? p0 : 0.f;
+        p1 = (c + 1 >= lo && c + 1 < hi) ? p1 : 0.f;
+      }
+      const f32x2 d2 = mul_f2(pack_f2(p0, p1),
+                              add_f2(pack_f2(__uint_as_float(dv[cur][2 * i]), __uint_as_float(dv[cur][2 * i + 1])),
+                                     nd(j)));
+      float d0, d1;
+      unpack_f2(d2, d0, d1);
+      if (STORE_P) pp[i] = bwd_pack<BF16>(p0, p1);
+      dsp[i] = bwd_pack<BF16>(d0, d1);
+    }
+    if (STORE_P) tmem_st8(s_addr + 8 * pc, pp);
+    tmem_st8(dp_addr + 8 * pc, dsp);
+    if (pc + 1 < 4) tmem_wait_ld_2x16(sv[cur ^ 1], dv[cur ^ 1]);
   }
 }
 
@@ -417,26 +463,13 @@ attn_bwd_kv(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
       tc_fence_after();
       const float* vec = reinterpret_cast<const float*>(sm.slot(n % Cfg::STAGES) + 2 * Cfg::TILE);
       const int qbase = step_qt(n) * 128 + 64 * c;
-#pragma unroll 1
-      for (int ch = 0; ch < 2; ++ch) {
-        uint32_t sv[32], dp[32], pp[16], dsp[16];
-        tmem_ld32(lane_addr + Cfg::S_COL + 64 * c + 32 * ch, sv);
-        tmem_ld32(lane_addr + Cfg::DP_COL + 64 * c + 32 * ch, dp);
-        tmem_wait_ld_regs(sv);
-        tmem_wait_ld_regs(dp);
-        const int col0 = 64 * c + 32 * ch, q0 = qbase + 32 * ch;
-        // visible queries of this key row: q >= key - shift (causal), q < Sq; none past Sk
-        const int lo = p.causal ? key - shift - q0 : 0;
-        const int hi = key < p.Sk ? min(32, p.Sq - q0) : 0;
-        const f32x2* nl2 = reinterpret_cast<const f32x2*>(vec + col0);
-        const f32x2* nd2 = reinterpret_cast<const f32x2*>(vec + 128 + col0);
-        f32x2 nl[16], nd[16];
-#pragma unroll
-        for (int i = 0; i < 16; ++i) { nl[i] = nl2[i]; nd[i] = nd2[i]; }
-        bwd_chunk<BF16>(sv, dp, c2x2, nl, nd, lo, hi, pp, dsp);
-        tmem_st16(lane_addr + Cfg::S_COL + 64 * c + 16 * ch, pp);
-        tmem_st16(lane_addr + Cfg::DP_COL + 64 * c + 16 * ch, dsp);
-      }
+      // visible queries of this key row: q >= key - shift (causal), q < Sq; none past Sk
+      const int lo = p.causal ? key - shift - qbase : 0;
+      const int hi = key < p.Sk ? min(64, p.Sq - qbase) : 0;
+      const f32x2* nl2 = reinterpret_cast<const f32x2*>(vec + 64 * c);
+      const f32x2* nd2 = reinterpret_cast<const f32x2*>(vec + 128 + 64 * c);
+      bwd_half<BF16, true>(lane_addr + Cfg::S_COL + 64 * c, lane_addr + Cfg::DP_COL + 64 * c, c2x2,
+                           [&](int j) { return nl2[j]; }, [&](int j) { return nd2[j]; }, lo, hi);
       tmem_wait_st();
       tc_fence_before();
       mbar_arrive(&sm.p_ready[c]);
@@ -556,28 +589,17 @@ attn_bwd_q(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUt
     const float nl1 = p.nlse2[vrow], nd1 = p.ndelta[vrow];
     const int klim = p.causal ? q + p.Sk - p.Sq : p.Sk - 1;          // last key this row sees
     const f32x2 c2x2 = pack_f2(p.c2, p.c2);
-    f32x2 nl[16], nd[16];
-#pragma unroll
-    for (int i = 0; i < 16; ++i) { nl[i] = pack_f2(nl1, nl1); nd[i] = pack_f2(nd1, nd1); }
+    const f32x2 nlp = pack_f2(nl1, nl1), ndp = pack_f2(nd1, nd1);
     bool ok = true;
     for (int n = 0; n < nsteps; ++n) {
       ok = mbar_wait_warp(&sm.s_ready[c], n & 1, sm.abort_flag, 77 + c);
       if (!ok) break;
       tc_fence_after();
       const int kbase = n * 128 + 64 * c;
-#pragma unroll 1
-      for (int ch = 0; ch < 2; ++ch) {
-        uint32_t sv[32], dp[32], pp[16], dsp[16];
-        tmem_ld32(lane_addr + Cfg::S_COL + 64 * c + 32 * ch, sv);
-        tmem_ld32(lane_addr + Cfg::DP_COL + 64 * c + 32 * ch, dp);
-        tmem_wait_ld_regs(sv);
-        tmem_wait_ld_regs(dp);
-        const int k0 = kbase + 32 * ch;
-        // visible keys of this row: k <= klim, k < Sk; none for padding rows
-        const int hi = q < p.Sq ? min(p.Sk, klim + 1) - k0 : 0;
-        bwd_chunk<BF16>(sv, dp, c2x2, nl, nd, 0, hi, pp, dsp);
-        tmem_st16(lane_addr + Cfg::DP_COL + 64 * c + 16 * ch, dsp);
-      }
+      // visible keys of this row: k <= klim, k < Sk; none for padding rows
+      const int hi = q < p.Sq ? min(p.Sk, klim + 1) - kbase : 0;
+      bwd_half<BF16, false>(lane_addr + Cfg::S_COL + 64 * c, lane_addr + Cfg::DP_COL + 64 * c, c2x2,
+                            [&](int) { return nlp; }, [&](int) { return ndp; }, 0, hi);
       tmem_wait_st();
       tc_fence_before();
       mbar_arrive(&sm.p_ready[c]);
