@@ -135,6 +135,12 @@ __device__ __forceinline__ void mma_ts_x4(uint32_t d_tmem, uint32_t a_tmem, uint
       ::"r"(d_tmem), "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(acc_first), "r"(1u) : "memory");
 }
 
+__device__ __forceinline__ f32x2 mul_f2(f32x2 a, f32x2 b) {
+  f32x2 d;
+  asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
+
 // 16-bit pair of two fp32 values (round to nearest even)
 template <bool BF16>
 __device__ __forceinline__ uint32_t bwd_pack(float lo, float hi) {

@@ -359,11 +359,6 @@ __device__ __forceinline__ f32x2 add_f2(f32x2 a, f32x2 b) {
   asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
   return d;
 }
-__device__ __forceinline__ f32x2 mul_f2(f32x2 a, f32x2 b) {
-  f32x2 d;
-  asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
-  return d;
-}
 // max of three fp32 values in one instruction (sm_100)
 __device__ __forceinline__ float max3f(float a, float b, float c) {
   float d;
