@@ -21,7 +21,7 @@ from __future__ import annotations
 
 import torch
 
-DTYPES = {"fp16": torch.float16, "bf16": torch.bfloat16}
+DTYPES = {"fp16": torch.float16, "bf16": torch.bfloat16, "fp32": torch.float32}
 
 
 def make_qkv(B, Sq, Sk, Hq, Hkv, D, dtype="fp16", seed=0, input_scale=1.0,
@@ -117,3 +117,21 @@ def make_dout(B, Sq, Hq, D, dtype="fp16", seed=0):
     g = torch.Generator(device="cpu")
     g.manual_seed(int(seed) + 7777)
     return torch.randn((B, Sq, Hq, D), generator=g, dtype=torch.float32).to(DTYPES[dtype]).contiguous()
+
+
+def quantize_e4m3(x):
+    """Per-tensor FP8 quantisation of a float tensor: descale = max |x| / 448 (448 is the
+    largest e4m3 value), codes = x / descale rounded to e4m3 (torch's float8_e4m3fn
+    conversion, round to nearest even), returned as a uint8 tensor of codes and the float
+    descale factor (x ~ value(codes) * descale)."""
+    amax = float(x.abs().max())
+    d = amax / 448.0 if amax > 0 else 1.0
+    return (x / d).to(torch.float8_e4m3fn).view(torch.uint8).contiguous(), d
+
+
+def make_qkv_fp8(B, Sq, Sk, Hq, Hkv, D, seed=0, input_scale=1.0, k_sink_rows=0, k_sink_factor=1.0):
+    """make_qkv's float32 draws (same recipe and seed), each tensor quantised to e4m3 with
+    its own descale: returns (q8, k8, v8, q_descale, k_descale, v_descale)."""
+    q, k, v = make_qkv(B, Sq, Sk, Hq, Hkv, D, "fp32", seed, input_scale, k_sink_rows, k_sink_factor)
+    (q8, qd), (k8, kd), (v8, vd) = quantize_e4m3(q), quantize_e4m3(k), quantize_e4m3(v)
+    return q8, k8, v8, qd, kd, vd

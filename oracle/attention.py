@@ -275,6 +275,28 @@ def attention_backward(q, k, v, do, scale, causal=False):
     return dq, dk, dv
 
 
+def decode_e4m3(codes):
+    """Values of 8-bit e4m3 codes (sign bit, 4-bit exponent with bias 7, 3-bit mantissa;
+    exponent 0 = subnormal m * 2^-9; 0x7f / 0xff = NaN; no infinities; largest 448) as
+    float64 -- the FP8 format the Stem page's fp8 prefill path and the StreamAttention
+    page's FP8 roadmap item name, written out from its definition."""
+    c = np.asarray(codes, dtype=np.uint8).astype(np.int64)
+    sign = np.where(c & 0x80, -1.0, 1.0)
+    e = (c >> 3) & 0xF
+    m = (c & 0x7).astype(np.float64)
+    val = np.where(e == 0, m * 2.0 ** -9, (1.0 + m / 8.0) * np.exp2(e.astype(np.float64) - 7.0))
+    val = np.where((c & 0x7F) == 0x7F, np.nan, val)
+    return sign * val
+
+
+def attention_fp8(q8, k8, v8, q_descale, k_descale, v_descale, scale, causal=False):
+    """Attention on FP8 inputs: :func:`attention` of the dequantised tensors
+    decode_e4m3(q8) * q_descale, decode_e4m3(k8) * k_descale, decode_e4m3(v8) * v_descale
+    (per-tensor descale factors).  Shapes as :func:`attention`."""
+    return attention(decode_e4m3(q8) * q_descale, decode_e4m3(k8) * k_descale, decode_e4m3(v8) * v_descale,
+                     scale, causal)
+
+
 def attention_blockwise(q, k, v, scale, causal=False, block=64):
     """The online-softmax recurrence, restated in float64 (TurboQuant page,
     ``online_softmax_attention``; StreamAttention page, "Kernel Design"): walk the

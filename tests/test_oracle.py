@@ -594,3 +594,35 @@ def test_backward_rows_without_keys_contribute_nothing():
     dq2, dk2, dv2 = attention_backward(q, k, v, do2, 0.8, True)
     np.testing.assert_allclose(dk2, dk, atol=TOL)
     np.testing.assert_allclose(dv2, dv, atol=TOL)
+
+
+# ---- FP8 (e4m3) inputs
+
+def test_decode_e4m3_known_codes():
+    from oracle import decode_e4m3
+    table = {0x00: 0.0, 0x38: 1.0, 0xB8: -1.0, 0x40: 2.0, 0x3C: 1.5, 0x7E: 448.0, 0xFE: -448.0,
+             0x08: 2.0 ** -6, 0x01: 2.0 ** -9, 0x07: 7 * 2.0 ** -9, 0x30: 0.5, 0x77: 240.0}
+    for code, val in table.items():
+        assert decode_e4m3([code])[0] == val, hex(code)
+    assert np.isnan(decode_e4m3([0x7F])[0]) and np.isnan(decode_e4m3([0xFF])[0])
+
+
+def test_decode_e4m3_matches_torch_float8():
+    # every code against the library's own float8_e4m3fn -> float conversion
+    import torch
+    from oracle import decode_e4m3
+    codes = np.arange(256, dtype=np.uint8)
+    lib = torch.from_numpy(codes).view(torch.float8_e4m3fn).to(torch.float64).numpy()
+    ours = decode_e4m3(codes)
+    np.testing.assert_array_equal(np.isnan(ours), np.isnan(lib))
+    np.testing.assert_array_equal(ours[~np.isnan(ours)], lib[~np.isnan(lib)])
+
+
+def test_attention_fp8_is_attention_of_the_dequantised_inputs():
+    from oracle import attention_fp8, decode_e4m3
+    rng = np.random.default_rng(3)
+    q8, k8, v8 = (rng.integers(0, 0x7E, size=s, dtype=np.uint8) for s in ((1, 5, 2, 4), (1, 7, 1, 4), (1, 7, 1, 4)))
+    O, L = attention_fp8(q8, k8, v8, 0.01, 0.02, 0.5, 0.7, True)
+    Od, Ld = attention(decode_e4m3(q8) * 0.01, decode_e4m3(k8) * 0.02, decode_e4m3(v8) * 0.5, 0.7, True)
+    np.testing.assert_allclose(O, Od, atol=TOL)
+    np.testing.assert_allclose(L, Ld, atol=TOL)
