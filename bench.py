@@ -200,7 +200,8 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
     ap.add_argument("--no-e2e", action="store_true")
-    ap.add_argument("--only", default="all", choices=["all", "prefill", "decode", "varlen", "sparse", "backward"],
+    ap.add_argument("--only", default="all",
+                    choices=["all", "prefill", "decode", "varlen", "sparse", "backward", "fp8"],
                     help="profiling aid: run only one half of the step (the JSON line is then partial)")
     ap.add_argument("--prefill-seq", type=int, default=0,
                     help="profiling aid: shorter prefill sequence (same heads, dtype, sinks)")
@@ -217,10 +218,11 @@ def main():
                                                    sa_attn_decode_paged_workspace_size,
                                                    sa_attn_decode_workspace_size, sa_attn_fwd,
                                                    sa_attn_fwd_block_sparse, sa_attn_fwd_block_sparse_workspace_size,
-                                                   sa_attn_bwd, sa_attn_bwd_workspace_size,
+                                                   sa_attn_bwd, sa_attn_bwd_workspace_size, sa_attn_fwd_fp8,
                                                    sa_attn_fwd_varlen, sa_check_status)
     from online_softmax_attention_sm_b200.dist import aggregate_throughput, max_over_ranks, rank_seed
-    from online_softmax_attention_sm_b200.inputs import make_dout, make_qkv, make_workload_inputs, stem_block_mask
+    from online_softmax_attention_sm_b200.inputs import (make_dout, make_qkv, make_qkv_fp8, make_workload_inputs,
+                                                         stem_block_mask)
     from online_softmax_attention_sm_b200.workloads import WORKLOADS, block_sparse_flops
 
     rank, world, local = dist_env()
@@ -240,6 +242,7 @@ def main():
     run_var = args.only in ("all", "varlen")
     run_sparse = args.only in ("all", "sparse")
     run_bwd = args.only in ("all", "backward")
+    run_fp8 = args.only in ("all", "fp8")
     q_h, k_h, v_h = make_workload_inputs(wp, seed=rank_seed(wp.seed, rank))
     dq_h, dk_h, dv_h = make_workload_inputs(wd, seed=rank_seed(wd.seed, rank))
     q, k, v = q_h.to(dev), k_h.to(dev), v_h.to(dev)
@@ -405,6 +408,28 @@ def main():
         bwd_ms = [a.elapsed_time(b) for a, b in bev]
         del dout, gq, gk, gv, bws
 
+    # FP8 forward: the prefill workload's draws quantised to e4m3 per tensor (same seed)
+    fp8_ms = [float("nan")]
+    if run_fp8:
+        q8, k8, v8, qd8, kd8, vd8 = make_qkv_fp8(wp.B, wp.Sq, wp.Sk, wp.Hq, wp.Hkv, wp.D, seed=rank_seed(wp.seed, rank),
+                                                 input_scale=wp.input_scale, k_sink_rows=wp.k_sink_rows,
+                                                 k_sink_factor=wp.k_sink_factor)
+        q8, k8, v8 = q8.to(dev), k8.to(dev), v8.to(dev)
+        o8 = torch.empty((wp.B, wp.Sq, wp.Hq, wp.D), dtype=torch.bfloat16, device=dev)
+        fev = []
+        for i in range(args.warmup + args.steps):
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            sa_attn_fwd_fp8(q8, k8, v8, qd8, kd8, vd8, causal=wp.causal, scale=wp.scale, out=o8, lse=lse,
+                            stream=stream)
+            e1.record(stream)
+            if i >= args.warmup:
+                fev.append((e0, e1))
+        torch.cuda.synchronize(dev)
+        sa_check_status(stream)
+        fp8_ms = [a.elapsed_time(b) for a, b in fev]
+        del q8, k8, v8, o8
+
     # e2e through the public API with host buffers: H2D of the step's inputs, D2H of outputs
     e2e_ms = None
     h2d = sum(t.numel() * t.element_size() for t in (q_h, k_h, v_h, dq_h, dk_h, dv_h))
@@ -441,6 +466,7 @@ def main():
     var_avg = max_over_ranks(sum(var_ms) / len(var_ms), dev)
     sp_avg = max_over_ranks(sum(sp_ms) / len(sp_ms), dev)
     bwd_avg = max_over_ranks(sum(bwd_ms) / len(bwd_ms), dev)
+    fp8_avg = max_over_ranks(sum(fp8_ms) / len(fp8_ms), dev)
     e2e_ms = max_over_ranks(e2e_ms, dev) if e2e_ms is not None else None
 
     if rank == 0:
@@ -501,6 +527,11 @@ def main():
                          "flops": "2.5 x the forward's (5 tile products against 2; the dQ kernel's "
                                   "recomputed S and dP are not credited)",
                          "kernels": "bwd_prep + attn_bwd_kv + attn_bwd_q"},
+            "prefill_fp8": {"workload": f"{PREFILL}, Q/K/V in e4m3 (per-tensor descale)",
+                            "value": wp.flops / (fp8_avg * 1e-3) / 1e12, "unit": "TFLOP/s", "bound": "tensor",
+                            "peak": 2 * peak, "peak_source": "measured bf16 burst x 2 (nominal fp8 : bf16)",
+                            "frac": wp.flops / (fp8_avg * 1e-3) / 1e12 / (2 * peak), "ms": fp8_avg,
+                            "kernel": "attn_fwd_sm100 (FP8 instance: kind::f8f6f4 QK and PV, e4m3 P)"},
             "prefill_ms": pre_avg,
             "gpu_launches": (int(run_pre) + 2 * int(run_dec)) * args.steps,
             "clocks": clk.summary(),

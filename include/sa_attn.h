@@ -119,6 +119,18 @@ int sa_attn_fwd_block_sparse(const void* q, const void* k, const void* v, void* 
                              void* workspace, size_t workspace_bytes, sa_stream_t stream);
 
 /*
+ * FP8 forward (the Stem page's fp8 prefill path; the StreamAttention page's FP8 roadmap
+ * item): q, k, v are e4m3 codes (one byte per element, layouts as sa_attn_fwd) with
+ * per-tensor descale factors, o is bf16 [B, Sq, Hq, D], lse fp32 [B, Hq, Sq] or NULL.
+ * Computes sa_attn_fwd of the dequantised tensors q*q_descale, k*k_descale, v*v_descale:
+ * S on kind::f8f6f4 tensor cores (exact products, fp32 sums), P rounded to e4m3 for P V.
+ * D must be 128 (else SA_ERR_UNSUPPORTED); descales finite and > 0 (else SA_ERR_INVALID).
+ */
+int sa_attn_fwd_fp8(const void* q, const void* k, const void* v, void* o, float* lse,
+                    int B, int Sq, int Sk, int Hq, int Hkv, int D, int causal, float scale,
+                    float q_descale, float k_descale, float v_descale, sa_stream_t stream);
+
+/*
  * Attention backward: dQ, dK, dV of the forward's O for an upstream gradient dO
  * (StreamAttention page, "Backward": the QK tiles are recomputed from the saved LSE and
  * dQ/dK/dV are streamed, never the attention matrix; flash-attn-volta page, backward).

@@ -45,14 +45,16 @@ constexpr int kUnitQueue = 4;    // unit indices the load warp may hand out ahea
 constexpr int kSparseMaxKTiles = 1024;                       // keys <= 131072
 constexpr int kSparseSlotBytes = 16 + 2 * kSparseMaxKTiles;  // header + longest list
 
-template <int D>
+// FP8: Q, K, V in e4m3 (one byte per element), the instance's products kind::f8f6f4.
+template <int D, bool FP8 = false>
 struct FwdCfg {
   static constexpr int BM = 128;                     // query rows per Q tile
   static constexpr int BN = 128;                     // keys per K/V tile
-  static constexpr int KCH = D / 64;                 // 128-byte chunks along D
-  static constexpr int CHUNK_BYTES = 128 * 128;      // one 128-row x 64-element box
+  static constexpr int CHUNK_ELEMS = FP8 ? 128 : 64; // elements in a 128-byte row
+  static constexpr int KCH = D / CHUNK_ELEMS;        // 128-byte chunks along D
+  static constexpr int CHUNK_BYTES = 128 * 128;      // one 128-row x 128-byte box
   static constexpr int TILE_BYTES = KCH * CHUNK_BYTES;
-  static constexpr int STAGES = (D == 128) ? 4 : 8;  // K/V ring slots
+  static constexpr int STAGES = TILE_BYTES == 2 * CHUNK_BYTES ? 4 : 8;  // K/V ring slots (128 KB)
   static constexpr int SMEM_Q = 2 * TILE_BYTES;
   static constexpr int SMEM_RING = STAGES * TILE_BYTES;
   static constexpr int SMEM_BARS = 1024;
@@ -102,6 +104,7 @@ struct FwdParams {
   // record (b * Hq + h) * n_qblk + query block.
   const uint16_t* sp;
   int sp_stride;
+  float o_mul;          // O scale in the epilogue: the V descale of the FP8 instance, else 1
 };
 
 struct UnitInfo {
@@ -190,9 +193,9 @@ __device__ __forceinline__ int fwd_unit_of(int round, int cta, int ncta) {
   return round * ncta + ((round & 1) ? (ncta - 1 - cta) : cta);
 }
 // Shared-memory map: Q tiles, K/V ring, then the barriers and two words.
-template <int D>
+template <int D, bool FP8 = false>
 struct FwdSmem {
-  using Cfg = FwdCfg<D>;
+  using Cfg = FwdCfg<D, FP8>;
   uint8_t* q;          // [2][TILE]
   uint8_t* ring;       // [STAGES][TILE]
   uint64_t* kv_full;   // [STAGES]
@@ -236,8 +239,8 @@ struct FwdSmem {
 // it, release the queue slot (one arrival per warp) unless the unit's shared-memory record
 // is still needed (block-sparse: released by fwd_release_unit at the unit's end).
 // Returns -1 if the wait gave up.
-template <int D>
-__device__ __forceinline__ int fwd_next_unit(const FwdSmem<D>& sm, int n, int where, bool release = true) {
+template <class SM>
+__device__ __forceinline__ int fwd_next_unit(const SM& sm, int n, int where, bool release = true) {
   const int slot = n % kUnitQueue;
   if (!mbar_wait_warp(&sm.unit_full[slot], (n / kUnitQueue) & 1, sm.abort_flag, where)) return -1;
   const int u = sm.uq[slot];
@@ -245,8 +248,8 @@ __device__ __forceinline__ int fwd_next_unit(const FwdSmem<D>& sm, int n, int wh
   return u;
 }
 
-template <int D>
-__device__ __forceinline__ void fwd_release_unit(const FwdSmem<D>& sm, int n) {
+template <class SM>
+__device__ __forceinline__ void fwd_release_unit(const SM& sm, int n) {
   mbar_arrive_warp(&sm.unit_empty[n % kUnitQueue]);
 }
 
@@ -255,8 +258,8 @@ __device__ __forceinline__ void fwd_release_unit(const FwdSmem<D>& sm, int n) {
 __device__ __forceinline__ const uint16_t* fwd_sparse_record(const FwdParams& p, const UnitInfo& x) {
   return p.sp + ((size_t)(x.b * p.Hq + x.h) * p.n_qblk + x.q0 / 256) * p.sp_stride;
 }
-template <int D>
-__device__ __forceinline__ void fwd_sparse_attach(const FwdSmem<D>& sm, int slot, UnitInfo& x) {
+template <class SM>
+__device__ __forceinline__ void fwd_sparse_attach(const SM& sm, int slot, UnitInfo& x) {
   const uint16_t* rec = reinterpret_cast<const uint16_t*>(sm.lists + slot * kSparseSlotBytes);
   x.nkv_max = rec[0];
   x.nkv[0] = rec[1];
@@ -265,11 +268,11 @@ __device__ __forceinline__ void fwd_sparse_attach(const FwdSmem<D>& sm, int slot
 }
 
 // ------------------------------------------------------------------ TMA producer
-template <int D, bool BF16, bool DYN, bool SPARSE>
+template <int D, bool BF16, bool DYN, bool SPARSE, bool FP8>
 __device__ __forceinline__ void fwd_producer(const CUtensorMap* tm_q, const CUtensorMap* tm_k,
                                              const CUtensorMap* tm_v, const FwdParams& p,
-                                             const FwdSmem<D>& sm, int lane, int cta, int ncta) {
-  using Cfg = FwdCfg<D>;
+                                             const FwdSmem<D, FP8>& sm, int lane, int cta, int ncta) {
+  using Cfg = FwdCfg<D, FP8>;
   if (lane == 0) {
     int slot = 0, ring_n = 0;            // ring position and total loads issued
     int q_load0 = 0, q_load1 = 0;        // Q tile loads issued
@@ -318,7 +321,8 @@ __device__ __forceinline__ void fwd_producer(const CUtensorMap* tm_q, const CUte
           const CUtensorMap* tm = kv ? tm_v : tm_k;
 #pragma unroll
           for (int c = 0; c < Cfg::KCH; ++c)
-            tma_load_4d(dst + c * Cfg::CHUNK_BYTES, tm, &sm.kv_full[slot], c * 64, x.kvh, x.kbase + kt * 128, x.mb);
+            tma_load_4d(dst + c * Cfg::CHUNK_BYTES, tm, &sm.kv_full[slot], c * Cfg::CHUNK_ELEMS, x.kvh,
+                        x.kbase + kt * 128, x.mb);
           ++ring_n;
           slot = (slot + 1 == Cfg::STAGES) ? 0 : slot + 1;
           if (j == 0 && kv == 0) {
@@ -334,7 +338,7 @@ __device__ __forceinline__ void fwd_producer(const CUtensorMap* tm_q, const CUte
               mbar_arrive_expect_tx(&sm.q_full[t], Cfg::TILE_BYTES);
 #pragma unroll
               for (int c = 0; c < Cfg::KCH; ++c)
-                tma_load_4d(qd + c * Cfg::CHUNK_BYTES, tm_q, &sm.q_full[t], c * 64, x.h,
+                tma_load_4d(qd + c * Cfg::CHUNK_BYTES, tm_q, &sm.q_full[t], c * Cfg::CHUNK_ELEMS, x.h,
                             x.qbase + x.q0 + t * 128, x.mb);
               ++ql;
             }
@@ -364,14 +368,59 @@ __device__ __forceinline__ void fwd_producer(const CUtensorMap* tm_q, const CUte
 }
 
 // ------------------------------------------------------------------ MMA issuer
-template <int D, bool BF16, bool DYN, bool SPARSE>
-__device__ __forceinline__ void fwd_mma(const FwdParams& p, const FwdSmem<D>& sm, uint32_t tmem_base,
+// 4 k-steps of a shared x shared product along one 128-byte row: kind::f16 (16 elements a
+// step) or, for FP8, kind::f8f6f4 (32 e4m3 elements a step); both step 32 bytes.
+template <bool FP8>
+__device__ __forceinline__ void qk_mma_x4(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
+                                          uint32_t acc_first) {
+  if constexpr (!FP8) {
+    mma_ss_x4(d_tmem, a_desc, b_desc, idesc, acc_first);
+  } else {
+    asm volatile(
+        "{\n .reg .pred e, p, q;\n .reg .b32 r;\n .reg .b64 a, b;\n"
+        " elect.sync r|e, 0xffffffff;\n setp.ne.b32 p, %4, 0;\n setp.ne.b32 q, %5, 0;\n"
+        " @e tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], %1, %2, %3, p;\n"
+        " add.s64 a, %1, 2;\n add.s64 b, %2, 2;\n"
+        " @e tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], a, b, %3, q;\n"
+        " add.s64 a, %1, 4;\n add.s64 b, %2, 4;\n"
+        " @e tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], a, b, %3, q;\n"
+        " add.s64 a, %1, 6;\n add.s64 b, %2, 6;\n"
+        " @e tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], a, b, %3, q;\n}\n"
+        ::"r"(d_tmem), "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(acc_first), "r"(1u) : "memory");
+  }
+}
+// kind::f8f6f4 with A (e4m3 P) in tensor memory: a k-step is 32 keys = 8 columns of 4
+// values; B (V, MN-major) steps 32 rows of 128 bytes (4096 bytes).  x3: keys 0-95, x1: one step.
+__device__ __forceinline__ void mma_ts_f8_x3(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc, uint32_t idesc,
+                                             uint32_t acc_first) {
+  asm volatile(
+      "{\n .reg .pred e, p, q;\n .reg .b32 r, a;\n .reg .b64 b;\n"
+      " elect.sync r|e, 0xffffffff;\n setp.ne.b32 p, %4, 0;\n setp.ne.b32 q, %5, 0;\n"
+      " @e tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], [%1], %2, %3, p;\n"
+      " add.u32 a, %1, 8;\n add.s64 b, %2, 256;\n"
+      " @e tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], [a], b, %3, q;\n"
+      " add.u32 a, %1, 16;\n add.s64 b, %2, 512;\n"
+      " @e tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], [a], b, %3, q;\n}\n"
+      ::"r"(d_tmem), "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(acc_first), "r"(1u) : "memory");
+}
+__device__ __forceinline__ void mma_ts_f8_x1(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc, uint32_t idesc,
+                                             uint32_t acc) {
+  asm volatile(
+      "{\n .reg .pred e, p;\n .reg .b32 r;\n"
+      " elect.sync r|e, 0xffffffff;\n setp.ne.b32 p, %4, 0;\n"
+      " @e tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], [%1], %2, %3, p;\n}\n"
+      ::"r"(d_tmem), "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(acc) : "memory");
+}
+
+template <int D, bool BF16, bool DYN, bool SPARSE, bool FP8>
+__device__ __forceinline__ void fwd_mma(const FwdParams& p, const FwdSmem<D, FP8>& sm, uint32_t tmem_base,
                                         int lane, int cta, int ncta) {
-  using Cfg = FwdCfg<D>;
+  using Cfg = FwdCfg<D, FP8>;
   (void)lane;
   {
-    constexpr uint32_t IDESC_QK = idesc_f16(BF16 ? 1 : 0, 128, 128, 0, 0);
-    constexpr uint32_t IDESC_PV = idesc_f16(BF16 ? 1 : 0, 128, D, 0, 1);
+    // (e4m3 is format 0 of kind::f8f6f4, in the same descriptor fields)
+    constexpr uint32_t IDESC_QK = idesc_f16((BF16 && !FP8) ? 1 : 0, 128, 128, 0, 0);
+    constexpr uint32_t IDESC_PV = idesc_f16((BF16 && !FP8) ? 1 : 0, 128, D, 0, 1);
     const uint32_t sQ_addr = smem_u32(sm.q);
     const uint32_t sRing_addr = smem_u32(sm.ring);
     int ring_n = 0;                       // ring position of this unit's first K tile
@@ -383,8 +432,8 @@ __device__ __forceinline__ void fwd_mma(const FwdParams& p, const FwdSmem<D>& sm
       // D / 16 k-steps: 4 per 64-element (128-byte) chunk of the head dimension
 #pragma unroll
       for (int c = 0; c < Cfg::KCH; ++c)
-        mma_ss_x4(tmem_base + Cfg::S_COL(t), smem_desc_sw128(q_addr + c * Cfg::CHUNK_BYTES, 16, 1024),
-                  smem_desc_sw128(k_addr + c * Cfg::CHUNK_BYTES, 16, 1024), IDESC_QK, c > 0);
+        qk_mma_x4<FP8>(tmem_base + Cfg::S_COL(t), smem_desc_sw128(q_addr + c * Cfg::CHUNK_BYTES, 16, 1024),
+                       smem_desc_sw128(k_addr + c * Cfg::CHUNK_BYTES, 16, 1024), IDESC_QK, c > 0);
       mma_commit_warp(&sm.s_full[t]);
     };
     // Issue order per K/V step j:  PV_0(j), QK_0(j+1), PV_1(j), QK_1(j+1).
@@ -443,13 +492,21 @@ __device__ __forceinline__ void fwd_mma(const FwdParams& p, const FwdSmem<D>& sm
             if (!ok) break;
             tc_fence_after();
             const uint32_t acc = SPARSE ? (npv[t] > 0 ? 1u : 0u) : (j > 0 ? 1u : 0u);
-            mma_ts_x6(tmem_base + Cfg::O_COL(t), tmem_base + Cfg::P_COL(t),
-                      smem_desc_sw128(v_addr, Cfg::CHUNK_BYTES, 1024), IDESC_PV, acc);
+            if (FP8)   // keys 0-95: three k-steps of 32 (8 columns of 4 e4m3 P values, 32 V rows each)
+              mma_ts_f8_x3(tmem_base + Cfg::O_COL(t), tmem_base + Cfg::P_COL(t),
+                           smem_desc_sw128(v_addr, Cfg::CHUNK_BYTES, 1024), IDESC_PV, acc);
+            else
+              mma_ts_x6(tmem_base + Cfg::O_COL(t), tmem_base + Cfg::P_COL(t),
+                        smem_desc_sw128(v_addr, Cfg::CHUNK_BYTES, 1024), IDESC_PV, acc);
             ok = mbar_wait_warp(&sm.p_full[t], (t ? pv1 : pv0) & 1, sm.abort_flag, 14);
             if (!ok) break;
             tc_fence_after();
-            mma_ts_x2(tmem_base + Cfg::O_COL(t), tmem_base + Cfg::P_COL(t) + 6 * 8,
-                      smem_desc_sw128(v_addr + 6 * 2048, Cfg::CHUNK_BYTES, 1024), IDESC_PV, 1u);
+            if (FP8)
+              mma_ts_f8_x1(tmem_base + Cfg::O_COL(t), tmem_base + Cfg::P_COL(t) + 3 * 8,
+                           smem_desc_sw128(v_addr + 3 * 4096, Cfg::CHUNK_BYTES, 1024), IDESC_PV, 1u);
+            else
+              mma_ts_x2(tmem_base + Cfg::O_COL(t), tmem_base + Cfg::P_COL(t) + 6 * 8,
+                        smem_desc_sw128(v_addr + 6 * 2048, Cfg::CHUNK_BYTES, 1024), IDESC_PV, 1u);
             const bool last = SPARSE ? (++npv[t] == x.nkv[t]) : (j + 1 == x.nkv[t]);
             if (last) mma_commit_warp(&sm.o_done[t]);   // O_t complete for the epilogue
             if (t) ++pv1; else ++pv0;
@@ -557,6 +614,49 @@ __device__ __forceinline__ void softmax_chunk(const uint32_t (&v)[32], const f32
   tmem_st16(taddr, pk);
 }
 
+// FP8 instance: the same chunk with P rounded to e4m3 (round to nearest even, saturating:
+// p <= 2^8 under the lazy reference, below e4m3's 448), 4 values per tensor-memory column
+// (key 4j in the low byte of column j), 8 columns at taddr; rs2 sums the e4m3 values the
+// MMA multiplies.
+template <int POLY>
+__device__ __forceinline__ void softmax_chunk_fp8(const uint32_t (&v)[32], const f32x2 scale2,
+                                                  const f32x2 negm2, f32x2 (&rs2)[2], f32x2 (&rse2)[2],
+                                                  const uint32_t taddr) {
+  uint32_t pk[8];
+#pragma unroll
+  for (int i = 0; i < 16; ++i) {
+    float x0, x1;
+    unpack_f2(fma_f2(pack_f2(__uint_as_float(v[2 * i]), __uint_as_float(v[2 * i + 1])), scale2, negm2), x0, x1);
+    float a, b2;
+    if (POLY > 0 && (i % (POLY > 0 ? POLY : 1)) == POLY - 1) {
+      exp2_poly_pair(x0, x1, a, b2);
+    } else {
+      a = ex2(x0);
+      b2 = ex2(x1);
+    }
+    rse2[i & 1] = add_f2(rse2[i & 1], pack_f2(a, b2));
+    uint16_t e8;          // low byte: key 2i, high byte: key 2i + 1
+    asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(e8) : "f"(b2), "f"(a));
+    uint32_t h2;          // the two e4m3 values back as f16x2, for the row sum
+    asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(h2) : "h"(e8));
+    const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&h2));
+    rs2[i & 1] = add_f2(rs2[i & 1], pack_f2(f.x, f.y));
+    if (i & 1) pk[i >> 1] |= (uint32_t)e8 << 16;
+    else pk[i >> 1] = e8;
+  }
+  asm volatile("tcgen05.st.sync.aligned.32x32b.x8.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8};"
+               ::"r"(taddr), "r"(pk[0]), "r"(pk[1]), "r"(pk[2]), "r"(pk[3]), "r"(pk[4]), "r"(pk[5]),
+                 "r"(pk[6]), "r"(pk[7])
+               : "memory");
+}
+
+template <bool BF16, bool FP8, int POLY>
+__device__ __forceinline__ void softmax_chunk_any(const uint32_t (&v)[32], const f32x2 scale2, const f32x2 negm2,
+                                                  f32x2 (&rs2)[2], f32x2 (&rse2)[2], const uint32_t p_addr, int c) {
+  if constexpr (FP8) softmax_chunk_fp8<POLY>(v, scale2, negm2, rs2, rse2, p_addr + c * 8);
+  else softmax_chunk<BF16, POLY>(v, scale2, negm2, rs2, rse2, p_addr + c * 16);
+}
+
 // Running max over a 32-score chunk on 8 chains.
 __device__ __forceinline__ void chunk_max(const uint32_t (&v)[32], float (&mx)[8]) {
 #pragma unroll
@@ -612,7 +712,7 @@ __device__ __forceinline__ void move_reference(const float m_tile, const bool fi
 // exponentials.  P overwrites S columns 0-63 only, so the second pass holds chunks 0-1
 // from the first and loads chunks 2-3 again, which keeps a quarter fewer registers live
 // through the exponentials.  The MMA warp may start on keys 0-95 at p_part.
-template <int D, bool BF16>
+template <int D, bool BF16, bool FP8>
 __device__ __forceinline__ void softmax_tile_full(const uint32_t s_addr, const uint32_t o_addr,
                                                   const uint32_t p_addr, const float c2, const bool first,
                                                   float& m_ref, float& l_sum, float& l_lse,
@@ -642,23 +742,23 @@ __device__ __forceinline__ void softmax_tile_full(const uint32_t s_addr, const u
   f32x2 rs2[2] = {0ull, 0ull}, rse2[2] = {0ull, 0ull};
   uint32_t v2[32], v3[32];
   tmem_ld32(s_addr + 64, v2);
-  softmax_chunk<BF16, kPolyEvery>(v0, scale2, negm2, rs2, rse2, p_addr);
-  softmax_chunk<BF16, kPolyEvery>(v1, scale2, negm2, rs2, rse2, p_addr + 16);
+  softmax_chunk_any<BF16, FP8, kPolyEvery>(v0, scale2, negm2, rs2, rse2, p_addr, 0);
+  softmax_chunk_any<BF16, FP8, kPolyEvery>(v1, scale2, negm2, rs2, rse2, p_addr, 1);
   tmem_wait_ld_regs(v2);
   tmem_ld32(s_addr + 96, v3);
-  softmax_chunk<BF16, kPolyEvery>(v2, scale2, negm2, rs2, rse2, p_addr + 32);
+  softmax_chunk_any<BF16, FP8, kPolyEvery>(v2, scale2, negm2, rs2, rse2, p_addr, 2);
   tmem_wait_st();
   tc_fence_before();
   mbar_arrive(p_part);
   tmem_wait_ld_regs(v3);
-  softmax_chunk<BF16, kPolyEvery>(v3, scale2, negm2, rs2, rse2, p_addr + 48);
+  softmax_chunk_any<BF16, FP8, kPolyEvery>(v3, scale2, negm2, rs2, rse2, p_addr, 3);
   sum_f2x2(rs2, l_sum);
   sum_f2x2(rse2, l_lse);
 }
 
 // A tile that crosses the causal diagonal or the ragged end of K (or a negative scale):
 // scores are scaled first and keys >= kl set to -inf, then max and exponentials.
-template <int D, bool BF16>
+template <int D, bool BF16, bool FP8>
 __device__ __forceinline__ void softmax_tile_masked(const uint32_t s_addr, const uint32_t o_addr,
                                                     const uint32_t p_addr, const float c2, const int kl,
                                                     const bool first, float& m_ref, float& l_sum,
@@ -684,7 +784,7 @@ __device__ __forceinline__ void softmax_tile_masked(const uint32_t s_addr, const
   f32x2 rs2[2] = {0ull, 0ull}, rse2[2] = {0ull, 0ull};
 #pragma unroll
   for (int c = 0; c < 4; ++c) {
-    softmax_chunk<BF16, 0>(v[c], scale2, negm2, rs2, rse2, p_addr + c * 16);
+    softmax_chunk_any<BF16, FP8, 0>(v[c], scale2, negm2, rs2, rse2, p_addr, c);
     if (c == 2) {
       tmem_wait_st();
       tc_fence_before();
@@ -695,10 +795,10 @@ __device__ __forceinline__ void softmax_tile_masked(const uint32_t s_addr, const
   sum_f2x2(rse2, l_lse);
 }
 
-template <int D, bool BF16, bool DYN, bool SPARSE>
-__device__ __forceinline__ void fwd_softmax(const FwdParams& p, const FwdSmem<D>& sm, uint32_t tmem_base,
+template <int D, bool BF16, bool DYN, bool SPARSE, bool FP8>
+__device__ __forceinline__ void fwd_softmax(const FwdParams& p, const FwdSmem<D, FP8>& sm, uint32_t tmem_base,
                                             int warp, int lane, int cta, int ncta) {
-  using Cfg = FwdCfg<D>;
+  using Cfg = FwdCfg<D, FP8>;
   const int t = warp >> 2;                  // Q tile of this warpgroup (warp: 0-7 here)
   const int wl = warp & 3;                  // TMEM lane quarter (physical warp index % 4)
   const int row_in_tile = wl * 32 + lane;
@@ -740,10 +840,10 @@ __device__ __forceinline__ void fwd_softmax(const FwdParams& p, const FwdSmem<D>
       ++s_n;
       tc_fence_after();
       if (kt < mask_from && c2 >= 0.f) {
-        softmax_tile_full<D, BF16>(s_addr, o_addr, p_addr, c2, first, m_ref, l_sum, l_lse, &sm.p_part[t]);
+        softmax_tile_full<D, BF16, FP8>(s_addr, o_addr, p_addr, c2, first, m_ref, l_sum, l_lse, &sm.p_part[t]);
       } else {
         const int kl = (kt >= mask_from) ? klim - kt * 128 : 128;   // keys >= kl: invisible to this row
-        softmax_tile_masked<D, BF16>(s_addr, o_addr, p_addr, c2, kl, first, m_ref, l_sum, l_lse,
+        softmax_tile_masked<D, BF16, FP8>(s_addr, o_addr, p_addr, c2, kl, first, m_ref, l_sum, l_lse,
                                      &sm.p_part[t]);
       }
       tmem_wait_st();
@@ -760,7 +860,7 @@ __device__ __forceinline__ void fwd_softmax(const FwdParams& p, const FwdSmem<D>
       tc_fence_after();
     }
     const bool store = row < x.sq;
-    const float inv_l = l_sum > 0.f ? 1.f / l_sum : 0.f;
+    const float inv_l = l_sum > 0.f ? p.o_mul / l_sum : 0.f;   // o_mul: FP8 V descale, else 1
     using T = typename std::conditional<BF16, __nv_bfloat16, __half>::type;
     T* orow = reinterpret_cast<T*>(p.o) + (((size_t)x.mb * p.Sq + x.qbase + row) * p.Hq + x.h) * D;
 #pragma unroll 1
@@ -811,15 +911,16 @@ __device__ __forceinline__ void fwd_teardown(bool owner, uint32_t tmem_base, uin
   }
 }
 
-template <int D, bool BF16, bool DYN, bool SPARSE>
+template <int D, bool BF16, bool DYN, bool SPARSE, bool FP8 = false>
 __global__ void __launch_bounds__(384, 1)
 attn_fwd_sm100(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                const __grid_constant__ CUtensorMap tm_v, const FwdParams p) {
-  using Cfg = FwdCfg<D>;
+  using Cfg = FwdCfg<D, FP8>;
   static_assert(DYN || !SPARSE, "the block-sparse units go through the dynamic unit queue");
+  static_assert(!FP8 || (BF16 && !SPARSE && D == 128), "FP8: D = 128, bf16 output, dense or packed");
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
-  const FwdSmem<D> sm(smem);
+  const FwdSmem<D, FP8> sm(smem);
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
   const int ncta = gridDim.x;
@@ -854,13 +955,13 @@ attn_fwd_sm100(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
     // load / MMA warpgroup gives registers away; warp 2 checks packed sequence offsets,
     // warp 3 has no role
     regs_dec<Cfg::REGS_OTHER>();
-    if (warp == kWarpLoad) fwd_producer<D, BF16, DYN, SPARSE>(&tm_q, &tm_k, &tm_v, p, sm, lane, cta, ncta);
-    else if (warp == kWarpMma) fwd_mma<D, BF16, DYN, SPARSE>(p, sm, tmem_base, lane, cta, ncta);
+    if (warp == kWarpLoad) fwd_producer<D, BF16, DYN, SPARSE, FP8>(&tm_q, &tm_k, &tm_v, p, sm, lane, cta, ncta);
+    else if (warp == kWarpMma) fwd_mma<D, BF16, DYN, SPARSE, FP8>(p, sm, tmem_base, lane, cta, ncta);
     else if (warp == 2 && p.cu_q) fwd_check_lengths(p, lane, cta, ncta);
     fwd_teardown(warp == kWarpMma, tmem_base, Cfg::TMEM_COLS);
   } else {
     regs_inc<Cfg::REGS_SOFTMAX>();
-    fwd_softmax<D, BF16, DYN, SPARSE>(p, sm, tmem_base, warp - 4, lane, cta, ncta);
+    fwd_softmax<D, BF16, DYN, SPARSE, FP8>(p, sm, tmem_base, warp - 4, lane, cta, ncta);
     fwd_teardown(false, tmem_base, Cfg::TMEM_COLS);
   }
 }

@@ -56,17 +56,24 @@ EncodeTiledFn get_encode() {
   return fn;
 }
 
-// View a [B, S, H, D] 16-bit tensor as 4-D (D, H, S, B); box = 64 elements x 1 head x
-// `rows` rows x 1 batch, 128-byte swizzle.  Rows past S read as zero.
+// Map element type for 8-bit (e4m3) tensors, next to SA_FP16 / SA_BF16.
+constexpr int kMapU8 = 100;
+
+// View a [B, S, H, D] 16-bit (or 8-bit) tensor as 4-D (D, H, S, B); box = one 128-byte row
+// of elements (64, or 128 for 8-bit) x 1 head x `rows` rows x 1 batch, 128-byte swizzle.
+// Rows past S read as zero.
 int make_map(CUtensorMap* m, const void* ptr, int dtype, int D, int H, int S, int B, int rows) {
   EncodeTiledFn enc = get_encode();
   if (!enc) return fail(SA_ERR_CUDA, "cuTensorMapEncodeTiled is not available from the driver");
+  const cuuint64_t eb = dtype == kMapU8 ? 1 : 2;
   cuuint64_t dims[4] = {(cuuint64_t)D, (cuuint64_t)H, (cuuint64_t)S, (cuuint64_t)B};
-  cuuint64_t strides[3] = {(cuuint64_t)D * 2, (cuuint64_t)H * D * 2, (cuuint64_t)S * H * D * 2};
-  cuuint32_t box[4] = {64, 1, (cuuint32_t)rows, 1};
+  cuuint64_t strides[3] = {(cuuint64_t)D * eb, (cuuint64_t)H * D * eb, (cuuint64_t)S * H * D * eb};
+  cuuint32_t box[4] = {(cuuint32_t)(128 / eb), 1, (cuuint32_t)rows, 1};
   cuuint32_t estr[4] = {1, 1, 1, 1};
-  CUresult r = enc(m, dtype == SA_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16,
-                   4, const_cast<void*>(ptr), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+  const CUtensorMapDataType ty = dtype == kMapU8 ? CU_TENSOR_MAP_DATA_TYPE_UINT8
+                                 : dtype == SA_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16
+                                                    : CU_TENSOR_MAP_DATA_TYPE_FLOAT16;
+  CUresult r = enc(m, ty, 4, const_cast<void*>(ptr), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
                    CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   if (r != CUDA_SUCCESS) return fail(SA_ERR_CUDA, "cuTensorMapEncodeTiled failed (CUresult %d)", (int)r);
@@ -213,24 +220,28 @@ int sparse_stride(int Sk) { return 8 + (((Sk + 127) / 128 + 7) / 8) * 8; }
 // Dense: q/o [B, Sq, Hq, D], k/v [B, Sk, Hkv, D].  Packed (vl.cu_q set): B sequences,
 // q/o [Sq, Hq, D] and k/v [Sk, Hkv, D] with Sq, Sk the totals, LSE [Hq, Sq].
 // Block-sparse (sparse.sp set, dense layout): the unit records built by sparse_unit_lists.
-template <int D, bool BF16>
+// FP8: q, k, v are e4m3, o bf16; `scale` already holds the Q and K descales, o_mul the V
+// descale.
+template <int D, bool BF16, bool FP8 = false>
 int launch_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Sq,
                int Sk, int Hq, int Hkv, int causal, float scale, cudaStream_t st,
-               const FwdVarlen& vl = FwdVarlen(), const FwdSparse& sparse = FwdSparse()) {
-  using Cfg = sa::FwdCfg<D>;
+               const FwdVarlen& vl = FwdVarlen(), const FwdSparse& sparse = FwdSparse(), float o_mul = 1.f) {
+  using Cfg = sa::FwdCfg<D, FP8>;
   const bool packed = vl.cu_q != nullptr;
   const int map_b = packed ? 1 : B;
+  const int map_ty = FP8 ? kMapU8 : (BF16 ? SA_BF16 : SA_FP16);
   CUtensorMap mq, mk, mv;
   int rc;
-  if ((rc = make_map(&mq, q, BF16, D, Hq, Sq, map_b, 128)) != SA_OK) return rc;
-  if ((rc = make_map(&mk, k, BF16, D, Hkv, Sk, map_b, 128)) != SA_OK) return rc;
-  if ((rc = make_map(&mv, v, BF16, D, Hkv, Sk, map_b, 128)) != SA_OK) return rc;
+  if ((rc = make_map(&mq, q, map_ty, D, Hq, Sq, map_b, 128)) != SA_OK) return rc;
+  if ((rc = make_map(&mk, k, map_ty, D, Hkv, Sk, map_b, 128)) != SA_OK) return rc;
+  if ((rc = make_map(&mv, v, map_ty, D, Hkv, Sk, map_b, 128)) != SA_OK) return rc;
   sa::FwdParams p;
   p.o = o; p.lse = lse;
   p.B = B; p.Sq = Sq; p.Sk = Sk; p.Hq = Hq; p.Hkv = Hkv; p.causal = causal;
   p.cu_q = vl.cu_q; p.cu_k = vl.cu_k;
   p.max_sq = packed ? vl.max_sq : Sq;
   p.sp = sparse.sp; p.sp_stride = sparse.stride;
+  p.o_mul = o_mul;
   const int seq_k = packed ? (vl.max_sk > 0 ? vl.max_sk : 1) : Sk;   // one sequence's keys, for L2 grouping
   p.n_qblk = (p.max_sq + 255) / 256;
   long long units = (long long)B * Hq * p.n_qblk;
@@ -247,7 +258,7 @@ int launch_fwd(const void* q, const void* k, const void* v, void* o, float* lse,
       l2 = 64 << 20;
     const int G = Hq / Hkv, n_bk = B * Hkv;
     const int ncta = p.n_units < num_sms() ? p.n_units : num_sms();
-    const double kv_bytes = 2.0 * seq_k * D * 2;       // K and V of one (b, KV head)
+    const double kv_bytes = 2.0 * seq_k * D * (FP8 ? 1 : 2);   // K and V of one (b, KV head)
     long long gmax = (long long)((l2 / 2) / kv_bytes);
     if (gmax < 1) gmax = 1;
     if (gmax > n_bk) gmax = n_bk;
@@ -275,9 +286,15 @@ int launch_fwd(const void* q, const void* k, const void* v, void* o, float* lse,
   const int grid = p.n_units < num_sms() ? p.n_units : num_sms();
   // packed lengths and block-sparse lists live on the device, so the static order's
   // balance is unknown: dynamic
-  auto kern = sparse.sp ? sa::attn_fwd_sm100<D, BF16, true, true>
-            : (packed || fwd_use_dynamic(p, D, grid)) ? sa::attn_fwd_sm100<D, BF16, true, false>
-                                                      : sa::attn_fwd_sm100<D, BF16, false, false>;
+  decltype(&sa::attn_fwd_sm100<D, BF16, false, false, FP8>) kern;
+  if constexpr (FP8) {
+    kern = (packed || fwd_use_dynamic(p, D, grid)) ? sa::attn_fwd_sm100<D, BF16, true, false, true>
+                                                   : sa::attn_fwd_sm100<D, BF16, false, false, true>;
+  } else {
+    kern = sparse.sp ? sa::attn_fwd_sm100<D, BF16, true, true>
+         : (packed || fwd_use_dynamic(p, D, grid)) ? sa::attn_fwd_sm100<D, BF16, true, false>
+                                                   : sa::attn_fwd_sm100<D, BF16, false, false>;
+  }
   const int smem = Cfg::SMEM_TOTAL + (sparse.sp ? Cfg::SMEM_SPARSE : 0);
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(attn_fwd_sm100)");
@@ -550,6 +567,24 @@ int sa_attn_fwd_block_sparse(const void* q, const void* k, const void* v, void* 
               : launch_fwd<64, false>(q, k, v, o, lse, B, Sq, Sk, Hq, Hkv, causal, scale, st, none, sp);
   return bf ? launch_fwd<128, true>(q, k, v, o, lse, B, Sq, Sk, Hq, Hkv, causal, scale, st, none, sp)
             : launch_fwd<128, false>(q, k, v, o, lse, B, Sq, Sk, Hq, Hkv, causal, scale, st, none, sp);
+}
+
+int sa_attn_fwd_fp8(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Sq, int Sk,
+                    int Hq, int Hkv, int D, int causal, float scale, float q_descale, float k_descale,
+                    float v_descale, sa_stream_t stream) {
+  int rc = check_dims(B, Sq, Sk, Hq, Hkv, D, SA_BF16, scale);
+  if (rc != SA_OK) return rc;
+  if (D != 128) return fail(SA_ERR_UNSUPPORTED, "the FP8 forward supports D = 128 (got %d)", D);
+  if (!(std::isfinite(q_descale) && q_descale > 0.f && std::isfinite(k_descale) && k_descale > 0.f &&
+        std::isfinite(v_descale) && v_descale > 0.f))
+    return fail(SA_ERR_INVALID, "descale factors must be finite and positive");
+  if (causal != 0 && causal != 1) return fail(SA_ERR_INVALID, "causal must be 0 or 1");
+  if (B == 0 || Sq == 0 || Hq == 0) return SA_OK;
+  if ((rc = check_ptrs(q, Sk ? k : q, Sk ? v : q, o, lse)) != SA_OK) return rc;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  if (Sk == 0) return launch_fill(o, (size_t)B * Sq * Hq * D, lse, (size_t)B * Hq * Sq, st);
+  return launch_fwd<128, true, true>(q, k, v, o, lse, B, Sq, Sk, Hq, Hkv, causal, scale * q_descale * k_descale,
+                                     st, FwdVarlen(), FwdSparse(), v_descale);
 }
 
 size_t sa_attn_bwd_workspace_size(int B, int Sq, int Hq) {

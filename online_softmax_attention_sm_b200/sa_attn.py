@@ -27,6 +27,7 @@ SIGNATURES = {
     "sa_attn_fwd_varlen": (_I, [_P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _I, _I, _F, _I, _P]),
     "sa_attn_fwd_block_sparse_workspace_size": (_Z, [_I, _I, _I, _I]),
     "sa_attn_bwd_workspace_size": (_Z, [_I, _I, _I]),
+    "sa_attn_fwd_fp8": (_I, [_P] * 5 + [_I] * 7 + [_F, _F, _F, _F, _P]),
     "sa_attn_bwd": (_I, [_P] * 9 + [_I] * 7 + [_F, _I, _P, _Z, _P]),
     "sa_attn_fwd_block_sparse": (_I, [_P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _F, _I, _P, _Z, _P]),
     "sa_attn_decode_workspace_size": (_Z, [_I, _I, _I, _I, _I, _I]),
@@ -190,6 +191,31 @@ def sa_attn_fwd_block_sparse(q, k, v, block_mask, causal=False, scale=None, work
                                           B, Sq, Sk, Hq, Hkv, D, int(bool(causal)), float(scale), _DT[q.dtype],
                                           _ptr(workspace), workspace.numel() * workspace.element_size(),
                                           _stream(stream)))
+    return out, lse
+
+
+def sa_attn_fwd_fp8(q8, k8, v8, q_descale, k_descale, v_descale, causal=False, scale=None, out=None, lse=None,
+                    return_lse=True, stream=None):
+    """FP8 attention forward.  q8 [B,Sq,Hq,D], k8/v8 [B,Sk,Hkv,D]: uint8 tensors of e4m3 codes
+    (CUDA, contiguous), per-tensor float descales.  Returns (o [B,Sq,Hq,D] bf16, lse [B,Hq,Sq])."""
+    B, Sq, Hq, D = q8.shape
+    Sk, Hkv = k8.shape[1], k8.shape[2]
+    if k8.shape != (B, Sk, Hkv, D) or v8.shape != k8.shape:
+        raise ValueError(f"shape mismatch q{tuple(q8.shape)} k{tuple(k8.shape)} v{tuple(v8.shape)}")
+    for n, t in (("q8", q8), ("k8", k8), ("v8", v8)):
+        _check_tensor(n, t, torch.uint8, q8.device)
+    if scale is None:
+        scale = 1.0 / math.sqrt(D)
+    if out is None:
+        out = torch.empty((B, Sq, Hq, D), dtype=torch.bfloat16, device=q8.device)
+    _check_tensor("out", out, torch.bfloat16, q8.device)
+    if return_lse and lse is None:
+        lse = torch.empty((B, Hq, Sq), dtype=torch.float32, device=q8.device)
+    if lse is not None:
+        _check_tensor("lse", lse, torch.float32, q8.device)
+    _check(lib().sa_attn_fwd_fp8(_ptr(q8), _ptr(k8), _ptr(v8), _ptr(out), _ptr(lse), B, Sq, Sk, Hq, Hkv, D,
+                                 int(bool(causal)), float(scale), float(q_descale), float(k_descale),
+                                 float(v_descale), _stream(stream)))
     return out, lse
 
 
