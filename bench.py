@@ -214,7 +214,7 @@ def main():
     import numpy as np
     import torch
     import torch.distributed as dist
-    from online_softmax_attention_sm_b200 import (sa_attn_decode, sa_attn_decode_paged,
+    from online_softmax_attention_sm_b200 import (sa_attn_decode, sa_attn_decode_paged, sa_attn_decode_single,
                                                    sa_attn_decode_paged_workspace_size,
                                                    sa_attn_decode_workspace_size, sa_attn_fwd,
                                                    sa_attn_fwd_block_sparse, sa_attn_fwd_block_sparse_workspace_size,
@@ -336,6 +336,35 @@ def main():
         sa_check_status(stream)
         paged_ms = [a.elapsed_time(b) for a, b in pev]
         del kc, vc
+
+    # the single-kernel decode (each tile's last split merges; no combine launch) on the same
+    # workload, and both decodes at batch 1 (the pages' small-batch case); same protocol
+    def cold_loop(call):
+        evs = []
+        for i in range(args.warmup + args.steps):
+            scrub.sum()
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            call()
+            e1.record(stream)
+            if i >= args.warmup:
+                evs.append((e0, e1))
+        torch.cuda.synchronize(dev)
+        sa_check_status(stream)
+        return [a.elapsed_time(b) for a, b in evs]
+
+    single_ms = b1_two_ms = b1_single_ms = [float("nan")]
+    if run_dec:
+        single_ms = cold_loop(lambda: sa_attn_decode_single(dq, dk, dv, scale=wd.scale, workspace=ws, out=do,
+                                                             lse=dlse, stream=stream))
+        dq1, dk1, dv1, do1, dl1 = dq[:1], dk[:1], dv[:1], do[:1], dlse[:1]
+        ws1 = torch.empty(max(16, sa_attn_decode_workspace_size(1, wd.Sk, wd.Hq, wd.Hkv, wd.D)), dtype=torch.uint8,
+                          device=dev)
+        b1_two_ms = cold_loop(lambda: sa_attn_decode(dq1, dk1, dv1, scale=wd.scale, workspace=ws1, out=do1, lse=dl1,
+                                                     stream=stream))
+        b1_single_ms = cold_loop(lambda: sa_attn_decode_single(dq1, dk1, dv1, scale=wd.scale, workspace=ws1,
+                                                               out=do1, lse=dl1, stream=stream))
+        del ws1
     del scrub
 
     # packed variable-length prefill: the long prefill's heads over 16 sequences of 32768
@@ -463,6 +492,9 @@ def main():
     dec_avg = max_over_ranks(sum(dec_ms) / len(dec_ms), dev)
     cold_avg = max_over_ranks(sum(cold_ms) / len(cold_ms), dev)
     paged_avg = max_over_ranks(sum(paged_ms) / len(paged_ms), dev)
+    single_avg = max_over_ranks(sum(single_ms) / len(single_ms), dev)
+    b1_two_avg = max_over_ranks(sum(b1_two_ms) / len(b1_two_ms), dev)
+    b1_single_avg = max_over_ranks(sum(b1_single_ms) / len(b1_single_ms), dev)
     var_avg = max_over_ranks(sum(var_ms) / len(var_ms), dev)
     sp_avg = max_over_ranks(sum(sp_ms) / len(sp_ms), dev)
     bwd_avg = max_over_ranks(sum(bwd_ms) / len(bwd_ms), dev)
@@ -508,7 +540,13 @@ def main():
                                  "frac": wd.kv_bytes / (paged_avg * 1e-3) / 1e9 / peaks["hbm_gbs"],
                                  "us": paged_avg * 1e3, "page_size": 64,
                                  "layout": "the same K/V in shuffled 64-token pages, full-length sequences",
-                                 "l2": "cold (4xL2 read scrub)"}},
+                                 "l2": "cold (4xL2 read scrub)"},
+                       "single_kernel": {"us": single_avg * 1e3,
+                                         "value": wd.kv_bytes / (single_avg * 1e-3) / 1e9, "unit": "GB/s",
+                                         "frac": wd.kv_bytes / (single_avg * 1e-3) / 1e9 / peaks["hbm_gbs"],
+                                         "kernel": "attn_decode_split (last split of each tile merges)"},
+                       "batch1": {"two_kernel_us": b1_two_avg * 1e3, "single_kernel_us": b1_single_avg * 1e3,
+                                  "workload": "the decode workload's first sequence alone (B1, 32768 keys)"}},
             "prefill_varlen": {"workload": VARLEN, "value": wv.flops / (var_avg * 1e-3) / 1e12,
                                "unit": "TFLOP/s", "bound": "tensor", "peak": peak,
                                "frac": wv.flops / (var_avg * 1e-3) / 1e12 / peak, "ms": var_avg,

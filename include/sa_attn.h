@@ -119,6 +119,19 @@ int sa_attn_fwd_block_sparse(const void* q, const void* k, const void* v, void* 
                              void* workspace, size_t workspace_bytes, sa_stream_t stream);
 
 /*
+ * Single-kernel split-KV decode (the StreamAttention page, "Engine Direction": the
+ * two-kernel prototype loses to launch and merge overhead at small batch).  Same arguments,
+ * workspace and result as sa_attn_decode; instead of a second (combine) launch, the last
+ * split CTA of each (batch, KV head, head group) tile -- found by an arrival counter --
+ * merges that tile's query heads.  At most 4096 such tiles (else SA_ERR_UNSUPPORTED); up to
+ * 16 calls may be in flight at once.  Measured against sa_attn_decode in the bench.
+ */
+int sa_attn_decode_single(const void* q, const void* k, const void* v, void* o, float* lse,
+                          int B, int Sk, int Hq, int Hkv, int D, float scale, int dtype,
+                          int num_splits, void* workspace, size_t workspace_bytes,
+                          sa_stream_t stream);
+
+/*
  * FP8 forward (the Stem page's fp8 prefill path; the StreamAttention page's FP8 roadmap
  * item): q, k, v are e4m3 codes (one byte per element, layouts as sa_attn_fwd) with
  * per-tensor descale factors, o is bf16 [B, Sq, Hq, D], lse fp32 [B, Hq, Sq] or NULL.

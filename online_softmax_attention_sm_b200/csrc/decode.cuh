@@ -63,6 +63,10 @@ struct DecParams {
   const int* block_table;   // [B, max_blocks]
   const int* seqlens;       // [B]
   int max_blocks, page_size;
+  // single-kernel instance (attn_decode_split<.., FUSED = true>): one arrival counter per
+  // (batch, KV head, head group) tile, zero at launch; the tile's last split merges and
+  // zeroes it again
+  unsigned int* sem;
 };
 
 __device__ __forceinline__ void ldsm_x4(uint32_t addr, uint32_t& r0, uint32_t& r1, uint32_t& r2, uint32_t& r3) {
@@ -179,7 +183,14 @@ struct DecMerge {
   static constexpr int MAX_SPLITS = (D == 64) ? 192 : 96;
 };
 
-template <int D, bool BF16, bool PAGED>
+template <int D, bool BF16>
+__device__ __forceinline__ void decode_merge_row(const DecParams& p, size_t row, float* s_w, float (*s_red)[4],
+                                                 float4* s_acc);
+
+// FUSED (the single-kernel instance, for small batches where a second launch costs more
+// than it saves): after writing its partial state, each CTA takes a ticket on its tile's
+// arrival counter, and the tile's last split merges the tile's query heads itself.
+template <int D, bool BF16, bool PAGED, bool FUSED = false>
 __global__ void __launch_bounds__(128, 3)
 attn_decode_split(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
                   const DecParams p) {
@@ -359,43 +370,49 @@ attn_decode_split(const __grid_constant__ CUtensorMap tm_k, const __grid_constan
     return;                                                   // outputs undefined; status word set
   }
   write_partial<D>(p, smem, b, h0, nrows, split, warp, lane, o, m0, m1, l0, l1, e0, e1);
+  if (FUSED) {
+    // every thread's partial-state stores are visible device-wide before the ticket
+    __threadfence();
+    __syncthreads();
+    volatile int* s_last = reinterpret_cast<volatile int*>(smem + region + 128);
+    const unsigned tile = ((unsigned)b * gridDim.y + blockIdx.y);
+    if (threadIdx.x == 0) *s_last = atomicAdd(p.sem + tile, 1u) == (unsigned)p.nsplit - 1u;
+    __syncthreads();
+    if (*s_last) {
+      __threadfence();
+      float* s_w = reinterpret_cast<float*>(smem);            // stages are drained
+      float (*s_red)[4] = reinterpret_cast<float (*)[4]>(s_w + DecMerge<D>::MAX_SPLITS);
+      float4* s_acc = reinterpret_cast<float4*>(s_w + DecMerge<D>::MAX_SPLITS + 16);
+      for (int r = 0; r < nrows; ++r) decode_merge_row<D, BF16>(p, (size_t)b * p.Hq + h0 + r, s_w, s_red, s_acc);
+      if (threadIdx.x == 0) p.sem[tile] = 0u;                  // ready for the next launch
+    }
+  }
 }
 
-// Merge of every split's partial state for one (batch, query head) row per CTA:
-//   M = max_s m_s,  w_s = 2^(m_s - M),  O = sum_s w_s O_s / sum_s w_s l_s,
-//   LSE = (M + log2 sum_s w_s e_s) * ln 2.
-// Launched with programmatic dependent launch right behind the split kernel: its CTAs are
-// resident before the split grid ends and proceed the moment its results are visible.
-// Every load (the split maxima/sums and the partial output rows) is issued up front, so
-// the merge costs one round trip to L2.  Thread t owns float4 column c = t % (D/4) and the
-// splits s = g, g + NG, ... with g = t / (D/4), NG = 128 / (D/4); the NG partial sums per
-// column are added through shared memory.
+// The merge of one (batch, query head) row by a block of 128 threads (scratch: s_w [MAX_SPLITS],
+// s_red [3][4], s_acc [128]).  Loads bypass L1 (.cg): in the single-kernel instance the
+// partial states were written by other CTAs of the same grid.
 template <int D, bool BF16>
-__global__ void __launch_bounds__(128)
-attn_decode_combine(const DecParams p) {
-  asm volatile("griddepcontrol.wait;" ::: "memory");
+__device__ __forceinline__ void decode_merge_row(const DecParams& p, size_t row, float* s_w, float (*s_red)[4],
+                                                 float4* s_acc) {
   constexpr int NC = D / 4, NG = 128 / NC;
   constexpr int MAXS = DecMerge<D>::MAX_SPLITS;
   constexpr int PER = (MAXS + NG - 1) / NG;                   // splits per thread, at most
   static_assert(MAXS <= 256, "two split maxima per thread");
-  __shared__ float s_w[MAXS];
-  __shared__ float s_red[3][4];
-  __shared__ float4 s_acc[128];
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const size_t row = blockIdx.x;                              // b * Hq + h
   const int ns = p.nsplit;
   const float4* ml = reinterpret_cast<const float4*>(p.ws_ml) + row * ns;
   const float4* os = reinterpret_cast<const float4*>(p.ws_o) + row * ns * NC;
   const int c = tid % NC, g = tid / NC;
   // all loads first
   const float4 ninf = make_float4(-INFINITY, 0.f, 0.f, 0.f);
-  const float4 mlA = tid < ns ? ml[tid] : ninf;
-  const float4 mlB = tid + 128 < ns ? ml[tid + 128] : ninf;
+  const float4 mlA = tid < ns ? __ldcg(ml + tid) : ninf;
+  const float4 mlB = tid + 128 < ns ? __ldcg(ml + tid + 128) : ninf;
   float4 v[PER];
 #pragma unroll
   for (int u = 0; u < PER; ++u) {
     const int s = g + u * NG;
-    v[u] = s < ns ? os[(size_t)s * NC + c] : make_float4(0.f, 0.f, 0.f, 0.f);
+    v[u] = s < ns ? __ldcg(os + (size_t)s * NC + c) : make_float4(0.f, 0.f, 0.f, 0.f);
   }
   // max over splits
   float M = fmaxf(mlA.x, mlB.x);
@@ -445,6 +462,26 @@ attn_decode_combine(const DecParams p) {
     reinterpret_cast<uint2*>(reinterpret_cast<uint16_t*>(p.o) + row * D)[tid] = packed;
   }
   if (p.lse && tid == 0) p.lse[row] = E > 0.f ? (M + __log2f(E)) * 0.69314718055994531f : -INFINITY;
+  __syncthreads();                                            // scratch free for the next row
+}
+
+// Merge of every split's partial state for one (batch, query head) row per CTA:
+//   M = max_s m_s,  w_s = 2^(m_s - M),  O = sum_s w_s O_s / sum_s w_s l_s,
+//   LSE = (M + log2 sum_s w_s e_s) * ln 2.
+// Launched with programmatic dependent launch right behind the split kernel: its CTAs are
+// resident before the split grid ends and proceed the moment its results are visible.
+// Every load (the split maxima/sums and the partial output rows) is issued up front, so
+// the merge costs one round trip to L2.  Thread t owns float4 column c = t % (D/4) and the
+// splits s = g, g + NG, ... with g = t / (D/4), NG = 128 / (D/4); the NG partial sums per
+// column are added through shared memory.
+template <int D, bool BF16>
+__global__ void __launch_bounds__(128)
+attn_decode_combine(const DecParams p) {
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+  __shared__ float s_w[DecMerge<D>::MAX_SPLITS];
+  __shared__ float s_red[3][4];
+  __shared__ float4 s_acc[128];
+  decode_merge_row<D, BF16>(p, blockIdx.x, s_w, s_red, s_acc);
 }
 
 }  // namespace sa

@@ -404,7 +404,33 @@ struct DecPaged {
   int max_blocks = 0, page_size = 0, num_pages = 0;
 };
 
-template <int D, bool BF16, bool PAGED>
+// Arrival counters of the single-kernel decode: kDecSemSlots sets of kDecSemTiles, zero with
+// the module; launches take sets in turn and every tile's last split zeroes its counter, so
+// up to kDecSemSlots single-kernel decodes may be in flight at once (on any streams).
+constexpr int kDecSemSlots = 16, kDecSemTiles = 4096;
+static __device__ unsigned int g_dec_sem[kDecSemSlots * kDecSemTiles];
+
+int dec_sem_slot(unsigned int** out) {
+  static std::mutex mu;
+  static unsigned int* addr[64] = {nullptr};
+  static unsigned int next[64] = {0};
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+  if (dev < 0 || dev >= 64) return fail(SA_ERR_UNSUPPORTED, "device ordinal %d out of range", dev);
+  std::lock_guard<std::mutex> lock(mu);
+  if (!addr[dev]) {
+    void* ptr = nullptr;
+    e = cudaGetSymbolAddress(&ptr, g_dec_sem);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaGetSymbolAddress(decode arrival counters)");
+    addr[dev] = static_cast<unsigned int*>(ptr);
+  }
+  *out = addr[dev] + (size_t)kDecSemTiles * (next[dev]++ % kDecSemSlots);
+  return SA_OK;
+}
+
+// FUSED: the single-kernel instance (the tile's last split merges; no combine launch).
+template <int D, bool BF16, bool PAGED, bool FUSED = false>
 int launch_decode(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Sk,
                   int Hq, int Hkv, float scale, const DecPlan& pl, void* ws, cudaStream_t st,
                   const DecPaged& pg = DecPaged()) {
@@ -425,15 +451,23 @@ int launch_decode(const void* q, const void* k, const void* v, void* o, float* l
   p.B = B; p.Sk = Sk; p.Hq = Hq; p.Hkv = Hkv; p.G = Hq / Hkv; p.ngrp = pl.ngrp;
   p.nsplit = pl.nsplit; p.chunk = pl.chunk;
   p.c2 = scale * kLog2e;
+  p.sem = nullptr;
   dim3 grid(pl.nsplit, Hkv * pl.ngrp, B);
   if ((long long)B * Hq > 0x7fffffffLL || grid.y > 65535 || grid.z > 65535)
     return fail(SA_ERR_UNSUPPORTED, "decode grid too large");
-  auto ks = sa::attn_decode_split<D, BF16, PAGED>;
+  if (FUSED) {
+    if ((long long)B * Hkv * pl.ngrp > kDecSemTiles)
+      return fail(SA_ERR_UNSUPPORTED, "single-kernel decode supports at most %d (batch, KV head, head group) "
+                  "tiles (got %lld)", kDecSemTiles, (long long)B * Hkv * pl.ngrp);
+    if ((rc = dec_sem_slot(&p.sem)) != SA_OK) return rc;
+  }
+  auto ks = sa::attn_decode_split<D, BF16, PAGED, FUSED>;
   cudaError_t e = cudaFuncSetAttribute(ks, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::SMEM_TOTAL);
   if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(attn_decode_split)");
   ks<<<grid, 128, Cfg::SMEM_TOTAL, st>>>(mk, mv, p);
   e = cudaGetLastError();
   if (e != cudaSuccess) return cuda_fail(e, "attn_decode_split launch");
+  if (FUSED) return SA_OK;
   // combine: programmatic dependent launch, resident and waiting when the split grid ends
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3((unsigned)(B * Hq));
@@ -680,6 +714,30 @@ int sa_attn_decode(const void* q, const void* k, const void* v, void* o, float* 
                          : launch_decode<64, false, false>(q, k, v, o, lse, B, Sk, Hq, Hkv, scale, pl, workspace, st);
   return bf ? launch_decode<128, true, false>(q, k, v, o, lse, B, Sk, Hq, Hkv, scale, pl, workspace, st)
             : launch_decode<128, false, false>(q, k, v, o, lse, B, Sk, Hq, Hkv, scale, pl, workspace, st);
+}
+
+int sa_attn_decode_single(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Sk,
+                          int Hq, int Hkv, int D, float scale, int dtype, int num_splits, void* workspace,
+                          size_t workspace_bytes, sa_stream_t stream) {
+  int rc = check_dims(B, 1, Sk, Hq, Hkv, D, dtype, scale);
+  if (rc != SA_OK) return rc;
+  if (num_splits < 0) return fail(SA_ERR_INVALID, "num_splits must be >= 0");
+  if (B == 0 || Hq == 0) return SA_OK;
+  if ((rc = check_ptrs(q, Sk ? k : q, Sk ? v : q, o, lse)) != SA_OK) return rc;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  if (Sk == 0) return launch_fill(o, (size_t)B * Hq * D, lse, (size_t)B * Hq, st);
+  DecPlan pl = plan_decode(B, Sk, Hq, Hkv, D, num_splits, num_sms());
+  const size_t need = dec_ws_bytes(B, Hq, pl.nsplit, D);
+  if (!workspace || workspace_bytes < need)
+    return fail(SA_ERR_WORKSPACE, "decode workspace of %zu bytes needed (got %zu)", need,
+                workspace ? workspace_bytes : (size_t)0);
+  if (!aligned16(workspace)) return fail(SA_ERR_INVALID, "workspace must be 16-byte aligned");
+  const bool bf = dtype == SA_BF16;
+  if (D == 64)
+    return bf ? launch_decode<64, true, false, true>(q, k, v, o, lse, B, Sk, Hq, Hkv, scale, pl, workspace, st)
+              : launch_decode<64, false, false, true>(q, k, v, o, lse, B, Sk, Hq, Hkv, scale, pl, workspace, st);
+  return bf ? launch_decode<128, true, false, true>(q, k, v, o, lse, B, Sk, Hq, Hkv, scale, pl, workspace, st)
+            : launch_decode<128, false, false, true>(q, k, v, o, lse, B, Sk, Hq, Hkv, scale, pl, workspace, st);
 }
 
 int sa_attn_decode_noalloc(const void* q, const void* k, const void* v, void* o, float* lse, int B,

@@ -28,6 +28,7 @@ SIGNATURES = {
     "sa_attn_fwd_block_sparse_workspace_size": (_Z, [_I, _I, _I, _I]),
     "sa_attn_bwd_workspace_size": (_Z, [_I, _I, _I]),
     "sa_attn_fwd_fp8": (_I, [_P] * 5 + [_I] * 7 + [_F, _F, _F, _F, _P]),
+    "sa_attn_decode_single": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _F, _I, _I, _P, _Z, _P]),
     "sa_attn_bwd": (_I, [_P] * 9 + [_I] * 7 + [_F, _I, _P, _Z, _P]),
     "sa_attn_fwd_block_sparse": (_I, [_P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _F, _I, _P, _Z, _P]),
     "sa_attn_decode_workspace_size": (_Z, [_I, _I, _I, _I, _I, _I]),
@@ -271,8 +272,10 @@ def sa_attn_decode_num_splits(B, Sk, Hq, Hkv, D):
 
 
 def sa_attn_decode(q, k, v, scale=None, num_splits=0, workspace=None, out=None, lse=None,
-                   return_lse=True, stream=None):
-    """Split-KV decode.  q [B,Hq,D], k/v [B,Sk,Hkv,D].  Returns (o [B,Hq,D], lse [B,Hq])."""
+                   return_lse=True, stream=None, single=False):
+    """Split-KV decode.  q [B,Hq,D], k/v [B,Sk,Hkv,D].  Returns (o [B,Hq,D], lse [B,Hq]).
+    single=True runs the single-kernel variant (sa_attn_decode_single: the last split of
+    each head tile merges, no combine launch)."""
     B, Hq, D = q.shape
     Sk, Hkv = k.shape[1], k.shape[2]
     if k.shape != (B, Sk, Hkv, D) or v.shape != k.shape:
@@ -290,10 +293,15 @@ def sa_attn_decode(q, k, v, scale=None, num_splits=0, workspace=None, out=None, 
     need = sa_attn_decode_workspace_size(B, Sk, Hq, Hkv, D, num_splits)
     if workspace is None:
         workspace = torch.empty(max(need, 16), dtype=torch.uint8, device=q.device)
-    _check(lib().sa_attn_decode(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse), B, Sk, Hq, Hkv, D,
-                                float(scale), _DT[q.dtype], int(num_splits), _ptr(workspace),
-                                workspace.numel() * workspace.element_size(), _stream(stream)))
+    fn = lib().sa_attn_decode_single if single else lib().sa_attn_decode
+    _check(fn(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse), B, Sk, Hq, Hkv, D, float(scale), _DT[q.dtype],
+              int(num_splits), _ptr(workspace), workspace.numel() * workspace.element_size(), _stream(stream)))
     return out, lse
+
+
+def sa_attn_decode_single(q, k, v, **kw):
+    """The single-kernel split-KV decode (same contract as :func:`sa_attn_decode`)."""
+    return sa_attn_decode(q, k, v, single=True, **kw)
 
 
 def sa_attn_decode_paged_workspace_size(B, Hq, Hkv, D, page_size, max_blocks, num_splits=0):

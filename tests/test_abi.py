@@ -272,6 +272,22 @@ def test_bwd_workspace_size(L):
     assert L.sa_attn_bwd_workspace_size(0, 300, 4) == 0
 
 
+@pytest.mark.parametrize("kw,code", [
+    (dict(q=NULL), sa.SA_ERR_INVALID),
+    (dict(Hq=3, Hkv=2), sa.SA_ERR_INVALID),
+    (dict(D=96), sa.SA_ERR_UNSUPPORTED),
+    (dict(ns=-1), sa.SA_ERR_INVALID),
+    (dict(ws=NULL), sa.SA_ERR_WORKSPACE),
+])
+def test_decode_single_rejects_invalid_arguments(L, kw, code):
+    args = dict(q=FAKE, k=FAKE, v=FAKE, o=FAKE, lse=NULL, B=1, Sk=64, Hq=2, Hkv=1, D=64, scale=0.125, dtype=0, ns=0,
+                ws=FAKE, wsb=1 << 20)
+    args.update(kw)
+    a = args
+    assert L.sa_attn_decode_single(a["q"], a["k"], a["v"], a["o"], a["lse"], a["B"], a["Sk"], a["Hq"], a["Hkv"],
+                                   a["D"], a["scale"], a["dtype"], a["ns"], a["ws"], a["wsb"], None) == code
+
+
 def test_version(L):
     assert re.fullmatch(r"\d+\.\d+\.\d+", sa.sa_version())
 
