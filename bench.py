@@ -219,6 +219,7 @@ def main():
                                                    sa_attn_decode_workspace_size, sa_attn_fwd,
                                                    sa_attn_fwd_block_sparse, sa_attn_fwd_block_sparse_workspace_size,
                                                    sa_attn_bwd, sa_attn_bwd_workspace_size, sa_attn_fwd_fp8,
+                                                   sa_attn_fwd_block_sparse_fp8,
                                                    sa_attn_fwd_varlen, sa_check_status)
     from online_softmax_attention_sm_b200.dist import aggregate_throughput, max_over_ranks, rank_seed
     from online_softmax_attention_sm_b200.inputs import (make_dout, make_qkv, make_qkv_fp8, make_workload_inputs,
@@ -438,7 +439,8 @@ def main():
         del dout, gq, gk, gv, bws
 
     # FP8 forward: the prefill workload's draws quantised to e4m3 per tensor (same seed)
-    fp8_ms = [float("nan")]
+    fp8_ms = sp8_ms = [float("nan")]
+    sp8_flops = float("nan")
     if run_fp8:
         q8, k8, v8, qd8, kd8, vd8 = make_qkv_fp8(wp.B, wp.Sq, wp.Sk, wp.Hq, wp.Hkv, wp.D, seed=rank_seed(wp.seed, rank),
                                                  input_scale=wp.input_scale, k_sink_rows=wp.k_sink_rows,
@@ -457,7 +459,25 @@ def main():
         torch.cuda.synchronize(dev)
         sa_check_status(stream)
         fp8_ms = [a.elapsed_time(b) for a, b in fev]
-        del q8, k8, v8, o8
+        # and block-sparse over the same e4m3 tensors (the Stem-shaped mask of the bf16 leg)
+        bmask8 = stem_block_mask(wp.B, wp.Hq, wp.Sq, wp.Sk, wp.causal, seed=wp.seed + 4)
+        sp8_flops = block_sparse_flops(bmask8.numpy(), wp.Sq, wp.Sk, wp.D, wp.causal)
+        bmask8 = bmask8.to(dev)
+        sws8 = torch.empty(max(16, sa_attn_fwd_block_sparse_workspace_size(wp.B, wp.Sq, wp.Sk, wp.Hq)),
+                           dtype=torch.uint8, device=dev)
+        fsev = []
+        for i in range(args.warmup + args.steps):
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            sa_attn_fwd_block_sparse_fp8(q8, k8, v8, bmask8, qd8, kd8, vd8, causal=wp.causal, scale=wp.scale,
+                                         workspace=sws8, out=o8, lse=lse, stream=stream)
+            e1.record(stream)
+            if i >= args.warmup:
+                fsev.append((e0, e1))
+        torch.cuda.synchronize(dev)
+        sa_check_status(stream)
+        sp8_ms = [a.elapsed_time(b) for a, b in fsev]
+        del q8, k8, v8, o8, bmask8, sws8
 
     # e2e through the public API with host buffers: H2D of the step's inputs, D2H of outputs
     e2e_ms = None
@@ -499,6 +519,7 @@ def main():
     sp_avg = max_over_ranks(sum(sp_ms) / len(sp_ms), dev)
     bwd_avg = max_over_ranks(sum(bwd_ms) / len(bwd_ms), dev)
     fp8_avg = max_over_ranks(sum(fp8_ms) / len(fp8_ms), dev)
+    sp8_avg = max_over_ranks(sum(sp8_ms) / len(sp8_ms), dev)
     e2e_ms = max_over_ranks(e2e_ms, dev) if e2e_ms is not None else None
 
     if rank == 0:
@@ -569,7 +590,10 @@ def main():
                             "value": wp.flops / (fp8_avg * 1e-3) / 1e12, "unit": "TFLOP/s", "bound": "tensor",
                             "peak": 2 * peak, "peak_source": "measured bf16 burst x 2 (nominal fp8 : bf16)",
                             "frac": wp.flops / (fp8_avg * 1e-3) / 1e12 / (2 * peak), "ms": fp8_avg,
-                            "kernel": "attn_fwd_sm100 (FP8 instance: kind::f8f6f4 QK and PV, e4m3 P)"},
+                            "kernel": "attn_fwd_sm100 (FP8 instance: kind::f8f6f4 QK and PV, e4m3 P)",
+                            "block_sparse": {"value": sp8_flops / (sp8_avg * 1e-3) / 1e12, "unit": "TFLOP/s",
+                                             "frac": sp8_flops / (sp8_avg * 1e-3) / 1e12 / (2 * peak),
+                                             "ms": sp8_avg, "mask": "the bf16 block-sparse leg's Stem-shaped mask"}},
             "prefill_ms": pre_avg,
             "gpu_launches": (int(run_pre) + 2 * int(run_dec)) * args.steps,
             "clocks": clk.summary(),

@@ -119,6 +119,18 @@ int sa_attn_fwd_block_sparse(const void* q, const void* k, const void* v, void* 
                              void* workspace, size_t workspace_bytes, sa_stream_t stream);
 
 /*
+ * FP8 block-sparse forward (the Stem page's serving backend: fp8 block-sparse prefill):
+ * sa_attn_fwd_block_sparse on e4m3 inputs with per-tensor descales, bf16 output, D = 128;
+ * inputs, outputs and descales as sa_attn_fwd_fp8, mask and workspace as
+ * sa_attn_fwd_block_sparse.
+ */
+int sa_attn_fwd_block_sparse_fp8(const void* q, const void* k, const void* v, void* o, float* lse,
+                                 const unsigned char* block_mask, int B, int Sq, int Sk, int Hq,
+                                 int Hkv, int D, int causal, float scale, float q_descale,
+                                 float k_descale, float v_descale, void* workspace,
+                                 size_t workspace_bytes, sa_stream_t stream);
+
+/*
  * Single-kernel split-KV decode (the StreamAttention page, "Engine Direction": the
  * two-kernel prototype loses to launch and merge overhead at small batch).  Same arguments,
  * workspace and result as sa_attn_decode; instead of a second (combine) launch, the last

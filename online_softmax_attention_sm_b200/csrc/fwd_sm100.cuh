@@ -917,7 +917,7 @@ attn_fwd_sm100(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
                const __grid_constant__ CUtensorMap tm_v, const FwdParams p) {
   using Cfg = FwdCfg<D, FP8>;
   static_assert(DYN || !SPARSE, "the block-sparse units go through the dynamic unit queue");
-  static_assert(!FP8 || (BF16 && !SPARSE && D == 128), "FP8: D = 128, bf16 output, dense or packed");
+  static_assert(!FP8 || (BF16 && D == 128), "FP8: D = 128, bf16 output");
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
   const FwdSmem<D, FP8> sm(smem);

@@ -288,7 +288,8 @@ int launch_fwd(const void* q, const void* k, const void* v, void* o, float* lse,
   // balance is unknown: dynamic
   decltype(&sa::attn_fwd_sm100<D, BF16, false, false, FP8>) kern;
   if constexpr (FP8) {
-    kern = (packed || fwd_use_dynamic(p, D, grid)) ? sa::attn_fwd_sm100<D, BF16, true, false, true>
+    kern = sparse.sp ? sa::attn_fwd_sm100<D, BF16, true, true, true>
+         : (packed || fwd_use_dynamic(p, D, grid)) ? sa::attn_fwd_sm100<D, BF16, true, false, true>
                                                    : sa::attn_fwd_sm100<D, BF16, false, false, true>;
   } else {
     kern = sparse.sp ? sa::attn_fwd_sm100<D, BF16, true, true>
@@ -511,6 +512,13 @@ int noalloc_scratch(void** out) {
   return SA_OK;
 }
 
+// Shared by the 16-bit and the FP8 block-sparse entry points (fp8: q, k, v e4m3, o bf16,
+// scale with the Q and K descales folded in, o_mul the V descale).
+int block_sparse_fwd(const void* q, const void* k, const void* v, void* o, float* lse,
+                     const unsigned char* block_mask, int B, int Sq, int Sk, int Hq, int Hkv, int D, int causal,
+                     float scale, int dtype, bool fp8, float o_mul, void* workspace, size_t workspace_bytes,
+                     cudaStream_t st);
+
 }  // namespace
 
 extern "C" {
@@ -570,10 +578,36 @@ int sa_attn_fwd_block_sparse(const void* q, const void* k, const void* v, void* 
                              size_t workspace_bytes, sa_stream_t stream) {
   int rc = check_dims(B, Sq, Sk, Hq, Hkv, D, dtype, scale);
   if (rc != SA_OK) return rc;
+  return block_sparse_fwd(q, k, v, o, lse, block_mask, B, Sq, Sk, Hq, Hkv, D, causal, scale, dtype, false, 1.f,
+                          workspace, workspace_bytes, reinterpret_cast<cudaStream_t>(stream));
+}
+
+int sa_attn_fwd_block_sparse_fp8(const void* q, const void* k, const void* v, void* o, float* lse,
+                                 const unsigned char* block_mask, int B, int Sq, int Sk, int Hq, int Hkv,
+                                 int D, int causal, float scale, float q_descale, float k_descale,
+                                 float v_descale, void* workspace, size_t workspace_bytes, sa_stream_t stream) {
+  int rc = check_dims(B, Sq, Sk, Hq, Hkv, D, SA_BF16, scale);
+  if (rc != SA_OK) return rc;
+  if (D != 128) return fail(SA_ERR_UNSUPPORTED, "the FP8 forward supports D = 128 (got %d)", D);
+  if (!(std::isfinite(q_descale) && q_descale > 0.f && std::isfinite(k_descale) && k_descale > 0.f &&
+        std::isfinite(v_descale) && v_descale > 0.f))
+    return fail(SA_ERR_INVALID, "descale factors must be finite and positive");
+  return block_sparse_fwd(q, k, v, o, lse, block_mask, B, Sq, Sk, Hq, Hkv, D, causal,
+                          scale * q_descale * k_descale, SA_BF16, true, v_descale, workspace, workspace_bytes,
+                          reinterpret_cast<cudaStream_t>(stream));
+}
+
+}  // extern "C"
+
+namespace {
+int block_sparse_fwd(const void* q, const void* k, const void* v, void* o, float* lse,
+                     const unsigned char* block_mask, int B, int Sq, int Sk, int Hq, int Hkv, int D, int causal,
+                     float scale, int dtype, bool fp8, float o_mul, void* workspace, size_t workspace_bytes,
+                     cudaStream_t st) {
+  int rc = SA_OK;
   if (causal != 0 && causal != 1) return fail(SA_ERR_INVALID, "causal must be 0 or 1");
   if (B == 0 || Sq == 0 || Hq == 0) return SA_OK;
   if ((rc = check_ptrs(q, Sk ? k : q, Sk ? v : q, o, lse)) != SA_OK) return rc;
-  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   if (Sk == 0) return launch_fill(o, (size_t)B * Sq * Hq * D, lse, (size_t)B * Hq * Sq, st);
   if (!block_mask) return fail(SA_ERR_INVALID, "block_mask must be non-null");
   if ((Sk + 127) / 128 > sa::kSparseMaxKTiles)
@@ -596,12 +630,16 @@ int sa_attn_fwd_block_sparse(const void* q, const void* k, const void* v, void* 
   if (e != cudaSuccess) return cuda_fail(e, "sparse_unit_lists launch");
   const bool bf = dtype == SA_BF16;
   const FwdVarlen none;
+  if (fp8) return launch_fwd<128, true, true>(q, k, v, o, lse, B, Sq, Sk, Hq, Hkv, causal, scale, st, none, sp, o_mul);
   if (D == 64)
     return bf ? launch_fwd<64, true>(q, k, v, o, lse, B, Sq, Sk, Hq, Hkv, causal, scale, st, none, sp)
               : launch_fwd<64, false>(q, k, v, o, lse, B, Sq, Sk, Hq, Hkv, causal, scale, st, none, sp);
   return bf ? launch_fwd<128, true>(q, k, v, o, lse, B, Sq, Sk, Hq, Hkv, causal, scale, st, none, sp)
             : launch_fwd<128, false>(q, k, v, o, lse, B, Sq, Sk, Hq, Hkv, causal, scale, st, none, sp);
 }
+}  // namespace
+
+extern "C" {
 
 int sa_attn_fwd_fp8(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Sq, int Sk,
                     int Hq, int Hkv, int D, int causal, float scale, float q_descale, float k_descale,

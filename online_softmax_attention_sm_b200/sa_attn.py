@@ -29,6 +29,7 @@ SIGNATURES = {
     "sa_attn_bwd_workspace_size": (_Z, [_I, _I, _I]),
     "sa_attn_fwd_fp8": (_I, [_P] * 5 + [_I] * 7 + [_F, _F, _F, _F, _P]),
     "sa_attn_decode_single": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _F, _I, _I, _P, _Z, _P]),
+    "sa_attn_fwd_block_sparse_fp8": (_I, [_P] * 6 + [_I] * 7 + [_F, _F, _F, _F, _P, _Z, _P]),
     "sa_attn_bwd": (_I, [_P] * 9 + [_I] * 7 + [_F, _I, _P, _Z, _P]),
     "sa_attn_fwd_block_sparse": (_I, [_P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _F, _I, _P, _Z, _P]),
     "sa_attn_decode_workspace_size": (_Z, [_I, _I, _I, _I, _I, _I]),
@@ -217,6 +218,36 @@ def sa_attn_fwd_fp8(q8, k8, v8, q_descale, k_descale, v_descale, causal=False, s
     _check(lib().sa_attn_fwd_fp8(_ptr(q8), _ptr(k8), _ptr(v8), _ptr(out), _ptr(lse), B, Sq, Sk, Hq, Hkv, D,
                                  int(bool(causal)), float(scale), float(q_descale), float(k_descale),
                                  float(v_descale), _stream(stream)))
+    return out, lse
+
+
+def sa_attn_fwd_block_sparse_fp8(q8, k8, v8, block_mask, q_descale, k_descale, v_descale, causal=False, scale=None,
+                                 workspace=None, out=None, lse=None, return_lse=True, stream=None):
+    """FP8 block-sparse forward: q8/k8/v8 uint8 e4m3 codes as in :func:`sa_attn_fwd_fp8`,
+    block_mask as in :func:`sa_attn_fwd_block_sparse`.  Returns (o bf16, lse)."""
+    B, Sq, Hq, D = q8.shape
+    Sk, Hkv = k8.shape[1], k8.shape[2]
+    if k8.shape != (B, Sk, Hkv, D) or v8.shape != k8.shape:
+        raise ValueError(f"shape mismatch q{tuple(q8.shape)} k{tuple(k8.shape)} v{tuple(v8.shape)}")
+    for n, t in (("q8", q8), ("k8", k8), ("v8", v8), ("block_mask", block_mask)):
+        _check_tensor(n, t, torch.uint8, q8.device)
+    want = (B, Hq, -(-Sq // 128), -(-Sk // 128))
+    if tuple(block_mask.shape) != want:
+        raise ValueError(f"block_mask must be {want}, got {tuple(block_mask.shape)}")
+    if scale is None:
+        scale = 1.0 / math.sqrt(D)
+    if out is None:
+        out = torch.empty((B, Sq, Hq, D), dtype=torch.bfloat16, device=q8.device)
+    _check_tensor("out", out, torch.bfloat16, q8.device)
+    if return_lse and lse is None:
+        lse = torch.empty((B, Hq, Sq), dtype=torch.float32, device=q8.device)
+    need = sa_attn_fwd_block_sparse_workspace_size(B, Sq, Sk, Hq)
+    if workspace is None:
+        workspace = torch.empty(max(need, 16), dtype=torch.uint8, device=q8.device)
+    _check(lib().sa_attn_fwd_block_sparse_fp8(_ptr(q8), _ptr(k8), _ptr(v8), _ptr(out), _ptr(lse), _ptr(block_mask),
+                                              B, Sq, Sk, Hq, Hkv, D, int(bool(causal)), float(scale),
+                                              float(q_descale), float(k_descale), float(v_descale), _ptr(workspace),
+                                              workspace.numel() * workspace.element_size(), _stream(stream)))
     return out, lse
 
 
