@@ -6,12 +6,12 @@ It shares no code with the CUDA path.  Every function here is pinned by
 ``tests/test_oracle.py`` to closed forms, invariants and brute force; none is
 "parity unpinned".
 """
-from .attention import (attention, attention_rows, attention_blockwise, attention_varlen,
+from .attention import (attention, attention_rows, attention_blockwise, attention_varlen, attention_paged_prefill,
                         attention_block_sparse, attention_block_sparse_rows, block_sparse_pairs,
                         attention_backward, decode_e4m3, attention_fp8, decode, decode_paged,
                         combine_lse)
 
-__all__ = ["attention", "attention_rows", "attention_blockwise", "attention_varlen",
+__all__ = ["attention", "attention_rows", "attention_blockwise", "attention_varlen", "attention_paged_prefill",
            "attention_block_sparse", "attention_block_sparse_rows", "block_sparse_pairs",
            "attention_backward", "decode_e4m3", "attention_fp8", "decode", "decode_paged",
            "combine_lse"]

@@ -297,6 +297,34 @@ def attention_fp8(q8, k8, v8, q_descale, k_descale, v_descale, scale, causal=Fal
                      scale, causal)
 
 
+def attention_paged_prefill(q, k_cache, v_cache, cu_seqlens_q, block_table, seqlens_k, scale, causal=False):
+    """Packed queries against a paged K/V cache (chunked prefill; the Stem / AngelSlim page's
+    serving backend, "varlen" and "paged" paths).  q [total_q, Hq, D]; k_cache/v_cache
+    [num_pages, page_size, Hkv, D]; sequence b owns query rows cu_seqlens_q[b] ..
+    cu_seqlens_q[b+1]-1 and keys 0 .. seqlens_k[b]-1, key t in page block_table[b, t //
+    page_size] at row t % page_size (lengths clamped to the table).  Each sequence is
+    :func:`attention` of its rows and its gathered keys (causal bottom-right within it).
+    Returns O [total_q, Hq, D], LSE [Hq, total_q]; rows outside every sequence: 0 / -inf."""
+    q = _f64(q)
+    cq = [int(x) for x in np.asarray(cu_seqlens_q)]
+    bt = np.asarray(block_table)
+    page_size = k_cache.shape[1]
+    total_q, Hq, D = q.shape
+    O = np.zeros((total_q, Hq, D))
+    LSE = np.full((Hq, total_q), NEG_INF)
+    for b in range(len(cq) - 1):
+        q0, q1 = cq[b], cq[b + 1]
+        if q1 <= q0:
+            continue
+        n = int(min(max(int(seqlens_k[b]), 0), page_size * bt.shape[1]))
+        t = np.arange(n)
+        kb = _f64(k_cache)[bt[b, t // page_size], t % page_size]    # [n, Hkv, D] in key order
+        vb = _f64(v_cache)[bt[b, t // page_size], t % page_size]
+        o, lse = attention(q[None, q0:q1], kb[None], vb[None], scale, causal)
+        O[q0:q1], LSE[:, q0:q1] = o[0], lse[0]
+    return O, LSE
+
+
 def attention_blockwise(q, k, v, scale, causal=False, block=64):
     """The online-softmax recurrence, restated in float64 (TurboQuant page,
     ``online_softmax_attention``; StreamAttention page, "Kernel Design"): walk the

@@ -626,3 +626,47 @@ def test_attention_fp8_is_attention_of_the_dequantised_inputs():
     Od, Ld = attention(decode_e4m3(q8) * 0.01, decode_e4m3(k8) * 0.02, decode_e4m3(v8) * 0.5, 0.7, True)
     np.testing.assert_allclose(O, Od, atol=TOL)
     np.testing.assert_allclose(L, Ld, atol=TOL)
+
+
+# ---- packed queries against a paged K/V cache
+
+def test_paged_prefill_is_varlen_over_gathered_keys():
+    from oracle import attention_paged_prefill
+    # two sequences; queries are chunks at the end of their keys (chunked prefill)
+    lens_q, lens_k, page = [3, 5], [9, 6], 4
+    rng = np.random.default_rng(0)
+    q = rng.standard_normal((8, 4, 3))
+    k = rng.standard_normal((15, 2, 3))
+    v = rng.standard_normal((15, 2, 3))
+    cq, ck = np.array([0, 3, 8]), np.array([0, 9, 15])
+    O, L = attention_varlen(q, k, v, cq, ck, 0.6, True)
+    # pages of 4 keys, shuffled: sequence 0 -> 3 pages, sequence 1 -> 2 pages
+    perm = rng.permutation(6)
+    kc, vc = np.zeros((6, page, 2, 3)), np.zeros((6, page, 2, 3))
+    table = np.full((2, 3), 0)
+    for b, (k0, n) in enumerate(((0, 9), (9, 6))):
+        for i in range(-(-n // page)):
+            slot = perm[3 * b + i] if b == 0 else perm[3 + i]
+            rows = range(k0 + i * page, min(k0 + n, k0 + (i + 1) * page))
+            kc[slot, :len(rows)], vc[slot, :len(rows)] = k[list(rows)], v[list(rows)]
+            table[b, i] = slot
+    Op, Lp = attention_paged_prefill(q, kc, vc, cq, table, np.array(lens_k), 0.6, True)
+    np.testing.assert_allclose(Op, O, atol=TOL)
+    np.testing.assert_allclose(Lp, L, atol=TOL)
+
+
+def test_paged_prefill_lengths_clamp_and_empty():
+    from oracle import attention_paged_prefill
+    rng = np.random.default_rng(1)
+    q = rng.standard_normal((4, 2, 3))
+    kc, vc = rng.standard_normal((3, 4, 1, 3)), rng.standard_normal((3, 4, 1, 3))
+    table = np.array([[2, 0], [1, 1]])
+    cq = np.array([0, 2, 4])
+    O, L = attention_paged_prefill(q, kc, vc, cq, table, np.array([100, 0]), 0.5, False)
+    # sequence 0 clamps to its 8 keys: pages 2 then 0
+    keys = np.concatenate([kc[2], kc[0]])[None]
+    vals = np.concatenate([vc[2], vc[0]])[None]
+    Od, Ld = attention(q[None, :2], keys, vals, 0.5, False)
+    np.testing.assert_allclose(O[:2], Od[0], atol=TOL)
+    np.testing.assert_allclose(L[:, :2], Ld[0], atol=TOL)
+    assert np.all(O[2:] == 0) and np.all(np.isneginf(L[:, 2:]))           # no keys
