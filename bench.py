@@ -219,7 +219,7 @@ def main():
                                                    sa_attn_decode_workspace_size, sa_attn_fwd,
                                                    sa_attn_fwd_block_sparse, sa_attn_fwd_block_sparse_workspace_size,
                                                    sa_attn_bwd, sa_attn_bwd_workspace_size, sa_attn_fwd_fp8,
-                                                   sa_attn_fwd_block_sparse_fp8,
+                                                   sa_attn_fwd_block_sparse_fp8, sa_attn_fwd_paged,
                                                    sa_attn_fwd_varlen, sa_check_status)
     from online_softmax_attention_sm_b200.dist import aggregate_throughput, max_over_ranks, rank_seed
     from online_softmax_attention_sm_b200.inputs import (make_dout, make_qkv, make_qkv_fp8, make_workload_inputs,
@@ -370,7 +370,7 @@ def main():
 
     # packed variable-length prefill: the long prefill's heads over 16 sequences of 32768
     # tokens in all (inputs and outputs exceed the L2)
-    var_ms = [float("nan")]
+    var_ms = pg_ms = [float("nan")]
     lens = wv.lengths
     if run_var:
         vq, vk, vv = (t[0].to(dev) for t in make_qkv(1, wv.Sq, wv.Sk, wv.Hq, wv.Hkv, wv.D, wv.dtype,
@@ -390,7 +390,36 @@ def main():
         torch.cuda.synchronize(dev)
         sa_check_status(stream)
         var_ms = [a.elapsed_time(b) for a, b in vev]
-        del vq, vk, vv, vo, vlse
+        # the same mix with its keys in a paged cache: 128-key pages in a fixed shuffled order
+        nbs = [-(-n // 128) for n in lens]
+        mb = max(nbs)
+        perm = torch.randperm(len(lens) * mb, generator=torch.Generator().manual_seed(wv.seed)).tolist()
+        kc = torch.zeros((len(lens) * mb, 128, wv.Hkv, wv.D), dtype=vk.dtype, device=dev)
+        vc = torch.zeros_like(kc)
+        table = torch.zeros((len(lens), mb), dtype=torch.int32)
+        k0 = 0
+        for b_, n in enumerate(lens):
+            for i in range(nbs[b_]):
+                slot, rows = perm[b_ * mb + i], min(128, n - i * 128)
+                table[b_, i] = slot
+                kc[slot, :rows] = vk[k0 + i * 128:k0 + i * 128 + rows]
+                vc[slot, :rows] = vv[k0 + i * 128:k0 + i * 128 + rows]
+            k0 += n
+        table = table.to(dev)
+        seqk = torch.tensor(lens, dtype=torch.int32, device=dev)
+        pgev = []
+        for i in range(args.warmup + args.steps):
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            sa_attn_fwd_paged(vq, kc, vc, cu, table, seqk, max(lens), causal=wv.causal, scale=wv.scale, out=vo,
+                              lse=vlse, stream=stream)
+            e1.record(stream)
+            if i >= args.warmup:
+                pgev.append((e0, e1))
+        torch.cuda.synchronize(dev)
+        sa_check_status(stream)
+        pg_ms = [a.elapsed_time(b) for a, b in pgev]
+        del vq, vk, vv, vo, vlse, kc, vc
 
     # block-sparse prefill: the prefill workload's tensors under a Stem-shaped block mask
     # (4 sink blocks, 4 window blocks, 10 % of the blocks between drawn at random); one API
@@ -545,6 +574,7 @@ def main():
     b1_two_avg = max_over_ranks(sum(b1_two_ms) / len(b1_two_ms), dev)
     b1_single_avg = max_over_ranks(sum(b1_single_ms) / len(b1_single_ms), dev)
     var_avg = max_over_ranks(sum(var_ms) / len(var_ms), dev)
+    pg_avg = max_over_ranks(sum(pg_ms) / len(pg_ms), dev)
     sp_avg = max_over_ranks(sum(sp_ms) / len(sp_ms), dev)
     bwd_avg = max_over_ranks(sum(bwd_ms) / len(bwd_ms), dev)
     fp8_avg = max_over_ranks(sum(fp8_ms) / len(fp8_ms), dev)
@@ -601,7 +631,10 @@ def main():
                                "unit": "TFLOP/s", "bound": "tensor", "peak": peak,
                                "frac": wv.flops / (var_avg * 1e-3) / 1e12 / peak, "ms": var_avg,
                                "sequences": len(lens), "lengths": f"{min(lens)}-{max(lens)}",
-                               "kernel": "attn_fwd_sm100 (dynamic unit order)"},
+                               "kernel": "attn_fwd_sm100 (dynamic unit order)",
+                               "paged": {"value": wv.flops / (pg_avg * 1e-3) / 1e12, "unit": "TFLOP/s",
+                                         "frac": wv.flops / (pg_avg * 1e-3) / 1e12 / peak, "ms": pg_avg,
+                                         "layout": "the same keys in shuffled 128-key pages (sa_attn_fwd_paged)"}},
             "prefill_block_sparse": {"workload": f"{PREFILL} + Stem-shaped block mask (4 sink, 4 window, "
                                                  "10 % of the blocks between)",
                                      "value": sp_flops / (sp_avg * 1e-3) / 1e12, "unit": "TFLOP/s",

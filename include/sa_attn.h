@@ -99,6 +99,22 @@ int sa_attn_fwd_varlen(const void* q, const void* k, const void* v, void* o, flo
                        sa_stream_t stream);
 
 /*
+ * Forward over a paged K/V cache with packed queries (chunked prefill against cached
+ * prefixes; the Stem page's serving backend names "varlen" and "paged" paths): q, o
+ * [total_q, Hq, D] and lse [Hq, total_q] as sa_attn_fwd_varlen (cu_seqlens_q, max_seqlen_q);
+ * k_cache, v_cache [num_pages, page_size, Hkv, D]; sequence b's key t sits in page
+ * block_table[b * max_blocks + t / page_size] (int32, device) at row t % page_size, its key
+ * count seqlens_k[b] (int32, device; clamped to [0, page_size * max_blocks]).  Causal is
+ * bottom-right aligned within each sequence.  page_size must be a positive multiple of
+ * 128 (SA_ERR_UNSUPPORTED).  A table entry outside [0, num_pages) reads zeros.
+ */
+int sa_attn_fwd_paged(const void* q, const void* k_cache, const void* v_cache, void* o, float* lse,
+                      const int* cu_seqlens_q, const int* block_table, const int* seqlens_k, int B,
+                      int max_seqlen_q, int total_q, int Hq, int Hkv, int D, int page_size,
+                      int max_blocks, int num_pages, int causal, float scale, int dtype,
+                      sa_stream_t stream);
+
+/*
  * Block-sparse forward (Stem / AngelSlim page, section 2.3: attention over the 128 x 128
  * blocks a top-k mask keeps, with the initial "sink" blocks and a sliding window of blocks
  * among them).  Same tensors, layouts and rules as sa_attn_fwd, plus:

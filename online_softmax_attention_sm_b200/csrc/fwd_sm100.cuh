@@ -100,6 +100,13 @@ struct FwdParams {
   const int* cu_q;
   const int* cu_k;
   int max_sq;
+  // Paged K/V for packed queries (block_table non-null; cu_k unused): k/v are caches
+  // [num_pages, page_size, Hkv, D], sequence b's key t in page block_table[b * max_blocks +
+  // t / page_size] at row t % page_size, its length seqlens_k[b] (clamped to the table);
+  // page_size a multiple of 128, so a K/V tile never crosses a page.
+  const int* block_table;
+  const int* seqlens_k;
+  int max_blocks, page_size;
   // Block-sparse (the kernel's SPARSE instance): unit records of sp_stride uint16 each,
   // record (b * Hq + h) * n_qblk + query block.
   const uint16_t* sp;
@@ -133,7 +140,7 @@ __device__ __forceinline__ int fwd_kv_tiles(int sq, int sk, int causal, int r0) 
 __device__ __forceinline__ void fwd_check_lengths(const FwdParams& p, int lane, int cta, int ncta) {
   for (int b = cta * 32 + lane; b < p.B; b += ncta * 32) {
     const int q0 = __ldg(p.cu_q + b), q1 = __ldg(p.cu_q + b + 1);
-    const int k0 = __ldg(p.cu_k + b), k1 = __ldg(p.cu_k + b + 1);
+    const int k0 = p.block_table ? 0 : __ldg(p.cu_k + b), k1 = p.block_table ? 0 : __ldg(p.cu_k + b + 1);  // paged: no cu_k
     if (q0 < 0 || q1 < q0 || q1 > p.Sq || q1 - q0 > p.max_sq || k0 < 0 || k1 < k0 || k1 > p.Sk)
       record_status(kStatusBadLengths, b);
   }
@@ -145,6 +152,10 @@ __device__ __forceinline__ void fwd_check_lengths(const FwdParams& p, int lane, 
 // fit in half the L2 and a (band, group) block fills about one round of the persistent
 // grid: the CTAs in flight then share K/V tiles through L2, and consecutive rounds hold
 // units of similar lengths (longest first overall, so the last units handed out are short).
+// PACKED: the instance may see packed sequences -- the dynamic one; the static instance
+// never does, and carries none of that code.  PAGED: the paged-cache instance (keys from
+// seqlens_k and the block table instead of cu_k).
+template <bool PACKED, bool PAGED = false>
 __device__ __forceinline__ UnitInfo fwd_unit(const FwdParams& p, int u) {
   UnitInfo x;
   const int G = p.Hq / p.Hkv;
@@ -164,13 +175,15 @@ __device__ __forceinline__ UnitInfo fwd_unit(const FwdParams& p, int u) {
   x.kvh = bk % p.Hkv;
   x.h = x.kvh * G + rem % G;
   x.q0 = qb * 256;
-  if (p.cu_q) {
+  if (PACKED && p.cu_q) {
     // clamped into the buffers: offsets that run backwards or past the end give an empty
     // or shortened sequence, never an access outside q/k/v/o
     const int q_lo = min(max(__ldg(p.cu_q + x.b), 0), p.Sq);
     const int q_hi = min(max(__ldg(p.cu_q + x.b + 1), q_lo), p.Sq);
-    const int k_lo = min(max(__ldg(p.cu_k + x.b), 0), p.Sk);
-    const int k_hi = min(max(__ldg(p.cu_k + x.b + 1), k_lo), p.Sk);
+    // paged: keys 0 .. seqlens_k[b]-1 of the sequence's pages (p.Sk = the table's capacity)
+    const int k_lo = PAGED ? 0 : min(max(__ldg(p.cu_k + x.b), 0), p.Sk);
+    const int k_hi = PAGED ? min(max(__ldg(p.seqlens_k + x.b), 0), p.Sk)
+                           : min(max(__ldg(p.cu_k + x.b + 1), k_lo), p.Sk);
     x.sq = q_hi - q_lo; x.sk = k_hi - k_lo;
     x.qbase = q_lo; x.kbase = k_lo; x.mb = 0;
   } else {
@@ -268,7 +281,7 @@ __device__ __forceinline__ void fwd_sparse_attach(const SM& sm, int slot, UnitIn
 }
 
 // ------------------------------------------------------------------ TMA producer
-template <int D, bool BF16, bool DYN, bool SPARSE, bool FP8>
+template <int D, bool BF16, bool DYN, bool SPARSE, bool FP8, bool PAGED>
 __device__ __forceinline__ void fwd_producer(const CUtensorMap* tm_q, const CUtensorMap* tm_k,
                                              const CUtensorMap* tm_v, const FwdParams& p,
                                              const FwdSmem<D, FP8>& sm, int lane, int cta, int ncta) {
@@ -294,7 +307,7 @@ __device__ __forceinline__ void fwd_producer(const CUtensorMap* tm_q, const CUte
         sm.uq[us] = u;
         if (SPARSE && u < p.n_units) {
           // the unit's K/V tile list lands in the queue slot with the posting itself
-          x = fwd_unit(p, u);
+          x = fwd_unit<DYN, PAGED>(p, u);
           const uint32_t bytes = (uint32_t)p.sp_stride * 2u;
           mbar_arrive_expect_tx(&sm.unit_full[us], bytes);
           bulk_copy_g2s(sm.lists + us * kSparseSlotBytes, fwd_sparse_record(p, x), bytes, &sm.unit_full[us]);
@@ -308,7 +321,7 @@ __device__ __forceinline__ void fwd_producer(const CUtensorMap* tm_q, const CUte
         }
       }
       if (u >= p.n_units) break;
-      if (!SPARSE) x = fwd_unit(p, u);
+      if (!SPARSE) x = fwd_unit<DYN, PAGED>(p, u);
       for (int j = 0; j < x.nkv_max && ok; ++j) {
         const int kt = SPARSE ? (int)(x.ent[j] & 0x3fffu) : j;   // key tile of this step
         for (int kv = 0; kv < 2 && ok; ++kv) {
@@ -319,10 +332,19 @@ __device__ __forceinline__ void fwd_producer(const CUtensorMap* tm_q, const CUte
           uint8_t* dst = sm.ring + slot * Cfg::TILE_BYTES;
           mbar_arrive_expect_tx(&sm.kv_full[slot], Cfg::TILE_BYTES);
           const CUtensorMap* tm = kv ? tm_v : tm_k;
+          {
+            // K/V tile coordinates: (key row, batch), or for a paged cache (row in page, page);
+            // a table entry outside the cache reads zeros (TMA fill), never other memory
+            int krow = x.kbase + kt * 128, kouter = x.mb;
+            if (PAGED) {
+              krow = (kt * 128) % p.page_size;
+              kouter = __ldg(p.block_table + (size_t)x.b * p.max_blocks + (kt * 128) / p.page_size);
+            }
 #pragma unroll
-          for (int c = 0; c < Cfg::KCH; ++c)
-            tma_load_4d(dst + c * Cfg::CHUNK_BYTES, tm, &sm.kv_full[slot], c * Cfg::CHUNK_ELEMS, x.kvh,
-                        x.kbase + kt * 128, x.mb);
+            for (int c = 0; c < Cfg::KCH; ++c)
+              tma_load_4d(dst + c * Cfg::CHUNK_BYTES, tm, &sm.kv_full[slot], c * Cfg::CHUNK_ELEMS, x.kvh, krow,
+                          kouter);
+          }
           ++ring_n;
           slot = (slot + 1 == Cfg::STAGES) ? 0 : slot + 1;
           if (j == 0 && kv == 0) {
@@ -412,7 +434,7 @@ __device__ __forceinline__ void mma_ts_f8_x1(uint32_t d_tmem, uint32_t a_tmem, u
       ::"r"(d_tmem), "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(acc) : "memory");
 }
 
-template <int D, bool BF16, bool DYN, bool SPARSE, bool FP8>
+template <int D, bool BF16, bool DYN, bool SPARSE, bool FP8, bool PAGED>
 __device__ __forceinline__ void fwd_mma(const FwdParams& p, const FwdSmem<D, FP8>& sm, uint32_t tmem_base,
                                         int lane, int cta, int ncta) {
   using Cfg = FwdCfg<D, FP8>;
@@ -445,7 +467,7 @@ __device__ __forceinline__ void fwd_mma(const FwdParams& p, const FwdSmem<D, FP8
       const int u = DYN ? fwd_next_unit(sm, n, 12, !SPARSE) : fwd_unit_of(n, cta, ncta);
       if (u < 0) { ok = false; break; }
       if (u >= p.n_units) break;
-      UnitInfo x = fwd_unit(p, u);
+      UnitInfo x = fwd_unit<DYN, PAGED>(p, u);
       if (SPARSE) fwd_sparse_attach(sm, n % kUnitQueue, x);
       if (x.nkv_max == 0) {
         if (SPARSE) fwd_release_unit(sm, n);
@@ -795,7 +817,7 @@ __device__ __forceinline__ void softmax_tile_masked(const uint32_t s_addr, const
   sum_f2x2(rse2, l_lse);
 }
 
-template <int D, bool BF16, bool DYN, bool SPARSE, bool FP8>
+template <int D, bool BF16, bool DYN, bool SPARSE, bool FP8, bool PAGED>
 __device__ __forceinline__ void fwd_softmax(const FwdParams& p, const FwdSmem<D, FP8>& sm, uint32_t tmem_base,
                                             int warp, int lane, int cta, int ncta) {
   using Cfg = FwdCfg<D, FP8>;
@@ -810,7 +832,7 @@ __device__ __forceinline__ void fwd_softmax(const FwdParams& p, const FwdSmem<D,
     const int u = DYN ? fwd_next_unit(sm, n, 23, !SPARSE) : fwd_unit_of(n, cta, ncta);
     if (u < 0) { ok = false; break; }
     if (u >= p.n_units) break;
-    UnitInfo x = fwd_unit(p, u);
+    UnitInfo x = fwd_unit<DYN, PAGED>(p, u);
     if (SPARSE) fwd_sparse_attach(sm, n % kUnitQueue, x);
     const int nkv = x.nkv[t];
     const int row = x.q0 + t * 128 + row_in_tile;
@@ -911,13 +933,14 @@ __device__ __forceinline__ void fwd_teardown(bool owner, uint32_t tmem_base, uin
   }
 }
 
-template <int D, bool BF16, bool DYN, bool SPARSE, bool FP8 = false>
+template <int D, bool BF16, bool DYN, bool SPARSE, bool FP8 = false, bool PAGED = false>
 __global__ void __launch_bounds__(384, 1)
 attn_fwd_sm100(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                const __grid_constant__ CUtensorMap tm_v, const FwdParams p) {
   using Cfg = FwdCfg<D, FP8>;
   static_assert(DYN || !SPARSE, "the block-sparse units go through the dynamic unit queue");
   static_assert(!FP8 || (BF16 && D == 128), "FP8: D = 128, bf16 output");
+  static_assert(!PAGED || (DYN && !SPARSE && !FP8), "the paged instance: dynamic, dense blocks, 16-bit");
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
   const FwdSmem<D, FP8> sm(smem);
@@ -955,13 +978,13 @@ attn_fwd_sm100(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
     // load / MMA warpgroup gives registers away; warp 2 checks packed sequence offsets,
     // warp 3 has no role
     regs_dec<Cfg::REGS_OTHER>();
-    if (warp == kWarpLoad) fwd_producer<D, BF16, DYN, SPARSE, FP8>(&tm_q, &tm_k, &tm_v, p, sm, lane, cta, ncta);
-    else if (warp == kWarpMma) fwd_mma<D, BF16, DYN, SPARSE, FP8>(p, sm, tmem_base, lane, cta, ncta);
+    if (warp == kWarpLoad) fwd_producer<D, BF16, DYN, SPARSE, FP8, PAGED>(&tm_q, &tm_k, &tm_v, p, sm, lane, cta, ncta);
+    else if (warp == kWarpMma) fwd_mma<D, BF16, DYN, SPARSE, FP8, PAGED>(p, sm, tmem_base, lane, cta, ncta);
     else if (warp == 2 && p.cu_q) fwd_check_lengths(p, lane, cta, ncta);
     fwd_teardown(warp == kWarpMma, tmem_base, Cfg::TMEM_COLS);
   } else {
     regs_inc<Cfg::REGS_SOFTMAX>();
-    fwd_softmax<D, BF16, DYN, SPARSE, FP8>(p, sm, tmem_base, warp - 4, lane, cta, ncta);
+    fwd_softmax<D, BF16, DYN, SPARSE, FP8, PAGED>(p, sm, tmem_base, warp - 4, lane, cta, ncta);
     fwd_teardown(false, tmem_base, Cfg::TMEM_COLS);
   }
 }

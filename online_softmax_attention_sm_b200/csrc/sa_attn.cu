@@ -205,6 +205,10 @@ struct FwdVarlen {
   const int* cu_q = nullptr;
   const int* cu_k = nullptr;
   int max_sq = 0, max_sk = 0;
+  // paged K/V (block_table set): caches [num_pages, page_size, Hkv, D], key lengths seqlens_k
+  const int* block_table = nullptr;
+  const int* seqlens_k = nullptr;
+  int max_blocks = 0, page_size = 0, num_pages = 0;
 };
 
 // Block-sparse unit records for launch_fwd (sp null: every key tile up to the diagonal).
@@ -233,12 +237,16 @@ int launch_fwd(const void* q, const void* k, const void* v, void* o, float* lse,
   CUtensorMap mq, mk, mv;
   int rc;
   if ((rc = make_map(&mq, q, map_ty, D, Hq, Sq, map_b, 128)) != SA_OK) return rc;
-  if ((rc = make_map(&mk, k, map_ty, D, Hkv, Sk, map_b, 128)) != SA_OK) return rc;
-  if ((rc = make_map(&mv, v, map_ty, D, Hkv, Sk, map_b, 128)) != SA_OK) return rc;
+  const bool paged = vl.block_table != nullptr;
+  const int k_rows = paged ? vl.page_size : Sk, k_outer = paged ? vl.num_pages : map_b;
+  if ((rc = make_map(&mk, k, map_ty, D, Hkv, k_rows, k_outer, 128)) != SA_OK) return rc;
+  if ((rc = make_map(&mv, v, map_ty, D, Hkv, k_rows, k_outer, 128)) != SA_OK) return rc;
   sa::FwdParams p;
   p.o = o; p.lse = lse;
   p.B = B; p.Sq = Sq; p.Sk = Sk; p.Hq = Hq; p.Hkv = Hkv; p.causal = causal;
   p.cu_q = vl.cu_q; p.cu_k = vl.cu_k;
+  p.block_table = vl.block_table; p.seqlens_k = vl.seqlens_k;
+  p.max_blocks = vl.max_blocks; p.page_size = vl.page_size;
   p.max_sq = packed ? vl.max_sq : Sq;
   p.sp = sparse.sp; p.sp_stride = sparse.stride;
   p.o_mul = o_mul;
@@ -293,6 +301,7 @@ int launch_fwd(const void* q, const void* k, const void* v, void* o, float* lse,
                                                    : sa::attn_fwd_sm100<D, BF16, false, false, true>;
   } else {
     kern = sparse.sp ? sa::attn_fwd_sm100<D, BF16, true, true>
+         : paged ? sa::attn_fwd_sm100<D, BF16, true, false, false, true>
          : (packed || fwd_use_dynamic(p, D, grid)) ? sa::attn_fwd_sm100<D, BF16, true, false>
                                                    : sa::attn_fwd_sm100<D, BF16, false, false>;
   }
@@ -564,6 +573,40 @@ int sa_attn_fwd_varlen(const void* q, const void* k, const void* v, void* o, flo
               : launch_fwd<64, false>(q, k, v, o, lse, B, total_q, total_k, Hq, Hkv, causal, scale, st, vl);
   return bf ? launch_fwd<128, true>(q, k, v, o, lse, B, total_q, total_k, Hq, Hkv, causal, scale, st, vl)
             : launch_fwd<128, false>(q, k, v, o, lse, B, total_q, total_k, Hq, Hkv, causal, scale, st, vl);
+}
+
+int sa_attn_fwd_paged(const void* q, const void* k_cache, const void* v_cache, void* o, float* lse,
+                      const int* cu_seqlens_q, const int* block_table, const int* seqlens_k, int B,
+                      int max_seqlen_q, int total_q, int Hq, int Hkv, int D, int page_size, int max_blocks,
+                      int num_pages, int causal, float scale, int dtype, sa_stream_t stream) {
+  int rc = check_dims(B, total_q, 1, Hq, Hkv, D, dtype, scale);
+  if (rc != SA_OK) return rc;
+  if (max_seqlen_q < 0) return fail(SA_ERR_INVALID, "negative max_seqlen_q");
+  if (causal != 0 && causal != 1) return fail(SA_ERR_INVALID, "causal must be 0 or 1");
+  if (page_size <= 0 || page_size % 128 != 0)
+    return fail(SA_ERR_UNSUPPORTED, "page_size must be a positive multiple of 128 (got %d)", page_size);
+  if (max_blocks <= 0 || num_pages <= 0) return fail(SA_ERR_INVALID, "max_blocks and num_pages must be positive");
+  if ((long long)max_blocks * page_size > 0x7fffffffLL) return fail(SA_ERR_UNSUPPORTED, "block table too long");
+  if (B == 0 || total_q == 0 || Hq == 0 || max_seqlen_q == 0) return SA_OK;
+  if (!cu_seqlens_q || !block_table || !seqlens_k)
+    return fail(SA_ERR_INVALID, "cu_seqlens_q, block_table and seqlens_k must be non-null");
+  if (((uintptr_t)cu_seqlens_q & 3u) || ((uintptr_t)block_table & 3u) || ((uintptr_t)seqlens_k & 3u))
+    return fail(SA_ERR_INVALID, "cu_seqlens_q, block_table and seqlens_k must be 4-byte aligned");
+  if ((rc = check_ptrs(q, k_cache, v_cache, o, lse)) != SA_OK) return rc;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  FwdVarlen vl;
+  vl.cu_q = cu_seqlens_q;
+  vl.max_sq = max_seqlen_q;
+  vl.max_sk = max_blocks * page_size;
+  vl.block_table = block_table; vl.seqlens_k = seqlens_k;
+  vl.max_blocks = max_blocks; vl.page_size = page_size; vl.num_pages = num_pages;
+  const int cap = max_blocks * page_size;
+  const bool bf = dtype == SA_BF16;
+  if (D == 64)
+    return bf ? launch_fwd<64, true>(q, k_cache, v_cache, o, lse, B, total_q, cap, Hq, Hkv, causal, scale, st, vl)
+              : launch_fwd<64, false>(q, k_cache, v_cache, o, lse, B, total_q, cap, Hq, Hkv, causal, scale, st, vl);
+  return bf ? launch_fwd<128, true>(q, k_cache, v_cache, o, lse, B, total_q, cap, Hq, Hkv, causal, scale, st, vl)
+            : launch_fwd<128, false>(q, k_cache, v_cache, o, lse, B, total_q, cap, Hq, Hkv, causal, scale, st, vl);
 }
 
 size_t sa_attn_fwd_block_sparse_workspace_size(int B, int Sq, int Sk, int Hq) {

@@ -30,6 +30,7 @@ SIGNATURES = {
     "sa_attn_fwd_fp8": (_I, [_P] * 5 + [_I] * 7 + [_F, _F, _F, _F, _P]),
     "sa_attn_decode_single": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _F, _I, _I, _P, _Z, _P]),
     "sa_attn_fwd_block_sparse_fp8": (_I, [_P] * 6 + [_I] * 7 + [_F, _F, _F, _F, _P, _Z, _P]),
+    "sa_attn_fwd_paged": (_I, [_P] * 8 + [_I] * 10 + [_F, _I, _P]),
     "sa_attn_bwd": (_I, [_P] * 9 + [_I] * 7 + [_F, _I, _P, _Z, _P]),
     "sa_attn_fwd_block_sparse": (_I, [_P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _F, _I, _P, _Z, _P]),
     "sa_attn_decode_workspace_size": (_Z, [_I, _I, _I, _I, _I, _I]),
@@ -287,6 +288,37 @@ def sa_attn_bwd(q, k, v, o, lse, dout, causal=False, scale=None, workspace=None,
                              _ptr(dv), B, Sq, Sk, Hq, Hkv, D, int(bool(causal)), float(scale), _DT[q.dtype],
                              _ptr(workspace), workspace.numel() * workspace.element_size(), _stream(stream)))
     return dq, dk, dv
+
+
+def sa_attn_fwd_paged(q, k_cache, v_cache, cu_seqlens_q, block_table, seqlens_k, max_seqlen_q, causal=False,
+                      scale=None, out=None, lse=None, return_lse=True, stream=None):
+    """Packed queries against a paged K/V cache.  q [total_q,Hq,D]; k_cache/v_cache
+    [num_pages, page_size, Hkv, D]; cu_seqlens_q int32 [B+1]; block_table int32 [B, max_blocks];
+    seqlens_k int32 [B] (all CUDA).  Returns (o [total_q,Hq,D], lse [Hq,total_q])."""
+    total_q, Hq, D = q.shape
+    num_pages, page_size, Hkv = k_cache.shape[0], k_cache.shape[1], k_cache.shape[2]
+    if k_cache.shape != (num_pages, page_size, Hkv, D) or v_cache.shape != k_cache.shape:
+        raise ValueError(f"shape mismatch q{tuple(q.shape)} k{tuple(k_cache.shape)} v{tuple(v_cache.shape)}")
+    if q.dtype not in _DT:
+        raise TypeError(f"unsupported dtype {q.dtype}")
+    for n, t in (("q", q), ("k_cache", k_cache), ("v_cache", v_cache)):
+        _check_tensor(n, t, q.dtype, q.device)
+    for n, t in (("cu_seqlens_q", cu_seqlens_q), ("block_table", block_table), ("seqlens_k", seqlens_k)):
+        _check_tensor(n, t, torch.int32, q.device)
+    B = cu_seqlens_q.numel() - 1
+    if block_table.dim() != 2 or block_table.shape[0] != B or seqlens_k.shape != (B,):
+        raise ValueError("block_table must be [B, max_blocks] and seqlens_k [B]")
+    if scale is None:
+        scale = 1.0 / math.sqrt(D)
+    if out is None:
+        out = torch.empty_like(q)
+    if return_lse and lse is None:
+        lse = torch.empty((Hq, total_q), dtype=torch.float32, device=q.device)
+    _check(lib().sa_attn_fwd_paged(_ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(out), _ptr(lse), _ptr(cu_seqlens_q),
+                                   _ptr(block_table), _ptr(seqlens_k), B, int(max_seqlen_q), total_q, Hq, Hkv, D,
+                                   page_size, block_table.shape[1], num_pages, int(bool(causal)), float(scale),
+                                   _DT[q.dtype], _stream(stream)))
+    return out, lse
 
 
 def sa_attn_fwd_simple(q, k, v, causal=False, scale=None, **kw):

@@ -288,6 +288,25 @@ def test_decode_single_rejects_invalid_arguments(L, kw, code):
                                    a["D"], a["scale"], a["dtype"], a["ns"], a["ws"], a["wsb"], None) == code
 
 
+@pytest.mark.parametrize("kw,code", [
+    (dict(q=NULL), sa.SA_ERR_INVALID),
+    (dict(bt=NULL), sa.SA_ERR_INVALID),
+    (dict(page=64), sa.SA_ERR_UNSUPPORTED),
+    (dict(page=200), sa.SA_ERR_UNSUPPORTED),
+    (dict(mb=0), sa.SA_ERR_INVALID),
+    (dict(npg=0), sa.SA_ERR_INVALID),
+    (dict(Hq=3, Hkv=2), sa.SA_ERR_INVALID),
+    (dict(causal=7), sa.SA_ERR_INVALID),
+])
+def test_fwd_paged_rejects_invalid_arguments(L, kw, code):
+    a = dict(q=FAKE, kc=FAKE, vc=FAKE, o=FAKE, lse=NULL, cq=FAKE, bt=FAKE, sk=FAKE, B=2, mq=64, tq=100, Hq=2, Hkv=1,
+             D=64, page=128, mb=4, npg=8, causal=1, scale=0.125, dtype=0)
+    a.update(kw)
+    assert L.sa_attn_fwd_paged(a["q"], a["kc"], a["vc"], a["o"], a["lse"], a["cq"], a["bt"], a["sk"], a["B"], a["mq"],
+                               a["tq"], a["Hq"], a["Hkv"], a["D"], a["page"], a["mb"], a["npg"], a["causal"],
+                               a["scale"], a["dtype"], None) == code
+
+
 def test_version(L):
     assert re.fullmatch(r"\d+\.\d+\.\d+", sa.sa_version())
 
