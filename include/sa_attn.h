@@ -19,6 +19,15 @@
  * Layouts (all contiguous, row-major, elements of `dtype` unless stated):
  *   prefill  q [B, Sq, Hq, D]   k, v [B, Sk, Hkv, D]   o [B, Sq, Hq, D]   lse [B, Hq, Sq] fp32
  *   decode   q [B, Hq, D]       k, v [B, Sk, Hkv, D]   o [B, Hq, D]       lse [B, Hq]     fp32
+ *   packed   q [total_q, Hq, D] k, v [total_k, Hkv, D] o [total_q, Hq, D] lse [Hq, total_q]
+ *   paged    k, v caches [num_pages, page_size, Hkv, D] with a block table per sequence
+ *   FP8      q, k, v e4m3 codes (1 byte), o bf16
+ *
+ * Entry points: sa_attn_fwd (prefill), sa_attn_fwd_varlen (packed sequences),
+ * sa_attn_fwd_paged (packed queries over a paged cache), sa_attn_fwd_block_sparse (a
+ * block mask), sa_attn_fwd_fp8 and sa_attn_fwd_block_sparse_fp8 (e4m3 inputs), sa_attn_bwd
+ * (dQ, dK, dV), sa_attn_decode / sa_attn_decode_single / sa_attn_decode_noalloc /
+ * sa_attn_decode_paged (single-token decode), plus workspace-size queries and status.
  *
  * Conventions shared by every entry point:
  *   - All tensor pointers are DEVICE pointers owned by the caller; the library keeps no
