@@ -272,7 +272,8 @@ __device__ __forceinline__ void bwd_init(const BwdSmem<D>& sm) {
 // The MMA warp's loop shared by both kernels: nsteps steps, each two halves; issue_s(n, h)
 // issues the S / dP products of half h of step n and commits s_ready[h]; issue_acc(n, h)
 // the accumulating products of half h of step n.  Step n's ring slot is released once its
-// products complete.  Returns false if a wait gave up.
+// accumulating products complete (not waiting for step n + 1's S / dP, so the load of step
+// n + 2 starts a product earlier).  Returns false if a wait gave up.
 template <int D, typename IssueS, typename IssueAcc>
 __device__ __forceinline__ bool bwd_mma_loop(const BwdSmem<D>& sm, int nsteps, IssueS issue_s, IssueAcc issue_acc) {
   using Cfg = BwdCfg<D>;
@@ -287,6 +288,8 @@ __device__ __forceinline__ bool bwd_mma_loop(const BwdSmem<D>& sm, int nsteps, I
       if (!mbar_wait_warp(&sm.p_ready[h], n & 1, sm.abort_flag, 61 + h)) return false;
       tc_fence_after();
       issue_acc(n, h);
+      // the slot's last reader is in the pipe: release it before step n + 1's second half
+      if (h == 1) mma_commit_warp(&sm.empty[n % Cfg::STAGES]);
       if (more) {
         if (h == 0) {
           const int m = n + 1;
@@ -296,7 +299,6 @@ __device__ __forceinline__ bool bwd_mma_loop(const BwdSmem<D>& sm, int nsteps, I
         issue_s(n + 1, h);
       }
     }
-    mma_commit_warp(&sm.empty[n % Cfg::STAGES]);
   }
   return true;
 }
