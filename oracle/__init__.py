@@ -8,10 +8,10 @@ It shares no code with the CUDA path.  Every function here is pinned by
 """
 from .attention import (attention, attention_rows, attention_blockwise, attention_varlen, attention_paged_prefill,
                         attention_block_sparse, attention_block_sparse_rows, block_sparse_pairs,
-                        attention_backward, decode_e4m3, attention_fp8, decode, decode_paged,
-                        combine_lse)
+                        attention_backward, attention_backward_rows, attention_backward_keys, decode_e4m3,
+                        attention_fp8, decode, decode_paged, combine_lse)
 
 __all__ = ["attention", "attention_rows", "attention_blockwise", "attention_varlen", "attention_paged_prefill",
            "attention_block_sparse", "attention_block_sparse_rows", "block_sparse_pairs",
-           "attention_backward", "decode_e4m3", "attention_fp8", "decode", "decode_paged",
-           "combine_lse"]
+           "attention_backward", "attention_backward_rows", "attention_backward_keys", "decode_e4m3",
+           "attention_fp8", "decode", "decode_paged", "combine_lse"]

@@ -275,6 +275,71 @@ def attention_backward(q, k, v, do, scale, causal=False):
     return dq, dk, dv
 
 
+def _probabilities(qm, km, scale, vis):
+    """Softmax weights P [n, Sk] of query rows qm [n, D] over keys km [Sk, D] (visible
+    where vis [n, Sk]); rows without a visible key get P = 0."""
+    s = np.where(vis, scale * (qm @ km.T), NEG_INF)
+    p = np.zeros_like(s)
+    has = vis.any(axis=1)
+    if has.any():
+        m = s[has].max(axis=1)
+        e = np.exp(s[has] - m[:, None])
+        p[has] = e / e.sum(axis=1, keepdims=True)
+    return p
+
+
+def attention_backward_rows(q, k, v, do, scale, causal, b, h, rows):
+    """dQ of selected query rows of one (batch, query head), for long sequences where
+    :func:`attention_backward`'s full score matrices would not fit.  A row's gradient
+    needs only its own softmax row (the StreamAttention page, "Backward": probabilities
+    recomputed from the scores): P_i over the visible keys, O_i = P_i V, dP_i = dO_i V^T,
+    Delta_i = dO_i . O_i, dS_i = P_i * (dP_i - Delta_i), dQ_i = scale * dS_i K.
+    Shapes as :func:`attention_backward`; returns dQ [len(rows), D] in float64."""
+    rows = np.asarray(rows, dtype=np.int64)
+    Sq, Hq = q.shape[1], q.shape[2]
+    Sk, Hkv = k.shape[1], k.shape[2]
+    kvh = h // (Hq // Hkv)
+    qm, dom = _f64(q[b, rows, h, :]), _f64(do[b, rows, h, :])
+    if Sk == 0:
+        return np.zeros_like(qm)
+    km, vm = _f64(k[b, :, kvh, :]), _f64(v[b, :, kvh, :])
+    p = _probabilities(qm, km, scale, _visible(Sq, Sk, causal, rows))
+    dp = dom @ vm.T
+    delta = (dom * (p @ vm)).sum(axis=1)
+    ds = p * (dp - delta[:, None])
+    return scale * (ds @ km)
+
+
+def attention_backward_keys(q, k, v, do, scale, causal, b, kvh, keys):
+    """dK and dV of selected keys of one (batch, KV head): the sums over the G query heads
+    of the group and over every query row that sees the key (dV_j = sum_i P_ij dO_i,
+    dK_j = scale * sum_i dS_ij Q_i, with P, dS of :func:`attention_backward_rows`).  Only
+    the rows that see some selected key are formed (causal: rows i >= min(keys) - (Sk - Sq)),
+    so keys near the end of a long causal sequence stay cheap.  Returns dK, dV
+    [len(keys), D] in float64."""
+    keys = np.asarray(keys, dtype=np.int64)
+    Sq, Hq, D = q.shape[1], q.shape[2], q.shape[3]
+    Sk, Hkv = k.shape[1], k.shape[2]
+    G = Hq // Hkv
+    dk = np.zeros((keys.size, D))
+    dv = np.zeros((keys.size, D))
+    if Sq == 0 or keys.size == 0:
+        return dk, dv
+    first = max(0, int(keys.min()) - (Sk - Sq)) if causal else 0
+    rows = np.arange(first, Sq)
+    vis = _visible(Sq, Sk, causal, rows)
+    km, vm = _f64(k[b, :, kvh, :]), _f64(v[b, :, kvh, :])
+    for h in range(kvh * G, (kvh + 1) * G):
+        qm, dom = _f64(q[b, rows, h, :]), _f64(do[b, rows, h, :])
+        p = _probabilities(qm, km, scale, vis)
+        dp = dom @ vm.T
+        delta = (dom * (p @ vm)).sum(axis=1)
+        ds = p * (dp - delta[:, None])
+        dv += p[:, keys].T @ dom
+        dk += scale * (ds[:, keys].T @ qm)
+    return dk, dv
+
+
 def decode_e4m3(codes):
     """Values of 8-bit e4m3 codes (sign bit, 4-bit exponent with bias 7, 3-bit mantissa;
     exponent 0 = subnormal m * 2^-9; 0x7f / 0xff = NaN; no infinities; largest 448) as

@@ -596,6 +596,53 @@ def test_backward_rows_without_keys_contribute_nothing():
     np.testing.assert_allclose(dv2, dv, atol=TOL)
 
 
+@pytest.mark.parametrize("causal,Sq,Sk", [(False, 7, 9), (True, 9, 9), (True, 6, 11), (True, 11, 6)])
+def test_backward_rows_and_keys_match_the_full_backward(causal, Sq, Sk):
+    # the sampled forms give the full backward's dQ rows and dK / dV keys, GQA included,
+    # for rows that see no key (Sq > Sk) and keys that no row sees in full
+    from oracle import attention_backward_keys, attention_backward_rows
+    q, k, v = qkv(B=2, Sq=Sq, Sk=Sk, Hq=6, Hkv=2, D=5, seed=81)
+    do = rnd(q.shape, 82)
+    dq, dk, dv = attention_backward(q, k, v, do, 0.6, causal)
+    rows = [0, Sq // 2, Sq - 1]
+    keys = [0, Sk // 3, Sk - 2, Sk - 1]
+    for b in range(2):
+        for h in range(6):
+            np.testing.assert_allclose(attention_backward_rows(q, k, v, do, 0.6, causal, b, h, rows),
+                                       dq[b, rows, h], atol=TOL)
+        for kvh in range(2):
+            gk, gv = attention_backward_keys(q, k, v, do, 0.6, causal, b, kvh, keys)
+            np.testing.assert_allclose(gk, dk[b, keys, kvh], atol=TOL)
+            np.testing.assert_allclose(gv, dv[b, keys, kvh], atol=TOL)
+
+
+def test_backward_rows_and_keys_match_central_differences():
+    # brute force on a tiny causal GQA case, independent of the full backward
+    from oracle import attention_backward_keys, attention_backward_rows
+    q, k, v = qkv(B=1, Sq=4, Sk=5, Hq=2, Hkv=1, D=3, seed=83)
+    do = rnd(q.shape, 84)
+    eps = 1e-6
+
+    def num_grad(x, idx):
+        old = x[idx]
+        x[idx] = old + eps
+        lp = loss(q, k, v, do, 0.7, True)
+        x[idx] = old - eps
+        lm = loss(q, k, v, do, 0.7, True)
+        x[idx] = old
+        return (lp - lm) / (2 * eps)
+
+    dq = attention_backward_rows(q, k, v, do, 0.7, True, 0, 1, [2, 3])
+    for r, i in enumerate([2, 3]):
+        for d in range(3):
+            assert abs(dq[r, d] - num_grad(q, (0, i, 1, d))) < 1e-7
+    dk, dv = attention_backward_keys(q, k, v, do, 0.7, True, 0, 0, [1, 4])
+    for r, j in enumerate([1, 4]):
+        for d in range(3):
+            assert abs(dk[r, d] - num_grad(k, (0, j, 0, d))) < 1e-7
+            assert abs(dv[r, d] - num_grad(v, (0, j, 0, d))) < 1e-7
+
+
 # ---- FP8 (e4m3) inputs
 
 def test_decode_e4m3_known_codes():
