@@ -175,6 +175,11 @@ int sa_attn_decode_single(const void* q, const void* k, const void* v, void* o, 
  * Computes sa_attn_fwd of the dequantised tensors q*q_descale, k*k_descale, v*v_descale:
  * S on kind::f8f6f4 tensor cores (exact products, fp32 sums), P rounded to e4m3 for P V.
  * D must be 128 (else SA_ERR_UNSUPPORTED); descales finite and > 0 (else SA_ERR_INVALID).
+ * Accuracy: each weight is rounded to e4m3 relative to its row's running reference max,
+ * and weights below 2^-10 of that reference become zero.  Up to about a thousand keys
+ * this loss is negligible.  On long rows dominated by a few keys (attention sinks) the many
+ * small weights can together carry much of the row's mass, and the result then departs
+ * from the dequantised attention by far more than e4m3 rounding alone would suggest.
  */
 int sa_attn_fwd_fp8(const void* q, const void* k, const void* v, void* o, float* lse,
                     int B, int Sq, int Sk, int Hq, int Hkv, int D, int causal, float scale,
