@@ -653,6 +653,9 @@ def main():
                             "peak": 2 * peak, "peak_source": "measured bf16 burst x 2 (nominal fp8 : bf16)",
                             "frac": wp.flops / (fp8_avg * 1e-3) / 1e12 / (2 * peak), "ms": fp8_avg,
                             "kernel": "attn_fwd_sm100 (FP8 instance: kind::f8f6f4 QK and PV, e4m3 P)",
+                            "accuracy": "open: e4m3 weights below 2^-10 of the row reference round to zero; "
+                                        "on this workload's long sink-dominated rows a host simulation of that "
+                                        "rounding gives per-row max |O error| median 0.013, 90th pct 1.05",
                             "block_sparse": {"value": sp8_flops / (sp8_avg * 1e-3) / 1e12, "unit": "TFLOP/s",
                                              "frac": sp8_flops / (sp8_avg * 1e-3) / 1e12 / (2 * peak),
                                              "ms": sp8_avg, "mask": "the bf16 block-sparse leg's Stem-shaped mask"}},
