@@ -10,7 +10,19 @@ O to bf16 (2^-8 |O|):
 with P the exact normalised weights.  Weights below e4m3's normal range (2^-6 of the
 reference) have an absolute rounding error of at most 2^-10 instead; `a` = 2e-3 covers
 their sum here (their errors are unbiased; at most a few hundredths of the mass sit there).
-The LSE uses fp32 sums of unrounded weights: 1e-3 as for the 16-bit forward."""
+The LSE uses fp32 sums of unrounded weights: 1e-3 as for the 16-bit forward.
+
+At the bench's 32768-token size the weights e4m3 cannot hold matter: p_j = 2^(s_j - m)
+below 2^-10 round to zero, and on long rows that a few keys dominate (the sink recipe)
+those weights can carry most of the mass.  There the check uses the rounding bound
+written out term by term: with the exact weights p_j relative to the row max (the
+kernel's reference is at or below the max, which only makes its weights larger and its
+rounding finer), |p~_j - p_j| <= e_j = max(u p_j, min(p_j, 2^-10)), and since
+O_gpu - O = sum_j (p~_j - p_j)(v_j - O) / sum_j p~_j,
+    |O_gpu - O| <= sum_j e_j |v_j - O| / (sum_j p_j - sum_j e_j)
+                   + 1e-4 sum_j P_j |v_j - O| + 2^-8 |O| + 2e-3,
+the 1e-4 term for the exponentials computed on the FMA pipe (relative error 7.6e-5).
+The LSE, from unrounded weights, keeps its 1e-3."""
 import math
 import zlib
 
@@ -20,7 +32,8 @@ import torch
 
 import oracle
 from online_softmax_attention_sm_b200 import sa_attn_fwd_block_sparse_fp8, sa_attn_fwd_fp8, sa_check_status
-from online_softmax_attention_sm_b200.inputs import make_qkv_fp8, stem_block_mask
+from online_softmax_attention_sm_b200.inputs import make_qkv_fp8, sample_rows, stem_block_mask
+from online_softmax_attention_sm_b200.workloads import WORKLOADS
 
 pytestmark = pytest.mark.gpu
 
@@ -102,3 +115,56 @@ def test_fp8_block_sparse_within_the_derived_bound(causal):
     fin = np.isfinite(L)
     assert np.array_equal(np.isneginf(lg), np.isneginf(L))
     assert np.abs(lg[fin] - L[fin]).max() <= 1e-3
+
+
+def rounding_bound_rows(k, v, q_rows, scale, rows, Sq, O):
+    """The flushed-weight bound of the module docstring for query rows `rows` (causal,
+    bottom-right) of one head: k, v [Sk, D] and q_rows [n, D] dequantised float64, O [n, D]
+    the oracle's output of those rows."""
+    Sk = k.shape[0]
+    out = np.zeros_like(O)
+    for r, i in enumerate(rows):
+        n = min(Sk, i + Sk - Sq + 1)
+        s = scale * (k[:n] @ q_rows[r])
+        p = np.exp(s - s.max())
+        e = np.maximum(U * p, np.minimum(p, 2.0 ** -10))
+        dev_ = np.abs(v[:n] - O[r])
+        out[r] = ((e @ dev_) / (p.sum() - e.sum()) + 1e-4 * (p @ dev_) / p.sum()
+                  + 2.0 ** -8 * np.abs(O[r]) + 2e-3)
+    return out
+
+
+def fp8_sampled_errors(q8, k8, v8, qd, kd, vd, scale, o, lse, heads, n_rows, seed):
+    """Largest |O - oracle| / bound and |LSE - oracle| over sampled rows of `heads`
+    (batch 0, causal): o [B, Sq, Hq, D] and lse [B, Hq, Sq] as float64 arrays."""
+    Sq, Hq = q8.shape[1], q8.shape[2]
+    G = Hq // k8.shape[2]
+    worst_o = worst_l = 0.0
+    for h in heads:
+        kvh = h // G
+        qh = oracle.decode_e4m3(q8[:, :, h:h + 1].numpy()) * qd
+        kh = oracle.decode_e4m3(k8[:, :, kvh:kvh + 1].numpy()) * kd
+        vh = oracle.decode_e4m3(v8[:, :, kvh:kvh + 1].numpy()) * vd
+        rows = sample_rows(Sq, n_rows, seed=seed + h, extra=(Sq - 1,))
+        O, L = oracle.attention_rows(qh, kh, vh, scale, True, 0, 0, rows)
+        bound = rounding_bound_rows(kh[0, :, 0], vh[0, :, 0], qh[0, rows, 0], scale, rows, Sq, O)
+        worst_o = max(worst_o, float((np.abs(o[0, rows, h] - O) / bound).max()))
+        worst_l = max(worst_l, float(np.abs(lse[0, h, rows] - L).max()))
+    return worst_o, worst_l
+
+
+def test_fp8_long_gqa_causal_sampled_rows():
+    # the bench's FP8 leg: the 32768-token GQA workload's draws (sinks included) in e4m3
+    w = WORKLOADS["gqa_causal_s32768_d128_bf16_sinks"]
+    q8, k8, v8, qd, kd, vd = make_qkv_fp8(w.B, w.Sq, w.Sk, w.Hq, w.Hkv, w.D, seed=w.seed,
+                                          input_scale=w.input_scale, k_sink_rows=w.k_sink_rows,
+                                          k_sink_factor=w.k_sink_factor)
+    dev = torch.device("cuda:0")
+    o, lse = sa_attn_fwd_fp8(q8.to(dev), k8.to(dev), v8.to(dev), qd, kd, vd, causal=True, scale=w.scale)
+    sa_check_status()
+    o, lse = o.double().cpu().numpy(), lse.double().cpu().numpy()
+    assert np.all(np.isfinite(o)) and np.all(np.isfinite(lse))
+    worst_o, worst_l = fp8_sampled_errors(q8, k8, v8, qd, kd, vd, w.scale, o, lse, heads=range(0, w.Hq, 4),
+                                          n_rows=24, seed=w.seed)
+    assert worst_o <= 1.0, f"max |O - oracle| / bound on sampled rows = {worst_o:.3f}"
+    assert worst_l <= 1e-3, f"max |LSE - oracle| on sampled rows = {worst_l:.3e}"
