@@ -1,4 +1,5 @@
-"""B200 (sm_100a) fused online-softmax attention: prefill forward and split-KV decode.
+"""B200 (sm_100a) fused online-softmax attention: prefill forward (dense, packed, paged,
+block-sparse, FP8), backward, and split-KV decode (dense, paged, single-launch).
 
 The computation runs in hand-written CUDA kernels behind the C ABI of
 ``include/sa_attn.h`` (``libsa_attn.so``); :mod:`.sa_attn` is its Python binding.
