@@ -94,6 +94,23 @@ def _check_tensor(name, t, dtype, device):
         raise ValueError(f"{name} must be contiguous")
 
 
+def _check_out(name, t, shape, dtype, device):
+    """A caller-supplied output buffer: dtype, device, contiguity and exactly `shape` (the
+    kernels write every element of that shape, so a smaller buffer would be overrun)."""
+    _check_tensor(name, t, dtype, device)
+    if tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name} must have shape {tuple(shape)}, got {tuple(t.shape)}")
+
+
+def _check_workspace(t, device):
+    """Device scratch: on the inputs' device and contiguous (its size is checked by the
+    library, which returns SA_ERR_WORKSPACE when it is short)."""
+    if t.device != device:
+        raise ValueError(f"workspace: on {t.device}, expected {device}")
+    if not t.is_contiguous():
+        raise ValueError("workspace must be contiguous")
+
+
 def sa_attn_fwd(q, k, v, causal=False, scale=None, out=None, lse=None, return_lse=True,
                 stream=None, simple=False):
     """Attention forward.  q [B,Sq,Hq,D], k/v [B,Sk,Hkv,D] (fp16/bf16, CUDA, contiguous).
@@ -110,11 +127,11 @@ def sa_attn_fwd(q, k, v, causal=False, scale=None, out=None, lse=None, return_ls
         scale = 1.0 / math.sqrt(D)
     if out is None:
         out = torch.empty_like(q)
-    _check_tensor("out", out, q.dtype, q.device)
+    _check_out("out", out, q.shape, q.dtype, q.device)
     if return_lse and lse is None:
         lse = torch.empty((B, Hq, Sq), dtype=torch.float32, device=q.device)
     if lse is not None:
-        _check_tensor("lse", lse, torch.float32, q.device)
+        _check_out("lse", lse, (B, Hq, Sq), torch.float32, q.device)
     fn = lib().sa_attn_fwd_simple if simple else lib().sa_attn_fwd
     _check(fn(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse), B, Sq, Sk, Hq, Hkv, D,
               int(bool(causal)), float(scale), _DT[q.dtype], _stream(stream)))
@@ -145,11 +162,11 @@ def sa_attn_fwd_varlen(q, k, v, cu_seqlens_q, cu_seqlens_k, max_seqlen_q, max_se
         scale = 1.0 / math.sqrt(D)
     if out is None:
         out = torch.empty_like(q)
-    _check_tensor("out", out, q.dtype, q.device)
+    _check_out("out", out, q.shape, q.dtype, q.device)
     if return_lse and lse is None:
         lse = torch.empty((Hq, total_q), dtype=torch.float32, device=q.device)
     if lse is not None:
-        _check_tensor("lse", lse, torch.float32, q.device)
+        _check_out("lse", lse, (Hq, total_q), torch.float32, q.device)
     _check(lib().sa_attn_fwd_varlen(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse), _ptr(cu_seqlens_q),
                                     _ptr(cu_seqlens_k), B, int(max_seqlen_q), int(max_seqlen_k), total_q,
                                     total_k, Hq, Hkv, D, int(bool(causal)), float(scale), _DT[q.dtype],
@@ -182,14 +199,15 @@ def sa_attn_fwd_block_sparse(q, k, v, block_mask, causal=False, scale=None, work
         scale = 1.0 / math.sqrt(D)
     if out is None:
         out = torch.empty_like(q)
-    _check_tensor("out", out, q.dtype, q.device)
+    _check_out("out", out, q.shape, q.dtype, q.device)
     if return_lse and lse is None:
         lse = torch.empty((B, Hq, Sq), dtype=torch.float32, device=q.device)
     if lse is not None:
-        _check_tensor("lse", lse, torch.float32, q.device)
+        _check_out("lse", lse, (B, Hq, Sq), torch.float32, q.device)
     need = sa_attn_fwd_block_sparse_workspace_size(B, Sq, Sk, Hq)
     if workspace is None:
         workspace = torch.empty(max(need, 16), dtype=torch.uint8, device=q.device)
+    _check_workspace(workspace, q.device)
     _check(lib().sa_attn_fwd_block_sparse(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse), _ptr(block_mask),
                                           B, Sq, Sk, Hq, Hkv, D, int(bool(causal)), float(scale), _DT[q.dtype],
                                           _ptr(workspace), workspace.numel() * workspace.element_size(),
@@ -211,11 +229,11 @@ def sa_attn_fwd_fp8(q8, k8, v8, q_descale, k_descale, v_descale, causal=False, s
         scale = 1.0 / math.sqrt(D)
     if out is None:
         out = torch.empty((B, Sq, Hq, D), dtype=torch.bfloat16, device=q8.device)
-    _check_tensor("out", out, torch.bfloat16, q8.device)
+    _check_out("out", out, (B, Sq, Hq, D), torch.bfloat16, q8.device)
     if return_lse and lse is None:
         lse = torch.empty((B, Hq, Sq), dtype=torch.float32, device=q8.device)
     if lse is not None:
-        _check_tensor("lse", lse, torch.float32, q8.device)
+        _check_out("lse", lse, (B, Hq, Sq), torch.float32, q8.device)
     _check(lib().sa_attn_fwd_fp8(_ptr(q8), _ptr(k8), _ptr(v8), _ptr(out), _ptr(lse), B, Sq, Sk, Hq, Hkv, D,
                                  int(bool(causal)), float(scale), float(q_descale), float(k_descale),
                                  float(v_descale), _stream(stream)))
@@ -239,12 +257,15 @@ def sa_attn_fwd_block_sparse_fp8(q8, k8, v8, block_mask, q_descale, k_descale, v
         scale = 1.0 / math.sqrt(D)
     if out is None:
         out = torch.empty((B, Sq, Hq, D), dtype=torch.bfloat16, device=q8.device)
-    _check_tensor("out", out, torch.bfloat16, q8.device)
+    _check_out("out", out, (B, Sq, Hq, D), torch.bfloat16, q8.device)
     if return_lse and lse is None:
         lse = torch.empty((B, Hq, Sq), dtype=torch.float32, device=q8.device)
+    if lse is not None:
+        _check_out("lse", lse, (B, Hq, Sq), torch.float32, q8.device)
     need = sa_attn_fwd_block_sparse_workspace_size(B, Sq, Sk, Hq)
     if workspace is None:
         workspace = torch.empty(max(need, 16), dtype=torch.uint8, device=q8.device)
+    _check_workspace(workspace, q8.device)
     _check(lib().sa_attn_fwd_block_sparse_fp8(_ptr(q8), _ptr(k8), _ptr(v8), _ptr(out), _ptr(lse), _ptr(block_mask),
                                               B, Sq, Sk, Hq, Hkv, D, int(bool(causal)), float(scale),
                                               float(q_descale), float(k_descale), float(v_descale), _ptr(workspace),
@@ -284,6 +305,7 @@ def sa_attn_bwd(q, k, v, o, lse, dout, causal=False, scale=None, workspace=None,
     need = sa_attn_bwd_workspace_size(B, Sq, Hq)
     if workspace is None:
         workspace = torch.empty(max(need, 16), dtype=torch.uint8, device=q.device)
+    _check_workspace(workspace, q.device)
     _check(lib().sa_attn_bwd(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), _ptr(dout), _ptr(dq), _ptr(dk),
                              _ptr(dv), B, Sq, Sk, Hq, Hkv, D, int(bool(causal)), float(scale), _DT[q.dtype],
                              _ptr(workspace), workspace.numel() * workspace.element_size(), _stream(stream)))
@@ -314,6 +336,9 @@ def sa_attn_fwd_paged(q, k_cache, v_cache, cu_seqlens_q, block_table, seqlens_k,
         out = torch.empty_like(q)
     if return_lse and lse is None:
         lse = torch.empty((Hq, total_q), dtype=torch.float32, device=q.device)
+    _check_out("out", out, q.shape, q.dtype, q.device)
+    if lse is not None:
+        _check_out("lse", lse, (Hq, total_q), torch.float32, q.device)
     _check(lib().sa_attn_fwd_paged(_ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(out), _ptr(lse), _ptr(cu_seqlens_q),
                                    _ptr(block_table), _ptr(seqlens_k), B, int(max_seqlen_q), total_q, Hq, Hkv, D,
                                    page_size, block_table.shape[1], num_pages, int(bool(causal)), float(scale),
@@ -353,9 +378,13 @@ def sa_attn_decode(q, k, v, scale=None, num_splits=0, workspace=None, out=None, 
         out = torch.empty_like(q)
     if return_lse and lse is None:
         lse = torch.empty((B, Hq), dtype=torch.float32, device=q.device)
+    _check_out("out", out, q.shape, q.dtype, q.device)
+    if lse is not None:
+        _check_out("lse", lse, (B, Hq), torch.float32, q.device)
     need = sa_attn_decode_workspace_size(B, Sk, Hq, Hkv, D, num_splits)
     if workspace is None:
         workspace = torch.empty(max(need, 16), dtype=torch.uint8, device=q.device)
+    _check_workspace(workspace, q.device)
     fn = lib().sa_attn_decode_single if single else lib().sa_attn_decode
     _check(fn(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse), B, Sk, Hq, Hkv, D, float(scale), _DT[q.dtype],
               int(num_splits), _ptr(workspace), workspace.numel() * workspace.element_size(), _stream(stream)))
@@ -397,9 +426,13 @@ def sa_attn_decode_paged(q, k_cache, v_cache, block_table, seqlens, scale=None, 
         out = torch.empty_like(q)
     if return_lse and lse is None:
         lse = torch.empty((B, Hq), dtype=torch.float32, device=q.device)
+    _check_out("out", out, q.shape, q.dtype, q.device)
+    if lse is not None:
+        _check_out("lse", lse, (B, Hq), torch.float32, q.device)
     need = sa_attn_decode_paged_workspace_size(B, Hq, Hkv, D, page_size, max_blocks, num_splits)
     if workspace is None:
         workspace = torch.empty(max(need, 16), dtype=torch.uint8, device=q.device)
+    _check_workspace(workspace, q.device)
     _check(lib().sa_attn_decode_paged(_ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(block_table), _ptr(seqlens),
                                       _ptr(out), _ptr(lse), B, Hq, Hkv, D, page_size, max_blocks, num_pages,
                                       float(scale), _DT[q.dtype], int(num_splits), _ptr(workspace),

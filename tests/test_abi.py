@@ -316,3 +316,46 @@ def test_library_has_no_cpu_path():
     import online_softmax_attention_sm_b200 as pkg
     src = open(os.path.join(os.path.dirname(pkg.__file__), "sa_attn.py")).read()
     assert "oracle" not in src and "scaled_dot_product" not in src and "softmax(" not in src
+
+
+def test_binding_rejects_wrong_output_and_workspace_buffers(L):
+    # a caller's out / lse of the wrong shape, or a workspace on another device, raises in the
+    # binding before anything is launched (host tensors: nothing here reaches a kernel)
+    import torch
+    f16, u8 = torch.float16, torch.uint8
+    q, k = torch.zeros(1, 8, 2, 64, dtype=f16), torch.zeros(1, 8, 1, 64, dtype=f16)
+    with pytest.raises(ValueError, match="out must have shape"):
+        sa.sa_attn_fwd(q, k, k, out=torch.empty(1, 7, 2, 64, dtype=f16))
+    with pytest.raises(ValueError, match="lse must have shape"):
+        sa.sa_attn_fwd(q, k, k, lse=torch.empty(1, 2, 7))
+    mask = torch.ones(1, 2, 1, 1, dtype=u8)
+    with pytest.raises(ValueError, match="lse must have shape"):
+        sa.sa_attn_fwd_block_sparse(q, k, k, mask, lse=torch.empty(2, 8))
+    with pytest.raises(ValueError, match="workspace: on meta"):
+        sa.sa_attn_fwd_block_sparse(q, k, k, mask, workspace=torch.empty(4096, dtype=u8, device="meta"))
+    qp, kp = torch.zeros(10, 2, 64, dtype=f16), torch.zeros(10, 1, 64, dtype=f16)
+    cu = torch.tensor([0, 10], dtype=torch.int32)
+    with pytest.raises(ValueError, match="lse must have shape"):
+        sa.sa_attn_fwd_varlen(qp, kp, kp, cu, cu, 10, 10, lse=torch.empty(1, 2, 10))
+    kc = torch.zeros(2, 128, 1, 64, dtype=f16)
+    table, seqk = torch.zeros(1, 2, dtype=torch.int32), torch.tensor([10], dtype=torch.int32)
+    with pytest.raises(ValueError, match="out must have shape"):
+        sa.sa_attn_fwd_paged(qp, kc, kc, cu, table, seqk, 10, out=torch.empty(9, 2, 64, dtype=f16))
+    q8, k8 = torch.zeros(1, 8, 2, 128, dtype=u8), torch.zeros(1, 8, 1, 128, dtype=u8)
+    with pytest.raises(ValueError, match="out must have shape"):
+        sa.sa_attn_fwd_fp8(q8, k8, k8, 1.0, 1.0, 1.0, out=torch.empty(1, 8, 2, 64, dtype=torch.bfloat16))
+    with pytest.raises(ValueError, match="lse must have shape"):
+        sa.sa_attn_fwd_block_sparse_fp8(q8, k8, k8, mask, 1.0, 1.0, 1.0, lse=torch.empty(1, 2, 9))
+    o, lse = torch.zeros_like(q), torch.zeros(1, 2, 8)
+    with pytest.raises(ValueError, match="workspace: on meta"):
+        sa.sa_attn_bwd(q, k, k, o, lse, o, workspace=torch.empty(4096, dtype=u8, device="meta"))
+    qd, kd = torch.zeros(2, 2, 64, dtype=f16), torch.zeros(2, 64, 1, 64, dtype=f16)
+    with pytest.raises(ValueError, match="out must have shape"):
+        sa.sa_attn_decode(qd, kd, kd, out=torch.empty(2, 2, 32, dtype=f16))
+    with pytest.raises(ValueError, match="lse must have shape"):
+        sa.sa_attn_decode(qd, kd, kd, lse=torch.empty(2, 3))
+    with pytest.raises(ValueError, match="workspace: on meta"):
+        sa.sa_attn_decode(qd, kd, kd, workspace=torch.empty(1 << 16, dtype=u8, device="meta"))
+    table2, seq2 = torch.zeros(2, 1, dtype=torch.int32), torch.tensor([10, 10], dtype=torch.int32)
+    with pytest.raises(ValueError, match="lse must have shape"):
+        sa.sa_attn_decode_paged(qd, kc, kc, table2, seq2, lse=torch.empty(2))
