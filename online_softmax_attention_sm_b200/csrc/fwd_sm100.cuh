@@ -79,6 +79,11 @@ constexpr int kWarpMma = 0;
 constexpr int kWarpLoad = 1;
 
 constexpr float kRescaleThresh = 8.0f;   // log2 units: the reference moves past this
+// FP8 weights: p = 2^(x - m_ref + kFp8Offset), so a row's largest weights sit near the top of
+// e4m3's range instead of at 1 (weights below 2^-10 of the top round to zero, and a long row
+// can hold many of them); the reference then moves once the max passes it by kFp8Thresh,
+// which keeps p <= 2^8.5 < 448.  O / l is unchanged, the LSE takes kFp8Offset off.
+constexpr float kFp8Offset = 8.0f, kFp8Thresh = 0.5f;
 constexpr int kPolyEvery = 4;            // full tiles: one exponential pair in kPolyEvery on the FMA pipe (0: none)
 
 struct FwdParams {
@@ -507,8 +512,8 @@ __device__ __forceinline__ void fwd_mma(const FwdParams& p, const FwdSmem<D, FP8
         const uint32_t k_addr = sRing_addr + (kpos % Cfg::STAGES) * Cfg::TILE_BYTES;
         bool k_ready = false;
         for (int t = 0; t < 2; ++t) {
-          if (!SPARSE && j >= x.nkv[t]) continue;
-          if (act(t, j)) {
+          const bool live = SPARSE || j < x.nkv[t];
+          if (live && act(t, j)) {
             // ---- O_t += P_t V_j: keys 0-95 as soon as their P is written, then 96-127
             ok = mbar_wait_warp(&sm.p_part[t], (t ? pv1 : pv0) & 1, sm.abort_flag, 17);
             if (!ok) break;
@@ -533,8 +538,10 @@ __device__ __forceinline__ void fwd_mma(const FwdParams& p, const FwdSmem<D, FP8
             if (last) mma_commit_warp(&sm.o_done[t]);   // O_t complete for the epilogue
             if (t) ++pv1; else ++pv0;
           }
+          // V_j's last reader is in the pipe: release its slot ahead of the second S
+          if (t == 1) mma_commit_warp(&sm.kv_empty[vpos % Cfg::STAGES]);
           // ---- S_t = Q_t K_{j+1}^T
-          if (act(t, j + 1)) {
+          if (live && act(t, j + 1)) {
             if (!k_ready) {
               ok = mbar_wait_warp(&sm.kv_full[kpos % Cfg::STAGES], (kpos / Cfg::STAGES) & 1, sm.abort_flag, 10);
               if (!ok) break;
@@ -551,7 +558,6 @@ __device__ __forceinline__ void fwd_mma(const FwdParams& p, const FwdSmem<D, FP8
           }
         }
         if (!ok) break;
-        mma_commit_warp(&sm.kv_empty[vpos % Cfg::STAGES]);
         if (j + 1 < x.nkv_max) {
           if (!k_ready) {
             // (cannot happen: the Q tile with the most K/V tiles needs K(j+1))
@@ -715,10 +721,10 @@ __device__ __forceinline__ void sum_f2x2(const f32x2 (&v)[2], float& acc) {
 // kRescaleThresh, rescaling both sums and (after the first tile) the O_t row by
 // 2^(m_ref - m_tile).  O_t holds P V up to the previous tile, complete: the commit that
 // signalled this tile's S covers every earlier MMA.
-template <int D>
+template <int D, bool FP8>
 __device__ __forceinline__ void move_reference(const float m_tile, const bool first, float& m_ref,
                                                float& l_sum, float& l_lse, const uint32_t o_addr) {
-  const bool need = m_tile > m_ref + kRescaleThresh;
+  const bool need = m_tile > m_ref + (FP8 ? kFp8Thresh : kRescaleThresh);
   float alpha = 1.f;
   if (need) {
     alpha = ex2(m_ref - m_tile);       // 0 when m_ref == -inf
@@ -758,9 +764,10 @@ __device__ __forceinline__ void softmax_tile_full(const uint32_t s_addr, const u
     chunk_max(v2, mx);
     chunk_max(v3, mx);
   }
-  move_reference<D>(max_of8(mx) * c2, first, m_ref, l_sum, l_lse, o_addr);
+  move_reference<D, FP8>(max_of8(mx) * c2, first, m_ref, l_sum, l_lse, o_addr);
   const float m_use = (m_ref == -INFINITY) ? 0.f : m_ref;
-  const f32x2 scale2 = pack_f2(c2, c2), negm2 = pack_f2(-m_use, -m_use);
+  const float nm = FP8 ? kFp8Offset - m_use : -m_use;
+  const f32x2 scale2 = pack_f2(c2, c2), negm2 = pack_f2(nm, nm);
   f32x2 rs2[2] = {0ull, 0ull}, rse2[2] = {0ull, 0ull};
   uint32_t v2[32], v3[32];
   tmem_ld32(s_addr + 64, v2);
@@ -800,9 +807,10 @@ __device__ __forceinline__ void softmax_tile_masked(const uint32_t s_addr, const
       v[c][i] = __float_as_uint((c * 32 + i < kl) ? __uint_as_float(v[c][i]) * c2 : -INFINITY);
     chunk_max(v[c], mx);
   }
-  move_reference<D>(max_of8(mx), first, m_ref, l_sum, l_lse, o_addr);
+  move_reference<D, FP8>(max_of8(mx), first, m_ref, l_sum, l_lse, o_addr);
   const float m_use = (m_ref == -INFINITY) ? 0.f : m_ref;
-  const f32x2 scale2 = pack_f2(1.f, 1.f), negm2 = pack_f2(-m_use, -m_use);
+  const float nm = FP8 ? kFp8Offset - m_use : -m_use;
+  const f32x2 scale2 = pack_f2(1.f, 1.f), negm2 = pack_f2(nm, nm);
   f32x2 rs2[2] = {0ull, 0ull}, rse2[2] = {0ull, 0ull};
 #pragma unroll
   for (int c = 0; c < 4; ++c) {
@@ -914,7 +922,8 @@ __device__ __forceinline__ void fwd_softmax(const FwdParams& p, const FwdSmem<D,
       }
     }
     if (store && p.lse) {
-      float lse = l_lse > 0.f ? (m_ref + __log2f(l_lse)) * 0.69314718055994531f : -INFINITY;
+      float lse = l_lse > 0.f ? ((FP8 ? m_ref - kFp8Offset : m_ref) + __log2f(l_lse)) * 0.69314718055994531f
+                              : -INFINITY;
       p.lse[((size_t)x.mb * p.Hq + x.h) * p.Sq + x.qbase + row] = lse;
     }
     tc_fence_before();

@@ -717,3 +717,61 @@ def test_paged_prefill_lengths_clamp_and_empty():
     np.testing.assert_allclose(O[:2], Od[0], atol=TOL)
     np.testing.assert_allclose(L[:, :2], Ld[0], atol=TOL)
     assert np.all(O[2:] == 0) and np.all(np.isneginf(L[:, 2:]))           # no keys
+
+
+def test_e4m3_quantisation_round_trip_fixes_the_descale_direction():
+    # the input recipe's per-tensor quantisation, then decode_e4m3(codes) * descale: every value
+    # comes back within half an e4m3 step (2^-4 relative in the normal range, 2^-10 * descale
+    # below it); dividing by the descale instead, or forgetting it, misses by orders of magnitude
+    import torch
+    from oracle import decode_e4m3
+    from online_softmax_attention_sm_b200.inputs import quantize_e4m3
+    x = torch.randn(4096, generator=torch.Generator().manual_seed(5), dtype=torch.float32) * 3.0
+    codes, d = quantize_e4m3(x)
+    back = decode_e4m3(codes.numpy()) * d
+    xs = x.double().numpy()
+    allowed = np.maximum(2.0 ** -4 * np.abs(xs), 2.0 ** -10 * d)
+    assert np.all(np.abs(back - xs) <= allowed * (1 + 1e-12))
+    assert np.abs(back).max() == pytest.approx(np.abs(xs).max(), rel=1e-6)   # amax maps to 448 exactly
+
+
+def test_attention_fp8_closed_forms_fix_each_descale():
+    from oracle import attention_fp8, decode_e4m3
+    rng = np.random.default_rng(11)
+    qd, kd, vd, scale = 0.03, 0.2, 1.7, 0.8
+    k8 = rng.integers(0x20, 0x60, size=(1, 6, 1, 4), dtype=np.uint8)
+    v8 = rng.integers(0x20, 0x60, size=(1, 6, 1, 4), dtype=np.uint8)
+    vals = (decode_e4m3(v8) * vd)[0, :, 0]                       # V as the caller means it
+    # Q = 0 (code 0): uniform weights, O = the mean of the dequantised V over the visible keys
+    q0 = np.zeros((1, 6, 2, 4), dtype=np.uint8)
+    O, L = attention_fp8(q0, k8, v8, qd, kd, vd, scale, causal=True)
+    for i in range(6):
+        np.testing.assert_allclose(O[0, i, 1], vals[: i + 1].mean(axis=0), atol=1e-12)
+        assert L[0, 1, i] == pytest.approx(math.log(i + 1), abs=1e-12)
+    # a single key: O = its V row, LSE = scale * (q qd) . (k kd), summed by hand
+    q8 = rng.integers(0x20, 0x60, size=(1, 3, 1, 4), dtype=np.uint8)
+    O, L = attention_fp8(q8, k8[:, :1], v8[:, :1], qd, kd, vd, scale, causal=False)
+    qv, kv = decode_e4m3(q8)[0, :, 0], decode_e4m3(k8)[0, 0, 0]
+    for i in range(3):
+        dot = sum(float(qv[i, d]) * qd * float(kv[d]) * kd for d in range(4))
+        assert L[0, 0, i] == pytest.approx(scale * dot, abs=1e-12)
+        np.testing.assert_allclose(O[0, i, 0], vals[0], atol=1e-12)
+
+
+def test_attention_fp8_approximates_attention_of_the_unquantised_inputs():
+    # quantise float inputs with the recipe, run the FP8 oracle, compare with attention of the
+    # original floats: close (quantisation error only), which fails if any descale is applied
+    # the wrong way round or to the wrong tensor
+    import torch
+    from oracle import attention_fp8
+    from online_softmax_attention_sm_b200.inputs import make_qkv_fp8, make_qkv
+    args = (1, 40, 40, 2, 1, 16)
+    q8, k8, v8, qd, kd, vd = make_qkv_fp8(*args, seed=9, input_scale=0.7)
+    q, k, v = (t.double().numpy() for t in make_qkv(*args, "fp32", 9, 0.7))
+    assert not (qd == kd or kd == vd or qd == vd)
+    O, L = attention_fp8(q8.numpy(), k8.numpy(), v8.numpy(), qd, kd, vd, 0.25, True)
+    Oe, Le = attention(q, k, v, 0.25, True)
+    assert np.abs(O - Oe).max() < 0.1 and np.abs(L - Le).max() < 0.1
+    for wrong in ((1 / qd, kd, vd), (qd, kd, 1 / vd), (vd, kd, qd), (qd, vd, kd)):
+        Ow, Lw = attention_fp8(q8.numpy(), k8.numpy(), v8.numpy(), *wrong, 0.25, True)
+        assert np.abs(Ow - Oe).max() > 0.1 or np.abs(Lw - Le).max() > 0.1
