@@ -7,7 +7,13 @@ One step = one pass of the whole hot path over one batch of synthetic input:
   * decode: the 32768-token GQA split-KV decode (fp16, B=4, Hq=14, Hkv=2, D=64),
     sa_attn_decode -> split-KV kernel + combine kernel (programmatic dependent launch).
 value = prefill FLOPs (4*B*Hq*Sq*Sk*D/2, causal) per second of whole step, TFLOP/s.
-The decode's KV bandwidth is reported beside it ("decode"), timed with its own events.
+The decode's KV bandwidth is reported beside it ("decode"), timed with its own events
+against a plain cold read of the same bytes ("floor"), and the other workloads -- the
+128-, 2048- and 4096-token forwards, packed / paged / block-sparse / FP8 prefill and the
+backward -- each as a leg of its own with its own roofline fraction.
+
+stdout: one compact JSON line (the figures); stderr: one JSON line with the same legs
+and their descriptions (kernels, layouts, protocols).
 
 Multi-GPU (torchrun): every rank runs its own independent copy of the workload (the
 work units -- batches and heads -- are independent, so nothing is exchanged); value is
@@ -192,6 +198,10 @@ def run_reference(args):
 
 
 # ------------------------------------------------------------------ our arm
+def mean(xs):
+    return sum(xs) / len(xs)
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -201,8 +211,8 @@ def main():
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--only", default="all",
-                    choices=["all", "prefill", "decode", "varlen", "sparse", "backward", "fp8"],
-                    help="profiling aid: run only one half of the step (the JSON line is then partial)")
+                    choices=["all", "prefill", "decode", "small", "varlen", "sparse", "backward", "fp8"],
+                    help="profiling aid: run only one part (the JSON line is then partial)")
     ap.add_argument("--prefill-seq", type=int, default=0,
                     help="profiling aid: shorter prefill sequence (same heads, dtype, sinks)")
     args = ap.parse_args()
@@ -220,7 +230,7 @@ def main():
                                                    sa_attn_fwd_block_sparse, sa_attn_fwd_block_sparse_workspace_size,
                                                    sa_attn_bwd, sa_attn_bwd_workspace_size, sa_attn_fwd_fp8,
                                                    sa_attn_fwd_block_sparse_fp8, sa_attn_fwd_paged,
-                                                   sa_attn_fwd_varlen, sa_check_status)
+                                                   sa_attn_fwd_varlen, sa_check_status, sa_diag_read_floor)
     from online_softmax_attention_sm_b200.dist import aggregate_throughput, max_over_ranks, rank_seed
     from online_softmax_attention_sm_b200.inputs import (make_dout, make_qkv, make_qkv_fp8, make_workload_inputs,
                                                          stem_block_mask)
@@ -239,11 +249,7 @@ def main():
         import dataclasses
         wp = dataclasses.replace(wp, name=f"{wp.name}_seq{args.prefill_seq}", Sq=args.prefill_seq,
                                  Sk=args.prefill_seq)
-    run_pre, run_dec = args.only in ("all", "prefill"), args.only in ("all", "decode")
-    run_var = args.only in ("all", "varlen")
-    run_sparse = args.only in ("all", "sparse")
-    run_bwd = args.only in ("all", "backward")
-    run_fp8 = args.only in ("all", "fp8")
+    run = {k: args.only in ("all", k) for k in ("prefill", "decode", "small", "varlen", "sparse", "backward", "fp8")}
     q_h, k_h, v_h = make_workload_inputs(wp, seed=rank_seed(wp.seed, rank))
     dq_h, dk_h, dv_h = make_workload_inputs(wd, seed=rank_seed(wd.seed, rank))
     q, k, v = q_h.to(dev), k_h.to(dev), v_h.to(dev)
@@ -256,15 +262,20 @@ def main():
                      device=dev)
     stream = torch.cuda.current_stream(dev)
 
+    def decode_call(qq, kk, vv, oo, ll, wsp):
+        return sa_attn_decode(qq, kk, vv, scale=wd.scale, workspace=wsp, out=oo, lse=ll, stream=stream)
+
+    launches_per_decode = 2                  # split kernel + combine
+
     def step(ev=None):
         if ev:
             ev[0].record(stream)
-        if run_pre:
+        if run["prefill"]:
             sa_attn_fwd(q, k, v, causal=True, scale=wp.scale, out=o, lse=lse, stream=stream)
         if ev:
             ev[1].record(stream)
-        if run_dec:
-            sa_attn_decode(dq, dk, dv, scale=wd.scale, workspace=ws, out=do, lse=dlse, stream=stream)
+        if run["decode"]:
+            decode_call(dq, dk, dv, do, dlse, ws)
         if ev:
             ev[2].record(stream)
 
@@ -291,27 +302,40 @@ def main():
     pre_ms = [e[0].elapsed_time(e[1]) for e in evs]
     dec_ms = [e[1].elapsed_time(e[2]) for e in evs]
 
-    # decode alone with a cold L2: between iterations, outside the events, READ a buffer of
-    # 4x the L2 size (a read leaves clean lines; a write scrub would make the decode pay
-    # for writing back up to an L2 of dirty lines)
+    # Everything below is timed per launch with CUDA events on `stream`.  "cold": before each
+    # iteration, outside the events, READ a buffer of 4x the L2 size (a read leaves clean
+    # lines; a write scrub would make the timed launch pay for writing back an L2 of dirty
+    # lines).  Used for every leg whose inputs fit in the L2.
     l2 = torch.cuda.get_device_properties(dev).L2_cache_size
     scrub = torch.ones(4 * l2 // 4, dtype=torch.float32, device=dev)
-    cold = []
-    for i in range(args.warmup + args.steps if run_dec else 0):
-        scrub.sum()
-        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        e0.record(stream)
-        sa_attn_decode(dq, dk, dv, scale=wd.scale, workspace=ws, out=do, lse=dlse, stream=stream)
-        e1.record(stream)
-        if i >= args.warmup:
-            cold.append((e0, e1))
-    torch.cuda.synchronize(dev)
-    cold_ms = [a.elapsed_time(b) for a, b in cold] or [float("nan")]
 
-    # the same decode over a paged cache: the K/V cut into 64-token pages, the pages
-    # shuffled (a fixed permutation), every sequence at full length; same cold-L2 protocol
-    paged_ms = [float("nan")]
-    if run_dec:
+    def timed(call, cold):
+        evs = []
+        for i in range(args.warmup + args.steps):
+            if cold:
+                scrub.sum()
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            call()
+            e1.record(stream)
+            if i >= args.warmup:
+                evs.append((e0, e1))
+        torch.cuda.synchronize(dev)
+        sa_check_status(stream)
+        return mean([a.elapsed_time(b) for a, b in evs])
+
+    nan = float("nan")
+    res = {}                 # leg -> mean ms on this rank
+
+    # ---- decode alone, cold; the floor (a plain read of the same K/V bytes, both ways); the
+    # paged layout, the single-kernel decode, and batch 1
+    if run["decode"]:
+        res["decode"] = timed(lambda: decode_call(dq, dk, dv, do, dlse, ws), True)
+        sink = torch.zeros(1, dtype=torch.int32, device=dev)
+        kv = torch.cat([dk.view(-1), dv.view(-1)])        # the decode's 64 MiB, one buffer
+        res["floor_ld"] = timed(lambda: sa_diag_read_floor(kv, sink, 0, stream=stream), True)
+        res["floor_bulk"] = timed(lambda: sa_diag_read_floor(kv, sink, 1, stream=stream), True)
+        del kv
         ps = 64
         nb = wd.Sk // ps
         perm = torch.randperm(wd.B * nb, generator=torch.Generator().manual_seed(wd.seed)).to(dev)
@@ -323,74 +347,45 @@ def main():
         seqlens = torch.full((wd.B,), wd.Sk, dtype=torch.int32, device=dev)
         pws = torch.empty(max(16, sa_attn_decode_paged_workspace_size(wd.B, wd.Hq, wd.Hkv, wd.D, ps, nb)),
                           dtype=torch.uint8, device=dev)
-        pev = []
-        for i in range(args.warmup + args.steps):
-            scrub.sum()
-            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-            e0.record(stream)
-            sa_attn_decode_paged(dq, kc, vc, table, seqlens, scale=wd.scale, workspace=pws, out=do, lse=dlse,
-                                 stream=stream)
-            e1.record(stream)
-            if i >= args.warmup:
-                pev.append((e0, e1))
-        torch.cuda.synchronize(dev)
-        sa_check_status(stream)
-        paged_ms = [a.elapsed_time(b) for a, b in pev]
+        res["decode_paged"] = timed(lambda: sa_attn_decode_paged(dq, kc, vc, table, seqlens, scale=wd.scale,
+                                                                 workspace=pws, out=do, lse=dlse, stream=stream),
+                                    True)
         del kc, vc
-
-    # the single-kernel decode (each tile's last split merges; no combine launch) on the same
-    # workload, and both decodes at batch 1 (the pages' small-batch case); same protocol
-    def cold_loop(call):
-        evs = []
-        for i in range(args.warmup + args.steps):
-            scrub.sum()
-            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-            e0.record(stream)
-            call()
-            e1.record(stream)
-            if i >= args.warmup:
-                evs.append((e0, e1))
-        torch.cuda.synchronize(dev)
-        sa_check_status(stream)
-        return [a.elapsed_time(b) for a, b in evs]
-
-    single_ms = b1_two_ms = b1_single_ms = [float("nan")]
-    if run_dec:
-        single_ms = cold_loop(lambda: sa_attn_decode_single(dq, dk, dv, scale=wd.scale, workspace=ws, out=do,
-                                                             lse=dlse, stream=stream))
+        res["decode_single"] = timed(lambda: sa_attn_decode_single(dq, dk, dv, scale=wd.scale, workspace=ws, out=do,
+                                                                   lse=dlse, stream=stream), True)
         dq1, dk1, dv1, do1, dl1 = dq[:1], dk[:1], dv[:1], do[:1], dlse[:1]
         ws1 = torch.empty(max(16, sa_attn_decode_workspace_size(1, wd.Sk, wd.Hq, wd.Hkv, wd.D)), dtype=torch.uint8,
                           device=dev)
-        b1_two_ms = cold_loop(lambda: sa_attn_decode(dq1, dk1, dv1, scale=wd.scale, workspace=ws1, out=do1, lse=dl1,
-                                                     stream=stream))
-        b1_single_ms = cold_loop(lambda: sa_attn_decode_single(dq1, dk1, dv1, scale=wd.scale, workspace=ws1,
-                                                               out=do1, lse=dl1, stream=stream))
+        res["decode_b1"] = timed(lambda: decode_call(dq1, dk1, dv1, do1, dl1, ws1), True)
+        res["decode_b1_single"] = timed(lambda: sa_attn_decode_single(dq1, dk1, dv1, scale=wd.scale, workspace=ws1,
+                                                                      out=do1, lse=dl1, stream=stream), True)
         del ws1
-    del scrub
 
-    # packed variable-length prefill: the long prefill's heads over 16 sequences of 32768
-    # tokens in all (inputs and outputs exceed the L2)
-    var_ms = pg_ms = [float("nan")]
+    # ---- the small forward workloads (inputs and outputs fit in the L2: cold protocol)
+    small = {}
+    if run["small"]:
+        for name in ("mha_s128_d64_fp16", "mha_causal_s2048_d64_fp16", "mha_s4096_d128_bf16",
+                     "mha_causal_s4096_d128_bf16"):
+            w = WORKLOADS[name]
+            sq, sk, sv = (t.to(dev) for t in make_workload_inputs(w, seed=rank_seed(w.seed, rank)))
+            so = torch.empty_like(sq)
+            sl = torch.empty((w.B, w.Hq, w.Sq), dtype=torch.float32, device=dev)
+            res[name] = timed(lambda: sa_attn_fwd(sq, sk, sv, causal=w.causal, scale=w.scale, out=so, lse=sl,
+                                                  stream=stream), True)
+            small[name] = w
+            del sq, sk, sv, so, sl
+
+    # ---- packed variable-length prefill: the long prefill's heads over 16 sequences of 32768
+    # tokens in all (inputs and outputs exceed the L2), and the same mix over a paged cache
     lens = wv.lengths
-    if run_var:
+    if run["varlen"]:
         vq, vk, vv = (t[0].to(dev) for t in make_qkv(1, wv.Sq, wv.Sk, wv.Hq, wv.Hkv, wv.D, wv.dtype,
                                                        seed=rank_seed(wv.seed, rank)))
         cu = torch.tensor(np.concatenate([[0], np.cumsum(lens)]), dtype=torch.int32, device=dev)
         vo = torch.empty_like(vq)
         vlse = torch.empty((wv.Hq, wv.Sq), dtype=torch.float32, device=dev)
-        vev = []
-        for i in range(args.warmup + args.steps):
-            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-            e0.record(stream)
-            sa_attn_fwd_varlen(vq, vk, vv, cu, cu, max(lens), max(lens), causal=wv.causal, scale=wv.scale,
-                               out=vo, lse=vlse, stream=stream)
-            e1.record(stream)
-            if i >= args.warmup:
-                vev.append((e0, e1))
-        torch.cuda.synchronize(dev)
-        sa_check_status(stream)
-        var_ms = [a.elapsed_time(b) for a, b in vev]
-        # the same mix with its keys in a paged cache: 128-key pages in a fixed shuffled order
+        res["varlen"] = timed(lambda: sa_attn_fwd_varlen(vq, vk, vv, cu, cu, max(lens), max(lens), causal=wv.causal,
+                                                         scale=wv.scale, out=vo, lse=vlse, stream=stream), False)
         nbs = [-(-n // 128) for n in lens]
         mb = max(nbs)
         perm = torch.randperm(len(lens) * mb, generator=torch.Generator().manual_seed(wv.seed)).tolist()
@@ -407,113 +402,72 @@ def main():
             k0 += n
         table = table.to(dev)
         seqk = torch.tensor(lens, dtype=torch.int32, device=dev)
-        pgev = []
-        for i in range(args.warmup + args.steps):
-            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-            e0.record(stream)
-            sa_attn_fwd_paged(vq, kc, vc, cu, table, seqk, max(lens), causal=wv.causal, scale=wv.scale, out=vo,
-                              lse=vlse, stream=stream)
-            e1.record(stream)
-            if i >= args.warmup:
-                pgev.append((e0, e1))
-        torch.cuda.synchronize(dev)
-        sa_check_status(stream)
-        pg_ms = [a.elapsed_time(b) for a, b in pgev]
+        res["varlen_paged"] = timed(lambda: sa_attn_fwd_paged(vq, kc, vc, cu, table, seqk, max(lens),
+                                                              causal=wv.causal, scale=wv.scale, out=vo, lse=vlse,
+                                                              stream=stream), False)
         del vq, vk, vv, vo, vlse, kc, vc
 
-    # block-sparse prefill: the prefill workload's tensors under a Stem-shaped block mask
-    # (4 sink blocks, 4 window blocks, 10 % of the blocks between drawn at random); one API
-    # call = the list-building kernel + the block-sparse forward
-    sp_ms, sp_flops = [float("nan")], float("nan")
-    if run_sparse:
+    # ---- block-sparse prefill: the prefill workload's tensors under a Stem-shaped block mask
+    # (4 sink, 4 window blocks, 10 % of the blocks between); one API call = the list kernel +
+    # the block-sparse forward
+    sp_flops = nan
+    bmask = None
+    if run["sparse"] or run["fp8"]:
         bmask = stem_block_mask(wp.B, wp.Hq, wp.Sq, wp.Sk, wp.causal, seed=wp.seed + 4)
         sp_flops = block_sparse_flops(bmask.numpy(), wp.Sq, wp.Sk, wp.D, wp.causal)
         bmask = bmask.to(dev)
         sws = torch.empty(max(16, sa_attn_fwd_block_sparse_workspace_size(wp.B, wp.Sq, wp.Sk, wp.Hq)),
                           dtype=torch.uint8, device=dev)
-        sev = []
-        for i in range(args.warmup + args.steps):
-            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-            e0.record(stream)
-            sa_attn_fwd_block_sparse(q, k, v, bmask, causal=wp.causal, scale=wp.scale, workspace=sws, out=o,
-                                     lse=lse, stream=stream)
-            e1.record(stream)
-            if i >= args.warmup:
-                sev.append((e0, e1))
-        torch.cuda.synchronize(dev)
-        sa_check_status(stream)
-        sp_ms = [a.elapsed_time(b) for a, b in sev]
-        del bmask, sws
+    if run["sparse"]:
+        res["block_sparse"] = timed(lambda: sa_attn_fwd_block_sparse(q, k, v, bmask, causal=wp.causal, scale=wp.scale,
+                                                                     workspace=sws, out=o, lse=lse, stream=stream),
+                                    False)
 
-    # backward of the prefill workload: dQ, dK, dV for a seeded dO (three kernels: prep,
-    # dK/dV, dQ); the forward's O and LSE are made once, outside the events
-    bwd_ms = [float("nan")]
-    if run_bwd:
+    # ---- backward of the prefill workload: dQ, dK, dV for a seeded dO (prep, dK/dV, dQ); the
+    # forward's O and LSE are made once, outside the events
+    if run["backward"]:
         dout = make_dout(wp.B, wp.Sq, wp.Hq, wp.D, wp.dtype, seed=rank_seed(wp.seed, rank)).to(dev)
         sa_attn_fwd(q, k, v, causal=wp.causal, scale=wp.scale, out=o, lse=lse, stream=stream)
         gq, gk, gv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
         bws = torch.empty(max(16, sa_attn_bwd_workspace_size(wp.B, wp.Sq, wp.Hq)), dtype=torch.uint8, device=dev)
-        bev = []
-        for i in range(args.warmup + args.steps):
-            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-            e0.record(stream)
-            sa_attn_bwd(q, k, v, o, lse, dout, causal=wp.causal, scale=wp.scale, workspace=bws, dq=gq, dk=gk,
-                        dv=gv, stream=stream)
-            e1.record(stream)
-            if i >= args.warmup:
-                bev.append((e0, e1))
-        torch.cuda.synchronize(dev)
-        sa_check_status(stream)
-        bwd_ms = [a.elapsed_time(b) for a, b in bev]
+        res["backward"] = timed(lambda: sa_attn_bwd(q, k, v, o, lse, dout, causal=wp.causal, scale=wp.scale,
+                                                    workspace=bws, dq=gq, dk=gk, dv=gv, stream=stream), False)
         del dout, gq, gk, gv, bws
 
-    # FP8 forward: the prefill workload's draws quantised to e4m3 per tensor (same seed)
-    fp8_ms = sp8_ms = [float("nan")]
-    sp8_flops = float("nan")
-    if run_fp8:
+    # ---- FP8 forward: the prefill workload's draws quantised to e4m3 per tensor (same seed);
+    # and block-sparse over the same e4m3 tensors.  Accuracy on the GPU: the 16-bit forward of
+    # the same dequantised values (e4m3 codes are exact in bf16; the descales go into the scale
+    # and onto O) stands in for the exact result -- that forward is itself checked against the
+    # fp64 oracle in the tests.
+    fp8_acc = None
+    if run["fp8"]:
         q8, k8, v8, qd8, kd8, vd8 = make_qkv_fp8(wp.B, wp.Sq, wp.Sk, wp.Hq, wp.Hkv, wp.D, seed=rank_seed(wp.seed, rank),
                                                  input_scale=wp.input_scale, k_sink_rows=wp.k_sink_rows,
                                                  k_sink_factor=wp.k_sink_factor)
         q8, k8, v8 = q8.to(dev), k8.to(dev), v8.to(dev)
         o8 = torch.empty((wp.B, wp.Sq, wp.Hq, wp.D), dtype=torch.bfloat16, device=dev)
-        fev = []
-        for i in range(args.warmup + args.steps):
-            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-            e0.record(stream)
-            sa_attn_fwd_fp8(q8, k8, v8, qd8, kd8, vd8, causal=wp.causal, scale=wp.scale, out=o8, lse=lse,
-                            stream=stream)
-            e1.record(stream)
-            if i >= args.warmup:
-                fev.append((e0, e1))
-        torch.cuda.synchronize(dev)
-        sa_check_status(stream)
-        fp8_ms = [a.elapsed_time(b) for a, b in fev]
-        # and block-sparse over the same e4m3 tensors (the Stem-shaped mask of the bf16 leg)
-        bmask8 = stem_block_mask(wp.B, wp.Hq, wp.Sq, wp.Sk, wp.causal, seed=wp.seed + 4)
-        sp8_flops = block_sparse_flops(bmask8.numpy(), wp.Sq, wp.Sk, wp.D, wp.causal)
-        bmask8 = bmask8.to(dev)
-        sws8 = torch.empty(max(16, sa_attn_fwd_block_sparse_workspace_size(wp.B, wp.Sq, wp.Sk, wp.Hq)),
-                           dtype=torch.uint8, device=dev)
-        fsev = []
-        for i in range(args.warmup + args.steps):
-            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-            e0.record(stream)
-            sa_attn_fwd_block_sparse_fp8(q8, k8, v8, bmask8, qd8, kd8, vd8, causal=wp.causal, scale=wp.scale,
-                                         workspace=sws8, out=o8, lse=lse, stream=stream)
-            e1.record(stream)
-            if i >= args.warmup:
-                fsev.append((e0, e1))
-        torch.cuda.synchronize(dev)
-        sa_check_status(stream)
-        sp8_ms = [a.elapsed_time(b) for a, b in fsev]
-        del q8, k8, v8, o8, bmask8, sws8
+        res["fp8"] = timed(lambda: sa_attn_fwd_fp8(q8, k8, v8, qd8, kd8, vd8, causal=wp.causal, scale=wp.scale,
+                                                   out=o8, lse=lse, stream=stream), False)
+        res["fp8_block_sparse"] = timed(lambda: sa_attn_fwd_block_sparse_fp8(
+            q8, k8, v8, bmask, qd8, kd8, vd8, causal=wp.causal, scale=wp.scale, workspace=sws, out=o8, lse=lse,
+            stream=stream), False)
+        sa_attn_fwd_fp8(q8, k8, v8, qd8, kd8, vd8, causal=wp.causal, scale=wp.scale, out=o8, lse=lse, stream=stream)
+        to16 = [t.view(torch.float8_e4m3fn).to(torch.bfloat16) for t in (q8, k8, v8)]
+        del q8, k8, v8
+        oref, _ = sa_attn_fwd(*to16, causal=wp.causal, scale=wp.scale * qd8 * kd8, return_lse=False, stream=stream)
+        del to16
+        diff = (o8.float() - oref.float() * vd8).abs()
+        fp8_acc = {"max_abs": float(diff.max()), "p999_abs": float(diff.view(-1)[::97].quantile(0.999))}
+        del o8, oref, diff
+    del scrub
+    if bmask is not None:
+        del bmask, sws
 
-    # e2e through the public API with host buffers: every step copies its inputs from pinned
-    # host memory and reads its outputs back.  Pipelined the way a serving loop runs it: three
-    # streams (host-to-device copies, compute, device-to-host copies) and two device buffer
-    # sets, so the copies of step i+1 and the read-back of step i-1 overlap the compute of
-    # step i; events keep a buffer set from being refilled before its step's compute and
-    # read-back are done.  The timed region spans the first copy to the last read-back.
+    # ---- e2e through the public API with host buffers: every step copies its inputs from
+    # pinned host memory and reads its outputs back, pipelined the way a serving loop runs it
+    # (copy-in / compute / copy-out streams over two device buffer sets; events keep a set from
+    # being refilled before its compute and read-back are done).  The timed region spans the
+    # first copy to the last read-back.
     e2e_ms = None
     h2d = sum(t.numel() * t.element_size() for t in (q_h, k_h, v_h, dq_h, dk_h, dv_h))
     d2h = sum(t.numel() * t.element_size() for t in (o, lse, do, dlse))
@@ -538,10 +492,10 @@ def main():
                 stream.wait_event(ev_in)
                 if i >= 2:
                     stream.wait_event(out_done[i - 2])         # set's outputs read back
-                if run_pre:
+                if run["prefill"]:
                     sa_attn_fwd(S[0], S[1], S[2], causal=True, scale=wp.scale, out=S[6], lse=S[7], stream=stream)
-                if run_dec:
-                    sa_attn_decode(S[3], S[4], S[5], scale=wd.scale, workspace=ws, out=S[8], lse=S[9], stream=stream)
+                if run["decode"]:
+                    decode_call(S[3], S[4], S[5], S[8], S[9], ws)
                 ev_c = torch.cuda.Event()
                 ev_c.record(stream)
                 comp_done.append(ev_c)
@@ -565,31 +519,21 @@ def main():
         sa_check_status(stream)
         del sets
 
+    # every rank reduces the same keys in the same order
     ms_step = max_over_ranks(ms_total / args.steps, dev)
-    pre_avg = max_over_ranks(sum(pre_ms) / len(pre_ms), dev)
-    dec_avg = max_over_ranks(sum(dec_ms) / len(dec_ms), dev)
-    cold_avg = max_over_ranks(sum(cold_ms) / len(cold_ms), dev)
-    paged_avg = max_over_ranks(sum(paged_ms) / len(paged_ms), dev)
-    single_avg = max_over_ranks(sum(single_ms) / len(single_ms), dev)
-    b1_two_avg = max_over_ranks(sum(b1_two_ms) / len(b1_two_ms), dev)
-    b1_single_avg = max_over_ranks(sum(b1_single_ms) / len(b1_single_ms), dev)
-    var_avg = max_over_ranks(sum(var_ms) / len(var_ms), dev)
-    pg_avg = max_over_ranks(sum(pg_ms) / len(pg_ms), dev)
-    sp_avg = max_over_ranks(sum(sp_ms) / len(sp_ms), dev)
-    bwd_avg = max_over_ranks(sum(bwd_ms) / len(bwd_ms), dev)
-    fp8_avg = max_over_ranks(sum(fp8_ms) / len(fp8_ms), dev)
-    sp8_avg = max_over_ranks(sum(sp8_ms) / len(sp8_ms), dev)
+    pre_avg = max_over_ranks(mean(pre_ms), dev)
+    dec_step = max_over_ranks(mean(dec_ms), dev)
+    for key in ("decode", "floor_ld", "floor_bulk", "decode_paged", "decode_single", "decode_b1", "decode_b1_single",
+                "mha_s128_d64_fp16", "mha_causal_s2048_d64_fp16", "mha_s4096_d128_bf16", "mha_causal_s4096_d128_bf16",
+                "varlen", "varlen_paged", "block_sparse", "backward", "fp8", "fp8_block_sparse"):
+        res[key] = max_over_ranks(res.get(key, nan), dev)
     e2e_ms = max_over_ranks(e2e_ms, dev) if e2e_ms is not None else None
 
     if rank == 0:
         peaks = load_peaks()
+        peak, hbm = peaks["bf16_tflops"], peaks["hbm_gbs"]
         value = aggregate_throughput(wp.flops, world, ms_step * 1e-3) / 1e12
         pre_tf = wp.flops / (pre_avg * 1e-3) / 1e12
-        # the timed loop is a fraction of a second at full clock, so the burst figure
-        # (cuBLAS timed alone) is the comparable -- and the stricter -- denominator
-        peak = peaks["bf16_tflops"]
-        dec_gbs_cold = wd.kv_bytes / (cold_avg * 1e-3) / 1e9
-        dec_gbs_step = wd.kv_bytes / (dec_avg * 1e-3) / 1e9 if run_dec else float("nan")
         traffic = None
         prof = os.path.join(ROOT, "profiles", "traffic.json")
         if os.path.exists(prof) and not args.prefill_seq:
@@ -597,81 +541,83 @@ def main():
             # only while the kernel is the one the counters were taken from
             if rec.get("kernel_source_sha256") == kernel_source_hash():
                 traffic = rec.get("bytes")
+
+        def r3(x):
+            return None if x is None or x != x else float(f"{x:.4g}")
+
+        def tf_leg(flops, ms, pk=peak):
+            tf = flops / (ms * 1e-3) / 1e12
+            return {"ms": r3(ms), "tflops": r3(tf), "frac": r3(tf / pk)}
+
+        def gb_leg(us):
+            gbs = wd.kv_bytes / (us * 1e-6) / 1e9
+            return {"us": r3(us), "gbs": r3(gbs), "frac": r3(gbs / hbm)}
+
+        dec_us = res["decode"] * 1e3
+        floor_us = min(res["floor_ld"], res["floor_bulk"]) * 1e3
+        legs = {
+            "backward": tf_leg(2.5 * wp.flops, res["backward"]),
+            "fp8": dict(tf_leg(wp.flops, res["fp8"], 2 * peak), acc=fp8_acc),
+            "fp8_block_sparse": tf_leg(sp_flops, res["fp8_block_sparse"], 2 * peak),
+            "block_sparse": tf_leg(sp_flops, res["block_sparse"]),
+            "varlen": tf_leg(wv.flops, res["varlen"]),
+            "varlen_paged": tf_leg(wv.flops, res["varlen_paged"]),
+            "c1_s128": {"us": r3(res["mha_s128_d64_fp16"] * 1e3),
+                        "tflops": r3(WORKLOADS["mha_s128_d64_fp16"].flops / (res["mha_s128_d64_fp16"] * 1e-3) / 1e12)},
+            "c3_s4096": tf_leg(WORKLOADS["mha_s4096_d128_bf16"].flops, res["mha_s4096_d128_bf16"]),
+            "c3_s4096_causal": tf_leg(WORKLOADS["mha_causal_s4096_d128_bf16"].flops, res["mha_causal_s4096_d128_bf16"]),
+            "c2_s2048_causal": tf_leg(WORKLOADS["mha_causal_s2048_d64_fp16"].flops, res["mha_causal_s2048_d64_fp16"]),
+            "decode": dict(gb_leg(dec_us), floor_us=r3(floor_us), floor_gbs=r3(wd.kv_bytes / (floor_us * 1e-6) / 1e9),
+                           over_floor_us=r3(dec_us - floor_us), paged_us=r3(res["decode_paged"] * 1e3),
+                           single_us=r3(res["decode_single"] * 1e3), b1_us=r3(res["decode_b1"] * 1e3),
+                           b1_single_us=r3(res["decode_b1_single"] * 1e3)),
+        }
         line = {
             "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_step,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
             "data": "synthetic",
-            "config": {"workload": f"{PREFILL} + {DECODE}",
-                       "prefill": {"B": wp.B, "Sq": wp.Sq, "Sk": wp.Sk, "Hq": wp.Hq, "Hkv": wp.Hkv, "D": wp.D,
-                                   "causal": True, "dtype": "bf16", "k_sink_rows": 4},
-                       "decode": {"B": wd.B, "Sk": wd.Sk, "Hq": wd.Hq, "Hkv": wd.Hkv, "D": wd.D, "dtype": "fp16"},
-                       "global_batch": wp.B * world, "seq_len": wp.Sq,
+            "config": {"workload": f"{PREFILL} + {DECODE}", "global_batch": wp.B * world, "seq_len": wp.Sq,
                        "parallelism": f"independent replicas x{world}" if world > 1 else "single GPU",
-                       "l2": "prefill inputs+outputs (640 MB) exceed L2; decode timed alone after reading 4xL2 of other data"},
+                       "l2": "step inputs exceed L2; legs whose inputs fit in L2 (decode, floor, c1-c3) timed cold "
+                             "after a 4xL2 read scrub"},
             "roofline": {"bound": "tensor", "kernel": "attn_fwd_sm100", "achieved": pre_tf, "peak": peak,
-                         "unit": "TFLOP/s", "frac": pre_tf / peak,
-                         "peak_source": f"{peaks['source']} bf16 cuBLAS burst (the timed loop is < 1 s)",
-                         "traffic": traffic},
-            "decode": {"value": dec_gbs_cold, "unit": "GB/s", "bound": "hbm", "peak": peaks["hbm_gbs"],
-                       "frac": dec_gbs_cold / peaks["hbm_gbs"], "us": cold_avg * 1e3, "l2": "cold (4xL2 read scrub)",
-                       "in_step_gbs": dec_gbs_step, "kernels": "attn_decode_split + attn_decode_combine (PDL)",
-                       "paged": {"value": wd.kv_bytes / (paged_avg * 1e-3) / 1e9, "unit": "GB/s",
-                                 "frac": wd.kv_bytes / (paged_avg * 1e-3) / 1e9 / peaks["hbm_gbs"],
-                                 "us": paged_avg * 1e3, "page_size": 64,
-                                 "layout": "the same K/V in shuffled 64-token pages, full-length sequences",
-                                 "l2": "cold (4xL2 read scrub)"},
-                       "single_kernel": {"us": single_avg * 1e3,
-                                         "value": wd.kv_bytes / (single_avg * 1e-3) / 1e9, "unit": "GB/s",
-                                         "frac": wd.kv_bytes / (single_avg * 1e-3) / 1e9 / peaks["hbm_gbs"],
-                                         "kernel": "attn_decode_split (last split of each tile merges)"},
-                       "batch1": {"two_kernel_us": b1_two_avg * 1e3, "single_kernel_us": b1_single_avg * 1e3,
-                                  "workload": "the decode workload's first sequence alone (B1, 32768 keys)"}},
-            "prefill_varlen": {"workload": VARLEN, "value": wv.flops / (var_avg * 1e-3) / 1e12,
-                               "unit": "TFLOP/s", "bound": "tensor", "peak": peak,
-                               "frac": wv.flops / (var_avg * 1e-3) / 1e12 / peak, "ms": var_avg,
-                               "sequences": len(lens), "lengths": f"{min(lens)}-{max(lens)}",
-                               "kernel": "attn_fwd_sm100 (dynamic unit order)",
-                               "paged": {"value": wv.flops / (pg_avg * 1e-3) / 1e12, "unit": "TFLOP/s",
-                                         "frac": wv.flops / (pg_avg * 1e-3) / 1e12 / peak, "ms": pg_avg,
-                                         "layout": "the same keys in shuffled 128-key pages (sa_attn_fwd_paged)"}},
-            "prefill_block_sparse": {"workload": f"{PREFILL} + Stem-shaped block mask (4 sink, 4 window, "
-                                                 "10 % of the blocks between)",
-                                     "value": sp_flops / (sp_avg * 1e-3) / 1e12, "unit": "TFLOP/s",
-                                     "bound": "tensor", "peak": peak,
-                                     "frac": sp_flops / (sp_avg * 1e-3) / 1e12 / peak, "ms": sp_avg,
-                                     "work_vs_dense_causal": sp_flops / wp.flops,
-                                     "kernels": "sparse_unit_lists + attn_fwd_sm100 (block-sparse instance)"},
-            "backward": {"workload": PREFILL, "value": 2.5 * wp.flops / (bwd_avg * 1e-3) / 1e12,
-                         "unit": "TFLOP/s", "bound": "tensor", "peak": peak,
-                         "frac": 2.5 * wp.flops / (bwd_avg * 1e-3) / 1e12 / peak, "ms": bwd_avg,
-                         "flops": "2.5 x the forward's (5 tile products against 2; the dQ kernel's "
-                                  "recomputed S and dP are not credited)",
-                         "kernels": "bwd_prep + attn_bwd_kv + attn_bwd_q"},
-            "prefill_fp8": {"workload": f"{PREFILL}, Q/K/V in e4m3 (per-tensor descale)",
-                            "value": wp.flops / (fp8_avg * 1e-3) / 1e12, "unit": "TFLOP/s", "bound": "tensor",
-                            "peak": 2 * peak, "peak_source": "measured bf16 burst x 2 (nominal fp8 : bf16)",
-                            "frac": wp.flops / (fp8_avg * 1e-3) / 1e12 / (2 * peak), "ms": fp8_avg,
-                            "kernel": "attn_fwd_sm100 (FP8 instance: kind::f8f6f4 QK and PV, e4m3 P)",
-                            "accuracy": "open: e4m3 weights below 2^-10 of the row reference round to zero; "
-                                        "on this workload's long sink-dominated rows a host simulation of that "
-                                        "rounding gives per-row max |O error| median 0.013, 90th pct 1.05",
-                            "block_sparse": {"value": sp8_flops / (sp8_avg * 1e-3) / 1e12, "unit": "TFLOP/s",
-                                             "frac": sp8_flops / (sp8_avg * 1e-3) / 1e12 / (2 * peak),
-                                             "ms": sp8_avg, "mask": "the bf16 block-sparse leg's Stem-shaped mask"}},
-            "prefill_ms": pre_avg,
-            "gpu_launches": (int(run_pre) + 2 * int(run_dec)) * args.steps,
+                         "unit": "TFLOP/s", "frac": pre_tf / peak, "ms": pre_avg,
+                         "peak_source": f"{peaks['source']} bf16 cuBLAS burst", "traffic": traffic},
+            "gpu_launches": (int(run["prefill"]) + launches_per_decode * int(run["decode"])) * args.steps,
             "clocks": clk.summary(),
         }
         if e2e_ms is not None:
             line["e2e"] = {"value": aggregate_throughput(wp.flops, world, e2e_ms * 1e-3) / 1e12, "unit": "TFLOP/s",
-                           "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms,
-                           "pipeline": "copy-in / compute / copy-out streams, two buffer sets"}
+                           "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms}
         if world == 1 and args.cpu_seconds > 0:
             f, el, desc = oracle_prefill_sample(wp, q_h, k_h, v_h, args.cpu_seconds)
             line["cpu_baseline"] = {"value": f / el / 1e12, "unit": "TFLOP/s", "cores": blas_threads(),
                                     "kind": "oracle", "sample": f"{desc}, {el:.1f} s"}
-        print(json.dumps(line), flush=True)
+        line["in_step_decode_us"] = r3(dec_step * 1e3)
+        line.update(legs)
+        print(json.dumps(line, separators=(",", ":")), flush=True)
+        details = {
+            "legs": {
+                "decode": f"{DECODE} alone, sa_attn_decode (split kernel + PDL combine), cold; GB/s of K+V read "
+                          "once vs MEASURED_PEAKS hbm_gbs; floor = sa_diag_read_floor of the same 64 MiB (best of "
+                          "128-bit loads and bulk copies), same protocol; paged = shuffled 64-token pages; single = "
+                          "sa_attn_decode_single; b1 = the first sequence alone",
+                "floor_ld_us": r3(res["floor_ld"] * 1e3), "floor_bulk_us": r3(res["floor_bulk"] * 1e3),
+                "c1_s128 / c2_s2048_causal / c3_s4096(_causal)": "mha_s128_d64_fp16, mha_causal_s2048_d64_fp16, "
+                          "mha_s4096_d128_bf16 (+ causal), sa_attn_fwd, cold; c1 is launch-bound",
+                "varlen": f"{VARLEN}: 16 packed sequences ({min(lens)}-{max(lens)} tokens), sa_attn_fwd_varlen; "
+                          "varlen_paged: the same keys in shuffled 128-key pages, sa_attn_fwd_paged",
+                "block_sparse": "prefill tensors + Stem-shaped block mask (4 sink, 4 window, 10 % between); FLOPs "
+                                f"per kept block ({sp_flops:.4g}); sparse_unit_lists + forward",
+                "backward": "sa_attn_bwd on the prefill workload, 2.5x the forward's FLOPs credited",
+                "fp8": "sa_attn_fwd_fp8 on the prefill draws in e4m3 (per-tensor descale), peak 2x the bf16 "
+                       "burst; acc = |O_fp8 - O_bf16 of the same dequantised values| (max; 99.9th percentile "
+                       "of every 97th element)",
+            },
+            "peaks": peaks,
+        }
+        print(json.dumps(details), file=sys.stderr, flush=True)
     if world > 1:
         dist.barrier()
         dist.destroy_process_group()

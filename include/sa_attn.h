@@ -40,6 +40,11 @@
  *   - Every device-side wait is bounded; if one expires the kernel records it in a device
  *     status word and returns early (outputs are then undefined).  sa_check_status()
  *     reports and clears that word.
+ *   - In-flight limits: every forward entry point (sa_attn_fwd and its packed, paged,
+ *     block-sparse and FP8 variants) may take its work units from counters in the
+ *     library's device image: at most 1024 such launches in flight per device (see
+ *     sa_attn_fwd).  sa_attn_decode_single: at most 16 calls in flight.  The other
+ *     entry points keep no state between calls beyond sa_attn_decode_noalloc's area.
  *   - D must be 64 or 128; dtype SA_FP16 or SA_BF16; Hq a positive multiple of Hkv.
  *   - B == 0, Sq == 0 or Hq == 0: SA_OK, nothing launched.  Sk == 0: O = 0, LSE = -inf.
  */
@@ -75,6 +80,13 @@ typedef enum {
  *   scale      : softmax scale, used as given (finite); callers usually pass 1/sqrt(D).
  *   dtype      : SA_FP16 or SA_BF16 for q, k, v and o.
  * Runs the persistent tcgen05 (tensor-memory) kernel.
+ * Concurrency: for shapes whose fixed work order would balance badly, the kernel takes its
+ * work units from a counter pair in the library's device image (1024 pairs, used in turn
+ * by successive launches and zeroed by each launch's end).  The packed, paged,
+ * block-sparse and FP8 forwards below always do.  At most 1024 such forward launches may
+ * be in flight on a device at once (on any streams or graphs); a launch that found its
+ * pair still in use by the launch 1024 before it would skip or repeat work units.  A CUDA
+ * graph keeps the pair it was captured with: replays of one graph must not overlap.
  */
 int sa_attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse,
                 int B, int Sq, int Sk, int Hq, int Hkv, int D, int causal,
@@ -160,8 +172,10 @@ int sa_attn_fwd_block_sparse_fp8(const void* q, const void* k, const void* v, vo
  * two-kernel prototype loses to launch and merge overhead at small batch).  Same arguments,
  * workspace and result as sa_attn_decode; instead of a second (combine) launch, the last
  * split CTA of each (batch, KV head, head group) tile -- found by an arrival counter --
- * merges that tile's query heads.  At most 4096 such tiles (else SA_ERR_UNSUPPORTED); up to
- * 16 calls may be in flight at once.  Measured against sa_attn_decode in the bench.
+ * merges that tile's query heads.  At most 4096 such tiles (else SA_ERR_UNSUPPORTED).  The
+ * arrival counters are 16 sets in the library's device image, used in turn by successive
+ * calls and zeroed by each tile's merge: up to 16 calls may be in flight on a device at once
+ * (any streams or graphs); replays of one captured graph must not overlap.
  */
 int sa_attn_decode_single(const void* q, const void* k, const void* v, void* o, float* lse,
                           int B, int Sk, int Hq, int Hkv, int D, float scale, int dtype,
@@ -175,11 +189,11 @@ int sa_attn_decode_single(const void* q, const void* k, const void* v, void* o, 
  * Computes sa_attn_fwd of the dequantised tensors q*q_descale, k*k_descale, v*v_descale:
  * S on kind::f8f6f4 tensor cores (exact products, fp32 sums), P rounded to e4m3 for P V.
  * D must be 128 (else SA_ERR_UNSUPPORTED); descales finite and > 0 (else SA_ERR_INVALID).
- * Accuracy: each weight is rounded to e4m3 relative to its row's running reference max,
- * and weights below 2^-10 of that reference become zero.  Up to about a thousand keys
- * this loss is negligible.  On long rows dominated by a few keys (attention sinks) the many
- * small weights can together carry much of the row's mass, and the result then departs
- * from the dequantised attention by far more than e4m3 rounding alone would suggest.
+ * Accuracy: each weight p = 2^(s - m_ref + 8) is rounded to e4m3 against its row's running
+ * reference max m_ref, which moves whenever the row max passes it by half a unit (log2),
+ * so the largest weights sit near 2^8 (under e4m3's 448) and only weights below 2^-18 of the
+ * row max round to zero.  O is normalised by the sum of the rounded weights; the LSE comes
+ * from fp32 sums of the unrounded ones (the offset taken off), as in sa_attn_fwd.
  */
 int sa_attn_fwd_fp8(const void* q, const void* k, const void* v, void* o, float* lse,
                     int B, int Sq, int Sk, int Hq, int Hkv, int D, int causal, float scale,
@@ -249,8 +263,14 @@ int sa_attn_decode(const void* q, const void* k, const void* v, void* o, float* 
  *   Limit: the split states must fit, B * Hq * splits * (D + 4) * 4 <= 8 MiB (splits as
  *   chosen by num_splits, see sa_attn_decode_workspace_size); larger problems return
  *   SA_ERR_UNSUPPORTED and leave the outputs untouched.
- *   The first call on a device looks up the area's device address (with that device
- *   current) and caches it; make that first call before any stream capture.
+ *   The area is part of the library's device code, which the CUDA runtime loads onto a
+ *   device when the library first uses it there (lazy module loading is the default):
+ *   the first call into the library on a device -- this entry point or any other --
+ *   takes the area's 8 MiB of device memory then.  A runtime that reserves the rest of
+ *   GPU memory afterwards must make one library call on each device before reserving.
+ *   The first call of this entry point on a device also looks up the area's device
+ *   address (with that device current) and caches it for the device's current context;
+ *   make that first call before any stream capture.
  *   Every call uses the same area: calls whose work may overlap on the GPU (other
  *   streams, other host threads) race and give undefined results.  Nothing in the area
  *   needs to start at zero; each call writes every byte it reads.
@@ -301,6 +321,27 @@ size_t sa_attn_decode_paged_workspace_size(int B, int Hq, int Hkv, int D, int pa
 int sa_attn_fwd_simple(const void* q, const void* k, const void* v, void* o, float* lse,
                        int B, int Sq, int Sk, int Hq, int Hkv, int D, int causal,
                        float scale, int dtype, sa_stream_t stream);
+
+/*
+ * Diagnostic: reads `bytes` of device memory at `src` once, with no attention arithmetic,
+ * and XORs it into *sink (device uint32, 4-byte aligned).  mode 0: 128-bit loads from four
+ * 256-thread blocks per SM, eight loads in flight per thread; mode 1: bulk asynchronous
+ * copies of 16 KB into a four-stage shared-memory ring, three blocks per SM -- the way the
+ * decode's split kernel streams K/V.  Gives the time one cold read of a buffer takes on
+ * this GPU, the floor of a kernel bound by reading those bytes (the decode's K/V).
+ * src 16-byte aligned and bytes a multiple of 16, sink non-null (else SA_ERR_INVALID);
+ * mode 0 or 1 (else SA_ERR_UNSUPPORTED).  bytes == 0: SA_OK, nothing launched.
+ */
+int sa_diag_read_floor(const void* src, size_t bytes, unsigned int* sink, int mode,
+                       sa_stream_t stream);
+
+/*
+ * Diagnostic: y[i] = 2^x[i] for i < n, computed by the FMA-pipe exponential the forward
+ * kernel uses for one exponential pair in four (range reduction to x = n + f, |f| <= 1/2,
+ * and a fitted cubic for 2^f; arguments below -126 are clamped there).  x, y: device
+ * float arrays of n elements (4-byte aligned).  For testing that exponential on its own.
+ */
+int sa_diag_exp2_poly(const float* x, float* y, int n, sa_stream_t stream);
 
 /* Thread-local description of the last non-OK return of this thread ("" if none). */
 const char* sa_last_error(void);

@@ -389,9 +389,52 @@ attn_decode_split(const __grid_constant__ CUtensorMap tm_k, const __grid_constan
   }
 }
 
+// The merge's summation order, written out so the combine kernel and the single-kernel
+// instance (which run the same row merge) give identical bits whatever the compiler does
+// around them.
+// With the split weights w_s = 2^(m_s - M), M the row max over the splits:
+//   * each of the two sums (of the 16-bit weights, of the fp32 weights), sum_s w_s y_s:
+//     virtual lane t of 128 (warp t / 32, lane t % 32) takes splits t and t + 128,
+//     x_t = fma(w_b, y_b, w_a * y_a); a butterfly over the 32 lanes of each virtual warp;
+//     then (x_0 + x_1) + (x_2 + x_3) over the 4 virtual warps;
+//   * each output float4 column c: group g of NG = 128 / (D/4) sums its splits g, g + NG, ...
+//     in order with fma from 0; then the NG group sums in order g = 0, 1, ...
+// Every operation is written with an explicit rounding so no contraction differs between
+// the two kernels.
+__device__ __forceinline__ float merge_pair(float wa, float ya, float wb, float yb) {
+  return __fmaf_rn(wb, yb, __fmul_rn(wa, ya));
+}
+__device__ __forceinline__ float butterfly_sum(float x) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) x = __fadd_rn(x, __shfl_xor_sync(0xffffffffu, x, o));
+  return x;                                                   // the same value in every lane
+}
+__device__ __forceinline__ float sum4(const float (&x)[4]) {
+  return __fadd_rn(__fadd_rn(x[0], x[1]), __fadd_rn(x[2], x[3]));
+}
+__device__ __forceinline__ void fma4(float4& acc, float w, const float4& v) {
+  acc.x = __fmaf_rn(w, v.x, acc.x); acc.y = __fmaf_rn(w, v.y, acc.y);
+  acc.z = __fmaf_rn(w, v.z, acc.z); acc.w = __fmaf_rn(w, v.w, acc.w);
+}
+__device__ __forceinline__ void add4(float4& a, const float4& b) {
+  a.x = __fadd_rn(a.x, b.x); a.y = __fadd_rn(a.y, b.y); a.z = __fadd_rn(a.z, b.z); a.w = __fadd_rn(a.w, b.w);
+}
+template <bool BF16>
+__device__ __forceinline__ void store_o4(const DecParams& p, size_t row, int D, int c, const float4& a, float L) {
+  const float inv = L > 0.f ? 1.f / L : 0.f;
+  uint2 packed;
+  packed.x = pack2<BF16>(__fmul_rn(a.x, inv), __fmul_rn(a.y, inv));
+  packed.y = pack2<BF16>(__fmul_rn(a.z, inv), __fmul_rn(a.w, inv));
+  reinterpret_cast<uint2*>(reinterpret_cast<uint16_t*>(p.o) + row * D)[c] = packed;
+}
+__device__ __forceinline__ float merged_lse(float M, float E) {
+  return E > 0.f ? __fmul_rn(__fadd_rn(M, __log2f(E)), 0.69314718055994531f) : -INFINITY;
+}
+
 // The merge of one (batch, query head) row by a block of 128 threads (scratch: s_w [MAX_SPLITS],
 // s_red [3][4], s_acc [128]).  Loads bypass L1 (.cg): in the single-kernel instance the
-// partial states were written by other CTAs of the same grid.
+// partial states were written by other CTAs of the same grid.  Thread t owns float4 column
+// c = t % (D/4) and the splits g, g + NG, ... with g = t / (D/4).
 template <int D, bool BF16>
 __device__ __forceinline__ void decode_merge_row(const DecParams& p, size_t row, float* s_w, float (*s_red)[4],
                                                  float4* s_acc) {
@@ -426,42 +469,27 @@ __device__ __forceinline__ void decode_merge_row(const DecParams& p, size_t row,
   const float wB = (mlB.x == -INFINITY) ? 0.f : ex2(mlB.x - M);
   if (tid < ns) s_w[tid] = wA;
   if (tid + 128 < ns) s_w[tid + 128] = wB;
-  float L = wA * mlA.y + wB * mlB.y, E = wA * mlA.z + wB * mlB.z;
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) {
-    L += __shfl_xor_sync(0xffffffffu, L, o);
-    E += __shfl_xor_sync(0xffffffffu, E, o);
-  }
+  const float L = butterfly_sum(merge_pair(wA, mlA.y, wB, mlB.y));
+  const float E = butterfly_sum(merge_pair(wA, mlA.z, wB, mlB.z));
   __syncthreads();                                            // s_red[0] consumed, s_w written
   if (lane == 0) { s_red[1][warp] = L; s_red[2][warp] = E; }
-  __syncthreads();
-  L = (s_red[1][0] + s_red[1][1]) + (s_red[1][2] + s_red[1][3]);
-  E = (s_red[2][0] + s_red[2][1]) + (s_red[2][2] + s_red[2][3]);
   // weighted sum of this thread's splits
   float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll
   for (int u = 0; u < PER; ++u) {
     const int s = g + u * NG;
-    const float w = s < ns ? s_w[s] : 0.f;
-    acc.x = fmaf(w, v[u].x, acc.x); acc.y = fmaf(w, v[u].y, acc.y);
-    acc.z = fmaf(w, v[u].z, acc.z); acc.w = fmaf(w, v[u].w, acc.w);
+    if (s < ns) fma4(acc, s_w[s], v[u]);
   }
   s_acc[tid] = acc;
   __syncthreads();
+  const float Lt = sum4(s_red[1]), Et = sum4(s_red[2]);
   if (tid < NC) {
     float4 a = s_acc[tid];
 #pragma unroll
-    for (int k = 1; k < NG; ++k) {
-      const float4 b2 = s_acc[k * NC + tid];
-      a.x += b2.x; a.y += b2.y; a.z += b2.z; a.w += b2.w;
-    }
-    const float inv = L > 0.f ? 1.f / L : 0.f;
-    uint2 packed;
-    packed.x = pack2<BF16>(a.x * inv, a.y * inv);
-    packed.y = pack2<BF16>(a.z * inv, a.w * inv);
-    reinterpret_cast<uint2*>(reinterpret_cast<uint16_t*>(p.o) + row * D)[tid] = packed;
+    for (int k = 1; k < NG; ++k) add4(a, s_acc[k * NC + tid]);
+    store_o4<BF16>(p, row, D, tid, a, Lt);
   }
-  if (p.lse && tid == 0) p.lse[row] = E > 0.f ? (M + __log2f(E)) * 0.69314718055994531f : -INFINITY;
+  if (p.lse && tid == 0) p.lse[row] = merged_lse(M, Et);
   __syncthreads();                                            // scratch free for the next row
 }
 

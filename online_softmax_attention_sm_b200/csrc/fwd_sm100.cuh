@@ -22,7 +22,8 @@
 //     S (tcgen05.ld 32x32b), computes the row max, p = 2^(c*s - m) with c = scale*log2(e),
 //     the row sums, writes P as 16-bit into tensor memory over S, and rescales its O row
 //     only when the reference max moves by more than kRescaleThresh (exact after the
-//     final division; keeps p <= 2^kRescaleThresh);
+//     final division; keeps p <= 2^kRescaleThresh; FP8: past half a unit, against an
+//     offset of 2^8);
 //   * the epilogue (same warpgroups) divides O by the row sum, rounds to the I/O dtype
 //     and writes O and the natural-log LSE.
 // Causal: K/V tiles past the diagonal are never loaded or multiplied; only tiles that
@@ -78,7 +79,7 @@ struct FwdCfg {
 constexpr int kWarpMma = 0;
 constexpr int kWarpLoad = 1;
 
-constexpr float kRescaleThresh = 8.0f;   // log2 units: the reference moves past this
+constexpr float kRescaleThresh = 8.0f;   // log2 units: the reference moves past this (16-bit P)
 // FP8 weights: p = 2^(x - m_ref + kFp8Offset), so a row's largest weights sit near the top of
 // e4m3's range instead of at 1 (weights below 2^-10 of the top round to zero, and a long row
 // can hold many of them); the reference then moves once the max passes it by kFp8Thresh,
@@ -585,10 +586,11 @@ __device__ __forceinline__ void fwd_mma(const FwdParams& p, const FwdSmem<D, FP8
 // bottleneck: 16 results per clock per SM).  x = n + f with n = round(x) taken from the
 // low mantissa bits of x + 1.5 * 2^23 and f in [-1/2, 1/2]; 2^f by a cubic fitted for
 // minimum relative error on that interval (max 7.6e-5, below the 16-bit rounding of P);
-// 2^n enters through the exponent field.  x is clamped at -126 so 2^n stays normal
-// (the result is then within 2^-126 of the true, smaller value).
+// 2^n enters through the exponent field.  x is clamped at -125: the cubic's value lies in
+// [0.7, 1.42), so with n >= -125 the exponent field stays >= 1 and the result normal (a
+// clamped argument gives 2^-125, within 2^-125 of the true, smaller value).
 __device__ __forceinline__ void exp2_poly_pair(float x0, float x1, float& a, float& b) {
-  const f32x2 x = pack_f2(fmaxf(x0, -126.f), fmaxf(x1, -126.f));
+  const f32x2 x = pack_f2(fmaxf(x0, -125.f), fmaxf(x1, -125.f));
   const f32x2 t = add_f2(x, pack_f2(12582912.f, 12582912.f));       // 1.5 * 2^23 + n
   const f32x2 f = fma_f2(add_f2(t, pack_f2(-12582912.f, -12582912.f)), pack_f2(-1.f, -1.f), x);
   f32x2 q = fma_f2(pack_f2(0.055174146f, 0.055174146f), f, pack_f2(0.24261758f, 0.24261758f));
@@ -602,14 +604,27 @@ __device__ __forceinline__ void exp2_poly_pair(float x0, float x1, float& a, flo
   b = __uint_as_float(__float_as_uint(q1) + (__float_as_uint(t1) << 23));
 }
 
+// Adds the two 16-bit values packed in pk (low half first) to two fp32 sums, one
+// mixed-precision add each (no unpacking into fp32 registers).
+template <bool BF16>
+__device__ __forceinline__ void add_16x2_to_f32(uint32_t pk, float& lo, float& hi) {
+  if (BF16)
+    asm("{\n .reg .b16 l, h;\n mov.b32 {l, h}, %2;\n add.rn.f32.bf16 %0, l, %0;\n add.rn.f32.bf16 %1, h, %1;\n}\n"
+        : "+f"(lo), "+f"(hi) : "r"(pk));
+  else
+    asm("{\n .reg .b16 l, h;\n mov.b32 {l, h}, %2;\n add.rn.f32.f16 %0, l, %0;\n add.rn.f32.f16 %1, h, %1;\n}\n"
+        : "+f"(lo), "+f"(hi) : "r"(pk));
+}
+
 // One 32-key chunk of a row (v: the 32 scores as raw fp32 bits): p = 2^(scale2 * s - m) on
 // pairs (one packed FMA per pair), P stored to tensor memory as 16-bit at taddr, both row
-// sums (rse2: the fp32 weights, for the LSE; rs2: the 16-bit weights the MMA multiplies,
-// so O / l is an exact weighted average of V).  With POLY > 0, one pair in POLY is
-// exponentiated by exp2_poly_pair (finite scores only).
+// sums (rse2: the fp32 weights, for the LSE; rs: the 16-bit weights the MMA multiplies, so
+// O / l is an exact weighted average of V -- the largest weights' rounding cancels, which
+// matters in rows one key dominates).  With POLY > 0, one pair in POLY is exponentiated
+// by exp2_poly_pair (finite scores only).
 template <bool BF16, int POLY>
 __device__ __forceinline__ void softmax_chunk(const uint32_t (&v)[32], const f32x2 scale2,
-                                              const f32x2 negm2, f32x2 (&rs2)[2], f32x2 (&rse2)[2],
+                                              const f32x2 negm2, float (&rs)[4], f32x2 (&rse2)[2],
                                               const uint32_t taddr) {
   uint32_t pk[16];
 #pragma unroll
@@ -624,26 +639,20 @@ __device__ __forceinline__ void softmax_chunk(const uint32_t (&v)[32], const f32
       b2 = ex2(x1);
     }
     rse2[i & 1] = add_f2(rse2[i & 1], pack_f2(a, b2));
-    float lo, hi;
     if (BF16) {
       __nv_bfloat162 h2 = __floats2bfloat162_rn(a, b2);
       pk[i] = *reinterpret_cast<uint32_t*>(&h2);
-      lo = __uint_as_float(pk[i] << 16);
-      hi = __uint_as_float(pk[i] & 0xffff0000u);
     } else {
       __half2 h2 = __floats2half2_rn(a, b2);
       pk[i] = *reinterpret_cast<uint32_t*>(&h2);
-      const float2 f = __half22float2(h2);
-      lo = f.x;
-      hi = f.y;
     }
-    rs2[i & 1] = add_f2(rs2[i & 1], pack_f2(lo, hi));
+    add_16x2_to_f32<BF16>(pk[i], rs[2 * (i & 1)], rs[2 * (i & 1) + 1]);
   }
   tmem_st16(taddr, pk);
 }
 
 // FP8 instance: the same chunk with P rounded to e4m3 (round to nearest even, saturating:
-// p <= 2^8 under the lazy reference, below e4m3's 448), 4 values per tensor-memory column
+// p <= 2^8.5 under the offset reference, below e4m3's 448), 4 values per tensor-memory column
 // (key 4j in the low byte of column j), 8 columns at taddr; rs2 sums the e4m3 values the
 // MMA multiplies.
 template <int POLY>
@@ -678,11 +687,24 @@ __device__ __forceinline__ void softmax_chunk_fp8(const uint32_t (&v)[32], const
                : "memory");
 }
 
+// rs2 (FP8: the e4m3 weights' sum as packed pairs) and rs (16-bit: four fp32 chains) hold
+// the sum of the weights the MMA multiplies.
 template <bool BF16, bool FP8, int POLY>
 __device__ __forceinline__ void softmax_chunk_any(const uint32_t (&v)[32], const f32x2 scale2, const f32x2 negm2,
-                                                  f32x2 (&rs2)[2], f32x2 (&rse2)[2], const uint32_t p_addr, int c) {
+                                                  f32x2 (&rs2)[2], float (&rs)[4], f32x2 (&rse2)[2],
+                                                  const uint32_t p_addr, int c) {
   if constexpr (FP8) softmax_chunk_fp8<POLY>(v, scale2, negm2, rs2, rse2, p_addr + c * 8);
-  else softmax_chunk<BF16, POLY>(v, scale2, negm2, rs2, rse2, p_addr + c * 16);
+  else softmax_chunk<BF16, POLY>(v, scale2, negm2, rs, rse2, p_addr + c * 16);
+}
+
+__device__ __forceinline__ void sum_rounded(const f32x2 (&rs2)[2], const float (&rs)[4], bool fp8, float& acc) {
+  if (fp8) {
+    float a0, a1;
+    unpack_f2(add_f2(rs2[0], rs2[1]), a0, a1);
+    acc += a0 + a1;
+  } else {
+    acc += (rs[0] + rs[1]) + (rs[2] + rs[3]);
+  }
 }
 
 // Running max over a 32-score chunk on 8 chains.
@@ -717,8 +739,8 @@ __device__ __forceinline__ void sum_f2x2(const f32x2 (&v)[2], float& acc) {
   acc += a0 + a1;
 }
 
-// Move the row's reference max to m_tile when it exceeds the reference by more than
-// kRescaleThresh, rescaling both sums and (after the first tile) the O_t row by
+// Move the row's reference max to m_tile when it exceeds the reference by more than the
+// instance's threshold, rescaling both sums and (after the first tile) the O_t row by
 // 2^(m_ref - m_tile).  O_t holds P V up to the previous tile, complete: the commit that
 // signalled this tile's S covers every earlier MMA.
 template <int D, bool FP8>
@@ -769,19 +791,20 @@ __device__ __forceinline__ void softmax_tile_full(const uint32_t s_addr, const u
   const float nm = FP8 ? kFp8Offset - m_use : -m_use;
   const f32x2 scale2 = pack_f2(c2, c2), negm2 = pack_f2(nm, nm);
   f32x2 rs2[2] = {0ull, 0ull}, rse2[2] = {0ull, 0ull};
+  float rs[4] = {0.f, 0.f, 0.f, 0.f};
   uint32_t v2[32], v3[32];
   tmem_ld32(s_addr + 64, v2);
-  softmax_chunk_any<BF16, FP8, kPolyEvery>(v0, scale2, negm2, rs2, rse2, p_addr, 0);
-  softmax_chunk_any<BF16, FP8, kPolyEvery>(v1, scale2, negm2, rs2, rse2, p_addr, 1);
+  softmax_chunk_any<BF16, FP8, kPolyEvery>(v0, scale2, negm2, rs2, rs, rse2, p_addr, 0);
+  softmax_chunk_any<BF16, FP8, kPolyEvery>(v1, scale2, negm2, rs2, rs, rse2, p_addr, 1);
   tmem_wait_ld_regs(v2);
   tmem_ld32(s_addr + 96, v3);
-  softmax_chunk_any<BF16, FP8, kPolyEvery>(v2, scale2, negm2, rs2, rse2, p_addr, 2);
+  softmax_chunk_any<BF16, FP8, kPolyEvery>(v2, scale2, negm2, rs2, rs, rse2, p_addr, 2);
   tmem_wait_st();
   tc_fence_before();
   mbar_arrive(p_part);
   tmem_wait_ld_regs(v3);
-  softmax_chunk_any<BF16, FP8, kPolyEvery>(v3, scale2, negm2, rs2, rse2, p_addr, 3);
-  sum_f2x2(rs2, l_sum);
+  softmax_chunk_any<BF16, FP8, kPolyEvery>(v3, scale2, negm2, rs2, rs, rse2, p_addr, 3);
+  sum_rounded(rs2, rs, FP8, l_sum);
   sum_f2x2(rse2, l_lse);
 }
 
@@ -812,16 +835,17 @@ __device__ __forceinline__ void softmax_tile_masked(const uint32_t s_addr, const
   const float nm = FP8 ? kFp8Offset - m_use : -m_use;
   const f32x2 scale2 = pack_f2(1.f, 1.f), negm2 = pack_f2(nm, nm);
   f32x2 rs2[2] = {0ull, 0ull}, rse2[2] = {0ull, 0ull};
+  float rs[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
   for (int c = 0; c < 4; ++c) {
-    softmax_chunk_any<BF16, FP8, 0>(v[c], scale2, negm2, rs2, rse2, p_addr, c);
+    softmax_chunk_any<BF16, FP8, 0>(v[c], scale2, negm2, rs2, rs, rse2, p_addr, c);
     if (c == 2) {
       tmem_wait_st();
       tc_fence_before();
       mbar_arrive(p_part);
     }
   }
-  sum_f2x2(rs2, l_sum);
+  sum_rounded(rs2, rs, FP8, l_sum);
   sum_f2x2(rse2, l_lse);
 }
 
@@ -851,8 +875,8 @@ __device__ __forceinline__ void fwd_softmax(const FwdParams& p, const FwdSmem<D,
     int kvis = x.sk;                        // keys every row of the tile can see
     if (p.causal) kvis = min(kvis, max(0, r0 + x.sk - x.sq + 1));
     const int mask_from = kvis / 128;
-    // l_sum: sum of the 16-bit weights (normalises O, matching what the MMA multiplied);
-    // l_lse: sum of the fp32 weights (gives the LSE without the 16-bit rounding bias)
+    // l_sum: sum of the rounded weights the MMA multiplied (normalises O); l_lse: sum of
+    // the fp32 weights (gives the LSE without the rounding bias)
     float m_ref = -INFINITY, l_sum = 0.f, l_lse = 0.f;
     const uint32_t s_addr = lane_addr + Cfg::S_COL(t), o_addr = lane_addr + Cfg::O_COL(t);
     const uint32_t p_addr = lane_addr + Cfg::P_COL(t);

@@ -8,13 +8,16 @@
 #include "bwd_sm100.cuh"
 #include "fwd_simple.cuh"
 #include "decode.cuh"
+#include "diag.cuh"
 
 #include <cmath>
 #include <cstdarg>
 #include <cstdio>
 #include <cstring>
 #include <map>
+#include <tuple>
 #include <mutex>
+#include <atomic>
 #include <vector>
 #include <algorithm>
 #include <string>
@@ -54,6 +57,46 @@ EncodeTiledFn get_encode() {
       fn = reinterpret_cast<EncodeTiledFn>(p);
   });
   return fn;
+}
+
+// Device address of a __device__ variable of this library on the current device, looked up
+// once per (device, context, variable) with that device current and cached.  Keyed by the
+// context too: after a device reset the runtime creates a new primary context and reloads
+// the module, and the old address would be stale.
+using CtxGetCurrentFn = CUresult (*)(CUcontext*);
+
+int device_symbol(const void* symbol, const char* what, void** out) {
+  static std::mutex mu;
+  static std::map<std::tuple<int, uintptr_t, uintptr_t>, void*> cache;
+  static CtxGetCurrentFn ctx_fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      ctx_fn = reinterpret_cast<CtxGetCurrentFn>(p);
+  });
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+  CUcontext ctx = nullptr;
+  if (ctx_fn && (ctx_fn(&ctx) != CUDA_SUCCESS || !ctx)) {
+    // no context current yet: the runtime makes the device's primary context current on
+    // first use, which a no-op free triggers
+    cudaFree(nullptr);
+    if (ctx_fn(&ctx) != CUDA_SUCCESS) ctx = nullptr;
+  }
+  const auto key = std::make_tuple(dev, reinterpret_cast<uintptr_t>(ctx), reinterpret_cast<uintptr_t>(symbol));
+  std::lock_guard<std::mutex> lock(mu);
+  auto it = cache.find(key);
+  if (it != cache.end()) { *out = it->second; return SA_OK; }
+  void* p = nullptr;
+  e = cudaGetSymbolAddress(&p, symbol);
+  if (e != cudaSuccess) return fail(SA_ERR_CUDA, "cudaGetSymbolAddress(%s): %s", what, cudaGetErrorString(e));
+  if (cache.size() < 4096) cache[key] = p;
+  *out = p;
+  return SA_OK;
 }
 
 // Map element type for 8-bit (e4m3) tensors, next to SA_FP16 / SA_BF16.
@@ -175,28 +218,19 @@ bool fwd_use_dynamic(const sa::FwdParams& p, int D, int ncta) {
 }
 
 // Dynamic-scheduling counters of the forward kernel: kFwdWorkSlots pairs (next unit, CTAs
-// done), zero-initialised with the module; launches take slots in turn and the last CTA of
-// a launch zeroes its pair, so up to kFwdWorkSlots forward launches may be in flight at once
-// (on any streams) without sharing a counter.
-constexpr int kFwdWorkSlots = 64;
+// done), zero-initialised with the module; launches of the dynamic instance take slots in
+// turn and the last CTA of a launch zeroes its pair, so up to kFwdWorkSlots of them may be in
+// flight at once (on any streams) without sharing a counter.  A launch that shared a pair
+// with a live one would skip or repeat units; the limit is stated in the C ABI's header.
+constexpr int kFwdWorkSlots = 1024;
 static __device__ unsigned int g_fwd_work[2 * kFwdWorkSlots];
 
 int fwd_work_slot(unsigned int** out) {
-  static std::mutex mu;
-  static unsigned int* addr[64] = {nullptr};
-  static unsigned int next[64] = {0};
-  int dev = 0;
-  cudaError_t e = cudaGetDevice(&dev);
-  if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
-  if (dev < 0 || dev >= 64) return fail(SA_ERR_UNSUPPORTED, "device ordinal %d out of range", dev);
-  std::lock_guard<std::mutex> lock(mu);
-  if (!addr[dev]) {
-    void* p = nullptr;
-    e = cudaGetSymbolAddress(&p, g_fwd_work);
-    if (e != cudaSuccess) return cuda_fail(e, "cudaGetSymbolAddress(forward work counters)");
-    addr[dev] = static_cast<unsigned int*>(p);
-  }
-  *out = addr[dev] + 2 * (next[dev]++ % kFwdWorkSlots);
+  static std::atomic<unsigned int> next{0};
+  void* base = nullptr;
+  int rc = device_symbol((const void*)&g_fwd_work, "forward work counters", &base);
+  if (rc != SA_OK) return rc;
+  *out = static_cast<unsigned int*>(base) + 2 * (next++ % kFwdWorkSlots);
   return SA_OK;
 }
 
@@ -421,21 +455,11 @@ constexpr int kDecSemSlots = 16, kDecSemTiles = 4096;
 static __device__ unsigned int g_dec_sem[kDecSemSlots * kDecSemTiles];
 
 int dec_sem_slot(unsigned int** out) {
-  static std::mutex mu;
-  static unsigned int* addr[64] = {nullptr};
-  static unsigned int next[64] = {0};
-  int dev = 0;
-  cudaError_t e = cudaGetDevice(&dev);
-  if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
-  if (dev < 0 || dev >= 64) return fail(SA_ERR_UNSUPPORTED, "device ordinal %d out of range", dev);
-  std::lock_guard<std::mutex> lock(mu);
-  if (!addr[dev]) {
-    void* ptr = nullptr;
-    e = cudaGetSymbolAddress(&ptr, g_dec_sem);
-    if (e != cudaSuccess) return cuda_fail(e, "cudaGetSymbolAddress(decode arrival counters)");
-    addr[dev] = static_cast<unsigned int*>(ptr);
-  }
-  *out = addr[dev] + (size_t)kDecSemTiles * (next[dev]++ % kDecSemSlots);
+  static std::atomic<unsigned int> next{0};
+  void* base = nullptr;
+  int rc = device_symbol((const void*)&g_dec_sem, "decode arrival counters", &base);
+  if (rc != SA_OK) return rc;
+  *out = static_cast<unsigned int*>(base) + (size_t)kDecSemTiles * (next++ % kDecSemSlots);
   return SA_OK;
 }
 
@@ -501,24 +525,9 @@ int launch_decode(const void* q, const void* k, const void* v, void* o, float* l
 constexpr size_t kNoAllocScratchBytes = 8u << 20;
 static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
 
-// Device address of g_noalloc_scratch on the current device (looked up on the first call
-// per device, with that device current).  Returns SA_OK or SA_ERR_CUDA.
+// Device address of g_noalloc_scratch on the current device.  Returns SA_OK or SA_ERR_CUDA.
 int noalloc_scratch(void** out) {
-  static std::mutex mu;
-  static void* addr[64] = {nullptr};
-  int dev = 0;
-  cudaError_t e = cudaGetDevice(&dev);
-  if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
-  if (dev < 0 || dev >= 64) return fail(SA_ERR_UNSUPPORTED, "device ordinal %d out of range", dev);
-  std::lock_guard<std::mutex> lock(mu);
-  if (!addr[dev]) {
-    void* p = nullptr;
-    e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
-    if (e != cudaSuccess) return cuda_fail(e, "cudaGetSymbolAddress(built-in decode scratch)");
-    addr[dev] = p;
-  }
-  *out = addr[dev];
-  return SA_OK;
+  return device_symbol((const void*)g_noalloc_scratch, "built-in decode scratch", out);
 }
 
 // Shared by the 16-bit and the FP8 block-sparse entry points (fp8: q, k, v e4m3, o bf16,
@@ -908,6 +917,37 @@ int sa_attn_decode_paged(const void* q, const void* k_cache, const void* v_cache
               : launch_decode<64, false, true>(q, k_cache, v_cache, o, lse, B, msl, Hq, Hkv, scale, pl, workspace, st, pg);
   return bf ? launch_decode<128, true, true>(q, k_cache, v_cache, o, lse, B, msl, Hq, Hkv, scale, pl, workspace, st, pg)
             : launch_decode<128, false, true>(q, k_cache, v_cache, o, lse, B, msl, Hq, Hkv, scale, pl, workspace, st, pg);
+}
+
+int sa_diag_read_floor(const void* src, size_t bytes, unsigned int* sink, int mode, sa_stream_t stream) {
+  if (!src || !sink) return fail(SA_ERR_INVALID, "src and sink must be non-null");
+  if (!aligned16(src) || (bytes & 15u)) return fail(SA_ERR_INVALID, "src must be 16-byte aligned, bytes a multiple of 16");
+  if ((uintptr_t)sink & 3u) return fail(SA_ERR_INVALID, "sink must be 4-byte aligned");
+  if (mode != 0 && mode != 1) return fail(SA_ERR_UNSUPPORTED, "mode must be 0 or 1 (got %d)", mode);
+  if (bytes == 0) return SA_OK;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  cudaError_t e;
+  if (mode == 0) {
+    sa::read_floor_ld<<<4 * num_sms(), sa::kFloorThreads, 0, st>>>(static_cast<const uint4*>(src), bytes / 16, sink);
+  } else {
+    const int smem = 1024 + sa::kBulkStages * sa::kBulkBytes + 64;
+    e = cudaFuncSetAttribute(sa::read_floor_bulk, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(read_floor_bulk)");
+    sa::read_floor_bulk<<<3 * num_sms(), 128, smem, st>>>(static_cast<const uint8_t*>(src), bytes / 16, sink);
+  }
+  e = cudaGetLastError();
+  return e == cudaSuccess ? SA_OK : cuda_fail(e, "read_floor launch");
+}
+
+int sa_diag_exp2_poly(const float* x, float* y, int n, sa_stream_t stream) {
+  if (n < 0) return fail(SA_ERR_INVALID, "negative n");
+  if (n == 0) return SA_OK;
+  if (!x || !y || ((uintptr_t)x & 3u) || ((uintptr_t)y & 3u))
+    return fail(SA_ERR_INVALID, "x and y must be non-null, 4-byte aligned device arrays");
+  const int pairs = (n + 1) / 2;
+  sa::diag_exp2_poly<<<(pairs + 255) / 256, 256, 0, reinterpret_cast<cudaStream_t>(stream)>>>(x, y, n);
+  cudaError_t e = cudaGetLastError();
+  return e == cudaSuccess ? SA_OK : cuda_fail(e, "diag_exp2_poly launch");
 }
 
 const char* sa_last_error(void) { return g_err.c_str(); }

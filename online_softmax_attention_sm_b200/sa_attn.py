@@ -43,6 +43,8 @@ SIGNATURES = {
     "sa_check_status": (_I, [_P]),
     "sa_version": (ctypes.c_char_p, []),
     "sa_selftest_bounded_wait": (_I, [_P]),
+    "sa_diag_read_floor": (_I, [_P, _Z, _P, _I, _P]),
+    "sa_diag_exp2_poly": (_I, [_P, _P, _I, _P]),
 }
 
 _lib = None
@@ -438,6 +440,28 @@ def sa_attn_decode_paged(q, k_cache, v_cache, block_table, seqlens, scale=None, 
                                       float(scale), _DT[q.dtype], int(num_splits), _ptr(workspace),
                                       workspace.numel() * workspace.element_size(), _stream(stream)))
     return out, lse
+
+
+def sa_diag_read_floor(buf, sink, mode=0, stream=None):
+    """Diagnostic: read every byte of the contiguous CUDA tensor `buf` once (no attention
+    arithmetic), folding it into the int32 CUDA tensor `sink` (one element).  mode 0:
+    128-bit loads; mode 1: bulk copies into a shared-memory ring (the decode's way)."""
+    if not buf.is_contiguous():
+        raise ValueError("buf must be contiguous")
+    if sink.dtype != torch.int32 or sink.device != buf.device or sink.numel() < 1:
+        raise ValueError("sink must be an int32 tensor on buf's device")
+    _check(lib().sa_diag_read_floor(_ptr(buf), buf.numel() * buf.element_size(), _ptr(sink), int(mode),
+                                    _stream(stream)))
+
+
+def sa_diag_exp2_poly(x, out=None, stream=None):
+    """Diagnostic: 2^x by the forward kernel's FMA-pipe exponential (x: float32 CUDA tensor)."""
+    _check_tensor("x", x, torch.float32, x.device)
+    if out is None:
+        out = torch.empty_like(x)
+    _check_out("out", out, x.shape, torch.float32, x.device)
+    _check(lib().sa_diag_exp2_poly(_ptr(x), _ptr(out), x.numel(), _stream(stream)))
+    return out
 
 
 def sa_check_status(stream=None):

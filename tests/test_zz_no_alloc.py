@@ -4,8 +4,11 @@ It serves callers that cannot give the library device memory for scratch (runtim
 reserve all GPU memory up front, hosts whose allocator is out of reach of the calling
 code); its scratch is a fixed area inside the library.  Checked here through the C ABI
 against the workspace-taking sa_attn_decode, on calls in a row that reuse the area with
-different shapes, plus the size limit.  This file is collected last on purpose: a run
-that stops at the first failure has already run every other test.
+different shapes: the two run the same kernels with the same split plan, so the results
+must be bit-identical (a stale or aliased byte in the shared area would show), plus the
+size limit.  The library's device code (the area included) is loaded by the first call
+into it -- here the reference decode, before any measured call.  This file is collected
+last on purpose: a run that stops at the first failure has already run every other test.
 """
 import ctypes
 
@@ -52,19 +55,21 @@ def test_noalloc_decode_matches_workspace_decode():
         lerr = (lse - ref_lse).abs().max().item()
         assert err <= O_TOL[dt], f"call {i}: max |O - O_ref| = {err:.3e}"
         assert lerr <= LSE_TOL, f"call {i}: max |LSE - LSE_ref| = {lerr:.3e}"
+        assert torch.equal(o, ref_o) and torch.equal(lse, ref_lse), f"call {i}: not bit-identical"
 
 
 def test_noalloc_rejects_problems_beyond_its_scratch():
-    B, Sk, Hq, Hkv, D = 64, 32768, 64, 8, 128      # with 96 splits: ~186 MB of split states
+    # 2 splits of 64 keys for 64 x 128 rows of D = 128: 8.65 MB of split states, over the 8 MiB
+    # area.  K/V really hold Sk rows, so even if the size check failed to stop the call it
+    # could only compute, never read outside the buffers.
+    B, Sk, Hq, Hkv, D, ns = 64, 128, 128, 8, 128, 2
+    assert B * Hq * ns * (D + 4) * 4 > 8 << 20
     q = torch.zeros((B, Hq, D), dtype=torch.bfloat16, device=DEV)
-    k = torch.zeros((B, 128, Hkv, D), dtype=torch.bfloat16, device=DEV)   # never read
+    k = torch.zeros((B, Sk, Hkv, D), dtype=torch.bfloat16, device=DEV)
+    v = torch.zeros_like(k)
     o = torch.full_like(q, 3.0)
     lse = torch.full((B, Hq), 3.0, dtype=torch.float32, device=DEV)
-    fake_k = ctypes.c_void_p(k.data_ptr())
-    rc = lib().sa_attn_decode_noalloc(ctypes.c_void_p(q.data_ptr()), fake_k, fake_k,
-                                      ctypes.c_void_p(o.data_ptr()), ctypes.c_void_p(lse.data_ptr()),
-                                      B, Sk, Hq, Hkv, D, ctypes.c_float(0.1), SA_BF16, 96,
-                                      ctypes.c_void_p(torch.cuda.current_stream().cuda_stream))
+    rc = noalloc(q, k, v, o, lse, 0.1, "bf16", num_splits=ns)
     assert rc == SA_ERR_UNSUPPORTED
     assert "scratch" in lib().sa_last_error().decode()
     sa_check_status()
