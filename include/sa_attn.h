@@ -343,6 +343,20 @@ int sa_diag_read_floor(const void* src, size_t bytes, unsigned int* sink, int mo
  */
 int sa_diag_exp2_poly(const float* x, float* y, int n, sa_stream_t stream);
 
+/*
+ * The same forward as sa_attn_fwd on a second kernel that runs each unit of 256 query rows
+ * on a pair of CTAs (a two-CTA cluster): 2-SM tensor-core products (each SM loads half of
+ * every K/V tile), S double-buffered in tensor memory so the softmax never waits for its
+ * own tile's next S, the softmax of each row split over two threads.  D = 128 only (else
+ * SA_ERR_UNSUPPORTED); dense layout; static work order.  Same arguments, conventions and
+ * results as sa_attn_fwd -- the two kernels give identical bits.  sa_attn_fwd does not use
+ * it: on this hardware both are bound by the softmax's exponentials per SM, and the pair's
+ * cross-CTA hand-offs made it about 20 % slower on the shapes measured.
+ */
+int sa_attn_fwd_pair(const void* q, const void* k, const void* v, void* o, float* lse,
+                     int B, int Sq, int Sk, int Hq, int Hkv, int D, int causal,
+                     float scale, int dtype, sa_stream_t stream);
+
 /* Thread-local description of the last non-OK return of this thread ("" if none). */
 const char* sa_last_error(void);
 

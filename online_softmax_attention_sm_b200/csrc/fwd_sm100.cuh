@@ -745,13 +745,13 @@ __device__ __forceinline__ void sum_f2x2(const f32x2 (&v)[2], float& acc) {
 // signalled this tile's S covers every earlier MMA.
 template <int D, bool FP8>
 __device__ __forceinline__ void move_reference(const float m_tile, const bool first, float& m_ref,
-                                               float& l_sum, float& l_lse, const uint32_t o_addr) {
+                                               float (&l_sum)[2], float (&l_lse)[2], const uint32_t o_addr) {
   const bool need = m_tile > m_ref + (FP8 ? kFp8Thresh : kRescaleThresh);
   float alpha = 1.f;
   if (need) {
     alpha = ex2(m_ref - m_tile);       // 0 when m_ref == -inf
-    l_sum *= alpha;
-    l_lse *= alpha;
+    l_sum[0] *= alpha; l_sum[1] *= alpha;
+    l_lse[0] *= alpha; l_lse[1] *= alpha;
     m_ref = m_tile;
   }
   if (!first && __any_sync(0xffffffffu, need)) rescale_o_row<D>(o_addr, alpha);
@@ -765,7 +765,7 @@ __device__ __forceinline__ void move_reference(const float m_tile, const bool fi
 template <int D, bool BF16, bool FP8>
 __device__ __forceinline__ void softmax_tile_full(const uint32_t s_addr, const uint32_t o_addr,
                                                   const uint32_t p_addr, const float c2, const bool first,
-                                                  float& m_ref, float& l_sum, float& l_lse,
+                                                  float& m_ref, float (&l_sum)[2], float (&l_lse)[2],
                                                   uint64_t* p_part) {
   uint32_t v0[32], v1[32];
   float mx[8];
@@ -790,22 +790,27 @@ __device__ __forceinline__ void softmax_tile_full(const uint32_t s_addr, const u
   const float m_use = (m_ref == -INFINITY) ? 0.f : m_ref;
   const float nm = FP8 ? kFp8Offset - m_use : -m_use;
   const f32x2 scale2 = pack_f2(c2, c2), negm2 = pack_f2(nm, nm);
-  f32x2 rs2[2] = {0ull, 0ull}, rse2[2] = {0ull, 0ull};
-  float rs[4] = {0.f, 0.f, 0.f, 0.f};
+  // the row's sums are kept per key half (keys 0-63, 64-127) and added at the end, the order
+  // the pair kernel's two half-row threads use, so both kernels give identical bits
+  f32x2 rs2[2][2] = {{0ull, 0ull}, {0ull, 0ull}}, rse2[2][2] = {{0ull, 0ull}, {0ull, 0ull}};
+  float rs[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
   uint32_t v2[32], v3[32];
   tmem_ld32(s_addr + 64, v2);
-  softmax_chunk_any<BF16, FP8, kPolyEvery>(v0, scale2, negm2, rs2, rs, rse2, p_addr, 0);
-  softmax_chunk_any<BF16, FP8, kPolyEvery>(v1, scale2, negm2, rs2, rs, rse2, p_addr, 1);
+  softmax_chunk_any<BF16, FP8, kPolyEvery>(v0, scale2, negm2, rs2[0], rs[0], rse2[0], p_addr, 0);
+  softmax_chunk_any<BF16, FP8, kPolyEvery>(v1, scale2, negm2, rs2[0], rs[0], rse2[0], p_addr, 1);
   tmem_wait_ld_regs(v2);
   tmem_ld32(s_addr + 96, v3);
-  softmax_chunk_any<BF16, FP8, kPolyEvery>(v2, scale2, negm2, rs2, rs, rse2, p_addr, 2);
+  softmax_chunk_any<BF16, FP8, kPolyEvery>(v2, scale2, negm2, rs2[1], rs[1], rse2[1], p_addr, 2);
   tmem_wait_st();
   tc_fence_before();
   mbar_arrive(p_part);
   tmem_wait_ld_regs(v3);
-  softmax_chunk_any<BF16, FP8, kPolyEvery>(v3, scale2, negm2, rs2, rs, rse2, p_addr, 3);
-  sum_rounded(rs2, rs, FP8, l_sum);
-  sum_f2x2(rse2, l_lse);
+  softmax_chunk_any<BF16, FP8, kPolyEvery>(v3, scale2, negm2, rs2[1], rs[1], rse2[1], p_addr, 3);
+#pragma unroll
+  for (int hh = 0; hh < 2; ++hh) {
+    sum_rounded(rs2[hh], rs[hh], FP8, l_sum[hh]);
+    sum_f2x2(rse2[hh], l_lse[hh]);
+  }
 }
 
 // A tile that crosses the causal diagonal or the ragged end of K (or a negative scale):
@@ -813,8 +818,8 @@ __device__ __forceinline__ void softmax_tile_full(const uint32_t s_addr, const u
 template <int D, bool BF16, bool FP8>
 __device__ __forceinline__ void softmax_tile_masked(const uint32_t s_addr, const uint32_t o_addr,
                                                     const uint32_t p_addr, const float c2, const int kl,
-                                                    const bool first, float& m_ref, float& l_sum,
-                                                    float& l_lse, uint64_t* p_part) {
+                                                    const bool first, float& m_ref, float (&l_sum)[2],
+                                                    float (&l_lse)[2], uint64_t* p_part) {
   uint32_t v[4][32];
 #pragma unroll
   for (int c = 0; c < 4; ++c) tmem_ld32(s_addr + c * 32, v[c]);
@@ -834,19 +839,22 @@ __device__ __forceinline__ void softmax_tile_masked(const uint32_t s_addr, const
   const float m_use = (m_ref == -INFINITY) ? 0.f : m_ref;
   const float nm = FP8 ? kFp8Offset - m_use : -m_use;
   const f32x2 scale2 = pack_f2(1.f, 1.f), negm2 = pack_f2(nm, nm);
-  f32x2 rs2[2] = {0ull, 0ull}, rse2[2] = {0ull, 0ull};
-  float rs[4] = {0.f, 0.f, 0.f, 0.f};
+  f32x2 rs2[2][2] = {{0ull, 0ull}, {0ull, 0ull}}, rse2[2][2] = {{0ull, 0ull}, {0ull, 0ull}};
+  float rs[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
 #pragma unroll
   for (int c = 0; c < 4; ++c) {
-    softmax_chunk_any<BF16, FP8, 0>(v[c], scale2, negm2, rs2, rs, rse2, p_addr, c);
+    softmax_chunk_any<BF16, FP8, 0>(v[c], scale2, negm2, rs2[c >> 1], rs[c >> 1], rse2[c >> 1], p_addr, c);
     if (c == 2) {
       tmem_wait_st();
       tc_fence_before();
       mbar_arrive(p_part);
     }
   }
-  sum_rounded(rs2, rs, FP8, l_sum);
-  sum_f2x2(rse2, l_lse);
+#pragma unroll
+  for (int hh = 0; hh < 2; ++hh) {
+    sum_rounded(rs2[hh], rs[hh], FP8, l_sum[hh]);
+    sum_f2x2(rse2[hh], l_lse[hh]);
+  }
 }
 
 template <int D, bool BF16, bool DYN, bool SPARSE, bool FP8, bool PAGED>
@@ -877,7 +885,7 @@ __device__ __forceinline__ void fwd_softmax(const FwdParams& p, const FwdSmem<D,
     const int mask_from = kvis / 128;
     // l_sum: sum of the rounded weights the MMA multiplied (normalises O); l_lse: sum of
     // the fp32 weights (gives the LSE without the rounding bias)
-    float m_ref = -INFINITY, l_sum = 0.f, l_lse = 0.f;
+    float m_ref = -INFINITY, l_sum[2] = {0.f, 0.f}, l_lse[2] = {0.f, 0.f};
     const uint32_t s_addr = lane_addr + Cfg::S_COL(t), o_addr = lane_addr + Cfg::O_COL(t);
     const uint32_t p_addr = lane_addr + Cfg::P_COL(t);
     int i = 0;                              // block-sparse: this tile's K/V steps so far
@@ -914,7 +922,8 @@ __device__ __forceinline__ void fwd_softmax(const FwdParams& p, const FwdSmem<D,
       tc_fence_after();
     }
     const bool store = row < x.sq;
-    const float inv_l = l_sum > 0.f ? p.o_mul / l_sum : 0.f;   // o_mul: FP8 V descale, else 1
+    const float L = l_sum[0] + l_sum[1], E = l_lse[0] + l_lse[1];
+    const float inv_l = L > 0.f ? p.o_mul / L : 0.f;           // o_mul: FP8 V descale, else 1
     using T = typename std::conditional<BF16, __nv_bfloat16, __half>::type;
     T* orow = reinterpret_cast<T*>(p.o) + (((size_t)x.mb * p.Sq + x.qbase + row) * p.Hq + x.h) * D;
 #pragma unroll 1
@@ -946,7 +955,7 @@ __device__ __forceinline__ void fwd_softmax(const FwdParams& p, const FwdSmem<D,
       }
     }
     if (store && p.lse) {
-      float lse = l_lse > 0.f ? ((FP8 ? m_ref - kFp8Offset : m_ref) + __log2f(l_lse)) * 0.69314718055994531f
+      float lse = E > 0.f ? ((FP8 ? m_ref - kFp8Offset : m_ref) + __log2f(E)) * 0.69314718055994531f
                               : -INFINITY;
       p.lse[((size_t)x.mb * p.Hq + x.h) * p.Sq + x.qbase + row] = lse;
     }

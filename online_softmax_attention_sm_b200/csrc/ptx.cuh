@@ -290,6 +290,200 @@ __device__ __forceinline__ void tmem_wait_st() {
 }
 
 // ----------------------------------------------------------------------------------
+// CTA pairs (a cluster of two CTAs whose tensor cores run one product together).
+// Written from the PTX ISA's descriptions; the pair forms are used by the pair kernel only
+// (a kernel uses one cta_group throughout).  Tensor-memory addresses and shared-memory
+// descriptors name the same columns / offsets in both CTAs.
+// ----------------------------------------------------------------------------------
+__device__ __forceinline__ uint32_t cluster_ctarank() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+  return r;
+}
+__device__ __forceinline__ uint32_t cluster_id_x() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%clusterid.x;" : "=r"(r));
+  return r;
+}
+__device__ __forceinline__ uint32_t nclusters_x() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%nclusterid.x;" : "=r"(r));
+  return r;
+}
+// The shared::cluster address of the same shared-memory offset in CTA `rank` of the cluster.
+__device__ __forceinline__ uint32_t map_shared_rank(const void* p, uint32_t rank) {
+  uint32_t r;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(smem_u32(p)), "r"(rank));
+  return r;
+}
+// One arrival on an mbarrier of another CTA of the cluster.  The default (CTA-scope) release:
+// what it signals is tensor-memory data ordered by tcgen05.wait / tcgen05.fence before it;
+// the cluster-scope release measured about 1500 cycles per arrival here.
+__device__ __forceinline__ void mbar_arrive_cluster(uint32_t cluster_addr) {
+  asm volatile("mbarrier.arrive.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr) : "memory");
+}
+// 4-D tiled load into this CTA's shared memory whose completion (bytes) is counted on an
+// mbarrier of either CTA of the pair (bar: a shared::cluster address); no multicast.
+__device__ __forceinline__ void tma_load_4d_pair(void* dst, const CUtensorMap* map, uint32_t bar_cluster,
+                                                 int c0, int c1, int c2, int c3) {
+  asm volatile(
+      "cp.async.bulk.tensor.4d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%2, %3, %4, %5}], [%6];"
+      ::"r"(smem_u32(dst)), "l"(reinterpret_cast<uint64_t>(map)), "r"(c0), "r"(c1), "r"(c2), "r"(c3),
+        "r"(bar_cluster)
+      : "memory");
+}
+__device__ __forceinline__ bool mbar_try_wait_cl(uint64_t* bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n .reg .pred p;\n"
+      " mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n"
+      " selp.u32 %0, 1, 0, p;\n}\n"
+      : "=r"(ok) : "r"(smem_u32(bar)), "r"(parity) : "memory");
+  return ok != 0;
+}
+// Bounded waits (as mbar_wait / mbar_wait_warp) with acquire at cluster scope, for barriers
+// that arrivals from the peer CTA or the pair's commits complete.
+__device__ __forceinline__ bool mbar_wait_cl(uint64_t* bar, uint32_t parity, volatile int* abort, int where) {
+  if (mbar_try_wait_cl(bar, parity)) return true;
+  const uint64_t t0 = globaltimer_ns();
+  for (uint32_t it = 1;; ++it) {
+    if (mbar_try_wait_cl(bar, parity)) return true;
+    if ((it & 255u) == 0) {
+      if (abort && *abort) return false;
+      if (globaltimer_ns() - t0 > kWaitLimitNs) {
+        record_timeout(where);
+        if (abort) *abort = 1;
+        return false;
+      }
+    }
+  }
+}
+__device__ __forceinline__ bool mbar_wait_warp_cl(uint64_t* bar, uint32_t parity, volatile int* abort, int where) {
+  if (__all_sync(0xffffffffu, mbar_try_wait_cl(bar, parity))) return true;
+  const uint64_t t0 = globaltimer_ns();
+  for (uint32_t it = 1;; ++it) {
+    if (__all_sync(0xffffffffu, mbar_try_wait_cl(bar, parity))) return true;
+    if ((it & 255u) == 0) {
+      if (__any_sync(0xffffffffu, abort != nullptr && *abort != 0)) return false;
+      if (__any_sync(0xffffffffu, globaltimer_ns() - t0 > kWaitLimitNs)) {
+        if ((threadIdx.x & 31) == 0) {
+          record_timeout(where);
+          if (abort) *abort = 1;
+        }
+        return false;
+      }
+    }
+  }
+}
+// Every thread of both CTAs: arrive and wait at the cluster barrier (release / acquire).
+__device__ __forceinline__ void cluster_sync_all() {
+  asm volatile("barrier.cluster.arrive.release.aligned;\n barrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+// Pair tensor memory: one warp of each CTA (the same warp index in both) allocates the same
+// columns in both CTAs' tensor memory; the same warps free them.
+__device__ __forceinline__ void tmem_alloc_pair(uint32_t* dst, uint32_t ncols) {
+  asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;"
+               ::"r"(smem_u32(dst)), "r"(ncols) : "memory");
+}
+__device__ __forceinline__ void tmem_relinquish_pair() {
+  asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void tmem_dealloc_pair(uint32_t taddr, uint32_t ncols) {
+  asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols) : "memory");
+}
+// Pair products, issued by the leader CTA: D rows 0-127 in the leader's tensor memory, rows
+// 128-255 in the peer's; each CTA supplies its own A rows and half of B (N / 2) at the same
+// shared-memory offsets.  x4: 4 k-steps of 16 elements along a 128-byte swizzled row (both
+// descriptors advance 32 bytes); ts_x4: 4 k-steps with A (16-bit P) in tensor memory, 8
+// columns per step, B stepping 16 rows of 128 bytes.
+__device__ __forceinline__ void mma_pair_ss_x4(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
+                                               uint32_t acc_first) {
+  asm volatile(
+      "{\n .reg .pred e, p, q;\n .reg .b32 r;\n .reg .b64 a, b;\n"
+      " elect.sync r|e, 0xffffffff;\n setp.ne.b32 p, %4, 0;\n setp.ne.b32 q, %5, 0;\n"
+      " @e tcgen05.mma.cta_group::2.kind::f16 [%0], %1, %2, %3, p;\n"
+      " add.s64 a, %1, 2;\n add.s64 b, %2, 2;\n"
+      " @e tcgen05.mma.cta_group::2.kind::f16 [%0], a, b, %3, q;\n"
+      " add.s64 a, %1, 4;\n add.s64 b, %2, 4;\n"
+      " @e tcgen05.mma.cta_group::2.kind::f16 [%0], a, b, %3, q;\n"
+      " add.s64 a, %1, 6;\n add.s64 b, %2, 6;\n"
+      " @e tcgen05.mma.cta_group::2.kind::f16 [%0], a, b, %3, q;\n}\n"
+      ::"r"(d_tmem), "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(acc_first), "r"(1u) : "memory");
+}
+//   ss_x8: 8 k-steps over two 128-byte chunks of both operands (chunk strides a_chunk and
+//          b_chunk, in descriptor units of 16 bytes); the first step accumulates iff acc_first.
+__device__ __forceinline__ void mma_pair_ss_x8(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
+                                               uint32_t acc_first, uint32_t a_chunk, uint32_t b_chunk) {
+  asm volatile(
+      "{\n .reg .pred e, p, q;\n .reg .b32 r;\n .reg .b64 a, b, a1, b1;\n"
+      " elect.sync r|e, 0xffffffff;\n setp.ne.b32 p, %4, 0;\n setp.ne.b32 q, %5, 0;\n"
+      " @e tcgen05.mma.cta_group::2.kind::f16 [%0], %1, %2, %3, p;\n"
+      " add.s64 a, %1, 2;\n add.s64 b, %2, 2;\n"
+      " @e tcgen05.mma.cta_group::2.kind::f16 [%0], a, b, %3, q;\n"
+      " add.s64 a, %1, 4;\n add.s64 b, %2, 4;\n"
+      " @e tcgen05.mma.cta_group::2.kind::f16 [%0], a, b, %3, q;\n"
+      " add.s64 a, %1, 6;\n add.s64 b, %2, 6;\n"
+      " @e tcgen05.mma.cta_group::2.kind::f16 [%0], a, b, %3, q;\n"
+      " cvt.u64.u32 a1, %6;\n cvt.u64.u32 b1, %7;\n add.s64 a1, %1, a1;\n add.s64 b1, %2, b1;\n"
+      " @e tcgen05.mma.cta_group::2.kind::f16 [%0], a1, b1, %3, q;\n"
+      " add.s64 a, a1, 2;\n add.s64 b, b1, 2;\n"
+      " @e tcgen05.mma.cta_group::2.kind::f16 [%0], a, b, %3, q;\n"
+      " add.s64 a, a1, 4;\n add.s64 b, b1, 4;\n"
+      " @e tcgen05.mma.cta_group::2.kind::f16 [%0], a, b, %3, q;\n"
+      " add.s64 a, a1, 6;\n add.s64 b, b1, 6;\n"
+      " @e tcgen05.mma.cta_group::2.kind::f16 [%0], a, b, %3, q;\n}\n"
+      ::"r"(d_tmem), "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(acc_first), "r"(1u), "r"(a_chunk), "r"(b_chunk)
+      : "memory");
+}
+//   ts_x8: 8 k-steps with A (16-bit P) in tensor memory at two column bases (keys 0-63 at a0,
+//          keys 64-127 at a1, 8 columns per step), B stepping 16 rows of 128 bytes.
+__device__ __forceinline__ void mma_pair_ts_x8(uint32_t d_tmem, uint32_t a0, uint32_t a1, uint64_t b_desc,
+                                               uint32_t idesc, uint32_t acc_first) {
+  asm volatile(
+      "{\n .reg .pred e, p, q;\n .reg .b32 r, a;\n .reg .b64 b;\n"
+      " elect.sync r|e, 0xffffffff;\n setp.ne.b32 p, %5, 0;\n setp.ne.b32 q, %6, 0;\n"
+      " @e tcgen05.mma.cta_group::2.kind::f16 [%0], [%1], %3, %4, p;\n"
+      " add.u32 a, %1, 8;\n add.s64 b, %3, 128;\n"
+      " @e tcgen05.mma.cta_group::2.kind::f16 [%0], [a], b, %4, q;\n"
+      " add.u32 a, %1, 16;\n add.s64 b, %3, 256;\n"
+      " @e tcgen05.mma.cta_group::2.kind::f16 [%0], [a], b, %4, q;\n"
+      " add.u32 a, %1, 24;\n add.s64 b, %3, 384;\n"
+      " @e tcgen05.mma.cta_group::2.kind::f16 [%0], [a], b, %4, q;\n"
+      " add.s64 b, %3, 512;\n"
+      " @e tcgen05.mma.cta_group::2.kind::f16 [%0], [%2], b, %4, q;\n"
+      " add.u32 a, %2, 8;\n add.s64 b, %3, 640;\n"
+      " @e tcgen05.mma.cta_group::2.kind::f16 [%0], [a], b, %4, q;\n"
+      " add.u32 a, %2, 16;\n add.s64 b, %3, 768;\n"
+      " @e tcgen05.mma.cta_group::2.kind::f16 [%0], [a], b, %4, q;\n"
+      " add.u32 a, %2, 24;\n add.s64 b, %3, 896;\n"
+      " @e tcgen05.mma.cta_group::2.kind::f16 [%0], [a], b, %4, q;\n}\n"
+      ::"r"(d_tmem), "r"(a0), "r"(a1), "l"(b_desc), "r"(idesc), "r"(acc_first), "r"(1u) : "memory");
+}
+__device__ __forceinline__ void mma_pair_ts_x4(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc, uint32_t idesc,
+                                               uint32_t acc_first) {
+  asm volatile(
+      "{\n .reg .pred e, p, q;\n .reg .b32 r, a;\n .reg .b64 b;\n"
+      " elect.sync r|e, 0xffffffff;\n setp.ne.b32 p, %4, 0;\n setp.ne.b32 q, %5, 0;\n"
+      " @e tcgen05.mma.cta_group::2.kind::f16 [%0], [%1], %2, %3, p;\n"
+      " add.u32 a, %1, 8;\n add.s64 b, %2, 128;\n"
+      " @e tcgen05.mma.cta_group::2.kind::f16 [%0], [a], b, %3, q;\n"
+      " add.u32 a, %1, 16;\n add.s64 b, %2, 256;\n"
+      " @e tcgen05.mma.cta_group::2.kind::f16 [%0], [a], b, %3, q;\n"
+      " add.u32 a, %1, 24;\n add.s64 b, %2, 384;\n"
+      " @e tcgen05.mma.cta_group::2.kind::f16 [%0], [a], b, %3, q;\n}\n"
+      ::"r"(d_tmem), "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(acc_first), "r"(1u) : "memory");
+}
+// Commit of the pair's products so far: one arrival on the mbarrier at this offset in each
+// CTA of the pair (mask 0b11) once they have completed.
+__device__ __forceinline__ void mma_commit_pair_warp(uint64_t* bar) {
+  asm volatile(
+      "{\n .reg .pred e;\n .reg .b32 r;\n .reg .b16 m;\n elect.sync r|e, 0xffffffff;\n mov.b16 m, 3;\n"
+      " @e tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64 [%0], m;\n}\n"
+      ::"r"(smem_u32(bar)) : "memory");
+}
+
+// ----------------------------------------------------------------------------------
 // UMMA descriptors (tcgen05 shared-memory matrix descriptor and instruction descriptor)
 // ----------------------------------------------------------------------------------
 // Shared-memory matrix descriptor, 128-byte swizzle, sm_100 version bits.

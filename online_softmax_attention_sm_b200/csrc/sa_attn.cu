@@ -4,6 +4,7 @@
 #include "../../include/sa_attn.h"
 #include "ptx.cuh"
 #include "fwd_sm100.cuh"
+#include "fwd_pair_sm100.cuh"
 #include "sparse_lists.cuh"
 #include "bwd_sm100.cuh"
 #include "fwd_simple.cuh"
@@ -234,6 +235,86 @@ int fwd_work_slot(unsigned int** out) {
   return SA_OK;
 }
 
+// Scheduling groups of the forward's unit order for ncta CTAs (or CTA pairs): (batch, KV
+// head) pairs whose K + V (seq_k keys, row_bytes per key of each) fit in half the L2; among
+// the admissible sizes the one whose band (ceil(ncta / (kv_group * G)) query blocks) fills
+// whole rounds most exactly, then the smaller.
+void plan_units(sa::FwdParams& p, int ncta, int seq_k, double row_bytes) {
+  int dev = 0, l2 = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || cudaDeviceGetAttribute(&l2, cudaDevAttrL2CacheSize, dev) != cudaSuccess)
+    l2 = 64 << 20;
+  const int G = p.Hq / p.Hkv, n_bk = p.B * p.Hkv;
+  const double kv_bytes = 2.0 * seq_k * row_bytes;   // K and V of one (b, KV head)
+  long long gmax = (long long)((l2 / 2) / kv_bytes);
+  if (gmax < 1) gmax = 1;
+  if (gmax > n_bk) gmax = n_bk;
+  int best_g = 1, best_band = 1;
+  double best_waste = 1e30;
+  for (int g = 1; g <= gmax; ++g) {
+    const int band = (ncta + g * G - 1) / (g * G);
+    const double waste = (double)((long long)band * g * G % ncta) / ncta;   // partial round
+    if (waste < best_waste - 1e-9) { best_waste = waste; best_g = g; best_band = band; }
+  }
+  p.kv_group = best_g;
+  p.band = best_band;
+  if (best_band >= p.n_qblk && p.n_qblk > 4) {
+    // short sequences: one band would hold every query block, so a round would mix the
+    // longest and shortest units of a few pairs; take the units longest first across
+    // all pairs instead (bands of one query block, one group).  Measured: 3-26 % faster
+    // for sequences of 2048-8192 tokens and packed mixes; at 1024 tokens (4 query
+    // blocks) the pair-by-pair order was 4 % faster and stays
+    p.band = 1;
+    p.kv_group = n_bk;
+  } else if (p.band > p.n_qblk) {
+    p.band = p.n_qblk;
+  }
+}
+
+// The dense 16-bit forward at D = 128 on CTA pairs (attn_fwd_pair_sm100): p holds the
+// problem (dense layout, static order); the grid is as many clusters of two as fit at once
+// (at most one per two SMs), the unit order planned for that many.
+template <bool BF16>
+int launch_fwd_pair(const void* q, const void* k, const void* v, sa::FwdParams p, int seq_k, cudaStream_t st) {
+  using Cfg = sa::PairCfg;
+  const int ty = BF16 ? SA_BF16 : SA_FP16;
+  CUtensorMap mq, mk, mv;
+  int rc;
+  if ((rc = make_map(&mq, q, ty, 128, p.Hq, p.Sq, p.B, 128)) != SA_OK) return rc;
+  if ((rc = make_map(&mk, k, ty, 128, p.Hkv, p.Sk, p.B, 64)) != SA_OK) return rc;     // 64-key halves
+  if ((rc = make_map(&mv, v, ty, 128, p.Hkv, p.Sk, p.B, 128)) != SA_OK) return rc;
+  auto kern = sa::attn_fwd_pair_sm100<BF16>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::SMEM_TOTAL);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(attn_fwd_pair_sm100)");
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 2;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cudaLaunchConfig_t cfg = {};
+  cfg.blockDim = dim3(Cfg::THREADS);
+  cfg.dynamicSmemBytes = Cfg::SMEM_TOTAL;
+  cfg.stream = st;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  static int max_cl[64] = {0};
+  int dev = 0;
+  if ((e = cudaGetDevice(&dev)) != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+  if (dev < 0 || dev >= 64) return fail(SA_ERR_UNSUPPORTED, "device ordinal %d out of range", dev);
+  if (!max_cl[dev]) {
+    cfg.gridDim = dim3(2 * (num_sms() / 2));
+    int n = 0;
+    e = cudaOccupancyMaxActiveClusters(&n, kern, &cfg);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaOccupancyMaxActiveClusters(attn_fwd_pair_sm100)");
+    if (n <= 0) return fail(SA_ERR_UNSUPPORTED, "no CTA pair of the forward fits on this device");
+    max_cl[dev] = n < num_sms() / 2 ? n : num_sms() / 2;
+  }
+  const int ncl = p.n_units < max_cl[dev] ? p.n_units : max_cl[dev];
+  plan_units(p, ncl, seq_k, 256.0);
+  cfg.gridDim = dim3(2 * ncl);
+  e = cudaLaunchKernelEx(&cfg, kern, mq, mk, mv, p);
+  return e == cudaSuccess ? SA_OK : cuda_fail(e, "attn_fwd_pair_sm100 launch");
+}
+
 // Packed variable-length sequences for launch_fwd (cu_q null: the dense layout).
 struct FwdVarlen {
   const int* cu_q = nullptr;
@@ -263,7 +344,8 @@ int sparse_stride(int Sk) { return 8 + (((Sk + 127) / 128 + 7) / 8) * 8; }
 template <int D, bool BF16, bool FP8 = false>
 int launch_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Sq,
                int Sk, int Hq, int Hkv, int causal, float scale, cudaStream_t st,
-               const FwdVarlen& vl = FwdVarlen(), const FwdSparse& sparse = FwdSparse(), float o_mul = 1.f) {
+               const FwdVarlen& vl = FwdVarlen(), const FwdSparse& sparse = FwdSparse(), float o_mul = 1.f,
+               bool force_pair = false) {
   using Cfg = sa::FwdCfg<D, FP8>;
   const bool packed = vl.cu_q != nullptr;
   const int map_b = packed ? 1 : B;
@@ -291,41 +373,13 @@ int launch_fwd(const void* q, const void* k, const void* v, void* o, float* lse,
   p.n_units = (int)units;
   p.c2 = scale * kLog2e;
   if ((rc = fwd_work_slot(&p.work)) != SA_OK) return rc;
-  {
-    // scheduling groups: (batch, KV head) pairs whose K + V fit in half the L2; among the
-    // admissible sizes take the one whose band (ceil(grid / (kv_group * G)) query blocks)
-    // fills whole rounds most exactly, then the smaller
-    int dev = 0, l2 = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess || cudaDeviceGetAttribute(&l2, cudaDevAttrL2CacheSize, dev) != cudaSuccess)
-      l2 = 64 << 20;
-    const int G = Hq / Hkv, n_bk = B * Hkv;
-    const int ncta = p.n_units < num_sms() ? p.n_units : num_sms();
-    const double kv_bytes = 2.0 * seq_k * D * (FP8 ? 1 : 2);   // K and V of one (b, KV head)
-    long long gmax = (long long)((l2 / 2) / kv_bytes);
-    if (gmax < 1) gmax = 1;
-    if (gmax > n_bk) gmax = n_bk;
-    int best_g = 1, best_band = 1;
-    double best_waste = 1e30;
-    for (int g = 1; g <= gmax; ++g) {
-      const int band = (ncta + g * G - 1) / (g * G);
-      const double waste = (double)((long long)band * g * G % ncta) / ncta;   // partial round
-      if (waste < best_waste - 1e-9) { best_waste = waste; best_g = g; best_band = band; }
-    }
-    p.kv_group = best_g;
-    p.band = best_band;
-    if (best_band >= p.n_qblk && p.n_qblk > 4) {
-      // short sequences: one band would hold every query block, so a round would mix the
-      // longest and shortest units of a few pairs; take the units longest first across
-      // all pairs instead (bands of one query block, one group).  Measured: 3-26 % faster
-      // for sequences of 2048-8192 tokens and packed mixes; at 1024 tokens (4 query
-      // blocks) the pair-by-pair order was 4 % faster and stays
-      p.band = 1;
-      p.kv_group = n_bk;
-    } else if (p.band > p.n_qblk) {
-      p.band = p.n_qblk;
-    }
-  }
+  plan_units(p, p.n_units < num_sms() ? p.n_units : num_sms(), seq_k, (double)D * (FP8 ? 1 : 2));
   const int grid = p.n_units < num_sms() ? p.n_units : num_sms();
+  // the CTA-pair kernel when asked for (sa_attn_fwd_pair; dense 16-bit, D = 128): measured
+  // slower than this kernel on every shape tried, so sa_attn_fwd does not take it
+  if constexpr (!FP8 && D == 128) {
+    if (force_pair && !packed && !paged && !sparse.sp) return launch_fwd_pair<BF16>(q, k, v, p, seq_k, st);
+  }
   // packed lengths and block-sparse lists live on the device, so the static order's
   // balance is unknown: dynamic
   decltype(&sa::attn_fwd_sm100<D, BF16, false, false, FP8>) kern;
@@ -768,6 +822,23 @@ int sa_attn_fwd_simple(const void* q, const void* k, const void* v, void* o, flo
                          : launch_simple<64, false>(q, k, v, o, lse, B, Sq, Sk, Hq, Hkv, causal, scale, st);
   return bf ? launch_simple<128, true>(q, k, v, o, lse, B, Sq, Sk, Hq, Hkv, causal, scale, st)
             : launch_simple<128, false>(q, k, v, o, lse, B, Sq, Sk, Hq, Hkv, causal, scale, st);
+}
+
+int sa_attn_fwd_pair(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Sq,
+                     int Sk, int Hq, int Hkv, int D, int causal, float scale, int dtype, sa_stream_t stream) {
+  int rc = check_dims(B, Sq, Sk, Hq, Hkv, D, dtype, scale);
+  if (rc != SA_OK) return rc;
+  if (D != 128) return fail(SA_ERR_UNSUPPORTED, "the CTA-pair forward supports D = 128 (got %d)", D);
+  if (causal != 0 && causal != 1) return fail(SA_ERR_INVALID, "causal must be 0 or 1");
+  if (B == 0 || Sq == 0 || Hq == 0) return SA_OK;
+  if ((rc = check_ptrs(q, Sk ? k : q, Sk ? v : q, o, lse)) != SA_OK) return rc;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  if (Sk == 0) return launch_fill(o, (size_t)B * Sq * Hq * D, lse, (size_t)B * Hq * Sq, st);
+  return dtype == SA_BF16
+             ? launch_fwd<128, true>(q, k, v, o, lse, B, Sq, Sk, Hq, Hkv, causal, scale, st, FwdVarlen(),
+                                     FwdSparse(), 1.f, true)
+             : launch_fwd<128, false>(q, k, v, o, lse, B, Sq, Sk, Hq, Hkv, causal, scale, st, FwdVarlen(),
+                                      FwdSparse(), 1.f, true);
 }
 
 int sa_attn_decode_num_splits(int B, int Sk, int Hq, int Hkv, int D) {

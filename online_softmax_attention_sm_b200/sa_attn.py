@@ -24,6 +24,7 @@ _P, _I, _F, _Z = ctypes.c_void_p, ctypes.c_int, ctypes.c_float, ctypes.c_size_t
 SIGNATURES = {
     "sa_attn_fwd": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _F, _I, _P]),
     "sa_attn_fwd_simple": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _F, _I, _P]),
+    "sa_attn_fwd_pair": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _F, _I, _P]),
     "sa_attn_fwd_varlen": (_I, [_P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _I, _I, _F, _I, _P]),
     "sa_attn_fwd_block_sparse_workspace_size": (_Z, [_I, _I, _I, _I]),
     "sa_attn_bwd_workspace_size": (_Z, [_I, _I, _I]),
@@ -114,7 +115,7 @@ def _check_workspace(t, device):
 
 
 def sa_attn_fwd(q, k, v, causal=False, scale=None, out=None, lse=None, return_lse=True,
-                stream=None, simple=False):
+                stream=None, simple=False, pair=False):
     """Attention forward.  q [B,Sq,Hq,D], k/v [B,Sk,Hkv,D] (fp16/bf16, CUDA, contiguous).
     Returns (o [B,Sq,Hq,D], lse [B,Hq,Sq] fp32 or None)."""
     B, Sq, Hq, D = q.shape
@@ -134,7 +135,7 @@ def sa_attn_fwd(q, k, v, causal=False, scale=None, out=None, lse=None, return_ls
         lse = torch.empty((B, Hq, Sq), dtype=torch.float32, device=q.device)
     if lse is not None:
         _check_out("lse", lse, (B, Hq, Sq), torch.float32, q.device)
-    fn = lib().sa_attn_fwd_simple if simple else lib().sa_attn_fwd
+    fn = lib().sa_attn_fwd_simple if simple else lib().sa_attn_fwd_pair if pair else lib().sa_attn_fwd
     _check(fn(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse), B, Sq, Sk, Hq, Hkv, D,
               int(bool(causal)), float(scale), _DT[q.dtype], _stream(stream)))
     return out, lse
@@ -346,6 +347,11 @@ def sa_attn_fwd_paged(q, k_cache, v_cache, cu_seqlens_q, block_table, seqlens_k,
                                    page_size, block_table.shape[1], num_pages, int(bool(causal)), float(scale),
                                    _DT[q.dtype], _stream(stream)))
     return out, lse
+
+
+def sa_attn_fwd_pair(q, k, v, causal=False, scale=None, **kw):
+    """The forward on the CTA-pair kernel whatever the shape (D = 128); as sa_attn_fwd."""
+    return sa_attn_fwd(q, k, v, causal, scale, pair=True, **kw)
 
 
 def sa_attn_fwd_simple(q, k, v, causal=False, scale=None, **kw):
