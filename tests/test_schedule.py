@@ -1,7 +1,8 @@
 """Host-side check of the prefill's unit enumeration (a mirror of the kernel's fwd_unit and
-of the host's choice of group and band): every (batch, head, query block) is produced
-exactly once, heads map to their KV head, and the order keeps the longest units first
-within each band."""
+of the host's choice of group and band, plan_units, including its short-sequence branch):
+every (batch, head, query block) is produced exactly once, heads map to their KV head, and
+the order keeps the longest units first within each band -- across every pair when the
+short-sequence branch applies."""
 import math
 
 import pytest
@@ -19,7 +20,11 @@ def choose(B, Sq, Sk, Hq, Hkv, D, ncta=148, l2=126 * 2 ** 20):
         waste = (band * g * G % ncta) / ncta
         if waste < best[0] - 1e-9:
             best = (waste, g, band)
-    return best[1], min(best[2], n_qblk)
+    kg, band = best[1], best[2]
+    if band >= n_qblk and n_qblk > 4:
+        # short sequences: bands of one query block over every (batch, KV head) pair
+        return n_bk, 1
+    return kg, min(band, n_qblk)
 
 
 def unit(u, B, Sq, Hq, Hkv, kv_group, band):
@@ -61,3 +66,16 @@ def test_unit_order_is_a_bijection(shape):
 def test_long_gqa_workload_choice():
     # 32768 tokens, 8 KV heads of 16.8 MB K+V each: one KV head per group, 37-block bands
     assert choose(1, 32768, 32768, 32, 8, 128) == (1, 37)
+
+
+def test_short_sequences_go_longest_first_across_all_pairs():
+    # 2048 tokens, 16 batches: one band would hold all 8 query blocks, so the host takes
+    # bands of one query block over all (batch, KV head) pairs
+    B, Sq, Sk, Hq, Hkv, D = 16, 2048, 2048, 8, 2, 128
+    kg, band = choose(B, Sq, Sk, Hq, Hkv, D)
+    assert (kg, band) == (B * Hkv, 1)
+    n_qblk = (Sq + 255) // 256
+    qbs = [unit(u, B, Sq, Hq, Hkv, kg, band)[2] for u in range(B * Hq * n_qblk)]
+    assert qbs == sorted(qbs, reverse=True)          # strictly longest query blocks first
+    assert len({(b, h, qb) for b, h, qb, _ in (unit(u, B, Sq, Hq, Hkv, kg, band)
+                                                for u in range(B * Hq * n_qblk))}) == B * Hq * n_qblk
