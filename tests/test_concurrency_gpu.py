@@ -1,8 +1,8 @@
 """Forward launches that take their work units from the library's shared counter pairs (the
 dynamic instance: every packed-sequence forward), many in flight at once on several streams:
-each must give exactly the result of a launch run alone.  More launches than the round-1
-pool had counter pairs (64), fewer than the current pool (1024), so a launch that picked up
-a pair still in use -- units skipped or run twice -- would show as a wrong output."""
+each must give exactly the result of a launch run alone.  More launches than a 64-pair pool
+would hold, fewer than the library's 1024 pairs, so a launch that picked up a pair still in
+use -- units skipped or run twice -- would show as a wrong output."""
 import numpy as np
 import pytest
 import torch
