@@ -301,11 +301,20 @@ __device__ __forceinline__ void fwd_producer(const CUtensorMap* tm_q, const CUte
       // ---- the next unit (an index past the list ends the CTA), posted to the other roles
       int u;
       UnitInfo x;
+      bool have_x = false;
+      const int us = n % kUnitQueue;
       if (!DYN) {
         u = fwd_unit_of(n, cta, ncta);       // every role computes the same index
       } else {
-        const int us = n % kUnitQueue;
         u = n == 0 ? cta : ncta + (int)atomicAdd(p.work, 1u);
+        if (!SPARSE && p.cu_q) {
+          // packed sequences shorter than the longest leave units without a single row
+          // (nothing to compute or write): take the next one instead of handing them out
+          for (; u < p.n_units; u = ncta + (int)atomicAdd(p.work, 1u)) {
+            x = fwd_unit<DYN, PAGED>(p, u);
+            if (x.q0 < x.sq) { have_x = true; break; }
+          }
+        }
         if (n >= kUnitQueue) {
           ok = mbar_wait(&sm.unit_empty[us], ((n / kUnitQueue) - 1) & 1, sm.abort_flag, 5);
           if (!ok) break;
@@ -327,7 +336,9 @@ __device__ __forceinline__ void fwd_producer(const CUtensorMap* tm_q, const CUte
         }
       }
       if (u >= p.n_units) break;
-      if (!SPARSE) x = fwd_unit<DYN, PAGED>(p, u);
+      // (dynamic order: the unit's coordinates from the posted index, read back, so that their
+      // arithmetic cannot be scheduled ahead of the posting the other roles wait for)
+      if (!SPARSE && !have_x) x = fwd_unit<DYN, PAGED>(p, DYN ? (int)sm.uq[us] : u);
       for (int j = 0; j < x.nkv_max && ok; ++j) {
         const int kt = SPARSE ? (int)(x.ent[j] & 0x3fffu) : j;   // key tile of this step
         for (int kv = 0; kv < 2 && ok; ++kv) {
