@@ -215,6 +215,8 @@ def main():
                     help="profiling aid: run only one part (the JSON line is then partial)")
     ap.add_argument("--prefill-seq", type=int, default=0,
                     help="profiling aid: shorter prefill sequence (same heads, dtype, sinks)")
+    ap.add_argument("--varlen-tokens", type=int, default=0,
+                    help="profiling aid: fewer tokens in the packed mix (same 16 sequences' recipe and heads)")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
@@ -249,6 +251,10 @@ def main():
         import dataclasses
         wp = dataclasses.replace(wp, name=f"{wp.name}_seq{args.prefill_seq}", Sq=args.prefill_seq,
                                  Sk=args.prefill_seq)
+    if args.varlen_tokens:
+        import dataclasses
+        wv = dataclasses.replace(wv, name=f"{wv.name}_t{args.varlen_tokens}", Sq=args.varlen_tokens,
+                                 Sk=args.varlen_tokens)
     run = {k: args.only in ("all", k) for k in ("prefill", "decode", "small", "varlen", "sparse", "backward", "fp8")}
     q_h, k_h, v_h = make_workload_inputs(wp, seed=rank_seed(wp.seed, rank))
     dq_h, dk_h, dv_h = make_workload_inputs(wd, seed=rank_seed(wd.seed, rank))
