@@ -190,7 +190,7 @@ int sa_attn_decode_single(const void* q, const void* k, const void* v, void* o, 
  * S on kind::f8f6f4 tensor cores (exact products, fp32 sums), P rounded to e4m3 for P V.
  * D must be 128 (else SA_ERR_UNSUPPORTED); descales finite and > 0 (else SA_ERR_INVALID).
  * Accuracy: each weight p = 2^(s - m_ref + 8) is rounded to e4m3 against its row's running
- * reference max m_ref, which moves whenever the row max passes it by half a unit (log2),
+ * reference max m_ref, which moves whenever the row max passes it by 0.75 (log2 units),
  * so the largest weights sit near 2^8 (under e4m3's 448) and only weights below 2^-18 of the
  * row max round to zero.  O is normalised by the sum of the rounded weights; the LSE comes
  * from fp32 sums of the unrounded ones (the offset taken off), as in sa_attn_fwd.

@@ -22,7 +22,7 @@
 //     S (tcgen05.ld 32x32b), computes the row max, p = 2^(c*s - m) with c = scale*log2(e),
 //     the row sums, writes P as 16-bit into tensor memory over S, and rescales its O row
 //     only when the reference max moves by more than kRescaleThresh (exact after the
-//     final division; keeps p <= 2^kRescaleThresh; FP8: past half a unit, against an
+//     final division; keeps p <= 2^kRescaleThresh; FP8: past three quarters of a unit, against an
 //     offset of 2^8);
 //   * the epilogue (same warpgroups) divides O by the row sum, rounds to the I/O dtype
 //     and writes O and the natural-log LSE.
@@ -83,8 +83,8 @@ constexpr float kRescaleThresh = 8.0f;   // log2 units: the reference moves past
 // FP8 weights: p = 2^(x - m_ref + kFp8Offset), so a row's largest weights sit near the top of
 // e4m3's range instead of at 1 (weights below 2^-10 of the top round to zero, and a long row
 // can hold many of them); the reference then moves once the max passes it by kFp8Thresh,
-// which keeps p <= 2^8.5 < 448.  O / l is unchanged, the LSE takes kFp8Offset off.
-constexpr float kFp8Offset = 8.0f, kFp8Thresh = 0.5f;
+// which keeps p <= 2^8.75 < 448.  O / l is unchanged, the LSE takes kFp8Offset off.
+constexpr float kFp8Offset = 8.0f, kFp8Thresh = 0.75f;
 constexpr int kPolyEvery = 4;            // full tiles: one exponential pair in kPolyEvery on the FMA pipe (0: none)
 
 struct FwdParams {
@@ -663,7 +663,7 @@ __device__ __forceinline__ void softmax_chunk(const uint32_t (&v)[32], const f32
 }
 
 // FP8 instance: the same chunk with P rounded to e4m3 (round to nearest even, saturating:
-// p <= 2^8.5 under the offset reference, below e4m3's 448), 4 values per tensor-memory column
+// p <= 2^8.75 under the offset reference, below e4m3's 448), 4 values per tensor-memory column
 // (key 4j in the low byte of column j), 8 columns at taddr; rs2 sums the e4m3 values the
 // MMA multiplies.
 template <int POLY>

@@ -13,10 +13,10 @@ row max, the kernel offsetting its weights by 2^8) have an absolute rounding err
 The LSE uses fp32 sums of unrounded weights: 1e-3 as for the 16-bit forward.
 
 At the bench's 32768-token size the weights below e4m3's normal range matter: the kernel
-writes them as p_j = 2^(s_j - m_ref + 8) with its reference m_ref at most half a unit (log2)
-below the row max, so a weight under 2^-14 of the row max (under 2^-6 after the offset) is
-subnormal, with an absolute rounding error of at most 2^-10, i.e. 2^-18 of the row max, and
-one under 2^-18 of the max rounds to zero.  On long rows that a few sink keys dominate, tens
+writes them as p_j = 2^(s_j - m_ref + 8) with its reference m_ref at most 0.75 (log2 units)
+below the row max, so only a weight under 2^-14 of the row max can be subnormal (under 2^-6
+after the offset), with an absolute rounding error of at most 2^-10, i.e. 2^-18 of the row
+max, and only one under 2^-18 of the max can round to zero.  On long rows that a few sink keys dominate, tens
 of thousands of weights sit there.  The check on sampled rows is the first-order bound of
 the normal-range weights plus one fixed absolute term,
     |O_gpu - O| <= (u/(1-u) + 1e-4) sum_j P_j |v_j - O| + 2^-8 |O| + 2e-3 + A,   A = 0.05,
