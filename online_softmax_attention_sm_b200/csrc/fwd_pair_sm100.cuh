@@ -311,17 +311,17 @@ __device__ __forceinline__ void pair_softmax(const FwdParams& p, const PairSmem&
       }
       const float m_use = (m_ref == -INFINITY) ? 0.f : m_ref;
       const f32x2 scale2 = full ? pack_f2(c2, c2) : pack_f2(1.f, 1.f), negm2 = pack_f2(-m_use, -m_use);
-      f32x2 rs2[2] = {0ull, 0ull}, rse2[2] = {0ull, 0ull};
+      f32x2 rse2[2] = {0ull, 0ull};
       float rs[4] = {0.f, 0.f, 0.f, 0.f};
       const uint32_t pa = lane_addr + PairCfg::P_COL(b, h);
       if (full) {
-        softmax_chunk_any<BF16, false, kPolyEvery>(v[0], scale2, negm2, rs2, rs, rse2, pa, 0);
-        softmax_chunk_any<BF16, false, kPolyEvery>(v[1], scale2, negm2, rs2, rs, rse2, pa, 1);
+        softmax_chunk_any<BF16, false, kPolyEvery>(v[0], scale2, negm2, rs, rse2, pa, 0);
+        softmax_chunk_any<BF16, false, kPolyEvery>(v[1], scale2, negm2, rs, rse2, pa, 1);
       } else {
-        softmax_chunk_any<BF16, false, 0>(v[0], scale2, negm2, rs2, rs, rse2, pa, 0);
-        softmax_chunk_any<BF16, false, 0>(v[1], scale2, negm2, rs2, rs, rse2, pa, 1);
+        softmax_chunk_any<BF16, false, 0>(v[0], scale2, negm2, rs, rse2, pa, 0);
+        softmax_chunk_any<BF16, false, 0>(v[1], scale2, negm2, rs, rse2, pa, 1);
       }
-      sum_rounded(rs2, rs, false, l_sum);
+      sum_rounded(rs, l_sum);
       sum_f2x2(rse2, l_lse);
       if (h == 0 && j > 0) {
         // O holds P V up to step j-1 once that product completes (its V slot's free barrier);

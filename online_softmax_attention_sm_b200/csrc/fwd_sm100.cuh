@@ -664,11 +664,11 @@ __device__ __forceinline__ void softmax_chunk(const uint32_t (&v)[32], const f32
 
 // FP8 instance: the same chunk with P rounded to e4m3 (round to nearest even, saturating:
 // p <= 2^8.75 under the offset reference, below e4m3's 448), 4 values per tensor-memory column
-// (key 4j in the low byte of column j), 8 columns at taddr; rs2 sums the e4m3 values the
-// MMA multiplies.
+// (key 4j in the low byte of column j), 8 columns at taddr; rs sums the e4m3 values the
+// MMA multiplies (each exact in f16, added to fp32 by mixed-precision adds).
 template <int POLY>
 __device__ __forceinline__ void softmax_chunk_fp8(const uint32_t (&v)[32], const f32x2 scale2,
-                                                  const f32x2 negm2, f32x2 (&rs2)[2], f32x2 (&rse2)[2],
+                                                  const f32x2 negm2, float (&rs)[4], f32x2 (&rse2)[2],
                                                   const uint32_t taddr) {
   uint32_t pk[8];
 #pragma unroll
@@ -687,8 +687,7 @@ __device__ __forceinline__ void softmax_chunk_fp8(const uint32_t (&v)[32], const
     asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(e8) : "f"(b2), "f"(a));
     uint32_t h2;          // the two e4m3 values back as f16x2, for the row sum
     asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(h2) : "h"(e8));
-    const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&h2));
-    rs2[i & 1] = add_f2(rs2[i & 1], pack_f2(f.x, f.y));
+    add_16x2_to_f32<false>(h2, rs[2 * (i & 1)], rs[2 * (i & 1) + 1]);
     if (i & 1) pk[i >> 1] |= (uint32_t)e8 << 16;
     else pk[i >> 1] = e8;
   }
@@ -698,24 +697,16 @@ __device__ __forceinline__ void softmax_chunk_fp8(const uint32_t (&v)[32], const
                : "memory");
 }
 
-// rs2 (FP8: the e4m3 weights' sum as packed pairs) and rs (16-bit: four fp32 chains) hold
-// the sum of the weights the MMA multiplies.
+// rs (four fp32 chains) holds the sum of the weights the MMA multiplies (16-bit or e4m3).
 template <bool BF16, bool FP8, int POLY>
 __device__ __forceinline__ void softmax_chunk_any(const uint32_t (&v)[32], const f32x2 scale2, const f32x2 negm2,
-                                                  f32x2 (&rs2)[2], float (&rs)[4], f32x2 (&rse2)[2],
-                                                  const uint32_t p_addr, int c) {
-  if constexpr (FP8) softmax_chunk_fp8<POLY>(v, scale2, negm2, rs2, rse2, p_addr + c * 8);
+                                                  float (&rs)[4], f32x2 (&rse2)[2], const uint32_t p_addr, int c) {
+  if constexpr (FP8) softmax_chunk_fp8<POLY>(v, scale2, negm2, rs, rse2, p_addr + c * 8);
   else softmax_chunk<BF16, POLY>(v, scale2, negm2, rs, rse2, p_addr + c * 16);
 }
 
-__device__ __forceinline__ void sum_rounded(const f32x2 (&rs2)[2], const float (&rs)[4], bool fp8, float& acc) {
-  if (fp8) {
-    float a0, a1;
-    unpack_f2(add_f2(rs2[0], rs2[1]), a0, a1);
-    acc += a0 + a1;
-  } else {
-    acc += (rs[0] + rs[1]) + (rs[2] + rs[3]);
-  }
+__device__ __forceinline__ void sum_rounded(const float (&rs)[4], float& acc) {
+  acc += (rs[0] + rs[1]) + (rs[2] + rs[3]);
 }
 
 // Running max over a 32-score chunk on 8 chains.
@@ -803,23 +794,23 @@ __device__ __forceinline__ void softmax_tile_full(const uint32_t s_addr, const u
   const f32x2 scale2 = pack_f2(c2, c2), negm2 = pack_f2(nm, nm);
   // the row's sums are kept per key half (keys 0-63, 64-127) and added at the end, the order
   // the pair kernel's two half-row threads use, so both kernels give identical bits
-  f32x2 rs2[2][2] = {{0ull, 0ull}, {0ull, 0ull}}, rse2[2][2] = {{0ull, 0ull}, {0ull, 0ull}};
+  f32x2 rse2[2][2] = {{0ull, 0ull}, {0ull, 0ull}};
   float rs[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
   uint32_t v2[32], v3[32];
   tmem_ld32(s_addr + 64, v2);
-  softmax_chunk_any<BF16, FP8, kPolyEvery>(v0, scale2, negm2, rs2[0], rs[0], rse2[0], p_addr, 0);
-  softmax_chunk_any<BF16, FP8, kPolyEvery>(v1, scale2, negm2, rs2[0], rs[0], rse2[0], p_addr, 1);
+  softmax_chunk_any<BF16, FP8, kPolyEvery>(v0, scale2, negm2, rs[0], rse2[0], p_addr, 0);
+  softmax_chunk_any<BF16, FP8, kPolyEvery>(v1, scale2, negm2, rs[0], rse2[0], p_addr, 1);
   tmem_wait_ld_regs(v2);
   tmem_ld32(s_addr + 96, v3);
-  softmax_chunk_any<BF16, FP8, kPolyEvery>(v2, scale2, negm2, rs2[1], rs[1], rse2[1], p_addr, 2);
+  softmax_chunk_any<BF16, FP8, kPolyEvery>(v2, scale2, negm2, rs[1], rse2[1], p_addr, 2);
   tmem_wait_st();
   tc_fence_before();
   mbar_arrive(p_part);
   tmem_wait_ld_regs(v3);
-  softmax_chunk_any<BF16, FP8, kPolyEvery>(v3, scale2, negm2, rs2[1], rs[1], rse2[1], p_addr, 3);
+  softmax_chunk_any<BF16, FP8, kPolyEvery>(v3, scale2, negm2, rs[1], rse2[1], p_addr, 3);
 #pragma unroll
   for (int hh = 0; hh < 2; ++hh) {
-    sum_rounded(rs2[hh], rs[hh], FP8, l_sum[hh]);
+    sum_rounded(rs[hh], l_sum[hh]);
     sum_f2x2(rse2[hh], l_lse[hh]);
   }
 }
@@ -850,11 +841,11 @@ __device__ __forceinline__ void softmax_tile_masked(const uint32_t s_addr, const
   const float m_use = (m_ref == -INFINITY) ? 0.f : m_ref;
   const float nm = FP8 ? kFp8Offset - m_use : -m_use;
   const f32x2 scale2 = pack_f2(1.f, 1.f), negm2 = pack_f2(nm, nm);
-  f32x2 rs2[2][2] = {{0ull, 0ull}, {0ull, 0ull}}, rse2[2][2] = {{0ull, 0ull}, {0ull, 0ull}};
+  f32x2 rse2[2][2] = {{0ull, 0ull}, {0ull, 0ull}};
   float rs[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
 #pragma unroll
   for (int c = 0; c < 4; ++c) {
-    softmax_chunk_any<BF16, FP8, 0>(v[c], scale2, negm2, rs2[c >> 1], rs[c >> 1], rse2[c >> 1], p_addr, c);
+    softmax_chunk_any<BF16, FP8, 0>(v[c], scale2, negm2, rs[c >> 1], rse2[c >> 1], p_addr, c);
     if (c == 2) {
       tmem_wait_st();
       tc_fence_before();
@@ -863,7 +854,7 @@ __device__ __forceinline__ void softmax_tile_masked(const uint32_t s_addr, const
   }
 #pragma unroll
   for (int hh = 0; hh < 2; ++hh) {
-    sum_rounded(rs2[hh], rs[hh], FP8, l_sum[hh]);
+    sum_rounded(rs[hh], l_sum[hh]);
     sum_f2x2(rse2[hh], l_lse[hh]);
   }
 }
