@@ -63,13 +63,16 @@ EncodeTiledFn get_encode() {
 // Device address of a __device__ variable of this library on the current device, looked up
 // once per (device, context, variable) with that device current and cached.  Keyed by the
 // context too: after a device reset the runtime creates a new primary context and reloads
-// the module, and the old address would be stale.
+// the module, and the old address would be stale.  The context is identified by its
+// process-unique id (cuCtxGetId), not its handle, which a new context could reuse.
 using CtxGetCurrentFn = CUresult (*)(CUcontext*);
+using CtxGetIdFn = CUresult (*)(CUcontext, unsigned long long*);
 
 int device_symbol(const void* symbol, const char* what, void** out) {
   static std::mutex mu;
-  static std::map<std::tuple<int, uintptr_t, uintptr_t>, void*> cache;
+  static std::map<std::tuple<int, unsigned long long, uintptr_t>, void*> cache;
   static CtxGetCurrentFn ctx_fn = nullptr;
+  static CtxGetIdFn id_fn = nullptr;
   static std::once_flag once;
   std::call_once(once, [] {
     void* p = nullptr;
@@ -77,6 +80,10 @@ int device_symbol(const void* symbol, const char* what, void** out) {
     if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &p, cudaEnableDefault, &q) == cudaSuccess &&
         q == cudaDriverEntryPointSuccess)
       ctx_fn = reinterpret_cast<CtxGetCurrentFn>(p);
+    p = nullptr;
+    if (cudaGetDriverEntryPoint("cuCtxGetId", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      id_fn = reinterpret_cast<CtxGetIdFn>(p);
   });
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
@@ -88,7 +95,10 @@ int device_symbol(const void* symbol, const char* what, void** out) {
     cudaFree(nullptr);
     if (ctx_fn(&ctx) != CUDA_SUCCESS) ctx = nullptr;
   }
-  const auto key = std::make_tuple(dev, reinterpret_cast<uintptr_t>(ctx), reinterpret_cast<uintptr_t>(symbol));
+  unsigned long long ctx_key = reinterpret_cast<uintptr_t>(ctx);
+  unsigned long long id = 0;
+  if (ctx && id_fn && id_fn(ctx, &id) == CUDA_SUCCESS) ctx_key = id;
+  const auto key = std::make_tuple(dev, ctx_key, reinterpret_cast<uintptr_t>(symbol));
   std::lock_guard<std::mutex> lock(mu);
   auto it = cache.find(key);
   if (it != cache.end()) { *out = it->second; return SA_OK; }
