@@ -523,6 +523,25 @@ __device__ __forceinline__ void fwd_mma(const FwdParams& p, const FwdSmem<D, FP8
         const uint32_t v_addr = sRing_addr + (vpos % Cfg::STAGES) * Cfg::TILE_BYTES;
         const uint32_t k_addr = sRing_addr + (kpos % Cfg::STAGES) * Cfg::TILE_BYTES;
         bool k_ready = false;
+        bool s_ahead[2] = {false, false};
+        if (SPARSE && FP8 && j + 1 < x.nkv_max) {
+          // FP8 block-sparse (8-slot ring of 16 KB tiles): a Q tile idle at this step but
+          // working at the next one gets its next S now, ahead of the other tile's P V, so that
+          // with alternating single-tile steps the two softmax warpgroups overlap -- only if
+          // K_{j+1} (and that tile's Q) have landed: waiting here would hold up that P V.
+          // (K_{j+1}'s slot held a tile of an earlier step, already waited for, so the parity
+          // test sees no older phase.)
+          for (int t = 0; t < 2; ++t) {
+            if (act(t, j) || !act(t, j + 1)) continue;
+            if (!k_ready)
+              k_ready = __all_sync(0xffffffffu, mbar_try_wait(&sm.kv_full[kpos % Cfg::STAGES], (kpos / Cfg::STAGES) & 1));
+            if (!k_ready) break;
+            if (q_wait[t]) continue;
+            tc_fence_after();
+            issue_qk(t, k_addr);
+            s_ahead[t] = true;
+          }
+        }
         for (int t = 0; t < 2; ++t) {
           const bool live = SPARSE || j < x.nkv[t];
           if (live && act(t, j)) {
@@ -553,7 +572,7 @@ __device__ __forceinline__ void fwd_mma(const FwdParams& p, const FwdSmem<D, FP8
           // V_j's last reader is in the pipe: release its slot ahead of the second S
           if (t == 1) mma_commit_warp(&sm.kv_empty[vpos % Cfg::STAGES]);
           // ---- S_t = Q_t K_{j+1}^T
-          if (live && act(t, j + 1)) {
+          if (live && act(t, j + 1) && !s_ahead[t]) {
             if (!k_ready) {
               ok = mbar_wait_warp(&sm.kv_full[kpos % Cfg::STAGES], (kpos / Cfg::STAGES) & 1, sm.abort_flag, 10);
               if (!ok) break;
