@@ -86,6 +86,13 @@ constexpr float kRescaleThresh = 8.0f;   // log2 units: the reference moves past
 // which keeps p <= 2^8.75 < 448.  O / l is unchanged, the LSE takes kFp8Offset off.
 constexpr float kFp8Offset = 8.0f, kFp8Thresh = 0.75f;
 constexpr int kPolyEvery = 4;            // full tiles: one exponential pair in kPolyEvery on the FMA pipe (0: none)
+// The FP8 block-sparse instance runs many single-tile steps, where one softmax warpgroup has
+// the MUFU to itself, on a softmax with fewer instructions per score: there the FMA-pipe
+// share only costs issue slots (measured 4 % slower at one pair in four), so it takes none.
+// (The 16-bit block-sparse instance keeps the dense share: with every block kept it gives the
+// dense forward's bits.)
+template <bool SPARSE, bool FP8>
+__host__ __device__ constexpr int poly_every() { return (SPARSE && FP8) ? 0 : kPolyEvery; }
 
 struct FwdParams {
   void* o;
@@ -783,7 +790,7 @@ __device__ __forceinline__ void move_reference(const float m_tile, const bool fi
 // exponentials.  P overwrites S columns 0-63 only, so the second pass holds chunks 0-1
 // from the first and loads chunks 2-3 again, which keeps a quarter fewer registers live
 // through the exponentials.  The MMA warp may start on keys 0-95 at p_part.
-template <int D, bool BF16, bool FP8>
+template <int D, bool BF16, bool FP8, int POLY>
 __device__ __forceinline__ void softmax_tile_full(const uint32_t s_addr, const uint32_t o_addr,
                                                   const uint32_t p_addr, const float c2, const bool first,
                                                   float& m_ref, float (&l_sum)[2], float (&l_lse)[2],
@@ -817,16 +824,16 @@ __device__ __forceinline__ void softmax_tile_full(const uint32_t s_addr, const u
   float rs[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
   uint32_t v2[32], v3[32];
   tmem_ld32(s_addr + 64, v2);
-  softmax_chunk_any<BF16, FP8, kPolyEvery>(v0, scale2, negm2, rs[0], rse2[0], p_addr, 0);
-  softmax_chunk_any<BF16, FP8, kPolyEvery>(v1, scale2, negm2, rs[0], rse2[0], p_addr, 1);
+  softmax_chunk_any<BF16, FP8, POLY>(v0, scale2, negm2, rs[0], rse2[0], p_addr, 0);
+  softmax_chunk_any<BF16, FP8, POLY>(v1, scale2, negm2, rs[0], rse2[0], p_addr, 1);
   tmem_wait_ld_regs(v2);
   tmem_ld32(s_addr + 96, v3);
-  softmax_chunk_any<BF16, FP8, kPolyEvery>(v2, scale2, negm2, rs[1], rse2[1], p_addr, 2);
+  softmax_chunk_any<BF16, FP8, POLY>(v2, scale2, negm2, rs[1], rse2[1], p_addr, 2);
   tmem_wait_st();
   tc_fence_before();
   mbar_arrive(p_part);
   tmem_wait_ld_regs(v3);
-  softmax_chunk_any<BF16, FP8, kPolyEvery>(v3, scale2, negm2, rs[1], rse2[1], p_addr, 3);
+  softmax_chunk_any<BF16, FP8, POLY>(v3, scale2, negm2, rs[1], rse2[1], p_addr, 3);
 #pragma unroll
   for (int hh = 0; hh < 2; ++hh) {
     sum_rounded(rs[hh], l_sum[hh]);
@@ -923,7 +930,8 @@ __device__ __forceinline__ void fwd_softmax(const FwdParams& p, const FwdSmem<D,
       ++s_n;
       tc_fence_after();
       if (kt < mask_from && c2 >= 0.f) {
-        softmax_tile_full<D, BF16, FP8>(s_addr, o_addr, p_addr, c2, first, m_ref, l_sum, l_lse, &sm.p_part[t]);
+        softmax_tile_full<D, BF16, FP8, poly_every<SPARSE, FP8>()>(s_addr, o_addr, p_addr, c2, first, m_ref, l_sum, l_lse,
+                                                            &sm.p_part[t]);
       } else {
         const int kl = (kt >= mask_from) ? klim - kt * 128 : 128;   // keys >= kl: invisible to this row
         softmax_tile_masked<D, BF16, FP8>(s_addr, o_addr, p_addr, c2, kl, first, m_ref, l_sum, l_lse,
