@@ -52,3 +52,20 @@ def test_our_arm_fails_loudly_without_a_gpu():
     r = run_bench("--steps", "1", "--warmup", "3", "--cpu-seconds", "0", "--no-e2e", timeout=300)
     assert r.returncode != 0
     assert not r.stdout.strip(), "no JSON line may come out of a run without the GPU path"
+
+
+def test_reference_arm_under_two_ranks_prints_once():
+    # launched the way the scaling run launches every arm; rank 0 alone runs the oracle
+    import socket
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        port = s.getsockname()[1]
+    r = subprocess.run([sys.executable, "-m", "torch.distributed.run", "--nnodes=1", "--nproc-per-node", "2",
+                        "--master-addr", "127.0.0.1", "--master-port", str(port),
+                        os.path.join(ROOT, "bench.py"), "--impl", "reference", "--gpus", "2", "--steps", "1",
+                        "--warmup", "3"], cwd=ROOT, capture_output=True, text=True, timeout=600)
+    assert r.returncode == 0, r.stderr[-2000:]
+    lines = [l for l in r.stdout.splitlines() if l.strip().startswith("{")]
+    assert len(lines) == 1, r.stdout[-2000:]
+    line = json.loads(lines[0])
+    assert line["impl"] == "reference" and line["n_gpus"] == 2 and line["cpu_baseline"]["cores"] >= 1
